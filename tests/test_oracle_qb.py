@@ -1,0 +1,219 @@
+"""Pins for the oracle's optimal-assignment balancing (QB + exact finish).
+
+Fixed by: brute-force enumeration on tiny instances, scipy's HiGHS LP solver on
+the relaxation (integral by the max-min argument), scipy's Hungarian solver
+for k = 1, the closed-form minimum of each dual sub-problem, the constraint
+sums, and the demo's qualitative claim that the bias evens the load.
+Source: "MoE travelogue 6: optimal assignment promotes balance"
+(kexue.fm/archives/11619): Linear programming eqs. (3)-(4), Max-min (7),
+Divide and conquer (8)-(11), Alternating iteration, Mind the pitfall, Demo code.
+"""
+import itertools
+
+import numpy as np
+import pytest
+from scipy.optimize import linear_sum_assignment, linprog
+
+import oracle
+import workloads as W
+
+
+def _objective(s, idx):
+    return float(np.take_along_axis(s.astype(np.float64), idx.astype(np.int64), 1).sum())
+
+
+def _brute(s, k):
+    """Best objective and every optimal assignment (as frozensets per token) by enumeration."""
+    m, n = s.shape
+    C = m * k // n
+    combos = list(itertools.combinations(range(n), k))
+    best, arg = -np.inf, []
+    for choice in itertools.product(combos, repeat=m):
+        cnt = np.zeros(n, int)
+        for ch in choice:
+            cnt[list(ch)] += 1
+        if (cnt != C).any():
+            continue
+        v = sum(float(s[i, list(ch)].astype(np.float64).sum()) for i, ch in enumerate(choice))
+        if v > best + 1e-12:
+            best, arg = v, [choice]
+        elif abs(v - best) <= 1e-12:
+            arg.append(choice)
+    return best, arg
+
+
+def _lp(s, k):
+    m, n = s.shape
+    C = m * k // n
+    A = np.zeros((m + n, m * n))
+    for i in range(m):
+        A[i, i * n:(i + 1) * n] = 1
+    for j in range(n):
+        A[m + j, j::n] = 1
+    r = linprog(-s.astype(np.float64).ravel(), A_eq=A, b_eq=[k] * m + [C] * n, bounds=(0, 1), method="highs")
+    assert r.status == 0
+    return -r.fun, r.x.reshape(m, n)
+
+
+def _check_balanced(idx, m, n, k):
+    assert idx.shape == (m, k)
+    for row in idx:
+        assert len(set(row.tolist())) == k and (np.diff(row) > 0).all()
+    assert (np.bincount(idx.ravel(), minlength=n) == m * k // n).all()
+
+
+@pytest.mark.parametrize("case", range(30))
+def test_bruteforce_tiny(case):
+    shapes = [(8, 4, 1), (6, 3, 1), (6, 4, 2), (4, 4, 2), (8, 2, 1), (6, 3, 2)]
+    m, n, k = shapes[case % len(shapes)]
+    rng = np.random.default_rng(100 + case)
+    s = (rng.standard_normal((m, n)) + 1.5 * rng.standard_normal(n)).astype(np.float32)
+    for rule in (oracle.QB_MIDPOINT, oracle.QB_BOUNDARY):
+        idx, _, info, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, rule=rule, max_iters=case % 4)
+        assert rc == oracle.OK and info[2] == 0
+        _check_balanced(idx, m, n, k)
+        best, arg = _brute(s, k)
+        assert _objective(s, idx) == pytest.approx(best, abs=1e-9)
+        if len(arg) == 1:
+            assert [set(r.tolist()) for r in idx] == [set(c) for c in arg[0]]
+
+
+@pytest.mark.parametrize("m,n,k,iters,seed", [(512, 16, 2, 0, 0), (512, 16, 2, 5, 1), (1024, 8, 1, 3, 2),
+                                              (768, 32, 4, 10, 3), (600, 12, 3, 2, 4)])
+def test_lp_medium(m, n, k, iters, seed):
+    s = W.make_qb_scores(m, n, seed=seed)
+    idx, _, info, rc = oracle.balance_assign(s, k, max_iters=iters)
+    assert rc == oracle.OK and info[2] == 0
+    _check_balanced(idx, m, n, k)
+    obj, x = _lp(s, k)
+    assert _objective(s, idx) == pytest.approx(obj, rel=1e-12, abs=1e-7)
+    # continuous random scores: the LP optimum is a unique 0/1 vertex, equal to ours
+    assert np.allclose(x, np.round(x), atol=1e-7)
+    ours = np.zeros((m, n))
+    np.put_along_axis(ours, idx.astype(np.int64), 1.0, 1)
+    assert (ours == np.round(x)).all()
+    assert oracle.is_optimal(s, idx)
+
+
+def test_hungarian_k1():
+    m, n = 120, 6
+    s = W.make_qb_scores(m, n, seed=7)
+    idx, _, info, rc = oracle.balance_assign(s, 1, max_iters=1)
+    _check_balanced(idx, m, n, 1)
+    C = m // n
+    cost = -np.repeat(s.astype(np.float64), C, axis=1)  # each expert column repeated C times
+    r, c = linear_sum_assignment(cost)
+    assert _objective(s, idx) == pytest.approx(-cost[r, c].sum(), rel=1e-12)
+    assert (idx[r, 0] == c // C).all()
+
+
+def test_dual_subproblem_minima_closed_form():
+    # eqs. (10)-(11): min over alpha of k*alpha + sum_j max(0, v_j - alpha) is the sum of the k largest v_j,
+    # attained anywhere between the k-th and (k+1)-th largest -- both rules pick such a point.
+    m, n, k = 64, 16, 3
+    s = W.make_qb_scores(m, n, seed=9)
+    beta = np.random.default_rng(1).standard_normal(n).astype(np.float32)
+    v = (s - beta[None, :]).astype(np.float32)
+    for rule in (oracle.QB_MIDPOINT, oracle.QB_BOUNDARY):
+        alpha, idx, _ = oracle.qb_row(s, k, beta, rule)
+        vs = -np.sort(-v.astype(np.float64), axis=1)
+        g = k * alpha.astype(np.float64) + np.maximum(0, v.astype(np.float64) - alpha[:, None]).sum(1)
+        assert np.allclose(g, vs[:, :k].sum(1), rtol=1e-12, atol=1e-9)
+        assert ((alpha >= vs[:, k]) & (alpha <= vs[:, k - 1])).all()
+        if rule == oracle.QB_BOUNDARY:
+            assert (alpha == vs[:, k]).all()  # the page's convention: the (k+1)-th largest
+        # the selection is the top-k of s - beta (ties to the lower index), listed best first
+        for i in range(m):
+            assert idx[i].tolist() == sorted(range(n), key=lambda j: (-v[i, j], j))[:k]
+    C = m * k // n
+    alpha, _, _ = oracle.qb_row(s, k, beta)
+    u = (s - alpha[:, None]).astype(np.float32).astype(np.float64)
+    for rule in (oracle.QB_MIDPOINT, oracle.QB_BOUNDARY):
+        b = oracle.qb_col(s, k, alpha, rule).astype(np.float64)
+        us = -np.sort(-u, axis=0)
+        g = C * b + np.maximum(0, u - b[None, :]).sum(0)
+        assert np.allclose(g, us[:C].sum(0), rtol=1e-12, atol=1e-9)
+        assert ((b >= us[C]) & (b <= us[C - 1])).all()
+
+
+def test_midpoint_value_is_fp32_mean_of_neighbours():
+    s = np.array([[4.0, 1.0, 3.0, 2.0]], np.float32)
+    alpha, idx, _ = oracle.qb_row(s, 2, np.zeros(4, np.float32), oracle.QB_MIDPOINT)
+    assert alpha[0] == np.float32(2.5) and idx.tolist() == [[0, 2]]
+    alpha_b, _, _ = oracle.qb_row(s, 2, np.zeros(4, np.float32), oracle.QB_BOUNDARY)
+    assert alpha_b[0] == np.float32(2.0)
+
+
+def test_step_mode_selects_with_old_beta():
+    # Mind the pitfall: x comes from the old beta; beta is updated afterwards.
+    m, n, k = 256, 16, 2
+    s = W.make_qb_scores(m, n, seed=11)
+    beta_old = np.random.default_rng(2).standard_normal(n).astype(np.float32) * np.float32(0.5)
+    idx, beta_new, info, rc = oracle.balance_assign(s, k, beta=beta_old, mode=oracle.QB_STEP)
+    alpha, sel, _ = oracle.qb_row(s, k, beta_old)
+    assert (np.sort(sel, axis=1) == idx).all()
+    assert (oracle.qb_col(s, k, alpha) == beta_new).all()
+    assert info[0] == 1 and info[1] == 0
+
+
+def test_solve_balances_and_repair_optimal_on_skewed_scores():
+    m, n, k = 2048, 32, 4
+    s = W.make_qb_scores(m, n, seed=0)
+    _, idx0, _ = oracle.qb_row(s, k, np.zeros(n, np.float32))
+    before = np.bincount(idx0.ravel(), minlength=n)
+    idx, beta, info, rc = oracle.balance_assign(s, k, max_iters=8)
+    assert rc == oracle.OK
+    _check_balanced(idx, m, n, k)
+    assert before.max() > m * k // n  # plain top-k was unbalanced
+    assert oracle.is_optimal(s, idx)
+    # repair alone from plain top-k reaches the same optimum
+    idx_r, _, info_r, _ = oracle.balance_assign(s, k, max_iters=0)
+    assert info_r[1] > 0 and (idx_r == idx).all()
+
+
+def test_certificate_rejects_a_worse_assignment():
+    m, n, k = 256, 8, 2
+    s = W.make_qb_scores(m, n, seed=5)
+    idx, _, _, _ = oracle.balance_assign(s, k)
+    assert oracle.is_optimal(s, idx)
+    # swap: token a trades expert p for q and token b trades q for p (counts unchanged) -> a worse objective
+    bad = idx.copy()
+    for a in range(m):
+        for b in range(a + 1, m):
+            p = [e for e in bad[a] if e not in bad[b]]
+            q = [e for e in bad[b] if e not in bad[a]]
+            if p and q:
+                pa, qb = p[0], q[0]
+                gain = s[a, qb] + s[b, pa] - s[a, pa] - s[b, qb]
+                if gain < -1e-3:
+                    bad[a][bad[a] == pa] = qb
+                    bad[b][bad[b] == qb] = pa
+                    break
+        else:
+            continue
+        break
+    bad.sort(axis=1)
+    assert (np.bincount(bad.ravel(), minlength=n) == m * k // n).all()
+    assert _objective(s, bad) < _objective(s, idx)
+    assert not oracle.is_optimal(s, bad)
+
+
+def test_demo_claim_bias_evens_the_load():
+    # Demo code: scores rand(m,n) + rand(n); the top-k after subtracting the QB bias is far more even.
+    rng = np.random.default_rng(0)
+    m, n, k = 20000, 64, 8
+    s = (rng.random((m, n)) + rng.random(n)).astype(np.float32)
+    _, i0, _ = oracle.qb_row(s, k, np.zeros(n, np.float32))
+    v0 = oracle.balance_stats(None, i0, m, n, k, m)["vio"]
+    _, beta, _, _ = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=5, max_repair=0, check=False)
+    _, i1, _ = oracle.qb_row(s, k, beta)
+    v1 = oracle.balance_stats(None, i1, m, n, k, m)["vio"]
+    assert v0[0] > 1.0 and v1[0] < 0.1 * v0[0]
+
+
+def test_argument_errors():
+    s = W.make_qb_scores(10, 4, seed=0)
+    with pytest.raises(oracle.OracleError):
+        oracle.balance_assign(s, 1)  # m*k = 10 not divisible by n = 4
+    with pytest.raises(oracle.OracleError):
+        oracle.balance_assign(W.make_qb_scores(8, 4), 4)  # k must be < n
