@@ -1,0 +1,235 @@
+/*
+ * moe.h -- C ABI of a B200 (sm_100a) MoE-layer forward library.
+ *
+ * One forward pass of a Switch / top-k mixture-of-experts layer, split into the
+ * stages the layer is made of: router + top-k, optimal-assignment balancing,
+ * capacity slots, dispatch, expert FFN, combine, load statistics. Every stage
+ * runs in hand-written CUDA kernels; there is no host fallback.
+ *
+ * Conventions (all calls):
+ *  - Every array pointer is a DEVICE pointer owned by the caller; the library
+ *    never allocates device memory. Calls that need scratch take a `workspace`
+ *    of at least the size returned by the matching *_workspace_size() query
+ *    (which is a pure host function and may be called without a GPU).
+ *  - Arrays are dense and row-major; shapes are given as [rows, cols].
+ *    Integer arrays are int32, floating-point statistics fp32.
+ *  - Every call is asynchronous: it validates its arguments on the host,
+ *    enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns. It does not synchronise, except where stated.
+ *  - Return value: MOE_OK, or an error code; the message of the last error on
+ *    the calling thread is available from moe_last_error(). Invalid arguments
+ *    are rejected before anything is enqueued. Conditions only the device can
+ *    see (an expert index out of range, more kept rows than a buffer holds)
+ *    set a device error word that moe_sync_status() reports.
+ *  - Notation follows the pages: m tokens, n experts, k experts per token,
+ *    d model width, d_ff expert hidden width, scores s_ij, capacity C.
+ *  - Limits: 1 <= k <= n <= 256; d a multiple of 8 (bf16) or 4 (fp32);
+ *    d_ff a multiple of 8; m * k < 2^31.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_NOT_CONVERGED = 5,
+    MOE_ERR_INTERNAL = 6
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_SOFTMAX = 0, MOE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_QB_STEP = 0, MOE_QB_SOLVE = 1 } moe_qb_mode;
+typedef enum { MOE_QB_MIDPOINT = 0, MOE_QB_BOUNDARY = 1 } moe_qb_threshold;
+
+/* Copies the message of the calling thread's last error (NUL-terminated, truncated to len). */
+MOE_API void moe_last_error(char* buf, size_t len);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device. Returns MOE_OK, or MOE_ERR_INTERNAL / MOE_ERR_INVALID_ARG
+ * for a condition a kernel detected (the message says which), or MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_sync_status(moe_stream_t stream);
+
+/*
+ * Router and top-k selection.
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Switch
+ * Routing Steps 1-3 (h = x W_r, p = softmax(h), i* = argmax p, gate p_i*) and
+ * selective precision (router projection and softmax in fp32); the Shazeer
+ * gate Softmax(TopK(x W_g)) for k >= 2; "MoE travelogue 6"
+ * (kexue.fm/archives/11619), Method review eq. (1): Loss-Free ranks by
+ * rho + b and weights by rho.
+ *
+ *  x          [m, d] activations, dtype x_dtype (MOE_F32 or MOE_BF16); upcast to fp32.
+ *  w_r        [d, n] fp32 router weight.
+ *  logits_in  [m, n] fp32, or NULL. When given, x and w_r are ignored and h = logits_in.
+ *  fn         MOE_SOFTMAX: p = softmax(h); MOE_SIGMOID: rho = 1 / (1 + exp(-h)).
+ *  renorm_topk  softmax with k >= 2 only: gate = softmax over the k selected
+ *             logits (p_sel / sum of selected p); otherwise gate = p_sel.
+ *  rank_bias  [n] fp32 Loss-Free bias b, or NULL. Ranking key fp32(score) + b
+ *             (fp32 add); without it the key is h (softmax) or rho (sigmoid).
+ *  probs_out  [m, n] fp32 scores p or rho, or NULL.
+ *  topk_idx   [m, k] out: selected experts, best key first; equal keys -> lower index first.
+ *  topk_gate  [m, k] out: fp32 gates (rho_sel for sigmoid).
+ * All h, p, rho and keys are fp32. Errors: MOE_ERR_INVALID_ARG for bad shapes
+ * or NULL required pointers.
+ */
+MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, const float* logits_in, int64_t m,
+                           int32_t d, int32_t n, int32_t k, moe_score_fn fn, int32_t renorm_topk,
+                           const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
+                           moe_stream_t stream);
+
+/*
+ * Optimal-assignment balancing (Quantile Balancing) with an exact finish.
+ * Passage: "MoE travelogue 6: optimal assignment promotes balance"
+ * (kexue.fm/archives/11619): Linear programming eq. (3) (maximise sum x_ij s_ij
+ * with sum_j x_ij = k and sum_i x_ij = C = m k / n), the dual (8)-(11), the
+ * alternating QB algorithm box, and its practical one-step form under
+ * "Mind the pitfall" (select with the old beta, then update beta).
+ *
+ *  s          [m, n] fp32 scores. (m * k) % n must be 0 and k < n.
+ *  beta       [n] fp32, in: previous beta (zeros for a cold start); out: new beta.
+ *  mode       MOE_QB_STEP: x = topk(s - beta_old); one alpha/beta update -> beta_new.
+ *             MOE_QB_SOLVE: alternate row/column passes until topk(s - beta) has
+ *             every column count equal to C or max_iters beta updates are done,
+ *             then move the remaining excess with successive shortest paths on
+ *             the n-expert graph (at most max_repair moves), which yields the
+ *             optimum of eq. (3). beta returns the last QB beta.
+ *  rule       threshold between the two neighbouring order statistics:
+ *             MOE_QB_MIDPOINT fp32(fp32(a + b) * 0.5) (default) or
+ *             MOE_QB_BOUNDARY the (k+1)-th / (C+1)-th largest (the page's convention).
+ *  topk_idx   [m, k] out: each token's experts in ascending index order.
+ *  info       [4] int32 device out: beta updates done, repair moves, excess left
+ *             (0 = balanced), tokens whose k-th and (k+1)-th values of s - beta
+ *             tie in the last row pass.
+ * SOLVE synchronises `stream` between phases (its loop length depends on the
+ * data) and returns MOE_ERR_NOT_CONVERGED if max_repair moves did not remove
+ * the excess. STEP is fully asynchronous.
+ */
+MOE_API size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k, moe_qb_mode mode);
+MOE_API moe_status moe_balance_assign(const float* s, int64_t m, int32_t n, int32_t k, float* beta, moe_qb_mode mode,
+                              moe_qb_threshold rule, int32_t max_iters, int32_t max_repair, int32_t* topk_idx,
+                              int32_t* info, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Capacity slots and the expert-major row layout.
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Expert
+ * Capacity and token drop (capacity = tokens / experts x capacity factor;
+ * overflow skips the expert and rides the residual connection); "Switch
+ * Transformer read for implementation" (molayo1419.me), the dispatch
+ * permutation and the expert capacity example.
+ *
+ * Within each segment of seg_len tokens (a micro-batch; seg_len = m for one
+ * segment), the assignments (token i, pick r) are visited in token order; the
+ * j-th assignment to expert e (j from 0) gets slot j, kept iff j < capacity.
+ *  topk_idx       [m, k] expert ids (a token lists distinct experts).
+ *  capacity       per expert per segment (>= seg_len * k: nothing is dropped).
+ *  slot           [m, k] out: slot or -1 (dropped).
+ *  dest_row       [m, k] out: row in the expert-major buffer, or -1.
+ *  src_token      [m * k] out: src_token[row] = token; the first `rows` entries are
+ *                 written, rows = expert_offsets[n] (rows of expert e are
+ *                 expert_offsets[e] .. expert_offsets[e+1]-1, segment by segment,
+ *                 token order inside).
+ *  expert_offsets [n + 1] out; routed_count, kept_count [m / seg_len, n] out
+ *                 (routed = before capacity, kept = min(routed, capacity)).
+ * Errors: MOE_ERR_INVALID_ARG (seg_len must divide m, capacity >= 0),
+ * MOE_ERR_WORKSPACE. An expert id outside [0, n) sets the device error word.
+ */
+MOE_API size_t moe_capacity_slots_workspace_size(int64_t m, int32_t k, int32_t n, int64_t seg_len);
+MOE_API moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_t k, int32_t n, int32_t capacity,
+                              int64_t seg_len, int32_t* slot, int32_t* dest_row, int32_t* src_token,
+                              int32_t* expert_offsets, int32_t* routed_count, int32_t* kept_count, void* workspace,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Dispatch: gather tokens into expert-major order.
+ * Passage: "Switch Transformer read for implementation" (molayo1419.me), the
+ * forward pass changes token order twice (first: group tokens by expert).
+ *  x [m, d] (dtype dt) -> xbuf [max_rows, d]: xbuf[r] = x[src_token[r]] for
+ *  r < expert_offsets[n] (read on the device). max_rows is the capacity of xbuf
+ *  in rows; more kept rows than that set the device error word.
+ */
+MOE_API moe_status moe_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, const int32_t* src_token,
+                        const int32_t* expert_offsets, int32_t n, int64_t max_rows, void* xbuf, moe_stream_t stream);
+
+/*
+ * Expert FFN on the expert-major rows: for the rows of expert e,
+ *   ybuf = max(0, xbuf W1_e + b1_e) W2_e + b2_e.
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Switch
+ * Layer: FFN(x) = max(0, x W1 + b1) W2 + b2 replicated per expert.
+ *  xbuf [max_rows, d], ybuf [max_rows, d]: dtype dt; rows per expert from
+ *       expert_offsets [n+1] (device; rows = expert_offsets[n] <= max_rows).
+ *  w1   [n, d_ff, d]: W1_e stored output-major (the nn.Linear weight layout, row j
+ *       holds the weights of hidden unit j); b1 [n, d_ff].
+ *  w2   [n, d, d_ff]: W2_e output-major; b2 [n, d]. Weights and biases have dtype dt.
+ *  bf16: bf16 x bf16 products with fp32 accumulation on the tensor cores; the
+ *  hidden activation is rounded to bf16 between the two GEMMs.
+ *  fp32: fp32 FMA throughout.
+ *  workspace holds the hidden activations [max_rows, d_ff] (dtype dt).
+ */
+MOE_API size_t moe_expert_ffn_workspace_size(moe_dtype dt, int64_t max_rows, int32_t d_ff);
+MOE_API moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2,
+                          const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d, int32_t d_ff,
+                          int64_t max_rows, void* ybuf, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine: inverse permute, gate, and join the residual path.
+ * Passage: "Switch Transformer read for implementation" (molayo1419.me):
+ * restore token order, multiply by the gate, join the residual; overflow
+ * tokens keep only the residual. "Switch Transformers paper review", Step 3.
+ *  y[i] = (residual ? residual[i] : 0) + sum over r with dest_row[i,r] >= 0 of
+ *         g_ir * ybuf[dest_row[i,r]]
+ *  fp32 accumulation; for dt = MOE_BF16 each gate is first rounded to bf16 (the
+ *  selective-precision recipe casts the gate back to bf16). y [m, d] has dtype dt.
+ *  residual may be NULL; it must not alias y.
+ */
+MOE_API moe_status moe_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
+                       const void* residual, int64_t m, int32_t k, int32_t d, void* y, moe_stream_t stream);
+
+/*
+ * Load statistics, auxiliary loss and the Loss-Free bias update.
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), auxiliary
+ * load balancing loss L = alpha N sum_i f_i P_i; "Qwen global-batch load
+ * balance" (agentlenshq.com): per-micro-batch loss averaged vs f_i pooled over
+ * the global batch; "MoE travelogue 6", Demo code (MaxVio/MinVio/AvgVio) and
+ * eq. (2) (b <- b - gamma sign(F - 1/n)).
+ *
+ *  probs     [m, n] router scores (p or rho), or NULL (then P and aux are not written).
+ *  topk_idx  [m, k] routing decision (counts are taken before capacity).
+ *  seg_len   micro-batch length (divides m); nseg = m / seg_len.
+ *  f, P      [nseg + 1, n] out (row nseg: whole batch). f_i = count_i / (k m_seg).
+ *  aux       [nseg + 2] out: per segment, the mean over segments (micro-batch
+ *            loss), and the loss on pooled f and P (global-batch loss).
+ *  vio       [3] out: MaxVio, MinVio, AvgVio of the pooled counts, or NULL.
+ *  bias_inout [n] Loss-Free bias updated in place with step gamma, or NULL; the
+ *            sign is decided exactly from the integer counts.
+ * Accumulation is fp64 in a fixed order (the results are deterministic).
+ */
+MOE_API size_t moe_balance_stats_workspace_size(int64_t m, int32_t n, int64_t seg_len);
+MOE_API moe_status moe_balance_stats(const float* probs, const int32_t* topk_idx, int64_t m, int32_t n, int32_t k,
+                             int64_t seg_len, float alpha, float* f, float* P, float* aux, float* vio,
+                             float* bias_inout, float gamma, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,246 @@
+"""Python binding of the B200 MoE-layer forward library (libmoe_b200.so).
+
+Argument marshalling only: each function takes torch tensors, checks dtypes,
+devices and shapes, optionally allocates outputs and workspaces through torch
+(device memory is PyTorch's job here), and calls the C entry point of the same
+name on the current CUDA stream. Every step of the computation runs in the
+library's CUDA kernels; there is no fallback. If the library is missing, the
+import of any function raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_SOFTMAX, MOE_SIGMOID = 0, 1
+MOE_QB_STEP, MOE_QB_SOLVE = 0, 1
+MOE_QB_MIDPOINT, MOE_QB_BOUNDARY = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_NOT_CONVERGED", 6: "MOE_ERR_INTERNAL"}
+
+# every symbol the C header declares
+EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk", "moe_balance_assign_workspace_size",
+           "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
+           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
+           "moe_balance_stats")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libmoe_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m load_balanced_dispatch_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        P, I64, I32, F, SZ = C.c_void_p, C.c_int64, C.c_int32, C.c_float, C.c_size_t
+        L.moe_last_error.argtypes = [C.c_char_p, SZ]
+        L.moe_last_error.restype = None
+        L.moe_sync_status.argtypes = [P]
+        L.moe_router_topk.argtypes = [P, I32, P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, P]
+        L.moe_balance_assign_workspace_size.argtypes = [I64, I32, I32, I32]
+        L.moe_balance_assign_workspace_size.restype = SZ
+        L.moe_balance_assign.argtypes = [P, I64, I32, I32, P, I32, I32, I32, I32, P, P, P, SZ, P]
+        L.moe_capacity_slots_workspace_size.argtypes = [I64, I32, I32, I64]
+        L.moe_capacity_slots_workspace_size.restype = SZ
+        L.moe_capacity_slots.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P, SZ, P]
+        L.moe_dispatch.argtypes = [P, I32, I64, I32, P, P, I32, I64, P, P]
+        L.moe_expert_ffn_workspace_size.argtypes = [I32, I64, I32]
+        L.moe_expert_ffn_workspace_size.restype = SZ
+        L.moe_expert_ffn.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, SZ, P]
+        L.moe_combine.argtypes = [P, I32, P, P, P, I64, I32, I32, P, P]
+        L.moe_balance_stats_workspace_size.argtypes = [I64, I32, I64]
+        L.moe_balance_stats_workspace_size.restype = SZ
+        L.moe_balance_stats.argtypes = [P, P, I64, I32, I32, I64, F, P, P, P, P, P, F, P, SZ, P]
+        for name in EXPORTS:
+            if name not in ("moe_last_error",) and not name.endswith("_workspace_size"):
+                getattr(L, name).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    buf = C.create_string_buffer(512)
+    lib().moe_last_error(buf, 512)
+    return buf.value.decode()
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MoEError(fn, code, last_error())
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t, dtype, shape, name):
+    if t is None:
+        return
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def sync_status(stream=None):
+    """Synchronise the stream and raise if a kernel recorded a device-side error."""
+    _check("moe_sync_status", lib().moe_sync_status(_stream(stream)))
+
+
+def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias=None, logits_in=None,
+                    probs_out=None, topk_idx=None, topk_gate=None, want_probs=True, stream=None):
+    """Router + top-k. Returns (topk_idx [m,k] int32, topk_gate [m,k] fp32, probs [m,n] fp32 or None)."""
+    if logits_in is not None:
+        m, d = logits_in.shape[0], 0
+        dev = logits_in.device
+        _need(logits_in, torch.float32, (m, n), "logits_in")
+        xdt = MOE_F32
+    else:
+        m, d = x.shape
+        dev = x.device
+        xdt = _dtype_code(x)
+        _need(x, x.dtype, (m, d), "x")
+        _need(w_r, torch.float32, (d, n), "w_r")
+    _need(rank_bias, torch.float32, (n,), "rank_bias")
+    if topk_idx is None:
+        topk_idx = torch.empty((m, k), dtype=torch.int32, device=dev)
+    if topk_gate is None:
+        topk_gate = torch.empty((m, k), dtype=torch.float32, device=dev)
+    if probs_out is None and want_probs:
+        probs_out = torch.empty((m, n), dtype=torch.float32, device=dev)
+    _check("moe_router_topk", lib().moe_router_topk(
+        _ptr(x), xdt, _ptr(w_r), _ptr(logits_in), m, d, n, k, score_fn, renorm_topk, _ptr(rank_bias),
+        _ptr(probs_out), _ptr(topk_idx), _ptr(topk_gate), _stream(stream)))
+    return topk_idx, topk_gate, probs_out
+
+
+def moe_capacity_slots(topk_idx, n, capacity, seg_len=None, out=None, workspace=None, stream=None):
+    """Capacity slots. Returns dict(slot, dest_row, src_token, expert_offsets, routed_count, kept_count)."""
+    m, k = topk_idx.shape
+    seg_len = m if seg_len is None else seg_len
+    dev = topk_idx.device
+    nseg = m // seg_len if seg_len > 0 else 1
+    if out is None:
+        out = dict(slot=torch.empty((m, k), dtype=torch.int32, device=dev),
+                   dest_row=torch.empty((m, k), dtype=torch.int32, device=dev),
+                   src_token=torch.empty((m * k,), dtype=torch.int32, device=dev),
+                   expert_offsets=torch.empty((n + 1,), dtype=torch.int32, device=dev),
+                   routed_count=torch.empty((nseg, n), dtype=torch.int32, device=dev),
+                   kept_count=torch.empty((nseg, n), dtype=torch.int32, device=dev))
+    ws_bytes = lib().moe_capacity_slots_workspace_size(m, k, n, seg_len)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _check("moe_capacity_slots", lib().moe_capacity_slots(
+        _ptr(topk_idx), m, k, n, capacity, seg_len, _ptr(out["slot"]), _ptr(out["dest_row"]), _ptr(out["src_token"]),
+        _ptr(out["expert_offsets"]), _ptr(out["routed_count"]), _ptr(out["kept_count"]), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_dispatch(x, src_token, expert_offsets, n, max_rows=None, xbuf=None, stream=None):
+    """xbuf[r] = x[src_token[r]] for the kept rows (expert-major). Returns xbuf [max_rows, d]."""
+    m, d = x.shape
+    max_rows = src_token.numel() if max_rows is None else max_rows
+    if xbuf is None:
+        xbuf = torch.empty((max_rows, d), dtype=x.dtype, device=x.device)
+    _check("moe_dispatch", lib().moe_dispatch(_ptr(x), _dtype_code(x), m, d, _ptr(src_token), _ptr(expert_offsets),
+                                              n, max_rows, _ptr(xbuf), _stream(stream)))
+    return xbuf
+
+
+def moe_expert_ffn(xbuf, w1, b1, w2, b2, expert_offsets, ybuf=None, workspace=None, stream=None):
+    """ybuf = max(0, xbuf W1_e + b1_e) W2_e + b2_e per expert group. w1 [n,d_ff,d], w2 [n,d,d_ff]."""
+    max_rows, d = xbuf.shape
+    n, d_ff, _ = w1.shape
+    dt = _dtype_code(xbuf)
+    for t, shp, name in ((w1, (n, d_ff, d), "w1"), (b1, (n, d_ff), "b1"), (w2, (n, d, d_ff), "w2"), (b2, (n, d), "b2")):
+        _need(t, xbuf.dtype, shp, name)
+    if ybuf is None:
+        ybuf = torch.empty((max_rows, d), dtype=xbuf.dtype, device=xbuf.device)
+    ws_bytes = lib().moe_expert_ffn_workspace_size(dt, max_rows, d_ff)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=xbuf.device)
+    _check("moe_expert_ffn", lib().moe_expert_ffn(
+        _ptr(xbuf), dt, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(expert_offsets), n, d, d_ff, max_rows,
+        _ptr(ybuf), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return ybuf
+
+
+def moe_combine(ybuf, dest_row, topk_gate, residual=None, y=None, stream=None):
+    """y[i] = residual[i] + sum_r g_ir ybuf[dest_row[i,r]] (kept picks only). Returns y [m, d]."""
+    m, k = dest_row.shape
+    d = ybuf.shape[1]
+    if y is None:
+        y = torch.empty((m, d), dtype=ybuf.dtype, device=ybuf.device)
+    _check("moe_combine", lib().moe_combine(_ptr(ybuf), _dtype_code(ybuf), _ptr(dest_row), _ptr(topk_gate),
+                                            _ptr(residual), m, k, d, _ptr(y), _stream(stream)))
+    return y
+
+
+def moe_balance_stats(probs, topk_idx, n, seg_len=None, alpha=1e-2, bias_inout=None, gamma=1e-3, out=None,
+                      workspace=None, stream=None):
+    """f, P [nseg+1, n], aux [nseg+2], vio [3]; updates bias_inout in place when given."""
+    m, k = topk_idx.shape
+    seg_len = m if seg_len is None else seg_len
+    nseg = m // seg_len
+    dev = topk_idx.device
+    if out is None:
+        out = dict(f=torch.empty((nseg + 1, n), dtype=torch.float32, device=dev),
+                   P=torch.empty((nseg + 1, n), dtype=torch.float32, device=dev),
+                   aux=torch.empty((nseg + 2,), dtype=torch.float32, device=dev),
+                   vio=torch.empty((3,), dtype=torch.float32, device=dev))
+    ws_bytes = lib().moe_balance_stats_workspace_size(m, n, seg_len)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _check("moe_balance_stats", lib().moe_balance_stats(
+        _ptr(probs), _ptr(topk_idx), m, n, k, seg_len, alpha, _ptr(out["f"]), _ptr(out["P"] if probs is not None else None),
+        _ptr(out["aux"] if probs is not None else None), _ptr(out["vio"]), _ptr(bias_inout), gamma, _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_balance_assign(s, k, beta=None, mode=MOE_QB_SOLVE, rule=MOE_QB_MIDPOINT, max_iters=64, max_repair=1 << 20,
+                       topk_idx=None, info=None, workspace=None, stream=None):
+    """Balanced assignment. Returns (topk_idx [m,k] ascending experts, beta [n] (updated in place), info [4])."""
+    m, n = s.shape
+    dev = s.device
+    if beta is None:
+        beta = torch.zeros((n,), dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty((m, k), dtype=torch.int32, device=dev)
+    if info is None:
+        info = torch.zeros((4,), dtype=torch.int32, device=dev)
+    ws_bytes = lib().moe_balance_assign_workspace_size(m, n, k, mode)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _check("moe_balance_assign", lib().moe_balance_assign(
+        _ptr(s), m, n, k, _ptr(beta), mode, rule, max_iters, max_repair, _ptr(topk_idx), _ptr(info), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return topk_idx, beta, info

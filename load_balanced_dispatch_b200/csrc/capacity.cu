@@ -1,0 +1,203 @@
+// capacity.cu -- capacity slots and the expert-major row layout.
+//
+// Switch Transformers paper review (tildalice.io/?p=118), Expert Capacity and
+// token drop; Switch Transformer read for implementation (molayo1419.me), the
+// dispatch permutation and the capacity example: within a micro-batch, the
+// j-th assignment (in token order) to expert e gets slot j and is kept iff
+// j < capacity; overflow rides the residual path.
+//
+// Three launches over chunks of kChunk tokens (a chunk never straddles a
+// segment):
+//   count  -- per-chunk expert histogram (shared-memory integer atomics);
+//   scan   -- one CTA, thread e walks the chunks of every segment in order:
+//             chunk prefix within its segment, routed/kept counts, the
+//             expert offsets (block exclusive scan over e) and each
+//             (segment, expert) base row;
+//   assign -- per chunk, a stable in-order rank for every assignment
+//             (warp __match_any_sync groups + per-warp running counters in
+//             shared memory, warps owning consecutive sub-ranges), then
+//             slot / dest_row / src_token.
+// Everything is integer arithmetic: the result is exact and deterministic.
+#include "common.cuh"
+
+namespace moe {
+
+namespace cap {
+constexpr int kChunk = 256;   // tokens per chunk
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+}  // namespace cap
+
+struct CapGeometry {
+    int64_t nseg, cps, nchunks;
+};
+
+static CapGeometry cap_geometry(int64_t m, int64_t seg_len) {
+    CapGeometry g;
+    g.nseg = m / seg_len;
+    g.cps = (seg_len + cap::kChunk - 1) / cap::kChunk;
+    g.nchunks = g.nseg * g.cps;
+    return g;
+}
+
+size_t capacity_workspace_bytes(int64_t m, int32_t k, int32_t n, int64_t seg_len) {
+    (void)k;
+    if (seg_len <= 0) return 0;
+    CapGeometry g = cap_geometry(m, seg_len);
+    return sizeof(int32_t) * (size_t)n * (size_t)(2 * g.nchunks + g.nseg);
+}
+
+__device__ __forceinline__ void chunk_range(int64_t chunk, int64_t cps, int64_t seg_len, int64_t& seg, int64_t& t0,
+                                            int64_t& t1) {
+    seg = chunk / cps;
+    const int64_t c = chunk - seg * cps;
+    t0 = seg * seg_len + c * cap::kChunk;
+    t1 = min(t0 + (int64_t)cap::kChunk, (seg + 1) * seg_len);
+}
+
+__global__ void __launch_bounds__(cap::kThreads)
+cap_count_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg_len, int64_t cps,
+                 int32_t* __restrict__ hist) {
+    __shared__ int cnt[kMaxExperts];
+    for (int e = threadIdx.x; e < n; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    int64_t seg, t0, t1;
+    chunk_range(blockIdx.x, cps, seg_len, seg, t0, t1);
+    const int64_t a0 = t0 * k, a1 = t1 * k;
+    for (int64_t q = a0 + threadIdx.x; q < a1; q += blockDim.x) {
+        const int e = idx[q];
+        if (e < 0 || e >= n) record_error(kErrExpertIndex);
+        else atomicAdd(&cnt[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x) hist[(int64_t)blockIdx.x * n + e] = cnt[e];
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x == 256), in a fixed order.
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* sh, int64_t& total) {
+    const int tid = threadIdx.x;
+    sh[tid] = v;
+    __syncthreads();
+    for (int o = 1; o < cap::kThreads; o <<= 1) {
+        int64_t add = tid >= o ? sh[tid - o] : 0;
+        __syncthreads();
+        sh[tid] += add;
+        __syncthreads();
+    }
+    total = sh[cap::kThreads - 1];
+    return sh[tid] - v;
+}
+
+__global__ void __launch_bounds__(cap::kThreads)
+cap_scan_kernel(const int32_t* __restrict__ hist, int n, int64_t nseg, int64_t cps, int32_t capacity,
+                int32_t* __restrict__ prefix, int32_t* __restrict__ seg_base, int32_t* __restrict__ expert_offsets,
+                int32_t* __restrict__ routed_count, int32_t* __restrict__ kept_count) {
+    __shared__ int64_t sh[cap::kThreads];
+    const int e = threadIdx.x;
+    int64_t kept_total = 0;
+    if (e < n) {
+        for (int64_t s = 0; s < nseg; ++s) {
+            int64_t run = 0;
+            for (int64_t c = 0; c < cps; ++c) {
+                const int64_t ch = s * cps + c;
+                prefix[ch * n + e] = (int32_t)run;
+                run += hist[ch * n + e];
+            }
+            const int64_t kept = run < capacity ? run : (int64_t)capacity;
+            routed_count[s * n + e] = (int32_t)run;
+            kept_count[s * n + e] = (int32_t)kept;
+            kept_total += kept;
+        }
+    }
+    int64_t total;
+    const int64_t off = block_exclusive_scan(kept_total, sh, total);
+    if (e < n) {
+        expert_offsets[e] = (int32_t)off;
+        int64_t base = off;
+        for (int64_t s = 0; s < nseg; ++s) {
+            seg_base[s * n + e] = (int32_t)base;
+            base += kept_count[s * n + e];
+        }
+    }
+    if (e == 0) expert_offsets[n] = (int32_t)total;
+}
+
+__global__ void __launch_bounds__(cap::kThreads)
+cap_assign_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg_len, int64_t cps, int32_t capacity,
+                  const int32_t* __restrict__ prefix, const int32_t* __restrict__ seg_base,
+                  int32_t* __restrict__ slot, int32_t* __restrict__ dest_row, int32_t* __restrict__ src_token) {
+    __shared__ int wcnt[cap::kWarps][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int q = tid; q < cap::kWarps * kMaxExperts; q += cap::kThreads) (&wcnt[0][0])[q] = 0;
+    __syncthreads();
+    int64_t seg, t0, t1;
+    const int64_t chunk = blockIdx.x;
+    chunk_range(chunk, cps, seg_len, seg, t0, t1);
+    const int64_t a0 = t0 * k, A = (t1 - t0) * k;
+    const int64_t per_warp = (A + cap::kWarps - 1) / cap::kWarps;
+    const int64_t w0 = a0 + min((int64_t)warp * per_warp, A), w1 = a0 + min((int64_t)(warp + 1) * per_warp, A);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+
+    // pass 1: per-warp expert counts over the warp's contiguous sub-range
+    for (int64_t b = w0; b < w1; b += 32) {
+        const int64_t q = b + lane;
+        int e = q < w1 ? idx[q] : -1;
+        if (e >= n) e = -1;
+        const uint32_t grp = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (grp & lt_mask) == 0) wcnt[warp][e] += __popc(grp);
+    }
+    __syncthreads();
+    // exclusive prefix over warps, seeded with the chunk's prefix within its segment
+    for (int e = tid; e < n; e += cap::kThreads) {
+        int run = prefix[chunk * n + e];
+        for (int w = 0; w < cap::kWarps; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    // pass 2: ranks in order
+    for (int64_t b = w0; b < w1; b += 32) {
+        const int64_t q = b + lane;
+        int e = q < w1 ? idx[q] : -1;
+        if (e >= n) e = -1;
+        const uint32_t grp = __match_any_sync(0xffffffffu, e);
+        int rank = 0;
+        if (e >= 0) rank = wcnt[warp][e] + __popc(grp & lt_mask);
+        __syncwarp();
+        if (e >= 0 && (grp & lt_mask) == 0) wcnt[warp][e] += __popc(grp);
+        __syncwarp();
+        if (q < w1) {
+            int32_t sl = -1, dr = -1;
+            if (e >= 0 && rank < capacity) {
+                sl = rank;
+                dr = seg_base[seg * n + e] + rank;
+                src_token[dr] = (int32_t)(q / k);
+            }
+            slot[q] = sl;
+            dest_row[q] = dr;
+        }
+    }
+}
+
+cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, int32_t capacity, int64_t seg_len,
+                            int32_t* slot, int32_t* dest_row, int32_t* src_token, int32_t* expert_offsets,
+                            int32_t* routed_count, int32_t* kept_count, void* workspace, cudaStream_t stream) {
+    CapGeometry g = cap_geometry(m, seg_len);
+    int32_t* hist = static_cast<int32_t*>(workspace);
+    int32_t* prefix = hist + g.nchunks * n;
+    int32_t* seg_base = prefix + g.nchunks * n;
+    if (g.nchunks > 0) {
+        cap_count_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(topk_idx, k, n, seg_len, g.cps, hist);
+    }
+    cap_scan_kernel<<<1, cap::kThreads, 0, stream>>>(hist, n, g.nseg, g.cps, capacity, prefix, seg_base,
+                                                     expert_offsets, routed_count, kept_count);
+    if (g.nchunks > 0) {
+        cap_assign_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(
+            topk_idx, k, n, seg_len, g.cps, capacity, prefix, seg_base, slot, dest_row, src_token);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

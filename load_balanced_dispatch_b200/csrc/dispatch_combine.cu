@@ -1,0 +1,104 @@
+// dispatch_combine.cu -- the two permutations of the layer and the gated combine.
+//
+// Switch Transformer read for implementation (molayo1419.me): the forward pass
+// changes token order twice -- group tokens by expert before the FFN, restore
+// token order after it, multiply by the gate and join the residual path;
+// overflow tokens keep only the residual. Switch Transformers paper review
+// (tildalice.io/?p=118), Step 3: y = p_i* E_i*(x).
+//
+// Both kernels are HBM-bound row copies: one warp per row, 16-byte vectors,
+// grid sized to a multiple of the SM count and striding over rows.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRowThreads = 256;
+
+static unsigned row_grid(int64_t rows) {
+    const int64_t per_block = kRowThreads / 32;
+    int64_t blocks = (rows + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)kNumSMs * 16;
+    if (blocks > cap) blocks = cap;
+    return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+
+// xbuf[r] = x[src_token[r]] for r < expert_offsets[n]; raw 16-byte copies.
+__global__ void __launch_bounds__(kRowThreads)
+dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, const int32_t* __restrict__ src_token,
+                const int32_t* __restrict__ expert_offsets, int n, int64_t max_rows, uint4* __restrict__ xbuf) {
+    int64_t rows = expert_offsets[n];
+    if (rows > max_rows) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) record_error(kErrRowOverflow);
+        rows = max_rows;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
+    for (int64_t r = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int32_t t = src_token[r];
+        if (t < 0 || t >= m) {
+            if (lane == 0) record_error(kErrTokenIndex);
+            continue;
+        }
+        const uint4* src = x + (int64_t)t * vec_per_row;
+        uint4* dst = xbuf + r * vec_per_row;
+        for (int64_t c = lane; c < vec_per_row; c += 32) dst[c] = src[c];
+    }
+}
+
+// y[i] = (residual[i]) + sum_r g_ir * ybuf[dest_row[i,r]]  (fp32 accumulation).
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads)
+combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row, const float* __restrict__ gate,
+               const T* __restrict__ residual, int64_t m, int k, int d, int gate_bf16, T* __restrict__ y) {
+    constexpr int V = Vec16<T>::N;
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / V;
+    const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
+    for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
+        for (int c = lane; c < nvec; c += 32) {
+            float acc[V];
+            if (residual) Vec16<T>::load(residual + i * d + (int64_t)c * V, acc);
+            else
+#pragma unroll
+                for (int q = 0; q < V; ++q) acc[q] = 0.f;
+            for (int r = 0; r < k; ++r) {
+                const int32_t row = dest_row[i * k + r];
+                if (row < 0) continue;
+                float g = gate[i * k + r];
+                if (gate_bf16) g = round_to_bf16(g);
+                float v[V];
+                Vec16<T>::load(ybuf + (int64_t)row * d + (int64_t)c * V, v);
+#pragma unroll
+                for (int q = 0; q < V; ++q) acc[q] = fmaf(g, v[q], acc[q]);
+            }
+            Vec16<T>::store(y + i * d + (int64_t)c * V, acc);
+        }
+    }
+}
+
+cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const int32_t* src_token,
+                            const int32_t* expert_offsets, int n, int64_t max_rows, void* xbuf,
+                            cudaStream_t stream) {
+    const int64_t bytes_per_row = (int64_t)d * (dt == MOE_BF16 ? 2 : 4);
+    dispatch_kernel<<<row_grid(max_rows), kRowThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), m, bytes_per_row / 16, src_token, expert_offsets, n, max_rows,
+        static_cast<uint4*>(xbuf));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
+                           const void* residual, int64_t m, int k, int d, void* y, cudaStream_t stream) {
+    if (m == 0) return cudaSuccess;
+    if (dt == MOE_BF16) {
+        combine_kernel<__nv_bfloat16><<<row_grid(m), kRowThreads, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(ybuf), dest_row, topk_gate,
+            static_cast<const __nv_bfloat16*>(residual), m, k, d, 1, static_cast<__nv_bfloat16*>(y));
+    } else {
+        combine_kernel<float><<<row_grid(m), kRowThreads, 0, stream>>>(
+            static_cast<const float*>(ybuf), dest_row, topk_gate, static_cast<const float*>(residual), m, k, d, 0,
+            static_cast<float*>(y));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

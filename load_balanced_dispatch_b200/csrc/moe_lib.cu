@@ -1,0 +1,10 @@
+// moe_lib.cu -- single translation unit of the library (one device error word
+// shared by every kernel without relocatable device code).
+#include "api.cu"
+#include "balance.cu"
+#include "capacity.cu"
+#include "dispatch_combine.cu"
+#include "ffn.cu"
+#include "ffn_simt.cu"
+#include "router.cu"
+#include "stats.cu"

@@ -1,0 +1,232 @@
+// router.cu -- router projection h = x W_r (fp32), score function, top-k and gates.
+//
+// Switch Transformers paper review (tildalice.io/?p=118), Switch Routing Steps
+// 1-3 with selective precision (projection and softmax in fp32); the Shazeer
+// gate Softmax(TopK(.)) for k >= 2; MoE travelogue 6 (kexue.fm/archives/11619)
+// eq. (1): a Loss-Free bias enters the ranking only.
+//
+// One CTA computes the fp32 logits of TM tokens against all n <= 256 experts
+// with SIMT FMAs (K-tiles of x and W_r staged in shared memory), parks the
+// logit tile in shared memory, and one warp per token row finishes the row in
+// registers: max/exp/sum (softmax) or the logistic function, the ranking key,
+// k rounds of a warp arg-max (ties -> lower index) and the gates. Logits never
+// reach HBM.
+#include "common.cuh"
+
+namespace moe {
+
+namespace router {
+constexpr int TM = 32;       // tokens per CTA
+constexpr int TK = 32;       // K-tile
+constexpr int XS = TM + 1;   // padded stride of the transposed x tile
+constexpr int kThreads = 256;
+}  // namespace router
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, int64_t avail, float* out);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, int64_t avail, float* out) {
+    if (avail >= 4 && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+        float4 v = *reinterpret_cast<const float4*>(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) out[q] = q < avail ? p[q] : 0.f;
+    }
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, int64_t avail, float* out) {
+    if (avail >= 4 && (reinterpret_cast<uintptr_t>(p) & 7) == 0) {
+        uint2 v = *reinterpret_cast<const uint2*>(p);
+        out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+        out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) out[q] = q < avail ? __bfloat162float(p[q]) : 0.f;
+    }
+}
+
+// Finish one token row held by a warp: lane owns experts j = lane + 32 q (q < NT).
+template <int NT>
+__device__ __forceinline__ void finish_row(const float (&h)[NT], int64_t row, int n, int k, int fn, int renorm,
+                                           const float* rank_bias, float* probs_out, int32_t* topk_idx,
+                                           float* topk_gate) {
+    const int lane = threadIdx.x & 31;
+    float p[NT], key[NT];
+    if (fn == MOE_SOFTMAX) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < NT; ++q) if (lane + 32 * q < n) mx = fmaxf(mx, h[q]);
+        mx = warp_max(mx);
+        float s = 0.f;
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+            p[q] = (lane + 32 * q < n) ? expf(h[q] - mx) : 0.f;
+            s += p[q];
+        }
+        s = warp_sum(s);
+#pragma unroll
+        for (int q = 0; q < NT; ++q) p[q] = p[q] / s;
+    } else {
+#pragma unroll
+        for (int q = 0; q < NT; ++q) p[q] = 1.f / (1.f + expf(-h[q]));
+    }
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+        const int j = lane + 32 * q;
+        if (j >= n) { key[q] = -INFINITY; continue; }
+        if (rank_bias) key[q] = __fadd_rn(p[q], rank_bias[j]);
+        else key[q] = (fn == MOE_SOFTMAX) ? h[q] : p[q];
+    }
+    if (probs_out) {
+#pragma unroll
+        for (int q = 0; q < NT; ++q)
+            if (lane + 32 * q < n) probs_out[row * n + lane + 32 * q] = p[q];
+    }
+    uint32_t taken = 0;
+    float selsum = 0.f;
+    float mysel_p = 0.f;   // lane r (< k) keeps the score of pick r
+    int mysel_i = 0;
+    for (int r = 0; r < k; ++r) {
+        float bk = -INFINITY;
+        int bi = 0x7fffffff;
+        float bp = 0.f;
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+            const int j = lane + 32 * q;
+            if (j < n && !(taken & (1u << q)) && ranks_before(key[q], j, bk, bi)) { bk = key[q]; bi = j; bp = p[q]; }
+        }
+        float wk = bk;
+        int wi = bi;
+        warp_best(wk, wi);
+        const int owner = wi & 31;
+        if (lane == owner && wi < n) taken |= 1u << (wi >> 5);
+        const float wp = __shfl_sync(0xffffffffu, bp, owner);
+        selsum += wp;
+        if (r < 32 && lane == r) { mysel_p = wp; mysel_i = wi; }
+        if (r >= 32 && lane == 0) {  // k > 32: write picks beyond the first 32 as they come
+            topk_idx[row * k + r] = wi;
+            topk_gate[row * k + r] = wp;  // divided by the selected sum below when renormalising
+        }
+    }
+    if (lane < k && lane < 32) {
+        topk_idx[row * k + lane] = mysel_i;
+        topk_gate[row * k + lane] = (fn == MOE_SOFTMAX && renorm) ? mysel_p / selsum : mysel_p;
+    }
+    if (k > 32 && fn == MOE_SOFTMAX && renorm) {
+        __syncwarp();
+        for (int r = 32 + lane; r < k; r += 32) topk_gate[row * k + r] = topk_gate[row * k + r] / selsum;
+    }
+}
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(router::kThreads)
+router_topk_kernel(const T* __restrict__ x, const float* __restrict__ w_r, const float* __restrict__ logits_in,
+                   int64_t m, int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
+                   float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+    using namespace router;
+    constexpr int NPAD = 32 * NT;
+    __shared__ __align__(16) float smem[(TK * XS + TK * NPAD) > (TM * (NPAD + 1)) ? (TK * XS + TK * NPAD)
+                                                                                   : (TM * (NPAD + 1))];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row0 = (int64_t)blockIdx.x * TM;
+
+    if (logits_in) {
+        for (int rr = warp; rr < TM; rr += kThreads / 32) {
+            const int64_t row = row0 + rr;
+            if (row >= m) break;
+            float h[NT];
+#pragma unroll
+            for (int q = 0; q < NT; ++q) h[q] = (lane + 32 * q < n) ? logits_in[row * n + lane + 32 * q] : 0.f;
+            finish_row<NT>(h, row, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+        }
+        return;
+    }
+
+    float* xs = smem;              // [TK][XS]: x tile transposed (k-major)
+    float* ws = smem + TK * XS;    // [TK][NPAD]
+    const int tx = lane, ty = warp;  // thread computes tokens ty*4 .. ty*4+3, experts tx + 32 q
+    float acc[4][NT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < NT; ++q) acc[i][q] = 0.f;
+
+    const int lr = tid >> 3, lc = tid & 7;  // x tile loader: row lr, k-chunk lc (4 elements)
+    for (int k0 = 0; k0 < d; k0 += TK) {
+        {
+            const int64_t gr = row0 + lr;
+            const int gk = k0 + lc * 4;
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            if (gr < m && gk < d) load4<T>(x + gr * d + gk, d - gk, v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xs[(lc * 4 + q) * XS + lr] = v[q];
+        }
+        for (int e = tid; e < TK * NPAD; e += kThreads) {
+            const int kk = e / NPAD, j = e - kk * NPAD;
+            const int gk = k0 + kk;
+            ws[e] = (gk < d && j < n) ? w_r[(int64_t)gk * n + j] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < TK; ++kk) {
+            float xv[4], wv[NT];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[i] = xs[kk * XS + ty * 4 + i];
+#pragma unroll
+            for (int q = 0; q < NT; ++q) wv[q] = ws[kk * NPAD + tx + 32 * q];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < NT; ++q) acc[i][q] = fmaf(xv[i], wv[q], acc[i][q]);
+        }
+        __syncthreads();
+    }
+    float* lg = smem;  // [TM][NPAD+1]
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < NT; ++q) lg[(ty * 4 + i) * (NPAD + 1) + tx + 32 * q] = acc[i][q];
+    __syncthreads();
+    for (int rr = warp; rr < TM; rr += kThreads / 32) {
+        const int64_t row = row0 + rr;
+        if (row >= m) break;
+        float h[NT];
+#pragma unroll
+        for (int q = 0; q < NT; ++q) h[q] = lg[rr * (NPAD + 1) + lane + 32 * q];
+        finish_row<NT>(h, row, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    }
+}
+
+template <typename T, int NT>
+static cudaError_t launch_router_t(const void* x, const float* w_r, const float* logits_in, int64_t m, int d, int n,
+                                   int k, int fn, int renorm, const float* rank_bias, float* probs_out,
+                                   int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    const int64_t blocks = (m + router::TM - 1) / router::TM;
+    if (blocks == 0) return cudaSuccess;
+    router_topk_kernel<T, NT><<<(unsigned)blocks, router::kThreads, 0, stream>>>(
+        static_cast<const T*>(x), w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_router_dt(const void* x, const float* w_r, const float* logits_in, int64_t m, int d, int n,
+                                    int k, int fn, int renorm, const float* rank_bias, float* probs_out,
+                                    int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    if (n <= 32) return launch_router_t<T, 1>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+    if (n <= 64) return launch_router_t<T, 2>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+    if (n <= 128) return launch_router_t<T, 4>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+    return launch_router_t<T, 8>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+}
+
+cudaError_t launch_router(const void* x, moe_dtype dt, const float* w_r, const float* logits_in, int64_t m, int d,
+                          int n, int k, int fn, int renorm, const float* rank_bias, float* probs_out,
+                          int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    if (dt == MOE_BF16)
+        return launch_router_dt<__nv_bfloat16>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out,
+                                               topk_idx, topk_gate, stream);
+    return launch_router_dt<float>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
+                                   topk_gate, stream);
+}
+
+}  // namespace moe

@@ -1,0 +1,107 @@
+"""One MoE-layer forward through the C ABI: buffers owned by torch, stages run in order.
+
+The runner only allocates device buffers once and calls the library's entry
+points in the order the layer defines (router -> [balance] -> capacity ->
+dispatch -> expert FFN -> combine -> statistics). All arithmetic happens in
+the library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import (MOE_QB_MIDPOINT, MOE_QB_STEP, MOE_SIGMOID, MOE_SOFTMAX, moe_balance_assign, moe_balance_stats,
+               moe_capacity_slots, moe_combine, moe_dispatch, moe_expert_ffn, moe_router_topk, lib)
+
+
+@dataclass
+class LayerShape:
+    m: int
+    d: int
+    n: int
+    k: int
+    d_ff: int
+    score_fn: str = "softmax"
+    dtype: torch.dtype = torch.bfloat16
+    capacity: int = 0
+    seg_len: int = 0
+    renorm_topk: int = 0
+    alpha: float = 1e-2
+    gamma: float = 1e-3
+    residual: bool = False
+    lossfree: bool = False   # update the Loss-Free ranking bias after each forward
+
+
+class MoELayer:
+    """Device-resident weights and preallocated buffers for repeated forwards."""
+
+    def __init__(self, shape: LayerShape, weights: dict, device="cuda"):
+        s = self.shape = shape
+        self.device = torch.device(device)
+        self.w = weights  # x-independent tensors on the device: w_r, w1, b1, w2, b2, rank_bias (optional)
+        m, n, k, d = s.m, s.n, s.k, s.d
+        seg = s.seg_len or m
+        self.seg_len = seg
+        nseg = m // seg
+        dev = self.device
+        i32, f32 = torch.int32, torch.float32
+        self.rows_max = m * k
+        self.buf = dict(
+            topk_idx=torch.empty((m, k), dtype=i32, device=dev),
+            topk_gate=torch.empty((m, k), dtype=f32, device=dev),
+            probs=torch.empty((m, n), dtype=f32, device=dev),
+            slot=torch.empty((m, k), dtype=i32, device=dev),
+            dest_row=torch.empty((m, k), dtype=i32, device=dev),
+            src_token=torch.empty((m * k,), dtype=i32, device=dev),
+            expert_offsets=torch.empty((n + 1,), dtype=i32, device=dev),
+            routed_count=torch.empty((nseg, n), dtype=i32, device=dev),
+            kept_count=torch.empty((nseg, n), dtype=i32, device=dev),
+            xbuf=torch.empty((self.rows_max, d), dtype=s.dtype, device=dev),
+            ybuf=torch.empty((self.rows_max, d), dtype=s.dtype, device=dev),
+            y=torch.empty((m, d), dtype=s.dtype, device=dev),
+            f=torch.empty((nseg + 1, n), dtype=f32, device=dev),
+            P=torch.empty((nseg + 1, n), dtype=f32, device=dev),
+            aux=torch.empty((nseg + 2,), dtype=f32, device=dev),
+            vio=torch.empty((3,), dtype=f32, device=dev),
+        )
+        L = lib()
+        dt = 1 if s.dtype == torch.bfloat16 else 0
+        self.ws = dict(
+            cap=torch.empty((max(L.moe_capacity_slots_workspace_size(m, k, n, seg), 1),), dtype=torch.uint8, device=dev),
+            ffn=torch.empty((L.moe_expert_ffn_workspace_size(dt, self.rows_max, s.d_ff),), dtype=torch.uint8,
+                            device=dev),
+            stats=torch.empty((max(L.moe_balance_stats_workspace_size(m, n, seg), 1),), dtype=torch.uint8,
+                              device=dev),
+        )
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        s, b, w = self.shape, self.buf, self.w
+        fn = MOE_SOFTMAX if s.score_fn == "softmax" else MOE_SIGMOID
+        moe_router_topk(x, w["w_r"], s.n, s.k, fn, s.renorm_topk, rank_bias=w.get("rank_bias"), probs_out=b["probs"],
+                        topk_idx=b["topk_idx"], topk_gate=b["topk_gate"], stream=stream)
+        cap = moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"],
+                                 stream=stream)
+        moe_dispatch(x, cap["src_token"], cap["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=stream)
+        moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], cap["expert_offsets"], ybuf=b["ybuf"],
+                       workspace=self.ws["ffn"], stream=stream)
+        moe_combine(b["ybuf"], cap["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
+                    stream=stream)
+        moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
+                          bias_inout=w.get("rank_bias") if s.lossfree else None, gamma=s.gamma, out=b,
+                          workspace=self.ws["stats"], stream=stream)
+        return b["y"]
+
+    # kernel launches per forward (router 1, capacity 3, dispatch 1, FFN 2, combine 1, stats 2)
+    launches_per_forward = 10
+
+
+def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:
+    """Move numpy inputs from `workloads.make_layer_inputs` to the device (bf16-representable values convert exactly)."""
+    out = {}
+    for key in ("w1", "b1", "w2", "b2"):
+        out[key] = torch.from_numpy(inp[key]).to(device=device, dtype=dtype).contiguous()
+    out["w_r"] = torch.from_numpy(inp["w_r"]).to(device=device, dtype=torch.float32).contiguous()
+    if inp.get("rank_bias") is not None:
+        out["rank_bias"] = torch.from_numpy(inp["rank_bias"]).to(device=device, dtype=torch.float32).contiguous()
+    return out

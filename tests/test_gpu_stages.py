@@ -1,0 +1,222 @@
+"""Per-call parity of the CUDA library against the CPU oracle, on the same seeded inputs.
+
+Integer outputs (selections, slots, rows, counts) and fp32 decisions are
+bit-exact; floating-point values are within the stated tolerances. Sizes span
+several tiles and a ragged tail; edge cases: empty experts, capacity 0 and
+>= m, k = n - 1, ties, several segments.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from gpu_util import MARGIN, TOL_STATS, dev, host, norm_err, tol, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+lb = pytest.importorskip("load_balanced_dispatch_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from load_balanced_dispatch_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    yield
+    lb.sync_status()
+
+
+# ---------------------------------------------------------------- router
+@pytest.mark.parametrize("m,n,k,renorm", [(1000, 8, 1, 0), (777, 64, 2, 1), (513, 128, 1, 0), (300, 200, 6, 0),
+                                          (256, 256, 8, 1), (97, 16, 15, 0), (64, 256, 40, 1)])
+def test_router_logits_in_softmax_bitexact(m, n, k, renorm):
+    rng = np.random.default_rng(m + n)
+    logits = rng.standard_normal((m, n)).astype(np.float32)
+    logits[::7] = np.round(logits[::7] * 2) / 2  # exact ties on some rows
+    p_ref, i_ref, g_ref, _ = oracle.router(None, None, m, 0, n, k, renorm=renorm, logits_in=logits)
+    idx, gate, probs = lb.moe_router_topk(None, None, n, k, lb.MOE_SOFTMAX, renorm, logits_in=dev(logits))
+    torch.cuda.synchronize()
+    assert (host(idx) == i_ref).all()
+    assert np.allclose(host(gate), g_ref, rtol=1e-5, atol=1e-7)
+    assert np.allclose(host(probs), p_ref, rtol=1e-5, atol=1e-8)
+
+
+@pytest.mark.parametrize("m,n,k,bias", [(1000, 64, 6, True), (333, 32, 4, False), (128, 256, 8, True)])
+def test_router_logits_in_sigmoid(m, n, k, bias):
+    rng = np.random.default_rng(n + k)
+    logits = rng.standard_normal((m, n)).astype(np.float32)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32) if bias else None
+    p_ref, i_ref, g_ref, margin = oracle.router(None, None, m, 0, n, k, fn=oracle.SIGMOID, rank_bias=b,
+                                                logits_in=logits)
+    idx, gate, probs = lb.moe_router_topk(None, None, n, k, lb.MOE_SIGMOID, 0, rank_bias=None if b is None else dev(b),
+                                          logits_in=dev(logits))
+    torch.cuda.synchronize()
+    ok = margin > MARGIN
+    assert ok.mean() > 0.9
+    assert (host(idx)[ok] == i_ref[ok]).all()
+    assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-6)
+    assert np.allclose(host(probs), p_ref, rtol=1e-6)
+
+
+@pytest.mark.parametrize("dtype,m,d,n,k", [("fp32", 1000, 64, 8, 1), ("bf16", 517, 768, 128, 1),
+                                           ("bf16", 300, 200, 64, 6), ("fp32", 129, 36, 256, 8)])
+def test_router_projection(dtype, m, d, n, k):
+    rng = np.random.default_rng(d)
+    x = rng.standard_normal((m, d)).astype(np.float32)
+    if dtype == "bf16":
+        x = W.round_to_bf16(x)
+    w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
+    p_ref, i_ref, g_ref, margin = oracle.router(x, w, m, d, n, k)
+    idx, gate, probs = lb.moe_router_topk(dev(x, torch_dtype(dtype)), dev(w), n, k)
+    torch.cuda.synchronize()
+    ok = margin > MARGIN
+    assert ok.mean() > 0.97
+    assert (host(idx)[ok] == i_ref[ok]).all()
+    assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-5)
+    assert np.allclose(host(probs), p_ref, rtol=1e-5, atol=1e-9)
+
+
+# ---------------------------------------------------------------- capacity
+@pytest.mark.parametrize("m,n,k,cap,seg", [(1000, 8, 1, 160, 1000), (8192, 128, 1, 80, 8192), (4096, 64, 2, 256, 512),
+                                           (777, 16, 3, 40, 777), (1536, 256, 8, 30, 256), (600, 5, 2, 0, 300),
+                                           (300, 4, 2, 10 ** 6, 100), (64, 64, 63, 1, 64)])
+def test_capacity_bitexact(m, n, k, cap, seg):
+    idx = W.make_topk_idx(m, n, k, seed=m * 7 + n)
+    ref = oracle.capacity(idx, m, k, n, cap, seg)
+    out = lb.moe_capacity_slots(dev(idx), n, cap, seg)
+    torch.cuda.synchronize()
+    rows = int(ref["expert_offsets"][-1])
+    for key in ("slot", "dest_row", "expert_offsets", "routed_count", "kept_count"):
+        assert (host(out[key]) == ref[key]).all(), key
+    assert (host(out["src_token"])[:rows] == ref["src_token"][:rows]).all()
+
+
+def test_capacity_golden_example(golden):
+    g = golden("capacity_example.txt")
+    routed = [int(v) for v in g["routed"]]
+    route = np.concatenate([np.full(c, e) for e, c in enumerate(routed)])
+    route = np.random.default_rng(0).permutation(route).astype(np.int32)[:, None]
+    for cf in ("1.0", "1.25"):
+        out = lb.moe_capacity_slots(dev(route), 4, int(g["capacity_" + cf][0]))
+        assert host(out["kept_count"])[0].tolist() == [int(v) for v in g["kept_" + cf]]
+        assert int((host(out["slot"]) < 0).sum()) == int(g["dropped_" + cf][0])
+
+
+def test_capacity_rejects_bad_expert_ids():
+    idx = np.array([[0], [9], [1]], np.int32)
+    lb.moe_capacity_slots(dev(idx), 4, 8)
+    with pytest.raises(lb.MoEError):
+        lb.sync_status()
+
+
+# ---------------------------------------------------------------- dispatch / combine
+@pytest.mark.parametrize("dtype,m,d,n,k,cap", [("bf16", 1000, 768, 16, 2, 100), ("fp32", 513, 64, 8, 1, 80),
+                                               ("bf16", 300, 4096, 64, 2, 0)])
+def test_dispatch_combine(dtype, m, d, n, k, cap):
+    rng = np.random.default_rng(d)
+    x = rng.standard_normal((m, d)).astype(np.float32)
+    if dtype == "bf16":
+        x = W.round_to_bf16(x)
+    idx = W.make_topk_idx(m, n, k, seed=1)
+    ref = oracle.capacity(idx, m, k, n, cap, m)
+    rows = int(ref["expert_offsets"][-1])
+    td = torch_dtype(dtype)
+    xd = dev(x, td)
+    out = lb.moe_capacity_slots(dev(idx), n, cap)
+    xbuf = lb.moe_dispatch(xd, out["src_token"], out["expert_offsets"], n, m * k)
+    torch.cuda.synchronize()
+    assert (host(xbuf)[:rows] == oracle.dispatch(x, ref["src_token"], rows)).all()
+    ybuf = rng.standard_normal((m * k, d)).astype(np.float32)
+    if dtype == "bf16":
+        ybuf = W.round_to_bf16(ybuf)
+    gate = rng.random((m, k)).astype(np.float32)
+    for residual in (None, xd):
+        y = lb.moe_combine(dev(ybuf, td), out["dest_row"], dev(gate), residual=residual)
+        torch.cuda.synchronize()
+        y_ref = oracle.combine(ybuf[:max(rows, 1)] if rows else np.zeros((1, d)), ref["dest_row"], gate,
+                               None if residual is None else x, m, k, d, gate_bf16=int(dtype == "bf16"))
+        assert norm_err(host(y), y_ref) <= (2 ** -8 if dtype == "bf16" else 1e-6)
+
+
+# ---------------------------------------------------------------- expert FFN
+@pytest.mark.parametrize("dtype,rows_per,d,d_ff", [("fp32", [100, 0, 37, 256, 1], 64, 256),
+                                                   ("bf16", [64, 80, 0, 3, 129, 77], 768, 3072),
+                                                   ("bf16", [130, 1, 0, 256], 2048, 1408),
+                                                   ("bf16", [0, 300], 256, 512)])
+def test_expert_ffn(dtype, rows_per, d, d_ff):
+    n = len(rows_per)
+    rng = np.random.default_rng(d + d_ff)
+    off = np.concatenate([[0], np.cumsum(rows_per)]).astype(np.int32)
+    rows = int(off[-1])
+    max_rows = rows + 19
+    st = (lambda a: W.round_to_bf16(a)) if dtype == "bf16" else (lambda a: a.astype(np.float32))
+    xbuf = st(rng.standard_normal((max_rows, d)).astype(np.float32))
+    w1 = st((rng.standard_normal((n, d_ff, d)) / np.sqrt(d)).astype(np.float32))
+    b1 = st((0.1 * rng.standard_normal((n, d_ff))).astype(np.float32))
+    w2 = st((rng.standard_normal((n, d, d_ff)) / np.sqrt(d_ff)).astype(np.float32))
+    b2 = st((0.1 * rng.standard_normal((n, d))).astype(np.float32))
+    td = torch_dtype(dtype)
+    ybuf = lb.moe_expert_ffn(dev(xbuf, td), dev(w1, td), dev(b1, td), dev(w2, td), dev(b2, td), dev(off))
+    torch.cuda.synchronize()
+    ref = oracle.expert_ffn(xbuf[:rows], off, w1, b1, w2, b2)
+    assert norm_err(host(ybuf)[:rows], ref) <= tol(dtype)
+
+
+# ---------------------------------------------------------------- statistics
+@pytest.mark.parametrize("m,n,k,seg", [(8192, 128, 1, 8192), (65536, 64, 2, 4096), (1000, 8, 1, 250),
+                                       (777, 256, 8, 777)])
+def test_balance_stats(m, n, k, seg):
+    rng = np.random.default_rng(n)
+    p = rng.random((m, n)).astype(np.float32)
+    p /= p.sum(1, keepdims=True)
+    idx = W.make_topk_idx(m, n, k, seed=3)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32)
+    ref = oracle.balance_stats(p, idx, m, n, k, seg, 1e-2, bias=b, gamma=1e-3)
+    bd = dev(b)
+    out = lb.moe_balance_stats(dev(p), dev(idx), n, seg, 1e-2, bias_inout=bd, gamma=1e-3)
+    torch.cuda.synchronize()
+    assert (host(out["f"]) == ref["f"].astype(np.float32)).all()
+    assert np.allclose(host(out["P"]), ref["P"], rtol=TOL_STATS, atol=0)
+    assert np.allclose(host(out["aux"]), ref["aux"], rtol=TOL_STATS, atol=0)
+    assert np.allclose(host(out["vio"]), ref["vio"], rtol=1e-6, atol=1e-7)
+    assert (host(bd) == ref["bias"]).all()
+
+
+def test_balance_stats_golden_identity(golden):
+    g = golden("aux_balanced.txt")
+    for n in (int(v) for v in g["experts"]):
+        m = 4 * n
+        out = lb.moe_balance_stats(dev(W.make_uniform_probs(m, n)), dev(W.make_round_robin_idx(m, n, 2)), n, m // 2,
+                                   float(g["alpha"][0]))
+        torch.cuda.synchronize()
+        assert (host(out["aux"]) == np.float32(g["expected_aux"][0])).all()
+        assert (host(out["vio"]) == 0).all()
+
+
+# ---------------------------------------------------------------- balanced assignment
+@pytest.mark.parametrize("m,n,k,rule", [(2048, 32, 4, 0), (4096, 64, 6, 1), (1000, 8, 2, 0), (768, 256, 8, 0),
+                                        (2560, 16, 15, 0)])
+def test_balance_step_bitexact(m, n, k, rule):
+    s = W.make_qb_scores(m, n, seed=m + k)
+    beta0 = (0.3 * np.random.default_rng(5).standard_normal(n)).astype(np.float32)
+    i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=beta0, mode=oracle.QB_STEP, rule=rule)
+    idx, beta, info = lb.moe_balance_assign(dev(s), k, beta=dev(beta0), mode=lb.MOE_QB_STEP, rule=rule)
+    torch.cuda.synchronize()
+    assert (host(idx) == i_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert host(info)[2] == info_ref[2] and host(info)[3] == info_ref[3]
+
+
+@pytest.mark.parametrize("m,n,k,iters,rule", [(2048, 32, 4, 8, 0), (2048, 32, 4, 0, 0), (1024, 16, 2, 3, 1),
+                                              (4096, 64, 8, 20, 0), (512, 8, 1, 2, 0)])
+def test_balance_solve_bitexact(m, n, k, iters, rule):
+    s = W.make_qb_scores(m, n, seed=m * 3 + n)
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, rule=rule, max_iters=iters)
+    assert rc == oracle.OK
+    idx, beta, info = lb.moe_balance_assign(dev(s), k, mode=lb.MOE_QB_SOLVE, rule=rule, max_iters=iters)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
+    assert (np.bincount(host(idx).ravel(), minlength=n) == m * k // n).all()
