@@ -1,0 +1,333 @@
+"""Benchmark of the MoE-layer forward on B200: one JSON line on rank 0.
+
+A step is one forward pass of the whole layer (router + top-k, capacity slots,
+dispatch, expert FFN, combine, load statistics) over one batch of the
+Switch-Base-like workload: m = 8192 tokens, d = 768, n = 128 experts, top-1
+softmax router in fp32, d_ff = 3072, capacity 80 (factor 1.25), bf16
+activations and weights, synthetic seeded inputs. The expert weights (1.2 GB)
+exceed the 126 MB L2, so every step streams them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+N > 1 runs under torchrun: every rank runs its own batch (weak scaling, no
+collective on the data path); the time is the max over ranks. `--impl
+reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer tokens/s (route+balance+dispatch+FFN+combine) and % roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name} MoE layer forward: m={cfg.m} d={cfg.d} n={cfg.n} k={cfg.k} {cfg.score_fn} "
+            f"d_ff={cfg.d_ff} capacity={cfg.capacity}/micro-batch seg_len={cfg.seg_len} {cfg.dtype}, fp32 router")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append(dict(ts=ts, sm=float(parts[2]), smax=float(parts[3]), active=parts[5],
+                                     hw=parts[6], hwt=parts[7], swt=parts[8], pcap=parts[9]))
+                except Exception:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 - 1 <= r["ts"] <= self.t1 + 1] or rows
+        load = [r for r in inside if r["sm"] > 0.5 * r["smax"]] or inside
+        reasons = set()
+        for r in inside:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_rate(cfg, inp, tokens: int):
+    """Time the CPU oracle on the first `tokens` tokens of the batch as one micro-batch
+    (capacity rescaled with the same factor). Returns (tokens/s, seconds)."""
+    import oracle
+    sub = W.scaled_config(cfg.name, m=tokens, seg_len=tokens,
+                          capacity=W.capacity_from_factor(1.25, tokens, cfg.k, cfg.n))
+    sub_inp = dict(inp, x=inp["x"][:tokens])
+    t = time.perf_counter()
+    oracle.layer_forward(sub_inp, sub)
+    dt = time.perf_counter() - t
+    return tokens / dt, dt
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    inp = W.make_layer_inputs(cfg, seed=0)
+    rate, _ = oracle_rate(cfg, inp, 32)                    # calibration
+    budget = 120.0                                        # seconds for the whole run
+    per_step = max(16, min(2048, int(budget * rate / max(1, args.steps + args.warmup))))
+    for _ in range(args.warmup):
+        oracle_rate(cfg, inp, per_step)
+    total_t = 0.0
+    for _ in range(args.steps):
+        _, dt = oracle_rate(cfg, inp, per_step)
+        total_t += dt
+    value = per_step * args.steps / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"first {per_step} tokens of the batch per step as one micro-batch "
+                                       f"(capacity factor 1.25), full layer forward in fp64 C"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def ffn_algorithmic_bytes(cfg, offsets, esz=2):
+    rows = np.diff(offsets)
+    used = int((rows > 0).sum())
+    per_expert = (2 * cfg.d * cfg.d_ff + cfg.d_ff + cfg.d) * esz
+    return used * per_expert + int(rows.sum()) * cfg.d * esz * 2
+
+
+def stage_bytes(cfg, offsets, esz=2):
+    m, d, n, k = cfg.m, cfg.d, cfg.n, cfg.k
+    rows = int(offsets[-1])
+    return {
+        "router": m * d * esz + d * n * 4 + m * n * 4 + m * k * 8,
+        "capacity": m * k * 4 * 4 + rows * 4,
+        "dispatch": 2 * rows * d * esz + rows * 4,
+        "ffn": ffn_algorithmic_bytes(cfg, offsets, esz),
+        "combine": rows * d * esz + m * d * esz + m * k * 8,
+        "stats": m * n * 4 + m * k * 4,
+    }
+
+
+def run_gpu(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import load_balanced_dispatch_b200 as lb
+    from load_balanced_dispatch_b200.layer import LayerShape, MoELayer, weights_to_device
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    lb.lib()
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    inp = W.make_layer_inputs(cfg, seed=rank)
+    w = weights_to_device(inp, dt)
+    shape = LayerShape(m=cfg.m, d=cfg.d, n=cfg.n, k=cfg.k, d_ff=cfg.d_ff, score_fn=cfg.score_fn, dtype=dt,
+                       capacity=cfg.capacity, seg_len=cfg.seg_len, renorm_topk=cfg.renorm_topk)
+    layer = MoELayer(shape, w)
+    x_host = torch.from_numpy(inp["x"]).to(dt).pin_memory()
+    x = x_host.to("cuda")
+    stream = torch.cuda.current_stream()
+    nst = len(MoELayer.STAGES)
+
+    # warm-up
+    for _ in range(args.warmup):
+        layer.forward(x)
+    lb.sync_status()
+
+    # timed region: K forwards, stage events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        layer.forward(x, events=evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    lb.sync_status()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, s in enumerate(MoELayer.STAGES)}
+    offsets = layer.buf["expert_offsets"].cpu().numpy()
+
+    # end-to-end through the public API: host x -> device, forward, y and the loss -> host, every step
+    y_host = torch.empty((cfg.m, cfg.d), dtype=dt).pin_memory()
+    aux_host = torch.empty(layer.buf["aux"].shape, dtype=torch.float32).pin_memory()
+    x_e2e = torch.empty_like(x)
+    for _ in range(2):
+        x_e2e.copy_(x_host, non_blocking=True)
+        layer.forward(x_e2e)
+        y_host.copy_(layer.buf["y"], non_blocking=True)
+        aux_host.copy_(layer.buf["aux"], non_blocking=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_e2e.copy_(x_host, non_blocking=True)
+        layer.forward(x_e2e)
+        y_host.copy_(layer.buf["y"], non_blocking=True)
+        aux_host.copy_(layer.buf["aux"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    lb.sync_status()
+
+    result = None
+    if rank == 0:
+        hbm, src = peaks()
+        sb = stage_bytes(cfg, offsets)
+        ffn_bytes = sb["ffn"]
+        ffn_s = stage_ms["ffn"] * 1e-3
+        achieved = ffn_bytes / ffn_s / 1e9
+        tokens = cfg.m * args.steps * world
+        value = tokens / (ms * 1e-3)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            rate, secs = oracle_rate(cfg, inp, args.cpu_tokens)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                   "sample": f"first {args.cpu_tokens} of the {cfg.m} tokens as one micro-batch (capacity factor "
+                             f"1.25), full layer forward in single-threaded fp64 C, {secs:.1f} s"}
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) expert weights; per rank)",
+            "config": {"workload": workload_desc(cfg), "m": cfg.m, "d_model": cfg.d, "experts": cfg.n, "k": cfg.k,
+                       "d_ff": cfg.d_ff, "capacity": cfg.capacity, "global_batch": cfg.m * world,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2: 1.2 GB of expert weights streamed every step"},
+            "roofline": {"kernel": "moe_expert_ffn (expert GEMM1 + GEMM2)", "bound": "hbm",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "peak_source": f"{src} hbm_gbs", "traffic": None,
+                         "algorithmic_bytes_per_launch": ffn_bytes, "launch_ms": stage_ms["ffn"]},
+            "stages": {s: {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9} for s in MoELayer.STAGES},
+            "rows_kept": int(offsets[-1]),
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": y_host.numel() * y_host.element_size() + aux_host.numel() * 4},
+            "clocks": clk,
+            "gpu_launches": args.steps * MoELayer.launches_per_forward,
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="switch", choices=sorted(W.CONFIGS))
+    ap.add_argument("--cpu-tokens", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = W.CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

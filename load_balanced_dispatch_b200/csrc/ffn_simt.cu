@@ -10,6 +10,7 @@
 // tiles, K-tiles of 16 staged in shared memory. fp32 inputs stay fp32 (a
 // tensor-core tf32 path would miss the fp32 tolerance).
 #include "common.cuh"
+#include "groups.cuh"
 
 namespace moe {
 
@@ -18,50 +19,22 @@ constexpr int BM = 64, BN = 64, BK = 16, kThreads = 256;
 constexpr int PAD = 4;
 }  // namespace simt
 
-// Tile list of a grouped GEMM, rebuilt per CTA from the device-side offsets.
-struct GroupTiles {
-    int tile_start[kMaxExperts + 1];
-    int row_start[kMaxExperts + 1];
-};
-
-__device__ __forceinline__ int find_group(const GroupTiles& g, int n, int tile) {
-    int lo = 0, hi = n;  // largest e with tile_start[e] <= tile
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (g.tile_start[mid] <= tile) lo = mid; else hi = mid;
-    }
-    return lo;
-}
-
 template <typename T, bool RELU>
 __global__ void __launch_bounds__(simt::kThreads)
 grouped_gemm_simt(const T* __restrict__ A, const T* __restrict__ B, const T* __restrict__ bias,
                   const int32_t* __restrict__ offsets, int n, int N, int K, int64_t max_rows, T* __restrict__ Cout) {
     using namespace simt;
-    __shared__ GroupTiles g;
+    __shared__ GroupTable g;
     __shared__ __align__(16) float As[BK][BM + PAD];
     __shared__ __align__(16) float Bs[BK][BN + PAD];
     const int tid = threadIdx.x;
     const int ntn = (N + BN - 1) / BN;
-    if (tid == 0) {
-        int acc = 0;
-        for (int e = 0; e < n; ++e) {
-            int r0 = offsets[e], r1 = offsets[e + 1];
-            if (r1 > max_rows) { record_error(kErrRowOverflow); r1 = (int)max_rows; }
-            if (r0 > r1) r0 = r1;
-            g.row_start[e] = r0;
-            g.tile_start[e] = acc;
-            acc += ((r1 - r0 + BM - 1) / BM) * ntn;
-        }
-        g.tile_start[n] = acc;
-        int rend = offsets[n];
-        g.row_start[n] = rend > max_rows ? (int)max_rows : rend;
-    }
+    if (tid < 32) build_group_table(offsets, n, ntn, BM, max_rows, g);
     __syncthreads();
     const int total = g.tile_start[n];
     const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads, each 4 x 4 outputs
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const int e = find_group(g, n, tile);
+        const int e = group_of_tile(g, n, tile);
         const int local = tile - g.tile_start[e];
         const int mt = local / ntn, nt = local - mt * ntn;
         const int64_t row0 = (int64_t)g.row_start[e] + (int64_t)mt * BM;

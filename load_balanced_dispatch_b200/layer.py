@@ -75,21 +75,33 @@ class MoELayer:
                               device=dev),
         )
 
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    STAGES = ("router", "capacity", "dispatch", "ffn", "combine", "stats")
+
+    def forward(self, x: torch.Tensor, stream=None, events=None) -> torch.Tensor:
+        """One forward. `events`: optional list of 7 CUDA events recorded on the stream around the 6 stages."""
         s, b, w = self.shape, self.buf, self.w
+        st = stream if stream is not None else torch.cuda.current_stream()
+        mark = (lambda i: events[i].record(st)) if events is not None else (lambda i: None)
         fn = MOE_SOFTMAX if s.score_fn == "softmax" else MOE_SIGMOID
+        mark(0)
         moe_router_topk(x, w["w_r"], s.n, s.k, fn, s.renorm_topk, rank_bias=w.get("rank_bias"), probs_out=b["probs"],
-                        topk_idx=b["topk_idx"], topk_gate=b["topk_gate"], stream=stream)
+                        topk_idx=b["topk_idx"], topk_gate=b["topk_gate"], stream=st)
+        mark(1)
         cap = moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"],
-                                 stream=stream)
-        moe_dispatch(x, cap["src_token"], cap["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=stream)
+                                 stream=st)
+        mark(2)
+        moe_dispatch(x, cap["src_token"], cap["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
+        mark(3)
         moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], cap["expert_offsets"], ybuf=b["ybuf"],
-                       workspace=self.ws["ffn"], stream=stream)
+                       workspace=self.ws["ffn"], stream=st)
+        mark(4)
         moe_combine(b["ybuf"], cap["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
-                    stream=stream)
+                    stream=st)
+        mark(5)
         moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
                           bias_inout=w.get("rank_bias") if s.lossfree else None, gamma=s.gamma, out=b,
-                          workspace=self.ws["stats"], stream=stream)
+                          workspace=self.ws["stats"], stream=st)
+        mark(6)
         return b["y"]
 
     # kernel launches per forward (router 1, capacity 3, dispatch 1, FFN 2, combine 1, stats 2)
