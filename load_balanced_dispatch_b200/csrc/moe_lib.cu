@@ -6,5 +6,6 @@
 #include "dispatch_combine.cu"
 #include "ffn.cu"
 #include "ffn_simt.cu"
+#include "ffn_tc.cu"
 #include "router.cu"
 #include "stats.cu"

@@ -29,11 +29,15 @@ import numpy as np
 
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); return float32."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    bits = a.view(np.uint32).astype(np.uint64)
-    lsb = (bits >> 16) & 1
-    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
-    return rounded.astype(np.uint32).view(np.float32)
+    a = np.array(a, dtype=np.float32, copy=True, order="C")
+    if not np.isfinite(a).all():
+        raise ValueError("round_to_bf16 expects finite values")
+    bits = a.view(np.uint32)
+    lsb = (bits >> np.uint32(16)) & np.uint32(1)
+    bits += np.uint32(0x7FFF)
+    bits += lsb
+    bits &= np.uint32(0xFFFF0000)
+    return a
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
