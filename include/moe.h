@@ -160,6 +160,31 @@ MOE_API moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_
                               size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Capacity slots with no caller-provided scratch. The pages have no
+ * counterpart: this is a convenience for callers that cannot allocate device
+ * memory or pass a workspace -- for example code reached through a fixed
+ * foreign-function signature that carries only inputs and outputs, or a host
+ * framework that owns all device memory and forbids its plugins to call
+ * cudaMalloc (which may also synchronise the device).
+ *  Arguments and results: exactly those of moe_capacity_slots, minus the workspace.
+ *  Scratch: a fixed 1 MiB array compiled into the library (every GPU that
+ *  loads the library keeps it until the process exits). A problem needing more
+ *  (moe_capacity_slots_workspace_size > 1 MiB) is rejected with
+ *  MOE_ERR_WORKSPACE before anything is enqueued; use moe_capacity_slots then.
+ *  The first call on a device looks up the array's device address with
+ *  cudaGetSymbolAddress while that device is current; make that first call
+ *  before any stream capture.
+ *  All calls share the one array and it keeps the last call's contents (no
+ *  word of it needs to start at zero: every word read is first written by the
+ *  same call). Calls that overlap on the GPU -- on different streams, or from
+ *  threads that do not order their streams -- race on it; order them.
+ */
+MOE_API moe_status moe_capacity_slots_static(const int32_t* topk_idx, int64_t m, int32_t k, int32_t n,
+                                             int32_t capacity, int64_t seg_len, int32_t* slot, int32_t* dest_row,
+                                             int32_t* src_token, int32_t* expert_offsets, int32_t* routed_count,
+                                             int32_t* kept_count, moe_stream_t stream);
+
+/*
  * Dispatch: gather tokens into expert-major order.
  * Passage: "Switch Transformer read for implementation" (molayo1419.me), the
  * forward pass changes token order twice (first: group tokens by expert).

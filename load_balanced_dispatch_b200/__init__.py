@@ -28,7 +28,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk", "moe_balance_assign_workspace_size",
            "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
-           "moe_balance_stats")
+           "moe_balance_stats", "moe_capacity_slots_static")
 
 
 class MoEError(RuntimeError):
@@ -58,6 +58,7 @@ def lib() -> C.CDLL:
         L.moe_capacity_slots_workspace_size.argtypes = [I64, I32, I32, I64]
         L.moe_capacity_slots_workspace_size.restype = SZ
         L.moe_capacity_slots.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P, SZ, P]
+        L.moe_capacity_slots_static.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P]
         L.moe_dispatch.argtypes = [P, I32, I64, I32, P, P, I32, I64, P, P]
         L.moe_expert_ffn_workspace_size.argtypes = [I32, I64, I32]
         L.moe_expert_ffn_workspace_size.restype = SZ
@@ -161,6 +162,26 @@ def moe_capacity_slots(topk_idx, n, capacity, seg_len=None, out=None, workspace=
         _ptr(topk_idx), m, k, n, capacity, seg_len, _ptr(out["slot"]), _ptr(out["dest_row"]), _ptr(out["src_token"]),
         _ptr(out["expert_offsets"]), _ptr(out["routed_count"]), _ptr(out["kept_count"]), _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_capacity_slots_static(topk_idx, n, capacity, seg_len=None, out=None, stream=None):
+    """moe_capacity_slots without a workspace: the library's fixed 1 MiB scratch array is used
+    instead, for callers that cannot allocate device memory. Same outputs as moe_capacity_slots."""
+    m, k = topk_idx.shape
+    seg_len = m if seg_len is None else seg_len
+    dev = topk_idx.device
+    nseg = m // seg_len if seg_len > 0 else 1
+    if out is None:
+        out = dict(slot=torch.empty((m, k), dtype=torch.int32, device=dev),
+                   dest_row=torch.empty((m, k), dtype=torch.int32, device=dev),
+                   src_token=torch.empty((m * k,), dtype=torch.int32, device=dev),
+                   expert_offsets=torch.empty((n + 1,), dtype=torch.int32, device=dev),
+                   routed_count=torch.empty((nseg, n), dtype=torch.int32, device=dev),
+                   kept_count=torch.empty((nseg, n), dtype=torch.int32, device=dev))
+    _check("moe_capacity_slots_static", lib().moe_capacity_slots_static(
+        _ptr(topk_idx), m, k, n, capacity, seg_len, _ptr(out["slot"]), _ptr(out["dest_row"]), _ptr(out["src_token"]),
+        _ptr(out["expert_offsets"]), _ptr(out["routed_count"]), _ptr(out["kept_count"]), _stream(stream)))
     return out
 
 

@@ -3,6 +3,7 @@
 #include "api.cu"
 #include "balance.cu"
 #include "capacity.cu"
+#include "capacity_static.cu"
 #include "dispatch_combine.cu"
 #include "ffn.cu"
 #include "ffn_simt.cu"
