@@ -155,6 +155,28 @@ def run_reference(args, cfg):
     return 0
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Every rank processes its own batch (weak scaling): all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (ms_max * 1e-3)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own synthetic batch and weights."""
+    return rank
+
+
 # ------------------------------------------------------------------ GPU arm
 def ffn_algorithmic_bytes(cfg, offsets, esz=2):
     rows = np.diff(offsets)
@@ -193,7 +215,7 @@ def run_gpu(args, cfg):
                                 device_id=torch.device("cuda", local))
     lb.lib()
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-    inp = W.make_layer_inputs(cfg, seed=rank)
+    inp = W.make_layer_inputs(cfg, seed=rank_seed(rank))
     w = weights_to_device(inp, dt)
     shape = LayerShape(m=cfg.m, d=cfg.d, n=cfg.n, k=cfg.k, d_ff=cfg.d_ff, score_fn=cfg.score_fn, dtype=dt,
                        capacity=cfg.capacity, seg_len=cfg.seg_len, renorm_topk=cfg.renorm_topk)
@@ -228,11 +250,7 @@ def run_gpu(args, cfg):
         dist.barrier()
     clk = clocks.stop()
     lb.sync_status()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), device="cuda")
     stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, s in enumerate(MoELayer.STAGES)}
     offsets = layer.buf["expert_offsets"].cpu().numpy()
@@ -258,11 +276,7 @@ def run_gpu(args, cfg):
         aux_host.copy_(layer.buf["aux"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), device="cuda")
     lb.sync_status()
 
     result = None
@@ -273,7 +287,7 @@ def run_gpu(args, cfg):
         ffn_s = stage_ms["ffn"] * 1e-3
         achieved = ffn_bytes / ffn_s / 1e9
         tokens = cfg.m * args.steps * world
-        value = tokens / (ms * 1e-3)
+        value = whole_job_tokens_per_s(cfg.m, args.steps, world, ms)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             import oracle
@@ -298,7 +312,7 @@ def run_gpu(args, cfg):
             "stages": {s: {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9} for s in MoELayer.STAGES},
             "rows_kept": int(offsets[-1]),
             "cpu_baseline": cpu,
-            "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_tokens_per_s(cfg.m, args.steps, world, ms_e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": y_host.numel() * y_host.element_size() + aux_host.numel() * 4},
             "clocks": clk,
