@@ -225,10 +225,18 @@ def run_gpu(args, cfg):
     stream = torch.cuda.current_stream()
     nst = len(MoELayer.STAGES)
 
-    # warm-up
+    # warm-up (eager), then record each stage into a CUDA graph unless --eager
     for _ in range(args.warmup):
         layer.forward(x)
     lb.sync_status()
+    if args.eager:
+        run = lambda events=None: layer.forward(x, events=events)  # noqa: E731
+    else:
+        layer.capture(x)
+        run = layer.replay
+        for _ in range(args.warmup):
+            run()
+        lb.sync_status()
 
     # timed region: K forwards, stage events on the launching stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
@@ -242,7 +250,7 @@ def run_gpu(args, cfg):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        layer.forward(x, events=evs[i])
+        run(events=evs[i])
     end.record(stream)
     torch.cuda.synchronize()
     clocks.mark("t1")
@@ -258,10 +266,9 @@ def run_gpu(args, cfg):
     # end-to-end through the public API: host x -> device, forward, y and the loss -> host, every step
     y_host = torch.empty((cfg.m, cfg.d), dtype=dt).pin_memory()
     aux_host = torch.empty(layer.buf["aux"].shape, dtype=torch.float32).pin_memory()
-    x_e2e = torch.empty_like(x)
     for _ in range(2):
-        x_e2e.copy_(x_host, non_blocking=True)
-        layer.forward(x_e2e)
+        x.copy_(x_host, non_blocking=True)
+        run()
         y_host.copy_(layer.buf["y"], non_blocking=True)
         aux_host.copy_(layer.buf["aux"], non_blocking=True)
     if world > 1:
@@ -270,8 +277,8 @@ def run_gpu(args, cfg):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        x_e2e.copy_(x_host, non_blocking=True)
-        layer.forward(x_e2e)
+        x.copy_(x_host, non_blocking=True)
+        run()
         y_host.copy_(layer.buf["y"], non_blocking=True)
         aux_host.copy_(layer.buf["aux"], non_blocking=True)
     e1.record(stream)
@@ -303,7 +310,7 @@ def run_gpu(args, cfg):
             "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) expert weights; per rank)",
             "config": {"workload": workload_desc(cfg), "m": cfg.m, "d_model": cfg.d, "experts": cfg.n, "k": cfg.k,
                        "d_ff": cfg.d_ff, "capacity": cfg.capacity, "global_batch": cfg.m * world,
-                       "parallelism": f"replicas x{world}",
+                       "parallelism": f"replicas x{world}", "launch": "eager" if args.eager else "cuda graphs per stage",
                        "l2": "inputs larger than L2: 1.2 GB of expert weights streamed every step"},
             "roofline": {"kernel": "moe_expert_ffn (expert GEMM1 + GEMM2)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -316,12 +323,67 @@ def run_gpu(args, cfg):
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": y_host.numel() * y_host.element_size() + aux_host.numel() * 4},
             "clocks": clk,
-            "gpu_launches": args.steps * MoELayer.launches_per_forward,
+            "gpu_launches": args.steps * layer.launches_per_forward(),
         }
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_gpu_qb(args):
+    """Balanced assignment of the 65536 x 256 skewed scores (k = 8): SOLVE mode per step."""
+    import torch
+
+    import load_balanced_dispatch_b200 as lb
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    q = W.QB_CONFIG
+    m, n, k = q["m"], q["n"], q["k"]
+    s = torch.from_numpy(W.make_qb_scores(m, n, seed=0, skew_std=q["skew_std"])).cuda()
+    beta = torch.zeros(n, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lb.lib().moe_balance_assign_workspace_size(m, n, k, lb.MOE_QB_SOLVE), dtype=torch.uint8,
+                     device="cuda")
+    idx = torch.empty((m, k), dtype=torch.int32, device="cuda")
+    info = torch.zeros(4, dtype=torch.int32, device="cuda")
+
+    def step():
+        beta.zero_()
+        lb.moe_balance_assign(s, k, beta=beta, mode=lb.MOE_QB_SOLVE, max_iters=args.qb_iters, topk_idx=idx,
+                              info=info, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    lb.sync_status()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    # one STEP (row pass + column pass, the practical per-training-step form) for the per-pass figures
+    st0, st1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st0.record(stream)
+    for _ in range(args.steps):
+        lb.moe_balance_assign(s, k, beta=beta, mode=lb.MOE_QB_STEP, topk_idx=idx, info=torch.zeros_like(info),
+                              workspace=ws)
+    st1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = st0.elapsed_time(st1) / args.steps
+    inf = info.cpu().tolist()
+    hbm, src = peaks()
+    line = {"metric": METRIC, "value": m / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (N(0,1) + per-expert skew N(0,1.5^2))",
+            "config": {"workload": f"optimal-assignment balancing SOLVE m={m} n={n} k={k} C={m * k // n}",
+                       "max_iters": args.qb_iters},
+            "solve_info": {"beta_updates": inf[0], "repair_moves": inf[1], "excess_left": inf[2], "ties": inf[3]},
+            "step_mode_ms": step_ms,
+            "step_mode_GB/s": (3 * m * n * 4) / (step_ms * 1e-3) / 1e9, "peak_hbm": hbm}
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -331,12 +393,16 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="switch", choices=sorted(W.CONFIGS))
+    ap.add_argument("--workload", default="switch", choices=sorted(W.CONFIGS) + ["qb"])
+    ap.add_argument("--qb-iters", type=int, default=32)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch every call from Python instead of CUDA graphs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload == "qb":
+        return run_gpu_qb(args)
     cfg = W.CONFIGS[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg)

@@ -89,13 +89,17 @@ MOE_API moe_status moe_sync_status(moe_stream_t stream);
  *  probs_out  [m, n] fp32 scores p or rho, or NULL.
  *  topk_idx   [m, k] out: selected experts, best key first; equal keys -> lower index first.
  *  topk_gate  [m, k] out: fp32 gates (rho_sel for sigmoid).
+ *  workspace  bf16 x with n <= 128: [3, n, d] bf16 split of W_r (w = w0 + w1 + w2, each
+ *             bf16) so the projection runs on the tensor cores with exact products and
+ *             fp32 accumulation; size from moe_router_topk_workspace_size (0 otherwise).
  * All h, p, rho and keys are fp32. Errors: MOE_ERR_INVALID_ARG for bad shapes
- * or NULL required pointers.
+ * or NULL required pointers; MOE_ERR_WORKSPACE for a missing or short workspace.
  */
+MOE_API size_t moe_router_topk_workspace_size(int32_t d, int32_t n, int32_t k, moe_dtype x_dtype);
 MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, const float* logits_in, int64_t m,
                            int32_t d, int32_t n, int32_t k, moe_score_fn fn, int32_t renorm_topk,
                            const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
-                           moe_stream_t stream);
+                           void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Optimal-assignment balancing (Quantile Balancing) with an exact finish.

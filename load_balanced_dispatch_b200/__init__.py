@@ -25,7 +25,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_NOT_CONVERGED", 6: "MOE_ERR_INTERNAL"}
 
 # every symbol the C header declares
-EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk", "moe_balance_assign_workspace_size",
+EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size", "moe_router_topk", "moe_balance_assign_workspace_size",
            "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
            "moe_balance_stats", "moe_capacity_slots_static")
@@ -51,7 +51,9 @@ def lib() -> C.CDLL:
         L.moe_last_error.argtypes = [C.c_char_p, SZ]
         L.moe_last_error.restype = None
         L.moe_sync_status.argtypes = [P]
-        L.moe_router_topk.argtypes = [P, I32, P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, P]
+        L.moe_router_topk_workspace_size.argtypes = [I32, I32, I32, I32]
+        L.moe_router_topk_workspace_size.restype = SZ
+        L.moe_router_topk.argtypes = [P, I32, P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
         L.moe_balance_assign_workspace_size.argtypes = [I64, I32, I32, I32]
         L.moe_balance_assign_workspace_size.restype = SZ
         L.moe_balance_assign.argtypes = [P, I64, I32, I32, P, I32, I32, I32, I32, P, P, P, SZ, P]
@@ -116,7 +118,7 @@ def sync_status(stream=None):
 
 
 def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias=None, logits_in=None,
-                    probs_out=None, topk_idx=None, topk_gate=None, want_probs=True, stream=None):
+                    probs_out=None, topk_idx=None, topk_gate=None, want_probs=True, workspace=None, stream=None):
     """Router + top-k. Returns (topk_idx [m,k] int32, topk_gate [m,k] fp32, probs [m,n] fp32 or None)."""
     if logits_in is not None:
         m, d = logits_in.shape[0], 0
@@ -136,9 +138,13 @@ def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias
         topk_gate = torch.empty((m, k), dtype=torch.float32, device=dev)
     if probs_out is None and want_probs:
         probs_out = torch.empty((m, n), dtype=torch.float32, device=dev)
+    ws_bytes = lib().moe_router_topk_workspace_size(d, n, k, xdt) if logits_in is None else 0
+    if workspace is None and ws_bytes:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
     _check("moe_router_topk", lib().moe_router_topk(
         _ptr(x), xdt, _ptr(w_r), _ptr(logits_in), m, d, n, k, score_fn, renorm_topk, _ptr(rank_bias),
-        _ptr(probs_out), _ptr(topk_idx), _ptr(topk_gate), _stream(stream)))
+        _ptr(probs_out), _ptr(topk_idx), _ptr(topk_gate), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream(stream)))
     return topk_idx, topk_gate, probs_out
 
 

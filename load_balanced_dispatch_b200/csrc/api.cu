@@ -10,7 +10,9 @@ namespace moe {
 
 cudaError_t launch_router(const void* x, moe_dtype dt, const float* w_r, const float* logits_in, int64_t m, int d,
                           int n, int k, int fn, int renorm, const float* rank_bias, float* probs_out,
-                          int32_t* topk_idx, float* topk_gate, cudaStream_t stream);
+                          int32_t* topk_idx, float* topk_gate, void* workspace, cudaStream_t stream);
+size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt);
+bool router_uses_tc(moe_dtype dt, const float* logits_in, int n, int k);
 cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, int32_t capacity, int64_t seg_len,
                             int32_t* slot, int32_t* dest_row, int32_t* src_token, int32_t* expert_offsets,
                             int32_t* routed_count, int32_t* kept_count, void* workspace, cudaStream_t stream);
@@ -84,10 +86,14 @@ moe_status moe_sync_status(moe_stream_t stream) {
     return MOE_OK;
 }
 
+size_t moe_router_topk_workspace_size(int32_t d, int32_t n, int32_t k, moe_dtype x_dtype) {
+    return router_uses_tc(x_dtype, nullptr, n, k) ? router_workspace_bytes(d, n, x_dtype) : 0;
+}
+
 moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, const float* logits_in, int64_t m,
                            int32_t d, int32_t n, int32_t k, moe_score_fn fn, int32_t renorm_topk,
                            const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
-                           moe_stream_t stream) {
+                           void* workspace, size_t ws_bytes, moe_stream_t stream) {
     REQUIRE(m >= 0, "m must be >= 0");
     REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
     REQUIRE(k >= 1 && k <= n, "k must be in [1, n]");
@@ -98,9 +104,17 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, c
     if (!logits_in) {
         REQUIRE(m == 0 || (x && w_r), "x and w_r are required when logits_in is NULL");
         REQUIRE(d >= 1, "d must be >= 1");
+        REQUIRE(x_dtype != MOE_BF16 || d % 8 == 0, "d must be a multiple of 8 for bf16 x");
+        REQUIRE(x_dtype != MOE_BF16 || m == 0 || aligned16(x), "bf16 x must be 16-byte aligned");
+    }
+    REQUIRE(!probs_out || aligned16(probs_out), "probs_out must be 16-byte aligned");
+    if (router_uses_tc(x_dtype, logits_in, n, k) && m > 0) {
+        const size_t need = router_workspace_bytes(d, n, x_dtype);
+        if (ws_bytes < need || !workspace || !aligned16(workspace))
+            return fail(MOE_ERR_WORKSPACE, "moe_router_topk: 16-byte aligned workspace of %zu bytes required", need);
     }
     return check_launch(launch_router(x, x_dtype, w_r, logits_in, m, d, n, k, (int)fn, renorm_topk, rank_bias,
-                                      probs_out, topk_idx, topk_gate, stream),
+                                      probs_out, topk_idx, topk_gate, workspace, stream),
                         "moe_router_topk");
 }
 
@@ -142,8 +156,9 @@ moe_status moe_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, const
 }
 
 size_t moe_expert_ffn_workspace_size(moe_dtype dt, int64_t max_rows, int32_t d_ff) {
+    // hidden activations [max_rows, d_ff], then (bf16) one int32 completion counter per expert
     const size_t esz = dt == MOE_BF16 ? 2 : 4;
-    return esz * (size_t)(max_rows < 0 ? 0 : max_rows) * (size_t)(d_ff < 0 ? 0 : d_ff) + 1024;
+    return esz * (size_t)(max_rows < 0 ? 0 : max_rows) * (size_t)(d_ff < 0 ? 0 : d_ff) + 2048;
 }
 
 moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2,

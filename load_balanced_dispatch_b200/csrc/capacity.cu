@@ -98,10 +98,17 @@ cap_scan_kernel(const int32_t* __restrict__ hist, int n, int64_t nseg, int64_t c
     if (e < n) {
         for (int64_t s = 0; s < nseg; ++s) {
             int64_t run = 0;
-            for (int64_t c = 0; c < cps; ++c) {
-                const int64_t ch = s * cps + c;
-                prefix[ch * n + e] = (int32_t)run;
-                run += hist[ch * n + e];
+            for (int64_t c0 = 0; c0 < cps; c0 += 8) {  // 8 loads in flight
+                int32_t h[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) h[u] = (c0 + u < cps) ? hist[(s * cps + c0 + u) * n + e] : 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (c0 + u < cps) {
+                        prefix[(s * cps + c0 + u) * n + e] = (int32_t)run;
+                        run += h[u];
+                    }
+                }
             }
             const int64_t kept = run < capacity ? run : (int64_t)capacity;
             routed_count[s * n + e] = (int32_t)run;

@@ -41,7 +41,20 @@ dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, con
         }
         const uint4* src = x + (int64_t)t * vec_per_row;
         uint4* dst = xbuf + r * vec_per_row;
-        for (int64_t c = lane; c < vec_per_row; c += 32) dst[c] = src[c];
+        // up to 8 independent 16-byte loads in flight per lane before the stores
+        for (int64_t c0 = lane; c0 < vec_per_row; c0 += 32 * 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t c = c0 + 32 * u;
+                if (c < vec_per_row) v[u] = src[c];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t c = c0 + 32 * u;
+                if (c < vec_per_row) dst[c] = v[u];
+            }
+        }
     }
 }
 
@@ -55,23 +68,35 @@ combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row,
     const int nvec = d / V;
     const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
     for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
-        for (int c = lane; c < nvec; c += 32) {
-            float acc[V];
-            if (residual) Vec16<T>::load(residual + i * d + (int64_t)c * V, acc);
-            else
+        // two 16-byte column chunks per lane at a time: their k row loads are independent
+        for (int c0 = lane; c0 < nvec; c0 += 64) {
+            const int c1 = c0 + 32;
+            const bool has1 = c1 < nvec;
+            float acc0[V], acc1[V];
+            if (residual) {
+                Vec16<T>::load(residual + i * d + (int64_t)c0 * V, acc0);
+                if (has1) Vec16<T>::load(residual + i * d + (int64_t)c1 * V, acc1);
+            } else {
 #pragma unroll
-                for (int q = 0; q < V; ++q) acc[q] = 0.f;
+                for (int q = 0; q < V; ++q) { acc0[q] = 0.f; acc1[q] = 0.f; }
+            }
             for (int r = 0; r < k; ++r) {
                 const int32_t row = dest_row[i * k + r];
                 if (row < 0) continue;
                 float g = gate[i * k + r];
                 if (gate_bf16) g = round_to_bf16(g);
-                float v[V];
-                Vec16<T>::load(ybuf + (int64_t)row * d + (int64_t)c * V, v);
+                float v0[V], v1[V];
+                const T* yr = ybuf + (int64_t)row * d;
+                Vec16<T>::load(yr + (int64_t)c0 * V, v0);
+                if (has1) Vec16<T>::load(yr + (int64_t)c1 * V, v1);
 #pragma unroll
-                for (int q = 0; q < V; ++q) acc[q] = fmaf(g, v[q], acc[q]);
+                for (int q = 0; q < V; ++q) {
+                    acc0[q] = fmaf(g, v0[q], acc0[q]);
+                    if (has1) acc1[q] = fmaf(g, v1[q], acc1[q]);
+                }
             }
-            Vec16<T>::store(y + i * d + (int64_t)c * V, acc);
+            Vec16<T>::store(y + i * d + (int64_t)c0 * V, acc0);
+            if (has1) Vec16<T>::store(y + i * d + (int64_t)c1 * V, acc1);
         }
     }
 }

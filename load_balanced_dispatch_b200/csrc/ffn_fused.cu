@@ -1,0 +1,255 @@
+// ffn_fused.cu -- the bf16 expert FFN as ONE persistent tcgen05 launch over both GEMMs.
+//
+// Switch Transformers paper review (tildalice.io/?p=118), Switch Layer:
+// FFN(x) = max(0, x W1 + b1) W2 + b2 per expert.
+//
+// The tile list holds every GEMM1 tile (h = relu(xbuf W1_e^T + b1_e), bf16)
+// followed by every GEMM2 tile (ybuf = h W2_e^T + b2_e). Each CTA walks its
+// tiles in increasing order, so it finishes all of its GEMM1 tiles before its
+// first GEMM2 tile; with every CTA resident at once (cooperative launch) each
+// GEMM1 tile therefore completes, and a GEMM2 tile of expert e only waits for
+// the GEMM1 tiles of e. That wait is a per-expert counter in global memory:
+// each epilogue warp of a GEMM1 tile stores its h rows, fences them for the
+// async (TMA) proxy and release-adds 1; the producer of a GEMM2 tile
+// acquire-polls the counter (bounded), fences, then loads h with TMA. One
+// launch instead of two removes the second kernel's prologue and the wave
+// tail between the GEMMs. Warp roles, pipeline and epilogue are those of the
+// two-launch kernel in ffn_tc.cu; every wait is bounded.
+#include "groups.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+
+namespace fz {
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kThreads = 192;
+constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
+constexpr int kEpiWarps = 4;
+}  // namespace fz
+
+struct FusedShared {
+    uint64_t full[fz::STAGES], empty[fz::STAGES], tfull[2], tempty[2];
+    uint32_t tmem_base;
+    int abort_flag;
+    GroupTable g1, g2;
+};
+
+constexpr size_t fused_smem_bytes() { return 1024 + (size_t)fz::STAGES * fz::STAGE_BYTES + sizeof(FusedShared); }
+
+struct FusedTile {
+    int phase, e, n0, N, K, mtiles1;
+    int64_t row0, row_end;
+};
+
+__device__ __forceinline__ FusedTile fused_decode(const FusedShared* sh, int tile, int T1, int n, int d, int d_ff) {
+    FusedTile t;
+    t.phase = tile < T1 ? 1 : 2;
+    const GroupTable& g = t.phase == 1 ? sh->g1 : sh->g2;
+    const int lt = t.phase == 1 ? tile : tile - T1;
+    t.e = group_of_tile(g, n, lt);
+    const int local = lt - g.tile_start[t.e];
+    const int rows_e = g.row_start[t.e + 1] - g.row_start[t.e];
+    const int mtiles = (rows_e + fz::BM - 1) / fz::BM;
+    const int nt = local / mtiles, mt = local - nt * mtiles;
+    t.row0 = (int64_t)g.row_start[t.e] + (int64_t)mt * fz::BM;
+    t.row_end = g.row_start[t.e + 1];
+    t.n0 = nt * fz::BN;
+    t.N = t.phase == 1 ? d_ff : d;
+    t.K = t.phase == 1 ? d : d_ff;
+    t.mtiles1 = mtiles;
+    return t;
+}
+
+__global__ void __launch_bounds__(fz::kThreads, 1)
+ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w1,
+             const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_w2,
+             const __nv_bfloat16* __restrict__ b1, const __nv_bfloat16* __restrict__ b2,
+             const int32_t* __restrict__ offsets, int n, int d, int d_ff, int64_t max_rows,
+             __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ y, int* __restrict__ done1) {
+    using namespace fz;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    FusedShared* sh = reinterpret_cast<FusedShared*>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntn1 = (d_ff + BN - 1) / BN, ntn2 = (d + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        sh->abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::prefetch_tensormap(&map_x);
+        ptx::prefetch_tensormap(&map_w1);
+        ptx::prefetch_tensormap(&map_h);
+        ptx::prefetch_tensormap(&map_w2);
+    }
+    if (warp == 1) ptx::tmem_alloc(&sh->tmem_base, TMEM_COLS);
+    if (warp == 2) build_group_table(offsets, n, ntn1, BM, max_rows, sh->g1);
+    if (warp == 3) build_group_table(offsets, n, ntn2, BM, max_rows, sh->g2);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = sh->tmem_base;
+    const int T1 = sh->g1.tile_start[n];
+    const int total = T1 + sh->g2.tile_start[n];
+    volatile int* abort_flag = &sh->abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
+                if (t.phase == 2) {
+                    // all GEMM1 tiles of expert e, each signalled by its 4 epilogue warps
+                    const int rows_e = sh->g1.row_start[t.e + 1] - sh->g1.row_start[t.e];
+                    const int need = ((rows_e + BM - 1) / BM) * ntn1 * kEpiWarps;
+                    const long long t0 = clock64();
+                    bool ok = true;
+                    while (ptx::ld_acquire_gpu(done1 + t.e) < need) {
+                        if (*abort_flag || clock64() - t0 > ptx::kWaitCycles) {
+                            if (!*abort_flag) { *abort_flag = 1; record_error(kErrPipelineTimeout); }
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    if (!ok) break;
+                    ptx::fence_proxy_async_global();
+                }
+                const CUtensorMap* ma = t.phase == 1 ? &map_x : &map_h;
+                const CUtensorMap* mb = t.phase == 1 ? &map_w1 : &map_w2;
+                const int nkb = (t.K + BK - 1) / BK;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    ptx::mbar_expect_tx(&sh->full[stage], STAGE_BYTES);
+                    ptx::tma_load_2d(sa, ma, &sh->full[stage], kb * BK, (int)t.row0);
+                    ptx::tma_load_3d(sa + A_BYTES, mb, &sh->full[stage], kb * BK, t.n0, t.e);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, aphase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const int K = tile < T1 ? d : d_ff;
+                const int nkb = (K + BK - 1) / BK;
+                if (!ptx::mbar_wait(&sh->tempty[acc], aphase ^ 1u, abort_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!ptx::mbar_wait(&sh->full[stage], phase, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = ptx::smem_u32(smem + stage * STAGE_BYTES);
+                    const uint64_t adesc = ptx::sw128_kmajor_desc(sa);
+                    const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        ptx::umma_bf16(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+                    ptx::umma_commit(&sh->empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::umma_commit(&sh->tfull[acc]);
+                if (++acc == 2) { acc = 0; aphase ^= 1u; }
+            }
+        }
+    } else {
+        const int quad = warp & 3;
+        int acc = 0;
+        uint32_t aphase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
+            if (!ptx::mbar_wait(&sh->tfull[acc], aphase, abort_flag)) break;
+            ptx::tc_fence_after();
+            const int64_t r = t.row0 + quad * 32 + lane;
+            const bool row_ok = r < t.row_end;
+            const bool relu = t.phase == 1;
+            const __nv_bfloat16* be = (t.phase == 1 ? b1 : b2) + (int64_t)t.e * t.N;
+            __nv_bfloat16* out = t.phase == 1 ? h : y;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int col0 = t.n0 + c * 32;
+                if (col0 >= t.N) break;  // warp-uniform
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
+#pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int col = col0 + g8 * 8;
+                    if (col >= t.N) break;
+                    float f[8], bv[8];
+                    Vec16<__nv_bfloat16>::load(be + col, bv);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        f[q] = __uint_as_float(v[g8 * 8 + q]) + bv[q];
+                        if (relu) f[q] = fmaxf(f[q], 0.f);
+                    }
+                    if (row_ok) Vec16<__nv_bfloat16>::store(out + r * t.N + col, f);
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&sh->tempty[acc]);
+            if (t.phase == 1) {
+                // publish this warp's h rows to the TMA loads of the GEMM2 tiles of expert e
+                ptx::fence_proxy_async_global();
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(done1 + t.e, 1);
+                }
+            }
+            if (++acc == 2) { acc = 0; aphase ^= 1u; }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
+                             const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
+                             int* done1, cudaStream_t stream) {
+    CUtensorMap mx, mw1, mh, mw2;
+    if (!map_2d(&mx, xbuf, (uint64_t)max_rows, (uint64_t)d, fz::BM)) return cudaErrorInvalidValue;
+    if (!map_3d(&mw1, w1, (uint64_t)n, (uint64_t)d_ff, (uint64_t)d, fz::BN)) return cudaErrorInvalidValue;
+    if (!map_2d(&mh, hbuf, (uint64_t)max_rows, (uint64_t)d_ff, fz::BM)) return cudaErrorInvalidValue;
+    if (!map_3d(&mw2, w2, (uint64_t)n, (uint64_t)d, (uint64_t)d_ff, fz::BN)) return cudaErrorInvalidValue;
+    static int grid = 0;
+    const size_t smem = fused_smem_bytes();
+    if (!grid) {
+        cudaError_t e = cudaFuncSetAttribute(ffn_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ffn_fused_tc, fz::kThreads, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        grid = num_sms();  // one CTA per SM (all resident: the cooperative launch checks it)
+    }
+    cudaError_t e = cudaMemsetAsync(done1, 0, sizeof(int) * (size_t)n, stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(fz::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ffn_fused_tc, mx, mw1, mh, mw2, static_cast<const __nv_bfloat16*>(b1),
+                              static_cast<const __nv_bfloat16*>(b2), offsets, n, d, d_ff, max_rows,
+                              static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), done1);
+}
+
+}  // namespace moe

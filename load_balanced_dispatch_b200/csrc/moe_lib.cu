@@ -8,5 +8,7 @@
 #include "ffn.cu"
 #include "ffn_simt.cu"
 #include "ffn_tc.cu"
+#include "ffn_fused.cu"
 #include "router.cu"
+#include "router_tc.cu"
 #include "stats.cu"

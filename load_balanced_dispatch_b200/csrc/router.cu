@@ -219,9 +219,24 @@ static cudaError_t launch_router_dt(const void* x, const float* w_r, const float
     return launch_router_t<T, 8>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
 }
 
+cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, int n, int k, int fn, int renorm,
+                             const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
+                             void* workspace, cudaStream_t stream);
+
+// bf16 activations projected on the tensor cores (W_r split into three bf16 parts) when the
+// expert row fits the register drain (n <= 128); fp32 activations, given logits or n > 128 use the
+// FMA kernel.
+bool router_tc_supported(int n, int k);
+bool router_uses_tc(moe_dtype dt, const float* logits_in, int n, int k) {
+    return dt == MOE_BF16 && !logits_in && router_tc_supported(n, k);
+}
+
 cudaError_t launch_router(const void* x, moe_dtype dt, const float* w_r, const float* logits_in, int64_t m, int d,
                           int n, int k, int fn, int renorm, const float* rank_bias, float* probs_out,
-                          int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+                          int32_t* topk_idx, float* topk_gate, void* workspace, cudaStream_t stream) {
+    if (router_uses_tc(dt, logits_in, n, k))
+        return launch_router_tc(x, w_r, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, workspace,
+                                stream);
     if (dt == MOE_BF16)
         return launch_router_dt<__nv_bfloat16>(x, w_r, logits_in, m, d, n, k, fn, renorm, rank_bias, probs_out,
                                                topk_idx, topk_gate, stream);

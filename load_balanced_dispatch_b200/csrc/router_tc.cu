@@ -1,0 +1,242 @@
+// router_tc.cu -- fp32-accurate router projection on the bf16 tensor cores, with the
+// score function, ranking and top-k fused into the TMEM epilogue.
+//
+// Switch Transformers paper review (tildalice.io/?p=118), selective precision:
+// the router runs in fp32. x is bf16 (exact in fp32); W_r is fp32. Each W_r
+// entry is split into three bf16 parts w = w0 + w1 + w2 (w0 = bf16(w),
+// w1 = bf16(w - w0), w2 = bf16(w - w0 - w1): 3 x 8 mantissa bits = fp32's 24),
+// so x.W_r = x.w0 + x.w1 + x.w2 where every bf16 x bf16 product is exact and
+// the tensor core accumulates in fp32: fp32-accurate logits at tensor-core speed.
+//
+//   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand)
+//   router_tc_kernel     one CTA per 128 tokens, 128 threads:
+//     warp 0 lane 0   TMA: x tile 128x64 + the three 64-wide W parts per stage
+//     warp 1 lane 0   tcgen05.mma kind::f16 M=128 N=np (3 parts x 4 K-steps per stage)
+//     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM
+//                     lane); each K block's product lands in a fresh TMEM accumulator
+//                     (two, ping-pong) and is added into fp32 registers with
+//                     round-to-nearest adds, which keeps the sum fp32-accurate;
+//                     then the warp parks its 32 rows in shared memory and finishes
+//                     them row by row (softmax or sigmoid, key, top-k, gates) with
+//                     the same routine as the FMA router.
+#include "tc_ptx.cuh"
+
+namespace moe {
+
+namespace rtc {
+constexpr int BM = 128, BK = 64, NMAX = 128, STAGES = 3;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 drain + epilogue
+constexpr int A_BYTES = BM * BK * 2;
+}  // namespace rtc
+
+struct RouterTcShared {
+    uint64_t full[rtc::STAGES], empty[rtc::STAGES], tfull[2], tempty[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__host__ __device__ inline int router_np(int n) { return ((n + 31) / 32) * 32; }
+__host__ __device__ inline int router_stage_bytes(int np) { return rtc::A_BYTES + 3 * np * 128; }
+__host__ __device__ inline uint32_t router_tmem_cols(int np) {
+    uint32_t c = 32;
+    while ((int)c < 2 * np) c <<= 1;
+    return c;
+}
+inline size_t router_tc_smem(int np) {
+    return 1024 + (size_t)rtc::STAGES * router_stage_bytes(np) + sizeof(RouterTcShared);
+}
+
+// W_r [d, n] fp32 -> out [3, n, d] bf16 with w = out[0] + out[1] + out[2] (32x32 tiles through shared memory).
+__global__ void router_split_kernel(const float* __restrict__ w_r, int d, int n, __nv_bfloat16* __restrict__ out) {
+    __shared__ float tile[32][33];
+    const int t0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+    for (int r = ty; r < 32; r += 8) {
+        const int t = t0 + r, j = j0 + tx;
+        tile[r][tx] = (t < d && j < n) ? w_r[(int64_t)t * n + j] : 0.f;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int j = j0 + r, t = t0 + tx;
+        if (j >= n || t >= d) continue;
+        const float w = tile[tx][r];
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(p1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r2);
+        const int64_t o = (int64_t)j * d + t, plane = (int64_t)n * d;
+        out[o] = p0;
+        out[plane + o] = p1;
+        out[2 * plane + o] = p2;
+    }
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(rtc::kThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
+                 int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
+                 float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+    using namespace rtc;
+    constexpr int NP = NCH * 32;
+    constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    RouterTcShared* sh = reinterpret_cast<RouterTcShared*>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = (d + BK - 1) / BK;
+    const uint32_t tcols = router_tmem_cols(NP);
+    const int64_t row0 = (int64_t)blockIdx.x * BM;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        sh->abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::prefetch_tensormap(&map_x);
+        ptx::prefetch_tensormap(&map_w);
+    }
+    if (warp == 1) ptx::tmem_alloc(&sh->tmem_base, tcols);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sh->tmem_base;
+    volatile int* abort_flag = &sh->abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) break;
+                uint8_t* st = smem + stage * STAGE_BYTES;
+                ptx::mbar_expect_tx(&sh->full[stage], (uint32_t)STAGE_BYTES);
+                ptx::tma_load_2d(st, &map_x, &sh->full[stage], kb * BK, (int)row0);
+                for (int part = 0; part < 3; ++part)
+                    ptx::tma_load_3d(st + A_BYTES + part * NP * 128, &map_w, &sh->full[stage], kb * BK, 0, part);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, NP);
+            int stage = 0, buf = 0;
+            uint32_t phase = 0, bphase = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!ptx::mbar_wait(&sh->tempty[buf], bphase ^ 1u, abort_flag)) break;
+                if (!ptx::mbar_wait(&sh->full[stage], phase, abort_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t sa = ptx::smem_u32(smem + stage * STAGE_BYTES);
+                const uint64_t adesc = ptx::sw128_kmajor_desc(sa);
+                // a fresh accumulator per K block; the small parts of W first, the leading part last
+                for (int part = 2; part >= 0; --part) {
+                    const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + A_BYTES + part * NP * 128);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        ptx::umma_bf16(tmem + (uint32_t)(buf * NP), adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                       (part != 2 || kk != 0) ? 1u : 0u);
+                }
+                ptx::umma_commit(&sh->empty[stage]);
+                ptx::umma_commit(&sh->tfull[buf]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (++buf == 2) { buf = 0; bphase ^= 1u; }
+            }
+        }
+    } else {
+        // drain: thread owns token row 32*(warp%4) + lane; block results added in fp32 (round to nearest)
+        const int quad = warp & 3;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        float acc[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) acc[j] = 0.f;
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                uint32_t v[32];
+                ptx::tmem_ld32(trow + (uint32_t)(buf * NP + c * 32), v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[q]));
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&sh->tempty[buf]);
+            if (++buf == 2) { buf = 0; bphase ^= 1u; }
+        }
+        // park the warp's 32 logit rows in the (now idle) stage memory, then finish them one row per
+        // step with the compact warp-per-row routine shared with the FMA router
+        if (ok) {
+            float* rows = reinterpret_cast<float*>(smem) + (size_t)quad * 32 * (NP + 1);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) rows[lane * (NP + 1) + j] = acc[j];
+            __syncwarp();
+            for (int rr = 0; rr < 32; ++rr) {
+                const int64_t r = row0 + quad * 32 + rr;
+                if (r >= m) break;
+                float hv[NCH];
+#pragma unroll
+                for (int q = 0; q < NCH; ++q) hv[q] = rows[rr * (NP + 1) + lane + 32 * q];
+                finish_row<NCH>(hv, r, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, tcols);
+    }
+}
+
+size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt) {
+    if (dt != MOE_BF16 || d < 1 || n < 1) return 0;
+    return (size_t)3 * n * d * 2 + 256;
+}
+
+template <int NCH>
+static cudaError_t launch_router_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
+                                      int fn, int renorm, const float* rank_bias, float* probs_out,
+                                      int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    const size_t smem = router_tc_smem(NCH * 32);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
+    router_tc_kernel<NCH><<<(unsigned)blocks, rtc::kThreads, smem, stream>>>(mx, mw, m, d, n, k, fn, renorm, rank_bias,
+                                                                             probs_out, topk_idx, topk_gate);
+    return cudaGetLastError();
+}
+
+// Tensor-core router for bf16 activations with n <= 128 (the drain keeps a token's n logits in registers).
+bool router_tc_supported(int n, int k) { (void)k; return n <= rtc::NMAX; }
+
+cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, int n, int k, int fn, int renorm,
+                             const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
+                             void* workspace, cudaStream_t stream) {
+    if (!router_tc_supported(n, k)) return cudaErrorNotSupported;
+    if (m == 0) return cudaSuccess;
+    __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(workspace);
+    {
+        dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
+        router_split_kernel<<<tg, tb, 0, stream>>>(w_r, d, n, wsplit);
+    }
+    const int np = router_np(n);
+    CUtensorMap mx, mw;
+    if (!map_2d(&mx, x, (uint64_t)m, (uint64_t)d, rtc::BM)) return cudaErrorInvalidValue;
+    if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)np)) return cudaErrorInvalidValue;
+    switch (np / 32) {
+        case 1: return launch_router_tc_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+        case 2: return launch_router_tc_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+        case 3: return launch_router_tc_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+        default: return launch_router_tc_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+    }
+}
+
+}  // namespace moe

@@ -10,10 +10,12 @@
 //
 // Two launches. `partial`: each CTA takes kRows consecutive rows of one
 // segment, sums the probabilities per expert in fp64 (column-parallel,
-// coalesced row reads, fixed order) and counts the routed picks. `final`: one
-// CTA folds the chunks in order, writes f and P per segment and for the whole
-// batch, and reduces the loss terms in a fixed tree order. No floating-point
-// atomics anywhere, so the results are bit-reproducible.
+// coalesced row reads, 8 loads in flight per thread, fixed order) and counts
+// the routed picks. `final`: one CTA; every thread folds the chunks of one
+// (segment, expert) pair in order, then one expert per thread folds the
+// segments for the whole batch, then warps reduce the loss terms in a fixed
+// tree order. No floating-point atomics anywhere, so the results are
+// bit-reproducible.
 #include "common.cuh"
 
 namespace moe {
@@ -37,8 +39,9 @@ static StatsGeometry stats_geometry(int64_t m, int64_t seg_len) {
 size_t stats_workspace_bytes(int64_t m, int32_t n, int64_t seg_len) {
     if (seg_len <= 0) return 0;
     StatsGeometry g = stats_geometry(m, seg_len);
-    // psum [nchunks][n] f64, prod [nseg + 1][n] f64, pcnt [nchunks][n] i32
-    return sizeof(double) * (size_t)n * (size_t)(g.nchunks + g.nseg + 1) + sizeof(int32_t) * (size_t)n * g.nchunks;
+    // psum [nchunks][n] f64, prod [nseg + 1][n] f64, segps [nseg][n] f64, pcnt [nchunks][n] i32, segcnt [nseg][n] i32
+    return sizeof(double) * (size_t)n * (size_t)(g.nchunks + 2 * g.nseg + 1) +
+           sizeof(int32_t) * (size_t)n * (size_t)(g.nchunks + g.nseg);
 }
 
 __global__ void __launch_bounds__(stats::kThreads)
@@ -63,8 +66,18 @@ stats_partial_kernel(const float* __restrict__ probs, const int32_t* __restrict_
         const int groups = stats::kThreads / npad > 0 ? stats::kThreads / npad : 1;
         const int e = tid % npad, gid = tid / npad;
         double s = 0.0;
-        if (gid < groups && e < n)
-            for (int64_t r = r0 + gid; r < r1; r += groups) s += (double)probs[r * n + e];
+        if (gid < groups && e < n) {
+            for (int64_t r = r0 + gid; r < r1; r += 8 * (int64_t)groups) {
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t rr = r + (int64_t)u * groups;
+                    v[u] = rr < r1 ? probs[rr * n + e] : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) s += (double)v[u];
+            }
+        }
         part[tid] = s;
         __syncthreads();
         if (tid < n) {
@@ -94,29 +107,55 @@ __global__ void __launch_bounds__(stats::kThreads)
 stats_final_kernel(const double* __restrict__ psum, const int32_t* __restrict__ pcnt, int has_probs, int64_t m, int n,
                    int k, int64_t seg_len, int64_t nseg, int64_t cps, float alpha, float* __restrict__ f,
                    float* __restrict__ P, float* __restrict__ aux, float* __restrict__ vio,
-                   float* __restrict__ bias, float gamma, double* __restrict__ prod) {
+                   float* __restrict__ bias, float gamma, double* __restrict__ prod, double* __restrict__ segps,
+                   int32_t* __restrict__ segcnt) {
     __shared__ double sh[stats::kThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // phase A: one (segment, expert) pair per thread folds its chunks in order, 8 loads in flight
+    for (int64_t pr = tid; pr < nseg * n; pr += stats::kThreads) {
+        const int64_t s = pr / n;
+        const int e = (int)(pr - s * n);
+        int64_t cs = 0;
+        double ps = 0.0;
+        for (int64_t c0 = 0; c0 < cps; c0 += 8) {
+            int32_t cv[8];
+            double pv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t c = c0 + u;
+                cv[u] = c < cps ? pcnt[(s * cps + c) * n + e] : 0;
+                pv[u] = (has_probs && c < cps) ? psum[(s * cps + c) * n + e] : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) { cs += cv[u]; ps += pv[u]; }
+        }
+        segcnt[s * n + e] = (int32_t)cs;
+        const double fv = (double)cs / ((double)k * (double)seg_len);
+        f[s * n + e] = (float)fv;
+        if (has_probs) {
+            segps[s * n + e] = ps;
+            const double pv = ps / (double)seg_len;
+            P[s * n + e] = (float)pv;
+            prod[s * n + e] = fv * pv;
+        }
+    }
+    __syncthreads();
+    // phase B: the whole batch, one expert per thread, segments in order
     const int e = tid;
     int64_t tot = 0;
     double pall = 0.0;
     if (e < n) {
-        for (int64_t s = 0; s < nseg; ++s) {
-            int64_t cs = 0;
-            double ps = 0.0;
-            for (int64_t c = 0; c < cps; ++c) {
-                cs += pcnt[(s * cps + c) * n + e];
-                if (has_probs) ps += psum[(s * cps + c) * n + e];
+        for (int64_t s0 = 0; s0 < nseg; s0 += 8) {
+            int32_t cv[8];
+            double pv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t s = s0 + u;
+                cv[u] = s < nseg ? segcnt[s * n + e] : 0;
+                pv[u] = (has_probs && s < nseg) ? segps[s * n + e] : 0.0;
             }
-            tot += cs;
-            pall += ps;
-            const double fv = (double)cs / ((double)k * (double)seg_len);
-            f[s * n + e] = (float)fv;
-            if (has_probs) {
-                const double pv = ps / (double)seg_len;
-                P[s * n + e] = (float)pv;
-                prod[s * n + e] = fv * pv;
-            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) { tot += cv[u]; pall += pv[u]; }
         }
         const double fg = (double)tot / ((double)k * (double)m);
         f[nseg * n + e] = (float)fg;
@@ -175,12 +214,15 @@ cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m,
     StatsGeometry g = stats_geometry(m, seg_len);
     double* psum = static_cast<double*>(workspace);
     double* prod = psum + g.nchunks * n;
-    int32_t* pcnt = reinterpret_cast<int32_t*>(prod + (g.nseg + 1) * n);
+    double* segps = prod + (g.nseg + 1) * n;
+    int32_t* pcnt = reinterpret_cast<int32_t*>(segps + g.nseg * n);
+    int32_t* segcnt = pcnt + g.nchunks * n;
     if (g.nchunks > 0)
         stats_partial_kernel<<<(unsigned)g.nchunks, stats::kThreads, 0, stream>>>(probs, topk_idx, n, k, seg_len,
                                                                                   g.cps, psum, pcnt);
     stats_final_kernel<<<1, stats::kThreads, 0, stream>>>(psum, pcnt, probs != nullptr, m, n, k, seg_len, g.nseg,
-                                                          g.cps, alpha, f, P, aux, vio, bias, gamma, prod);
+                                                          g.cps, alpha, f, P, aux, vio, bias, gamma, prod, segps,
+                                                          segcnt);
     return cudaGetLastError();
 }
 

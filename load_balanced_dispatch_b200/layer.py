@@ -68,6 +68,8 @@ class MoELayer:
         L = lib()
         dt = 1 if s.dtype == torch.bfloat16 else 0
         self.ws = dict(
+            router=torch.empty((max(L.moe_router_topk_workspace_size(d, n, k, dt), 1),), dtype=torch.uint8,
+                               device=dev),
             cap=torch.empty((max(L.moe_capacity_slots_workspace_size(m, k, n, seg), 1),), dtype=torch.uint8, device=dev),
             ffn=torch.empty((L.moe_expert_ffn_workspace_size(dt, self.rows_max, s.d_ff),), dtype=torch.uint8,
                             device=dev),
@@ -77,35 +79,72 @@ class MoELayer:
 
     STAGES = ("router", "capacity", "dispatch", "ffn", "combine", "stats")
 
-    def forward(self, x: torch.Tensor, stream=None, events=None) -> torch.Tensor:
-        """One forward. `events`: optional list of 7 CUDA events recorded on the stream around the 6 stages."""
+    def _stage(self, i: int, x: torch.Tensor, st) -> None:
         s, b, w = self.shape, self.buf, self.w
-        st = stream if stream is not None else torch.cuda.current_stream()
-        mark = (lambda i: events[i].record(st)) if events is not None else (lambda i: None)
-        fn = MOE_SOFTMAX if s.score_fn == "softmax" else MOE_SIGMOID
-        mark(0)
-        moe_router_topk(x, w["w_r"], s.n, s.k, fn, s.renorm_topk, rank_bias=w.get("rank_bias"), probs_out=b["probs"],
-                        topk_idx=b["topk_idx"], topk_gate=b["topk_gate"], stream=st)
-        mark(1)
-        cap = moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"],
-                                 stream=st)
-        mark(2)
-        moe_dispatch(x, cap["src_token"], cap["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
-        mark(3)
-        moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], cap["expert_offsets"], ybuf=b["ybuf"],
-                       workspace=self.ws["ffn"], stream=st)
-        mark(4)
-        moe_combine(b["ybuf"], cap["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
-                    stream=st)
-        mark(5)
-        moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
-                          bias_inout=w.get("rank_bias") if s.lossfree else None, gamma=s.gamma, out=b,
-                          workspace=self.ws["stats"], stream=st)
-        mark(6)
-        return b["y"]
+        if i == 0:
+            fn = MOE_SOFTMAX if s.score_fn == "softmax" else MOE_SIGMOID
+            moe_router_topk(x, w["w_r"], s.n, s.k, fn, s.renorm_topk, rank_bias=w.get("rank_bias"),
+                            probs_out=b["probs"], topk_idx=b["topk_idx"], topk_gate=b["topk_gate"],
+                            workspace=self.ws["router"], stream=st)
+        elif i == 1:
+            moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"], stream=st)
+        elif i == 2:
+            moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
+        elif i == 3:
+            moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"], ybuf=b["ybuf"],
+                           workspace=self.ws["ffn"], stream=st)
+        elif i == 4:
+            moe_combine(b["ybuf"], b["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
+                        stream=st)
+        else:
+            moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
+                              bias_inout=w.get("rank_bias") if s.lossfree else None, gamma=s.gamma, out=b,
+                              workspace=self.ws["stats"], stream=st)
 
-    # kernel launches per forward (router 1, capacity 3, dispatch 1, FFN 2, combine 1, stats 2)
-    launches_per_forward = 10
+    def forward(self, x: torch.Tensor, stream=None, events=None) -> torch.Tensor:
+        """One forward through the C ABI. `events`: optional 7 CUDA events recorded around the 6 stages."""
+        st = stream if stream is not None else torch.cuda.current_stream()
+        for i in range(len(self.STAGES)):
+            if events is not None:
+                events[i].record(st)
+            self._stage(i, x, st)
+        if events is not None:
+            events[len(self.STAGES)].record(st)
+        return self.buf["y"]
+
+    def capture(self, x: torch.Tensor) -> None:
+        """Record each stage of forward(x) into its own CUDA graph (x's address is baked in).
+        The first forward runs eagerly so one-time host set-up happens outside the capture."""
+        self.forward(x)
+        torch.cuda.synchronize()
+        self.graphs = []
+        for i in range(len(self.STAGES)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._stage(i, x, torch.cuda.current_stream())
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def replay(self, events=None) -> torch.Tensor:
+        """Replay the captured forward on the current stream, events (optional) between the stages."""
+        st = torch.cuda.current_stream()
+        for i, g in enumerate(self.graphs):
+            if events is not None:
+                events[i].record(st)
+            g.replay()
+        if events is not None:
+            events[len(self.graphs)].record(st)
+        return self.buf["y"]
+
+    def launches_per_forward(self) -> int:
+        """Kernel launches of one forward: router (split + tensor-core kernel for bf16 with n <= 128, else 1),
+        capacity 3, dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
+        combine 1, statistics 2."""
+        s = self.shape
+        bf16 = s.dtype == torch.bfloat16
+        router = 2 if (bf16 and s.n <= 128) else 1
+        ffn = 1 if bf16 else 2
+        return router + 3 + 1 + ffn + 1 + 2
 
 
 def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:

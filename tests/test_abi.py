@@ -43,6 +43,8 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_workspace_queries_are_host_only(L):
+    assert L.moe_router_topk_workspace_size(768, 128, 1, 1) >= 3 * 768 * 128 * 2
+    assert L.moe_router_topk_workspace_size(64, 8, 1, 0) == 0  # fp32 activations: FMA path, no scratch
     assert L.moe_capacity_slots_workspace_size(8192, 1, 128, 8192) > 0
     assert L.moe_expert_ffn_workspace_size(1, 8192, 3072) >= 8192 * 3072 * 2
     assert L.moe_balance_stats_workspace_size(65536, 64, 4096) > 0
@@ -62,7 +64,7 @@ def test_invalid_arguments_rejected_before_any_launch(L):
     rc = L.moe_capacity_slots(fake, 100, 1, 8, 10, 30, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None)
     assert rc == 1 and "seg_len" in _err(L)
     # k > n
-    rc = L.moe_router_topk(fake, 1, fake, None, 16, 8, 4, 5, 0, 0, None, None, fake, fake, None)
+    rc = L.moe_router_topk(fake, 1, fake, None, 16, 8, 4, 5, 0, 0, None, None, fake, fake, None, 0, None)
     assert rc == 1 and "k must be" in _err(L)
     # m*k not divisible by n for the balanced assignment
     rc = L.moe_balance_assign(fake, 10, 4, 1, fake, 1, 0, 4, 4, fake, fake, fake, 1 << 30, None)
@@ -70,6 +72,9 @@ def test_invalid_arguments_rejected_before_any_launch(L):
     # k must be < n for the balanced assignment
     rc = L.moe_balance_assign(fake, 8, 4, 4, fake, 1, 0, 4, 4, fake, fake, fake, 1 << 30, None)
     assert rc == 1
+    # bf16 router without its workspace
+    rc = L.moe_router_topk(fake, 1, fake, None, 16, 64, 8, 2, 0, 0, None, None, fake, fake, None, 0, None)
+    assert rc == 3 and "workspace" in _err(L)
     # workspace too small
     rc = L.moe_capacity_slots(fake, 64, 1, 8, 10, 64, fake, fake, fake, fake, fake, fake, fake, 0, None)
     assert rc == 3 and "workspace" in _err(L)

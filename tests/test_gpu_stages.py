@@ -59,16 +59,22 @@ def test_router_logits_in_sigmoid(m, n, k, bias):
     assert np.allclose(host(probs), p_ref, rtol=1e-6)
 
 
-@pytest.mark.parametrize("dtype,m,d,n,k", [("fp32", 1000, 64, 8, 1), ("bf16", 517, 768, 128, 1),
-                                           ("bf16", 300, 200, 64, 6), ("fp32", 129, 36, 256, 8)])
-def test_router_projection(dtype, m, d, n, k):
-    rng = np.random.default_rng(d)
+@pytest.mark.parametrize("dtype,m,d,n,k,fn,renorm,bias", [
+    ("fp32", 1000, 64, 8, 1, 0, 0, False), ("bf16", 517, 768, 128, 1, 0, 0, False),
+    ("bf16", 300, 200, 64, 6, 0, 1, False), ("fp32", 129, 36, 256, 8, 0, 0, False),
+    ("bf16", 700, 2048, 64, 6, 1, 0, True), ("bf16", 259, 128, 256, 8, 0, 1, False),
+    ("bf16", 1000, 96, 40, 3, 1, 0, False), ("bf16", 131, 4096, 64, 2, 0, 1, False),
+    ("bf16", 64, 64, 16, 12, 0, 0, False)])
+def test_router_projection(dtype, m, d, n, k, fn, renorm, bias):
+    rng = np.random.default_rng(d + n)
     x = rng.standard_normal((m, d)).astype(np.float32)
     if dtype == "bf16":
         x = W.round_to_bf16(x)
     w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
-    p_ref, i_ref, g_ref, margin = oracle.router(x, w, m, d, n, k)
-    idx, gate, probs = lb.moe_router_topk(dev(x, torch_dtype(dtype)), dev(w), n, k)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32) if bias else None
+    p_ref, i_ref, g_ref, margin = oracle.router(x, w, m, d, n, k, fn, renorm, b)
+    idx, gate, probs = lb.moe_router_topk(dev(x, torch_dtype(dtype)), dev(w), n, k, fn, renorm,
+                                          rank_bias=None if b is None else dev(b))
     torch.cuda.synchronize()
     ok = margin > MARGIN
     assert ok.mean() > 0.97
@@ -209,7 +215,8 @@ def test_balance_step_bitexact(m, n, k, rule):
 
 
 @pytest.mark.parametrize("m,n,k,iters,rule", [(2048, 32, 4, 8, 0), (2048, 32, 4, 0, 0), (1024, 16, 2, 3, 1),
-                                              (4096, 64, 8, 20, 0), (512, 8, 1, 2, 0)])
+                                              (4096, 64, 8, 20, 0), (512, 8, 1, 2, 0), (4096, 64, 8, 40, 0),
+                                              (2048, 16, 3, 33, 1)])
 def test_balance_solve_bitexact(m, n, k, iters, rule):
     s = W.make_qb_scores(m, n, seed=m * 3 + n)
     i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, rule=rule, max_iters=iters)
@@ -220,3 +227,17 @@ def test_balance_solve_bitexact(m, n, k, iters, rule):
     assert (host(beta) == b_ref).all()
     assert (host(idx) == i_ref).all()
     assert (np.bincount(host(idx).ravel(), minlength=n) == m * k // n).all()
+
+
+@pytest.mark.parametrize("m,n,k,seed", [(1024, 8, 2, 0), (2048, 16, 2, 2), (4096, 32, 4, 1), (512, 4, 1, 0)])
+def test_balance_solve_converges_inside_a_batch(m, n, k, seed):
+    # mild skew: QB alone reaches exact balance after 6..45 beta updates (no repair), so the
+    # early exit happens inside, or at the edge of, a batch of enqueued iterations
+    s = W.make_qb_scores(m, n, seed=seed, skew_std=0.5)
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=60)
+    assert rc == oracle.OK and info_ref[1] == 0 and info_ref[0] < 60
+    idx, beta, info = lb.moe_balance_assign(dev(s), k, mode=lb.MOE_QB_SOLVE, max_iters=60)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
