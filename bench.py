@@ -263,25 +263,50 @@ def run_gpu(args, cfg):
                 for j, s in enumerate(MoELayer.STAGES)}
     offsets = layer.buf["expert_offsets"].cpu().numpy()
 
-    # end-to-end through the public API: host x -> device, forward, y and the loss -> host, every step
-    y_host = torch.empty((cfg.m, cfg.d), dtype=dt).pin_memory()
-    aux_host = torch.empty(layer.buf["aux"].shape, dtype=torch.float32).pin_memory()
-    for _ in range(2):
-        x.copy_(x_host, non_blocking=True)
-        run()
-        y_host.copy_(layer.buf["y"], non_blocking=True)
-        aux_host.copy_(layer.buf["aux"], non_blocking=True)
+    # end-to-end through the public API, as a serving loop runs it: every step copies its input
+    # from pinned host memory, runs the layer and reads the output and the loss back. Two layer
+    # instances (shared weights, own buffers) alternate so step t's copies overlap the neighbours'
+    # compute; events order the reuse of each instance's buffers.
+    layers = [layer, MoELayer(shape, w)]
+    xs = [x, torch.empty_like(x)]
+    if not args.eager:
+        layers[1].capture(xs[1])
+    runs = [run, (lambda events=None: layers[1].forward(xs[1], events=events)) if args.eager else layers[1].replay]
+    y_host = [torch.empty((cfg.m, cfg.d), dtype=dt).pin_memory() for _ in range(2)]
+    aux_host = [torch.empty(layer.buf["aux"].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(t):
+        b = t % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[b])          # the instance's previous forward has read its input
+            xs[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            s_cmp.wait_event(ev_out[b])         # its previous output has been read back
+            runs[b]()
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            y_host[b].copy_(layers[b].buf["y"], non_blocking=True)
+            aux_host[b].copy_(layers[b].buf["aux"], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    torch.cuda.synchronize()
+    for t in range(4):
+        e2e_step(t)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        x.copy_(x_host, non_blocking=True)
-        run()
-        y_host.copy_(layer.buf["y"], non_blocking=True)
-        aux_host.copy_(layer.buf["aux"], non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    for t in range(args.steps):
+        e2e_step(t)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), device="cuda")
     lb.sync_status()
@@ -321,7 +346,8 @@ def run_gpu(args, cfg):
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_tokens_per_s(cfg.m, args.steps, world, ms_e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-                    "d2h_bytes_per_step": y_host.numel() * y_host.element_size() + aux_host.numel() * 4},
+                    "d2h_bytes_per_step": y_host[0].numel() * y_host[0].element_size() + aux_host[0].numel() * 4,
+                    "pipelined": "host copies of step t overlap compute of steps t-1 and t+1 (3 streams)"},
             "clocks": clk,
             "gpu_launches": args.steps * layer.launches_per_forward(),
         }

@@ -358,67 +358,121 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
 }
 
 namespace qb {
-constexpr int kArcThreads = 512;     // 16 warps scan the tokens
+constexpr int kArcThreads = 512;     // 16 warps
+constexpr int kArcBatch = 4;         // members per warp step (their loads in flight together)
+constexpr int kArcWords = 512;       // bitmap words compacted per pass: at most 16384 members
+constexpr int kMemberCap = kArcWords * 32;
 constexpr int kStepThreads = 1024;   // 4 threads per expert column in the shortest-path rounds
+constexpr size_t kArcSmem = (size_t)(kArcThreads / 32) * kMaxExperts * (8 + 4) + (size_t)kMemberCap * 4;
 }  // namespace qb
+
+// Membership bitmap: bit i of row e is set when token i holds expert e.
+__global__ void qb_member_bits_kernel(const int32_t* __restrict__ topk_idx, int64_t m, int k, int64_t words,
+                                      uint32_t* __restrict__ mem) {
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= m * k) return;
+    const int64_t i = q / k;
+    const int e = topk_idx[q];
+    atomicOr(&mem[(int64_t)e * words + (i >> 5)], 1u << (i & 31));
+}
 
 // Arc costs of the expert graph for the listed rows a = rows[blockIdx.x]:
 // W[a][b] = min over tokens i holding a but not b of s_ia - s_ib (fp64), A[a][b] = that token
-// (lowest token among equal costs). Each warp scans chunks of 32 tokens, finds the members of a
-// by ballot, and for each member the lanes test their columns b = lane + 32 q against its k
-// experts; the 16 warps' minima are folded in warp order at the end.
+// (lowest token among equal costs). The members of a come from the bitmap (compacted into shared
+// memory, kMemberCap at a time); warp w takes members in batches of kArcBatch, lanes own columns
+// b = lane + 32 q; the 32 warps' minima are folded in warp order at the end.
 template <int NT>
-__global__ void __launch_bounds__(qb::kArcThreads)
+__global__ void __launch_bounds__(qb::kArcThreads, 1)
 qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_t* __restrict__ topk_idx,
-              const int32_t* __restrict__ rows, const int32_t* __restrict__ nrows, double* __restrict__ W,
-              int32_t* __restrict__ A, const int32_t* __restrict__ status) {
+              const uint32_t* __restrict__ mem, int64_t words, const int32_t* __restrict__ rows,
+              const int32_t* __restrict__ nrows, double* __restrict__ W, int32_t* __restrict__ A,
+              const int32_t* __restrict__ status) {
     if (status[qb::kStError] || status[qb::kStDone]) return;
     if ((int)blockIdx.x >= *nrows) return;
-    constexpr int NW = qb::kArcThreads / 32;
-    __shared__ double bw[NW][kMaxExperts];
-    __shared__ int32_t ba[NW][kMaxExperts];
+    constexpr int NW = qb::kArcThreads / 32, B = qb::kArcBatch;
+    extern __shared__ unsigned char arc_smem[];
+    double* bw = reinterpret_cast<double*>(arc_smem);                       // [NW][256]
+    int32_t* ba = reinterpret_cast<int32_t*>(bw + NW * kMaxExperts);         // [NW][256]
+    int32_t* list = ba + NW * kMaxExperts;                                   // [kMemberCap]
+    __shared__ int nlist;
     const int a = rows[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t* row = mem + (int64_t)a * words;
     double best[NT];
     int32_t arg[NT];
 #pragma unroll
     for (int q = 0; q < NT; ++q) { best[q] = INFINITY; arg[q] = 0x7fffffff; }
-    for (int64_t base = (int64_t)warp * 32; base < m; base += (int64_t)NW * 32) {
-        const int64_t i = base + lane;
-        bool mem = false;
-        if (i < m)
-            for (int r = 0; r < k; ++r) mem |= topk_idx[i * k + r] == a;
-        uint32_t bal = __ballot_sync(0xffffffffu, mem);
-        while (bal) {
-            const int src = __ffs(bal) - 1;
-            bal &= bal - 1;
-            const int64_t ti = base + src;
-            uint32_t in = 0;  // bit q: column lane + 32 q belongs to the token's set
-            for (int r = 0; r < k; ++r) {
-                const int e = topk_idx[ti * k + r];
+    for (int64_t w0 = 0; w0 < words; w0 += qb::kArcWords) {
+        // compact the members held in the next kArcWords bitmap words (token order is not needed:
+        // ties go to the lowest token explicitly)
+        if (threadIdx.x == 0) nlist = 0;
+        __syncthreads();
+        {
+            const int64_t wi = w0 + threadIdx.x;
+            const uint32_t bits = (threadIdx.x < qb::kArcWords && wi < words) ? row[wi] : 0u;
+            const int c = __popc(bits);
+            int incl = c;
 #pragma unroll
-                for (int q = 0; q < NT; ++q) in |= (e == lane + 32 * q) ? (1u << q) : 0u;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
             }
-            const double sa = (double)s[ti * n + a];
+            int base = 0;
+            if (lane == 31 && incl) base = atomicAdd(&nlist, incl);
+            base = __shfl_sync(0xffffffffu, base, 31);
+            int pos = base + incl - c;
+            uint32_t bb = bits;
+            while (bb) {
+                const int bit = __ffs(bb) - 1;
+                bb &= bb - 1;
+                list[pos++] = (int32_t)((wi << 5) + bit);
+            }
+        }
+        __syncthreads();
+        const int cnt = nlist;
+        for (int p0 = warp * B; p0 < cnt; p0 += NW * B) {
+            int32_t id[B];
+            float sa[B], sb[B][NT];
+            int32_t ex[B];
 #pragma unroll
-            for (int q = 0; q < NT; ++q) {
-                const int b = lane + 32 * q;
-                if (b < n && !((in >> q) & 1u)) {
-                    const double c = sa - (double)s[ti * n + b];
-                    if (c < best[q] || (c == best[q] && ti < arg[q])) { best[q] = c; arg[q] = (int32_t)ti; }
+            for (int u = 0; u < B; ++u) {
+                id[u] = p0 + u < cnt ? list[p0 + u] : -1;
+                const int64_t ti = id[u] >= 0 ? id[u] : 0;
+                sa[u] = s[ti * n + a];
+                ex[u] = lane < k ? topk_idx[ti * k + lane] : -1;
+#pragma unroll
+                for (int q = 0; q < NT; ++q) sb[u][q] = (lane + 32 * q < n) ? s[ti * n + lane + 32 * q] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                if (id[u] < 0) continue;  // warp-uniform
+                uint32_t in = 0;  // bit q: column lane + 32 q belongs to the member's set
+                for (int r = 0; r < k; ++r) {
+                    const int e = k <= 32 ? __shfl_sync(0xffffffffu, ex[u], r & 31) : topk_idx[(int64_t)id[u] * k + r];
+#pragma unroll
+                    for (int q = 0; q < NT; ++q) in |= (e == lane + 32 * q) ? (1u << q) : 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const int b = lane + 32 * q;
+                    if (b < n && !((in >> q) & 1u)) {
+                        const double c = (double)sa[u] - (double)sb[u][q];
+                        if (c < best[q] || (c == best[q] && id[u] < arg[q])) { best[q] = c; arg[q] = id[u]; }
+                    }
                 }
             }
         }
+        __syncthreads();
     }
 #pragma unroll
-    for (int q = 0; q < NT; ++q) { bw[warp][lane + 32 * q] = best[q]; ba[warp][lane + 32 * q] = arg[q]; }
+    for (int q = 0; q < NT; ++q) { bw[warp * kMaxExperts + lane + 32 * q] = best[q]; ba[warp * kMaxExperts + lane + 32 * q] = arg[q]; }
     __syncthreads();
     for (int b = threadIdx.x; b < n; b += blockDim.x) {
         double bb = INFINITY;
         int32_t aa = -1;
         for (int w = 0; w < NW; ++w) {
-            const double c = bw[w][b];
-            const int32_t t = ba[w][b];
+            const double c = bw[w * kMaxExperts + b];
+            const int32_t t = ba[w * kMaxExperts + b];
             if (c < bb || (c == bb && c != INFINITY && t < aa)) { bb = c; aa = t; }
         }
         W[(int64_t)a * n + b] = bb;
@@ -433,10 +487,11 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
 __global__ void __launch_bounds__(qb::kStepThreads)
 qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, const int32_t* __restrict__ A,
                       int32_t* __restrict__ counts, int32_t* __restrict__ topk_idx, int32_t* __restrict__ status,
-                      int32_t* __restrict__ rows, int32_t* __restrict__ nrows) {
+                      int32_t* __restrict__ rows, int32_t* __restrict__ nrows, uint32_t* __restrict__ mem,
+                      int64_t words) {
     __shared__ double dist[kMaxExperts], part_d[4][kMaxExperts];
     __shared__ int part_p[4][kMaxExperts], pred[kMaxExperts];
-    __shared__ int any_over, changed;
+    __shared__ int any_over;
     __shared__ uint32_t touched[kMaxExperts / 32];
     const int tid = threadIdx.x;
     const int b = tid & 255, part = tid >> 8;  // 4 threads per column b, each a quarter of the a range
@@ -454,20 +509,39 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         if (tid == 0) { status[qb::kStDone] = 1; *nrows = 0; }
         return;
     }
-    const int qa = (n + 3) / 4, a0 = part * qa, a1 = min(n, a0 + qa);
+    // Jacobi rounds over the frontier: only experts whose distance changed in the previous round
+    // can improve another one, so each round reads just their rows of W (same fixpoint as full rounds)
+    __shared__ int front[kMaxExperts], nfront;
+    __shared__ unsigned char chg[kMaxExperts];
+    if (tid < kMaxExperts) chg[tid] = (tid < n && dist[tid] == 0.0) ? 1 : 0;
+    __syncthreads();
     bool settled = false;
     for (int round = 0; round <= n; ++round) {
-        if (tid == 0) changed = 0;
+        if (tid == 0) {
+            int c = 0;
+            for (int a = 0; a < n; ++a)
+                if (chg[a]) front[c++] = a;
+            nfront = c;
+        }
+        __syncthreads();
+        const int nf = nfront;
+        if (nf == 0) { settled = true; break; }
         double bestd = INFINITY;
         if (b < n) {
-            for (int a = a0; a < a1; a += 8) {
+            // this thread's quarter of the frontier, 8 loads in flight
+            for (int f0 = part; f0 < nf; f0 += 4 * 8) {
                 double w8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) w8[u] = (a + u < a1) ? W[(int64_t)(a + u) * n + b] : INFINITY;
+                int a8[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int aa = a + u;
-                    if (aa < a1 && aa != b && dist[aa] != INFINITY && w8[u] != INFINITY) {
+                    const int fi = f0 + 4 * u;
+                    a8[u] = fi < nf ? front[fi] : -1;
+                    w8[u] = a8[u] >= 0 ? W[(int64_t)a8[u] * n + b] : INFINITY;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int aa = a8[u];
+                    if (aa >= 0 && aa != b && w8[u] != INFINITY) {
                         const double c = dist[aa] + w8[u];
                         if (c < bestd) bestd = c;
                     }
@@ -476,23 +550,26 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         }
         part_d[part][b] = bestd;
         __syncthreads();
-        if (part == 0 && b < n) {
-            double nd = dist[b];
-            for (int p = 0; p < 4; ++p) nd = fmin(nd, part_d[p][b]);
-            if (nd != dist[b]) changed = 1;
-            part_d[0][b] = nd;
+        if (part == 0) {
+            if (b < n) {
+                double nd = dist[b];
+                for (int p = 0; p < 4; ++p) nd = fmin(nd, part_d[p][b]);
+                chg[b] = nd != dist[b];
+                part_d[0][b] = nd;
+            } else {
+                chg[b] = 0;
+            }
         }
         __syncthreads();
-        const int ch = changed;
         if (part == 0 && b < n) dist[b] = part_d[0][b];
         __syncthreads();
-        if (!ch) { settled = true; break; }
     }
-    if (!settled) {
+    if (!settled) {  // still improving after n rounds: a negative cycle, which an optimal start excludes
         if (tid == 0) { status[qb::kStError] = 1; record_error(kErrRepair); *nrows = 0; }
         return;
     }
-    // predecessor: lowest a with dist[a] + W[a][b] == dist[b]
+    // predecessor: lowest a with dist[a] + W[a][b] == dist[b] (4 threads per column, a quarter each)
+    const int qa = (n + 3) / 4, a0 = part * qa, a1 = min(n, a0 + qa);
     int pa = 0x7fffffff;
     if (b < n && dist[b] != INFINITY) {
         for (int a = a0; a < a1; ++a) {
@@ -534,6 +611,8 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
             }
             if (pos < 0 || hasb) { ok = false; break; }
             touched[bb >> 5] |= 1u << (bb & 31);
+            mem[(int64_t)a * words + (i >> 5)] &= ~(1u << (i & 31));
+            mem[(int64_t)bb * words + (i >> 5)] |= 1u << (i & 31);
             int r = pos;
             row[r] = bb;
             while (r > 0 && row[r - 1] > row[r]) { const int t2 = row[r - 1]; row[r - 1] = row[r]; row[r] = t2; --r; }
@@ -580,6 +659,7 @@ struct QBWorkspace {
     int32_t* A;
     int32_t* rows;
     int32_t* nrows;
+    uint32_t* mem;   // [n][ceil(m / 32)] membership bitmap
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -597,6 +677,7 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     p = take(sizeof(int32_t) * (size_t)n * n);          if (w) w->A = (int32_t*)p;
     p = take(sizeof(int32_t) * (size_t)n);              if (w) w->rows = (int32_t*)p;
     p = take(sizeof(int32_t));                          if (w) w->nrows = (int32_t*)p;
+    p = take(sizeof(uint32_t) * (size_t)n * (size_t)((m + 31) / 32)); if (w) w->mem = (uint32_t*)p;
     return off;
 }
 
@@ -622,16 +703,24 @@ static void launch_row(const float* s, int64_t m, int n, int k, const float* bet
     else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, stream);
 }
 
+template <int NT>
+static void launch_arc_t(const float* s, int64_t m, int n, int k, const int32_t* topk_idx, const QBWorkspace& w,
+                         cudaStream_t stream) {
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(qb_arc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qb::kArcSmem);
+        attr = true;
+    }
+    qb_arc_kernel<NT><<<n, qb::kArcThreads, qb::kArcSmem, stream>>>(s, m, n, k, topk_idx, w.mem, (m + 31) / 32,
+                                                                    w.rows, w.nrows, w.W, w.A, w.status);
+}
+
 static void launch_arc(const float* s, int64_t m, int n, int k, const int32_t* topk_idx, const QBWorkspace& w,
                        cudaStream_t stream) {
-    if (n <= 32)
-        qb_arc_kernel<1><<<n, qb::kArcThreads, 0, stream>>>(s, m, n, k, topk_idx, w.rows, w.nrows, w.W, w.A, w.status);
-    else if (n <= 64)
-        qb_arc_kernel<2><<<n, qb::kArcThreads, 0, stream>>>(s, m, n, k, topk_idx, w.rows, w.nrows, w.W, w.A, w.status);
-    else if (n <= 128)
-        qb_arc_kernel<4><<<n, qb::kArcThreads, 0, stream>>>(s, m, n, k, topk_idx, w.rows, w.nrows, w.W, w.A, w.status);
-    else
-        qb_arc_kernel<8><<<n, qb::kArcThreads, 0, stream>>>(s, m, n, k, topk_idx, w.rows, w.nrows, w.W, w.A, w.status);
+    if (n <= 32) launch_arc_t<1>(s, m, n, k, topk_idx, w, stream);
+    else if (n <= 64) launch_arc_t<2>(s, m, n, k, topk_idx, w, stream);
+    else if (n <= 128) launch_arc_t<4>(s, m, n, k, topk_idx, w, stream);
+    else launch_arc_t<8>(s, m, n, k, topk_idx, w, stream);
 }
 
 // Returns a moe_status; SOLVE synchronises the stream between phases.
@@ -695,11 +784,18 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
         // exact finish: one shortest-path move per unit of excess; W is built for every row once,
         // then only the rows a move invalidates are recomputed
         const int64_t moves = excess < max_repair ? excess : max_repair;
-        if (moves > 0) qb_all_rows_kernel<<<1, 256, 0, stream>>>(n, w.rows, w.nrows);
+        if (moves > 0) {
+            const int64_t words = (m + 31) / 32;
+            if ((ce = cudaMemsetAsync(w.mem, 0, sizeof(uint32_t) * (size_t)n * (size_t)words, stream)) != cudaSuccess)
+                goto cuda_fail;
+            qb_member_bits_kernel<<<(unsigned)((m * k + 255) / 256), 256, 0, stream>>>(topk_idx, m, k, words, w.mem);
+            qb_all_rows_kernel<<<1, 256, 0, stream>>>(n, w.rows, w.nrows);
+        }
         for (int64_t a = 0; a < moves; ++a) {
             launch_arc(s, m, n, k, topk_idx, w, stream);
             qb_repair_step_kernel<<<1, qb::kStepThreads, 0, stream>>>(n, C, k, w.W, w.A, final_counts, topk_idx,
-                                                                      w.status, w.rows, w.nrows);
+                                                                      w.status, w.rows, w.nrows, w.mem,
+                                                                      (m + 31) / 32);
         }
         qb_info_kernel<<<1, 32, 0, stream>>>(final_counts, n, C, w.status, iters,
                                              iters % 2 ? qb::kStTies1 : qb::kStTies0, info);

@@ -4,17 +4,28 @@
 // FFN(x) = max(0, x W1 + b1) W2 + b2 per expert.
 //
 // The tile list holds every GEMM1 tile (h = relu(xbuf W1_e^T + b1_e), bf16)
-// followed by every GEMM2 tile (ybuf = h W2_e^T + b2_e). Each CTA walks its
-// tiles in increasing order, so it finishes all of its GEMM1 tiles before its
-// first GEMM2 tile; with every CTA resident at once (cooperative launch) each
-// GEMM1 tile therefore completes, and a GEMM2 tile of expert e only waits for
-// the GEMM1 tiles of e. That wait is a per-expert counter in global memory:
+// followed by every GEMM2 tile (ybuf = h W2_e^T + b2_e). CTAs take tiles from
+// a global ticket counter (dynamic scheduling balances the unequal tiles: a
+// GEMM2 tile streams four times the weight bytes of a GEMM1 tile at the
+// Switch-Base shape). Tickets are taken in list order and only by running
+// CTAs, so every GEMM1 tile a GEMM2 tile waits for is held by a running CTA
+// that needs nothing else to finish it: no deadlock without co-residency.
+// A GEMM2 tile of expert e waits for a per-expert counter in global memory:
 // each epilogue warp of a GEMM1 tile stores its h rows, fences them for the
 // async (TMA) proxy and release-adds 1; the producer of a GEMM2 tile
 // acquire-polls the counter (bounded), fences, then loads h with TMA. One
 // launch instead of two removes the second kernel's prologue and the wave
-// tail between the GEMMs. Warp roles, pipeline and epilogue are those of the
-// two-launch kernel in ffn_tc.cu; every wait is bounded.
+// tail between the GEMMs.
+//
+// One CTA per SM, 192 threads: warp 0 takes tickets and runs the TMA producer
+// (4-stage ring of a 128x64 A tile and a 256x64 B tile, 128-byte swizzle,
+// K-major, no multicast); warp 1's lane 0 issues tcgen05.mma kind::f16
+// (M=128, N=256, K=16, bf16 x bf16 -> fp32 in TMEM) and commits each stage
+// back; warps 2-5 drain one of two TMEM accumulators (tcgen05.ld, + bias,
+// ReLU for GEMM1, bf16, 16-byte stores) while the other fills. Row tails past
+// an expert's end are computed and masked; column and K tails are TMA zero
+// fill. Every wait is bounded (about 2 s), after which the device error word
+// and an abort flag are set and all roles leave their loops.
 #include "groups.cuh"
 #include "tc_ptx.cuh"
 
@@ -27,10 +38,14 @@ constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTE
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
 constexpr int kEpiWarps = 4;
+constexpr int RING = 4;   // tile ids handed from the producer to the MMA and epilogue warps
 }  // namespace fz
 
 struct FusedShared {
     uint64_t full[fz::STAGES], empty[fz::STAGES], tfull[2], tempty[2];
+    uint64_t tready[fz::RING], tfree[fz::RING];
+    int tile_ring[fz::RING];
+    __align__(16) __nv_bfloat16 bias_stage[fz::kEpiWarps][fz::BN];  // each epilogue warp's copy of its tile's bias
     uint32_t tmem_base;
     int abort_flag;
     GroupTable g1, g2;
@@ -67,7 +82,8 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
              const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_w2,
              const __nv_bfloat16* __restrict__ b1, const __nv_bfloat16* __restrict__ b2,
              const int32_t* __restrict__ offsets, int n, int d, int d_ff, int64_t max_rows,
-             __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ y, int* __restrict__ done1) {
+             __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ y, int* __restrict__ done1,
+             int* __restrict__ next_tile) {
     using namespace fz;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -78,6 +94,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
         for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        for (int r = 0; r < RING; ++r) { ptx::mbar_init(&sh->tready[r], 1); ptx::mbar_init(&sh->tfree[r], 1 + kEpiWarps); }
         sh->abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::prefetch_tensormap(&map_x);
@@ -98,9 +115,16 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
 
     if (warp == 0) {
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int stage = 0, slot = 0;
+            uint32_t phase = 0, rphase = 0;
+            for (;;) {
+                // take the next tile of the launch and hand its id to the MMA and epilogue warps
+                if (!ptx::mbar_wait(&sh->tfree[slot], rphase ^ 1u, abort_flag)) break;
+                const int tile = atomicAdd(next_tile, 1);
+                sh->tile_ring[slot] = tile < total ? tile : -1;
+                ptx::mbar_arrive(&sh->tready[slot]);
+                if (++slot == RING) { slot = 0; rphase ^= 1u; }
+                if (tile >= total) break;
                 const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
                 if (t.phase == 2) {
                     // all GEMM1 tiles of expert e, each signalled by its 4 epilogue warps
@@ -136,9 +160,14 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, aphase = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int stage = 0, acc = 0, slot = 0;
+            uint32_t phase = 0, aphase = 0, rphase = 0;
+            for (;;) {
+                if (!ptx::mbar_wait(&sh->tready[slot], rphase, abort_flag)) break;
+                const int tile = *(volatile int*)&sh->tile_ring[slot];
+                ptx::mbar_arrive(&sh->tfree[slot]);
+                if (++slot == RING) { slot = 0; rphase ^= 1u; }
+                if (tile < 0) break;
                 const int K = tile < T1 ? d : d_ff;
                 const int nkb = (K + BK - 1) / BK;
                 if (!ptx::mbar_wait(&sh->tempty[acc], aphase ^ 1u, abort_flag)) break;
@@ -164,16 +193,30 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         }
     } else {
         const int quad = warp & 3;
-        int acc = 0;
-        uint32_t aphase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        int acc = 0, slot = 0;
+        uint32_t aphase = 0, rphase = 0;
+        for (;;) {
+            if (!ptx::mbar_wait(&sh->tready[slot], rphase, abort_flag)) break;
+            const int tile = *(volatile int*)&sh->tile_ring[slot];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sh->tfree[slot]);
+            if (++slot == RING) { slot = 0; rphase ^= 1u; }
+            if (tile < 0) break;
             const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
+            // stage the tile's 256 bias values in shared memory while the accumulator fills
+            __nv_bfloat16* be = sh->bias_stage[warp - 2];
+            {
+                const __nv_bfloat16* gb = (t.phase == 1 ? b1 : b2) + (int64_t)t.e * t.N;
+                const int col = t.n0 + lane * 8;
+                if (col < t.N)
+                    *reinterpret_cast<uint4*>(be + lane * 8) = *reinterpret_cast<const uint4*>(gb + col);
+                __syncwarp();
+            }
             if (!ptx::mbar_wait(&sh->tfull[acc], aphase, abort_flag)) break;
             ptx::tc_fence_after();
             const int64_t r = t.row0 + quad * 32 + lane;
             const bool row_ok = r < t.row_end;
             const bool relu = t.phase == 1;
-            const __nv_bfloat16* be = (t.phase == 1 ? b1 : b2) + (int64_t)t.e * t.N;
             __nv_bfloat16* out = t.phase == 1 ? h : y;
             for (int c = 0; c < BN / 32; ++c) {
                 const int col0 = t.n0 + c * 32;
@@ -185,7 +228,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                     const int col = col0 + g8 * 8;
                     if (col >= t.N) break;
                     float f[8], bv[8];
-                    Vec16<__nv_bfloat16>::load(be + col, bv);
+                    Vec16<__nv_bfloat16>::load(be + (col - t.n0), bv);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         f[q] = __uint_as_float(v[g8 * 8 + q]) + bv[q];
@@ -218,38 +261,27 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
 
 cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
                              const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
-                             int* done1, cudaStream_t stream) {
+                             int* counters, cudaStream_t stream) {
     CUtensorMap mx, mw1, mh, mw2;
     if (!map_2d(&mx, xbuf, (uint64_t)max_rows, (uint64_t)d, fz::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw1, w1, (uint64_t)n, (uint64_t)d_ff, (uint64_t)d, fz::BN)) return cudaErrorInvalidValue;
     if (!map_2d(&mh, hbuf, (uint64_t)max_rows, (uint64_t)d_ff, fz::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw2, w2, (uint64_t)n, (uint64_t)d, (uint64_t)d_ff, fz::BN)) return cudaErrorInvalidValue;
-    static int grid = 0;
+    static bool attr = false;
     const size_t smem = fused_smem_bytes();
-    if (!grid) {
+    if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(ffn_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ffn_fused_tc, fz::kThreads, smem);
-        if (e != cudaSuccess) return e;
-        if (per_sm < 1) return cudaErrorInvalidConfiguration;
-        grid = num_sms();  // one CTA per SM (all resident: the cooperative launch checks it)
+        attr = true;
     }
-    cudaError_t e = cudaMemsetAsync(done1, 0, sizeof(int) * (size_t)n, stream);
+    // counters[0..n-1]: GEMM1 completions per expert; counters[n]: next tile ticket
+    cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(fz::kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ffn_fused_tc, mx, mw1, mh, mw2, static_cast<const __nv_bfloat16*>(b1),
-                              static_cast<const __nv_bfloat16*>(b2), offsets, n, d, d_ff, max_rows,
-                              static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), done1);
+    ffn_fused_tc<<<num_sms(), fz::kThreads, smem, stream>>>(
+        mx, mw1, mh, mw2, static_cast<const __nv_bfloat16*>(b1), static_cast<const __nv_bfloat16*>(b2), offsets, n,
+        d, d_ff, max_rows, static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), counters,
+        counters + n);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

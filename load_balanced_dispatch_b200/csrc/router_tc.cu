@@ -72,6 +72,57 @@ __global__ void router_split_kernel(const float* __restrict__ w_r, int d, int n,
     }
 }
 
+constexpr int KTHREAD = 8;  // largest k finished one row per thread
+
+// Finish one token row in one thread: h[0..n) in shared memory (stride-1 within the row).
+// Same definitions as finish_row: softmax / logistic in fp32, key = score + bias or the
+// logit (softmax) / rho (sigmoid), top-k with ties to the lower index, gates.
+__device__ __noinline__ void finish_row_thread(const float* __restrict__ h, int64_t row, int n, int k, int fn,
+                                               int renorm, const float* __restrict__ rank_bias,
+                                               float* __restrict__ probs_out, int32_t* __restrict__ topk_idx,
+                                               float* __restrict__ topk_gate) {
+    float mx = -INFINITY, sum = 0.f;
+    if (fn == MOE_SOFTMAX) {
+        for (int j = 0; j < n; ++j) mx = fmaxf(mx, h[j]);
+        for (int j = 0; j < n; ++j) sum += expf(h[j] - mx);
+    }
+    float kk[KTHREAD], kp[KTHREAD];
+    int ki[KTHREAD];
+#pragma unroll
+    for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
+    float* prow = probs_out ? probs_out + row * n : nullptr;
+    for (int j = 0; j < n; ++j) {
+        const float hj = h[j];
+        const float p = (fn == MOE_SOFTMAX) ? expf(hj - mx) / sum : 1.f / (1.f + expf(-hj));
+        if (prow) prow[j] = p;
+        const float key = rank_bias ? __fadd_rn(p, rank_bias[j]) : (fn == MOE_SOFTMAX ? hj : p);
+        // insert into the best-first list of length k (ties: the lower index ranks first)
+        bool placed = false;
+#pragma unroll
+        for (int t = KTHREAD - 1; t >= 0; --t) {
+            if (t < k && !placed) {
+                const int u = t > 0 ? t - 1 : 0;
+                if (t > 0 && ranks_before(key, j, kk[u], ki[u])) {
+                    kk[t] = kk[u]; ki[t] = ki[u]; kp[t] = kp[u];
+                } else {
+                    if (ranks_before(key, j, kk[t], ki[t])) { kk[t] = key; ki[t] = j; kp[t] = p; }
+                    placed = true;
+                }
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int t = 0; t < KTHREAD; ++t) if (t < k) s += kp[t];
+#pragma unroll
+    for (int t = 0; t < KTHREAD; ++t) {
+        if (t < k) {
+            topk_idx[row * k + t] = ki[t];
+            topk_gate[row * k + t] = (fn == MOE_SOFTMAX && renorm) ? kp[t] / s : kp[t];
+        }
+    }
+}
+
 template <int NCH>
 __global__ void __launch_bounds__(rtc::kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
@@ -173,13 +224,21 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 #pragma unroll
             for (int j = 0; j < NP; ++j) rows[lane * (NP + 1) + j] = acc[j];
             __syncwarp();
-            for (int rr = 0; rr < 32; ++rr) {
-                const int64_t r = row0 + quad * 32 + rr;
-                if (r >= m) break;
-                float hv[NCH];
+            if (k <= KTHREAD) {
+                // one thread per token row: compact loops over the experts, top-k in registers
+                const int64_t r = row0 + quad * 32 + lane;
+                if (r < m)
+                    finish_row_thread(rows + lane * (NP + 1), r, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
+                                      topk_gate);
+            } else {
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int64_t r = row0 + quad * 32 + rr;
+                    if (r >= m) break;
+                    float hv[NCH];
 #pragma unroll
-                for (int q = 0; q < NCH; ++q) hv[q] = rows[rr * (NP + 1) + lane + 32 * q];
-                finish_row<NCH>(hv, r, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+                    for (int q = 0; q < NCH; ++q) hv[q] = rows[rr * (NP + 1) + lane + 32 * q];
+                    finish_row<NCH>(hv, r, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+                }
             }
         }
     }

@@ -8,21 +8,23 @@
 // whole batch; MoE travelogue 6 (kexue.fm/archives/11619), Demo code
 // (MaxVio/MinVio/AvgVio) and eq. (2) b <- b - gamma sign(F - 1/n).
 //
-// Two launches. `partial`: each CTA takes kRows consecutive rows of one
-// segment, sums the probabilities per expert in fp64 (column-parallel,
-// coalesced row reads, 8 loads in flight per thread, fixed order) and counts
-// the routed picks. `final`: one CTA; every thread folds the chunks of one
-// (segment, expert) pair in order, then one expert per thread folds the
-// segments for the whole batch, then warps reduce the loss terms in a fixed
-// tree order. No floating-point atomics anywhere, so the results are
-// bit-reproducible.
+// One launch. Each CTA (1024 threads) takes kRows consecutive rows of one
+// segment: thread (expert e, group g) sums its rows' probabilities in fp64
+// with 16 loads issued together, the groups are folded in order, and the
+// routed picks are counted. The CTA publishes its partial sums, fences, and
+// takes a ticket; the last CTA of a segment folds that segment's chunks in
+// chunk order (f, P and the loss of the segment), and the last segment to
+// finish folds the segments in order (the whole batch, the micro-batch mean
+// and global loss, the violations, the bias update). The fold order never
+// depends on which CTA finishes last, and there are no floating-point atomics,
+// so the results are bit-reproducible.
 #include "common.cuh"
 
 namespace moe {
 
 namespace stats {
-constexpr int kRows = 128;      // rows per partial CTA
-constexpr int kThreads = 256;
+constexpr int kRows = 512;      // rows per CTA
+constexpr int kThreads = 1024;
 }  // namespace stats
 
 struct StatsGeometry {
@@ -36,61 +38,35 @@ static StatsGeometry stats_geometry(int64_t m, int64_t seg_len) {
     return g;
 }
 
+struct StatsWs {
+    double *psum, *segps, *segaux;
+    int32_t *pcnt, *segcnt, *tickets;  // tickets: one per segment, then one for the batch
+};
+
+static size_t stats_layout(int64_t m, int32_t n, int64_t seg_len, StatsWs* w, char* base) {
+    StatsGeometry g = stats_geometry(m, seg_len);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char* p = base ? base + off : nullptr;
+        off += (bytes + 255) & ~(size_t)255;
+        return p;
+    };
+    char* p;
+    p = take(sizeof(double) * (size_t)n * g.nchunks);   if (w) w->psum = (double*)p;
+    p = take(sizeof(double) * (size_t)n * g.nseg);      if (w) w->segps = (double*)p;
+    p = take(sizeof(double) * (size_t)g.nseg);          if (w) w->segaux = (double*)p;
+    p = take(sizeof(int32_t) * (size_t)n * g.nchunks);  if (w) w->pcnt = (int32_t*)p;
+    p = take(sizeof(int32_t) * (size_t)n * g.nseg);     if (w) w->segcnt = (int32_t*)p;
+    p = take(sizeof(int32_t) * (size_t)(g.nseg + 1));   if (w) w->tickets = (int32_t*)p;
+    return off;
+}
+
 size_t stats_workspace_bytes(int64_t m, int32_t n, int64_t seg_len) {
     if (seg_len <= 0) return 0;
-    StatsGeometry g = stats_geometry(m, seg_len);
-    // psum [nchunks][n] f64, prod [nseg + 1][n] f64, segps [nseg][n] f64, pcnt [nchunks][n] i32, segcnt [nseg][n] i32
-    return sizeof(double) * (size_t)n * (size_t)(g.nchunks + 2 * g.nseg + 1) +
-           sizeof(int32_t) * (size_t)n * (size_t)(g.nchunks + g.nseg);
+    return stats_layout(m, n, seg_len, nullptr, nullptr);
 }
 
-__global__ void __launch_bounds__(stats::kThreads)
-stats_partial_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, int n, int k, int64_t seg_len,
-                     int64_t cps, double* __restrict__ psum, int32_t* __restrict__ pcnt) {
-    __shared__ int cnt[kMaxExperts];
-    __shared__ double part[stats::kThreads];
-    const int tid = threadIdx.x;
-    const int64_t chunk = blockIdx.x;
-    const int64_t seg = chunk / cps, c = chunk - seg * cps;
-    const int64_t r0 = seg * seg_len + c * stats::kRows;
-    const int64_t r1 = min(r0 + (int64_t)stats::kRows, (seg + 1) * seg_len);
-    for (int e = tid; e < n; e += stats::kThreads) cnt[e] = 0;
-    __syncthreads();
-    for (int64_t q = r0 * k + tid; q < r1 * k; q += stats::kThreads) {
-        const int e = idx[q];
-        if (e < 0 || e >= n) record_error(kErrExpertIndex);
-        else atomicAdd(&cnt[e], 1);
-    }
-    if (probs) {
-        const int npad = (n + 31) & ~31;
-        const int groups = stats::kThreads / npad > 0 ? stats::kThreads / npad : 1;
-        const int e = tid % npad, gid = tid / npad;
-        double s = 0.0;
-        if (gid < groups && e < n) {
-            for (int64_t r = r0 + gid; r < r1; r += 8 * (int64_t)groups) {
-                float v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int64_t rr = r + (int64_t)u * groups;
-                    v[u] = rr < r1 ? probs[rr * n + e] : 0.f;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) s += (double)v[u];
-            }
-        }
-        part[tid] = s;
-        __syncthreads();
-        if (tid < n) {
-            double t = 0.0;
-            for (int g = 0; g < groups; ++g) t += part[g * npad + tid];
-            psum[chunk * n + tid] = t;
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < n; e += stats::kThreads) pcnt[chunk * n + e] = cnt[e];
-}
-
-// Fixed-order block reduction of one double per thread (256 threads).
+// Fixed-order block reductions of one double per thread.
 __device__ __forceinline__ double block_sum_d(double v, double* sh) {
     const int tid = threadIdx.x;
     v = warp_sum_d(v);
@@ -98,23 +74,83 @@ __device__ __forceinline__ double block_sum_d(double v, double* sh) {
     if ((tid & 31) == 0) sh[tid >> 5] = v;
     __syncthreads();
     double t = 0.0;
-    for (int w = 0; w < stats::kThreads / 32; ++w) t += sh[w];
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh[w];
+    __syncthreads();
+    return t;
+}
+__device__ __forceinline__ double block_max_d(double v, double* sh) {
+    const int tid = threadIdx.x;
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if ((tid & 31) == 0) sh[tid >> 5] = v;
+    __syncthreads();
+    double t = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = fmax(t, sh[w]);
     __syncthreads();
     return t;
 }
 
 __global__ void __launch_bounds__(stats::kThreads)
-stats_final_kernel(const double* __restrict__ psum, const int32_t* __restrict__ pcnt, int has_probs, int64_t m, int n,
-                   int k, int64_t seg_len, int64_t nseg, int64_t cps, float alpha, float* __restrict__ f,
-                   float* __restrict__ P, float* __restrict__ aux, float* __restrict__ vio,
-                   float* __restrict__ bias, float gamma, double* __restrict__ prod, double* __restrict__ segps,
-                   int32_t* __restrict__ segcnt) {
+stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, int64_t m, int n, int k,
+             int64_t seg_len, int64_t cps, int64_t nseg, float alpha, float* __restrict__ f, float* __restrict__ P,
+             float* __restrict__ aux, float* __restrict__ vio, float* __restrict__ bias, float gamma, StatsWs w) {
+    __shared__ int cnt[kMaxExperts];
+    __shared__ double part[stats::kThreads];
     __shared__ double sh[stats::kThreads / 32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // phase A: one (segment, expert) pair per thread folds its chunks in order, 8 loads in flight
-    for (int64_t pr = tid; pr < nseg * n; pr += stats::kThreads) {
-        const int64_t s = pr / n;
-        const int e = (int)(pr - s * n);
+    __shared__ int s_last;
+    const int tid = threadIdx.x;
+    const int64_t chunk = blockIdx.x;
+    const int64_t seg = chunk / cps, c = chunk - seg * cps;
+    const int64_t r0 = seg * seg_len + c * stats::kRows;
+    const int64_t r1 = min(r0 + (int64_t)stats::kRows, (seg + 1) * seg_len);
+    const bool has_probs = probs != nullptr;
+
+    // ---- this chunk: counts and per-expert probability sums
+    for (int e = tid; e < n; e += stats::kThreads) cnt[e] = 0;
+    __syncthreads();
+    for (int64_t q = r0 * k + tid; q < r1 * k; q += stats::kThreads) {
+        const int e = idx[q];
+        if (e < 0 || e >= n) record_error(kErrExpertIndex);
+        else atomicAdd(&cnt[e], 1);
+    }
+    if (has_probs) {
+        const int npad = (n + 31) & ~31;
+        const int groups = stats::kThreads / npad;
+        const int e = tid % npad, gid = tid / npad;
+        double s = 0.0;
+        if (gid < groups && e < n) {
+            for (int64_t r = r0 + gid; r < r1; r += 16 * (int64_t)groups) {
+                float v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int64_t rr = r + (int64_t)u * groups;
+                    v[u] = rr < r1 ? probs[rr * n + e] : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) s += (double)v[u];
+            }
+        }
+        part[tid] = s;
+        __syncthreads();
+        if (tid < n) {
+            double t = 0.0;
+            for (int g = 0; g < groups; ++g) t += part[g * npad + tid];
+            w.psum[chunk * n + tid] = t;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < n; e += stats::kThreads) w.pcnt[chunk * n + e] = cnt[e];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&w.tickets[seg], 1) == (int)cps - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // ---- last CTA of the segment: fold its chunks in chunk order
+    double prod = 0.0;
+    if (tid < n) {
+        const int e = tid;
         int64_t cs = 0;
         double ps = 0.0;
         for (int64_t c0 = 0; c0 < cps; c0 += 8) {
@@ -122,37 +158,48 @@ stats_final_kernel(const double* __restrict__ psum, const int32_t* __restrict__ 
             double pv[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t c = c0 + u;
-                cv[u] = c < cps ? pcnt[(s * cps + c) * n + e] : 0;
-                pv[u] = (has_probs && c < cps) ? psum[(s * cps + c) * n + e] : 0.0;
+                const int64_t cc = c0 + u;
+                cv[u] = cc < cps ? w.pcnt[(seg * cps + cc) * n + e] : 0;
+                pv[u] = (has_probs && cc < cps) ? w.psum[(seg * cps + cc) * n + e] : 0.0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) { cs += cv[u]; ps += pv[u]; }
         }
-        segcnt[s * n + e] = (int32_t)cs;
+        w.segcnt[seg * n + e] = (int32_t)cs;
         const double fv = (double)cs / ((double)k * (double)seg_len);
-        f[s * n + e] = (float)fv;
+        f[seg * n + e] = (float)fv;
         if (has_probs) {
-            segps[s * n + e] = ps;
+            w.segps[seg * n + e] = ps;
             const double pv = ps / (double)seg_len;
-            P[s * n + e] = (float)pv;
-            prod[s * n + e] = fv * pv;
+            P[seg * n + e] = (float)pv;
+            prod = fv * pv;
         }
     }
+    if (has_probs) {
+        const double a = (double)alpha * (double)n * block_sum_d(prod, sh);
+        if (tid == 0) { aux[seg] = (float)a; w.segaux[seg] = a; }
+    }
+    __threadfence();
     __syncthreads();
-    // phase B: the whole batch, one expert per thread, segments in order
-    const int e = tid;
+    if (tid == 0) s_last = atomicAdd(&w.tickets[nseg], 1) == (int)nseg - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // ---- last segment: the whole batch, in segment order
     int64_t tot = 0;
-    double pall = 0.0;
-    if (e < n) {
+    double pall = 0.0, gprod = 0.0;
+    const bool valid = tid < n;
+    if (valid) {
+        const int e = tid;
         for (int64_t s0 = 0; s0 < nseg; s0 += 8) {
             int32_t cv[8];
             double pv[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t s = s0 + u;
-                cv[u] = s < nseg ? segcnt[s * n + e] : 0;
-                pv[u] = (has_probs && s < nseg) ? segps[s * n + e] : 0.0;
+                const int64_t ss = s0 + u;
+                cv[u] = ss < nseg ? w.segcnt[ss * n + e] : 0;
+                pv[u] = (has_probs && ss < nseg) ? w.segps[ss * n + e] : 0.0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) { tot += cv[u]; pall += pv[u]; }
@@ -162,49 +209,31 @@ stats_final_kernel(const double* __restrict__ psum, const int32_t* __restrict__ 
         if (has_probs) {
             const double pg = pall / (double)m;
             P[nseg * n + e] = (float)pg;
-            prod[nseg * n + e] = fg * pg;
+            gprod = fg * pg;
         }
     }
-    __syncthreads();
     if (has_probs) {
-        // per-segment losses: warp w folds segments w, w+8, ... ; its running sum of losses in order
-        double wsum = 0.0;
-        for (int64_t s = warp; s < nseg + 1; s += stats::kThreads / 32) {
-            double t = 0.0;
-            for (int j = lane; j < n; j += 32) t += prod[s * n + j];
-            t = warp_sum_d(t);
-            const double a = (double)alpha * (double)n * t;
-            if (lane == 0) aux[s < nseg ? s : nseg + 1] = (float)a;
-            if (s < nseg) wsum += a;
-        }
-        if (lane != 0) wsum = 0.0;
-        const double micro = block_sum_d(wsum, sh);
-        if (tid == 0) aux[nseg] = (float)(micro / (double)nseg);
-    }
-    // MaxVio / MinVio / AvgVio of the pooled counts
-    const double F = (e < n) ? (double)tot / ((double)m * (double)k) * (double)n - 1.0 : 0.0;
-    if (vio) {
-        const double av = block_sum_d(e < n ? fabs(F) : 0.0, sh);
-        double mx = (e < n) ? F : -INFINITY, mn = (e < n) ? F : INFINITY;
-        for (int o = 16; o > 0; o >>= 1) {
-            mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        }
-        __shared__ double smx[stats::kThreads / 32], smn[stats::kThreads / 32];
-        if (lane == 0) { smx[warp] = mx; smn[warp] = mn; }
-        __syncthreads();
+        const double g = (double)alpha * (double)n * block_sum_d(gprod, sh);
         if (tid == 0) {
-            double a = -INFINITY, b = INFINITY;
-            for (int w = 0; w < stats::kThreads / 32; ++w) { a = fmax(a, smx[w]); b = fmin(b, smn[w]); }
-            vio[0] = (float)a; vio[1] = (float)b; vio[2] = (float)(av / (double)n);
+            double micro = 0.0;
+            for (int64_t s = 0; s < nseg; ++s) micro += w.segaux[s];
+            aux[nseg] = (float)(micro / (double)nseg);
+            aux[nseg + 1] = (float)g;
         }
     }
-    if (bias && e < n) {
+    const double F = valid ? (double)tot / ((double)m * (double)k) * (double)n - 1.0 : 0.0;
+    if (vio) {
+        const double av = block_sum_d(valid ? fabs(F) : 0.0, sh);
+        const double mx = block_max_d(valid ? F : -INFINITY, sh);
+        const double mn = -block_max_d(valid ? -F : -INFINITY, sh);
+        if (tid == 0) { vio[0] = (float)mx; vio[1] = (float)mn; vio[2] = (float)(av / (double)n); }
+    }
+    if (bias && valid) {
         const int64_t lhs = tot * (int64_t)n, rhs = m * (int64_t)k;
-        float b = bias[e];
+        float b = bias[tid];
         if (lhs > rhs) b = __fsub_rn(b, gamma);
         else if (lhs < rhs) b = __fadd_rn(b, gamma);
-        bias[e] = b;
+        bias[tid] = b;
     }
 }
 
@@ -212,17 +241,12 @@ cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m,
                          float alpha, float* f, float* P, float* aux, float* vio, float* bias, float gamma,
                          void* workspace, cudaStream_t stream) {
     StatsGeometry g = stats_geometry(m, seg_len);
-    double* psum = static_cast<double*>(workspace);
-    double* prod = psum + g.nchunks * n;
-    double* segps = prod + (g.nseg + 1) * n;
-    int32_t* pcnt = reinterpret_cast<int32_t*>(segps + g.nseg * n);
-    int32_t* segcnt = pcnt + g.nchunks * n;
-    if (g.nchunks > 0)
-        stats_partial_kernel<<<(unsigned)g.nchunks, stats::kThreads, 0, stream>>>(probs, topk_idx, n, k, seg_len,
-                                                                                  g.cps, psum, pcnt);
-    stats_final_kernel<<<1, stats::kThreads, 0, stream>>>(psum, pcnt, probs != nullptr, m, n, k, seg_len, g.nseg,
-                                                          g.cps, alpha, f, P, aux, vio, bias, gamma, prod, segps,
-                                                          segcnt);
+    StatsWs w;
+    stats_layout(m, n, seg_len, &w, static_cast<char*>(workspace));
+    cudaError_t e = cudaMemsetAsync(w.tickets, 0, sizeof(int32_t) * (size_t)(g.nseg + 1), stream);
+    if (e != cudaSuccess) return e;
+    stats_kernel<<<(unsigned)g.nchunks, stats::kThreads, 0, stream>>>(probs, topk_idx, m, n, k, seg_len, g.cps,
+                                                                      g.nseg, alpha, f, P, aux, vio, bias, gamma, w);
     return cudaGetLastError();
 }
 

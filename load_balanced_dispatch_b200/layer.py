@@ -139,12 +139,12 @@ class MoELayer:
     def launches_per_forward(self) -> int:
         """Kernel launches of one forward: router (split + tensor-core kernel for bf16 with n <= 128, else 1),
         capacity 3, dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
-        combine 1, statistics 2."""
+        combine 1, statistics 1."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
         router = 2 if (bf16 and s.n <= 128) else 1
         ffn = 1 if bf16 else 2
-        return router + 3 + 1 + ffn + 1 + 2
+        return router + 3 + 1 + ffn + 1 + 1
 
 
 def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:
