@@ -11,14 +11,17 @@
 //
 // Kernels:
 //   qb_row     one warp per token: v = s_i - beta in registers (n/32 values per
-//              lane), k + 1 rounds of a warp arg-max give the top-k set, the
-//              k-th and (k+1)-th values (alpha) and a tie flag; the set is
-//              written in ascending expert order and counted per expert.
+//              lane); the keys that can be among the k + 1 best are found from
+//              the lane maxima and gathered one per lane, then k + 1 rounds of a
+//              warp arg-max give the top-k set, the k-th and (k+1)-th values
+//              (alpha) and a tie flag; the set is written in ascending expert
+//              order and counted per expert.
 //   transpose  s [m, n] -> sT [n, m] once per call, so each column is contiguous.
-//   qb_col     one CTA per expert column: exact radix select (four 8-bit
-//              digit passes over order-preserving uint32 keys of u) for the
-//              C-th largest, then the (C+1)-th from the tie count or one max
-//              pass.
+//   qb_col     one CTA per expert column: one sweep keeps the keys of u near
+//              the previous beta_j in shared memory and counts those above;
+//              the C-th and (C+1)-th largest are then selected there (radix
+//              digits over order-preserving uint32 keys). When they are not
+//              inside that window, an exact radix select over the column.
 //   repair     successive shortest paths on the n-expert graph (exact finish
 //              when the QB iterate is not yet balanced): arc a -> b costs
 //              W[a][b] = min over tokens i holding a but not b of s_ia - s_ib
@@ -56,11 +59,102 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Top-(k+1) of one row held by a warp (lane owns j = lane + 32 q). Each round takes the
-// best untaken key: lane-local scan (lowest q on ties), then __reduce_max_sync over the
-// order-preserving keys and __reduce_min_sync over the candidate indices (lowest j among
-// equal keys) -- two warp instructions per round. R rows are interleaved per warp so the
-// rounds of independent rows overlap.
+// Top-(k+1) of one row held by a warp: lane owns j = lane + 32 q (q < NT); key = float_key(v),
+// 0 for j >= n (every real key is above 0). Output: `taken` (bit q: j = lane + 32 q is among the
+// k best), the k-th and (k+1)-th best values vk, vk1. Ranking: larger key first, equal keys by
+// lower j.
+//
+// Rounds: each of the k + 1 rounds takes the best untaken key: a lane-local scan (lowest q on
+// ties), __reduce_max_sync over keys, __reduce_min_sync over the candidate indices.
+template <int NT>
+__device__ __forceinline__ void row_topk_rounds(const uint32_t (&key)[NT], const float (&v)[NT], int n, int k,
+                                                uint32_t& taken, float& vk, float& vk1) {
+    const int lane = threadIdx.x & 31;
+    taken = 0;
+    vk = vk1 = 0.f;
+    for (int r = 0; r <= k; ++r) {
+        uint32_t lb = 0;
+        int lq = -1;
+        float lv = 0.f;
+#pragma unroll
+        for (int q = 0; q < NT; ++q)
+            if (!((taken >> q) & 1u) && key[q] > lb) { lb = key[q]; lq = q; lv = v[q]; }
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, lb);
+        const uint32_t cand = (lq >= 0 && lb == mx) ? (uint32_t)(lq * 32 + lane) : 0xffffffffu;
+        const uint32_t wj = __reduce_min_sync(0xffffffffu, cand);
+        const float wv = __shfl_sync(0xffffffffu, lv, (int)(wj & 31u));
+        if (r < k && wj < (uint32_t)n && (int)(wj & 31u) == lane) taken |= 1u << (wj >> 5);
+        if (r == k - 1) vk = wv;
+        if (r == k) vk1 = wv;
+    }
+}
+
+// Same result, usually far fewer instructions (k < 32, k < n): the (k+1)-th largest of the 32
+// lane maxima (with multiplicity) is a lower bound T of the row's (k+1)-th largest key, since k+1
+// distinct keys reach it. Every pick therefore has key >= T. When at most 32 keys reach T they
+// are gathered one per lane (through this warp's 32 shared slots) and the k + 1 rounds run over
+// single values. Returns false (nothing written) when more than 32 keys reach T.
+template <int NT>
+__device__ __forceinline__ bool row_topk_pruned(const uint32_t (&key)[NT], const float (&v)[NT], int n, int k,
+                                                uint32_t* sk, int* sj, float* sv, uint32_t& taken, float& vk,
+                                                float& vk1) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t full = 0xffffffffu;
+    uint32_t lm = 0;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) lm = max(lm, key[q]);
+    // T: walk the distinct lane maxima from the top until k + 1 of them are counted
+    uint32_t cur = lm, T = 1;
+    int need = k + 1;
+    for (;;) {
+        const uint32_t mx = __reduce_max_sync(full, cur);
+        if (mx == 0) break;  // fewer than k + 1 lane maxima: every key is a candidate
+        const int c = __popc(__ballot_sync(full, cur == mx));
+        if (c >= need) { T = mx; break; }
+        need -= c;
+        if (cur == mx) cur = 0;
+    }
+    int c = 0;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) c += key[q] >= T ? 1 : 0;
+    const int N = (int)__reduce_add_sync(full, (unsigned)c);
+    if (N > 32) return false;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(full, incl, o);
+        if (lane >= o) incl += y;
+    }
+    int pos = incl - c;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+        if (key[q] >= T) { sk[pos] = key[q]; sj[pos] = lane + 32 * q; sv[pos] = v[q]; ++pos; }
+    }
+    __syncwarp();
+    uint32_t ck = lane < N ? sk[lane] : 0u;
+    const uint32_t cj = lane < N ? (uint32_t)sj[lane] : 0xffffffffu;
+    const float cv = lane < N ? sv[lane] : 0.f;
+    __syncwarp();
+    taken = 0;
+    vk = vk1 = 0.f;
+    for (int r = 0; r <= k; ++r) {
+        const uint32_t mx = __reduce_max_sync(full, ck);
+        const uint32_t cand = (ck != 0 && ck == mx) ? cj : 0xffffffffu;
+        const uint32_t wj = __reduce_min_sync(full, cand);
+        const uint32_t src = __ballot_sync(full, cand == wj && cand != 0xffffffffu);
+        const float wv = __shfl_sync(full, cv, src ? __ffs(src) - 1 : 0);
+        if (r < k) {
+            if (wj < (uint32_t)n && (int)(wj & 31u) == lane) taken |= 1u << (wj >> 5);
+            if (cj == wj) ck = 0;
+        }
+        if (r == k - 1) vk = wv;
+        if (r == k) vk1 = wv;
+    }
+    return true;
+}
+
+// One warp per token, R tokens interleaved per warp so their loads overlap; each row takes the
+// pruned selection, or the plain rounds when it does not apply.
 template <int NT, int R>
 __global__ void __launch_bounds__(qb::kRowThreads)
 qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
@@ -70,21 +164,23 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
     __shared__ float sb[kMaxExperts];
     __shared__ int cnt[kMaxExperts];
     __shared__ int nties;
+    __shared__ uint32_t s_key[qb::kRowThreads];
+    __shared__ int s_j[qb::kRowThreads];
+    __shared__ float s_v[qb::kRowThreads];
     const int tid = threadIdx.x, lane = tid & 31;
+    const int wbase = tid & ~31;  // this warp's 32 shared slots
     for (int j = tid; j < n; j += blockDim.x) { sb[j] = beta[j]; cnt[j] = 0; }
     if (tid == 0) nties = 0;
     __syncthreads();
     const uint32_t lt = (1u << lane) - 1u;
+    const bool prune = k < 32 && k < n;
     const int64_t warps = (int64_t)gridDim.x * (qb::kRowThreads / 32);
     for (int64_t i0 = ((int64_t)blockIdx.x * (qb::kRowThreads / 32) + (tid >> 5)) * R; i0 < m; i0 += warps * R) {
         float v[R][NT];
-        uint32_t key[R][NT], taken[R];
-        float vk[R], vk1[R];
+        uint32_t key[R][NT];
 #pragma unroll
         for (int u = 0; u < R; ++u) {
             const int64_t i = i0 + u;
-            taken[u] = 0;
-            vk[u] = vk1[u] = 0.f;
 #pragma unroll
             for (int q = 0; q < NT; ++q) {
                 const int j = lane + 32 * q;
@@ -93,36 +189,23 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
                 key[u][q] = ok ? float_key(v[u][q]) : 0u;
             }
         }
-        for (int r = 0; r <= k; ++r) {
-#pragma unroll
-            for (int u = 0; u < R; ++u) {
-                uint32_t lb = 0;
-                int lq = -1;
-                float lv = 0.f;
-#pragma unroll
-                for (int q = 0; q < NT; ++q)
-                    if (!((taken[u] >> q) & 1u) && key[u][q] > lb) { lb = key[u][q]; lq = q; lv = v[u][q]; }
-                const uint32_t mx = __reduce_max_sync(0xffffffffu, lb);
-                const uint32_t cand = (lq >= 0 && lb == mx) ? (uint32_t)(lq * 32 + lane) : 0xffffffffu;
-                const uint32_t wj = __reduce_min_sync(0xffffffffu, cand);
-                const float wv = __shfl_sync(0xffffffffu, lv, (int)(wj & 31u));
-                if (r < k && wj < (uint32_t)n && (int)(wj & 31u) == lane) taken[u] |= 1u << (wj >> 5);
-                if (r == k - 1) vk[u] = wv;
-                if (r == k) vk1[u] = wv;
-            }
-        }
 #pragma unroll
         for (int u = 0; u < R; ++u) {
             const int64_t i = i0 + u;
             if (i >= m) break;
+            uint32_t taken;
+            float vk, vk1;
+            if (!(prune && row_topk_pruned<NT>(key[u], v[u], n, k, s_key + wbase, s_j + wbase, s_v + wbase, taken,
+                                               vk, vk1)))
+                row_topk_rounds<NT>(key[u], v[u], n, k, taken, vk, vk1);
             if (lane == 0) {
-                alpha[i] = qb_threshold(vk[u], vk1[u], rule);
-                if (vk[u] == vk1[u]) atomicAdd(&nties, 1);
+                alpha[i] = qb_threshold(vk, vk1, rule);
+                if (vk == vk1) atomicAdd(&nties, 1);
             }
             int pos = 0;
 #pragma unroll
             for (int q = 0; q < NT; ++q) {
-                const bool bit = (taken[u] >> q) & 1u;
+                const bool bit = (taken >> q) & 1u;
                 const uint32_t mask = __ballot_sync(0xffffffffu, bit);
                 if (bit) {
                     topk_idx[i * k + pos + __popc(mask & lt)] = lane + 32 * q;
@@ -214,19 +297,135 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, unsigned* red) {
     return r;
 }
 
+__device__ __forceinline__ unsigned block_sum_u32(unsigned v, unsigned* red) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    unsigned r = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += red[w];
+    __syncthreads();
+    return r;
+}
+
 namespace qb {
 constexpr int kCandCap = 16384;                         // candidate keys kept in shared memory
 constexpr size_t kColSmem = 4096 * 4 + kColThreads * 4 + kCandCap * 4;
+// key-space half-widths of the window around the previous beta_j
+constexpr uint32_t kWinDefault = 1u << 18, kWinMin = 1u << 12, kWinMax = 1u << 26;
 }  // namespace qb
 
+// Visit every key float_key(fp32(col[i] - alpha[i])) of a column, warp-uniformly (f gets
+// ok = false for padding lanes). 16-byte loads, two of each operand in flight per thread,
+// when m is a multiple of 4 (then every column of sT starts on a 16-byte boundary).
+template <typename F>
+__device__ __forceinline__ void for_each_col_key(const float* __restrict__ col, const float* __restrict__ alpha,
+                                                 int64_t m, F&& f) {
+    const int tid = threadIdx.x, T = blockDim.x;
+    if ((m & 3) == 0) {
+        const float4* c4 = reinterpret_cast<const float4*>(col);
+        const float4* a4 = reinterpret_cast<const float4*>(alpha);
+        const int64_t m4 = m >> 2;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t base = 0; base < m4; base += 2 * T) {
+            const int64_t v0 = base + tid, v1 = v0 + T;
+            const bool ok0 = v0 < m4, ok1 = v1 < m4;
+            const float4 c0 = ok0 ? c4[v0] : z, a0 = ok0 ? a4[v0] : z;
+            const float4 c1 = ok1 ? c4[v1] : z, a1 = ok1 ? a4[v1] : z;
+            f(ok0, float_key(__fsub_rn(c0.x, a0.x)));
+            f(ok0, float_key(__fsub_rn(c0.y, a0.y)));
+            f(ok0, float_key(__fsub_rn(c0.z, a0.z)));
+            f(ok0, float_key(__fsub_rn(c0.w, a0.w)));
+            f(ok1, float_key(__fsub_rn(c1.x, a1.x)));
+            f(ok1, float_key(__fsub_rn(c1.y, a1.y)));
+            f(ok1, float_key(__fsub_rn(c1.z, a1.z)));
+            f(ok1, float_key(__fsub_rn(c1.w, a1.w)));
+        }
+    } else {
+        for (int64_t base = 0; base < m; base += T) {
+            const int64_t i = base + tid;
+            const bool ok = i < m;
+            f(ok, ok ? float_key(__fsub_rn(col[i], alpha[i])) : 0u);
+        }
+    }
+}
+
+// Append `key` to the shared list for every lane with `in` (warp-uniform call; one shared
+// atomic per warp). Positions past kCandCap are counted but not stored.
+__device__ __forceinline__ void warp_append(unsigned* list, unsigned* count, bool in, uint32_t key) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (!bal) return;
+    const int lane = threadIdx.x & 31;
+    unsigned wbase = 0;
+    if (lane == 0) wbase = atomicAdd(count, (unsigned)__popc(bal));
+    wbase = __shfl_sync(0xffffffffu, wbase, 0);
+    const unsigned pos = wbase + __popc(bal & ((1u << lane) - 1u));
+    if (in && pos < (unsigned)qb::kCandCap) list[pos] = key;
+}
+
+// The want-th largest key (1-based, want <= ncand) of the shared list: three digit passes
+// (bits 31..20, 19..8, 7..0). Also gives its multiplicity and the number of list keys above it.
+__device__ void select_in_list(const unsigned* list, unsigned ncand, int64_t want, unsigned* hist, unsigned* scan,
+                               uint32_t* key_out, unsigned* mult_out, int64_t* greater_out) {
+    const int tid = threadIdx.x, T = blockDim.x;
+    int s1, s2, s3;
+    int64_t w1, w2, w3;
+    unsigned c1, c2, c3;
+    for (int b = tid; b < 4096; b += T) hist[b] = 0;
+    __syncthreads();
+    for (unsigned base = 0; base < ncand; base += T) {
+        const unsigned c = base + tid;
+        const bool ok = c < ncand;
+        warp_hist_add(hist, ok, (ok ? list[c] : 0u) >> 20);
+    }
+    __syncthreads();
+    block_select_bin(hist, 4096, want, scan, &s1, &w1, &c1);
+    for (int b = tid; b < 4096; b += T) hist[b] = 0;
+    __syncthreads();
+    for (unsigned base = 0; base < ncand; base += T) {
+        const unsigned c = base + tid;
+        const uint32_t key = c < ncand ? list[c] : 0u;
+        warp_hist_add(hist, c < ncand && (key >> 20) == (uint32_t)s1, (key >> 8) & 0xfffu);
+    }
+    __syncthreads();
+    block_select_bin(hist, 4096, w1, scan, &s2, &w2, &c2);
+    const uint32_t pre = ((uint32_t)s1 << 20) | ((uint32_t)s2 << 8);
+    for (int b = tid; b < 256; b += T) hist[b] = 0;
+    __syncthreads();
+    for (unsigned base = 0; base < ncand; base += T) {
+        const unsigned c = base + tid;
+        const uint32_t key = c < ncand ? list[c] : 0u;
+        warp_hist_add(hist, c < ncand && (key & 0xffffff00u) == pre, key & 0xffu);
+    }
+    __syncthreads();
+    block_select_bin(hist, 256, w2, scan, &s3, &w3, &c3);
+    *key_out = pre | (uint32_t)s3;
+    *mult_out = c3;
+    *greater_out = want - w3;
+}
+
+// Largest list key strictly below `bound` (0 if none), block-wide.
+__device__ __forceinline__ uint32_t list_max_below(const unsigned* list, unsigned ncand, uint32_t bound,
+                                                   unsigned* scan) {
+    uint32_t best = 0;
+    for (unsigned c = threadIdx.x; c < ncand; c += blockDim.x) {
+        const uint32_t key = list[c];
+        if (key < bound && key > best) best = key;
+    }
+    return block_max_u32(best, scan);
+}
+
 // beta_j = threshold between the C-th and (C+1)-th largest key of column j of u = fp32(s - alpha).
-// Pass 1 (global): histogram of the top 12 key bits. Pass 2 (global): keep the keys of the selected
-// bin in shared memory and the largest key below it. Then digits 19..8 and 7..0 over the kept keys.
-// If the bin holds more keys than fit, the two remaining digits stream from global memory instead.
+// Window pass: one sweep counts the keys above a window around the previous beta_j and keeps
+// the keys inside it in shared memory; when the C-th largest falls inside (the usual case once
+// the iteration settles) both order statistics come from the kept keys. Otherwise the full
+// radix path: a 12-bit digit histogram sweep, a sweep keeping the selected bin's keys (the
+// largest key below the bin is tracked), then the low digits over the kept keys (streamed from
+// global memory if the bin overflows the list). Both paths return the same two keys.
 __global__ void __launch_bounds__(qb::kColThreads)
 qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const float* __restrict__ alpha, int rule,
               float* __restrict__ beta, const int32_t* __restrict__ counts, int32_t* __restrict__ counts_next,
-              int32_t* __restrict__ status, int iter, int check) {
+              int32_t* __restrict__ status, int iter, int check, uint32_t* __restrict__ win) {
     if (check) {
         // stop once the previous row pass is balanced; otherwise CTA 0 prepares the next row pass
         if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
@@ -253,108 +452,115 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
     unsigned* scan = hist + 4096;              // blockDim
     unsigned* cand = scan + qb::kColThreads;   // kCandCap
     __shared__ unsigned s_ncand;
-    const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31;
+    const int tid = threadIdx.x, T = blockDim.x;
     const int j = blockIdx.x;
     const float* col = sT + (int64_t)j * m;
-    auto key_at = [&](int64_t i) { return float_key(__fsub_rn(col[i], alpha[i])); };
 
-    for (int b = tid; b < 4096; b += T) hist[b] = 0;
+    // ---- window pass around the previous beta_j (only this CTA reads or writes beta[j])
+    const uint32_t pk = float_key(beta[j]);
+    const uint32_t w = win[j] ? win[j] : qb::kWinDefault;
+    const uint32_t lo = pk > w ? pk - w : 0u, hi = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
     if (tid == 0) s_ncand = 0;
     __syncthreads();
-    for (int64_t base = 0; base < m; base += T) {
-        const int64_t i = base + tid;
-        const bool ok = i < m;
-        const uint32_t key = ok ? key_at(i) : 0u;
-        warp_hist_add(hist, ok, key >> 20);
-    }
-    __syncthreads();
-    int sel1;
-    int64_t want1;
-    unsigned cnt1;
-    block_select_bin(hist, 4096, C, scan, &sel1, &want1, &cnt1);
-
+    unsigned above = 0;
     uint32_t below = 0;
-    for (int64_t base = 0; base < m; base += T) {
-        const int64_t i = base + tid;
-        const bool ok = i < m;
-        const uint32_t key = ok ? key_at(i) : 0u;
-        const uint32_t d = key >> 20;
-        if (ok && d < (uint32_t)sel1 && key > below) below = key;
-        const bool in = ok && d == (uint32_t)sel1;
-        const uint32_t bal = __ballot_sync(0xffffffffu, in);
-        unsigned wbase = 0;
-        if (lane == 0 && bal) wbase = atomicAdd(&s_ncand, (unsigned)__popc(bal));
-        wbase = __shfl_sync(0xffffffffu, wbase, 0);
-        const unsigned pos = wbase + __popc(bal & ((1u << lane) - 1u));
-        if (in && pos < (unsigned)qb::kCandCap) cand[pos] = key;
-    }
+    for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+        above += (ok && key > hi) ? 1u : 0u;
+        if (ok && key < lo && key > below) below = key;
+        warp_append(cand, &s_ncand, ok && key >= lo && key <= hi, key);
+    });
+    above = block_sum_u32(above, scan);
     below = block_max_u32(below, scan);
-    const unsigned ncand = s_ncand;
-    const bool kept = ncand <= (unsigned)qb::kCandCap;
+    unsigned ncand = s_ncand;
+    const bool hit = ncand <= (unsigned)qb::kCandCap && (int64_t)above < C && (int64_t)above + ncand >= C;
 
-    // digits 19..8, then 7..0, within the selected top bin
-    int sel2, sel3;
-    int64_t want2, want3;
-    unsigned cnt2, cnt3;
-    for (int b = tid; b < 4096; b += T) hist[b] = 0;
-    __syncthreads();
-    if (kept) {
-        for (unsigned base = 0; base < ncand; base += T) {
-            const unsigned c = base + tid;
-            const bool ok = c < ncand;
-            const uint32_t key = ok ? cand[c] : 0u;
-            warp_hist_add(hist, ok, (key >> 8) & 0xfffu);
+    uint32_t akey, bkey;
+    if (hit) {
+        unsigned mult;
+        int64_t greater;
+        select_in_list(cand, ncand, C - (int64_t)above, hist, scan, &akey, &mult, &greater);
+        greater += above;
+        if (greater + (int64_t)mult >= C + 1) {
+            bkey = akey;
+        } else {
+            const uint32_t best = list_max_below(cand, ncand, akey, scan);
+            bkey = best ? best : below;
         }
     } else {
-        for (int64_t base = 0; base < m; base += T) {
-            const int64_t i = base + tid;
-            const uint32_t key = i < m ? key_at(i) : 0u;
-            warp_hist_add(hist, i < m && (key >> 20) == (uint32_t)sel1, (key >> 8) & 0xfffu);
-        }
-    }
-    __syncthreads();
-    block_select_bin(hist, 4096, want1, scan, &sel2, &want2, &cnt2);
-    const uint32_t pre2 = ((uint32_t)sel1 << 20) | ((uint32_t)sel2 << 8);
-    for (int b = tid; b < 256; b += T) hist[b] = 0;
-    __syncthreads();
-    if (kept) {
-        for (unsigned base = 0; base < ncand; base += T) {
-            const unsigned c = base + tid;
-            const uint32_t key = c < ncand ? cand[c] : 0u;
-            warp_hist_add(hist, c < ncand && (key & 0xffffff00u) == pre2, key & 0xffu);
-        }
-    } else {
-        for (int64_t base = 0; base < m; base += T) {
-            const int64_t i = base + tid;
-            const uint32_t key = i < m ? key_at(i) : 0u;
-            warp_hist_add(hist, i < m && (key & 0xffffff00u) == pre2, key & 0xffu);
-        }
-    }
-    __syncthreads();
-    block_select_bin(hist, 256, want2, scan, &sel3, &want3, &cnt3);
-    const uint32_t akey = pre2 | (uint32_t)sel3;
-    const int64_t greater = C - want3;
-    uint32_t bkey;
-    if (greater + (int64_t)cnt3 >= C + 1) {
-        bkey = akey;
-    } else {
-        // the (C+1)-th largest is the largest key below akey: inside the top bin, else below it
-        uint32_t best = 0;
-        if (kept) {
-            for (unsigned c = tid; c < ncand; c += T) {
-                const uint32_t key = cand[c];
-                if (key < akey && key > best) best = key;
+        // ---- full radix path
+        for (int b = tid; b < 4096; b += T) hist[b] = 0;
+        __syncthreads();
+        for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) { warp_hist_add(hist, ok, key >> 20); });
+        __syncthreads();
+        int sel1;
+        int64_t want1;
+        unsigned cnt1;
+        block_select_bin(hist, 4096, C, scan, &sel1, &want1, &cnt1);
+        if (tid == 0) s_ncand = 0;
+        __syncthreads();
+        below = 0;
+        for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+            const uint32_t d = key >> 20;
+            if (ok && d < (uint32_t)sel1 && key > below) below = key;
+            warp_append(cand, &s_ncand, ok && d == (uint32_t)sel1, key);
+        });
+        below = block_max_u32(below, scan);
+        ncand = s_ncand;
+        if (ncand <= (unsigned)qb::kCandCap) {
+            unsigned mult;
+            int64_t greater;
+            select_in_list(cand, ncand, want1, hist, scan, &akey, &mult, &greater);
+            greater += C - want1;
+            if (greater + (int64_t)mult >= C + 1) {
+                bkey = akey;
+            } else {
+                const uint32_t best = list_max_below(cand, ncand, akey, scan);
+                bkey = best ? best : below;
             }
         } else {
-            for (int64_t i = tid; i < m; i += T) {
-                const uint32_t key = key_at(i);
-                if ((key >> 20) == (uint32_t)sel1 && key < akey && key > best) best = key;
+            // the bin overflows the list: its low digits stream from global memory
+            int sel2, sel3;
+            int64_t want2, want3;
+            unsigned cnt2, cnt3;
+            for (int b = tid; b < 4096; b += T) hist[b] = 0;
+            __syncthreads();
+            for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+                warp_hist_add(hist, ok && (key >> 20) == (uint32_t)sel1, (key >> 8) & 0xfffu);
+            });
+            __syncthreads();
+            block_select_bin(hist, 4096, want1, scan, &sel2, &want2, &cnt2);
+            const uint32_t pre2 = ((uint32_t)sel1 << 20) | ((uint32_t)sel2 << 8);
+            for (int b = tid; b < 256; b += T) hist[b] = 0;
+            __syncthreads();
+            for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+                warp_hist_add(hist, ok && (key & 0xffffff00u) == pre2, key & 0xffu);
+            });
+            __syncthreads();
+            block_select_bin(hist, 256, want2, scan, &sel3, &want3, &cnt3);
+            akey = pre2 | (uint32_t)sel3;
+            const int64_t greater = C - want3;
+            if (greater + (int64_t)cnt3 >= C + 1) {
+                bkey = akey;
+            } else {
+                uint32_t best = 0;
+                for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+                    if (ok && (key >> 20) == (uint32_t)sel1 && key < akey && key > best) best = key;
+                });
+                best = block_max_u32(best, scan);
+                bkey = best ? best : below;
             }
         }
-        best = block_max_u32(best, scan);
-        bkey = best ? best : below;
     }
-    if (tid == 0) beta[j] = qb_threshold(key_float(akey), key_float(bkey), rule);
+    if (tid == 0) {
+        const float bnew = qb_threshold(key_float(akey), key_float(bkey), rule);
+        beta[j] = bnew;
+        // next window: centred on the new beta, as wide as this move plus the gap it splits
+        const uint32_t nk = float_key(bnew);
+        const uint64_t dist = nk > pk ? (uint64_t)(nk - pk) : (uint64_t)(pk - nk);
+        uint64_t wn = dist + (uint64_t)(akey - bkey) + qb::kWinMin;
+        if (wn > qb::kWinMax) wn = qb::kWinMax;
+        win[j] = (uint32_t)wn;
+    }
 }
 
 namespace qb {
@@ -446,11 +652,10 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
 #pragma unroll
             for (int u = 0; u < B; ++u) {
                 if (id[u] < 0) continue;  // warp-uniform
-                uint32_t in = 0;  // bit q: column lane + 32 q belongs to the member's set
+                uint32_t in = 0;  // bit q: column lane + 32 q belongs to the member's set (set by its owner lane)
                 for (int r = 0; r < k; ++r) {
                     const int e = k <= 32 ? __shfl_sync(0xffffffffu, ex[u], r & 31) : topk_idx[(int64_t)id[u] * k + r];
-#pragma unroll
-                    for (int q = 0; q < NT; ++q) in |= (e == lane + 32 * q) ? (1u << q) : 0u;
+                    if ((e & 31) == lane) in |= 1u << (e >> 5);
                 }
 #pragma unroll
                 for (int q = 0; q < NT; ++q) {
@@ -478,6 +683,32 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
         W[(int64_t)a * n + b] = bb;
         A[(int64_t)a * n + b] = bb == INFINITY ? -1 : aa;
     }
+}
+
+// Compact the indices a < n with flag[a] != 0, in increasing order, into out[] and *count
+// (block-wide; threads 0..255 each own one flag, a ballot per warp and a prefix over the warps).
+// Ends with a barrier, so out and *count are visible to every thread.
+__device__ __forceinline__ void compact_flags(const unsigned char* flag, int n, int32_t* out, int32_t* count,
+                                              int* wcount) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool f = tid < n && flag[tid];
+    uint32_t bal = 0;
+    if (tid < kMaxExperts) {
+        bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) wcount[warp] = __popc(bal);
+    }
+    __syncthreads();
+    if (tid < kMaxExperts) {
+        int off = 0;
+        for (int w = 0; w < warp; ++w) off += wcount[w];
+        if (f) out[off + __popc(bal & ((1u << lane) - 1u))] = tid;
+        if (tid == kMaxExperts - 1) {
+            int tot = 0;
+            for (int w = 0; w < kMaxExperts / 32; ++w) tot += wcount[w];
+            *count = tot;
+        }
+    }
+    __syncthreads();
 }
 
 // One augmentation (one unit of excess): Jacobi Bellman-Ford rounds from the over-full experts,
@@ -513,17 +744,12 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     // can improve another one, so each round reads just their rows of W (same fixpoint as full rounds)
     __shared__ int front[kMaxExperts], nfront;
     __shared__ unsigned char chg[kMaxExperts];
+    __shared__ int wcount[kMaxExperts / 32];
     if (tid < kMaxExperts) chg[tid] = (tid < n && dist[tid] == 0.0) ? 1 : 0;
     __syncthreads();
     bool settled = false;
     for (int round = 0; round <= n; ++round) {
-        if (tid == 0) {
-            int c = 0;
-            for (int a = 0; a < n; ++a)
-                if (chg[a]) front[c++] = a;
-            nfront = c;
-        }
-        __syncthreads();
+        compact_flags(chg, n, front, &nfront, wcount);
         const int nf = nfront;
         if (nf == 0) { settled = true; break; }
         double bestd = INFINITY;
@@ -568,13 +794,29 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         if (tid == 0) { status[qb::kStError] = 1; record_error(kErrRepair); *nrows = 0; }
         return;
     }
-    // predecessor: lowest a with dist[a] + W[a][b] == dist[b] (4 threads per column, a quarter each)
-    const int qa = (n + 3) / 4, a0 = part * qa, a1 = min(n, a0 + qa);
+    // predecessor: lowest a with dist[a] + W[a][b] == dist[b], over the reachable experts only
+    // (4 threads per column take every 4th of them, 8 loads in flight; the minimum over the four)
+    if (tid < kMaxExperts) chg[tid] = (tid < n && dist[tid] != INFINITY) ? 1 : 0;
+    __syncthreads();
+    compact_flags(chg, n, front, &nfront, wcount);
+    const int nr = nfront;
     int pa = 0x7fffffff;
     if (b < n && dist[b] != INFINITY) {
-        for (int a = a0; a < a1; ++a) {
-            const double w = W[(int64_t)a * n + b];
-            if (a != b && dist[a] != INFINITY && w != INFINITY && dist[a] + w == dist[b]) { pa = a; break; }
+        const double db = dist[b];
+        for (int f0 = part; f0 < nr; f0 += 4 * 8) {
+            double w8[8];
+            int a8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int fi = f0 + 4 * u;
+                a8[u] = fi < nr ? front[fi] : -1;
+                w8[u] = a8[u] >= 0 ? W[(int64_t)a8[u] * n + b] : INFINITY;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int aa = a8[u];
+                if (aa >= 0 && aa != b && w8[u] != INFINITY && dist[aa] + w8[u] == db && aa < pa) pa = aa;
+            }
         }
     }
     part_p[part][b] = pa;
@@ -626,12 +868,15 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
             counts[node] -= 1;
             counts[t] += 1;
             status[qb::kStAugments] += 1;
-            int c = 0;
-            for (int e = 0; e < n; ++e)
-                if ((touched[e >> 5] >> (e & 31)) & 1u) rows[c++] = e;
-            *nrows = c;
         }
+        any_over = ok;
     }
+    __syncthreads();
+    if (!any_over) return;
+    // the rows of W this move invalidated, in expert order, for the next arc pass
+    if (tid < kMaxExperts) chg[tid] = (tid < n && ((touched[tid >> 5] >> (tid & 31)) & 1u)) ? 1 : 0;
+    __syncthreads();
+    compact_flags(chg, n, rows, nrows, wcount);
 }
 
 __global__ void qb_all_rows_kernel(int n, int32_t* __restrict__ rows, int32_t* __restrict__ nrows) {
@@ -660,6 +905,7 @@ struct QBWorkspace {
     int32_t* rows;
     int32_t* nrows;
     uint32_t* mem;   // [n][ceil(m / 32)] membership bitmap
+    uint32_t* win;   // [n] window half-widths of the column pass (0: default)
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -678,6 +924,7 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     p = take(sizeof(int32_t) * (size_t)n);              if (w) w->rows = (int32_t*)p;
     p = take(sizeof(int32_t));                          if (w) w->nrows = (int32_t*)p;
     p = take(sizeof(uint32_t) * (size_t)n * (size_t)((m + 31) / 32)); if (w) w->mem = (uint32_t*)p;
+    p = take(sizeof(uint32_t) * (size_t)n);             if (w) w->win = (uint32_t*)p;
     return off;
 }
 
@@ -740,6 +987,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
     }
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto cuda_fail;
     if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
+    if ((ce = cudaMemsetAsync(w.win, 0, sizeof(uint32_t) * n, stream)) != cudaSuccess) goto cuda_fail;
     {
         dim3 tb(32, 8), tg((unsigned)((m + 31) / 32), (unsigned)((n + 31) / 32));
         transpose_kernel<<<tg, tb, 0, stream>>>(s, m, n, w.sT);
@@ -747,7 +995,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
     if (mode == MOE_QB_STEP) {
         launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, stream);
         qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(w.sT, m, n, C, w.alpha, rule, beta, w.counts,
-                                                                    w.counts + n, w.status, 0, 0);
+                                                                    w.counts + n, w.status, 0, 0, w.win);
         qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
         if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
         return MOE_OK;
@@ -763,7 +1011,8 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
                            u % 2 ? qb::kStTies1 : qb::kStTies0, 1, stream);
                 if (u < max_iters)
                     qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(
-                        w.sT, m, n, C, w.alpha, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, w.status, u, 1);
+                        w.sT, m, n, C, w.alpha, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, w.status, u, 1,
+                        w.win);
             }
             if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
             if ((ce = cudaMemcpyAsync(hstatus, w.status, sizeof(hstatus), cudaMemcpyDeviceToHost, stream)) !=

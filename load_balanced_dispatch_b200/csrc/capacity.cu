@@ -6,13 +6,14 @@
 // j-th assignment (in token order) to expert e gets slot j and is kept iff
 // j < capacity; overflow rides the residual path.
 //
-// Three launches over chunks of kChunk tokens (a chunk never straddles a
+// Two launches over chunks of kChunk tokens (a chunk never straddles a
 // segment):
-//   count  -- per-chunk expert histogram (shared-memory integer atomics);
-//   scan   -- one CTA, thread e walks the chunks of every segment in order:
-//             chunk prefix within its segment, routed/kept counts, the
-//             expert offsets (block exclusive scan over e) and each
-//             (segment, expert) base row;
+//   count+scan -- per-chunk expert histogram (shared-memory integer atomics);
+//             the last CTA to finish (ticket after a fence) runs the scan:
+//             thread e walks the chunks of every segment in order: chunk
+//             prefix within its segment, routed/kept counts, the expert
+//             offsets (block exclusive scan over e) and each (segment,
+//             expert) base row;
 //   assign -- per chunk, a stable in-order rank for every assignment
 //             (warp __match_any_sync groups + per-warp running counters in
 //             shared memory, warps owning consecutive sub-ranges), then
@@ -40,11 +41,12 @@ static CapGeometry cap_geometry(int64_t m, int64_t seg_len) {
     return g;
 }
 
+// Workspace: hist [nchunks][n], prefix [nchunks][n], seg_base [nseg][n], then one ticket word.
 size_t capacity_workspace_bytes(int64_t m, int32_t k, int32_t n, int64_t seg_len) {
     (void)k;
     if (seg_len <= 0) return 0;
     CapGeometry g = cap_geometry(m, seg_len);
-    return sizeof(int32_t) * (size_t)n * (size_t)(2 * g.nchunks + g.nseg);
+    return sizeof(int32_t) * ((size_t)n * (size_t)(2 * g.nchunks + g.nseg) + 1);
 }
 
 __device__ __forceinline__ void chunk_range(int64_t chunk, int64_t cps, int64_t seg_len, int64_t& seg, int64_t& t0,
@@ -53,24 +55,6 @@ __device__ __forceinline__ void chunk_range(int64_t chunk, int64_t cps, int64_t 
     const int64_t c = chunk - seg * cps;
     t0 = seg * seg_len + c * cap::kChunk;
     t1 = min(t0 + (int64_t)cap::kChunk, (seg + 1) * seg_len);
-}
-
-__global__ void __launch_bounds__(cap::kThreads)
-cap_count_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg_len, int64_t cps,
-                 int32_t* __restrict__ hist) {
-    __shared__ int cnt[kMaxExperts];
-    for (int e = threadIdx.x; e < n; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
-    int64_t seg, t0, t1;
-    chunk_range(blockIdx.x, cps, seg_len, seg, t0, t1);
-    const int64_t a0 = t0 * k, a1 = t1 * k;
-    for (int64_t q = a0 + threadIdx.x; q < a1; q += blockDim.x) {
-        const int e = idx[q];
-        if (e < 0 || e >= n) record_error(kErrExpertIndex);
-        else atomicAdd(&cnt[e], 1);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < n; e += blockDim.x) hist[(int64_t)blockIdx.x * n + e] = cnt[e];
 }
 
 // Block-wide exclusive scan of one value per thread (blockDim.x == 256), in a fixed order.
@@ -88,10 +72,12 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* sh, 
     return sh[tid] - v;
 }
 
-__global__ void __launch_bounds__(cap::kThreads)
-cap_scan_kernel(const int32_t* __restrict__ hist, int n, int64_t nseg, int64_t cps, int32_t capacity,
-                int32_t* __restrict__ prefix, int32_t* __restrict__ seg_base, int32_t* __restrict__ expert_offsets,
-                int32_t* __restrict__ routed_count, int32_t* __restrict__ kept_count) {
+// The scan, run by the last CTA of the count phase: thread e walks the chunks of every segment in
+// order. hist was written by other CTAs of this launch, so it is read through L2 (__ldcg).
+__device__ __forceinline__ void cap_scan_body(const int32_t* hist, int n, int64_t nseg, int64_t cps, int32_t capacity,
+                                              int32_t* __restrict__ prefix, int32_t* __restrict__ seg_base,
+                                              int32_t* __restrict__ expert_offsets, int32_t* __restrict__ routed_count,
+                                              int32_t* __restrict__ kept_count) {
     __shared__ int64_t sh[cap::kThreads];
     const int e = threadIdx.x;
     int64_t kept_total = 0;
@@ -101,7 +87,7 @@ cap_scan_kernel(const int32_t* __restrict__ hist, int n, int64_t nseg, int64_t c
             for (int64_t c0 = 0; c0 < cps; c0 += 8) {  // 8 loads in flight
                 int32_t h[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) h[u] = (c0 + u < cps) ? hist[(s * cps + c0 + u) * n + e] : 0;
+                for (int u = 0; u < 8; ++u) h[u] = (c0 + u < cps) ? __ldcg(hist + (s * cps + c0 + u) * n + e) : 0;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     if (c0 + u < cps) {
@@ -127,6 +113,36 @@ cap_scan_kernel(const int32_t* __restrict__ hist, int n, int64_t nseg, int64_t c
         }
     }
     if (e == 0) expert_offsets[n] = (int32_t)total;
+}
+
+// Per-chunk expert histogram (shared-memory integer atomics); the last CTA to finish (a ticket
+// taken after a fence) then runs the scan over all chunks.
+__global__ void __launch_bounds__(cap::kThreads)
+cap_count_scan_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg_len, int64_t cps, int64_t nchunks,
+                      int64_t nseg, int32_t capacity, int32_t* hist, int32_t* __restrict__ prefix,
+                      int32_t* __restrict__ seg_base, int32_t* __restrict__ expert_offsets,
+                      int32_t* __restrict__ routed_count, int32_t* __restrict__ kept_count, int32_t* ticket) {
+    __shared__ int cnt[kMaxExperts];
+    __shared__ int s_last;
+    for (int e = threadIdx.x; e < n; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    int64_t seg, t0, t1;
+    chunk_range(blockIdx.x, cps, seg_len, seg, t0, t1);
+    const int64_t a0 = t0 * k, a1 = t1 * k;
+    for (int64_t q = a0 + threadIdx.x; q < a1; q += blockDim.x) {
+        const int e = idx[q];
+        if (e < 0 || e >= n) record_error(kErrExpertIndex);
+        else atomicAdd(&cnt[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x) hist[(int64_t)blockIdx.x * n + e] = cnt[e];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == (int)(nchunks - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    cap_scan_body(hist, n, nseg, cps, capacity, prefix, seg_base, expert_offsets, routed_count, kept_count);
 }
 
 __global__ void __launch_bounds__(cap::kThreads)
@@ -195,12 +211,21 @@ cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, in
     int32_t* hist = static_cast<int32_t*>(workspace);
     int32_t* prefix = hist + g.nchunks * n;
     int32_t* seg_base = prefix + g.nchunks * n;
-    if (g.nchunks > 0) {
-        cap_count_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(topk_idx, k, n, seg_len, g.cps, hist);
+    int32_t* ticket = seg_base + g.nseg * n;
+    if (g.nchunks == 0) {
+        // no tokens: empty layout, nothing to count
+        cudaError_t e = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (size_t)(n + 1), stream);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
-    cap_scan_kernel<<<1, cap::kThreads, 0, stream>>>(hist, n, g.nseg, g.cps, capacity, prefix, seg_base,
-                                                     expert_offsets, routed_count, kept_count);
-    if (g.nchunks > 0) {
+    {
+        cudaError_t e = cudaMemsetAsync(ticket, 0, sizeof(int32_t), stream);
+        if (e != cudaSuccess) return e;
+    }
+    cap_count_scan_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(
+        topk_idx, k, n, seg_len, g.cps, g.nchunks, g.nseg, capacity, hist, prefix, seg_base, expert_offsets,
+        routed_count, kept_count, ticket);
+    {
         cap_assign_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(
             topk_idx, k, n, seg_len, g.cps, capacity, prefix, seg_base, slot, dest_row, src_token);
     }

@@ -198,6 +198,42 @@ router_topk_kernel(const T* __restrict__ x, const float* __restrict__ w_r, const
     }
 }
 
+// Finish rows whose fp32 logits are already in memory: h [m, n]. `probs_out` may be h itself
+// (each warp loads its whole row into registers before writing any of it), so neither pointer
+// is declared restrict. One warp per row, grid-stride over rows.
+constexpr int kFinishThreads = 256;
+template <int NT>
+__global__ void __launch_bounds__(kFinishThreads)
+router_finish_kernel(const float* h, int64_t m, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
+                     float* probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kFinishThreads / 32);
+    for (int64_t row = (int64_t)blockIdx.x * (kFinishThreads / 32) + (threadIdx.x >> 5); row < m; row += warps) {
+        float hv[NT];
+#pragma unroll
+        for (int q = 0; q < NT; ++q) hv[q] = (lane + 32 * q < n) ? h[row * n + lane + 32 * q] : 0.f;
+        __syncwarp();
+        finish_row<NT>(hv, row, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    }
+}
+
+cudaError_t launch_router_finish(const float* h, int64_t m, int n, int k, int fn, int renorm, const float* rank_bias,
+                                 float* probs_out, int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    if (m == 0) return cudaSuccess;
+    int64_t blocks = (m + kFinishThreads / 32 - 1) / (kFinishThreads / 32);
+    const int64_t cap = (int64_t)kNumSMs * 8;
+    if (blocks > cap) blocks = cap;
+    if (n <= 32)
+        router_finish_kernel<1><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    else if (n <= 64)
+        router_finish_kernel<2><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    else if (n <= 128)
+        router_finish_kernel<4><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    else
+        router_finish_kernel<8><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    return cudaGetLastError();
+}
+
 template <typename T, int NT>
 static cudaError_t launch_router_t(const void* x, const float* w_r, const float* logits_in, int64_t m, int d, int n,
                                    int k, int fn, int renorm, const float* rank_bias, float* probs_out,

@@ -9,16 +9,19 @@
 // the tensor core accumulates in fp32: fp32-accurate logits at tensor-core speed.
 //
 //   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand)
-//   router_tc_kernel     one CTA per 128 tokens, 128 threads:
+//   router_tc_kernel     one CTA per 128 tokens and column tile of experts (64 wide when
+//                        the logits go to memory, all n otherwise), 192 threads:
 //     warp 0 lane 0   TMA: x tile 128x64 + the three 64-wide W parts per stage
-//     warp 1 lane 0   tcgen05.mma kind::f16 M=128 N=np (3 parts x 4 K-steps per stage)
+//     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = the tile width (3 parts x 4 K-steps per stage)
 //     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM
 //                     lane); each K block's product lands in a fresh TMEM accumulator
 //                     (two, ping-pong) and is added into fp32 registers with
 //                     round-to-nearest adds, which keeps the sum fp32-accurate;
-//                     then the warp parks its 32 rows in shared memory and finishes
-//                     them row by row (softmax or sigmoid, key, top-k, gates) with
-//                     the same routine as the FMA router.
+//                     then the warp parks its 32 rows in shared memory. With probs_out
+//                     the rows are stored there as fp32 logits (coalesced) and
+//                     router_finish_kernel (one warp per row over the whole GPU) turns
+//                     them into scores, keys, top-k and gates in place; without it the
+//                     drain threads finish their rows themselves (nothing to store).
 #include "tc_ptx.cuh"
 
 namespace moe {
@@ -138,6 +141,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     const int nkb = (d + BK - 1) / BK;
     const uint32_t tcols = router_tmem_cols(NP);
     const int64_t row0 = (int64_t)blockIdx.x * BM;
+    const int col0 = blockIdx.y * NP;  // first expert of this CTA's column tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
@@ -164,7 +168,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                 ptx::mbar_expect_tx(&sh->full[stage], (uint32_t)STAGE_BYTES);
                 ptx::tma_load_2d(st, &map_x, &sh->full[stage], kb * BK, (int)row0);
                 for (int part = 0; part < 3; ++part)
-                    ptx::tma_load_3d(st + A_BYTES + part * NP * 128, &map_w, &sh->full[stage], kb * BK, 0, part);
+                    ptx::tma_load_3d(st + A_BYTES + part * NP * 128, &map_w, &sh->full[stage], kb * BK, col0, part);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
         }
@@ -224,7 +228,19 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 #pragma unroll
             for (int j = 0; j < NP; ++j) rows[lane * (NP + 1) + j] = acc[j];
             __syncwarp();
-            if (k <= KTHREAD) {
+            if (probs_out) {
+                // logits out, coalesced (a warp stores one row's 128-byte runs per instruction);
+                // router_finish_kernel turns them into scores and picks in place
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int64_t r = row0 + quad * 32 + rr;
+                    if (r >= m) break;
+#pragma unroll
+                    for (int q = 0; q < NCH; ++q) {
+                        const int j = col0 + lane + 32 * q;
+                        if (j < n) probs_out[r * n + j] = rows[rr * (NP + 1) + lane + 32 * q];
+                    }
+                }
+            } else if (k <= KTHREAD) {
                 // one thread per token row: compact loops over the experts, top-k in registers
                 const int64_t r = row0 + quad * 32 + lane;
                 if (r < m)
@@ -268,8 +284,9 @@ static cudaError_t launch_router_tc_t(const CUtensorMap& mx, const CUtensorMap& 
         attr = true;
     }
     const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
-    router_tc_kernel<NCH><<<(unsigned)blocks, rtc::kThreads, smem, stream>>>(mx, mw, m, d, n, k, fn, renorm, rank_bias,
-                                                                             probs_out, topk_idx, topk_gate);
+    const unsigned ctiles = (unsigned)((router_np(n) + NCH * 32 - 1) / (NCH * 32));
+    router_tc_kernel<NCH><<<dim3((unsigned)blocks, ctiles), rtc::kThreads, smem, stream>>>(
+        mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
     return cudaGetLastError();
 }
 
@@ -286,16 +303,24 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, 
         dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
         router_split_kernel<<<tg, tb, 0, stream>>>(w_r, d, n, wsplit);
     }
+    // With probs_out the logits go to memory, so the experts split into 64-wide column tiles
+    // (twice the CTAs, half the W traffic and drain work each); without it each CTA keeps whole
+    // rows for the in-kernel finish.
     const int np = router_np(n);
+    const int tile = probs_out ? (np < 64 ? np : 64) : np;
     CUtensorMap mx, mw;
     if (!map_2d(&mx, x, (uint64_t)m, (uint64_t)d, rtc::BM)) return cudaErrorInvalidValue;
-    if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)np)) return cudaErrorInvalidValue;
-    switch (np / 32) {
-        case 1: return launch_router_tc_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
-        case 2: return launch_router_tc_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
-        case 3: return launch_router_tc_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
-        default: return launch_router_tc_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+    if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)tile)) return cudaErrorInvalidValue;
+    cudaError_t e;
+    switch (tile / 32) {
+        case 1: e = launch_router_tc_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
+        case 2: e = launch_router_tc_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
+        case 3: e = launch_router_tc_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
+        default: e = launch_router_tc_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
     }
+    if (e != cudaSuccess || !probs_out) return e;
+    // the tensor-core kernel left the fp32 logits in probs_out: finish them there, one warp per row
+    return launch_router_finish(probs_out, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
 }
 
 }  // namespace moe

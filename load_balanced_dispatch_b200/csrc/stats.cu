@@ -8,10 +8,10 @@
 // whole batch; MoE travelogue 6 (kexue.fm/archives/11619), Demo code
 // (MaxVio/MinVio/AvgVio) and eq. (2) b <- b - gamma sign(F - 1/n).
 //
-// One launch. Each CTA (1024 threads) takes kRows consecutive rows of one
-// segment: thread (expert e, group g) sums its rows' probabilities in fp64
-// with 16 loads issued together, the groups are folded in order, and the
-// routed picks are counted. The CTA publishes its partial sums, fences, and
+// One launch. Each CTA (256 threads) takes kRows consecutive rows of one
+// segment: thread (four experts, row group g) sums its rows' probabilities in
+// fp64 from 16-byte loads, eight in flight, the groups are folded in order,
+// and the routed picks are counted. The CTA publishes its partial sums, fences, and
 // takes a ticket; the last CTA of a segment folds that segment's chunks in
 // chunk order (f, P and the loss of the segment), and the last segment to
 // finish folds the segments in order (the whole batch, the micro-batch mean
@@ -23,8 +23,9 @@
 namespace moe {
 
 namespace stats {
-constexpr int kRows = 512;      // rows per CTA
-constexpr int kThreads = 1024;
+constexpr int kRows = 256;      // rows per CTA
+constexpr int kThreads = 256;
+constexpr int kBatch = 8;       // loads in flight per thread
 }  // namespace stats
 
 struct StatsGeometry {
@@ -90,12 +91,54 @@ __device__ __forceinline__ double block_max_d(double v, double* sh) {
     return t;
 }
 
-__global__ void __launch_bounds__(stats::kThreads)
+// Fold `cnt` [nblk][n] and `ps` [nblk][n] over the blocks in a fixed order, all threads taking part:
+// thread (e, p) sums blocks p, p + P, ... (P = threads / padded n), then thread e adds the P partial
+// sums in p order. Thread e < n gets the totals; barriers inside.
+// The blocks were written by other CTAs of this launch: read them through L2 (__ldcg), never the
+// read-only path.
+__device__ __forceinline__ void fold_blocks(const int32_t* cnt, const double* ps,
+                                            int64_t nblk, int n, bool has_ps, long long* pc, double* pp,
+                                            int64_t* cnt_out, double* ps_out) {
+    const int tid = threadIdx.x;
+    const int npad = (n + 31) & ~31;
+    const int P = stats::kThreads / npad;
+    const int e = tid % npad, p = tid / npad;
+    long long cs = 0;
+    double s = 0.0;
+    if (p < P && e < n) {
+        for (int64_t b0 = p; b0 < nblk; b0 += (int64_t)P * stats::kBatch) {
+            int32_t cv[stats::kBatch];
+            double pv[stats::kBatch];
+#pragma unroll
+            for (int u = 0; u < stats::kBatch; ++u) {
+                const int64_t b = b0 + (int64_t)u * P;
+                cv[u] = b < nblk ? __ldcg(cnt + b * n + e) : 0;
+                pv[u] = (has_ps && b < nblk) ? __ldcg(ps + b * n + e) : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < stats::kBatch; ++u) { cs += cv[u]; s += pv[u]; }
+        }
+    }
+    pc[tid] = cs;
+    pp[tid] = s;
+    __syncthreads();
+    if (tid < n) {
+        long long c = 0;
+        double t = 0.0;
+        for (int q = 0; q < P; ++q) { c += pc[q * npad + tid]; t += pp[q * npad + tid]; }
+        *cnt_out = c;
+        *ps_out = t;
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(stats::kThreads, 2)
 stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, int64_t m, int n, int k,
              int64_t seg_len, int64_t cps, int64_t nseg, float alpha, float* __restrict__ f, float* __restrict__ P,
              float* __restrict__ aux, float* __restrict__ vio, float* __restrict__ bias, float gamma, StatsWs w) {
     __shared__ int cnt[kMaxExperts];
-    __shared__ double part[stats::kThreads];
+    __shared__ double part[stats::kThreads * 4];
+    __shared__ long long pc[stats::kThreads];
     __shared__ double sh[stats::kThreads / 32];
     __shared__ int s_last;
     const int tid = threadIdx.x;
@@ -114,28 +157,58 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
         else atomicAdd(&cnt[e], 1);
     }
     if (has_probs) {
-        const int npad = (n + 31) & ~31;
-        const int groups = stats::kThreads / npad;
-        const int e = tid % npad, gid = tid / npad;
-        double s = 0.0;
-        if (gid < groups && e < n) {
-            for (int64_t r = r0 + gid; r < r1; r += 16 * (int64_t)groups) {
-                float v[16];
+        if ((n & 3) == 0) {
+            // 16-byte loads: thread (column quad c4, row group g); rows g, g + G, ... of the chunk
+            const int c4n = n >> 2, G = stats::kThreads / c4n;
+            const int c4 = tid % c4n, g = tid / c4n;
+            const float4* p4 = reinterpret_cast<const float4*>(probs);
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+            if (g < G) {
+                for (int64_t r = r0 + g; r < r1; r += (int64_t)G * stats::kBatch) {
+                    float4 v[stats::kBatch];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int64_t rr = r + (int64_t)u * groups;
-                    v[u] = rr < r1 ? probs[rr * n + e] : 0.f;
+                    for (int u = 0; u < stats::kBatch; ++u) {
+                        const int64_t rr = r + (int64_t)u * G;
+                        v[u] = rr < r1 ? p4[rr * c4n + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < stats::kBatch; ++u) {
+                        s0 += (double)v[u].x; s1 += (double)v[u].y; s2 += (double)v[u].z; s3 += (double)v[u].w;
+                    }
                 }
-#pragma unroll
-                for (int u = 0; u < 16; ++u) s += (double)v[u];
             }
-        }
-        part[tid] = s;
-        __syncthreads();
-        if (tid < n) {
-            double t = 0.0;
-            for (int g = 0; g < groups; ++g) t += part[g * npad + tid];
-            w.psum[chunk * n + tid] = t;
+            part[tid * 4 + 0] = s0; part[tid * 4 + 1] = s1; part[tid * 4 + 2] = s2; part[tid * 4 + 3] = s3;
+            __syncthreads();
+            if (tid < n) {
+                const int cq = tid >> 2, q = tid & 3;
+                double t = 0.0;
+                for (int gg = 0; gg < G; ++gg) t += part[(gg * c4n + cq) * 4 + q];
+                w.psum[chunk * n + tid] = t;
+            }
+        } else {
+            const int npad = (n + 31) & ~31;
+            const int G = stats::kThreads / npad;
+            const int e = tid % npad, g = tid / npad;
+            double s = 0.0;
+            if (g < G && e < n) {
+                for (int64_t r = r0 + g; r < r1; r += (int64_t)G * stats::kBatch) {
+                    float v[stats::kBatch];
+#pragma unroll
+                    for (int u = 0; u < stats::kBatch; ++u) {
+                        const int64_t rr = r + (int64_t)u * G;
+                        v[u] = rr < r1 ? probs[rr * n + e] : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < stats::kBatch; ++u) s += (double)v[u];
+                }
+            }
+            part[tid] = s;
+            __syncthreads();
+            if (tid < n) {
+                double t = 0.0;
+                for (int gg = 0; gg < G; ++gg) t += part[gg * npad + tid];
+                w.psum[chunk * n + tid] = t;
+            }
         }
     }
     __syncthreads();
@@ -147,24 +220,13 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
     if (!s_last) return;
     __threadfence();
 
-    // ---- last CTA of the segment: fold its chunks in chunk order
+    // ---- last CTA of the segment: fold its chunks
+    int64_t cs = 0;
+    double ps = 0.0;
+    fold_blocks(w.pcnt + seg * cps * n, w.psum + seg * cps * n, cps, n, has_probs, pc, part, &cs, &ps);
     double prod = 0.0;
     if (tid < n) {
         const int e = tid;
-        int64_t cs = 0;
-        double ps = 0.0;
-        for (int64_t c0 = 0; c0 < cps; c0 += 8) {
-            int32_t cv[8];
-            double pv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int64_t cc = c0 + u;
-                cv[u] = cc < cps ? w.pcnt[(seg * cps + cc) * n + e] : 0;
-                pv[u] = (has_probs && cc < cps) ? w.psum[(seg * cps + cc) * n + e] : 0.0;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) { cs += cv[u]; ps += pv[u]; }
-        }
         w.segcnt[seg * n + e] = (int32_t)cs;
         const double fv = (double)cs / ((double)k * (double)seg_len);
         f[seg * n + e] = (float)fv;
@@ -189,21 +251,10 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
     // ---- last segment: the whole batch, in segment order
     int64_t tot = 0;
     double pall = 0.0, gprod = 0.0;
+    fold_blocks(w.segcnt, w.segps, nseg, n, has_probs, pc, part, &tot, &pall);
     const bool valid = tid < n;
     if (valid) {
         const int e = tid;
-        for (int64_t s0 = 0; s0 < nseg; s0 += 8) {
-            int32_t cv[8];
-            double pv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int64_t ss = s0 + u;
-                cv[u] = ss < nseg ? w.segcnt[ss * n + e] : 0;
-                pv[u] = (has_probs && ss < nseg) ? w.segps[ss * n + e] : 0.0;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) { tot += cv[u]; pall += pv[u]; }
-        }
         const double fg = (double)tot / ((double)k * (double)m);
         f[nseg * n + e] = (float)fg;
         if (has_probs) {
@@ -216,7 +267,7 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
         const double g = (double)alpha * (double)n * block_sum_d(gprod, sh);
         if (tid == 0) {
             double micro = 0.0;
-            for (int64_t s = 0; s < nseg; ++s) micro += w.segaux[s];
+            for (int64_t s = 0; s < nseg; ++s) micro += __ldcg(w.segaux + s);
             aux[nseg] = (float)(micro / (double)nseg);
             aux[nseg + 1] = (float)g;
         }

@@ -2,8 +2,8 @@
 
 The runner only allocates device buffers once and calls the library's entry
 points in the order the layer defines (router -> [balance] -> capacity ->
-dispatch -> expert FFN -> combine -> statistics). All arithmetic happens in
-the library's kernels.
+dispatch -> expert FFN -> combine, and the statistics beside them once the
+router is done). All arithmetic happens in the library's kernels.
 """
 from __future__ import annotations
 
@@ -102,19 +102,34 @@ class MoELayer:
                               workspace=self.ws["stats"], stream=st)
 
     def forward(self, x: torch.Tensor, stream=None, events=None) -> torch.Tensor:
-        """One forward through the C ABI. `events`: optional 7 CUDA events recorded around the 6 stages."""
+        """One forward through the C ABI on `stream`. The statistics read only the router's outputs, so
+        they run on a side stream (forked after the router, joined at the end) beside capacity, dispatch,
+        FFN and combine. `events`: optional 7 CUDA events; then the 6 stages run one after another on
+        `stream` with the events recorded between them (per-stage timing)."""
         st = stream if stream is not None else torch.cuda.current_stream()
-        for i in range(len(self.STAGES)):
-            if events is not None:
-                events[i].record(st)
-            self._stage(i, x, st)
         if events is not None:
+            for i in range(len(self.STAGES)):
+                events[i].record(st)
+                self._stage(i, x, st)
             events[len(self.STAGES)].record(st)
+            return self.buf["y"]
+        if not hasattr(self, "_side"):
+            self._side = torch.cuda.Stream(device=self.device)
+            self._fork, self._join = torch.cuda.Event(), torch.cuda.Event()
+        self._stage(0, x, st)
+        self._fork.record(st)
+        self._side.wait_event(self._fork)
+        self._stage(5, x, self._side)
+        for i in range(1, 5):
+            self._stage(i, x, st)
+        self._join.record(self._side)
+        st.wait_event(self._join)
         return self.buf["y"]
 
     def capture(self, x: torch.Tensor) -> None:
-        """Record each stage of forward(x) into its own CUDA graph (x's address is baked in).
-        The first forward runs eagerly so one-time host set-up happens outside the capture."""
+        """Record forward(x) as one CUDA graph, and each stage into a graph of its own for per-stage
+        timing (x's address is baked in). The first forward runs eagerly so one-time host set-up
+        happens outside the capture."""
         self.forward(x)
         torch.cuda.synchronize()
         self.graphs = []
@@ -123,28 +138,34 @@ class MoELayer:
             with torch.cuda.graph(g):
                 self._stage(i, x, torch.cuda.current_stream())
             self.graphs.append(g)
+        self.graph_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_all):
+            self.forward(x, stream=torch.cuda.current_stream())
         torch.cuda.synchronize()
 
     def replay(self, events=None) -> torch.Tensor:
-        """Replay the captured forward on the current stream, events (optional) between the stages."""
+        """Replay the captured forward on the current stream: the whole-forward graph, or with
+        `events` (7 CUDA events) the per-stage graphs with the events recorded between them."""
         st = torch.cuda.current_stream()
+        if events is None:
+            self.graph_all.replay()
+            return self.buf["y"]
         for i, g in enumerate(self.graphs):
-            if events is not None:
-                events[i].record(st)
+            events[i].record(st)
             g.replay()
-        if events is not None:
-            events[len(self.graphs)].record(st)
+        events[len(self.graphs)].record(st)
         return self.buf["y"]
 
     def launches_per_forward(self) -> int:
-        """Kernel launches of one forward: router (split + tensor-core kernel for bf16 with n <= 128, else 1),
-        capacity 3, dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
+        """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection and
+        the finish kernel; else 1),
+        capacity 2 (count + scan, assign), dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
         combine 1, statistics 1."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
-        router = 2 if (bf16 and s.n <= 128) else 1
+        router = 3 if (bf16 and s.n <= 128) else 1
         ffn = 1 if bf16 else 2
-        return router + 3 + 1 + ffn + 1 + 1
+        return router + 2 + 1 + ffn + 1 + 1
 
 
 def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:

@@ -214,6 +214,38 @@ def test_balance_step_bitexact(m, n, k, rule):
     assert host(info)[2] == info_ref[2] and host(info)[3] == info_ref[3]
 
 
+@pytest.mark.parametrize("m,n,k", [(8192, 64, 4), (65536, 256, 8), (3000, 24, 5), (1002, 6, 3)])
+def test_balance_step_chain(m, n, k):
+    # each STEP starts from the previous one's beta, so the column pass finds the new thresholds
+    # inside its window around the old ones (the first step, from beta = 0, takes the full select)
+    s = W.make_qb_scores(m, n, seed=11)
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(3):
+        i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=b, mode=oracle.QB_STEP)
+        idx, beta, info = lb.moe_balance_assign(dev(s), k, beta=dev(b), mode=lb.MOE_QB_STEP)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(beta) == b_ref).all()
+        assert host(info)[2] == info_ref[2] and host(info)[3] == info_ref[3]
+        b = b_ref
+
+
+@pytest.mark.parametrize("m,n,k", [(65536, 4, 1), (32768, 8, 2)])
+def test_balance_step_heavy_ties(m, n, k):
+    # integer-grid scores: u = s - alpha repeats a few values thousands of times per column (signed
+    # zeros among them); at (65536, 4, 1) the selected key alone outnumbers the shared-memory
+    # candidate list, so the column pass streams its last digits from global memory
+    s = np.round(W.make_qb_scores(m, n, seed=7, skew_std=0.0)).astype(np.float32)
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(2):
+        i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=b, mode=oracle.QB_STEP)
+        idx, beta, info = lb.moe_balance_assign(dev(s), k, beta=dev(b), mode=lb.MOE_QB_STEP)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(beta) == b_ref).all()
+        b = b_ref
+
+
 @pytest.mark.parametrize("m,n,k,iters,rule", [(2048, 32, 4, 8, 0), (2048, 32, 4, 0, 0), (1024, 16, 2, 3, 1),
                                               (4096, 64, 8, 20, 0), (512, 8, 1, 2, 0), (4096, 64, 8, 40, 0),
                                               (2048, 16, 3, 33, 1)])
