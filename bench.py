@@ -35,15 +35,56 @@ import workloads as W  # noqa: E402
 METRIC = "MoE layer tokens/s (route+balance+dispatch+FFN+combine) and % roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0            # burst
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # seconds-long loop under the power cap
 
 
 def peaks():
+    """(HBM GB/s, source) from the measured peaks file, else the fallback figure."""
+    return peaks_all()["hbm_gbs"], peaks_all()["source"]
+
+
+def peaks_all():
     try:
         with open(PEAKS_FILE) as fh:
             p = json.load(fh)
-        return float(p["hbm_gbs"]), "measured"
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED, "source": "fallback"}
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch, from the ncu capture
+# summarised in profiles/ffn_fused_tc_switch.md (the Switch-Base-like shape only). Must be reset
+# to None whenever the kernel changes.
+FFN_DRAM_TRAFFIC = {"switch": 1273.434e6 + 63.501e6}
+
+
+def ffn_roofline(cfg, offsets, ffn_ms, esz=2):
+    """The expert FFN against the roofline that binds it at this shape: HBM (algorithmic bytes:
+    the weights of every expert with rows, xbuf read and ybuf written once) or the tensor cores
+    (4 rows d d_ff flop), whichever takes longer at the measured peaks. The tensor peak is the
+    sustained bf16 figure: the FFN is timed inside a loop of whole forwards."""
+    pk = peaks_all()
+    rows = int(offsets[-1])
+    nbytes = ffn_algorithmic_bytes(cfg, offsets, esz)
+    flops = 4.0 * rows * cfg.d * cfg.d_ff
+    s = ffn_ms * 1e-3
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops_sustained"] * 1e12)
+    common = {"kernel": "moe_expert_ffn (expert GEMM1 + GEMM2, one launch)",
+              "traffic": FFN_DRAM_TRAFFIC.get(cfg.name),
+              "algorithmic_bytes_per_launch": nbytes, "flop_per_launch": flops, "launch_ms": ffn_ms}
+    if t_tc > t_hbm:
+        achieved = flops / s / 1e12
+        return dict(common, bound="tensor", achieved=achieved, peak=pk["bf16_tflops_sustained"], unit="TFLOP/s",
+                    frac=achieved / pk["bf16_tflops_sustained"],
+                    peak_source=f"{pk['source']} bf16_tflops_sustained")
+    achieved = nbytes / s / 1e9
+    return dict(common, bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                frac=achieved / pk["hbm_gbs"], peak_source=f"{pk['source']} hbm_gbs")
 
 
 def workload_desc(cfg):
@@ -185,15 +226,17 @@ def ffn_algorithmic_bytes(cfg, offsets, esz=2):
     return used * per_expert + int(rows.sum()) * cfg.d * esz * 2
 
 
-def stage_bytes(cfg, offsets, esz=2):
+def stage_bytes(cfg, offsets, src_tokens_read, esz=2):
+    """Algorithmic HBM bytes per stage: each input read once, each output written once
+    (dispatch reads each token with a kept row once, however many of its rows are kept)."""
     m, d, n, k = cfg.m, cfg.d, cfg.n, cfg.k
     rows = int(offsets[-1])
     return {
         "router": m * d * esz + d * n * 4 + m * n * 4 + m * k * 8,
         "capacity": m * k * 4 * 4 + rows * 4,
-        "dispatch": 2 * rows * d * esz + rows * 4,
+        "dispatch": (src_tokens_read + rows) * d * esz + rows * 4,
         "ffn": ffn_algorithmic_bytes(cfg, offsets, esz),
-        "combine": rows * d * esz + m * d * esz + m * k * 8,
+        "combine": rows * d * esz + m * d * esz * (2 if cfg.residual else 1) + m * k * 8,
         "stats": m * n * 4 + m * k * 4,
     }
 
@@ -218,8 +261,12 @@ def run_gpu(args, cfg):
     inp = W.make_layer_inputs(cfg, seed=rank_seed(rank))
     w = weights_to_device(inp, dt)
     shape = LayerShape(m=cfg.m, d=cfg.d, n=cfg.n, k=cfg.k, d_ff=cfg.d_ff, score_fn=cfg.score_fn, dtype=dt,
-                       capacity=cfg.capacity, seg_len=cfg.seg_len, renorm_topk=cfg.renorm_topk)
+                       capacity=cfg.capacity, seg_len=cfg.seg_len, renorm_topk=cfg.renorm_topk, alpha=cfg.alpha,
+                       gamma=cfg.gamma, residual=bool(cfg.residual), lossfree=cfg.lossfree_bias > 0)
     layer = MoELayer(shape, w)
+    if world > 1:
+        # data-parallel replicas: the global-batch statistics pool every rank's counts
+        layer.enable_global_stats(cfg.m * world)
     x_host = torch.from_numpy(inp["x"]).to(dt).pin_memory()
     x = x_host.to("cuda")
     stream = torch.cuda.current_stream()
@@ -230,10 +277,18 @@ def run_gpu(args, cfg):
         layer.forward(x)
     lb.sync_status()
     if args.eager:
-        run = lambda events=None: layer.forward(x, events=events)  # noqa: E731
+        fwd = lambda events=None: layer.forward(x, events=events)  # noqa: E731
     else:
         layer.capture(x)
-        run = layer.replay
+        fwd = layer.replay
+
+    def run(events=None):
+        """One step: the forward, then (data-parallel replicas) the cross-rank statistics."""
+        fwd(events=events)
+        if world > 1:
+            layer.sync_global_stats()
+
+    if not args.eager:
         for _ in range(args.warmup):
             run()
         lb.sync_status()
@@ -269,16 +324,26 @@ def run_gpu(args, cfg):
     stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, s in enumerate(MoELayer.STAGES)}
     offsets = layer.buf["expert_offsets"].cpu().numpy()
+    src_read = int(torch.unique(layer.buf["src_token"][: int(offsets[-1])]).numel())
 
     # end-to-end through the public API, as a serving loop runs it: every step copies its input
     # from pinned host memory, runs the layer and reads the output and the loss back. Two layer
     # instances (shared weights, own buffers) alternate so step t's copies overlap the neighbours'
     # compute; events order the reuse of each instance's buffers.
     layers = [layer, MoELayer(shape, w)]
+    if world > 1:
+        layers[1].enable_global_stats(cfg.m * world)
     xs = [x, torch.empty_like(x)]
     if not args.eager:
         layers[1].capture(xs[1])
-    runs = [run, (lambda events=None: layers[1].forward(xs[1], events=events)) if args.eager else layers[1].replay]
+    fwd1 = (lambda events=None: layers[1].forward(xs[1], events=events)) if args.eager else layers[1].replay
+
+    def run1(events=None):
+        fwd1(events=events)
+        if world > 1:
+            layers[1].sync_global_stats()
+
+    runs = [run, run1]
     y_host = [torch.empty((cfg.m, cfg.d), dtype=dt).pin_memory() for _ in range(2)]
     aux_host = [torch.empty(layer.buf["aux"].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -321,10 +386,7 @@ def run_gpu(args, cfg):
     result = None
     if rank == 0:
         hbm, src = peaks()
-        sb = stage_bytes(cfg, offsets)
-        ffn_bytes = sb["ffn"]
-        ffn_s = stage_ms["ffn"] * 1e-3
-        achieved = ffn_bytes / ffn_s / 1e9
+        sb = stage_bytes(cfg, offsets, src_read)
         tokens = cfg.m * args.steps * world
         value = whole_job_tokens_per_s(cfg.m, args.steps, world, ms)
         cpu = None
@@ -342,13 +404,13 @@ def run_gpu(args, cfg):
             "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) expert weights; per rank)",
             "config": {"workload": workload_desc(cfg), "m": cfg.m, "d_model": cfg.d, "experts": cfg.n, "k": cfg.k,
                        "d_ff": cfg.d_ff, "capacity": cfg.capacity, "global_batch": cfg.m * world,
-                       "parallelism": f"replicas x{world}", "launch": "eager" if args.eager else "one cuda graph per forward",
-                       "l2": "inputs larger than L2: 1.2 GB of expert weights streamed every step"},
-            "roofline": {"kernel": "moe_expert_ffn (expert GEMM1 + GEMM2)", "bound": "hbm",
-                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_source": f"{src} hbm_gbs", "traffic": None,
-                         "algorithmic_bytes_per_launch": ffn_bytes, "launch_ms": stage_ms["ffn"]},
-            "stages": {s: {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9} for s in MoELayer.STAGES},
+                       "parallelism": (f"dp{world}: replicated experts, one all-reduce of 2n fp64 per step for the "
+                                       f"global-batch statistics") if world > 1 else "one GPU", "launch": "eager" if args.eager else "one cuda graph per forward",
+                       "l2": f"inputs larger than L2: {ffn_algorithmic_bytes(cfg, offsets) / 1e9:.2f} GB of expert weights and "
+                             f"rows streamed every step"},
+            "roofline": ffn_roofline(cfg, offsets, stage_ms["ffn"]),
+            "stages": {s: {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9,
+                           "hbm_frac": sb[s] / (stage_ms[s] * 1e-3) / 1e9 / hbm} for s in MoELayer.STAGES},
             "stages_note": "per-stage graphs with events between them, a separate run of K forwards",
             "rows_kept": int(offsets[-1]),
             "cpu_baseline": cpu,
@@ -357,7 +419,7 @@ def run_gpu(args, cfg):
                     "d2h_bytes_per_step": y_host[0].numel() * y_host[0].element_size() + aux_host[0].numel() * 4,
                     "pipelined": "host copies of step t overlap compute of steps t-1 and t+1 (3 streams)"},
             "clocks": clk,
-            "gpu_launches": args.steps * layer.launches_per_forward(),
+            "gpu_launches": args.steps * (layer.launches_per_forward() + (2 if world > 1 else 0)),
         }
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -398,15 +460,20 @@ def run_gpu_qb(args):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    # one STEP (row pass + column pass, the practical per-training-step form) for the per-pass figures
+    # STEP (row pass + column pass from the converged beta, the practical per-training-step form):
+    # 20 calls after 3 warm-up calls, for the per-pass figure
+    info_step = torch.zeros_like(info)
+    for _ in range(3):
+        lb.moe_balance_assign(s, k, beta=beta, mode=lb.MOE_QB_STEP, topk_idx=idx, info=info_step, workspace=ws)
+    torch.cuda.synchronize()
     st0, st1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_step = 20
     st0.record(stream)
-    for _ in range(args.steps):
-        lb.moe_balance_assign(s, k, beta=beta, mode=lb.MOE_QB_STEP, topk_idx=idx, info=torch.zeros_like(info),
-                              workspace=ws)
+    for _ in range(n_step):
+        lb.moe_balance_assign(s, k, beta=beta, mode=lb.MOE_QB_STEP, topk_idx=idx, info=info_step, workspace=ws)
     st1.record(stream)
     torch.cuda.synchronize()
-    step_ms = st0.elapsed_time(st1) / args.steps
+    step_ms = st0.elapsed_time(st1) / n_step
     inf = info.cpu().tolist()
     hbm, src = peaks()
     line = {"metric": METRIC, "value": m / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,

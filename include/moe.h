@@ -257,6 +257,44 @@ MOE_API moe_status moe_balance_stats(const float* probs, const int32_t* topk_idx
                              int64_t seg_len, float alpha, float* f, float* P, float* aux, float* vio,
                              float* bias_inout, float gamma, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * Global-batch statistics across data-parallel ranks, step 1 of 3: this rank's totals.
+ * Passage: "Qwen global-batch load balance for MoE LLM training" (agentlenshq.com):
+ * the global batch spans every data-parallel rank, so f_i is synchronised across the
+ * ranks (the counts are summed) before the loss is computed on the pooled values.
+ *
+ *  probs     [m, n] router scores of this rank's m tokens, or NULL (then row 1 is 0).
+ *  topk_idx  [m, k] routing decision of this rank's tokens.
+ *  totals    [2, n] fp64 out: row 0 = routed copies per expert (exact integers),
+ *            row 1 = sum over the m tokens of probs[:, e] (fixed-order fp64).
+ *  workspace moe_balance_totals_workspace_size(m, n) bytes.
+ * Step 2 (the caller's): sum `totals` element-wise over the ranks (one all-reduce of
+ * 2 n doubles, e.g. NCCL on the device buffer). Step 3: moe_balance_global.
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE.
+ */
+MOE_API size_t moe_balance_totals_workspace_size(int64_t m, int32_t n);
+MOE_API moe_status moe_balance_totals(const float* probs, const int32_t* topk_idx, int64_t m, int32_t n, int32_t k,
+                              double* totals, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Global-batch statistics across data-parallel ranks, step 3 of 3.
+ * Passage: as moe_balance_totals; the loss L = alpha N sum_i f_i P_i of
+ * "Switch Transformers paper review" (tildalice.io/?p=118) and the Loss-Free
+ * update b <- b - gamma sign(F - 1/n) of "MoE travelogue 6" eq. (2), taken on the
+ * pooled counts so every rank applies the same update.
+ *
+ *  totals    [2, n] fp64: the element-wise sum of every rank's moe_balance_totals.
+ *  m_total   tokens over all ranks.  has_probs: row 1 holds probability sums.
+ *  f, P      [n] out: f_i = count_i / (k m_total), P_i = psum_i / m_total (P only with has_probs).
+ *  aux       [1] out (with has_probs): alpha n sum_i f_i P_i.
+ *  vio       [3] out or NULL: MaxVio, MinVio, AvgVio of the pooled counts.
+ *  bias_inout [n] Loss-Free bias updated in place, or NULL.
+ * A count that is not a non-negative integer sets the device error word.
+ */
+MOE_API moe_status moe_balance_global(const double* totals, int64_t m_total, int32_t n, int32_t k, int32_t has_probs,
+                              float alpha, float* f, float* P, float* aux, float* vio, float* bias_inout, float gamma,
+                              moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size", "moe_router_topk", "moe_balance_assign_workspace_size",
            "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
-           "moe_balance_stats", "moe_capacity_slots_static")
+           "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
+           "moe_balance_totals", "moe_balance_global")
 
 
 class MoEError(RuntimeError):
@@ -69,6 +70,10 @@ def lib() -> C.CDLL:
         L.moe_balance_stats_workspace_size.argtypes = [I64, I32, I64]
         L.moe_balance_stats_workspace_size.restype = SZ
         L.moe_balance_stats.argtypes = [P, P, I64, I32, I32, I64, F, P, P, P, P, P, F, P, SZ, P]
+        L.moe_balance_totals_workspace_size.argtypes = [I64, I32]
+        L.moe_balance_totals_workspace_size.restype = SZ
+        L.moe_balance_totals.argtypes = [P, P, I64, I32, I32, P, P, SZ, P]
+        L.moe_balance_global.argtypes = [P, I64, I32, I32, I32, F, P, P, P, P, P, F, P]
         for name in EXPORTS:
             if name not in ("moe_last_error",) and not name.endswith("_workspace_size"):
                 getattr(L, name).restype = C.c_int
@@ -250,6 +255,41 @@ def moe_balance_stats(probs, topk_idx, n, seg_len=None, alpha=1e-2, bias_inout=N
         _ptr(probs), _ptr(topk_idx), m, n, k, seg_len, alpha, _ptr(out["f"]), _ptr(out["P"] if probs is not None else None),
         _ptr(out["aux"] if probs is not None else None), _ptr(out["vio"]), _ptr(bias_inout), gamma, _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_balance_totals(probs, topk_idx, n, totals=None, workspace=None, stream=None):
+    """This rank's [2, n] fp64 totals: routed copies per expert and probability sums (row 1 is 0 without probs)."""
+    m, k = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, torch.int32, (m, k), "topk_idx")
+    _need(probs, torch.float32, (m, n), "probs")
+    if totals is None:
+        totals = torch.empty((2, n), dtype=torch.float64, device=dev)
+    _need(totals, torch.float64, (2, n), "totals")
+    ws_bytes = lib().moe_balance_totals_workspace_size(m, n)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _check("moe_balance_totals", lib().moe_balance_totals(
+        _ptr(probs), _ptr(topk_idx), m, n, k, _ptr(totals), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return totals
+
+
+def moe_balance_global(totals, m_total, k, has_probs=True, alpha=1e-2, bias_inout=None, gamma=1e-3, out=None,
+                       stream=None):
+    """Global-batch f, P [n], aux [1], vio [3] from totals summed over the ranks (m_total tokens in all)."""
+    n = totals.shape[1]
+    dev = totals.device
+    _need(totals, torch.float64, (2, n), "totals")
+    _need(bias_inout, torch.float32, (n,), "bias_inout")
+    if out is None:
+        out = dict(f=torch.empty((n,), dtype=torch.float32, device=dev),
+                   P=torch.empty((n,), dtype=torch.float32, device=dev),
+                   aux=torch.empty((1,), dtype=torch.float32, device=dev),
+                   vio=torch.empty((3,), dtype=torch.float32, device=dev))
+    _check("moe_balance_global", lib().moe_balance_global(
+        _ptr(totals), m_total, n, k, 1 if has_probs else 0, alpha, _ptr(out["f"]), _ptr(out["P"]), _ptr(out["aux"]),
+        _ptr(out["vio"]), _ptr(bias_inout), gamma, _stream(stream)))
     return out
 
 

@@ -27,7 +27,10 @@ cudaError_t launch_ffn(const void* xbuf, moe_dtype dt, const void* w1, const voi
 size_t stats_workspace_bytes(int64_t m, int32_t n, int64_t seg_len);
 cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m, int n, int k, int64_t seg_len,
                          float alpha, float* f, float* P, float* aux, float* vio, float* bias, float gamma,
-                         void* workspace, cudaStream_t stream);
+                         void* workspace, cudaStream_t stream, double* totals);
+cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, int k, int has_probs, float alpha,
+                                float* f, float* P, float* aux, float* vio, float* bias, float gamma,
+                                cudaStream_t stream);
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k);
 int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int mode, int rule, int max_iters,
                        int max_repair, int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream,
@@ -79,6 +82,7 @@ moe_status moe_sync_status(moe_stream_t stream) {
             case kErrTokenIndex: return fail(MOE_ERR_INVALID_ARG, "device: src_token outside [0, m)");
             case kErrPipelineTimeout: return fail(MOE_ERR_INTERNAL, "device: a pipeline wait timed out");
             case kErrRepair: return fail(MOE_ERR_INTERNAL, "device: balanced-assignment repair failed");
+            case kErrTotals: return fail(MOE_ERR_INVALID_ARG, "device: a routed-count total is not a non-negative integer");
             default: return fail(MOE_ERR_INTERNAL, "device error code %d", code);
         }
     }
@@ -209,8 +213,37 @@ moe_status moe_balance_stats(const float* probs, const int32_t* topk_idx, int64_
     const size_t need = stats_workspace_bytes(m, n, seg_len);
     if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
     return check_launch(launch_stats(probs, topk_idx, m, n, k, seg_len, alpha, f, P, aux, vio, bias_inout, gamma,
-                                     workspace, stream),
+                                     workspace, stream, nullptr),
                         "moe_balance_stats");
+}
+
+size_t moe_balance_totals_workspace_size(int64_t m, int32_t n) { return stats_workspace_bytes(m, n, m); }
+
+moe_status moe_balance_totals(const float* probs, const int32_t* topk_idx, int64_t m, int32_t n, int32_t k,
+                              double* totals, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(m >= 1, "m must be >= 1");
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(k >= 1 && k <= n, "k must be in [1, n]");
+    REQUIRE(m * (int64_t)k < ((int64_t)1 << 31), "m * k must be < 2^31");
+    REQUIRE(topk_idx && totals, "topk_idx and totals are required");
+    const size_t need = stats_workspace_bytes(m, n, m);
+    if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+    return check_launch(launch_stats(probs, topk_idx, m, n, k, m, 0.f, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                     0.f, workspace, stream, totals),
+                        "moe_balance_totals");
+}
+
+moe_status moe_balance_global(const double* totals, int64_t m_total, int32_t n, int32_t k, int32_t has_probs,
+                              float alpha, float* f, float* P, float* aux, float* vio, float* bias_inout, float gamma,
+                              moe_stream_t stream) {
+    REQUIRE(m_total >= 1, "m_total must be >= 1");
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(k >= 1 && k <= n, "k must be in [1, n]");
+    REQUIRE(totals && f, "totals and f are required");
+    REQUIRE(!has_probs || (P && aux), "P and aux are required when has_probs is set");
+    return check_launch(launch_stats_global(totals, m_total, n, k, has_probs ? 1 : 0, alpha, f, P, aux, vio,
+                                            bias_inout, gamma, stream),
+                        "moe_balance_global");
 }
 
 size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k, moe_qb_mode mode) {

@@ -89,72 +89,68 @@ __device__ __forceinline__ void row_topk_rounds(const uint32_t (&key)[NT], const
     }
 }
 
-// Same result, usually far fewer instructions (k < 32, k < n): the (k+1)-th largest of the 32
-// lane maxima (with multiplicity) is a lower bound T of the row's (k+1)-th largest key, since k+1
-// distinct keys reach it. Every pick therefore has key >= T. When at most 32 keys reach T they
-// are gathered one per lane (through this warp's 32 shared slots) and the k + 1 rounds run over
-// single values. Returns false (nothing written) when more than 32 keys reach T.
+// Same result, far fewer instructions (k < 32, k < n), and the picks are written here.
+// T = the (k+1)-th largest of the 32 lane maxima, counted with multiplicity, is a lower bound of
+// the row's (k+1)-th largest key: k + 1 distinct keys reach it. So every pick has key >= T.
+// When at most 32 keys reach T, they are gathered one per lane in ascending j through this
+// warp's 32 shared slots. Each candidate's rank is then the number of candidates ranking before
+// it (a larger key, or an equal key at a lower j, that is at a lower slot). Ranks below k are
+// the picks, already in ascending j, and ranks k - 1 and k give vk and vk1.
+// Returns false, with nothing written, when more than 32 keys reach T.
 template <int NT>
-__device__ __forceinline__ bool row_topk_pruned(const uint32_t (&key)[NT], const float (&v)[NT], int n, int k,
-                                                uint32_t* sk, int* sj, float* sv, uint32_t& taken, float& vk,
-                                                float& vk1) {
+__device__ __forceinline__ bool row_topk_ranked(const uint32_t (&key)[NT], const float (&v)[NT], int k, int64_t i,
+                                                uint32_t* sk, int* sj, float* sv, int32_t* __restrict__ topk_idx,
+                                                int* cnt, float& vk, float& vk1) {
     const int lane = threadIdx.x & 31;
-    const uint32_t full = 0xffffffffu;
-    uint32_t lm = 0;
+    const uint32_t full = 0xffffffffu, lt = (1u << lane) - 1u;
+    uint32_t cur = 0;
 #pragma unroll
-    for (int q = 0; q < NT; ++q) lm = max(lm, key[q]);
-    // T: walk the distinct lane maxima from the top until k + 1 of them are counted
-    uint32_t cur = lm, T = 1;
-    int need = k + 1;
-    for (;;) {
+    for (int q = 0; q < NT; ++q) cur = max(cur, key[q]);
+    // remove the largest remaining lane maximum k times (one lane at a time); T = the next one
+    for (int r = 0; r < k; ++r) {
         const uint32_t mx = __reduce_max_sync(full, cur);
-        if (mx == 0) break;  // fewer than k + 1 lane maxima: every key is a candidate
-        const int c = __popc(__ballot_sync(full, cur == mx));
-        if (c >= need) { T = mx; break; }
-        need -= c;
-        if (cur == mx) cur = 0;
+        const uint32_t own = __ballot_sync(full, cur == mx);
+        if (lane == __ffs(own) - 1) cur = 0;
     }
-    int c = 0;
-#pragma unroll
-    for (int q = 0; q < NT; ++q) c += key[q] >= T ? 1 : 0;
-    const int N = (int)__reduce_add_sync(full, (unsigned)c);
-    if (N > 32) return false;
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(full, incl, o);
-        if (lane >= o) incl += y;
-    }
-    int pos = incl - c;
+    uint32_t T = __reduce_max_sync(full, cur);
+    if (T == 0) T = 1;  // fewer than k + 1 lanes hold keys: every key is a candidate
+    // gather the keys >= T in ascending j (q-major, then lane)
+    int N = 0;
 #pragma unroll
     for (int q = 0; q < NT; ++q) {
-        if (key[q] >= T) { sk[pos] = key[q]; sj[pos] = lane + 32 * q; sv[pos] = v[q]; ++pos; }
+        const bool c = key[q] >= T;
+        const uint32_t b = __ballot_sync(full, c);
+        const int pos = N + __popc(b & lt);
+        N += __popc(b);
+        if (c && pos < 32) { sk[pos] = key[q]; sj[pos] = lane + 32 * q; sv[pos] = v[q]; }
     }
+    if (N > 32) return false;
     __syncwarp();
-    uint32_t ck = lane < N ? sk[lane] : 0u;
-    const uint32_t cj = lane < N ? (uint32_t)sj[lane] : 0xffffffffu;
-    const float cv = lane < N ? sv[lane] : 0.f;
+    const bool has = lane < N;
+    const uint32_t ck = has ? sk[lane] : 0u;
+    const int cj = has ? sj[lane] : 0;
+    const float cv = has ? sv[lane] : 0.f;
     __syncwarp();
-    taken = 0;
-    vk = vk1 = 0.f;
-    for (int r = 0; r <= k; ++r) {
-        const uint32_t mx = __reduce_max_sync(full, ck);
-        const uint32_t cand = (ck != 0 && ck == mx) ? cj : 0xffffffffu;
-        const uint32_t wj = __reduce_min_sync(full, cand);
-        const uint32_t src = __ballot_sync(full, cand == wj && cand != 0xffffffffu);
-        const float wv = __shfl_sync(full, cv, src ? __ffs(src) - 1 : 0);
-        if (r < k) {
-            if (wj < (uint32_t)n && (int)(wj & 31u) == lane) taken |= 1u << (wj >> 5);
-            if (cj == wj) ck = 0;
-        }
-        if (r == k - 1) vk = wv;
-        if (r == k) vk1 = wv;
+    int rank = 0;
+    for (int c = 0; c < N; ++c) {
+        const uint32_t kc = __shfl_sync(full, ck, c);
+        rank += (kc > ck || (kc == ck && c < lane)) ? 1 : 0;
     }
+    const bool pick = has && rank < k;
+    const uint32_t pb = __ballot_sync(full, pick);
+    if (pick) {
+        topk_idx[i * k + __popc(pb & lt)] = cj;
+        atomicAdd(&cnt[cj], 1);
+    }
+    const uint32_t bk = __ballot_sync(full, has && rank == k - 1);
+    const uint32_t bk1 = __ballot_sync(full, has && rank == k);
+    vk = __shfl_sync(full, cv, __ffs(bk) - 1);
+    vk1 = __shfl_sync(full, cv, __ffs(bk1) - 1);
     return true;
 }
 
 // One warp per token, R tokens interleaved per warp so their loads overlap; each row takes the
-// pruned selection, or the plain rounds when it does not apply.
+// ranked selection, or the plain rounds when it does not apply.
 template <int NT, int R>
 __global__ void __launch_bounds__(qb::kRowThreads)
 qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
@@ -193,25 +189,26 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
         for (int u = 0; u < R; ++u) {
             const int64_t i = i0 + u;
             if (i >= m) break;
-            uint32_t taken;
             float vk, vk1;
-            if (!(prune && row_topk_pruned<NT>(key[u], v[u], n, k, s_key + wbase, s_j + wbase, s_v + wbase, taken,
-                                               vk, vk1)))
+            if (!(prune && row_topk_ranked<NT>(key[u], v[u], k, i, s_key + wbase, s_j + wbase, s_v + wbase,
+                                               topk_idx, cnt, vk, vk1))) {
+                uint32_t taken;
                 row_topk_rounds<NT>(key[u], v[u], n, k, taken, vk, vk1);
+                int pos = 0;
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const bool bit = (taken >> q) & 1u;
+                    const uint32_t mask = __ballot_sync(0xffffffffu, bit);
+                    if (bit) {
+                        topk_idx[i * k + pos + __popc(mask & lt)] = lane + 32 * q;
+                        atomicAdd(&cnt[lane + 32 * q], 1);
+                    }
+                    pos += __popc(mask);
+                }
+            }
             if (lane == 0) {
                 alpha[i] = qb_threshold(vk, vk1, rule);
                 if (vk == vk1) atomicAdd(&nties, 1);
-            }
-            int pos = 0;
-#pragma unroll
-            for (int q = 0; q < NT; ++q) {
-                const bool bit = (taken >> q) & 1u;
-                const uint32_t mask = __ballot_sync(0xffffffffu, bit);
-                if (bit) {
-                    topk_idx[i * k + pos + __popc(mask & lt)] = lane + 32 * q;
-                    atomicAdd(&cnt[lane + 32 * q], 1);
-                }
-                pos += __popc(mask);
             }
         }
     }

@@ -21,6 +21,7 @@ enum : int {
     kErrTokenIndex = 3,    // src_token outside [0, m)
     kErrPipelineTimeout = 4,  // a bounded pipeline wait gave up
     kErrRepair = 5,        // balanced-assignment repair found no valid path
+    kErrTotals = 6,        // a routed-count total is not a non-negative integer
 };
 __device__ int g_error = 0;
 

@@ -1,5 +1,5 @@
 // router_tc.cu -- fp32-accurate router projection on the bf16 tensor cores, with the
-// score function, ranking and top-k fused into the TMEM epilogue.
+// score function, ranking and top-k fused into the epilogue.
 //
 // Switch Transformers paper review (tildalice.io/?p=118), selective precision:
 // the router runs in fp32. x is bf16 (exact in fp32); W_r is fp32. Each W_r
@@ -9,31 +9,34 @@
 // the tensor core accumulates in fp32: fp32-accurate logits at tensor-core speed.
 //
 //   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand)
-//   router_tc_kernel     one CTA per 128 tokens and column tile of experts (64 wide when
-//                        the logits go to memory, all n otherwise), 192 threads:
-//     warp 0 lane 0   TMA: x tile 128x64 + the three 64-wide W parts per stage
+//   router_tc_kernel     one CTA per 128 tokens and 64-wide column tile of experts
+//                        (n <= 128, so one or two tiles), 192 threads:
+//     warp 0 lane 0   TMA: x tile 128x64 + the three W parts of the tile per stage
 //     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = the tile width (3 parts x 4 K-steps per stage)
 //     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM
 //                     lane); each K block's product lands in a fresh TMEM accumulator
 //                     (two, ping-pong) and is added into fp32 registers with
 //                     round-to-nearest adds, which keeps the sum fp32-accurate;
-//                     then the warp parks its 32 rows in shared memory. With probs_out
-//                     the rows are stored there as fp32 logits (coalesced) and
-//                     router_finish_kernel (one warp per row over the whole GPU) turns
-//                     them into scores, keys, top-k and gates in place; without it the
-//                     drain threads finish their rows themselves (nothing to store).
+//                     then the warp parks its 32 rows in shared memory.
+//   Finish. With probs_out the logits are stored (coalesced) and router_finish_kernel
+//   (one warp per row, the whole GPU) finishes them in place. Without it, for k <= 8
+//   the CTAs of the two column tiles of the same tokens form a 2-CTA cluster: thread
+//   r of each finishes row r over its own columns and trades the row maximum, the
+//   exp-sum and its local top-k with the peer through distributed shared memory, and
+//   rank 0 writes the picks. For larger k without probs_out each CTA takes whole rows
+//   (one tile of all n experts) and a warp finishes each row.
 #include "tc_ptx.cuh"
 
 namespace moe {
 
 namespace rtc {
-constexpr int BM = 128, BK = 64, NMAX = 128, STAGES = 3;
+constexpr int BM = 128, BK = 64, NMAX = 128, kMaxStages = 5;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 drain + epilogue
 constexpr int A_BYTES = BM * BK * 2;
 }  // namespace rtc
 
 struct RouterTcShared {
-    uint64_t full[rtc::STAGES], empty[rtc::STAGES], tfull[2], tempty[2];
+    uint64_t full[rtc::kMaxStages], empty[rtc::kMaxStages], tfull[2], tempty[2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -45,8 +48,8 @@ __host__ __device__ inline uint32_t router_tmem_cols(int np) {
     while ((int)c < 2 * np) c <<= 1;
     return c;
 }
-inline size_t router_tc_smem(int np) {
-    return 1024 + (size_t)rtc::STAGES * router_stage_bytes(np) + sizeof(RouterTcShared);
+inline size_t router_tc_smem(int np, int stages) {
+    return 1024 + (size_t)stages * router_stage_bytes(np) + sizeof(RouterTcShared);
 }
 
 // W_r [d, n] fp32 -> out [3, n, d] bf16 with w = out[0] + out[1] + out[2] (32x32 tiles through shared memory).
@@ -77,60 +80,160 @@ __global__ void router_split_kernel(const float* __restrict__ w_r, int d, int n,
 
 constexpr int KTHREAD = 8;  // largest k finished one row per thread
 
-// Finish one token row in one thread: h[0..n) in shared memory (stride-1 within the row).
-// Same definitions as finish_row: softmax / logistic in fp32, key = score + bias or the
-// logit (softmax) / rho (sigmoid), top-k with ties to the lower index, gates.
-__device__ __noinline__ void finish_row_thread(const float* __restrict__ h, int64_t row, int n, int k, int fn,
-                                               int renorm, const float* __restrict__ rank_bias,
-                                               float* __restrict__ probs_out, int32_t* __restrict__ topk_idx,
-                                               float* __restrict__ topk_gate) {
-    float mx = -INFINITY, sum = 0.f;
-    if (fn == MOE_SOFTMAX) {
-        for (int j = 0; j < n; ++j) mx = fmaxf(mx, h[j]);
-        for (int j = 0; j < n; ++j) sum += expf(h[j] - mx);
-    }
-    float kk[KTHREAD], kp[KTHREAD];
-    int ki[KTHREAD];
+namespace rtc {
+enum { kModeLogits = 0, kModeFused = 1, kModeRows = 2 };
+}  // namespace rtc
+
+// Insert (key, j, p) into a best-first list of length k <= KTHREAD (ties: the lower index first).
+__device__ __forceinline__ void topk_insert(float (&kk)[KTHREAD], int (&ki)[KTHREAD], float (&kp)[KTHREAD], int k,
+                                            float key, int j, float p) {
+    bool placed = false;
 #pragma unroll
-    for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
-    float* prow = probs_out ? probs_out + row * n : nullptr;
-    for (int j = 0; j < n; ++j) {
-        const float hj = h[j];
-        const float p = (fn == MOE_SOFTMAX) ? expf(hj - mx) / sum : 1.f / (1.f + expf(-hj));
-        if (prow) prow[j] = p;
-        const float key = rank_bias ? __fadd_rn(p, rank_bias[j]) : (fn == MOE_SOFTMAX ? hj : p);
-        // insert into the best-first list of length k (ties: the lower index ranks first)
-        bool placed = false;
-#pragma unroll
-        for (int t = KTHREAD - 1; t >= 0; --t) {
-            if (t < k && !placed) {
-                const int u = t > 0 ? t - 1 : 0;
-                if (t > 0 && ranks_before(key, j, kk[u], ki[u])) {
-                    kk[t] = kk[u]; ki[t] = ki[u]; kp[t] = kp[u];
-                } else {
-                    if (ranks_before(key, j, kk[t], ki[t])) { kk[t] = key; ki[t] = j; kp[t] = p; }
-                    placed = true;
-                }
+    for (int t = KTHREAD - 1; t >= 0; --t) {
+        if (t < k && !placed) {
+            const int u = t > 0 ? t - 1 : 0;
+            if (t > 0 && ranks_before(key, j, kk[u], ki[u])) {
+                kk[t] = kk[u]; ki[t] = ki[u]; kp[t] = kp[u];
+            } else {
+                if (ranks_before(key, j, kk[t], ki[t])) { kk[t] = key; ki[t] = j; kp[t] = p; }
+                placed = true;
             }
-        }
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int t = 0; t < KTHREAD; ++t) if (t < k) s += kp[t];
-#pragma unroll
-    for (int t = 0; t < KTHREAD; ++t) {
-        if (t < k) {
-            topk_idx[row * k + t] = ki[t];
-            topk_gate[row * k + t] = (fn == MOE_SOFTMAX && renorm) ? kp[t] / s : kp[t];
         }
     }
 }
 
-template <int NCH>
+// Score function, ranking and top-k of 128 token rows whose logits are parked in shared memory
+// (`rows`, pitch NP + 1, this CTA's expert columns col0 .. col0 + NP - 1), one row per thread of
+// warps 2-5. With `paired`, the other CTA of the 2-CTA cluster holds the other column tile of the
+// same rows: the row maximum, the exp-sum and the local top-k lists are exchanged through
+// distributed shared memory (`xch`, read by the peer), and the peer's partial sums are added in
+// cluster-rank order so both CTAs agree bit for bit. CTA rank 0 writes the picks and gates; each
+// CTA stores its own columns of probs_out, coalesced. Called by all 192 threads of both CTAs:
+// every barrier is reached by every thread whatever happened before (`ok` only gates the work).
+template <int NP>
+__device__ void fused_finish(float* rows, float* xch, bool paired, bool ok, int64_t row0, int col0, int64_t m, int n,
+                             int k, int fn, int renorm, const float* __restrict__ rank_bias,
+                             float* __restrict__ probs_out, int32_t* __restrict__ topk_idx,
+                             float* __restrict__ topk_gate) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool worker = warp >= 2 && ok;
+    const int quad = warp & 3, r = quad * 32 + lane;
+    float* h = rows + r * (NP + 1);
+    float* xmax = xch;                                   // [128]
+    float* xsum = xch + 128;                             // [128]
+    float* lkey = xch + 256;                             // [128][KTHREAD]
+    int* lidx = reinterpret_cast<int*>(xch + 256 + 128 * KTHREAD);
+    float* lp = xch + 256 + 2 * 128 * KTHREAD;
+    const int nloc = max(0, min(NP, n - col0));          // real experts in this tile
+    const uint32_t peer = paired ? (ptx::cluster_ctarank() ^ 1u) : 0u;
+    const bool first = !paired || ptx::cluster_ctarank() == 0;
+    auto sync = [&]() {
+        if (paired) ptx::cluster_sync();
+        else __syncthreads();
+    };
+    auto peer_addr = [&](const void* p) { return ptx::mapa_shared(ptx::smem_u32(p), peer); };
+    const bool softmax = fn == MOE_SOFTMAX;
+
+    // 1. row maximum (softmax)
+    float mx = -INFINITY;
+    if (worker && softmax)
+        for (int j = 0; j < nloc; ++j) mx = fmaxf(mx, h[j]);
+    if (worker) xmax[r] = mx;
+    sync();
+    if (worker && paired && softmax) mx = fmaxf(mx, ptx::ld_cluster_f32(peer_addr(xmax + r)));
+    // 2. sum of exp(h - max), added in cluster-rank order
+    float s = 0.f;
+    if (worker && softmax)
+        for (int j = 0; j < nloc; ++j) s += expf(h[j] - mx);
+    if (worker) xsum[r] = s;
+    sync();
+    if (worker && paired && softmax) {
+        const float so = ptx::ld_cluster_f32(peer_addr(xsum + r));
+        s = first ? s + so : so + s;
+    }
+    // 3. scores (parked back over the logits), keys, this tile's top-k
+    float kk[KTHREAD], kp[KTHREAD];
+    int ki[KTHREAD];
+#pragma unroll
+    for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
+    if (worker) {
+        for (int j = 0; j < nloc; ++j) {
+            const float hj = h[j];
+            const float p = softmax ? expf(hj - mx) / s : 1.f / (1.f + expf(-hj));
+            h[j] = p;
+            const float key = rank_bias ? __fadd_rn(p, rank_bias[col0 + j]) : (softmax ? hj : p);
+            topk_insert(kk, ki, kp, k, key, col0 + j, p);
+        }
+#pragma unroll
+        for (int t = 0; t < KTHREAD; ++t)
+            if (t < k) { lkey[r * KTHREAD + t] = kk[t]; lidx[r * KTHREAD + t] = ki[t]; lp[r * KTHREAD + t] = kp[t]; }
+    }
+    sync();
+    // 4. merge with the peer's list: each entry's place = its own rank + the other list's entries
+    //    ranking before it (a strict order, so the places are a permutation); rank 0 writes
+    const int64_t row = row0 + r;
+    if (worker && first && row < m) {
+        float ok2[KTHREAD], op[KTHREAD];
+        int oi[KTHREAD];
+#pragma unroll
+        for (int t = 0; t < KTHREAD; ++t) {
+            ok2[t] = -INFINITY; oi[t] = 0x7fffffff; op[t] = 0.f;
+            if (paired && t < k) {
+                ok2[t] = ptx::ld_cluster_f32(peer_addr(lkey + r * KTHREAD + t));
+                oi[t] = ptx::ld_cluster_s32(peer_addr(lidx + r * KTHREAD + t));
+                op[t] = ptx::ld_cluster_f32(peer_addr(lp + r * KTHREAD + t));
+            }
+        }
+        int pa[KTHREAD], pb[KTHREAD];
+        float selsum = 0.f;
+#pragma unroll
+        for (int t = 0; t < KTHREAD; ++t) {
+            int ca = t, cb = t;
+#pragma unroll
+            for (int u = 0; u < KTHREAD; ++u) {
+                if (u < k && ranks_before(ok2[u], oi[u], kk[t], ki[t])) ++ca;
+                if (u < k && ranks_before(kk[u], ki[u], ok2[t], oi[t])) ++cb;
+            }
+            pa[t] = t < k ? ca : KTHREAD;
+            pb[t] = t < k ? cb : KTHREAD;
+            if (pa[t] < k) selsum += kp[t];
+            if (pb[t] < k) selsum += op[t];
+        }
+        const bool renorm_gate = softmax && renorm;
+#pragma unroll
+        for (int t = 0; t < KTHREAD; ++t) {
+            if (pa[t] < k) {
+                topk_idx[row * k + pa[t]] = ki[t];
+                topk_gate[row * k + pa[t]] = renorm_gate ? kp[t] / selsum : kp[t];
+            }
+            if (pb[t] < k) {
+                topk_idx[row * k + pb[t]] = oi[t];
+                topk_gate[row * k + pb[t]] = renorm_gate ? op[t] / selsum : op[t];
+            }
+        }
+    }
+    // 5. this tile's scores out, coalesced: the warp stores its 32 rows
+    if (worker && probs_out) {
+        __syncwarp();
+        for (int rr = 0; rr < 32; ++rr) {
+            const int64_t rw = row0 + quad * 32 + rr;
+            if (rw >= m) break;
+#pragma unroll
+            for (int q = 0; q < NP / 32; ++q) {
+                const int j = lane + 32 * q;
+                if (j < nloc) probs_out[rw * n + col0 + j] = rows[(quad * 32 + rr) * (NP + 1) + j];
+            }
+        }
+    }
+    sync();  // the peer has finished reading this CTA's exchange area
+}
+
+template <int NCH, int STAGES>
 __global__ void __launch_bounds__(rtc::kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
                  int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
-                 float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+                 float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                 int mode) {
     using namespace rtc;
     constexpr int NP = NCH * 32;
     constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
@@ -157,6 +260,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     ptx::tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     volatile int* abort_flag = &sh->abort_flag;
+    bool drain_ok = true;  // this drain thread received every K block
 
     if (warp == 0) {
         if (lane == 0) {
@@ -206,9 +310,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
         for (int j = 0; j < NP; ++j) acc[j] = 0.f;
         int buf = 0;
         uint32_t bphase = 0;
-        bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-            if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { drain_ok = false; break; }
             ptx::tc_fence_after();
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
@@ -221,14 +324,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             ptx::mbar_arrive(&sh->tempty[buf]);
             if (++buf == 2) { buf = 0; bphase ^= 1u; }
         }
-        // park the warp's 32 logit rows in the (now idle) stage memory, then finish them one row per
-        // step with the compact warp-per-row routine shared with the FMA router
-        if (ok) {
+        // park the warp's 32 logit rows in the (now idle) stage memory
+        if (drain_ok) {
             float* rows = reinterpret_cast<float*>(smem) + (size_t)quad * 32 * (NP + 1);
 #pragma unroll
             for (int j = 0; j < NP; ++j) rows[lane * (NP + 1) + j] = acc[j];
             __syncwarp();
-            if (probs_out) {
+            if (mode == kModeLogits) {
                 // logits out, coalesced (a warp stores one row's 128-byte runs per instruction);
                 // router_finish_kernel turns them into scores and picks in place
                 for (int rr = 0; rr < 32; ++rr) {
@@ -240,13 +342,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                         if (j < n) probs_out[r * n + j] = rows[rr * (NP + 1) + lane + 32 * q];
                     }
                 }
-            } else if (k <= KTHREAD) {
-                // one thread per token row: compact loops over the experts, top-k in registers
-                const int64_t r = row0 + quad * 32 + lane;
-                if (r < m)
-                    finish_row_thread(rows + lane * (NP + 1), r, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
-                                      topk_gate);
-            } else {
+            } else if (mode == kModeRows) {
+                // whole rows in this CTA (k > KTHREAD, no scores out): a warp finishes each row
                 for (int rr = 0; rr < 32; ++rr) {
                     const int64_t r = row0 + quad * 32 + rr;
                     if (r >= m) break;
@@ -258,6 +355,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             }
         }
     }
+    if (mode == kModeFused)
+        fused_finish<NP>(reinterpret_cast<float*>(smem), reinterpret_cast<float*>(smem) + BM * (NP + 1),
+                         gridDim.y == 2, drain_ok, row0, col0, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
+                         topk_gate);
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -271,23 +372,55 @@ size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt) {
     return (size_t)3 * n * d * 2 + 256;
 }
 
-template <int NCH>
-static cudaError_t launch_router_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
-                                      int fn, int renorm, const float* rank_bias, float* probs_out,
-                                      int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
-    const size_t smem = router_tc_smem(NCH * 32);
+template <int NCH, int ST>
+static cudaError_t launch_router_tc_st(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
+                                       int fn, int renorm, const float* rank_bias, float* probs_out,
+                                       int32_t* topk_idx, float* topk_gate, dim3 grid, int mode,
+                                       cudaStream_t stream) {
+    const size_t smem = router_tc_smem(NCH * 32, ST);
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NCH, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(rtc::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    if (mode == rtc::kModeFused && grid.y == 2) {
+        // the two column tiles of the same 128 tokens form a cluster (exchange through DSMEM)
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 1;
+        at[0].val.clusterDim.y = 2;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, router_tc_kernel<NCH, ST>, mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out,
+                              topk_idx, topk_gate, mode);
+}
+
+// When every CTA has an SM to itself the ring is as deep as shared memory allows (five 40 KB
+// stages for a 64-wide tile, three 64 KB stages for a 128-wide one): the x tiles come from HBM
+// and the deeper ring keeps more of them in flight. When the grid is larger than the GPU, two
+// stages, so that two CTAs (each with its own TMEM accumulators) share an SM.
+template <int NCH>
+static cudaError_t launch_router_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
+                                      int fn, int renorm, const float* rank_bias, float* probs_out,
+                                      int32_t* topk_idx, float* topk_gate, int mode, cudaStream_t stream) {
     const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
     const unsigned ctiles = (unsigned)((router_np(n) + NCH * 32 - 1) / (NCH * 32));
-    router_tc_kernel<NCH><<<dim3((unsigned)blocks, ctiles), rtc::kThreads, smem, stream>>>(
-        mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
-    return cudaGetLastError();
+    const dim3 grid((unsigned)blocks, ctiles);
+    if (blocks * ctiles > num_sms())
+        return launch_router_tc_st<NCH, 2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate,
+                                           grid, mode, stream);
+    constexpr int kDeep = NCH <= 2 ? 5 : 3;
+    return launch_router_tc_st<NCH, kDeep>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
+                                           topk_gate, grid, mode, stream);
 }
 
 // Tensor-core router for bf16 activations with n <= 128 (the drain keeps a token's n logits in registers).
@@ -303,22 +436,25 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, 
         dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
         router_split_kernel<<<tg, tb, 0, stream>>>(w_r, d, n, wsplit);
     }
-    // With probs_out the logits go to memory, so the experts split into 64-wide column tiles
-    // (twice the CTAs, half the W traffic and drain work each); without it each CTA keeps whole
-    // rows for the in-kernel finish.
+    // With probs_out the logits go to memory in 64-wide column tiles and router_finish_kernel (a
+    // warp per row, the whole GPU) finishes them in place: measured faster than finishing in this
+    // kernel, where only four warps per SM share the rows. Without probs_out (nothing to store
+    // them in) the rows are finished here: for k <= KTHREAD by the paired-tile cluster, one row
+    // per thread; for larger k each CTA keeps whole rows and a warp finishes each.
     const int np = router_np(n);
-    const int tile = probs_out ? (np < 64 ? np : 64) : np;
+    const int mode = probs_out ? rtc::kModeLogits : (k <= KTHREAD ? rtc::kModeFused : rtc::kModeRows);
+    const int tile = mode == rtc::kModeRows ? np : (np < 64 ? np : 64);
     CUtensorMap mx, mw;
     if (!map_2d(&mx, x, (uint64_t)m, (uint64_t)d, rtc::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)tile)) return cudaErrorInvalidValue;
     cudaError_t e;
     switch (tile / 32) {
-        case 1: e = launch_router_tc_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
-        case 2: e = launch_router_tc_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
-        case 3: e = launch_router_tc_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
-        default: e = launch_router_tc_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream); break;
+        case 1: e = launch_router_tc_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, mode, stream); break;
+        case 2: e = launch_router_tc_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, mode, stream); break;
+        case 3: e = launch_router_tc_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, mode, stream); break;
+        default: e = launch_router_tc_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, mode, stream); break;
     }
-    if (e != cudaSuccess || !probs_out) return e;
+    if (e != cudaSuccess || mode != rtc::kModeLogits) return e;
     // the tensor-core kernel left the fp32 logits in probs_out: finish them there, one warp per row
     return launch_router_finish(probs_out, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
 }

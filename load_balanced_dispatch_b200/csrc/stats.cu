@@ -132,10 +132,49 @@ __device__ __forceinline__ void fold_blocks(const int32_t* cnt, const double* ps
     __syncthreads();
 }
 
+// Whole-batch results from the batch totals held by thread e < n (routed copies `tot`, probability
+// sum `pall`) over m tokens: f and P rows, the loss on them, the violations and the Loss-Free
+// update. Every thread of the block calls it (block reductions inside). Optional outputs may be NULL.
+__device__ void finish_batch(int64_t tot, double pall, int64_t m, int n, int k, bool has_probs, float alpha,
+                             float* __restrict__ f_row, float* __restrict__ P_row, float* __restrict__ aux_out,
+                             float* __restrict__ vio, float* __restrict__ bias, float gamma, double* sh) {
+    const int tid = threadIdx.x;
+    const bool valid = tid < n;
+    double gprod = 0.0;
+    if (valid) {
+        const double fg = (double)tot / ((double)k * (double)m);
+        if (f_row) f_row[tid] = (float)fg;
+        if (has_probs) {
+            const double pg = pall / (double)m;
+            if (P_row) P_row[tid] = (float)pg;
+            gprod = fg * pg;
+        }
+    }
+    if (has_probs) {
+        const double g = (double)alpha * (double)n * block_sum_d(gprod, sh);
+        if (tid == 0 && aux_out) *aux_out = (float)g;
+    }
+    const double F = valid ? (double)tot / ((double)m * (double)k) * (double)n - 1.0 : 0.0;
+    if (vio) {
+        const double av = block_sum_d(valid ? fabs(F) : 0.0, sh);
+        const double mx = block_max_d(valid ? F : -INFINITY, sh);
+        const double mn = -block_max_d(valid ? -F : -INFINITY, sh);
+        if (tid == 0) { vio[0] = (float)mx; vio[1] = (float)mn; vio[2] = (float)(av / (double)n); }
+    }
+    if (bias && valid) {
+        const int64_t lhs = tot * (int64_t)n, rhs = m * (int64_t)k;
+        float b = bias[tid];
+        if (lhs > rhs) b = __fsub_rn(b, gamma);
+        else if (lhs < rhs) b = __fadd_rn(b, gamma);
+        bias[tid] = b;
+    }
+}
+
 __global__ void __launch_bounds__(stats::kThreads, 2)
 stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, int64_t m, int n, int k,
              int64_t seg_len, int64_t cps, int64_t nseg, float alpha, float* __restrict__ f, float* __restrict__ P,
-             float* __restrict__ aux, float* __restrict__ vio, float* __restrict__ bias, float gamma, StatsWs w) {
+             float* __restrict__ aux, float* __restrict__ vio, float* __restrict__ bias, float gamma, StatsWs w,
+             double* __restrict__ totals) {
     __shared__ int cnt[kMaxExperts];
     __shared__ double part[stats::kThreads * 4];
     __shared__ long long pc[stats::kThreads];
@@ -229,17 +268,17 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
         const int e = tid;
         w.segcnt[seg * n + e] = (int32_t)cs;
         const double fv = (double)cs / ((double)k * (double)seg_len);
-        f[seg * n + e] = (float)fv;
+        if (f) f[seg * n + e] = (float)fv;
         if (has_probs) {
             w.segps[seg * n + e] = ps;
             const double pv = ps / (double)seg_len;
-            P[seg * n + e] = (float)pv;
+            if (P) P[seg * n + e] = (float)pv;
             prod = fv * pv;
         }
     }
     if (has_probs) {
         const double a = (double)alpha * (double)n * block_sum_d(prod, sh);
-        if (tid == 0) { aux[seg] = (float)a; w.segaux[seg] = a; }
+        if (tid == 0) { if (aux) aux[seg] = (float)a; w.segaux[seg] = a; }
     }
     __threadfence();
     __syncthreads();
@@ -250,54 +289,55 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
 
     // ---- last segment: the whole batch, in segment order
     int64_t tot = 0;
-    double pall = 0.0, gprod = 0.0;
+    double pall = 0.0;
     fold_blocks(w.segcnt, w.segps, nseg, n, has_probs, pc, part, &tot, &pall);
-    const bool valid = tid < n;
-    if (valid) {
-        const int e = tid;
-        const double fg = (double)tot / ((double)k * (double)m);
-        f[nseg * n + e] = (float)fg;
-        if (has_probs) {
-            const double pg = pall / (double)m;
-            P[nseg * n + e] = (float)pg;
-            gprod = fg * pg;
-        }
+    if (totals && tid < n) { totals[tid] = (double)tot; totals[n + tid] = has_probs ? pall : 0.0; }
+    if (has_probs && aux && tid == 0) {
+        double micro = 0.0;
+        for (int64_t s = 0; s < nseg; ++s) micro += __ldcg(w.segaux + s);
+        aux[nseg] = (float)(micro / (double)nseg);
     }
-    if (has_probs) {
-        const double g = (double)alpha * (double)n * block_sum_d(gprod, sh);
-        if (tid == 0) {
-            double micro = 0.0;
-            for (int64_t s = 0; s < nseg; ++s) micro += __ldcg(w.segaux + s);
-            aux[nseg] = (float)(micro / (double)nseg);
-            aux[nseg + 1] = (float)g;
-        }
+    finish_batch(tot, pall, m, n, k, has_probs, alpha, f ? f + nseg * n : nullptr, P ? P + nseg * n : nullptr,
+                 aux ? aux + nseg + 1 : nullptr, vio, bias, gamma, sh);
+}
+
+// Global-batch results from totals [2, n] summed over data-parallel ranks (m_total tokens).
+__global__ void __launch_bounds__(stats::kThreads)
+stats_global_kernel(const double* __restrict__ totals, int64_t m_total, int n, int k, int has_probs, float alpha,
+                    float* __restrict__ f, float* __restrict__ P, float* __restrict__ aux, float* __restrict__ vio,
+                    float* __restrict__ bias, float gamma) {
+    __shared__ double sh[stats::kThreads / 32];
+    const int tid = threadIdx.x;
+    int64_t tot = 0;
+    double pall = 0.0;
+    if (tid < n) {
+        const double c = totals[tid];
+        tot = (c >= 0.0 && c < 9.0e15) ? (int64_t)c : 0;
+        if (c < 0.0 || c >= 9.0e15 || c != (double)tot) record_error(kErrExpertIndex);
+        pall = totals[n + tid];
     }
-    const double F = valid ? (double)tot / ((double)m * (double)k) * (double)n - 1.0 : 0.0;
-    if (vio) {
-        const double av = block_sum_d(valid ? fabs(F) : 0.0, sh);
-        const double mx = block_max_d(valid ? F : -INFINITY, sh);
-        const double mn = -block_max_d(valid ? -F : -INFINITY, sh);
-        if (tid == 0) { vio[0] = (float)mx; vio[1] = (float)mn; vio[2] = (float)(av / (double)n); }
-    }
-    if (bias && valid) {
-        const int64_t lhs = tot * (int64_t)n, rhs = m * (int64_t)k;
-        float b = bias[tid];
-        if (lhs > rhs) b = __fsub_rn(b, gamma);
-        else if (lhs < rhs) b = __fadd_rn(b, gamma);
-        bias[tid] = b;
-    }
+    finish_batch(tot, pall, m_total, n, k, has_probs != 0, alpha, f, P, aux, vio, bias, gamma, sh);
 }
 
 cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m, int n, int k, int64_t seg_len,
                          float alpha, float* f, float* P, float* aux, float* vio, float* bias, float gamma,
-                         void* workspace, cudaStream_t stream) {
+                         void* workspace, cudaStream_t stream, double* totals) {
     StatsGeometry g = stats_geometry(m, seg_len);
     StatsWs w;
     stats_layout(m, n, seg_len, &w, static_cast<char*>(workspace));
     cudaError_t e = cudaMemsetAsync(w.tickets, 0, sizeof(int32_t) * (size_t)(g.nseg + 1), stream);
     if (e != cudaSuccess) return e;
     stats_kernel<<<(unsigned)g.nchunks, stats::kThreads, 0, stream>>>(probs, topk_idx, m, n, k, seg_len, g.cps,
-                                                                      g.nseg, alpha, f, P, aux, vio, bias, gamma, w);
+                                                                      g.nseg, alpha, f, P, aux, vio, bias, gamma, w,
+                                                                      totals);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, int k, int has_probs, float alpha,
+                                float* f, float* P, float* aux, float* vio, float* bias, float gamma,
+                                cudaStream_t stream) {
+    stats_global_kernel<<<1, stats::kThreads, 0, stream>>>(totals, m_total, n, k, has_probs, alpha, f, P, aux, vio,
+                                                           bias, gamma);
     return cudaGetLastError();
 }
 

@@ -76,6 +76,9 @@ class MoELayer:
             stats=torch.empty((max(L.moe_balance_stats_workspace_size(m, n, seg), 1),), dtype=torch.uint8,
                               device=dev),
         )
+        # data-parallel replicas: set by enable_global_stats(); the Loss-Free bias then follows the
+        # pooled counts of every rank instead of this rank's
+        self.global_stats = None
 
     STAGES = ("router", "capacity", "dispatch", "ffn", "combine", "stats")
 
@@ -97,8 +100,9 @@ class MoELayer:
             moe_combine(b["ybuf"], b["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
                         stream=st)
         else:
+            local_bias = s.lossfree and self.global_stats is None
             moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
-                              bias_inout=w.get("rank_bias") if s.lossfree else None, gamma=s.gamma, out=b,
+                              bias_inout=w.get("rank_bias") if local_bias else None, gamma=s.gamma, out=b,
                               workspace=self.ws["stats"], stream=st)
 
     def forward(self, x: torch.Tensor, stream=None, events=None) -> torch.Tensor:
@@ -156,14 +160,40 @@ class MoELayer:
         events[len(self.graphs)].record(st)
         return self.buf["y"]
 
+    def enable_global_stats(self, m_total: int, group=None) -> None:
+        """Pool the statistics over data-parallel ranks: after each forward, `sync_global_stats`
+        sums this rank's totals with every other rank's (one all-reduce of 2 n doubles) and
+        computes the global-batch f, P, loss and violations, and the Loss-Free update, which
+        then no longer follows this rank's counts alone."""
+        from . import lib as _lib
+        n, m = self.shape.n, self.shape.m
+        dev = self.device
+        self.global_stats = dict(
+            m_total=m_total, group=group,
+            totals=torch.empty((2, n), dtype=torch.float64, device=dev),
+            ws=torch.empty((max(_lib().moe_balance_totals_workspace_size(m, n), 1),), dtype=torch.uint8, device=dev),
+            out=dict(f=torch.empty((n,), dtype=torch.float32, device=dev),
+                     P=torch.empty((n,), dtype=torch.float32, device=dev),
+                     aux=torch.empty((1,), dtype=torch.float32, device=dev),
+                     vio=torch.empty((3,), dtype=torch.float32, device=dev)))
+
+    def sync_global_stats(self, stream=None) -> dict:
+        """The cross-rank step of a data-parallel forward (see enable_global_stats)."""
+        from .dp import global_batch_stats
+        g, s, b = self.global_stats, self.shape, self.buf
+        return global_batch_stats(b["probs"], b["topk_idx"], s.n, g["m_total"], alpha=s.alpha,
+                                  bias_inout=self.w.get("rank_bias") if s.lossfree else None, gamma=s.gamma,
+                                  group=g["group"], totals=g["totals"], workspace=g["ws"], out=g["out"],
+                                  stream=stream)
+
     def launches_per_forward(self) -> int:
-        """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection and
-        the finish kernel; else 1),
+        """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection
+        and the finish kernel; else 1),
         capacity 2 (count + scan, assign), dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
         combine 1, statistics 1."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
-        router = 3 if (bf16 and s.n <= 128) else 1
+        router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
         ffn = 1 if bf16 else 2
         return router + 2 + 1 + ffn + 1 + 1
 

@@ -78,6 +78,16 @@ def test_invalid_arguments_rejected_before_any_launch(L):
     # workspace too small
     rc = L.moe_capacity_slots(fake, 64, 1, 8, 10, 64, fake, fake, fake, fake, fake, fake, fake, 0, None)
     assert rc == 3 and "workspace" in _err(L)
+    # global-batch statistics: totals required, m_total >= 1, workspace sized by the query
+    rc = L.moe_balance_totals(fake, fake, 64, 8, 2, None, fake, 1 << 20, None)
+    assert rc == 1 and "totals" in _err(L)
+    rc = L.moe_balance_totals(fake, fake, 64, 8, 2, fake, fake, 0, None)
+    assert rc == 3 and "workspace" in _err(L)
+    assert L.moe_balance_totals_workspace_size(64, 8) > 0
+    rc = L.moe_balance_global(fake, 0, 8, 2, 1, C.c_float(0.01), fake, fake, fake, None, None, C.c_float(1e-3), None)
+    assert rc == 1 and "m_total" in _err(L)
+    rc = L.moe_balance_global(fake, 64, 8, 2, 1, C.c_float(0.01), fake, None, None, None, None, C.c_float(1e-3), None)
+    assert rc == 1 and "P and aux" in _err(L)
     # d not a multiple of 8 for bf16 dispatch
     rc = L.moe_dispatch(fake, 1, 4, 12, fake, fake, 8, 4, fake, None)
     assert rc == 1

@@ -64,7 +64,9 @@ def test_router_logits_in_sigmoid(m, n, k, bias):
     ("bf16", 300, 200, 64, 6, 0, 1, False), ("fp32", 129, 36, 256, 8, 0, 0, False),
     ("bf16", 700, 2048, 64, 6, 1, 0, True), ("bf16", 259, 128, 256, 8, 0, 1, False),
     ("bf16", 1000, 96, 40, 3, 1, 0, False), ("bf16", 131, 4096, 64, 2, 0, 1, False),
-    ("bf16", 64, 64, 16, 12, 0, 0, False)])
+    ("bf16", 64, 64, 16, 12, 0, 0, False), ("bf16", 600, 256, 100, 8, 0, 1, False),
+    ("bf16", 300, 128, 96, 5, 1, 0, True), ("bf16", 257, 192, 65, 2, 0, 0, False),
+    ("bf16", 200, 64, 128, 4, 0, 0, True)])
 def test_router_projection(dtype, m, d, n, k, fn, renorm, bias):
     rng = np.random.default_rng(d + n)
     x = rng.standard_normal((m, d)).astype(np.float32)
@@ -81,6 +83,27 @@ def test_router_projection(dtype, m, d, n, k, fn, renorm, bias):
     assert (host(idx)[ok] == i_ref[ok]).all()
     assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-5)
     assert np.allclose(host(probs), p_ref, rtol=1e-5, atol=1e-9)
+
+
+@pytest.mark.parametrize("m,d,n,k,fn,renorm,bias", [(517, 768, 128, 1, 0, 0, False), (300, 200, 64, 6, 0, 1, False),
+                                                      (700, 512, 64, 6, 1, 0, True), (64, 64, 16, 12, 0, 0, False),
+                                                      (400, 128, 100, 8, 1, 0, True)])
+def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
+    # no probs_out: the tensor-core path finishes the rows in the kernel (paired tiles for n > 64,
+    # whole rows for k > 8) and stores nothing but the picks and gates
+    rng = np.random.default_rng(d * 3 + n)
+    x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
+    w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32) if bias else None
+    _, i_ref, g_ref, margin = oracle.router(x, w, m, d, n, k, fn, renorm, b)
+    idx, gate, probs = lb.moe_router_topk(dev(x, torch.bfloat16), dev(w), n, k, fn, renorm,
+                                          rank_bias=None if b is None else dev(b), want_probs=False)
+    torch.cuda.synchronize()
+    assert probs is None
+    ok = margin > MARGIN
+    assert ok.mean() > 0.97
+    assert (host(idx)[ok] == i_ref[ok]).all()
+    assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-5)
 
 
 # ---------------------------------------------------------------- capacity
@@ -198,6 +221,36 @@ def test_balance_stats_golden_identity(golden):
         torch.cuda.synchronize()
         assert (host(out["aux"]) == np.float32(g["expected_aux"][0])).all()
         assert (host(out["vio"]) == 0).all()
+
+
+@pytest.mark.parametrize("m,n,k,ranks,with_probs", [(8192, 128, 1, 2, True), (6000, 64, 6, 3, True),
+                                                   (4096, 24, 3, 4, False)])
+def test_balance_global_across_ranks(m, n, k, ranks, with_probs):
+    # one batch split over `ranks` pretend ranks: per-rank totals, summed, then the global
+    # statistics = the oracle's whole-batch row on the unsplit batch
+    rng = np.random.default_rng(m + n)
+    p = rng.random((m, n)).astype(np.float32)
+    p /= p.sum(1, keepdims=True)
+    idx = W.make_topk_idx(m, n, k, seed=9, skew=1.2)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32)
+    ref = oracle.balance_stats(p if with_probs else None, idx, m, n, k, m, 1e-2, bias=b, gamma=1e-3)
+    total = torch.zeros((2, n), dtype=torch.float64, device="cuda")
+    cuts = [r * m // ranks for r in range(ranks + 1)]
+    for r in range(ranks):
+        lo, hi = cuts[r], cuts[r + 1]
+        t = lb.moe_balance_totals(dev(p[lo:hi]) if with_probs else None, dev(idx[lo:hi]), n)
+        total += t
+    bd = dev(b)
+    out = lb.moe_balance_global(total, m, k, has_probs=with_probs, alpha=1e-2, bias_inout=bd, gamma=1e-3)
+    torch.cuda.synchronize()
+    lb.sync_status()
+    assert (host(total)[0] == np.bincount(idx.ravel(), minlength=n)).all()
+    assert (host(out["f"]) == ref["f"][-1].astype(np.float32)).all()
+    if with_probs:
+        assert np.allclose(host(out["P"]), ref["P"][-1], rtol=TOL_STATS, atol=0)
+        assert np.allclose(host(out["aux"])[0], ref["aux"][-1], rtol=TOL_STATS, atol=0)
+    assert np.allclose(host(out["vio"]), ref["vio"], rtol=1e-6, atol=1e-7)
+    assert (host(bd) == ref["bias"]).all()
 
 
 # ---------------------------------------------------------------- balanced assignment
