@@ -56,10 +56,10 @@ def peaks_all():
                 "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED, "source": "fallback"}
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch, from the ncu capture
-# summarised in profiles/ffn_fused_tc_switch.md (the Switch-Base-like shape only). Must be reset
-# to None whenever the kernel changes.
-FFN_DRAM_TRAFFIC = {"switch": 1273.434e6 + 63.501e6}
+# dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch at a shape, from the
+# ncu capture summarised under profiles/. Emptied whenever the kernel changes (the figure would be
+# stale), refilled from the next capture.
+FFN_DRAM_TRAFFIC = {}
 
 
 def ffn_roofline(cfg, offsets, ffn_ms, esz=2):
@@ -409,8 +409,10 @@ def run_gpu(args, cfg):
                        "l2": f"inputs larger than L2: {ffn_algorithmic_bytes(cfg, offsets) / 1e9:.2f} GB of expert weights and "
                              f"rows streamed every step"},
             "roofline": ffn_roofline(cfg, offsets, stage_ms["ffn"]),
-            "stages": {s: {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9,
-                           "hbm_frac": sb[s] / (stage_ms[s] * 1e-3) / 1e9 / hbm} for s in MoELayer.STAGES},
+            "stages": {s: ({"ms": stage_ms[s], "fused_into": "ffn (second GEMM epilogue)"}
+                           if s == "combine" and layer.ffn_combine else
+                           {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9,
+                            "hbm_frac": sb[s] / (stage_ms[s] * 1e-3) / 1e9 / hbm}) for s in MoELayer.STAGES},
             "stages_note": "per-stage graphs with events between them, a separate run of K forwards",
             "rows_kept": int(offsets[-1]),
             "cpu_baseline": cpu,

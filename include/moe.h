@@ -57,7 +57,7 @@ typedef enum {
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 typedef enum { MOE_SOFTMAX = 0, MOE_SIGMOID = 1 } moe_score_fn;
 typedef enum { MOE_QB_STEP = 0, MOE_QB_SOLVE = 1 } moe_qb_mode;
-typedef enum { MOE_QB_MIDPOINT = 0, MOE_QB_BOUNDARY = 1 } moe_qb_threshold;
+typedef enum { MOE_QB_MIDPOINT = 0, MOE_QB_BOUNDARY = 1, MOE_QB_BIP = 2 } moe_qb_threshold;
 
 /* Copies the message of the calling thread's last error (NUL-terminated, truncated to len). */
 MOE_API void moe_last_error(char* buf, size_t len);
@@ -119,7 +119,10 @@ MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float
  *             optimum of eq. (3). beta returns the last QB beta.
  *  rule       threshold between the two neighbouring order statistics:
  *             MOE_QB_MIDPOINT fp32(fp32(a + b) * 0.5) (default) or
- *             MOE_QB_BOUNDARY the (k+1)-th / (C+1)-th largest (the page's convention).
+ *             MOE_QB_BOUNDARY the (k+1)-th / (C+1)-th largest (the page's convention);
+ *             MOE_QB_BIP the BIP variant ("Related work", problem (12) with inequality
+ *             constraints and non-negative duals): the (k+1)-th / (C+1)-th largest
+ *             clipped at zero, max(0, .).
  *  topk_idx   [m, k] out: each token's experts in ascending index order.
  *  info       [4] int32 device out: beta updates done, repair moves, excess left
  *             (0 = balanced), tokens whose k-th and (k+1)-th values of s - beta
@@ -132,6 +135,23 @@ MOE_API size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k
 MOE_API moe_status moe_balance_assign(const float* s, int64_t m, int32_t n, int32_t k, float* beta, moe_qb_mode mode,
                               moe_qb_threshold rule, int32_t max_iters, int32_t max_repair, int32_t* topk_idx,
                               int32_t* info, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * One SignSGD step on beta, in place of the quantile update.
+ * Passage: "MoE travelogue 6" (kexue.fm/archives/11619), "Gradient descent",
+ * eqs. (15)-(17): with alpha given, l(beta) = sum_ij max(0, s_ij - alpha_i - beta_j)
+ * + (m k / n) sum_j beta_j has dl/dbeta_j = m k / n - sum_i chi(s_ij - alpha_i - beta_j > 0),
+ * and beta_j <- beta_j - gamma sign(dl/dbeta_j).
+ *  The row pass selects x = topk(s - beta_old) and sets alpha by `rule`, as the
+ *  STEP mode of moe_balance_assign. Then count_j = #{i : fp32(s_ij - alpha_i) > beta_j}
+ *  (exact integers) and beta_j moves by gamma (one fp32 add or subtract; no move
+ *  when count_j = m k / n).
+ *  s, beta, rule, topk_idx, info, workspace: as moe_balance_assign (STEP).
+ *  The workspace of moe_balance_assign_workspace_size(m, n, k, MOE_QB_STEP) serves.
+ */
+MOE_API moe_status moe_balance_sign_step(const float* s, int64_t m, int32_t n, int32_t k, float* beta, float gamma,
+                                 moe_qb_threshold rule, int32_t* topk_idx, int32_t* info, void* workspace,
+                                 size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Capacity slots and the expert-major row layout.
@@ -218,6 +238,27 @@ MOE_API size_t moe_expert_ffn_workspace_size(moe_dtype dt, int64_t max_rows, int
 MOE_API moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2,
                           const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d, int32_t d_ff,
                           int64_t max_rows, void* ybuf, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Expert FFN and combine in one call, for one pick per token (k = 1, bf16).
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Switch
+ * Routing Step 3 (y = p_i* E_i*(x)) with "Switch Transformer read for
+ * implementation" (molayo1419.me): with top-1 routing each expert-major row
+ * belongs to one token, so the FFN's second GEMM writes that token's output
+ * directly, gated, and ybuf is never formed.
+ *  Arguments as moe_expert_ffn (without ybuf) and moe_combine with k = 1:
+ *  src_token [rows] and dest_row [m] from moe_capacity_slots, topk_gate [m],
+ *  residual [m, d] or NULL (must not alias y), y [m, d] out.
+ *  Results: bit for bit those of moe_expert_ffn followed by moe_combine (the
+ *  same roundings in the same order); dropped tokens get the residual or zeros.
+ *  max_rows <= m. bf16 only: MOE_ERR_UNSUPPORTED for fp32 (call the two
+ *  entry points). Workspace: moe_expert_ffn_workspace_size.
+ */
+MOE_API moe_status moe_expert_ffn_combine(const void* xbuf, moe_dtype dt, const void* w1, const void* b1,
+                                  const void* w2, const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d,
+                                  int32_t d_ff, int64_t max_rows, const int32_t* src_token, const int32_t* dest_row,
+                                  const float* topk_gate, const void* residual, int64_t m, void* y, void* workspace,
+                                  size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Combine: inverse permute, gate, and join the residual path.

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_F32, MOE_BF16 = 0, 1
 MOE_SOFTMAX, MOE_SIGMOID = 0, 1
 MOE_QB_STEP, MOE_QB_SOLVE = 0, 1
-MOE_QB_MIDPOINT, MOE_QB_BOUNDARY = 0, 1
+MOE_QB_MIDPOINT, MOE_QB_BOUNDARY, MOE_QB_BIP = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_NOT_CONVERGED", 6: "MOE_ERR_INTERNAL"}
 
@@ -29,7 +29,7 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
-           "moe_balance_totals", "moe_balance_global")
+           "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step")
 
 
 class MoEError(RuntimeError):
@@ -67,9 +67,12 @@ def lib() -> C.CDLL:
         L.moe_expert_ffn_workspace_size.restype = SZ
         L.moe_expert_ffn.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, SZ, P]
         L.moe_combine.argtypes = [P, I32, P, P, P, I64, I32, I32, P, P]
+        L.moe_expert_ffn_combine.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, P, P, I64, P, P, SZ,
+                                             P]
         L.moe_balance_stats_workspace_size.argtypes = [I64, I32, I64]
         L.moe_balance_stats_workspace_size.restype = SZ
         L.moe_balance_stats.argtypes = [P, P, I64, I32, I32, I64, F, P, P, P, P, P, F, P, SZ, P]
+        L.moe_balance_sign_step.argtypes = [P, I64, I32, I32, P, F, I32, P, P, P, SZ, P]
         L.moe_balance_totals_workspace_size.argtypes = [I64, I32]
         L.moe_balance_totals_workspace_size.restype = SZ
         L.moe_balance_totals.argtypes = [P, P, I64, I32, I32, P, P, SZ, P]
@@ -225,6 +228,31 @@ def moe_expert_ffn(xbuf, w1, b1, w2, b2, expert_offsets, ybuf=None, workspace=No
     return ybuf
 
 
+def moe_expert_ffn_combine(xbuf, w1, b1, w2, b2, expert_offsets, src_token, dest_row, topk_gate, residual=None,
+                           y=None, workspace=None, stream=None):
+    """k = 1, bf16: y[t] = residual[t] + g_t FFN_e(xbuf[row of t]) with the combine done by the FFN's second
+    GEMM (no ybuf); tokens without a kept row get the residual or zeros. Returns y [m, d]."""
+    max_rows, d = xbuf.shape
+    n, d_ff, _ = w1.shape
+    m, k = dest_row.shape
+    if k != 1:
+        raise ValueError("moe_expert_ffn_combine: one pick per token (k = 1)")
+    dt = _dtype_code(xbuf)
+    for t, shp, name in ((w1, (n, d_ff, d), "w1"), (b1, (n, d_ff), "b1"), (w2, (n, d, d_ff), "w2"), (b2, (n, d), "b2")):
+        _need(t, xbuf.dtype, shp, name)
+    _need(residual, xbuf.dtype, (m, d), "residual")
+    if y is None:
+        y = torch.empty((m, d), dtype=xbuf.dtype, device=xbuf.device)
+    ws_bytes = lib().moe_expert_ffn_workspace_size(dt, max_rows, d_ff)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=xbuf.device)
+    _check("moe_expert_ffn_combine", lib().moe_expert_ffn_combine(
+        _ptr(xbuf), dt, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(expert_offsets), n, d, d_ff, min(max_rows, m),
+        _ptr(src_token), _ptr(dest_row), _ptr(topk_gate), _ptr(residual), m, _ptr(y), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return y
+
+
 def moe_combine(ybuf, dest_row, topk_gate, residual=None, y=None, stream=None):
     """y[i] = residual[i] + sum_r g_ir ybuf[dest_row[i,r]] (kept picks only). Returns y [m, d]."""
     m, k = dest_row.shape
@@ -291,6 +319,26 @@ def moe_balance_global(totals, m_total, k, has_probs=True, alpha=1e-2, bias_inou
         _ptr(totals), m_total, n, k, 1 if has_probs else 0, alpha, _ptr(out["f"]), _ptr(out["P"]), _ptr(out["aux"]),
         _ptr(out["vio"]), _ptr(bias_inout), gamma, _stream(stream)))
     return out
+
+
+def moe_balance_sign_step(s, k, beta, gamma, rule=MOE_QB_MIDPOINT, topk_idx=None, info=None, workspace=None,
+                          stream=None):
+    """One SignSGD step on beta (in place): (topk_idx [m,k] ascending experts, beta, info [4])."""
+    m, n = s.shape
+    dev = s.device
+    _need(s, torch.float32, (m, n), "s")
+    _need(beta, torch.float32, (n,), "beta")
+    if topk_idx is None:
+        topk_idx = torch.empty((m, k), dtype=torch.int32, device=dev)
+    if info is None:
+        info = torch.zeros((4,), dtype=torch.int32, device=dev)
+    ws_bytes = lib().moe_balance_assign_workspace_size(m, n, k, MOE_QB_STEP)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    _check("moe_balance_sign_step", lib().moe_balance_sign_step(
+        _ptr(s), m, n, k, _ptr(beta), gamma, rule, _ptr(topk_idx), _ptr(info), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return topk_idx, beta, info
 
 
 def moe_balance_assign(s, k, beta=None, mode=MOE_QB_SOLVE, rule=MOE_QB_MIDPOINT, max_iters=64, max_repair=1 << 20,

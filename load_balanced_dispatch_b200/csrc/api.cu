@@ -24,6 +24,10 @@ cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_r
 cudaError_t launch_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2, const void* b2,
                        const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
                        cudaStream_t stream);
+cudaError_t launch_ffn_tc_combine(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
+                                  const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* hbuf,
+                                  const int32_t* src_token, const int32_t* dest_row, const float* gate,
+                                  const void* residual, int64_t m, void* y, cudaStream_t stream);
 size_t stats_workspace_bytes(int64_t m, int32_t n, int64_t seg_len);
 cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m, int n, int k, int64_t seg_len,
                          float alpha, float* f, float* P, float* aux, float* vio, float* bias, float gamma,
@@ -32,6 +36,8 @@ cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, in
                                 float* f, float* P, float* aux, float* vio, float* bias, float gamma,
                                 cudaStream_t stream);
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k);
+int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, float gamma, int rule,
+                          int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream, const char** err);
 int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int mode, int rule, int max_iters,
                        int max_repair, int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream,
                        const char** err);
@@ -185,6 +191,34 @@ moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1, const 
                         "moe_expert_ffn");
 }
 
+moe_status moe_expert_ffn_combine(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2,
+                                  const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d, int32_t d_ff,
+                                  int64_t max_rows, const int32_t* src_token, const int32_t* dest_row,
+                                  const float* topk_gate, const void* residual, int64_t m, void* y, void* workspace,
+                                  size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
+    if (dt != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_expert_ffn_combine: bf16 only (use moe_expert_ffn + moe_combine)");
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(max_rows >= 0 && max_rows < ((int64_t)1 << 31), "bad max_rows");
+    REQUIRE(m >= 0 && max_rows <= m, "one pick per token: max_rows must be <= m");
+    REQUIRE(d >= 8 && d % 8 == 0, "d must be a positive multiple of 8");
+    REQUIRE(d_ff >= 8 && d_ff % 8 == 0, "d_ff must be a positive multiple of 8");
+    REQUIRE(expert_offsets && w1 && b1 && w2 && b2, "weights, biases and expert_offsets are required");
+    REQUIRE(m == 0 || (y && dest_row && topk_gate && src_token), "y, src_token, dest_row and topk_gate are required");
+    REQUIRE(max_rows == 0 || xbuf, "xbuf is required");
+    REQUIRE(aligned16(xbuf) && aligned16(y) && aligned16(residual) && aligned16(w1) && aligned16(w2) &&
+                aligned16(workspace),
+            "xbuf, y, residual, w1, w2 and the workspace must be 16-byte aligned");
+    REQUIRE(residual == nullptr || residual != y, "residual must not alias y");
+    const size_t need = moe_expert_ffn_workspace_size(dt, max_rows, d_ff);
+    if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+    if (m == 0) return MOE_OK;
+    return check_launch(launch_ffn_tc_combine(xbuf, w1, b1, w2, b2, expert_offsets, n, d, d_ff, max_rows, workspace,
+                                              src_token, dest_row, topk_gate, residual, m, y, stream),
+                        "moe_expert_ffn_combine");
+}
+
 moe_status moe_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
                        const void* residual, int64_t m, int32_t k, int32_t d, void* y, moe_stream_t stream) {
     REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
@@ -246,6 +280,25 @@ moe_status moe_balance_global(const double* totals, int64_t m_total, int32_t n, 
                         "moe_balance_global");
 }
 
+moe_status moe_balance_sign_step(const float* s, int64_t m, int32_t n, int32_t k, float* beta, float gamma,
+                                 moe_qb_threshold rule, int32_t* topk_idx, int32_t* info, void* workspace,
+                                 size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(m >= 1, "m must be >= 1");
+    REQUIRE(n >= 2 && n <= kMaxExperts, "n must be in [2, %d]", kMaxExperts);
+    REQUIRE(k >= 1 && k < n, "k must be in [1, n - 1]");
+    REQUIRE(m * (int64_t)k < ((int64_t)1 << 31) && m * (int64_t)n < ((int64_t)1 << 34), "m too large");
+    REQUIRE((m * k) % n == 0, "m * k must be divisible by n (every expert gets exactly m k / n tokens)");
+    REQUIRE(rule == MOE_QB_MIDPOINT || rule == MOE_QB_BOUNDARY || rule == MOE_QB_BIP, "unknown threshold rule");
+    REQUIRE(gamma >= 0.f && gamma == gamma, "gamma must be a non-negative number");
+    REQUIRE(s && beta && topk_idx && info, "s, beta, topk_idx and info are required");
+    const size_t need = balance_workspace_bytes(m, n, k);
+    if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+    const char* err = "";
+    const int rc = run_balance_sign_step(s, m, n, k, beta, gamma, rule, topk_idx, info, workspace, stream, &err);
+    if (rc != MOE_OK) return fail((moe_status)rc, "moe_balance_sign_step: %s", err);
+    return MOE_OK;
+}
+
 size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k, moe_qb_mode mode) {
     (void)mode;
     if (m < 1 || n < 1 || n > kMaxExperts || k < 1) return 0;
@@ -261,7 +314,7 @@ moe_status moe_balance_assign(const float* s, int64_t m, int32_t n, int32_t k, f
     REQUIRE(m * (int64_t)k < ((int64_t)1 << 31) && m * (int64_t)n < ((int64_t)1 << 34), "m too large");
     REQUIRE((m * k) % n == 0, "m * k must be divisible by n (every expert gets exactly m k / n tokens)");
     REQUIRE(mode == MOE_QB_STEP || mode == MOE_QB_SOLVE, "unknown mode");
-    REQUIRE(rule == MOE_QB_MIDPOINT || rule == MOE_QB_BOUNDARY, "unknown threshold rule");
+    REQUIRE(rule == MOE_QB_MIDPOINT || rule == MOE_QB_BOUNDARY || rule == MOE_QB_BIP, "unknown threshold rule");
     REQUIRE(max_iters >= 0 && max_repair >= 0, "max_iters and max_repair must be >= 0");
     REQUIRE(s && beta && topk_idx && info, "s, beta, topk_idx and info are required");
     const size_t need = balance_workspace_bytes(m, n, k);

@@ -16,7 +16,8 @@
 //              warp arg-max give the top-k set, the k-th and (k+1)-th values
 //              (alpha) and a tie flag; the set is written in ascending expert
 //              order and counted per expert.
-//   transpose  s [m, n] -> sT [n, m] once per call, so each column is contiguous.
+//              The first row pass of a call also writes s transposed (sT [n, m]),
+//              so each expert's column is contiguous for the column pass.
 //   qb_col     one CTA per expert column: one sweep keeps the keys of u near
 //              the previous beta_j in shared memory and counts those above;
 //              the C-th and (C+1)-th largest are then selected there (radix
@@ -45,8 +46,12 @@ enum { kStDone = 0, kStAugments = 1, kStError = 2, kStQbDone = 4, kStIters = 5, 
 constexpr int kBatch = 16;  // QB iterations enqueued between host checks
 }  // namespace qb
 
+// Threshold between the q-th (a) and (q+1)-th (b) largest: midpoint, the (q+1)-th, or the
+// (q+1)-th clipped at zero (BIP's non-negative duals).
 __device__ __forceinline__ float qb_threshold(float a, float b, int rule) {
-    return rule == MOE_QB_BOUNDARY ? b : __fmul_rn(__fadd_rn(a, b), 0.5f);
+    if (rule == MOE_QB_BOUNDARY) return b;
+    if (rule == MOE_QB_BIP) return b > 0.f ? b : 0.f;
+    return __fmul_rn(__fadd_rn(a, b), 0.5f);
 }
 
 // order-preserving key: larger float -> larger key; -0 is folded onto +0
@@ -155,8 +160,10 @@ template <int NT, int R>
 __global__ void __launch_bounds__(qb::kRowThreads)
 qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
               float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
-              int32_t* __restrict__ status, int tie_slot, int skip_if_done) {
+              int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT) {
     if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
+    constexpr int ROWS = (qb::kRowThreads / 32) * R;  // token rows per CTA step
+    __shared__ float tile[ROWS][kMaxExperts + 1];      // the step's rows of s, for the transposed copy
     __shared__ float sb[kMaxExperts];
     __shared__ int cnt[kMaxExperts];
     __shared__ int nties;
@@ -170,8 +177,10 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
     __syncthreads();
     const uint32_t lt = (1u << lane) - 1u;
     const bool prune = k < 32 && k < n;
-    const int64_t warps = (int64_t)gridDim.x * (qb::kRowThreads / 32);
-    for (int64_t i0 = ((int64_t)blockIdx.x * (qb::kRowThreads / 32) + (tid >> 5)) * R; i0 < m; i0 += warps * R) {
+    // CTA-uniform steps of ROWS consecutive tokens (warp w takes rows w R .. w R + R - 1), so the
+    // optional transposed copy can use block barriers
+    for (int64_t base = (int64_t)blockIdx.x * ROWS; base < m; base += (int64_t)gridDim.x * ROWS) {
+        const int64_t i0 = base + (tid >> 5) * R;
         float v[R][NT];
         uint32_t key[R][NT];
 #pragma unroll
@@ -181,8 +190,27 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
             for (int q = 0; q < NT; ++q) {
                 const int j = lane + 32 * q;
                 const bool ok = i < m && j < n;
-                v[u][q] = ok ? __fsub_rn(s[i * n + j], sb[j]) : 0.f;
+                const float sv = ok ? s[i * n + j] : 0.f;
+                if (sT && j < n) tile[(tid >> 5) * R + u][j] = sv;
+                v[u][q] = ok ? __fsub_rn(sv, sb[j]) : 0.f;
                 key[u][q] = ok ? float_key(v[u][q]) : 0u;
+            }
+        }
+        if (sT) {
+            // the first row pass also writes s transposed (sT [n, m], each expert's column
+            // contiguous for the column pass): thread j stores column j of the step's rows
+            __syncthreads();
+            const int64_t nr = min((int64_t)ROWS, m - base);
+            for (int j = tid; j < n; j += blockDim.x) {
+                float* dst = sT + (int64_t)j * m + base;
+                if (nr == ROWS && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+#pragma unroll
+                    for (int r4 = 0; r4 < ROWS; r4 += 4)
+                        *reinterpret_cast<float4*>(dst + r4) =
+                            make_float4(tile[r4][j], tile[r4 + 1][j], tile[r4 + 2][j], tile[r4 + 3][j]);
+                } else {
+                    for (int r = 0; r < nr; ++r) dst[r] = tile[r][j];
+                }
             }
         }
 #pragma unroll
@@ -211,29 +239,12 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
                 if (vk == vk1) atomicAdd(&nties, 1);
             }
         }
+        if (sT) __syncthreads();  // the tile is rewritten by the next step
     }
     __syncthreads();
     for (int j = tid; j < n; j += blockDim.x)
         if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
     if (tid == 0 && nties) atomicAdd(&status[tie_slot], nties);
-}
-
-__global__ void transpose_kernel(const float* __restrict__ s, int64_t m, int n, float* __restrict__ sT) {
-    __shared__ float tile[32][33];
-    const int64_t i0 = (int64_t)blockIdx.x * 32;
-    const int j0 = blockIdx.y * 32;
-    const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
-    for (int r = ty; r < 32; r += 8) {
-        const int64_t i = i0 + r;
-        const int j = j0 + tx;
-        tile[r][tx] = (i < m && j < n) ? s[i * n + j] : 0.f;
-    }
-    __syncthreads();
-    for (int r = ty; r < 32; r += 8) {
-        const int j = j0 + r;
-        const int64_t i = i0 + tx;
-        if (j < n && i < m) sT[(int64_t)j * m + i] = tile[tx][r];
-    }
 }
 
 // Block-wide bin selection: scanning bins from the top, the bin where the cumulative count
@@ -561,9 +572,10 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
 }
 
 namespace qb {
-constexpr int kArcThreads = 512;     // 16 warps
+constexpr int kArcThreads = 256;     // 8 warps
 constexpr int kArcBatch = 4;         // members per warp step (their loads in flight together)
-constexpr int kArcWords = 512;       // bitmap words compacted per pass: at most 16384 members
+constexpr int kArcWords = 256;       // bitmap words compacted per pass: at most 8192 members
+constexpr int kArcSlices = 8;        // CTAs per row of W, each over 1/8 of the tokens
 constexpr int kMemberCap = kArcWords * 32;
 constexpr int kStepThreads = 1024;   // 4 threads per expert column in the shortest-path rounds
 constexpr size_t kArcSmem = (size_t)(kArcThreads / 32) * kMaxExperts * (8 + 4) + (size_t)kMemberCap * 4;
@@ -581,17 +593,23 @@ __global__ void qb_member_bits_kernel(const int32_t* __restrict__ topk_idx, int6
 
 // Arc costs of the expert graph for the listed rows a = rows[blockIdx.x]:
 // W[a][b] = min over tokens i holding a but not b of s_ia - s_ib (fp64), A[a][b] = that token
-// (lowest token among equal costs). The members of a come from the bitmap (compacted into shared
-// memory, kMemberCap at a time); warp w takes members in batches of kArcBatch, lanes own columns
-// b = lane + 32 q; the 32 warps' minima are folded in warp order at the end.
+// (lowest token among equal costs). Each row is split over gridDim.y CTAs, slice y taking the
+// y-th range of bitmap words (tokens), so the few rows a repair move invalidates still spread
+// over the GPU. The members of a in the slice come from the bitmap (compacted into shared memory,
+// kMemberCap at a time); warp w takes members in batches of kArcBatch, lanes own columns
+// b = lane + 32 q; the warps' minima are folded in warp order, and the last slice of the row to
+// finish folds the slices' partials in slice order.
 template <int NT>
-__global__ void __launch_bounds__(qb::kArcThreads, 1)
+__global__ void __launch_bounds__(qb::kArcThreads, 2)
 qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_t* __restrict__ topk_idx,
               const uint32_t* __restrict__ mem, int64_t words, const int32_t* __restrict__ rows,
               const int32_t* __restrict__ nrows, double* __restrict__ W, int32_t* __restrict__ A,
-              const int32_t* __restrict__ status) {
+              const int32_t* __restrict__ status, double* Wp, int32_t* Ap, int32_t* tickets) {
     if (status[qb::kStError] || status[qb::kStDone]) return;
     if ((int)blockIdx.x >= *nrows) return;
+    const int S = gridDim.y, slice = blockIdx.y;
+    const int64_t per = (words + S - 1) / S;
+    const int64_t wbeg = min(words, (int64_t)slice * per), wend = min(words, wbeg + per);
     constexpr int NW = qb::kArcThreads / 32, B = qb::kArcBatch;
     extern __shared__ unsigned char arc_smem[];
     double* bw = reinterpret_cast<double*>(arc_smem);                       // [NW][256]
@@ -605,14 +623,14 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
     int32_t arg[NT];
 #pragma unroll
     for (int q = 0; q < NT; ++q) { best[q] = INFINITY; arg[q] = 0x7fffffff; }
-    for (int64_t w0 = 0; w0 < words; w0 += qb::kArcWords) {
+    for (int64_t w0 = wbeg; w0 < wend; w0 += qb::kArcWords) {
         // compact the members held in the next kArcWords bitmap words (token order is not needed:
         // ties go to the lowest token explicitly)
         if (threadIdx.x == 0) nlist = 0;
         __syncthreads();
         {
             const int64_t wi = w0 + threadIdx.x;
-            const uint32_t bits = (threadIdx.x < qb::kArcWords && wi < words) ? row[wi] : 0u;
+            const uint32_t bits = (threadIdx.x < qb::kArcWords && wi < wend) ? row[wi] : 0u;
             const int c = __popc(bits);
             int incl = c;
 #pragma unroll
@@ -669,6 +687,8 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
 #pragma unroll
     for (int q = 0; q < NT; ++q) { bw[warp * kMaxExperts + lane + 32 * q] = best[q]; ba[warp * kMaxExperts + lane + 32 * q] = arg[q]; }
     __syncthreads();
+    // fold the warps in order; with one slice that is the row of W, else this slice's partial
+    const int64_t pslot = ((int64_t)blockIdx.x * S + slice) * n;
     for (int b = threadIdx.x; b < n; b += blockDim.x) {
         double bb = INFINITY;
         int32_t aa = -1;
@@ -677,9 +697,37 @@ qb_arc_kernel(const float* __restrict__ s, int64_t m, int n, int k, const int32_
             const int32_t t = ba[w * kMaxExperts + b];
             if (c < bb || (c == bb && c != INFINITY && t < aa)) { bb = c; aa = t; }
         }
+        if (S == 1) {
+            W[(int64_t)a * n + b] = bb;
+            A[(int64_t)a * n + b] = bb == INFINITY ? -1 : aa;
+        } else {
+            Wp[pslot + b] = bb;
+            Ap[pslot + b] = aa;
+        }
+    }
+    if (S == 1) return;
+    // the last slice to finish folds the slices in slice order (token ranges ascend with the slice,
+    // so the lowest token among equal costs wins as in one pass) and re-arms the row's ticket
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&tickets[blockIdx.x], 1) == S - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int b = threadIdx.x; b < n; b += blockDim.x) {
+        double bb = INFINITY;
+        int32_t aa = -1;
+        for (int sl = 0; sl < S; ++sl) {
+            const int64_t ps = ((int64_t)blockIdx.x * S + sl) * n + b;
+            const double c = __ldcg(Wp + ps);
+            const int32_t t = __ldcg(Ap + ps);
+            if (c < bb || (c == bb && c != INFINITY && t < aa)) { bb = c; aa = t; }
+        }
         W[(int64_t)a * n + b] = bb;
         A[(int64_t)a * n + b] = bb == INFINITY ? -1 : aa;
     }
+    if (threadIdx.x == 0) tickets[blockIdx.x] = 0;
 }
 
 // Compact the indices a < n with flag[a] != 0, in increasing order, into out[] and *count
@@ -903,6 +951,9 @@ struct QBWorkspace {
     int32_t* nrows;
     uint32_t* mem;   // [n][ceil(m / 32)] membership bitmap
     uint32_t* win;   // [n] window half-widths of the column pass (0: default)
+    double* Wp;      // [n][kArcSlices][n] per-slice partial arc costs
+    int32_t* Ap;     // [n][kArcSlices][n] their tokens
+    int32_t* arc_tickets;  // [n] slices done per row (re-armed by the folding slice)
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -922,6 +973,9 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     p = take(sizeof(int32_t));                          if (w) w->nrows = (int32_t*)p;
     p = take(sizeof(uint32_t) * (size_t)n * (size_t)((m + 31) / 32)); if (w) w->mem = (uint32_t*)p;
     p = take(sizeof(uint32_t) * (size_t)n);             if (w) w->win = (uint32_t*)p;
+    p = take(sizeof(double) * (size_t)n * qb::kArcSlices * n);  if (w) w->Wp = (double*)p;
+    p = take(sizeof(int32_t) * (size_t)n * qb::kArcSlices * n); if (w) w->Ap = (int32_t*)p;
+    p = take(sizeof(int32_t) * (size_t)n);              if (w) w->arc_tickets = (int32_t*)p;
     return off;
 }
 
@@ -929,22 +983,23 @@ size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k) { return qb_layo
 
 template <int NT>
 static void launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
-                         int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip,
+                         int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
                          cudaStream_t stream) {
     int64_t blocks = (m + 2 * (qb::kRowThreads / 32) - 1) / (2 * (qb::kRowThreads / 32));
     if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
     if (blocks < 1) blocks = 1;
     qb_row_kernel<NT, 2><<<(unsigned)blocks, qb::kRowThreads, 0, stream>>>(s, m, n, k, beta, rule, alpha, topk_idx,
-                                                                           counts, status, tie_slot, skip);
+                                                                           counts, status, tie_slot, skip, sT);
 }
 
+// sT != nullptr: this row pass also writes s transposed into sT (the first pass of a call).
 static void launch_row(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
-                       int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip,
+                       int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
                        cudaStream_t stream) {
-    if (n <= 32) launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, stream);
-    else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, stream);
-    else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, stream);
-    else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, stream);
+    if (n <= 32) launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+    else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+    else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+    else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
 }
 
 template <int NT>
@@ -955,8 +1010,9 @@ static void launch_arc_t(const float* s, int64_t m, int n, int k, const int32_t*
         cudaFuncSetAttribute(qb_arc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qb::kArcSmem);
         attr = true;
     }
-    qb_arc_kernel<NT><<<n, qb::kArcThreads, qb::kArcSmem, stream>>>(s, m, n, k, topk_idx, w.mem, (m + 31) / 32,
-                                                                    w.rows, w.nrows, w.W, w.A, w.status);
+    qb_arc_kernel<NT><<<dim3((unsigned)n, qb::kArcSlices), qb::kArcThreads, qb::kArcSmem, stream>>>(
+        s, m, n, k, topk_idx, w.mem, (m + 31) / 32, w.rows, w.nrows, w.W, w.A, w.status, w.Wp, w.Ap,
+        w.arc_tickets);
 }
 
 static void launch_arc(const float* s, int64_t m, int n, int k, const int32_t* topk_idx, const QBWorkspace& w,
@@ -965,6 +1021,74 @@ static void launch_arc(const float* s, int64_t m, int n, int k, const int32_t* t
     else if (n <= 64) launch_arc_t<2>(s, m, n, k, topk_idx, w, stream);
     else if (n <= 128) launch_arc_t<4>(s, m, n, k, topk_idx, w, stream);
     else launch_arc_t<8>(s, m, n, k, topk_idx, w, stream);
+}
+
+// SignSGD on beta: count_j = #{i : fp32(s_ij - alpha_i) > beta_j} over the rows of s (one warp
+// per token, lane counters for the columns lane + 32 q, folded per CTA in shared memory).
+template <int NT>
+__global__ void __launch_bounds__(256)
+qb_sign_count_kernel(const float* __restrict__ s, int64_t m, int n, const float* __restrict__ alpha,
+                     const float* __restrict__ beta, int32_t* __restrict__ counts) {
+    __shared__ int cnt[kMaxExperts];
+    __shared__ float sb[kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int j = tid; j < n; j += blockDim.x) { cnt[j] = 0; sb[j] = beta[j]; }
+    __syncthreads();
+    int c[NT];
+#pragma unroll
+    for (int q = 0; q < NT; ++q) c[q] = 0;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t i = (int64_t)blockIdx.x * (blockDim.x / 32) + (tid >> 5); i < m; i += warps) {
+        const float a = alpha[i];
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+            const int j = lane + 32 * q;
+            if (j < n && __fsub_rn(s[i * n + j], a) > sb[j]) ++c[q];
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < NT; ++q)
+        if (lane + 32 * q < n && c[q]) atomicAdd(&cnt[lane + 32 * q], c[q]);
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x)
+        if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
+}
+
+__global__ void qb_sign_update_kernel(const int32_t* __restrict__ counts, int n, int64_t C, float gamma,
+                                      float* __restrict__ beta) {
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const int64_t c = counts[j];
+        if (c > C) beta[j] = __fadd_rn(beta[j], gamma);        // gradient C - c < 0
+        else if (c < C) beta[j] = __fsub_rn(beta[j], gamma);   // gradient > 0
+    }
+}
+
+int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, float gamma, int rule,
+                          int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream, const char** err) {
+    QBWorkspace w;
+    qb_layout(m, n, k, &w, static_cast<char*>(workspace));
+    const int64_t C = m * k / n;
+    cudaError_t ce;
+    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto fail;
+    if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto fail;
+    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
+    {
+        int64_t blocks = (m + 7) / 8;
+        if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
+        if (blocks < 1) blocks = 1;
+        int32_t* sc = w.counts + n;  // chi counts, separate from the pick counts
+        if (n <= 32) qb_sign_count_kernel<1><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
+        else if (n <= 64) qb_sign_count_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
+        else if (n <= 128) qb_sign_count_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
+        else qb_sign_count_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
+        qb_sign_update_kernel<<<1, 256, 0, stream>>>(sc, n, C, gamma, beta);
+    }
+    qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
+    if ((ce = cudaGetLastError()) != cudaSuccess) goto fail;
+    return MOE_OK;
+fail:
+    *err = cudaGetErrorString(ce);
+    return MOE_ERR_CUDA;
 }
 
 // Returns a moe_status; SOLVE synchronises the stream between phases.
@@ -985,12 +1109,8 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto cuda_fail;
     if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
     if ((ce = cudaMemsetAsync(w.win, 0, sizeof(uint32_t) * n, stream)) != cudaSuccess) goto cuda_fail;
-    {
-        dim3 tb(32, 8), tg((unsigned)((m + 31) / 32), (unsigned)((n + 31) / 32));
-        transpose_kernel<<<tg, tb, 0, stream>>>(s, m, n, w.sT);
-    }
     if (mode == MOE_QB_STEP) {
-        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, stream);
+        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, w.sT, stream);
         qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(w.sT, m, n, C, w.alpha, rule, beta, w.counts,
                                                                     w.counts + n, w.status, 0, 0, w.win);
         qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
@@ -1005,7 +1125,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
             for (int u = u0; u <= u1; ++u) {
                 int32_t* cnt = w.counts + (u % 2) * n;
                 launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, cnt, w.status,
-                           u % 2 ? qb::kStTies1 : qb::kStTies0, 1, stream);
+                           u % 2 ? qb::kStTies1 : qb::kStTies0, 1, u == 0 ? w.sT : nullptr, stream);
                 if (u < max_iters)
                     qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(
                         w.sT, m, n, C, w.alpha, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, w.status, u, 1,
@@ -1033,6 +1153,8 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
         if (moves > 0) {
             const int64_t words = (m + 31) / 32;
             if ((ce = cudaMemsetAsync(w.mem, 0, sizeof(uint32_t) * (size_t)n * (size_t)words, stream)) != cudaSuccess)
+                goto cuda_fail;
+            if ((ce = cudaMemsetAsync(w.arc_tickets, 0, sizeof(int32_t) * (size_t)n, stream)) != cudaSuccess)
                 goto cuda_fail;
             qb_member_bits_kernel<<<(unsigned)((m * k + 255) / 256), 256, 0, stream>>>(topk_idx, m, k, words, w.mem);
             qb_all_rows_kernel<<<1, 256, 0, stream>>>(n, w.rows, w.nrows);

@@ -124,6 +124,8 @@ cap_count_scan_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg
                       int32_t* __restrict__ routed_count, int32_t* __restrict__ kept_count, int32_t* ticket) {
     __shared__ int cnt[kMaxExperts];
     __shared__ int s_last;
+    pdl_trigger();
+    pdl_wait();
     for (int e = threadIdx.x; e < n; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     int64_t seg, t0, t1;
@@ -151,6 +153,8 @@ cap_assign_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg_len
                   int32_t* __restrict__ slot, int32_t* __restrict__ dest_row, int32_t* __restrict__ src_token) {
     __shared__ int wcnt[cap::kWarps][kMaxExperts];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();
+    pdl_wait();
     for (int q = tid; q < cap::kWarps * kMaxExperts; q += cap::kThreads) (&wcnt[0][0])[q] = 0;
     __syncthreads();
     int64_t seg, t0, t1;
@@ -222,14 +226,13 @@ cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, in
         cudaError_t e = cudaMemsetAsync(ticket, 0, sizeof(int32_t), stream);
         if (e != cudaSuccess) return e;
     }
-    cap_count_scan_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(
-        topk_idx, k, n, seg_len, g.cps, g.nchunks, g.nseg, capacity, hist, prefix, seg_base, expert_offsets,
-        routed_count, kept_count, ticket);
-    {
-        cap_assign_kernel<<<(unsigned)g.nchunks, cap::kThreads, 0, stream>>>(
-            topk_idx, k, n, seg_len, g.cps, capacity, prefix, seg_base, slot, dest_row, src_token);
-    }
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(cap_count_scan_kernel, dim3((unsigned)g.nchunks), dim3(cap::kThreads), 0, stream,
+                               topk_idx, k, n, seg_len, g.cps, g.nchunks, g.nseg, capacity, hist, prefix, seg_base,
+                               expert_offsets, routed_count, kept_count, ticket);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(cap_assign_kernel, dim3((unsigned)g.nchunks), dim3(cap::kThreads), 0, stream, topk_idx, k, n,
+                      seg_len, g.cps, capacity, (const int32_t*)prefix, (const int32_t*)seg_base, slot, dest_row,
+                      src_token);
 }
 
 }  // namespace moe

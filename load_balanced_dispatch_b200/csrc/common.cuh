@@ -105,4 +105,28 @@ template <> struct Vec16<__nv_bfloat16> {
 
 __device__ __forceinline__ float round_to_bf16(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
+// Programmatic dependent launch. A kernel started with launch_pdl may begin while its predecessor
+// in the stream is still running: it calls pdl_wait() before it reads or writes any global memory
+// (pdl_wait returns once the predecessor grid has completed and its writes are visible), and
+// pdl_trigger() to let its own successor start early the same way. For a kernel launched without
+// the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace moe

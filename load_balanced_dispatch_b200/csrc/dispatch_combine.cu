@@ -26,6 +26,8 @@ static unsigned row_grid(int64_t rows) {
 __global__ void __launch_bounds__(kRowThreads)
 dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, const int32_t* __restrict__ src_token,
                 const int32_t* __restrict__ expert_offsets, int n, int64_t max_rows, uint4* __restrict__ xbuf) {
+    pdl_trigger();
+    pdl_wait();
     int64_t rows = expert_offsets[n];
     if (rows > max_rows) {
         if (blockIdx.x == 0 && threadIdx.x == 0) record_error(kErrRowOverflow);
@@ -65,6 +67,8 @@ combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row,
                const T* __restrict__ residual, int64_t m, int k, int d, int gate_bf16, T* __restrict__ y) {
     constexpr int V = Vec16<T>::N;
     const int lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();
     const int nvec = d / V;
     const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
     for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
@@ -105,25 +109,22 @@ cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const
                             const int32_t* expert_offsets, int n, int64_t max_rows, void* xbuf,
                             cudaStream_t stream) {
     const int64_t bytes_per_row = (int64_t)d * (dt == MOE_BF16 ? 2 : 4);
-    dispatch_kernel<<<row_grid(max_rows), kRowThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), m, bytes_per_row / 16, src_token, expert_offsets, n, max_rows,
-        static_cast<uint4*>(xbuf));
-    return cudaGetLastError();
+    return launch_pdl(dispatch_kernel, dim3(row_grid(max_rows)), dim3(kRowThreads), 0, stream,
+                      static_cast<const uint4*>(x), m, bytes_per_row / 16, src_token, expert_offsets, n, max_rows,
+                      static_cast<uint4*>(xbuf));
 }
 
 cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
                            const void* residual, int64_t m, int k, int d, void* y, cudaStream_t stream) {
     if (m == 0) return cudaSuccess;
     if (dt == MOE_BF16) {
-        combine_kernel<__nv_bfloat16><<<row_grid(m), kRowThreads, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(ybuf), dest_row, topk_gate,
-            static_cast<const __nv_bfloat16*>(residual), m, k, d, 1, static_cast<__nv_bfloat16*>(y));
-    } else {
-        combine_kernel<float><<<row_grid(m), kRowThreads, 0, stream>>>(
-            static_cast<const float*>(ybuf), dest_row, topk_gate, static_cast<const float*>(residual), m, k, d, 0,
-            static_cast<float*>(y));
+        return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(row_grid(m)), dim3(kRowThreads), 0, stream,
+                          static_cast<const __nv_bfloat16*>(ybuf), dest_row, topk_gate,
+                          static_cast<const __nv_bfloat16*>(residual), m, k, d, 1, static_cast<__nv_bfloat16*>(y));
     }
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<float>, dim3(row_grid(m)), dim3(kRowThreads), 0, stream,
+                      static_cast<const float*>(ybuf), dest_row, topk_gate, static_cast<const float*>(residual), m, k,
+                      d, 0, static_cast<float*>(y));
 }
 
 }  // namespace moe

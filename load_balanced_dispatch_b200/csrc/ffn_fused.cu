@@ -26,6 +26,11 @@
 // an expert's end are computed and masked; column and K tails are TMA zero
 // fill. Every wait is bounded (about 2 s), after which the device error word
 // and an abort flag are set and all roles leave their loops.
+//
+// With one pick per token (k = 1) the GEMM2 epilogue can also do the gated
+// combine (moe_expert_ffn_combine): each output row is written, gated, to its
+// token's row of y, so ybuf and the combine launch disappear; the few dropped
+// tokens get their residual (or zeros) from combine_dropped_kernel.
 #include "groups.cuh"
 #include "tc_ptx.cuh"
 
@@ -52,6 +57,19 @@ struct FusedShared {
 };
 
 constexpr size_t fused_smem_bytes() { return 1024 + (size_t)fz::STAGES * fz::STAGE_BYTES + sizeof(FusedShared); }
+
+// The gated combine for one pick per token (k = 1), done by the GEMM2 epilogue: row r of the
+// expert-major output belongs to token src_token[r] alone, so the epilogue writes
+// y[token] = bf16(fma(bf16(gate[token]), bf16(out_r), residual[token] or 0)) -- the same
+// operations, in the same order, as the combine kernel applied to ybuf. y == nullptr: the
+// epilogue writes ybuf instead.
+struct FusedCombine {
+    const int32_t* src_token;
+    const float* gate;                 // [m] (k = 1)
+    const __nv_bfloat16* residual;     // [m, d] or nullptr
+    __nv_bfloat16* y;                  // [m, d] or nullptr
+    int64_t m;
+};
 
 struct FusedTile {
     int phase, e, n0, N, K, mtiles1;
@@ -83,7 +101,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
              const __nv_bfloat16* __restrict__ b1, const __nv_bfloat16* __restrict__ b2,
              const int32_t* __restrict__ offsets, int n, int d, int d_ff, int64_t max_rows,
              __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ y, int* __restrict__ done1,
-             int* __restrict__ next_tile) {
+             int* __restrict__ next_tile, FusedCombine cmb) {
     using namespace fz;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -103,6 +121,8 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         ptx::prefetch_tensormap(&map_w2);
     }
     if (warp == 1) ptx::tmem_alloc(&sh->tmem_base, TMEM_COLS);
+    pdl_trigger();
+    pdl_wait();  // expert_offsets, xbuf and the counters come from earlier launches
     if (warp == 2) build_group_table(offsets, n, ntn1, BM, max_rows, sh->g1);
     if (warp == 3) build_group_table(offsets, n, ntn2, BM, max_rows, sh->g2);
     ptx::tc_fence_before();
@@ -215,14 +235,37 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
             if (!ptx::mbar_wait(&sh->tfull[acc], aphase, abort_flag)) break;
             ptx::tc_fence_after();
             const int64_t r = t.row0 + quad * 32 + lane;
-            const bool row_ok = r < t.row_end;
+            bool row_ok = r < t.row_end;
             const bool relu = t.phase == 1;
             __nv_bfloat16* out = t.phase == 1 ? h : y;
-            for (int c = 0; c < BN / 32; ++c) {
-                const int col0 = t.n0 + c * 32;
-                if (col0 >= t.N) break;  // warp-uniform
-                uint32_t v[32];
-                ptx::tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
+            // combined output: this row goes straight to its token's row of y, scaled by its gate
+            const bool comb = t.phase == 2 && cmb.y != nullptr;
+            int64_t tok = 0;
+            float gk = 0.f;
+            if (comb && row_ok) {
+                tok = cmb.src_token[r];
+                if (tok < 0 || tok >= cmb.m) {
+                    record_error(kErrTokenIndex);
+                    row_ok = false;
+                } else {
+                    gk = round_to_bf16(cmb.gate[tok]);
+                }
+            }
+            // two 32-column chunks in flight per wait
+            for (int c2 = 0; c2 < BN / 32; c2 += 2) {
+                const int colA = t.n0 + c2 * 32;
+                if (colA >= t.N) break;  // warp-uniform
+                const bool hasB = colA + 32 < t.N;
+                uint32_t v2[2][32];
+                const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN + c2 * 32);
+                ptx::tmem_ld32_issue(tbase, v2[0]);
+                if (hasB) ptx::tmem_ld32_issue(tbase + 32, v2[1]);
+                ptx::tmem_wait_ld();
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                if (half == 1 && !hasB) break;
+                const int col0 = colA + half * 32;
+                const uint32_t (&v)[32] = v2[half];
 #pragma unroll
                 for (int g8 = 0; g8 < 4; ++g8) {
                     const int col = col0 + g8 * 8;
@@ -234,8 +277,23 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                         f[q] = __uint_as_float(v[g8 * 8 + q]) + bv[q];
                         if (relu) f[q] = fmaxf(f[q], 0.f);
                     }
-                    if (row_ok) Vec16<__nv_bfloat16>::store(out + r * t.N + col, f);
+                    if (!row_ok) continue;
+                    if (comb) {
+                        float acc[8];
+                        if (cmb.residual) {
+                            Vec16<__nv_bfloat16>::load(cmb.residual + tok * t.N + col, acc);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[q] = fmaf(gk, round_to_bf16(f[q]), acc[q]);
+                        Vec16<__nv_bfloat16>::store(cmb.y + tok * t.N + col, acc);
+                    } else {
+                        Vec16<__nv_bfloat16>::store(out + r * t.N + col, f);
+                    }
                 }
+              }
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&sh->tempty[acc]);
@@ -259,9 +317,41 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     }
 }
 
+// y rows of tokens whose pick was dropped (k = 1, dest_row < 0): the residual, or zeros.
+__global__ void __launch_bounds__(256)
+combine_dropped_kernel(const int32_t* __restrict__ dest_row, const uint4* __restrict__ residual, int64_t m,
+                       int64_t vec_per_row, uint4* __restrict__ y) {
+    const int lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    for (int64_t i0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * 32; i0 < m; i0 += warps * 32) {
+        const int64_t i = i0 + lane;
+        const bool dropped = i < m && dest_row[i] < 0;
+        uint32_t mask = __ballot_sync(0xffffffffu, dropped);
+        while (mask) {  // the warp copies (or clears) each dropped row of its 32 tokens
+            const int b = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int64_t tok = i0 + b;
+            for (int64_t c = lane; c < vec_per_row; c += 32)
+                y[tok * vec_per_row + c] = residual ? residual[tok * vec_per_row + c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+cudaError_t launch_combine_dropped(const int32_t* dest_row, const void* residual, int64_t m, int d, void* y,
+                                   cudaStream_t stream) {
+    if (m == 0) return cudaSuccess;
+    int64_t blocks = (m + 255) / 256;
+    if (blocks > (int64_t)num_sms() * 4) blocks = (int64_t)num_sms() * 4;
+    return launch_pdl(combine_dropped_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, dest_row,
+                      static_cast<const uint4*>(residual), m, (int64_t)d * 2 / 16, static_cast<uint4*>(y));
+}
+
 cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
                              const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
-                             int* counters, cudaStream_t stream) {
+                             int* counters, cudaStream_t stream, const FusedCombine* cmb = nullptr,
+                             bool zero_counters = true) {
     CUtensorMap mx, mw1, mh, mw2;
     if (!map_2d(&mx, xbuf, (uint64_t)max_rows, (uint64_t)d, fz::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw1, w1, (uint64_t)n, (uint64_t)d_ff, (uint64_t)d, fz::BN)) return cudaErrorInvalidValue;
@@ -275,13 +365,46 @@ cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, c
         attr = true;
     }
     // counters[0..n-1]: GEMM1 completions per expert; counters[n]: next tile ticket
-    cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
-    if (e != cudaSuccess) return e;
-    ffn_fused_tc<<<num_sms(), fz::kThreads, smem, stream>>>(
-        mx, mw1, mh, mw2, static_cast<const __nv_bfloat16*>(b1), static_cast<const __nv_bfloat16*>(b2), offsets, n,
-        d, d_ff, max_rows, static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), counters,
-        counters + n);
-    return cudaGetLastError();
+    if (zero_counters) {
+        cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(ffn_fused_tc, dim3(num_sms()), dim3(fz::kThreads), smem, stream, mx, mw1, mh, mw2,
+                      static_cast<const __nv_bfloat16*>(b1), static_cast<const __nv_bfloat16*>(b2), offsets, n, d,
+                      d_ff, max_rows, static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), counters,
+                      counters + n, cmb ? *cmb : FusedCombine{nullptr, nullptr, nullptr, nullptr, 0});
+}
+
+// Both GEMMs in one persistent launch; its counters (per-expert completions, tile ticket) follow h.
+static int* ffn_counters(void* hbuf, int64_t max_rows, int d_ff) {
+    const size_t hbytes = ((size_t)max_rows * (size_t)d_ff * 2 + 255) & ~(size_t)255;
+    return reinterpret_cast<int*>(static_cast<char*>(hbuf) + hbytes);
+}
+
+cudaError_t launch_ffn_tc(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
+                          const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
+                          cudaStream_t stream) {
+    return launch_ffn_fused(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf,
+                            ffn_counters(hbuf, max_rows, d_ff), stream);
+}
+
+// The FFN with the k = 1 gated combine in its GEMM2 epilogue, plus the dropped tokens' rows.
+cudaError_t launch_ffn_tc_combine(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
+                                  const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* hbuf,
+                                  const int32_t* src_token, const int32_t* dest_row, const float* gate,
+                                  const void* residual, int64_t m, void* y, cudaStream_t stream) {
+    // counters first, so that the FFN directly follows a kernel (programmatic dependent launch)
+    int* counters = ffn_counters(hbuf, max_rows, d_ff);
+    if (max_rows > 0) {
+        cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_combine_dropped(dest_row, residual, m, d, y, stream);
+    if (e != cudaSuccess || max_rows == 0) return e;
+    const FusedCombine cmb{src_token, gate, static_cast<const __nv_bfloat16*>(residual),
+                           static_cast<__nv_bfloat16*>(y), m};
+    return launch_ffn_fused(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, nullptr, hbuf, counters, stream,
+                            &cmb, false);
 }
 
 }  // namespace moe

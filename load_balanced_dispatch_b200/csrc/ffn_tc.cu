@@ -59,17 +59,4 @@ static int num_sms() {
     return sms;
 }
 
-cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
-                             const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
-                             int* counters, cudaStream_t stream);
-
-// Both GEMMs in one persistent launch; its counters (per-expert completions, tile ticket) follow h.
-cudaError_t launch_ffn_tc(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
-                          const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
-                          cudaStream_t stream) {
-    const size_t hbytes = ((size_t)max_rows * (size_t)d_ff * 2 + 255) & ~(size_t)255;
-    int* done1 = reinterpret_cast<int*>(static_cast<char*>(hbuf) + hbytes);
-    return launch_ffn_fused(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf, done1, stream);
-}
-
 }  // namespace moe

@@ -207,6 +207,8 @@ __global__ void __launch_bounds__(kFinishThreads)
 router_finish_kernel(const float* h, int64_t m, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
                      float* probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
     const int lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();
     const int64_t warps = (int64_t)gridDim.x * (kFinishThreads / 32);
     for (int64_t row = (int64_t)blockIdx.x * (kFinishThreads / 32) + (threadIdx.x >> 5); row < m; row += warps) {
         float hv[NT];
@@ -224,13 +226,13 @@ cudaError_t launch_router_finish(const float* h, int64_t m, int n, int k, int fn
     const int64_t cap = (int64_t)kNumSMs * 8;
     if (blocks > cap) blocks = cap;
     if (n <= 32)
-        router_finish_kernel<1><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+        return launch_pdl(router_finish_kernel<1>, dim3((unsigned)blocks), dim3(kFinishThreads), 0, stream, h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
     else if (n <= 64)
-        router_finish_kernel<2><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+        return launch_pdl(router_finish_kernel<2>, dim3((unsigned)blocks), dim3(kFinishThreads), 0, stream, h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
     else if (n <= 128)
-        router_finish_kernel<4><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+        return launch_pdl(router_finish_kernel<4>, dim3((unsigned)blocks), dim3(kFinishThreads), 0, stream, h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
     else
-        router_finish_kernel<8><<<(unsigned)blocks, kFinishThreads, 0, stream>>>(h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+        return launch_pdl(router_finish_kernel<8>, dim3((unsigned)blocks), dim3(kFinishThreads), 0, stream, h, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
     return cudaGetLastError();
 }
 

@@ -55,6 +55,8 @@ inline size_t router_tc_smem(int np, int stages) {
 // W_r [d, n] fp32 -> out [3, n, d] bf16 with w = out[0] + out[1] + out[2] (32x32 tiles through shared memory).
 __global__ void router_split_kernel(const float* __restrict__ w_r, int d, int n, __nv_bfloat16* __restrict__ out) {
     __shared__ float tile[32][33];
+    pdl_trigger();
+    pdl_wait();
     const int t0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
     const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
     for (int r = ty; r < 32; r += 8) {
@@ -258,6 +260,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
+    pdl_trigger();
+    pdl_wait();  // the W split and x come from earlier launches
     const uint32_t tmem = sh->tmem_base;
     volatile int* abort_flag = &sh->abort_flag;
     bool drain_ok = true;  // this drain thread received every K block
@@ -313,13 +317,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
         for (int kb = 0; kb < nkb; ++kb) {
             if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { drain_ok = false; break; }
             ptx::tc_fence_after();
+            // every column chunk of the block in flight at once, one wait
+            uint32_t v[NCH][32];
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) {
-                uint32_t v[32];
-                ptx::tmem_ld32(trow + (uint32_t)(buf * NP + c * 32), v);
+            for (int c = 0; c < NCH; ++c) ptx::tmem_ld32_issue(trow + (uint32_t)(buf * NP + c * 32), v[c]);
+            ptx::tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 32; ++q) acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[q]));
-            }
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int q = 0; q < 32; ++q) acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[c][q]));
             ptx::tc_fence_before();
             ptx::mbar_arrive(&sh->tempty[buf]);
             if (++buf == 2) { buf = 0; bphase ^= 1u; }
@@ -390,15 +396,18 @@ static cudaError_t launch_router_tc_st(const CUtensorMap& mx, const CUtensorMap&
     cfg.blockDim = dim3(rtc::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
     if (mode == rtc::kModeFused && grid.y == 2) {
         // the two column tiles of the same 128 tokens form a cluster (exchange through DSMEM)
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = 1;
-        at[0].val.clusterDim.y = 2;
-        at[0].val.clusterDim.z = 1;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
+        at[1].id = cudaLaunchAttributeClusterDimension;
+        at[1].val.clusterDim.x = 1;
+        at[1].val.clusterDim.y = 2;
+        at[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     }
     return cudaLaunchKernelEx(&cfg, router_tc_kernel<NCH, ST>, mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out,
                               topk_idx, topk_gate, mode);
@@ -434,7 +443,8 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, 
     __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(workspace);
     {
         dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
-        router_split_kernel<<<tg, tb, 0, stream>>>(w_r, d, n, wsplit);
+        const cudaError_t e = launch_pdl(router_split_kernel, tg, tb, 0, stream, w_r, d, n, wsplit);
+        if (e != cudaSuccess) return e;
     }
     // With probs_out the logits go to memory in 64-wide column tiles and router_finish_kernel (a
     // warp per row, the whole GPU) finishes them in place: measured faster than finishing in this

@@ -181,6 +181,8 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
     __shared__ double sh[stats::kThreads / 32];
     __shared__ int s_last;
     const int tid = threadIdx.x;
+    pdl_trigger();
+    pdl_wait();
     const int64_t chunk = blockIdx.x;
     const int64_t seg = chunk / cps, c = chunk - seg * cps;
     const int64_t r0 = seg * seg_len + c * stats::kRows;
@@ -327,10 +329,8 @@ cudaError_t launch_stats(const float* probs, const int32_t* topk_idx, int64_t m,
     stats_layout(m, n, seg_len, &w, static_cast<char*>(workspace));
     cudaError_t e = cudaMemsetAsync(w.tickets, 0, sizeof(int32_t) * (size_t)(g.nseg + 1), stream);
     if (e != cudaSuccess) return e;
-    stats_kernel<<<(unsigned)g.nchunks, stats::kThreads, 0, stream>>>(probs, topk_idx, m, n, k, seg_len, g.cps,
-                                                                      g.nseg, alpha, f, P, aux, vio, bias, gamma, w,
-                                                                      totals);
-    return cudaGetLastError();
+    return launch_pdl(stats_kernel, dim3((unsigned)g.nchunks), dim3(stats::kThreads), 0, stream, probs, topk_idx, m,
+                      n, k, seg_len, g.cps, g.nseg, alpha, f, P, aux, vio, bias, gamma, w, totals);
 }
 
 cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, int k, int has_probs, float alpha,

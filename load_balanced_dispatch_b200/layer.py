@@ -12,7 +12,8 @@ from dataclasses import dataclass
 import torch
 
 from . import (MOE_QB_MIDPOINT, MOE_QB_STEP, MOE_SIGMOID, MOE_SOFTMAX, moe_balance_assign, moe_balance_stats,
-               moe_capacity_slots, moe_combine, moe_dispatch, moe_expert_ffn, moe_router_topk, lib)
+               moe_capacity_slots, moe_combine, moe_dispatch, moe_expert_ffn, moe_expert_ffn_combine,
+               moe_router_topk, lib)
 
 
 @dataclass
@@ -76,6 +77,8 @@ class MoELayer:
             stats=torch.empty((max(L.moe_balance_stats_workspace_size(m, n, seg), 1),), dtype=torch.uint8,
                               device=dev),
         )
+        # one pick per token in bf16: the combine runs in the FFN's second GEMM (moe_expert_ffn_combine)
+        self.ffn_combine = s.k == 1 and s.dtype == torch.bfloat16
         # data-parallel replicas: set by enable_global_stats(); the Loss-Free bias then follows the
         # pooled counts of every rank instead of this rank's
         self.global_stats = None
@@ -94,11 +97,18 @@ class MoELayer:
         elif i == 2:
             moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
         elif i == 3:
-            moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"], ybuf=b["ybuf"],
-                           workspace=self.ws["ffn"], stream=st)
+            if self.ffn_combine:
+                moe_expert_ffn_combine(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"],
+                                       b["src_token"], b["dest_row"], b["topk_gate"],
+                                       residual=x if s.residual else None, y=b["y"], workspace=self.ws["ffn"],
+                                       stream=st)
+            else:
+                moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"], ybuf=b["ybuf"],
+                               workspace=self.ws["ffn"], stream=st)
         elif i == 4:
-            moe_combine(b["ybuf"], b["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
-                        stream=st)
+            if not self.ffn_combine:  # otherwise done by the FFN's second GEMM
+                moe_combine(b["ybuf"], b["dest_row"], b["topk_gate"], residual=x if s.residual else None, y=b["y"],
+                            stream=st)
         else:
             local_bias = s.lossfree and self.global_stats is None
             moe_balance_stats(b["probs"], b["topk_idx"], s.n, self.seg_len, s.alpha,
@@ -138,6 +148,9 @@ class MoELayer:
         torch.cuda.synchronize()
         self.graphs = []
         for i in range(len(self.STAGES)):
+            if i == 4 and self.ffn_combine:  # nothing to launch: the combine ran in the FFN stage
+                self.graphs.append(None)
+                continue
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 self._stage(i, x, torch.cuda.current_stream())
@@ -156,7 +169,8 @@ class MoELayer:
             return self.buf["y"]
         for i, g in enumerate(self.graphs):
             events[i].record(st)
-            g.replay()
+            if g is not None:
+                g.replay()
         events[len(self.graphs)].record(st)
         return self.buf["y"]
 
@@ -190,11 +204,14 @@ class MoELayer:
         """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection
         and the finish kernel; else 1),
         capacity 2 (count + scan, assign), dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
-        combine 1, statistics 1."""
+        combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus one
+        launch for the dropped tokens' rows."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
         router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
         ffn = 1 if bf16 else 2
+        if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped tokens' rows
+            return router + 2 + 1 + 2 + 0 + 1
         return router + 2 + 1 + ffn + 1 + 1
 
 

@@ -20,7 +20,7 @@ _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
 SOFTMAX, SIGMOID = 0, 1
 QB_STEP, QB_SOLVE = 0, 1
-QB_MIDPOINT, QB_BOUNDARY = 0, 1
+QB_MIDPOINT, QB_BOUNDARY, QB_BIP = 0, 1, 2
 OK, ERR_ARG, ERR_NOT_CONVERGED, ERR_INTERNAL = 0, 1, 5, 6
 
 
@@ -57,6 +57,7 @@ def lib():
         _lib.orc_qb_col.argtypes = [P, L, I, L, P, I, P]
         _lib.orc_qb_col.restype = None
         _lib.orc_is_optimal.argtypes = [P, L, I, P, I, D]
+        _lib.orc_qb_sign_step.argtypes = [P, L, I, I, P, F, I, P, P]
     return _lib
 
 
@@ -164,6 +165,19 @@ def balance_assign(s, k, beta=None, mode=QB_SOLVE, rule=QB_MIDPOINT, max_iters=6
     if check and rc not in (OK, ERR_NOT_CONVERGED):
         raise OracleError("orc_balance_assign", rc)
     return idx, beta, info, rc
+
+
+def qb_sign_step(s, k, beta, gamma, rule=QB_MIDPOINT):
+    """One SignSGD-on-beta step: returns (topk_idx [m,k] ascending experts, beta_out [n] f32, info [4])."""
+    s = _f32(s)
+    m, n = s.shape
+    beta = np.array(beta, dtype=np.float32, copy=True)
+    idx = np.empty((m, k), np.int32)
+    info = np.zeros(4, np.int32)
+    rc = lib().orc_qb_sign_step(_p(s), m, n, k, _p(beta), np.float32(gamma), rule, _p(idx), _p(info))
+    if rc:
+        raise OracleError("orc_qb_sign_step", rc)
+    return idx, beta, info
 
 
 def qb_row(s, k, beta, rule=QB_MIDPOINT):

@@ -49,6 +49,7 @@
 #define ORC_QB_SOLVE 1
 #define ORC_QB_MIDPOINT 0
 #define ORC_QB_BOUNDARY 1
+#define ORC_QB_BIP 2
 
 /* Ranking order used everywhere: larger key first, equal keys -> lower index first. */
 static int ranks_before(double ka, int ia, double kb, int ib) {
@@ -364,10 +365,13 @@ static int cmp_desc(const void* pa, const void* pb) {
     return (a->i < b->i) ? -1 : (a->i > b->i);
 }
 
-/* Threshold between the q-th and (q+1)-th largest of a list sorted descending (q counted from 1). */
+/* Threshold between the q-th and (q+1)-th largest of a list sorted descending (q counted from 1).
+ * BIP ([QB], "Related work", the inequality-constrained problem (12)-(14)): the (q+1)-th value
+ * clipped at zero, max(0, b), since its duals must stay non-negative. */
 static float threshold_of(const orc_kv* sorted, int64_t q, int rule) {
     float a = sorted[q - 1].v, b = sorted[q].v;
     if (rule == ORC_QB_BOUNDARY) return b;
+    if (rule == ORC_QB_BIP) return b > 0.0f ? b : 0.0f;
     volatile float sum = a + b;
     volatile float half = sum * 0.5f;
     return half;
@@ -531,7 +535,7 @@ int orc_balance_assign(const float* s, int64_t m, int n, int k, float* beta_inou
                        int max_iters, int max_repair, int32_t* topk_idx, int32_t* info) {
     if (n < 2 || k < 1 || k >= n || m < 1 || ((m * k) % n) != 0) return ORC_ERR_ARG;
     if (mode != ORC_QB_STEP && mode != ORC_QB_SOLVE) return ORC_ERR_ARG;
-    if (rule != ORC_QB_MIDPOINT && rule != ORC_QB_BOUNDARY) return ORC_ERR_ARG;
+    if (rule != ORC_QB_MIDPOINT && rule != ORC_QB_BOUNDARY && rule != ORC_QB_BIP) return ORC_ERR_ARG;
     int64_t C = m * k / n;
     float* alpha = (float*)malloc(sizeof(float) * (size_t)m);
     unsigned char* X = (unsigned char*)malloc((size_t)m * n);
@@ -569,6 +573,48 @@ int orc_balance_assign(const float* s, int64_t m, int n, int k, float* beta_inou
     if (info) { info[0] = iters; info[1] = augments; info[2] = (int32_t)excess; info[3] = (int32_t)ties; }
     free(alpha); free(X); free(cnt); free(buf);
     return status;
+}
+
+/*
+ * SignSGD on beta ([QB], "Gradient descent", eqs. (15)-(17)): with alpha from the row pass, the
+ * loss l(beta) = sum_ij max(0, s_ij - alpha_i - beta_j) + (m k / n) sum_j beta_j has
+ *   dl/dbeta_j = m k / n - sum_i chi(s_ij - alpha_i - beta_j > 0),
+ * and the step is beta_j <- beta_j - gamma sign(dl/dbeta_j), used in place of the quantile
+ * update. One step: the row pass selects the top-k of s - beta (old beta) and sets alpha by
+ * `rule`; then count_j = #{i : fp32(s_ij - alpha_i) > beta_j} (the sign of the second fp32
+ * subtraction is that of the exact difference, so this is the indicator as written; sign(0) = 0
+ * leaves beta_j unchanged) and beta_j moves by gamma with one fp32 add or subtract.
+ * topk_idx / info as orc_balance_assign's STEP.
+ */
+int orc_qb_sign_step(const float* s, int64_t m, int n, int k, float* beta_inout, float gamma, int rule,
+                     int32_t* topk_idx, int32_t* info) {
+    if (n < 2 || k < 1 || k >= n || m < 1 || ((m * k) % n) != 0) return ORC_ERR_ARG;
+    if (rule != ORC_QB_MIDPOINT && rule != ORC_QB_BOUNDARY && rule != ORC_QB_BIP) return ORC_ERR_ARG;
+    const int64_t C = m * k / n;
+    float* alpha = (float*)malloc(sizeof(float) * (size_t)m);
+    unsigned char* X = (unsigned char*)malloc((size_t)m * n);
+    int64_t* cnt = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
+    orc_kv* buf = (orc_kv*)malloc(sizeof(orc_kv) * (size_t)n);
+    int64_t ties = 0;
+    qb_row_pass(s, m, n, k, beta_inout, rule, alpha, X, cnt, &ties, buf);
+    int64_t excess = 0;
+    for (int e = 0; e < n; ++e) if (cnt[e] > C) excess += cnt[e] - C;
+    for (int j = 0; j < n; ++j) {
+        int64_t c = 0;
+        for (int64_t i = 0; i < m; ++i) {
+            volatile float u = s[i * n + j] - alpha[i];
+            if (u > beta_inout[j]) c++;
+        }
+        if (c > C) beta_inout[j] = add_f32(beta_inout[j], gamma);        /* gradient < 0 */
+        else if (c < C) beta_inout[j] = add_f32(beta_inout[j], -gamma);  /* gradient > 0 */
+    }
+    for (int64_t i = 0; i < m; ++i) {
+        int r = 0;
+        for (int j = 0; j < n; ++j) if (X[i * n + j]) topk_idx[i * k + (r++)] = j;
+    }
+    if (info) { info[0] = 1; info[1] = 0; info[2] = (int32_t)excess; info[3] = (int32_t)ties; }
+    free(alpha); free(X); free(cnt); free(buf);
+    return ORC_OK;
 }
 
 /* One QB row pass alone: alpha_i, the top-k of s_i - beta (best first) and the per-expert counts. */

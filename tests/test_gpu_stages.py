@@ -192,6 +192,35 @@ def test_expert_ffn(dtype, rows_per, d, d_ff):
     assert norm_err(host(ybuf)[:rows], ref) <= tol(dtype)
 
 
+@pytest.mark.parametrize("m,n,d,d_ff,cap", [(2048, 16, 768, 3072, 150), (1000, 8, 256, 512, 100),
+                                            (513, 5, 2048, 1408, 1000), (300, 4, 256, 256, 0)])
+def test_expert_ffn_combine_matches_two_calls(m, n, d, d_ff, cap):
+    # k = 1: the FFN's second GEMM writes the gated combine straight into y. Bit for bit the
+    # result of moe_expert_ffn followed by moe_combine, with and without the residual; capacity
+    # 0 drops every token (no FFN rows at all)
+    rng = np.random.default_rng(m + d)
+    x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
+    idx = W.make_topk_idx(m, n, 1, seed=4, skew=1.5)
+    gate = rng.random((m, 1)).astype(np.float32)
+    w1 = W.round_to_bf16((rng.standard_normal((n, d_ff, d)) / np.sqrt(d)).astype(np.float32))
+    b1 = W.round_to_bf16((0.1 * rng.standard_normal((n, d_ff))).astype(np.float32))
+    w2 = W.round_to_bf16((rng.standard_normal((n, d, d_ff)) / np.sqrt(d_ff)).astype(np.float32))
+    b2 = W.round_to_bf16((0.1 * rng.standard_normal((n, d))).astype(np.float32))
+    bf = torch.bfloat16
+    xd = dev(x, bf)
+    out = lb.moe_capacity_slots(dev(idx), n, cap)
+    xbuf = lb.moe_dispatch(xd, out["src_token"], out["expert_offsets"], n, m)
+    wd = [dev(a, bf) for a in (w1, b1, w2, b2)]
+    ybuf = lb.moe_expert_ffn(xbuf, *wd, out["expert_offsets"])
+    for residual in (None, xd):
+        y2 = lb.moe_combine(ybuf, out["dest_row"], dev(gate), residual=residual)
+        y1 = lb.moe_expert_ffn_combine(xbuf, *wd, out["expert_offsets"], out["src_token"], out["dest_row"],
+                                       dev(gate), residual=residual)
+        torch.cuda.synchronize()
+        lb.sync_status()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
 # ---------------------------------------------------------------- statistics
 @pytest.mark.parametrize("m,n,k,seg", [(8192, 128, 1, 8192), (65536, 64, 2, 4096), (1000, 8, 1, 250),
                                        (777, 256, 8, 777)])
@@ -296,6 +325,50 @@ def test_balance_step_heavy_ties(m, n, k):
         torch.cuda.synchronize()
         assert (host(idx) == i_ref).all()
         assert (host(beta) == b_ref).all()
+        b = b_ref
+
+
+@pytest.mark.parametrize("m,n,k,shift", [(4096, 32, 4, 0.0), (2048, 16, 2, -1.0), (65536, 256, 8, 0.0),
+                                         (1002, 6, 3, 2.0)])
+def test_balance_bip_steps_bitexact(m, n, k, shift):
+    # BIP thresholds (the (k+1)-th / (C+1)-th values clipped at zero), three chained STEPs
+    s = W.make_qb_scores(m, n, seed=m + n) + np.float32(shift)
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(3):
+        i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=b, mode=oracle.QB_STEP, rule=oracle.QB_BIP)
+        idx, beta, info = lb.moe_balance_assign(dev(s), k, beta=dev(b), mode=lb.MOE_QB_STEP, rule=lb.MOE_QB_BIP)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(beta) == b_ref).all()
+        assert (host(info) == info_ref).all()
+        b = b_ref
+
+
+def test_balance_bip_solve_bitexact():
+    s = W.make_qb_scores(2048, 16, seed=9)
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, 2, mode=oracle.QB_SOLVE, rule=oracle.QB_BIP, max_iters=12)
+    assert rc == oracle.OK
+    idx, beta, info = lb.moe_balance_assign(dev(s), 2, mode=lb.MOE_QB_SOLVE, rule=lb.MOE_QB_BIP, max_iters=12)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
+
+
+@pytest.mark.parametrize("m,n,k,gamma,rule", [(4096, 32, 4, 0.05, 0), (65536, 256, 8, 0.01, 0), (1002, 6, 3, 0.1, 1),
+                                              (2048, 16, 2, 0.02, 2)])
+def test_balance_sign_steps_bitexact(m, n, k, gamma, rule):
+    # SignSGD on beta: five chained steps, picks, beta and info identical to the oracle
+    s = W.make_qb_scores(m, n, seed=m * 5 + n)
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(5):
+        i_ref, b_ref, info_ref = oracle.qb_sign_step(s, k, b, gamma, rule=rule)
+        bd = dev(b)
+        idx, _, info = lb.moe_balance_sign_step(dev(s), k, bd, gamma, rule=rule)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(bd) == b_ref).all()
+        assert (host(info) == info_ref).all()
         b = b_ref
 
 

@@ -217,3 +217,87 @@ def test_argument_errors():
         oracle.balance_assign(s, 1)  # m*k = 10 not divisible by n = 4
     with pytest.raises(oracle.OracleError):
         oracle.balance_assign(W.make_qb_scores(8, 4), 4)  # k must be < n
+
+
+# ---------------------------------------------------------------- balancing variants
+# "MoE travelogue 6", Related work (BIP: inequality constraints, duals clipped at zero) and
+# Gradient descent (SignSGD on beta, eqs. (15)-(17)).
+
+def test_bip_hand_example():
+    # m=4, n=2, k=1, C=2. Tokens 0, 1 prefer expert 0; tokens 2, 3 prefer expert 1.
+    # All scores negative: alpha_i = max(0, 2nd value) = 0, u = s, and each column's 3rd largest
+    # value is negative, so beta = max(0, .) = 0 for both experts.
+    s = np.array([[3, 1], [2, 0], [1, 4], [0, 5]], np.float32) - 10
+    alpha, idx, _ = oracle.qb_row(s, 1, np.zeros(2, np.float32), rule=oracle.QB_BIP)
+    assert (alpha == 0).all() and idx[:, 0].tolist() == [0, 0, 1, 1]
+    assert (oracle.qb_col(s, 1, alpha, rule=oracle.QB_BIP) == 0).all()
+    # shifted up by 20 (scores [[13, 11], [12, 10], [11, 14], [10, 15]]) the clip is inactive on
+    # alpha: the 2nd values 11, 10, 11, 10; column 0 of s - alpha is [2, 2, 0, 0] and column 1 is
+    # [0, 0, 3, 5]: both 3rd largest values are 0
+    alpha, _, _ = oracle.qb_row(s + 20, 1, np.zeros(2, np.float32), rule=oracle.QB_BIP)
+    assert alpha.tolist() == [11, 10, 11, 10]
+    assert oracle.qb_col(s + 20, 1, alpha, rule=oracle.QB_BIP).tolist() == [0.0, 0.0]
+
+
+def test_bip_equals_boundary_when_thresholds_are_positive():
+    # the clip max(0, .) only acts on negative thresholds: where the (k+1)-th / (C+1)-th values
+    # are positive (scores far above zero, alpha = 0 for the column pass) BIP is the page's
+    # boundary rule exactly; where they are negative it returns 0
+    s = W.make_qb_scores(2048, 16, seed=3) + np.float32(50)
+    b0 = np.zeros(16, np.float32)
+    a_b, i_b, _ = oracle.qb_row(s, 2, b0, rule=oracle.QB_BOUNDARY)
+    a_p, i_p, _ = oracle.qb_row(s, 2, b0, rule=oracle.QB_BIP)
+    assert (a_b > 0).all() and (a_b == a_p).all() and (i_b == i_p).all()
+    zero = np.zeros(2048, np.float32)
+    beta_b = oracle.qb_col(s, 2, zero, rule=oracle.QB_BOUNDARY)
+    assert (beta_b > 0).all() and (oracle.qb_col(s, 2, zero, rule=oracle.QB_BIP) == beta_b).all()
+    assert (oracle.qb_col(s - 100, 2, zero, rule=oracle.QB_BIP) == 0).all()
+    assert (oracle.qb_row(s - 100, 2, b0, rule=oracle.QB_BIP)[0] == 0).all()
+
+
+def test_bip_duals_never_negative():
+    s = W.make_qb_scores(3000, 24, seed=5) - np.float32(1.0)
+    beta = np.zeros(24, np.float32)
+    for _ in range(4):
+        _, beta, _, _ = oracle.balance_assign(s, 3, beta=beta, mode=oracle.QB_STEP, rule=oracle.QB_BIP)
+        assert (beta >= 0).all()
+        alpha, _, _ = oracle.qb_row(s, 3, beta, rule=oracle.QB_BIP)
+        assert (alpha >= 0).all()
+
+
+def test_sign_step_hand_example():
+    # m=4, n=2, k=1, C=2: tokens 0-2 prefer expert 0 (s = [1, 0]), token 3 expert 1 (s = [0, 1]).
+    # MIDPOINT alpha_i = 0.5 for every token. count_0 = #{s_i0 - 0.5 > 0} = 3 > C: the gradient
+    # C - 3 < 0, so beta_0 rises by gamma; count_1 = 1 < C: beta_1 falls by gamma.
+    s = np.array([[1, 0], [1, 0], [1, 0], [0, 1]], np.float32)
+    idx, beta, info = oracle.qb_sign_step(s, 1, np.zeros(2, np.float32), 0.125)
+    assert idx[:, 0].tolist() == [0, 0, 0, 1]
+    assert beta.tolist() == [0.125, -0.125]
+    assert info.tolist() == [1, 0, 1, 0]  # one update, no repair, excess 1, no ties
+    # balanced selection: both counts equal C, sign(0) = 0, beta unchanged
+    s2 = np.array([[1, 0], [1, 0], [0, 1], [0, 1]], np.float32)
+    _, beta2, info2 = oracle.qb_sign_step(s2, 1, np.array([0.25, -0.5], np.float32), 0.125)
+    assert beta2.tolist() == [0.25, -0.5] and info2[2] == 0
+
+
+def test_sign_steps_shrink_the_violation():
+    # repeated SignSGD steps move load from the crowded experts to the empty ones (the page puts
+    # its effect between Loss-Free and QB)
+    m, n, k = 4096, 16, 2
+    s = W.make_qb_scores(m, n, seed=7, skew_std=1.0)
+    beta = np.zeros(n, np.float32)
+    idx0, _, _ = oracle.qb_sign_step(s, k, beta, 0.0)
+    v0 = oracle.balance_stats(None, idx0, m, n, k, m)["vio"][0]
+    for _ in range(60):
+        idx, beta, _ = oracle.qb_sign_step(s, k, beta, 0.05)
+    v1 = oracle.balance_stats(None, idx, m, n, k, m)["vio"][0]
+    assert v1 < 0.5 * v0
+
+
+def test_sign_step_with_zero_gamma_is_plain_topk():
+    s = W.make_qb_scores(512, 8, seed=2)
+    beta = np.linspace(-0.3, 0.3, 8).astype(np.float32)
+    idx, beta_out, _ = oracle.qb_sign_step(s, 2, beta, 0.0)
+    assert (beta_out == beta).all()
+    _, ref, _ = oracle.qb_row(s, 2, beta)
+    assert (np.sort(ref, axis=1) == idx).all()
