@@ -476,6 +476,39 @@ def run_gpu_qb(args):
     st1.record(stream)
     torch.cuda.synchronize()
     step_ms = st0.elapsed_time(st1) / n_step
+    # one SignSGD step on beta (row pass + chi counts + sign update), same timing
+    sign_beta = beta.clone()
+    for _ in range(3):
+        lb.moe_balance_sign_step(s, k, sign_beta, 0.01, topk_idx=idx, info=info_step, workspace=ws)
+    torch.cuda.synchronize()
+    st0.record(stream)
+    for _ in range(n_step):
+        lb.moe_balance_sign_step(s, k, sign_beta, 0.01, topk_idx=idx, info=info_step, workspace=ws)
+    st1.record(stream)
+    torch.cuda.synchronize()
+    sign_ms = st0.elapsed_time(st1) / n_step
+
+    # the balancing variants on the same scores, from beta = 0: MaxVio of the step's picks
+    # (selected with the step's incoming beta) after 1, 8 and 32 steps
+    def max_vio():
+        return float(lb.moe_balance_stats(None, idx, n)["vio"][0].item())
+
+    variants = {}
+    for name, one in (("qb_step_midpoint", lambda b: lb.moe_balance_assign(
+                            s, k, beta=b, mode=lb.MOE_QB_STEP, topk_idx=idx, info=info_step, workspace=ws)),
+                      ("bip_step", lambda b: lb.moe_balance_assign(
+                            s, k, beta=b, mode=lb.MOE_QB_STEP, rule=lb.MOE_QB_BIP, topk_idx=idx, info=info_step,
+                            workspace=ws)),
+                      ("signsgd_gamma_0.01", lambda b: lb.moe_balance_sign_step(
+                            s, k, b, 0.01, topk_idx=idx, info=info_step, workspace=ws))):
+        b = torch.zeros(n, dtype=torch.float32, device="cuda")
+        vio = {}
+        for t in range(1, 33):
+            one(b)
+            if t in (1, 8, 32):
+                vio[f"after_{t}"] = max_vio()
+        variants[name] = vio
+    lb.sync_status()
     inf = info.cpu().tolist()
     hbm, src = peaks()
     line = {"metric": METRIC, "value": m / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
@@ -484,7 +517,8 @@ def run_gpu_qb(args):
             "config": {"workload": f"optimal-assignment balancing SOLVE m={m} n={n} k={k} C={m * k // n}",
                        "max_iters": args.qb_iters},
             "solve_info": {"beta_updates": inf[0], "repair_moves": inf[1], "excess_left": inf[2], "ties": inf[3]},
-            "step_mode_ms": step_ms,
+            "step_mode_ms": step_ms, "sign_step_ms": sign_ms,
+            "variants_maxvio": variants,
             "step_mode_GB/s": (3 * m * n * 4) / (step_ms * 1e-3) / 1e9, "peak_hbm": hbm}
     print(json.dumps(line), flush=True)
     return 0
