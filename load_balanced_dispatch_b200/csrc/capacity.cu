@@ -72,39 +72,75 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* sh, 
     return sh[tid] - v;
 }
 
-// The scan, run by the last CTA of the count phase: thread e walks the chunks of every segment in
-// order. hist was written by other CTAs of this launch, so it is read through L2 (__ldcg).
+// The scan, run by the last CTA of the count phase. Thread (e, g): expert e = tid % npad, group
+// g = tid / npad of P = blockDim / npad groups; group g takes the g-th contiguous range of each
+// segment's chunks, holding up to kRun histogram entries in registers. The groups' sums are
+// added in group order, so each chunk's prefix (the earlier chunks of its segment, in chunk
+// order) is exact. hist was written by other CTAs of this launch, so it is read through L2
+// (__ldcg). Ranges longer than kRun (more chunks per segment than P kRun) re-read hist.
+namespace cap {
+constexpr int kRun = 16;
+}
 __device__ __forceinline__ void cap_scan_body(const int32_t* hist, int n, int64_t nseg, int64_t cps, int32_t capacity,
                                               int32_t* __restrict__ prefix, int32_t* __restrict__ seg_base,
                                               int32_t* __restrict__ expert_offsets, int32_t* __restrict__ routed_count,
                                               int32_t* __restrict__ kept_count) {
     __shared__ int64_t sh[cap::kThreads];
-    const int e = threadIdx.x;
+    __shared__ int64_t part[cap::kThreads];
+    const int tid = threadIdx.x;
+    const int npad = (n + 31) & ~31;
+    const int P = cap::kThreads / npad;
+    const int e = tid % npad, g = tid / npad;
+    const bool act = g < P && e < n;
+    const int64_t per = (cps + P - 1) / P;
+    const int64_t c0 = min(cps, (int64_t)g * per), c1 = min(cps, c0 + per);
     int64_t kept_total = 0;
-    if (e < n) {
-        for (int64_t s = 0; s < nseg; ++s) {
-            int64_t run = 0;
-            for (int64_t c0 = 0; c0 < cps; c0 += 8) {  // 8 loads in flight
-                int32_t h[8];
+    for (int64_t s = 0; s < nseg; ++s) {
+        const int32_t* hs = hist + s * cps * n;
+        int32_t h[cap::kRun];
+        int64_t sum = 0;
+        if (act) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) h[u] = (c0 + u < cps) ? __ldcg(hist + (s * cps + c0 + u) * n + e) : 0;
+            for (int u = 0; u < cap::kRun; ++u) {
+                h[u] = (c0 + u < c1) ? __ldcg(hs + (c0 + u) * n + e) : 0;
+                sum += h[u];
+            }
+            for (int64_t c = c0 + cap::kRun; c < c1; ++c) sum += __ldcg(hs + c * n + e);
+        }
+        part[tid] = sum;
+        __syncthreads();
+        int64_t run = 0, total = 0;
+        if (act) {
+            for (int q = 0; q < P; ++q) {
+                const int64_t v = part[q * npad + e];
+                if (q < g) run += v;
+                total += v;
+            }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if (c0 + u < cps) {
-                        prefix[(s * cps + c0 + u) * n + e] = (int32_t)run;
-                        run += h[u];
-                    }
+            for (int u = 0; u < cap::kRun; ++u) {
+                if (c0 + u < c1) {
+                    prefix[(s * cps + c0 + u) * n + e] = (int32_t)run;
+                    run += h[u];
                 }
             }
-            const int64_t kept = run < capacity ? run : (int64_t)capacity;
-            routed_count[s * n + e] = (int32_t)run;
-            kept_count[s * n + e] = (int32_t)kept;
-            kept_total += kept;
+            for (int64_t c = c0 + cap::kRun; c < c1; ++c) {
+                prefix[(s * cps + c) * n + e] = (int32_t)run;
+                run += __ldcg(hs + c * n + e);
+            }
+            if (g == 0) {
+                const int64_t kept = total < capacity ? total : (int64_t)capacity;
+                routed_count[s * n + e] = (int32_t)total;
+                kept_count[s * n + e] = (int32_t)kept;
+                kept_total += kept;
+            }
         }
+        __syncthreads();
     }
+    // expert offsets: exclusive scan over the experts of their kept totals (held by group 0)
     int64_t total;
-    const int64_t off = block_exclusive_scan(kept_total, sh, total);
-    if (e < n) {
+    const int64_t off = block_exclusive_scan((g == 0 && e < n) ? kept_total : 0, sh, total);
+    // thread tid's scan slot is tid; the expert of group 0 is e = tid there
+    if (g == 0 && e < n) {
         expert_offsets[e] = (int32_t)off;
         int64_t base = off;
         for (int64_t s = 0; s < nseg; ++s) {
@@ -112,7 +148,7 @@ __device__ __forceinline__ void cap_scan_body(const int32_t* hist, int n, int64_
             base += kept_count[s * n + e];
         }
     }
-    if (e == 0) expert_offsets[n] = (int32_t)total;
+    if (tid == 0) expert_offsets[n] = (int32_t)total;
 }
 
 // Per-chunk expert histogram (shared-memory integer atomics); the last CTA to finish (a ticket

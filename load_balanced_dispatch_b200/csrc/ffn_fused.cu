@@ -76,11 +76,41 @@ struct FusedTile {
     int64_t row0, row_end;
 };
 
-__device__ __forceinline__ FusedTile fused_decode(const FusedShared* sh, int tile, int T1, int n, int d, int d_ff) {
+// Ticket order. Pair j = 0 .. n + L - 1 holds expert j's GEMM1 tiles (j < n) and then expert
+// (j - L)'s GEMM2 tiles (j >= L), so an expert's second GEMM follows its first by L experts'
+// worth of tiles; L = n puts every GEMM2 tile after every GEMM1 tile. For any L every GEMM2
+// tile comes after all GEMM1 tiles of its expert in ticket order, which keeps the launch free
+// of deadlock (tickets are taken in order, by running CTAs only).
+__device__ __forceinline__ int pair_start(const FusedShared* sh, int n, int L, int j) {
+    const int a = j < n ? j : n;
+    int b = j - L;
+    b = b < 0 ? 0 : (b > n ? n : b);
+    return sh->g1.tile_start[a] + sh->g2.tile_start[b];
+}
+// ticket -> (phase, index of the tile in its phase's list)
+__device__ __forceinline__ void ticket_decode(const FusedShared* sh, int n, int L, int ticket, int& phase, int& lt) {
+    int lo = 0, hi = n + L;  // the largest pair j with pair_start(j) <= ticket
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pair_start(sh, n, L, mid) <= ticket) lo = mid;
+        else hi = mid;
+    }
+    const int off = ticket - pair_start(sh, n, L, lo);
+    const int len1 = lo < n ? sh->g1.tile_start[lo + 1] - sh->g1.tile_start[lo] : 0;
+    if (off < len1) {
+        phase = 1;
+        lt = sh->g1.tile_start[lo] + off;
+    } else {
+        phase = 2;
+        lt = sh->g2.tile_start[lo - L] + (off - len1);
+    }
+}
+
+__device__ __forceinline__ FusedTile fused_decode(const FusedShared* sh, int ticket, int L, int n, int d, int d_ff) {
     FusedTile t;
-    t.phase = tile < T1 ? 1 : 2;
+    int lt;
+    ticket_decode(sh, n, L, ticket, t.phase, lt);
     const GroupTable& g = t.phase == 1 ? sh->g1 : sh->g2;
-    const int lt = t.phase == 1 ? tile : tile - T1;
     t.e = group_of_tile(g, n, lt);
     const int local = lt - g.tile_start[t.e];
     const int rows_e = g.row_start[t.e + 1] - g.row_start[t.e];
@@ -131,12 +161,17 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     const uint32_t tmem_base = sh->tmem_base;
     const int T1 = sh->g1.tile_start[n];
     const int total = T1 + sh->g2.tile_start[n];
+    // Lag between an expert's two GEMMs. A lag of about one wave was measured: it kept h in L2 but
+    // GEMM2 producers then waited on GEMM1 tiles still in flight (each producer runs up to RING
+    // tiles ahead) and the launch got slower, so every GEMM2 tile follows every GEMM1 tile.
+    const int L = n;
     volatile int* abort_flag = &sh->abort_flag;
 
     if (warp == 0) {
         if (lane == 0) {
             int stage = 0, slot = 0;
             uint32_t phase = 0, rphase = 0;
+            const uint64_t wpolicy = ptx::l2_policy_evict_first();
             for (;;) {
                 // take the next tile of the launch and hand its id to the MMA and epilogue warps
                 if (!ptx::mbar_wait(&sh->tfree[slot], rphase ^ 1u, abort_flag)) break;
@@ -145,7 +180,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                 ptx::mbar_arrive(&sh->tready[slot]);
                 if (++slot == RING) { slot = 0; rphase ^= 1u; }
                 if (tile >= total) break;
-                const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
+                const FusedTile t = fused_decode(sh, tile, L, n, d, d_ff);
                 if (t.phase == 2) {
                     // all GEMM1 tiles of expert e, each signalled by its 4 epilogue warps
                     const int rows_e = sh->g1.row_start[t.e + 1] - sh->g1.row_start[t.e];
@@ -172,7 +207,13 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     ptx::mbar_expect_tx(&sh->full[stage], STAGE_BYTES);
                     ptx::tma_load_2d(sa, ma, &sh->full[stage], kb * BK, (int)t.row0);
-                    ptx::tma_load_3d(sa + A_BYTES, mb, &sh->full[stage], kb * BK, t.n0, t.e);
+                    // an expert with one row tile reads each weight tile once: evict-first, so the
+                    // hidden rows h that the GEMM2 tiles read back stay in L2 (with more row tiles
+                    // the weight tiles are re-read and keep the normal policy)
+                    if (t.mtiles1 == 1)
+                        ptx::tma_load_3d_hint(sa + A_BYTES, mb, &sh->full[stage], kb * BK, t.n0, t.e, wpolicy);
+                    else
+                        ptx::tma_load_3d(sa + A_BYTES, mb, &sh->full[stage], kb * BK, t.n0, t.e);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -188,7 +229,9 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                 ptx::mbar_arrive(&sh->tfree[slot]);
                 if (++slot == RING) { slot = 0; rphase ^= 1u; }
                 if (tile < 0) break;
-                const int K = tile < T1 ? d : d_ff;
+                int ph, lt_unused;
+                ticket_decode(sh, n, L, tile, ph, lt_unused);
+                const int K = ph == 1 ? d : d_ff;
                 const int nkb = (K + BK - 1) / BK;
                 if (!ptx::mbar_wait(&sh->tempty[acc], aphase ^ 1u, abort_flag)) break;
                 ptx::tc_fence_after();
@@ -222,7 +265,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
             if (lane == 0) ptx::mbar_arrive(&sh->tfree[slot]);
             if (++slot == RING) { slot = 0; rphase ^= 1u; }
             if (tile < 0) break;
-            const FusedTile t = fused_decode(sh, tile, T1, n, d, d_ff);
+            const FusedTile t = fused_decode(sh, tile, L, n, d, d_ff);
             // stage the tile's 256 bias values in shared memory while the accumulator fills
             __nv_bfloat16* be = sh->bias_stage[warp - 2];
             {
