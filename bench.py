@@ -59,7 +59,7 @@ def peaks_all():
 # dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch at a shape, from the
 # ncu capture summarised under profiles/. Emptied whenever the kernel changes (the figure would be
 # stale), refilled from the next capture.
-FFN_DRAM_TRAFFIC = {"switch": 1.24e9 + 37.99e6}
+FFN_DRAM_TRAFFIC = {"switch": 1.24e9 + 36.06e6}
 
 
 def ffn_roofline(cfg, offsets, ffn_ms, esz=2):
@@ -411,6 +411,8 @@ def run_gpu(args, cfg):
             "roofline": ffn_roofline(cfg, offsets, stage_ms["ffn"]),
             "stages": {s: ({"ms": stage_ms[s], "fused_into": "ffn (second GEMM epilogue)"}
                            if s == "combine" and layer.ffn_combine else
+                           {"ms": stage_ms[s], "fused_into": "ffn (first GEMM gathers its rows from x)"}
+                           if s == "dispatch" and layer.gather else
                            {"ms": stage_ms[s], "GB/s": sb[s] / (stage_ms[s] * 1e-3) / 1e9,
                             "hbm_frac": sb[s] / (stage_ms[s] * 1e-3) / 1e9 / hbm}) for s in MoELayer.STAGES},
             "stages_note": "per-stage graphs with events between them, a separate run of K forwards",

@@ -240,6 +240,24 @@ MOE_API moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1
                           int64_t max_rows, void* ybuf, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Expert FFN reading its rows straight from the token-major activations (bf16).
+ * Passage: "Switch Transformer read for implementation" (molayo1419.me): the
+ * dispatch permutation groups tokens by expert before the FFN; here the FFN's
+ * first GEMM loads row r of the expert-major order as x[src_token[r]], so the
+ * permuted copy xbuf is never formed.
+ *  x [m, d] token-major; src_token [rows] from moe_capacity_slots; other
+ *  arguments as moe_expert_ffn. ybuf [max_rows, d] out, expert-major.
+ *  Results: bit for bit those of moe_dispatch followed by moe_expert_ffn. Measured
+ *  slower than that pair on the B200 (the row gather feeds the tensor cores more slowly
+ *  than tile loads of xbuf); its use is saving the xbuf buffer (max_rows x d elements).
+ *  bf16 only (MOE_ERR_UNSUPPORTED for fp32). Workspace: moe_expert_ffn_workspace_size.
+ */
+MOE_API moe_status moe_expert_ffn_gather(const void* x, moe_dtype dt, const void* w1, const void* b1, const void* w2,
+                                 const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d, int32_t d_ff,
+                                 int64_t max_rows, const int32_t* src_token, int64_t m, void* ybuf, void* workspace,
+                                 size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Expert FFN and combine in one call, for one pick per token (k = 1, bf16).
  * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Switch
  * Routing Step 3 (y = p_i* E_i*(x)) with "Switch Transformer read for

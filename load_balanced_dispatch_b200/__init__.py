@@ -29,7 +29,8 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_balance_assign", "moe_capacity_slots_workspace_size", "moe_capacity_slots", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
-           "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step")
+           "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step",
+           "moe_expert_ffn_gather")
 
 
 class MoEError(RuntimeError):
@@ -69,6 +70,7 @@ def lib() -> C.CDLL:
         L.moe_combine.argtypes = [P, I32, P, P, P, I64, I32, I32, P, P]
         L.moe_expert_ffn_combine.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, P, P, I64, P, P, SZ,
                                              P]
+        L.moe_expert_ffn_gather.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, I64, P, P, SZ, P]
         L.moe_balance_stats_workspace_size.argtypes = [I64, I32, I64]
         L.moe_balance_stats_workspace_size.restype = SZ
         L.moe_balance_stats.argtypes = [P, P, I64, I32, I32, I64, F, P, P, P, P, P, F, P, SZ, P]
@@ -228,6 +230,26 @@ def moe_expert_ffn(xbuf, w1, b1, w2, b2, expert_offsets, ybuf=None, workspace=No
     return ybuf
 
 
+def moe_expert_ffn_gather(x, w1, b1, w2, b2, expert_offsets, src_token, max_rows=None, ybuf=None, workspace=None,
+                          stream=None):
+    """bf16: ybuf = the FFN of x[src_token[r]] per expert group, rows gathered by the FFN itself (no xbuf)."""
+    m, d = x.shape
+    n, d_ff, _ = w1.shape
+    max_rows = src_token.numel() if max_rows is None else max_rows
+    dt = _dtype_code(x)
+    for t, shp, name in ((w1, (n, d_ff, d), "w1"), (b1, (n, d_ff), "b1"), (w2, (n, d, d_ff), "w2"), (b2, (n, d), "b2")):
+        _need(t, x.dtype, shp, name)
+    if ybuf is None:
+        ybuf = torch.empty((max_rows, d), dtype=x.dtype, device=x.device)
+    ws_bytes = lib().moe_expert_ffn_workspace_size(dt, max_rows, d_ff)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=x.device)
+    _check("moe_expert_ffn_gather", lib().moe_expert_ffn_gather(
+        _ptr(x), dt, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(expert_offsets), n, d, d_ff, max_rows,
+        _ptr(src_token), m, _ptr(ybuf), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return ybuf
+
+
 def moe_expert_ffn_combine(xbuf, w1, b1, w2, b2, expert_offsets, src_token, dest_row, topk_gate, residual=None,
                            y=None, workspace=None, stream=None):
     """k = 1, bf16: y[t] = residual[t] + g_t FFN_e(xbuf[row of t]) with the combine done by the FFN's second
@@ -237,6 +259,7 @@ def moe_expert_ffn_combine(xbuf, w1, b1, w2, b2, expert_offsets, src_token, dest
     m, k = dest_row.shape
     if k != 1:
         raise ValueError("moe_expert_ffn_combine: one pick per token (k = 1)")
+    max_rows = min(max_rows, m)
     dt = _dtype_code(xbuf)
     for t, shp, name in ((w1, (n, d_ff, d), "w1"), (b1, (n, d_ff), "b1"), (w2, (n, d, d_ff), "w2"), (b2, (n, d), "b2")):
         _need(t, xbuf.dtype, shp, name)
@@ -247,7 +270,7 @@ def moe_expert_ffn_combine(xbuf, w1, b1, w2, b2, expert_offsets, src_token, dest
     if workspace is None:
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=xbuf.device)
     _check("moe_expert_ffn_combine", lib().moe_expert_ffn_combine(
-        _ptr(xbuf), dt, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(expert_offsets), n, d, d_ff, min(max_rows, m),
+        _ptr(xbuf), dt, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(expert_offsets), n, d, d_ff, max_rows,
         _ptr(src_token), _ptr(dest_row), _ptr(topk_gate), _ptr(residual), m, _ptr(y), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return y

@@ -24,6 +24,9 @@ cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_r
 cudaError_t launch_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2, const void* b2,
                        const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
                        cudaStream_t stream);
+cudaError_t launch_ffn_tc_gather(const void* x, const int32_t* src_token, int64_t m, const void* w1, const void* b1,
+                                 const void* w2, const void* b2, const int32_t* offsets, int n, int d, int d_ff,
+                                 int64_t max_rows, void* ybuf, void* hbuf, cudaStream_t stream);
 cudaError_t launch_ffn_tc_combine(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
                                   const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* hbuf,
                                   const int32_t* src_token, const int32_t* dest_row, const float* gate,
@@ -189,6 +192,30 @@ moe_status moe_expert_ffn(const void* xbuf, moe_dtype dt, const void* w1, const 
     return check_launch(launch_ffn(xbuf, dt, w1, b1, w2, b2, expert_offsets, n, d, d_ff, max_rows, ybuf, workspace,
                                    stream),
                         "moe_expert_ffn");
+}
+
+moe_status moe_expert_ffn_gather(const void* x, moe_dtype dt, const void* w1, const void* b1, const void* w2,
+                                 const void* b2, const int32_t* expert_offsets, int32_t n, int32_t d, int32_t d_ff,
+                                 int64_t max_rows, const int32_t* src_token, int64_t m, void* ybuf, void* workspace,
+                                 size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
+    if (dt != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_expert_ffn_gather: bf16 only (use moe_dispatch + moe_expert_ffn)");
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(max_rows >= 0 && max_rows < ((int64_t)1 << 31), "bad max_rows");
+    REQUIRE(m >= 0 && m < ((int64_t)1 << 31), "bad m");
+    REQUIRE(d >= 8 && d % 8 == 0, "d must be a positive multiple of 8");
+    REQUIRE(d_ff >= 8 && d_ff % 8 == 0, "d_ff must be a positive multiple of 8");
+    REQUIRE(expert_offsets && w1 && b1 && w2 && b2, "weights, biases and expert_offsets are required");
+    REQUIRE(max_rows == 0 || (x && ybuf && src_token && m > 0), "x, src_token and ybuf are required");
+    REQUIRE(aligned16(x) && aligned16(ybuf) && aligned16(w1) && aligned16(w2) && aligned16(workspace),
+            "x, ybuf, w1, w2 and the workspace must be 16-byte aligned");
+    const size_t need = moe_expert_ffn_workspace_size(dt, max_rows, d_ff);
+    if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+    if (max_rows == 0) return MOE_OK;
+    return check_launch(launch_ffn_tc_gather(x, src_token, m, w1, b1, w2, b2, expert_offsets, n, d, d_ff, max_rows,
+                                             ybuf, workspace, stream),
+                        "moe_expert_ffn_gather");
 }
 
 moe_status moe_expert_ffn_combine(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2,

@@ -38,7 +38,9 @@ namespace moe {
 
 namespace fz {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kLoadWarps = 4;
+// warp 0 TMA, warp 1 MMA, warps 2-5 epilogue; with the row gather also warps 6-9
+constexpr int threads(bool gather) { return gather ? 320 : 192; }
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
@@ -68,6 +70,18 @@ struct FusedCombine {
     const float* gate;                 // [m] (k = 1)
     const __nv_bfloat16* residual;     // [m, d] or nullptr
     __nv_bfloat16* y;                  // [m, d] or nullptr
+    int64_t m;
+};
+
+// Dispatch fused into the first GEMM (the GATHER instantiation): the GEMM1 A tiles are gathered
+// straight from the token-major activations, row r of the expert-major order being
+// x[src_token[r]], by four loader warps (16-byte cp.async into the 128-byte-swizzled K-major
+// layout, a proxy fence, then an arrival on the stage's mbarrier), so xbuf is never formed.
+// Measured slower than dispatch + TMA tile loads (the loaders cannot feed the tensor cores at
+// the rate one TMA tile load per stage does); it saves the xbuf buffer, rows x d elements.
+struct FusedGather {
+    const __nv_bfloat16* x;     // [m, d] or nullptr (A tiles from xbuf by TMA)
+    const int32_t* src_token;   // [rows]
     int64_t m;
 };
 
@@ -125,13 +139,14 @@ __device__ __forceinline__ FusedTile fused_decode(const FusedShared* sh, int tic
     return t;
 }
 
-__global__ void __launch_bounds__(fz::kThreads, 1)
+template <bool GATHER>
+__global__ void __launch_bounds__(fz::threads(GATHER), 1)
 ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w1,
              const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_w2,
              const __nv_bfloat16* __restrict__ b1, const __nv_bfloat16* __restrict__ b2,
              const int32_t* __restrict__ offsets, int n, int d, int d_ff, int64_t max_rows,
              __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ y, int* __restrict__ done1,
-             int* __restrict__ next_tile, FusedCombine cmb) {
+             int* __restrict__ next_tile, FusedCombine cmb, FusedGather gth) {
     using namespace fz;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -140,9 +155,17 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     const int ntn1 = (d_ff + BN - 1) / BN, ntn2 = (d + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
+        const bool gather = GATHER;
+        // full: the producer's arrival (+ TMA bytes), and with the gather the 128 loader threads'
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&sh->full[s], 1 + (gather ? 32 * kLoadWarps : 0));
+            ptx::mbar_init(&sh->empty[s], 1);
+        }
         for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
-        for (int r = 0; r < RING; ++r) { ptx::mbar_init(&sh->tready[r], 1); ptx::mbar_init(&sh->tfree[r], 1 + kEpiWarps); }
+        for (int r = 0; r < RING; ++r) {
+            ptx::mbar_init(&sh->tready[r], 1);
+            ptx::mbar_init(&sh->tfree[r], 1 + kEpiWarps + (gather ? kLoadWarps : 0));
+        }
         sh->abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::prefetch_tensormap(&map_x);
@@ -201,12 +224,13 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                 const CUtensorMap* ma = t.phase == 1 ? &map_x : &map_h;
                 const CUtensorMap* mb = t.phase == 1 ? &map_w1 : &map_w2;
                 const int nkb = (t.K + BK - 1) / BK;
+                const bool a_by_tma = t.phase == 2 || !GATHER;  // else the loader warps gather A
                 bool ok = true;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + stage * STAGE_BYTES;
-                    ptx::mbar_expect_tx(&sh->full[stage], STAGE_BYTES);
-                    ptx::tma_load_2d(sa, ma, &sh->full[stage], kb * BK, (int)t.row0);
+                    ptx::mbar_expect_tx(&sh->full[stage], a_by_tma ? STAGE_BYTES : B_BYTES);
+                    if (a_by_tma) ptx::tma_load_2d(sa, ma, &sh->full[stage], kb * BK, (int)t.row0);
                     // an expert with one row tile reads each weight tile once: evict-first, so the
                     // hidden rows h that the GEMM2 tiles read back stay in L2 (with more row tiles
                     // the weight tiles are re-read and keep the normal policy)
@@ -252,6 +276,66 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                 if (!ok) break;
                 ptx::umma_commit(&sh->tfull[acc]);
                 if (++acc == 2) { acc = 0; aphase ^= 1u; }
+            }
+        }
+    } else if (warp >= 2 + kEpiWarps) {
+        // row gather (warps 6-9): thread l copies row l of each GEMM1 A tile, 8 x 16 bytes per
+        // K block, from x[src_token[row]] (zeros past the expert's rows or past d); the arrival
+        // for a stage waits until the next stage's copies are issued, so two are in flight
+        if (GATHER) {
+            const int ltid = (warp - 2 - kEpiWarps) * 32 + lane;
+            int stage = 0, slot = 0, pend = -1;
+            uint32_t phase = 0, rphase = 0;
+            bool ok = true;
+            for (;;) {
+                bool w = true;
+                if (lane == 0) w = ptx::mbar_wait(&sh->tready[slot], rphase, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                const int tile = *(volatile int*)&sh->tile_ring[slot];
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sh->tfree[slot]);
+                if (++slot == RING) { slot = 0; rphase ^= 1u; }
+                if (tile < 0) break;
+                const FusedTile t = fused_decode(sh, tile, L, n, d, d_ff);
+                const int64_t r = t.row0 + ltid;
+                bool valid = t.phase == 1 && r < t.row_end;
+                int64_t tok = 0;
+                if (valid) {
+                    tok = gth.src_token[r];
+                    if (tok < 0 || tok >= gth.m) { record_error(kErrTokenIndex); valid = false; tok = 0; }
+                }
+                const __nv_bfloat16* xrow = gth.x + tok * d;
+                const int nkb = (t.K + BK - 1) / BK;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    bool e = true;
+                    if (lane == 0) e = ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag);
+                    if (!__shfl_sync(0xffffffffu, e, 0)) { ok = false; break; }
+                    if (t.phase == 1) {
+                        const uint32_t dst = ptx::smem_u32(smem + stage * STAGE_BYTES) + (uint32_t)ltid * 128u;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int col = kb * BK + c * 8;
+                            const bool in = valid && col < d;
+                            ptx::cp_async16(dst + ((uint32_t)(c ^ (ltid & 7)) << 4), in ? (const void*)(xrow + col)
+                                                                                         : (const void*)gth.x,
+                                            in ? 16u : 0u);
+                        }
+                    }
+                    ptx::cp_async_commit();
+                    if (pend >= 0) {
+                        ptx::cp_async_wait_group<1>();
+                        ptx::fence_proxy_async_shared();
+                        ptx::mbar_arrive(&sh->full[pend]);
+                    }
+                    pend = stage;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            if (ok && pend >= 0) {
+                ptx::cp_async_wait_group<0>();
+                ptx::fence_proxy_async_shared();
+                ptx::mbar_arrive(&sh->full[pend]);
             }
         }
     } else {
@@ -391,19 +475,25 @@ cudaError_t launch_combine_dropped(const int32_t* dest_row, const void* residual
                       static_cast<const uint4*>(residual), m, (int64_t)d * 2 / 16, static_cast<uint4*>(y));
 }
 
+// xbuf: the expert-major rows [max_rows, d], or with gth the token-major x [gth->m, d] whose
+// rows the kernel gathers by gth->src_token.
 cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
                              const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
                              int* counters, cudaStream_t stream, const FusedCombine* cmb = nullptr,
-                             bool zero_counters = true) {
+                             bool zero_counters = true, const FusedGather* gth = nullptr) {
     CUtensorMap mx, mw1, mh, mw2;
-    if (!map_2d(&mx, xbuf, (uint64_t)max_rows, (uint64_t)d, fz::BM)) return cudaErrorInvalidValue;
+    const uint64_t xrows = gth ? (uint64_t)gth->m : (uint64_t)max_rows;  // the A map is unused when gathering
+    if (!map_2d(&mx, xbuf, xrows, (uint64_t)d, fz::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw1, w1, (uint64_t)n, (uint64_t)d_ff, (uint64_t)d, fz::BN)) return cudaErrorInvalidValue;
     if (!map_2d(&mh, hbuf, (uint64_t)max_rows, (uint64_t)d_ff, fz::BM)) return cudaErrorInvalidValue;
     if (!map_3d(&mw2, w2, (uint64_t)n, (uint64_t)d, (uint64_t)d_ff, fz::BN)) return cudaErrorInvalidValue;
     static bool attr = false;
     const size_t smem = fused_smem_bytes();
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(ffn_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(ffn_fused_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(ffn_fused_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
@@ -412,10 +502,16 @@ cudaError_t launch_ffn_fused(const void* xbuf, const void* w1, const void* b1, c
         cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(ffn_fused_tc, dim3(num_sms()), dim3(fz::kThreads), smem, stream, mx, mw1, mh, mw2,
+    const FusedCombine c = cmb ? *cmb : FusedCombine{nullptr, nullptr, nullptr, nullptr, 0};
+    if (gth)
+        return launch_pdl(ffn_fused_tc<true>, dim3(num_sms()), dim3(fz::threads(true)), smem, stream, mx, mw1, mh,
+                          mw2, static_cast<const __nv_bfloat16*>(b1), static_cast<const __nv_bfloat16*>(b2), offsets,
+                          n, d, d_ff, max_rows, static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf),
+                          counters, counters + n, c, *gth);
+    return launch_pdl(ffn_fused_tc<false>, dim3(num_sms()), dim3(fz::threads(false)), smem, stream, mx, mw1, mh, mw2,
                       static_cast<const __nv_bfloat16*>(b1), static_cast<const __nv_bfloat16*>(b2), offsets, n, d,
                       d_ff, max_rows, static_cast<__nv_bfloat16*>(hbuf), static_cast<__nv_bfloat16*>(ybuf), counters,
-                      counters + n, cmb ? *cmb : FusedCombine{nullptr, nullptr, nullptr, nullptr, 0});
+                      counters + n, c, FusedGather{nullptr, nullptr, 0});
 }
 
 // Both GEMMs in one persistent launch; its counters (per-expert completions, tile ticket) follow h.
@@ -429,6 +525,15 @@ cudaError_t launch_ffn_tc(const void* xbuf, const void* w1, const void* b1, cons
                           cudaStream_t stream) {
     return launch_ffn_fused(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf,
                             ffn_counters(hbuf, max_rows, d_ff), stream);
+}
+
+// The FFN reading its rows straight from x by src_token (the dispatch fused into the first GEMM).
+cudaError_t launch_ffn_tc_gather(const void* x, const int32_t* src_token, int64_t m, const void* w1, const void* b1,
+                                 const void* w2, const void* b2, const int32_t* offsets, int n, int d, int d_ff,
+                                 int64_t max_rows, void* ybuf, void* hbuf, cudaStream_t stream) {
+    const FusedGather gth{static_cast<const __nv_bfloat16*>(x), src_token, m};
+    return launch_ffn_fused(x, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf,
+                            ffn_counters(hbuf, max_rows, d_ff), stream, nullptr, true, &gth);
 }
 
 // The FFN with the k = 1 gated combine in its GEMM2 epilogue, plus the dropped tokens' rows.

@@ -13,7 +13,7 @@ import torch
 
 from . import (MOE_QB_MIDPOINT, MOE_QB_STEP, MOE_SIGMOID, MOE_SOFTMAX, moe_balance_assign, moe_balance_stats,
                moe_capacity_slots, moe_combine, moe_dispatch, moe_expert_ffn, moe_expert_ffn_combine,
-               moe_router_topk, lib)
+               moe_expert_ffn_gather, moe_router_topk, lib)
 
 
 @dataclass
@@ -47,6 +47,7 @@ class MoELayer:
         nseg = m // seg
         dev = self.device
         i32, f32 = torch.int32, torch.float32
+        bf16 = s.dtype == torch.bfloat16
         self.rows_max = m * k
         self.buf = dict(
             topk_idx=torch.empty((m, k), dtype=i32, device=dev),
@@ -58,8 +59,8 @@ class MoELayer:
             expert_offsets=torch.empty((n + 1,), dtype=i32, device=dev),
             routed_count=torch.empty((nseg, n), dtype=i32, device=dev),
             kept_count=torch.empty((nseg, n), dtype=i32, device=dev),
-            xbuf=torch.empty((self.rows_max, d), dtype=s.dtype, device=dev),
-            ybuf=torch.empty((self.rows_max, d), dtype=s.dtype, device=dev),
+            xbuf=torch.empty((self.rows_max, d), dtype=s.dtype, device=dev),  # k = 1 bf16 needs no ybuf
+            ybuf=torch.empty((0 if (bf16 and k == 1) else self.rows_max, d), dtype=s.dtype, device=dev),
             y=torch.empty((m, d), dtype=s.dtype, device=dev),
             f=torch.empty((nseg + 1, n), dtype=f32, device=dev),
             P=torch.empty((nseg + 1, n), dtype=f32, device=dev),
@@ -77,7 +78,10 @@ class MoELayer:
             stats=torch.empty((max(L.moe_balance_stats_workspace_size(m, n, seg), 1),), dtype=torch.uint8,
                               device=dev),
         )
-        # one pick per token in bf16: the combine runs in the FFN's second GEMM (moe_expert_ffn_combine)
+        # one pick per token in bf16: the combine runs in the FFN's second GEMM (moe_expert_ffn_combine).
+        # gather = True would let the FFN read its rows from x (moe_expert_ffn_gather: no dispatch, no
+        # xbuf); measured slower, it is off
+        self.gather = False
         self.ffn_combine = s.k == 1 and s.dtype == torch.bfloat16
         # data-parallel replicas: set by enable_global_stats(); the Loss-Free bias then follows the
         # pooled counts of every rank instead of this rank's
@@ -95,13 +99,17 @@ class MoELayer:
         elif i == 1:
             moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"], stream=st)
         elif i == 2:
-            moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
+            if not self.gather:  # otherwise the FFN gathers its rows from x
+                moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
         elif i == 3:
             if self.ffn_combine:
                 moe_expert_ffn_combine(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"],
                                        b["src_token"], b["dest_row"], b["topk_gate"],
                                        residual=x if s.residual else None, y=b["y"], workspace=self.ws["ffn"],
                                        stream=st)
+            elif self.gather:
+                moe_expert_ffn_gather(x, w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"], b["src_token"],
+                                      max_rows=self.rows_max, ybuf=b["ybuf"], workspace=self.ws["ffn"], stream=st)
             else:
                 moe_expert_ffn(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"], ybuf=b["ybuf"],
                                workspace=self.ws["ffn"], stream=st)
@@ -148,7 +156,7 @@ class MoELayer:
         torch.cuda.synchronize()
         self.graphs = []
         for i in range(len(self.STAGES)):
-            if i == 4 and self.ffn_combine:  # nothing to launch: the combine ran in the FFN stage
+            if (i == 4 and self.ffn_combine) or (i == 2 and self.gather):  # done inside the FFN stage
                 self.graphs.append(None)
                 continue
             g = torch.cuda.CUDAGraph()
@@ -210,8 +218,10 @@ class MoELayer:
         bf16 = s.dtype == torch.bfloat16
         router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
         ffn = 1 if bf16 else 2
-        if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped tokens' rows
-            return router + 2 + 1 + 2 + 0 + 1
+        if self.ffn_combine:  # the FFN (gathering its rows) with the combine in its epilogue + the dropped rows
+            return router + 2 + 0 + 2 + 0 + 1
+        if self.gather:       # the FFN gathering its rows, then the combine
+            return router + 2 + 0 + 1 + 1 + 1
         return router + 2 + 1 + ffn + 1 + 1
 
 

@@ -221,6 +221,31 @@ def test_expert_ffn_combine_matches_two_calls(m, n, d, d_ff, cap):
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+@pytest.mark.parametrize("m,n,k,d,d_ff,cap", [(2000, 16, 2, 768, 3072, 300), (1000, 64, 6, 2048, 1408, 10 ** 6),
+                                              (777, 8, 3, 256, 512, 40), (512, 4, 1, 128, 256, 0)])
+def test_expert_ffn_gather_matches_dispatch(m, n, k, d, d_ff, cap):
+    # the FFN loading its rows from x by src_token gives bit for bit the FFN of the dispatched
+    # copy, including dropped picks, ragged experts and a capacity that empties every expert
+    rng = np.random.default_rng(m * 3 + d)
+    x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
+    idx = W.make_topk_idx(m, n, k, seed=6, skew=1.3)
+    bf = torch.bfloat16
+    wd = [dev(W.round_to_bf16(a), bf) for a in (
+        (rng.standard_normal((n, d_ff, d)) / np.sqrt(d)).astype(np.float32),
+        (0.1 * rng.standard_normal((n, d_ff))).astype(np.float32),
+        (rng.standard_normal((n, d, d_ff)) / np.sqrt(d_ff)).astype(np.float32),
+        (0.1 * rng.standard_normal((n, d))).astype(np.float32))]
+    xd = dev(x, bf)
+    out = lb.moe_capacity_slots(dev(idx), n, cap)
+    xbuf = lb.moe_dispatch(xd, out["src_token"], out["expert_offsets"], n, m * k)
+    y_ref = lb.moe_expert_ffn(xbuf, *wd, out["expert_offsets"])
+    y = lb.moe_expert_ffn_gather(xd, *wd, out["expert_offsets"], out["src_token"], max_rows=m * k)
+    torch.cuda.synchronize()
+    lb.sync_status()
+    rows = int(host(out["expert_offsets"])[-1])
+    assert torch.equal(y[:rows].view(torch.int16), y_ref[:rows].view(torch.int16))
+
+
 # ---------------------------------------------------------------- statistics
 @pytest.mark.parametrize("m,n,k,seg", [(8192, 128, 1, 8192), (65536, 64, 2, 4096), (1000, 8, 1, 250),
                                        (777, 256, 8, 777)])
