@@ -32,6 +32,7 @@
 //              token. The number of moves equals the excess, so the host
 //              enqueues exactly that many rounds without waiting in between.
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 
@@ -577,7 +578,6 @@ constexpr int kArcBatch = 4;         // members per warp step (their loads in fl
 constexpr int kArcWords = 256;       // bitmap words compacted per pass: at most 8192 members
 constexpr int kArcSlices = 8;        // CTAs per row of W, each over 1/8 of the tokens
 constexpr int kMemberCap = kArcWords * 32;
-constexpr int kStepThreads = 1024;   // 4 threads per expert column in the shortest-path rounds
 constexpr size_t kArcSmem = (size_t)(kArcThreads / 32) * kMaxExperts * (8 + 4) + (size_t)kMemberCap * 4;
 }  // namespace qb
 
@@ -756,126 +756,133 @@ __device__ __forceinline__ void compact_flags(const unsigned char* flag, int n, 
     __syncthreads();
 }
 
-// One augmentation (one unit of excess): Jacobi Bellman-Ford rounds from the over-full experts,
-// the nearest under-full expert (lowest index on ties), the path by lowest-index predecessors, and
-// the moves of each arc's token. Writes the rows of W that the moves invalidate (the old set of
-// every moved token, plus the expert it moved to) for the next arc launch.
-__global__ void __launch_bounds__(qb::kStepThreads)
+namespace qb {
+constexpr int kRepCtas = 8;       // one cluster of 8 CTAs
+constexpr int kRepThreads = 256;  // thread (part 0..7, column 0..31)
+constexpr int kRepCols = 32;      // columns of W per CTA (n <= 256)
+}  // namespace qb
+
+// One augmentation (one unit of excess) on one 8-CTA cluster. CTA c owns the columns
+// b = 32 c .. 32 c + 31 of W, held in its shared memory. Jacobi Bellman-Ford rounds from the
+// over-full experts: each round every CTA relaxes its own columns from the experts whose
+// distance changed in the previous round (the frontier; the same fixpoint as full rounds), then
+// writes its columns' new distances and change flags into the next-round buffers of every CTA
+// of the cluster (distributed shared memory) and one cluster barrier ends the round, so every
+// CTA holds the same full distance vector. Then the predecessors (lowest a with
+// dist[a] + W[a][b] == dist[b]) of each CTA's columns go to CTA 0, whose thread 0 takes the
+// nearest under-full expert (lowest index on ties), walks the path and moves each arc's token,
+// and CTA 0 lists the rows of W the moves invalidate (the old set of every moved token, plus the
+// expert it moved to) for the next arc launch. All decisions that end loops or return are made
+// on data every CTA holds identically, so every CTA reaches every cluster barrier.
+__global__ void __launch_bounds__(qb::kRepThreads, 1)
 qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, const int32_t* __restrict__ A,
                       int32_t* __restrict__ counts, int32_t* __restrict__ topk_idx, int32_t* __restrict__ status,
                       int32_t* __restrict__ rows, int32_t* __restrict__ nrows, uint32_t* __restrict__ mem,
                       int64_t words) {
-    __shared__ double dist[kMaxExperts], part_d[4][kMaxExperts];
-    __shared__ int part_p[4][kMaxExperts], pred[kMaxExperts];
+    extern __shared__ double wsl[];  // [n][32]: this CTA's columns of W
+    __shared__ double dist[2][kMaxExperts];
+    __shared__ unsigned char chg[2][kMaxExperts];
+    __shared__ double part_d[8][qb::kRepCols];
+    __shared__ double nd_own[qb::kRepCols];
+    __shared__ unsigned char nc_own[qb::kRepCols];
+    __shared__ int part_p[8][qb::kRepCols];
+    __shared__ int pred[kMaxExperts];
+    __shared__ int front[kMaxExperts], nfront, wcount[kMaxExperts / 32];
     __shared__ int any_over;
     __shared__ uint32_t touched[kMaxExperts / 32];
-    const int tid = threadIdx.x;
-    const int b = tid & 255, part = tid >> 8;  // 4 threads per column b, each a quarter of the a range
+    const int tid = threadIdx.x, bl = tid & 31, part = tid >> 5;
+    const uint32_t crank = ptx::cluster_ctarank();
+    const int b = (int)crank * qb::kRepCols + bl;
+    const bool own = b < n;
+    // status is read by every CTA before any of them can change it (CTA 0 writes it at the end)
     if (status[qb::kStError] || status[qb::kStDone]) return;
+    for (int q = tid; q < n * qb::kRepCols; q += blockDim.x) {
+        const int a = q / qb::kRepCols, j = (int)crank * qb::kRepCols + (q % qb::kRepCols);
+        wsl[q] = j < n ? W[(int64_t)a * n + j] : INFINITY;
+    }
     if (tid == 0) any_over = 0;
     if (tid < kMaxExperts / 32) touched[tid] = 0;
     __syncthreads();
-    if (part == 0 && b < n) {
-        const bool over = counts[b] > C;
-        dist[b] = over ? 0.0 : INFINITY;
+    for (int e = tid; e < kMaxExperts; e += blockDim.x) {
+        const bool over = e < n && counts[e] > C;
+        dist[0][e] = over ? 0.0 : INFINITY;
+        dist[1][e] = INFINITY;
+        chg[0][e] = over ? 1 : 0;
+        chg[1][e] = 0;
+        pred[e] = -1;
         if (over) atomicOr(&any_over, 1);
     }
     __syncthreads();
-    if (!any_over) {
-        if (tid == 0) { status[qb::kStDone] = 1; *nrows = 0; }
+    if (!any_over) {  // the same counts in every CTA: all return here together
+        if (crank == 0 && tid == 0) { status[qb::kStDone] = 1; *nrows = 0; }
         return;
     }
-    // Jacobi rounds over the frontier: only experts whose distance changed in the previous round
-    // can improve another one, so each round reads just their rows of W (same fixpoint as full rounds)
-    __shared__ int front[kMaxExperts], nfront;
-    __shared__ unsigned char chg[kMaxExperts];
-    __shared__ int wcount[kMaxExperts / 32];
-    if (tid < kMaxExperts) chg[tid] = (tid < n && dist[tid] == 0.0) ? 1 : 0;
-    __syncthreads();
+    ptx::cluster_sync();  // every CTA's buffers are initialised before any remote write
+    int cur = 0;
     bool settled = false;
     for (int round = 0; round <= n; ++round) {
-        compact_flags(chg, n, front, &nfront, wcount);
+        compact_flags(chg[cur], n, front, &nfront, wcount);
         const int nf = nfront;
         if (nf == 0) { settled = true; break; }
-        double bestd = INFINITY;
-        if (b < n) {
-            // this thread's quarter of the frontier, 8 loads in flight
-            for (int f0 = part; f0 < nf; f0 += 4 * 8) {
-                double w8[8];
-                int a8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int fi = f0 + 4 * u;
-                    a8[u] = fi < nf ? front[fi] : -1;
-                    w8[u] = a8[u] >= 0 ? W[(int64_t)a8[u] * n + b] : INFINITY;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int aa = a8[u];
-                    if (aa >= 0 && aa != b && w8[u] != INFINITY) {
-                        const double c = dist[aa] + w8[u];
-                        if (c < bestd) bestd = c;
-                    }
+        double best = INFINITY;
+        if (own) {
+            for (int f = part; f < nf; f += 8) {
+                const int a = front[f];
+                const double w = wsl[a * qb::kRepCols + bl];
+                if (a != b && w != INFINITY) {
+                    const double c = dist[cur][a] + w;
+                    if (c < best) best = c;
                 }
             }
         }
-        part_d[part][b] = bestd;
+        part_d[part][bl] = best;
         __syncthreads();
-        if (part == 0) {
-            if (b < n) {
-                double nd = dist[b];
-                for (int p = 0; p < 4; ++p) nd = fmin(nd, part_d[p][b]);
-                chg[b] = nd != dist[b];
-                part_d[0][b] = nd;
-            } else {
-                chg[b] = 0;
-            }
+        if (part == 0 && own) {
+            double nd = dist[cur][b];
+            for (int p = 0; p < 8; ++p) nd = fmin(nd, part_d[p][bl]);
+            nd_own[bl] = nd;
+            nc_own[bl] = nd != dist[cur][b] ? 1 : 0;
         }
         __syncthreads();
-        if (part == 0 && b < n) dist[b] = part_d[0][b];
-        __syncthreads();
+        if (own) {  // thread (part = target CTA, bl): this column into that CTA's next-round buffers
+            ptx::st_cluster_f64(ptx::mapa_shared(ptx::smem_u32(&dist[cur ^ 1][b]), (uint32_t)part), nd_own[bl]);
+            ptx::st_cluster_u8(ptx::mapa_shared(ptx::smem_u32(&chg[cur ^ 1][b]), (uint32_t)part), nc_own[bl]);
+        }
+        ptx::cluster_sync();
+        cur ^= 1;
     }
     if (!settled) {  // still improving after n rounds: a negative cycle, which an optimal start excludes
-        if (tid == 0) { status[qb::kStError] = 1; record_error(kErrRepair); *nrows = 0; }
+        if (crank == 0 && tid == 0) { status[qb::kStError] = 1; record_error(kErrRepair); *nrows = 0; }
         return;
     }
-    // predecessor: lowest a with dist[a] + W[a][b] == dist[b], over the reachable experts only
-    // (4 threads per column take every 4th of them, 8 loads in flight; the minimum over the four)
-    if (tid < kMaxExperts) chg[tid] = (tid < n && dist[tid] != INFINITY) ? 1 : 0;
+    // predecessors of this CTA's columns, over the reachable experts, to CTA 0
+    for (int e = tid; e < kMaxExperts; e += blockDim.x) chg[cur ^ 1][e] = (e < n && dist[cur][e] != INFINITY) ? 1 : 0;
     __syncthreads();
-    compact_flags(chg, n, front, &nfront, wcount);
+    compact_flags(chg[cur ^ 1], n, front, &nfront, wcount);
     const int nr = nfront;
     int pa = 0x7fffffff;
-    if (b < n && dist[b] != INFINITY) {
-        const double db = dist[b];
-        for (int f0 = part; f0 < nr; f0 += 4 * 8) {
-            double w8[8];
-            int a8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int fi = f0 + 4 * u;
-                a8[u] = fi < nr ? front[fi] : -1;
-                w8[u] = a8[u] >= 0 ? W[(int64_t)a8[u] * n + b] : INFINITY;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int aa = a8[u];
-                if (aa >= 0 && aa != b && w8[u] != INFINITY && dist[aa] + w8[u] == db && aa < pa) pa = aa;
-            }
+    if (own && dist[cur][b] != INFINITY) {
+        const double db = dist[cur][b];
+        for (int f = part; f < nr; f += 8) {
+            const int a = front[f];
+            const double w = wsl[a * qb::kRepCols + bl];
+            if (a != b && w != INFINITY && dist[cur][a] + w == db && a < pa) pa = a;
         }
     }
-    part_p[part][b] = pa;
+    part_p[part][bl] = pa;
     __syncthreads();
-    if (part == 0 && b < n) {
+    if (part == 0 && own) {
         int p = 0x7fffffff;
-        for (int q = 0; q < 4; ++q) p = min(p, part_p[q][b]);
-        pred[b] = p == 0x7fffffff ? -1 : p;
+        for (int q = 0; q < 8; ++q) p = min(p, part_p[q][bl]);
+        ptx::st_cluster_s32(ptx::mapa_shared(ptx::smem_u32(&pred[b]), 0u), p == 0x7fffffff ? -1 : p);
     }
-    __syncthreads();
+    ptx::cluster_sync();  // after this, no CTA touches another's shared memory
+    if (crank != 0) return;
+    const double* dd = dist[cur];
     if (tid == 0) {
         int t = -1;
         for (int e = 0; e < n; ++e)
-            if (counts[e] < C && dist[e] != INFINITY && (t < 0 || dist[e] < dist[t])) t = e;
+            if (counts[e] < C && dd[e] != INFINITY && (t < 0 || dd[e] < dd[t])) t = e;
         bool ok = t >= 0;
         int node = t, len = 0;
         int path[kMaxExperts + 1];
@@ -919,9 +926,37 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     __syncthreads();
     if (!any_over) return;
     // the rows of W this move invalidated, in expert order, for the next arc pass
-    if (tid < kMaxExperts) chg[tid] = (tid < n && ((touched[tid >> 5] >> (tid & 31)) & 1u)) ? 1 : 0;
+    for (int e = tid; e < kMaxExperts; e += blockDim.x)
+        chg[cur ^ 1][e] = (e < n && ((touched[e >> 5] >> (e & 31)) & 1u)) ? 1 : 0;
     __syncthreads();
-    compact_flags(chg, n, rows, nrows, wcount);
+    compact_flags(chg[cur ^ 1], n, rows, nrows, wcount);
+}
+
+static cudaError_t launch_repair_step(int n, int64_t C, int k, const double* W, const int32_t* A, int32_t* counts,
+                                      int32_t* topk_idx, int32_t* status, int32_t* rows, int32_t* nrows,
+                                      uint32_t* mem, int64_t words, cudaStream_t stream) {
+    const size_t smem = (size_t)n * qb::kRepCols * sizeof(double);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(qb_repair_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)((size_t)kMaxExperts * qb::kRepCols * sizeof(double)));
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(qb::kRepCtas);
+    cfg.blockDim = dim3(qb::kRepThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = qb::kRepCtas;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qb_repair_step_kernel, n, C, k, W, A, counts, topk_idx, status, rows, nrows, mem,
+                              words);
 }
 
 __global__ void qb_all_rows_kernel(int n, int32_t* __restrict__ rows, int32_t* __restrict__ nrows) {
@@ -1161,9 +1196,9 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
         }
         for (int64_t a = 0; a < moves; ++a) {
             launch_arc(s, m, n, k, topk_idx, w, stream);
-            qb_repair_step_kernel<<<1, qb::kStepThreads, 0, stream>>>(n, C, k, w.W, w.A, final_counts, topk_idx,
-                                                                      w.status, w.rows, w.nrows, w.mem,
-                                                                      (m + 31) / 32);
+            if ((ce = launch_repair_step(n, C, k, w.W, w.A, final_counts, topk_idx, w.status, w.rows, w.nrows,
+                                         w.mem, (m + 31) / 32, stream)) != cudaSuccess)
+                goto cuda_fail;
         }
         qb_info_kernel<<<1, 32, 0, stream>>>(final_counts, n, C, w.status, iters,
                                              iters % 2 ? qb::kStTies1 : qb::kStTies0, info);

@@ -221,6 +221,15 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
     asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
 }
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u8(uint32_t addr, unsigned char v) {
+    asm volatile("st.shared::cluster.u8 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_s32(uint32_t addr, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 // Every thread of every CTA in the cluster arrives (release) and waits (acquire); called
 // convergently by whole warps.
 __device__ __forceinline__ void cluster_sync() {
