@@ -12,21 +12,25 @@
 // Kernels:
 //   qb_row     one warp per token: v = s_i - beta in registers (n/32 values per
 //              lane); the keys that can be among the k + 1 best are found from
-//              the lane maxima and gathered one per lane, then k + 1 rounds of a
-//              warp arg-max give the top-k set, the k-th and (k+1)-th values
-//              (alpha) and a tie flag; the set is written in ascending expert
-//              order and counted per expert.
-//              The first row pass of a call also writes s transposed (sT [n, m]),
-//              so each expert's column is contiguous for the column pass.
-//   qb_col     one CTA per expert column: one sweep keeps the keys of u near
-//              the previous beta_j in shared memory and counts those above;
-//              the C-th and (C+1)-th largest are then selected there (radix
-//              digits over order-preserving uint32 keys). When they are not
-//              inside that window, an exact radix select over the column.
+//              the lane maxima and gathered one per lane, and their ranks give
+//              the top-k set, the k-th and (k+1)-th values (alpha) and a tie
+//              flag (k + 1 rounds of a warp arg-max when that does not apply);
+//              the set is written in ascending expert order and counted per
+//              expert. The first row pass of a SOLVE also writes s transposed
+//              (sT [n, m]) for the column pass's full path.
+//   qb_colwin  the column pass's window sweep, over row-major s by the whole
+//              GPU: per column, the keys of u above a window around the
+//              previous beta_j are counted and those inside are listed.
+//   qb_col     one CTA per expert column: when the C-th largest fell inside
+//              the window, the C-th and (C+1)-th largest come from the column's
+//              list (radix digits over order-preserving uint32 keys); otherwise
+//              an exact radix select over the whole column (from sT, or from s
+//              with stride n).
 //   repair     successive shortest paths on the n-expert graph (exact finish
 //              when the QB iterate is not yet balanced): arc a -> b costs
 //              W[a][b] = min over tokens i holding a but not b of s_ia - s_ib
-//              (fp64, lowest token on ties); one CTA runs Jacobi Bellman-Ford
+//              (fp64, lowest token on ties); an 8-CTA cluster (W's columns
+//              split over the CTAs' shared memory) runs Jacobi Bellman-Ford
 //              rounds from the over-full experts, picks the nearest under-full
 //              expert (lowest index on ties) and moves each arc's argmin
 //              token. The number of moves equals the excess, so the host
@@ -319,42 +323,64 @@ __device__ __forceinline__ unsigned block_sum_u32(unsigned v, unsigned* red) {
 
 namespace qb {
 constexpr int kCandCap = 16384;                         // candidate keys kept in shared memory
+constexpr int kColUnroll = 4;                           // float4 pairs in flight per thread in a column sweep
+constexpr int kGCap = 8192;                             // window candidates kept per column (global lists)
+constexpr int kWinThreads = 256;                        // qb_colwin_kernel block size
+constexpr int kPairCap = 4096;                          // (column, key) pairs buffered per window-sweep CTA
+constexpr int kWinRows = 4;                             // rows in flight per warp in the window sweep
 constexpr size_t kColSmem = 4096 * 4 + kColThreads * 4 + kCandCap * 4;
 // key-space half-widths of the window around the previous beta_j
-constexpr uint32_t kWinDefault = 1u << 18, kWinMin = 1u << 12, kWinMax = 1u << 26;
+// kWinSweep: the sweep's windows are at most this wide
+constexpr uint32_t kWinDefault = 1u << 18, kWinMin = 1u << 12, kWinMax = 1u << 26, kWinSweep = 1u << 21;
 }  // namespace qb
 
-// Visit every key float_key(fp32(col[i] - alpha[i])) of a column, warp-uniformly (f gets
-// ok = false for padding lanes). 16-byte loads, two of each operand in flight per thread,
-// when m is a multiple of 4 (then every column of sT starts on a 16-byte boundary).
+// Visit every key float_key(fp32(col[i * stride] - alpha[i])) of a column, warp-uniformly (f gets
+// ok = false for padding lanes). A contiguous column (stride 1, m a multiple of 4: every column
+// of sT starts on a 16-byte boundary) is read with 16-byte loads, kColUnroll of each operand in
+// flight per thread; a strided one (a column of row-major s) with 8 scalar loads in flight.
 template <typename F>
-__device__ __forceinline__ void for_each_col_key(const float* __restrict__ col, const float* __restrict__ alpha,
-                                                 int64_t m, F&& f) {
+__device__ __forceinline__ void for_each_col_key(const float* __restrict__ col, int64_t stride,
+                                                 const float* __restrict__ alpha, int64_t m, F&& f) {
     const int tid = threadIdx.x, T = blockDim.x;
-    if ((m & 3) == 0) {
+    if (stride == 1 && (m & 3) == 0) {
+        // kColUnroll float4 pairs (column, alpha) per thread in flight before any is used
+        constexpr int U = qb::kColUnroll;
         const float4* c4 = reinterpret_cast<const float4*>(col);
         const float4* a4 = reinterpret_cast<const float4*>(alpha);
         const int64_t m4 = m >> 2;
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int64_t base = 0; base < m4; base += 2 * T) {
-            const int64_t v0 = base + tid, v1 = v0 + T;
-            const bool ok0 = v0 < m4, ok1 = v1 < m4;
-            const float4 c0 = ok0 ? c4[v0] : z, a0 = ok0 ? a4[v0] : z;
-            const float4 c1 = ok1 ? c4[v1] : z, a1 = ok1 ? a4[v1] : z;
-            f(ok0, float_key(__fsub_rn(c0.x, a0.x)));
-            f(ok0, float_key(__fsub_rn(c0.y, a0.y)));
-            f(ok0, float_key(__fsub_rn(c0.z, a0.z)));
-            f(ok0, float_key(__fsub_rn(c0.w, a0.w)));
-            f(ok1, float_key(__fsub_rn(c1.x, a1.x)));
-            f(ok1, float_key(__fsub_rn(c1.y, a1.y)));
-            f(ok1, float_key(__fsub_rn(c1.z, a1.z)));
-            f(ok1, float_key(__fsub_rn(c1.w, a1.w)));
+        for (int64_t base = 0; base < m4; base += U * T) {
+            float4 c[U], a[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t v = base + tid + (int64_t)u * T;
+                c[u] = v < m4 ? c4[v] : z;
+                a[u] = v < m4 ? a4[v] : z;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const bool ok = base + tid + (int64_t)u * T < m4;
+                f(ok, float_key(__fsub_rn(c[u].x, a[u].x)));
+                f(ok, float_key(__fsub_rn(c[u].y, a[u].y)));
+                f(ok, float_key(__fsub_rn(c[u].z, a[u].z)));
+                f(ok, float_key(__fsub_rn(c[u].w, a[u].w)));
+            }
         }
     } else {
-        for (int64_t base = 0; base < m; base += T) {
-            const int64_t i = base + tid;
-            const bool ok = i < m;
-            f(ok, ok ? float_key(__fsub_rn(col[i], alpha[i])) : 0u);
+        constexpr int U = 8;
+        for (int64_t base = 0; base < m; base += U * T) {
+            float c[U], a[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t i = base + tid + (int64_t)u * T;
+                c[u] = i < m ? col[i * stride] : 0.f;
+                a[u] = i < m ? alpha[i] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const bool ok = base + tid + (int64_t)u * T < m;
+                f(ok, ok ? float_key(__fsub_rn(c[u], a[u])) : 0u);
+            }
         }
     }
 }
@@ -424,30 +450,192 @@ __device__ __forceinline__ uint32_t list_max_below(const unsigned* list, unsigne
     return block_max_u32(best, scan);
 }
 
-// beta_j = threshold between the C-th and (C+1)-th largest key of column j of u = fp32(s - alpha).
-// Window pass: one sweep counts the keys above a window around the previous beta_j and keeps
-// the keys inside it in shared memory; when the C-th largest falls inside (the usual case once
-// the iteration settles) both order statistics come from the kept keys. Otherwise the full
-// radix path: a 12-bit digit histogram sweep, a sweep keeping the selected bin's keys (the
-// largest key below the bin is tracked), then the low digits over the kept keys (streamed from
-// global memory if the bin overflows the list). Both paths return the same two keys.
-__global__ void __launch_bounds__(qb::kColThreads)
-qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const float* __restrict__ alpha, int rule,
-              float* __restrict__ beta, const int32_t* __restrict__ counts, int32_t* __restrict__ counts_next,
-              int32_t* __restrict__ status, int iter, int check, uint32_t* __restrict__ win) {
+// Column pass, part 1: the window sweep over row-major s. For every column j the keys of
+// u_ij = fp32(s_ij - alpha_i) are compared with a window [lo_j, hi_j] around the previous beta_j
+// (half-width min(win_j, kWinSweep)): keys above it are counted and keys inside it are appended
+// to column j's candidate list (g_cand[j], kGCap long; the count g_ncand[j] goes on past it).
+// Warp per row, kWinRows rows in flight per warp; lane owns the columns win_col(lane, q) (VEC:
+// 16-byte loads, four adjacent columns per load). The per-key work is branch-free; a row with a
+// key inside some window takes the append path. A CTA buffers its (column, key) pairs in shared
+// memory and reserves room in the global lists once per column at the end; a column whose pairs
+// did not fit is marked full (its count pushed past kGCap), so it takes the exact full path.
+// All SMs sweep together, so the pass runs at the rate of one read of s.
+// check: stop at once when the row pass just made left every count at C (sets kStQbDone).
+template <bool VEC>
+__device__ __forceinline__ int win_col(int lane, int q) {
+    return VEC ? 128 * (q >> 2) + 4 * lane + (q & 3) : lane + 32 * q;
+}
+
+// float_key with -0 folded by an IEEE add of +0 (branch-free; the same key for every float)
+__device__ __forceinline__ uint32_t float_key_nz(float f) {
+    const uint32_t b = __float_as_uint(__fadd_rn(f, 0.0f));
+    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+}
+
+template <int NT, bool VEC>
+__global__ void __launch_bounds__(qb::kWinThreads, 2)
+qb_colwin_kernel(const float* __restrict__ s, int64_t m, int n, int64_t C, const float* __restrict__ alpha,
+                 const float* __restrict__ beta, const uint32_t* __restrict__ win, const int32_t* __restrict__ counts,
+                 int32_t* __restrict__ status, int check, uint32_t* __restrict__ g_above,
+                 uint32_t* __restrict__ g_ncand, uint32_t* __restrict__ g_cand) {
+    static_assert(!VEC || NT % 4 == 0, "vector columns come in fours");
+    constexpr int R = qb::kWinRows;
+    __shared__ uint32_t sabove[kMaxExperts], scnt[kMaxExperts], sbase[kMaxExperts];
+    __shared__ unsigned char sfull[kMaxExperts];
+    __shared__ uint2 pairs[qb::kPairCap];
+    __shared__ unsigned npairs;
+    __shared__ int balanced;
+    const int tid = threadIdx.x, lane = tid & 31;
     if (check) {
-        // stop once the previous row pass is balanced; otherwise CTA 0 prepares the next row pass
         if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
-        __shared__ int balanced;
-        if (threadIdx.x == 0) balanced = 1;
+        if (tid == 0) balanced = 1;
         __syncthreads();
-        for (int e = threadIdx.x; e < n; e += blockDim.x)
+        for (int e = tid; e < n; e += blockDim.x)
             if (counts[e] != C) balanced = 0;
         __syncthreads();
         if (balanced) {
-            if (blockIdx.x == 0 && threadIdx.x == 0) status[qb::kStQbDone] = 1;
+            if (blockIdx.x == 0 && tid == 0) status[qb::kStQbDone] = 1;
             return;
         }
+    }
+    for (int j = tid; j < n; j += blockDim.x) { sabove[j] = 0; scnt[j] = 0; sfull[j] = 0; }
+    if (tid == 0) npairs = 0;
+    // padding columns get the empty window lo = hi = the largest key, which no float reaches
+    uint32_t lo[NT], hi[NT], above[NT];
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+        const int j = win_col<VEC>(lane, q);
+        above[q] = 0;
+        lo[q] = 0xffffffffu;
+        hi[q] = 0xffffffffu;
+        if (j < n) {
+            const uint32_t pk = float_key(beta[j]);
+            uint32_t w = win[j] ? win[j] : qb::kWinDefault;
+            if (w > qb::kWinSweep) w = qb::kWinSweep;
+            lo[q] = pk > w ? pk - w : 0u;
+            hi[q] = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
+        }
+    }
+    __syncthreads();
+    constexpr int WPB = qb::kWinThreads / 32;
+    const int64_t nw = (int64_t)gridDim.x * WPB;
+    for (int64_t i0 = (int64_t)blockIdx.x * WPB + (tid >> 5); i0 < m; i0 += R * nw) {
+        float a[R], v[R][NT];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t i = i0 + r * nw;
+            const bool ok = i < m;
+            a[r] = ok ? alpha[i] : 0.f;
+            if (VEC) {
+#pragma unroll
+                for (int h = 0; h < NT / 4; ++h) {
+                    const int c = 128 * h + 4 * lane;
+                    const float4 t = (ok && c < n) ? *reinterpret_cast<const float4*>(s + i * n + c)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[r][4 * h] = t.x;
+                    v[r][4 * h + 1] = t.y;
+                    v[r][4 * h + 2] = t.z;
+                    v[r][4 * h + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const int j = lane + 32 * q;
+                    v[r][q] = (ok && j < n) ? s[i * n + j] : 0.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const bool ok = i0 + r * nw < m;  // warp-uniform
+            uint32_t inw = 0;
+#pragma unroll
+            for (int q = 0; q < NT; ++q) {
+                const uint32_t key = float_key_nz(__fsub_rn(v[r][q], a[r]));
+                above[q] += (ok && key > hi[q]) ? 1u : 0u;
+                inw |= (ok && key >= lo[q] && key <= hi[q]) ? (1u << q) : 0u;
+            }
+            if (__any_sync(0xffffffffu, inw != 0)) {
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    if ((inw >> q) & 1u) {
+                        const int j = win_col<VEC>(lane, q);
+                        const unsigned p = atomicAdd(&npairs, 1u);
+                        if (p < (unsigned)qb::kPairCap)
+                            pairs[p] = make_uint2((uint32_t)j, float_key_nz(__fsub_rn(v[r][q], a[r])));
+                        else
+                            sfull[j] = 1;
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+        const int j = win_col<VEC>(lane, q);
+        if (j < n && above[q]) atomicAdd(&sabove[j], above[q]);
+    }
+    __syncthreads();
+    const unsigned np = min(npairs, (unsigned)qb::kPairCap);
+    for (unsigned p = tid; p < np; p += blockDim.x) atomicAdd(&scnt[pairs[p].x], 1u);
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x) {
+        if (sabove[j]) atomicAdd(&g_above[j], sabove[j]);
+        // a full column: its count goes past kGCap, its pairs are not stored
+        const uint32_t add = sfull[j] ? scnt[j] + (uint32_t)qb::kGCap + 1u : scnt[j];
+        sbase[j] = add ? atomicAdd(&g_ncand[j], add) : 0u;
+        if (sfull[j]) sbase[j] = (uint32_t)qb::kGCap;
+        scnt[j] = 0;
+    }
+    __syncthreads();
+    for (unsigned p = tid; p < np; p += blockDim.x) {
+        const uint2 pr = pairs[p];
+        const uint32_t pos = sbase[pr.x] + atomicAdd(&scnt[pr.x], 1u);
+        if (pos < (uint32_t)qb::kGCap) g_cand[(int64_t)pr.x * qb::kGCap + pos] = pr.y;
+    }
+}
+
+// The want-th and (want+1)-th largest keys (1-based, want + 1 <= ncand) of a short shared list,
+// by ranks: a key holds rank r when fewer than r keys are above it and at least r are at or
+// above it. One candidate per thread (ncand <= blockDim.x), four list keys per shared load.
+__device__ __forceinline__ void rank_select2(const unsigned* list, unsigned ncand, int64_t want, uint32_t* out) {
+    const unsigned c = threadIdx.x;
+    if (c < ncand) {
+        const uint32_t kc = list[c];
+        unsigned g = 0, e = 0;
+        const unsigned n4 = ncand & ~3u;
+        for (unsigned x = 0; x < n4; x += 4) {
+            const uint4 q = *reinterpret_cast<const uint4*>(list + x);
+            g += (q.x > kc) + (q.y > kc) + (q.z > kc) + (q.w > kc);
+            e += (q.x == kc) + (q.y == kc) + (q.z == kc) + (q.w == kc);
+        }
+        for (unsigned x = n4; x < ncand; ++x) {
+            g += list[x] > kc;
+            e += list[x] == kc;
+        }
+        if ((int64_t)g < want && want <= (int64_t)(g + e)) out[0] = kc;
+        if ((int64_t)g < want + 1 && want + 1 <= (int64_t)(g + e)) out[1] = kc;
+    }
+    __syncthreads();
+}
+
+// Column pass, part 2: beta_j = threshold between the C-th and (C+1)-th largest key of column j
+// of u = fp32(s - alpha). When both fell inside the window of part 1 (the usual case once the
+// iteration settles) they come from the column's candidate list, copied into shared memory:
+// by ranks when the list is short, else by radix digits. Otherwise the full radix path over the
+// column: a 12-bit digit histogram sweep, a sweep keeping the selected bin's keys (the largest
+// key below the bin is tracked), then the low digits over the kept keys (streamed from global
+// memory if the bin overflows the list). The column is read from sT (contiguous) when it
+// exists, else from s (stride n). Every path returns the same two keys. Part 1's counters are
+// cleared for the next pass. check: nothing to do once kStQbDone is set; otherwise CTA 0
+// prepares the next row pass.
+__global__ void __launch_bounds__(qb::kColThreads)
+qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t m, int n, int64_t C,
+              const float* __restrict__ alpha, int rule, float* __restrict__ beta, int32_t* __restrict__ counts_next,
+              int32_t* __restrict__ status, int iter, int check, uint32_t* __restrict__ win,
+              uint32_t* __restrict__ g_above, uint32_t* __restrict__ g_ncand, const uint32_t* __restrict__ g_cand) {
+    if (check) {
+        if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
         if (blockIdx.x == 0) {
             for (int e = threadIdx.x; e < n; e += blockDim.x) counts_next[e] = 0;
             if (threadIdx.x == 0) {
@@ -461,45 +649,39 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
     unsigned* scan = hist + 4096;              // blockDim
     unsigned* cand = scan + qb::kColThreads;   // kCandCap
     __shared__ unsigned s_ncand;
+    __shared__ uint32_t s_sel[2];
     const int tid = threadIdx.x, T = blockDim.x;
     const int j = blockIdx.x;
-    const float* col = sT + (int64_t)j * m;
+    const float* col = sT ? sT + (int64_t)j * m : s + j;
+    const int64_t stride = sT ? 1 : n;
 
-    // ---- window pass around the previous beta_j (only this CTA reads or writes beta[j])
     const uint32_t pk = float_key(beta[j]);
-    const uint32_t w = win[j] ? win[j] : qb::kWinDefault;
-    const uint32_t lo = pk > w ? pk - w : 0u, hi = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
-    if (tid == 0) s_ncand = 0;
+    const unsigned above = __ldcg(&g_above[j]);
+    unsigned ncand = __ldcg(&g_ncand[j]);
+    // both order statistics inside the window
+    const bool hit = ncand <= (unsigned)qb::kGCap && (int64_t)above < C && (int64_t)above + ncand >= C + 1;
+    if (hit)
+        for (unsigned c = tid; c < ncand; c += T) cand[c] = __ldcg(&g_cand[(int64_t)j * qb::kGCap + c]);
     __syncthreads();
-    unsigned above = 0;
-    uint32_t below = 0;
-    for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
-        above += (ok && key > hi) ? 1u : 0u;
-        if (ok && key < lo && key > below) below = key;
-        warp_append(cand, &s_ncand, ok && key >= lo && key <= hi, key);
-    });
-    above = block_sum_u32(above, scan);
-    below = block_max_u32(below, scan);
-    unsigned ncand = s_ncand;
-    const bool hit = ncand <= (unsigned)qb::kCandCap && (int64_t)above < C && (int64_t)above + ncand >= C;
+    if (tid == 0) { g_above[j] = 0; g_ncand[j] = 0; }
 
     uint32_t akey, bkey;
-    if (hit) {
+    if (hit && ncand <= (unsigned)T) {
+        rank_select2(cand, ncand, C - (int64_t)above, s_sel);
+        akey = s_sel[0];
+        bkey = s_sel[1];
+    } else if (hit) {
         unsigned mult;
         int64_t greater;
         select_in_list(cand, ncand, C - (int64_t)above, hist, scan, &akey, &mult, &greater);
         greater += above;
-        if (greater + (int64_t)mult >= C + 1) {
-            bkey = akey;
-        } else {
-            const uint32_t best = list_max_below(cand, ncand, akey, scan);
-            bkey = best ? best : below;
-        }
+        bkey = greater + (int64_t)mult >= C + 1 ? akey : list_max_below(cand, ncand, akey, scan);
     } else {
         // ---- full radix path
+        uint32_t below = 0;
         for (int b = tid; b < 4096; b += T) hist[b] = 0;
         __syncthreads();
-        for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) { warp_hist_add(hist, ok, key >> 20); });
+        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) { warp_hist_add(hist, ok, key >> 20); });
         __syncthreads();
         int sel1;
         int64_t want1;
@@ -507,8 +689,7 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
         block_select_bin(hist, 4096, C, scan, &sel1, &want1, &cnt1);
         if (tid == 0) s_ncand = 0;
         __syncthreads();
-        below = 0;
-        for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
             const uint32_t d = key >> 20;
             if (ok && d < (uint32_t)sel1 && key > below) below = key;
             warp_append(cand, &s_ncand, ok && d == (uint32_t)sel1, key);
@@ -533,7 +714,7 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
             unsigned cnt2, cnt3;
             for (int b = tid; b < 4096; b += T) hist[b] = 0;
             __syncthreads();
-            for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+            for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
                 warp_hist_add(hist, ok && (key >> 20) == (uint32_t)sel1, (key >> 8) & 0xfffu);
             });
             __syncthreads();
@@ -541,7 +722,7 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
             const uint32_t pre2 = ((uint32_t)sel1 << 20) | ((uint32_t)sel2 << 8);
             for (int b = tid; b < 256; b += T) hist[b] = 0;
             __syncthreads();
-            for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+            for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
                 warp_hist_add(hist, ok && (key & 0xffffff00u) == pre2, key & 0xffu);
             });
             __syncthreads();
@@ -552,7 +733,7 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
                 bkey = akey;
             } else {
                 uint32_t best = 0;
-                for_each_col_key(col, alpha, m, [&](bool ok, uint32_t key) {
+                for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
                     if (ok && (key >> 20) == (uint32_t)sel1 && key < akey && key > best) best = key;
                 });
                 best = block_max_u32(best, scan);
@@ -563,10 +744,10 @@ qb_col_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t C, const f
     if (tid == 0) {
         const float bnew = qb_threshold(key_float(akey), key_float(bkey), rule);
         beta[j] = bnew;
-        // next window: centred on the new beta, as wide as this move plus the gap it splits
+        // next window: centred on the new beta, twice as wide as this move, plus the gap it splits
         const uint32_t nk = float_key(bnew);
         const uint64_t dist = nk > pk ? (uint64_t)(nk - pk) : (uint64_t)(pk - nk);
-        uint64_t wn = dist + (uint64_t)(akey - bkey) + qb::kWinMin;
+        uint64_t wn = 2 * dist + (uint64_t)(akey - bkey) + qb::kWinMin;
         if (wn > qb::kWinMax) wn = qb::kWinMax;
         win[j] = (uint32_t)wn;
     }
@@ -989,6 +1170,9 @@ struct QBWorkspace {
     double* Wp;      // [n][kArcSlices][n] per-slice partial arc costs
     int32_t* Ap;     // [n][kArcSlices][n] their tokens
     int32_t* arc_tickets;  // [n] slices done per row (re-armed by the folding slice)
+    uint32_t* g_above;     // [n] column pass: keys above the window (cleared by the select kernel)
+    uint32_t* g_ncand;     // [n] column pass: keys inside the window
+    uint32_t* g_cand;      // [n][kGCap] column pass: the keys inside the window
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -1011,6 +1195,8 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     p = take(sizeof(double) * (size_t)n * qb::kArcSlices * n);  if (w) w->Wp = (double*)p;
     p = take(sizeof(int32_t) * (size_t)n * qb::kArcSlices * n); if (w) w->Ap = (int32_t*)p;
     p = take(sizeof(int32_t) * (size_t)n);              if (w) w->arc_tickets = (int32_t*)p;
+    p = take(sizeof(uint32_t) * (size_t)2 * n);         if (w) { w->g_above = (uint32_t*)p; w->g_ncand = w->g_above + n; }
+    p = take(sizeof(uint32_t) * (size_t)n * qb::kGCap); if (w) w->g_cand = (uint32_t*)p;
     return off;
 }
 
@@ -1035,6 +1221,37 @@ static void launch_row(const float* s, int64_t m, int n, int k, const float* bet
     else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
     else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
     else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+}
+
+template <int NT, bool VEC>
+static void launch_colwin_t(const float* s, int64_t m, int n, int64_t C, const QBWorkspace& w, const float* beta,
+                            const int32_t* counts, int check, cudaStream_t stream) {
+    constexpr int WPB = qb::kWinThreads / 32;
+    int64_t blocks = (m + qb::kWinRows * WPB - 1) / (qb::kWinRows * WPB);
+    if (blocks > (int64_t)kNumSMs * 2) blocks = (int64_t)kNumSMs * 2;
+    if (blocks < 1) blocks = 1;
+    qb_colwin_kernel<NT, VEC><<<(unsigned)blocks, qb::kWinThreads, 0, stream>>>(
+        s, m, n, C, w.alpha, beta, w.win, counts, w.status, check, w.g_above, w.g_ncand, w.g_cand);
+}
+
+// The column pass: the window sweep over s, then one select CTA per column. sT: s transposed
+// (SOLVE), read by the select kernel's full path when the window missed; nullptr: that path
+// reads the column from s with stride n.
+static void launch_col(const float* s, const float* sT, int64_t m, int n, int64_t C, const QBWorkspace& w, int rule,
+                       float* beta, const int32_t* counts, int32_t* counts_next, int iter, int check,
+                       cudaStream_t stream) {
+    // 16-byte rows when every row of s starts on a 16-byte boundary
+    const bool vec = n % 4 == 0 && (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    if (vec) {
+        if (n <= 128) launch_colwin_t<4, true>(s, m, n, C, w, beta, counts, check, stream);
+        else launch_colwin_t<8, true>(s, m, n, C, w, beta, counts, check, stream);
+    } else if (n <= 32) launch_colwin_t<1, false>(s, m, n, C, w, beta, counts, check, stream);
+    else if (n <= 64) launch_colwin_t<2, false>(s, m, n, C, w, beta, counts, check, stream);
+    else if (n <= 128) launch_colwin_t<4, false>(s, m, n, C, w, beta, counts, check, stream);
+    else launch_colwin_t<8, false>(s, m, n, C, w, beta, counts, check, stream);
+    qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(s, sT, m, n, C, w.alpha, rule, beta, counts_next,
+                                                                w.status, iter, check, w.win, w.g_above, w.g_ncand,
+                                                                w.g_cand);
 }
 
 template <int NT>
@@ -1144,10 +1361,11 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto cuda_fail;
     if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
     if ((ce = cudaMemsetAsync(w.win, 0, sizeof(uint32_t) * n, stream)) != cudaSuccess) goto cuda_fail;
+    if ((ce = cudaMemsetAsync(w.g_above, 0, sizeof(uint32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
     if (mode == MOE_QB_STEP) {
-        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, w.sT, stream);
-        qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(w.sT, m, n, C, w.alpha, rule, beta, w.counts,
-                                                                    w.counts + n, w.status, 0, 0, w.win);
+        // one pass each; a window miss reads its column from s (no transposed copy)
+        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
+        launch_col(s, nullptr, m, n, C, w, rule, beta, w.counts, w.counts + n, 0, 0, stream);
         qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
         if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
         return MOE_OK;
@@ -1162,9 +1380,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
                 launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, cnt, w.status,
                            u % 2 ? qb::kStTies1 : qb::kStTies0, 1, u == 0 ? w.sT : nullptr, stream);
                 if (u < max_iters)
-                    qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(
-                        w.sT, m, n, C, w.alpha, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, w.status, u, 1,
-                        w.win);
+                    launch_col(s, w.sT, m, n, C, w, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, u, 1, stream);
             }
             if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
             if ((ce = cudaMemcpyAsync(hstatus, w.status, sizeof(hstatus), cudaMemcpyDeviceToHost, stream)) !=

@@ -99,7 +99,7 @@ class MoELayer:
         elif i == 1:
             moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"], stream=st)
         elif i == 2:
-            if not self.gather:  # otherwise the FFN gathers its rows from x
+            if self.uses_dispatch():  # otherwise the FFN gathers its rows from x
                 moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
         elif i == 3:
             if self.ffn_combine:
@@ -148,6 +148,10 @@ class MoELayer:
         st.wait_event(self._join)
         return self.buf["y"]
 
+    def uses_dispatch(self) -> bool:
+        """Whether the forward forms xbuf with moe_dispatch (the fused-combine FFN always reads xbuf)."""
+        return self.ffn_combine or not self.gather
+
     def capture(self, x: torch.Tensor) -> None:
         """Record forward(x) as one CUDA graph, and each stage into a graph of its own for per-stage
         timing (x's address is baked in). The first forward runs eagerly so one-time host set-up
@@ -156,7 +160,7 @@ class MoELayer:
         torch.cuda.synchronize()
         self.graphs = []
         for i in range(len(self.STAGES)):
-            if (i == 4 and self.ffn_combine) or (i == 2 and self.gather):  # done inside the FFN stage
+            if (i == 4 and self.ffn_combine) or (i == 2 and not self.uses_dispatch()):  # done inside the FFN stage
                 self.graphs.append(None)
                 continue
             g = torch.cuda.CUDAGraph()
@@ -210,19 +214,19 @@ class MoELayer:
 
     def launches_per_forward(self) -> int:
         """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection
-        and the finish kernel; else 1),
-        capacity 2 (count + scan, assign), dispatch 1, FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
-        combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus one
-        launch for the dropped tokens' rows."""
+        and the finish kernel; else 1), capacity 2
+        (count + scan, assign), dispatch 1 (0 when the FFN gathers its rows from x), FFN (bf16: one fused
+        launch, after a memset of its counters; fp32: 2), combine 1, statistics 1. With one pick per token
+        in bf16 the combine is the FFN's epilogue plus one launch for the dropped tokens' rows."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
         router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
-        ffn = 1 if bf16 else 2
-        if self.ffn_combine:  # the FFN (gathering its rows) with the combine in its epilogue + the dropped rows
-            return router + 2 + 0 + 2 + 0 + 1
-        if self.gather:       # the FFN gathering its rows, then the combine
-            return router + 2 + 0 + 1 + 1 + 1
-        return router + 2 + 1 + ffn + 1 + 1
+        dispatch = 1 if self.uses_dispatch() else 0
+        if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped rows
+            ffn, combine = 2, 0
+        else:
+            ffn, combine = (1 if bf16 else 2), 1
+        return router + 2 + dispatch + ffn + combine + 1
 
 
 def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:
