@@ -628,12 +628,25 @@ __device__ __forceinline__ void rank_select2(const unsigned* list, unsigned ncan
 // memory if the bin overflows the list). The column is read from sT (contiguous) when it
 // exists, else from s (stride n). Every path returns the same two keys. Part 1's counters are
 // cleared for the next pass. check: nothing to do once kStQbDone is set; otherwise CTA 0
-// prepares the next row pass.
+// prepares the next row pass. info (one STEP): CTA 0 also writes the call's info words from the
+// row pass's counts.
 __global__ void __launch_bounds__(qb::kColThreads)
 qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t m, int n, int64_t C,
               const float* __restrict__ alpha, int rule, float* __restrict__ beta, int32_t* __restrict__ counts_next,
               int32_t* __restrict__ status, int iter, int check, uint32_t* __restrict__ win,
-              uint32_t* __restrict__ g_above, uint32_t* __restrict__ g_ncand, const uint32_t* __restrict__ g_cand) {
+              uint32_t* __restrict__ g_above, uint32_t* __restrict__ g_ncand, const uint32_t* __restrict__ g_cand,
+              const int32_t* __restrict__ info_counts, int tie_slot, int32_t* __restrict__ info) {
+    if (info && blockIdx.x == 0 && threadIdx.x < 32) {
+        int64_t ex = 0;
+        for (int e = threadIdx.x; e < n; e += 32) ex += info_counts[e] > C ? info_counts[e] - C : 0;
+        for (int o = 16; o > 0; o >>= 1) ex += __shfl_xor_sync(0xffffffffu, ex, o);
+        if (threadIdx.x == 0) {
+            info[0] = 1;
+            info[1] = status[qb::kStAugments];
+            info[2] = (int32_t)ex;
+            info[3] = status[tie_slot];
+        }
+    }
     if (check) {
         if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
         if (blockIdx.x == 0) {
@@ -958,7 +971,7 @@ constexpr int kRepCols = 32;      // columns of W per CTA (n <= 256)
 __global__ void __launch_bounds__(qb::kRepThreads, 1)
 qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, const int32_t* __restrict__ A,
                       int32_t* __restrict__ counts, int32_t* __restrict__ topk_idx, int32_t* __restrict__ status,
-                      int32_t* __restrict__ rows, int32_t* __restrict__ nrows, uint32_t* __restrict__ mem,
+                      int32_t* __restrict__ moves, int32_t* __restrict__ nmoves, uint32_t* __restrict__ mem,
                       int64_t words) {
     extern __shared__ double wsl[];  // [n][32]: this CTA's columns of W
     __shared__ double dist[2][kMaxExperts];
@@ -970,7 +983,6 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     __shared__ int pred[kMaxExperts];
     __shared__ int front[kMaxExperts], nfront, wcount[kMaxExperts / 32];
     __shared__ int any_over;
-    __shared__ uint32_t touched[kMaxExperts / 32];
     const int tid = threadIdx.x, bl = tid & 31, part = tid >> 5;
     const uint32_t crank = ptx::cluster_ctarank();
     const int b = (int)crank * qb::kRepCols + bl;
@@ -982,7 +994,6 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         wsl[q] = j < n ? W[(int64_t)a * n + j] : INFINITY;
     }
     if (tid == 0) any_over = 0;
-    if (tid < kMaxExperts / 32) touched[tid] = 0;
     __syncthreads();
     for (int e = tid; e < kMaxExperts; e += blockDim.x) {
         const bool over = e < n && counts[e] > C;
@@ -995,7 +1006,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     }
     __syncthreads();
     if (!any_over) {  // the same counts in every CTA: all return here together
-        if (crank == 0 && tid == 0) { status[qb::kStDone] = 1; *nrows = 0; }
+        if (crank == 0 && tid == 0) { status[qb::kStDone] = 1; nmoves[0] = 0; nmoves[1] = 0; }
         return;
     }
     ptx::cluster_sync();  // every CTA's buffers are initialised before any remote write
@@ -1033,7 +1044,12 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         cur ^= 1;
     }
     if (!settled) {  // still improving after n rounds: a negative cycle, which an optimal start excludes
-        if (crank == 0 && tid == 0) { status[qb::kStError] = 1; record_error(kErrRepair); *nrows = 0; }
+        if (crank == 0 && tid == 0) {
+            status[qb::kStError] = 1;
+            record_error(kErrRepair);
+            nmoves[0] = 0;
+            nmoves[1] = 0;
+        }
         return;
     }
     // predecessors of this CTA's columns, over the reachable experts, to CTA 0
@@ -1072,6 +1088,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
             while (pred[node] >= 0 && len <= n) { node = pred[node]; path[len++] = node; }
             ok = len <= n && counts[node] > C;
         }
+        int nm = 0;
         for (int p = len - 1; ok && p > 0; --p) {
             const int a = path[p], bb = path[p - 1];
             const int32_t i = A[(int64_t)a * n + bb];
@@ -1082,39 +1099,36 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
             for (int r = 0; r < k; ++r) {
                 if (row[r] == a) pos = r;
                 if (row[r] == bb) hasb = true;
-                touched[row[r] >> 5] |= 1u << (row[r] & 31);  // the token's old set
             }
             if (pos < 0 || hasb) { ok = false; break; }
-            touched[bb >> 5] |= 1u << (bb & 31);
             mem[(int64_t)a * words + (i >> 5)] &= ~(1u << (i & 31));
             mem[(int64_t)bb * words + (i >> 5)] |= 1u << (i & 31);
             int r = pos;
             row[r] = bb;
             while (r > 0 && row[r - 1] > row[r]) { const int t2 = row[r - 1]; row[r - 1] = row[r]; row[r] = t2; --r; }
             while (r + 1 < k && row[r + 1] < row[r]) { const int t2 = row[r + 1]; row[r + 1] = row[r]; row[r] = t2; ++r; }
+            // the move, for the arc update that follows: token i went from a to bb
+            moves[3 * nm] = i;
+            moves[3 * nm + 1] = a;
+            moves[3 * nm + 2] = bb;
+            ++nm;
         }
         if (!ok) {
             status[qb::kStError] = 1;
             record_error(kErrRepair);
-            *nrows = 0;
+            nm = 0;
         } else {
             counts[node] -= 1;
             counts[t] += 1;
             status[qb::kStAugments] += 1;
         }
-        any_over = ok;
+        nmoves[0] = nm;
+        nmoves[1] = 0;  // entries queued for recomputation by the next arc update
     }
-    __syncthreads();
-    if (!any_over) return;
-    // the rows of W this move invalidated, in expert order, for the next arc pass
-    for (int e = tid; e < kMaxExperts; e += blockDim.x)
-        chg[cur ^ 1][e] = (e < n && ((touched[e >> 5] >> (e & 31)) & 1u)) ? 1 : 0;
-    __syncthreads();
-    compact_flags(chg[cur ^ 1], n, rows, nrows, wcount);
 }
 
 static cudaError_t launch_repair_step(int n, int64_t C, int k, const double* W, const int32_t* A, int32_t* counts,
-                                      int32_t* topk_idx, int32_t* status, int32_t* rows, int32_t* nrows,
+                                      int32_t* topk_idx, int32_t* status, int32_t* moves, int32_t* nmoves,
                                       uint32_t* mem, int64_t words, cudaStream_t stream) {
     const size_t smem = (size_t)n * qb::kRepCols * sizeof(double);
     static bool attr = false;
@@ -1136,8 +1150,117 @@ static cudaError_t launch_repair_step(int n, int64_t C, int k, const double* W, 
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, qb_repair_step_kernel, n, C, k, W, A, counts, topk_idx, status, rows, nrows, mem,
-                              words);
+    return cudaLaunchKernelEx(&cfg, qb_repair_step_kernel, n, C, k, W, A, counts, topk_idx, status, moves, nmoves,
+                              mem, words);
+}
+
+// Arc costs after a repair move, updated in place instead of rebuilding rows. An entry
+// W[x][y] is a minimum over the eligible tokens (holding x, not y), taken on (cost, token). A
+// move changes the eligibility of its moved tokens only: a token that became eligible enters
+// the minimum; a token that stopped being eligible changes the entry only if it was the
+// recorded argmin, and those entries are queued for recomputation from the membership
+// bitmaps. A minimum over a set that lost a token other than its argmin is unchanged, so the
+// result equals the rebuilt rows bit for bit. CTA x takes row x, thread y column y; the moved
+// tokens' expert sets after the move come from topk_idx (before it: bb replaced by a).
+__global__ void __launch_bounds__(kMaxExperts)
+qb_arc_inc_kernel(const float* __restrict__ s, int n, int k, const int32_t* __restrict__ topk_idx,
+                  const int32_t* __restrict__ moves, int32_t* __restrict__ nmoves, const int32_t* __restrict__ status,
+                  double* __restrict__ W, int32_t* __restrict__ A, int32_t* __restrict__ rec) {
+    if (status[qb::kStError] || status[qb::kStDone]) return;
+    const int L = nmoves[0];
+    if (L <= 0) return;
+    __shared__ uint32_t nset[kMaxExperts][kMaxExperts / 32];
+    __shared__ int32_t mv[kMaxExperts][3];
+    const int tid = threadIdx.x;
+    for (int q = tid; q < L * (kMaxExperts / 32); q += blockDim.x) nset[q / (kMaxExperts / 32)][q % (kMaxExperts / 32)] = 0;
+    for (int q = tid; q < 3 * L; q += blockDim.x) mv[q / 3][q % 3] = moves[q];
+    __syncthreads();
+    for (int q = tid; q < L * k; q += blockDim.x) {
+        const int p = q / k;
+        const int e = topk_idx[(int64_t)mv[p][0] * k + (q - p * k)];
+        atomicOr(&nset[p][e >> 5], 1u << (e & 31));
+    }
+    __syncthreads();
+    const int x = blockIdx.x, y = tid;
+    if (y >= n || x == y) return;
+    const int64_t at = (int64_t)x * n + y;
+    double w = W[at];
+    int32_t t = A[at];
+    bool re = false, changed = false;
+    for (int p = 0; p < L; ++p) {
+        const int32_t i = mv[p][0];
+        const int a = mv[p][1], bb = mv[p][2];
+        const bool xn = (nset[p][x >> 5] >> (x & 31)) & 1u, yn = (nset[p][y >> 5] >> (y & 31)) & 1u;
+        const bool xo = x == a ? true : (x == bb ? false : xn);
+        const bool yo = y == a ? true : (y == bb ? false : yn);
+        const bool el_new = xn && !yn, el_old = xo && !yo;
+        if (el_old && !el_new) {
+            if (t == i) re = true;
+        } else if (el_new && !el_old) {
+            const double c = (double)s[(int64_t)i * n + x] - (double)s[(int64_t)i * n + y];
+            if (c < w || (c == w && i < t)) { w = c; t = i; changed = true; }
+        }
+    }
+    if (re) rec[atomicAdd(&nmoves[1], 1)] = (int32_t)at;
+    else if (changed) { W[at] = w; A[at] = t; }
+}
+
+// The queued entries, recomputed from the membership bitmaps: W[x][y] = min over tokens in
+// mem[x] and not in mem[y] of s_tx - s_ty (fp64, lowest token on ties). One CTA per entry.
+__global__ void __launch_bounds__(256)
+qb_arc_recompute_kernel(const float* __restrict__ s, int64_t m, int n, const uint32_t* __restrict__ mem,
+                        int64_t words, const int32_t* __restrict__ nmoves, const int32_t* __restrict__ rec,
+                        const int32_t* __restrict__ status, double* __restrict__ W, int32_t* __restrict__ A) {
+    if (status[qb::kStError] || status[qb::kStDone]) return;
+    const int nrec = nmoves[1];
+    __shared__ double rw[8];
+    __shared__ int32_t rt[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = blockIdx.x; e < nrec; e += gridDim.x) {
+        const int32_t at = rec[e];
+        const int x = at / n, y = at - x * n;
+        const uint32_t* mx = mem + (int64_t)x * words;
+        const uint32_t* my = mem + (int64_t)y * words;
+        double best = INFINITY;
+        int32_t arg = 0x7fffffff;
+        for (int64_t w0 = 0; w0 < words; w0 += 4 * (int64_t)blockDim.x) {
+            uint32_t bits[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t wi = w0 + tid + (int64_t)u * blockDim.x;
+                bits[u] = wi < words ? (mx[wi] & ~my[wi]) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t wi = w0 + tid + (int64_t)u * blockDim.x;
+                uint32_t b = bits[u];
+                while (b) {
+                    const int bit = __ffs(b) - 1;
+                    b &= b - 1;
+                    const int64_t ti = (wi << 5) + bit;
+                    if (ti >= m) break;
+                    const double c = (double)s[ti * n + x] - (double)s[ti * n + y];
+                    if (c < best || (c == best && (int32_t)ti < arg)) { best = c; arg = (int32_t)ti; }
+                }
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int32_t oa = __shfl_xor_sync(0xffffffffu, arg, o);
+            if (ob < best || (ob == best && oa < arg)) { best = ob; arg = oa; }
+        }
+        if (lane == 0) { rw[warp] = best; rt[warp] = arg; }
+        __syncthreads();
+        if (tid == 0) {
+            double bw = INFINITY;
+            int32_t ba = 0x7fffffff;
+            for (int q = 0; q < (int)(blockDim.x >> 5); ++q)
+                if (rw[q] < bw || (rw[q] == bw && rt[q] < ba)) { bw = rw[q]; ba = rt[q]; }
+            W[at] = bw;
+            A[at] = bw == INFINITY ? -1 : ba;
+        }
+        __syncthreads();
+    }
 }
 
 __global__ void qb_all_rows_kernel(int n, int32_t* __restrict__ rows, int32_t* __restrict__ nrows) {
@@ -1173,6 +1296,9 @@ struct QBWorkspace {
     uint32_t* g_above;     // [n] column pass: keys above the window (cleared by the select kernel)
     uint32_t* g_ncand;     // [n] column pass: keys inside the window
     uint32_t* g_cand;      // [n][kGCap] column pass: the keys inside the window
+    int32_t* moves;        // [n][3] the last repair move: token, from, to per hop
+    int32_t* nmoves;       // [2] hops of the last move, entries queued for recomputation
+    int32_t* rec;          // [n * n] queued entries x * n + y
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -1184,19 +1310,27 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     char* p;
     p = take(sizeof(float) * (size_t)m * n);            if (w) w->sT = (float*)p;
     p = take(sizeof(float) * (size_t)m);                if (w) w->alpha = (float*)p;
-    p = take(sizeof(int32_t) * (size_t)2 * n);          if (w) w->counts = (int32_t*)p;
-    p = take(sizeof(int32_t) * qb::kStWords);           if (w) w->status = (int32_t*)p;
+    // the words every call clears, in one block: status, counts (2 n), win (n), g_above (n), g_ncand (n)
+    p = take(sizeof(int32_t) * ((size_t)qb::kStWords + 5 * (size_t)n));
+    if (w) {
+        w->status = (int32_t*)p;
+        w->counts = w->status + qb::kStWords;
+        w->win = (uint32_t*)(w->counts + 2 * n);
+        w->g_above = w->win + n;
+        w->g_ncand = w->g_above + n;
+    }
     p = take(sizeof(double) * (size_t)n * n);           if (w) w->W = (double*)p;
     p = take(sizeof(int32_t) * (size_t)n * n);          if (w) w->A = (int32_t*)p;
     p = take(sizeof(int32_t) * (size_t)n);              if (w) w->rows = (int32_t*)p;
     p = take(sizeof(int32_t));                          if (w) w->nrows = (int32_t*)p;
     p = take(sizeof(uint32_t) * (size_t)n * (size_t)((m + 31) / 32)); if (w) w->mem = (uint32_t*)p;
-    p = take(sizeof(uint32_t) * (size_t)n);             if (w) w->win = (uint32_t*)p;
     p = take(sizeof(double) * (size_t)n * qb::kArcSlices * n);  if (w) w->Wp = (double*)p;
     p = take(sizeof(int32_t) * (size_t)n * qb::kArcSlices * n); if (w) w->Ap = (int32_t*)p;
     p = take(sizeof(int32_t) * (size_t)n);              if (w) w->arc_tickets = (int32_t*)p;
-    p = take(sizeof(uint32_t) * (size_t)2 * n);         if (w) { w->g_above = (uint32_t*)p; w->g_ncand = w->g_above + n; }
     p = take(sizeof(uint32_t) * (size_t)n * qb::kGCap); if (w) w->g_cand = (uint32_t*)p;
+    p = take(sizeof(int32_t) * 3 * (size_t)(n + 1));    if (w) w->moves = (int32_t*)p;
+    p = take(sizeof(int32_t) * 2);                      if (w) w->nmoves = (int32_t*)p;
+    p = take(sizeof(int32_t) * (size_t)n * n);          if (w) w->rec = (int32_t*)p;
     return off;
 }
 
@@ -1239,7 +1373,7 @@ static void launch_colwin_t(const float* s, int64_t m, int n, int64_t C, const Q
 // reads the column from s with stride n.
 static void launch_col(const float* s, const float* sT, int64_t m, int n, int64_t C, const QBWorkspace& w, int rule,
                        float* beta, const int32_t* counts, int32_t* counts_next, int iter, int check,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, int32_t* info = nullptr) {
     // 16-byte rows when every row of s starts on a 16-byte boundary
     const bool vec = n % 4 == 0 && (reinterpret_cast<uintptr_t>(s) & 15) == 0;
     if (vec) {
@@ -1251,7 +1385,7 @@ static void launch_col(const float* s, const float* sT, int64_t m, int n, int64_
     else launch_colwin_t<8, false>(s, m, n, C, w, beta, counts, check, stream);
     qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(s, sT, m, n, C, w.alpha, rule, beta, counts_next,
                                                                 w.status, iter, check, w.win, w.g_above, w.g_ncand,
-                                                                w.g_cand);
+                                                                w.g_cand, counts, qb::kStTies0, info);
 }
 
 template <int NT>
@@ -1274,6 +1408,15 @@ static void launch_arc(const float* s, int64_t m, int n, int k, const int32_t* t
     else if (n <= 128) launch_arc_t<4>(s, m, n, k, topk_idx, w, stream);
     else launch_arc_t<8>(s, m, n, k, topk_idx, w, stream);
 }
+
+static void launch_arc_update(const float* s, int64_t m, int n, int k, const int32_t* topk_idx, const QBWorkspace& w,
+                              cudaStream_t stream) {
+    qb_arc_inc_kernel<<<n, kMaxExperts, 0, stream>>>(s, n, k, topk_idx, w.moves, w.nmoves, w.status, w.W, w.A,
+                                                     w.rec);
+    qb_arc_recompute_kernel<<<kNumSMs * 4, 256, 0, stream>>>(s, m, n, w.mem, (m + 31) / 32, w.nmoves, w.rec,
+                                                             w.status, w.W, w.A);
+}
+
 
 // SignSGD on beta: count_j = #{i : fp32(s_ij - alpha_i) > beta_j} over the rows of s (one warp
 // per token, lane counters for the columns lane + 32 q, folded per CTA in shared memory).
@@ -1321,8 +1464,8 @@ int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, 
     qb_layout(m, n, k, &w, static_cast<char*>(workspace));
     const int64_t C = m * k / n;
     cudaError_t ce;
-    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto fail;
-    if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto fail;
+    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 2 * n), stream)) != cudaSuccess)
+        goto fail;
     launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
     {
         int64_t blocks = (m + 7) / 8;
@@ -1358,15 +1501,13 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
             goto cuda_fail;
         col_attr = true;
     }
-    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * qb::kStWords, stream)) != cudaSuccess) goto cuda_fail;
-    if ((ce = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
-    if ((ce = cudaMemsetAsync(w.win, 0, sizeof(uint32_t) * n, stream)) != cudaSuccess) goto cuda_fail;
-    if ((ce = cudaMemsetAsync(w.g_above, 0, sizeof(uint32_t) * 2 * n, stream)) != cudaSuccess) goto cuda_fail;
+    // status, counts, windows and the column pass's counters: one block, one clear
+    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 5 * n), stream)) != cudaSuccess)
+        goto cuda_fail;
     if (mode == MOE_QB_STEP) {
         // one pass each; a window miss reads its column from s (no transposed copy)
         launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
-        launch_col(s, nullptr, m, n, C, w, rule, beta, w.counts, w.counts + n, 0, 0, stream);
-        qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
+        launch_col(s, nullptr, m, n, C, w, rule, beta, w.counts, w.counts + n, 0, 0, stream, info);
         if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
         return MOE_OK;
     }
@@ -1399,7 +1540,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
         for (int e = 0; e < n; ++e)
             if (hcounts[(iters % 2) * n + e] > C) excess += hcounts[(iters % 2) * n + e] - C;
         // exact finish: one shortest-path move per unit of excess; W is built for every row once,
-        // then only the rows a move invalidates are recomputed
+        // then updated entry by entry after each move
         const int64_t moves = excess < max_repair ? excess : max_repair;
         if (moves > 0) {
             const int64_t words = (m + 31) / 32;
@@ -1411,8 +1552,9 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
             qb_all_rows_kernel<<<1, 256, 0, stream>>>(n, w.rows, w.nrows);
         }
         for (int64_t a = 0; a < moves; ++a) {
-            launch_arc(s, m, n, k, topk_idx, w, stream);
-            if ((ce = launch_repair_step(n, C, k, w.W, w.A, final_counts, topk_idx, w.status, w.rows, w.nrows,
+            if (a == 0) launch_arc(s, m, n, k, topk_idx, w, stream);           // every row once
+            else launch_arc_update(s, m, n, k, topk_idx, w, stream);          // the entries the last move changed
+            if ((ce = launch_repair_step(n, C, k, w.W, w.A, final_counts, topk_idx, w.status, w.moves, w.nmoves,
                                          w.mem, (m + 31) / 32, stream)) != cudaSuccess)
                 goto cuda_fail;
         }
