@@ -42,6 +42,7 @@ namespace moe {
 
 namespace qb {
 constexpr int kRowThreads = 256;
+constexpr int kRowTile = 32;      // rows of s per shared-memory tile of the row pass (one bulk copy)
 constexpr int kColThreads = 512;  // qb_col_kernel block size (its scan buffer is sized by it)
 // status words kept in the workspace
 // kStDone: repair finished; kStQbDone: a row pass found every count equal to C (later passes return at once);
@@ -159,74 +160,104 @@ __device__ __forceinline__ bool row_topk_ranked(const uint32_t (&key)[NT], const
     return true;
 }
 
-// One warp per token, R tokens interleaved per warp so their loads overlap; each row takes the
-// ranked selection, or the plain rounds when it does not apply.
-template <int NT, int R>
-__global__ void __launch_bounds__(qb::kRowThreads)
+// One warp per token. CTAs stream tiles of kRowTile consecutive rows of s into shared memory
+// with bulk copies, two tiles in flight (double buffer, one mbarrier each; the partial last tile
+// and unaligned inputs take plain loads), so the selection reads its rows from shared memory.
+// Each row takes the ranked selection, or the plain rounds when it does not apply. beta for the
+// lane's columns stays in registers. TRANS: the tile is also written out transposed (sT [n, m],
+// each expert's column contiguous) for the column pass's full path.
+template <int NT, bool TRANS>
+__global__ void __launch_bounds__(qb::kRowThreads, 3)
 qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
               float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
-              int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT) {
+              int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT, int bulk) {
     if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
-    constexpr int ROWS = (qb::kRowThreads / 32) * R;  // token rows per CTA step
-    __shared__ float tile[ROWS][kMaxExperts + 1];      // the step's rows of s, for the transposed copy
-    __shared__ float sb[kMaxExperts];
+    constexpr int RT = qb::kRowTile;
+    extern __shared__ __align__(128) float rtile[];  // [2][RT * n]
+    __shared__ __align__(8) uint64_t bar[2];
     __shared__ int cnt[kMaxExperts];
     __shared__ int nties;
+    __shared__ int abort_flag;
     __shared__ uint32_t s_key[qb::kRowThreads];
     __shared__ int s_j[qb::kRowThreads];
     __shared__ float s_v[qb::kRowThreads];
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wbase = tid & ~31;  // this warp's 32 shared slots
-    for (int j = tid; j < n; j += blockDim.x) { sb[j] = beta[j]; cnt[j] = 0; }
-    if (tid == 0) nties = 0;
+    const int64_t ntiles = (m + RT - 1) / RT;
+    const int64_t tile_floats = (int64_t)RT * n;
+    const uint32_t tile_bytes = (uint32_t)(tile_floats * sizeof(float));
+    for (int j = tid; j < n; j += blockDim.x) cnt[j] = 0;
+    if (tid == 0) {
+        nties = 0;
+        abort_flag = 0;
+        ptx::mbar_init(&bar[0], 1);
+        ptx::mbar_init(&bar[1], 1);
+        ptx::fence_barrier_init();
+    }
     __syncthreads();
+    float bq[NT];
+#pragma unroll
+    for (int q = 0; q < NT; ++q) bq[q] = lane + 32 * q < n ? beta[lane + 32 * q] : 0.f;
     const uint32_t lt = (1u << lane) - 1u;
     const bool prune = k < 32 && k < n;
-    // CTA-uniform steps of ROWS consecutive tokens (warp w takes rows w R .. w R + R - 1), so the
-    // optional transposed copy can use block barriers
-    for (int64_t base = (int64_t)blockIdx.x * ROWS; base < m; base += (int64_t)gridDim.x * ROWS) {
-        const int64_t i0 = base + (tid >> 5) * R;
-        float v[R][NT];
-        uint32_t key[R][NT];
-#pragma unroll
-        for (int u = 0; u < R; ++u) {
-            const int64_t i = i0 + u;
-#pragma unroll
-            for (int q = 0; q < NT; ++q) {
-                const int j = lane + 32 * q;
-                const bool ok = i < m && j < n;
-                const float sv = ok ? s[i * n + j] : 0.f;
-                if (sT && j < n) tile[(tid >> 5) * R + u][j] = sv;
-                v[u][q] = ok ? __fsub_rn(sv, sb[j]) : 0.f;
-                key[u][q] = ok ? float_key(v[u][q]) : 0u;
+    // copies issued and consumed per buffer (thread 0's bookkeeping, for a clean exit on abort)
+    int issued[2] = {0, 0}, consumed[2] = {0, 0};
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            const int64_t t = blockIdx.x + (int64_t)b * gridDim.x;
+            if (bulk && t < ntiles && (t + 1) * RT <= m) {
+                ptx::mbar_expect_tx(&bar[b], tile_bytes);
+                ptx::bulk_load(rtile + b * tile_floats, s + t * tile_floats, tile_bytes, &bar[b]);
+                ++issued[b];
             }
         }
-        if (sT) {
-            // the first row pass also writes s transposed (sT [n, m], each expert's column
-            // contiguous for the column pass): thread j stores column j of the step's rows
-            __syncthreads();
-            const int64_t nr = min((int64_t)ROWS, m - base);
+    }
+    int u = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++u) {
+        const int b = u & 1;
+        float* tl = rtile + b * tile_floats;
+        const int64_t i0 = t * RT;
+        const int rows = (int)min((int64_t)RT, m - i0);
+        if (bulk && rows == RT) {
+            ptx::mbar_wait(&bar[b], (uint32_t)((u >> 1) & 1), &abort_flag);
+            if (tid == 0) ++consumed[b];
+        } else {
+            for (int64_t q = tid; q < (int64_t)rows * n; q += blockDim.x) tl[q] = s[i0 * n + q];
+        }
+        __syncthreads();
+        if (abort_flag) break;  // the same value in every thread after the barrier
+        if (TRANS) {
+            // thread j stores column j of the tile's rows: 16-byte pieces when they are aligned
             for (int j = tid; j < n; j += blockDim.x) {
-                float* dst = sT + (int64_t)j * m + base;
-                if (nr == ROWS && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+                float* dst = sT + (int64_t)j * m + i0;
+                if (rows == RT && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
 #pragma unroll
-                    for (int r4 = 0; r4 < ROWS; r4 += 4)
+                    for (int r4 = 0; r4 < RT; r4 += 4)
                         *reinterpret_cast<float4*>(dst + r4) =
-                            make_float4(tile[r4][j], tile[r4 + 1][j], tile[r4 + 2][j], tile[r4 + 3][j]);
+                            make_float4(tl[r4 * n + j], tl[(r4 + 1) * n + j], tl[(r4 + 2) * n + j],
+                                        tl[(r4 + 3) * n + j]);
                 } else {
-                    for (int r = 0; r < nr; ++r) dst[r] = tile[r][j];
+                    for (int r = 0; r < rows; ++r) dst[r] = tl[r * n + j];
                 }
             }
         }
+        for (int r = warp; r < rows; r += qb::kRowThreads / 32) {
+            const int64_t i = i0 + r;
+            const float* row = tl + r * n;
+            float v[NT];
+            uint32_t key[NT];
 #pragma unroll
-        for (int u = 0; u < R; ++u) {
-            const int64_t i = i0 + u;
-            if (i >= m) break;
+            for (int q = 0; q < NT; ++q) {
+                const int j = lane + 32 * q;
+                const bool ok = j < n;
+                v[q] = ok ? __fsub_rn(row[j], bq[q]) : 0.f;
+                key[q] = ok ? float_key(v[q]) : 0u;
+            }
             float vk, vk1;
-            if (!(prune && row_topk_ranked<NT>(key[u], v[u], k, i, s_key + wbase, s_j + wbase, s_v + wbase,
-                                               topk_idx, cnt, vk, vk1))) {
+            if (!(prune && row_topk_ranked<NT>(key, v, k, i, s_key + wbase, s_j + wbase, s_v + wbase, topk_idx, cnt,
+                                               vk, vk1))) {
                 uint32_t taken;
-                row_topk_rounds<NT>(key[u], v[u], n, k, taken, vk, vk1);
+                row_topk_rounds<NT>(key, v, n, k, taken, vk, vk1);
                 int pos = 0;
 #pragma unroll
                 for (int q = 0; q < NT; ++q) {
@@ -244,7 +275,26 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
                 if (vk == vk1) atomicAdd(&nties, 1);
             }
         }
-        if (sT) __syncthreads();  // the tile is rewritten by the next step
+        __syncthreads();  // every warp is done with the buffer
+        if (tid == 0) {
+            const int64_t tn = t + 2 * (int64_t)gridDim.x;
+            if (bulk && tn < ntiles && (tn + 1) * RT <= m) {
+                ptx::mbar_expect_tx(&bar[b], tile_bytes);
+                ptx::bulk_load(tl, s + tn * tile_floats, tile_bytes, &bar[b]);
+                ++issued[b];
+            }
+        }
+    }
+    if (abort_flag) {
+        // a wait gave up: let this CTA's copies still in flight land before it exits (bounded)
+        if (tid == 0) {
+            for (int b = 0; b < 2; ++b)
+                for (int c = consumed[b]; c < issued[b]; ++c)
+                    for (int it = 0; it < (1 << 22) && !ptx::mbar_try_wait(&bar[b], (uint32_t)(c & 1)); ++it) {
+                    }
+            status[qb::kStError] = 1;
+        }
+        return;
     }
     __syncthreads();
     for (int j = tid; j < n; j += blockDim.x)
@@ -1336,15 +1386,35 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
 
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k) { return qb_layout(m, n, k, nullptr, nullptr); }
 
+template <int NT, bool TRANS>
+static void launch_row_tt(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
+                          int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
+                          cudaStream_t stream) {
+    const size_t smem = 2 * (size_t)qb::kRowTile * n * sizeof(float);
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(qb_row_kernel<NT, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(2 * (size_t)qb::kRowTile * kMaxExperts * sizeof(float)));
+        attr = true;
+    }
+    // tiles spread evenly: every CTA takes the same number of tiles (the last ones one fewer)
+    const int64_t ntiles = (m + qb::kRowTile - 1) / qb::kRowTile;
+    const int64_t slots = (int64_t)kNumSMs * 3;
+    const int64_t per = (ntiles + slots - 1) / slots;
+    int64_t blocks = per > 0 ? (ntiles + per - 1) / per : 1;
+    if (blocks < 1) blocks = 1;
+    // bulk copies need a 16-byte aligned s (every tile then starts on a 16-byte boundary)
+    const int bulk = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    qb_row_kernel<NT, TRANS><<<(unsigned)blocks, qb::kRowThreads, smem, stream>>>(
+        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk);
+}
+
 template <int NT>
 static void launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                          int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
                          cudaStream_t stream) {
-    int64_t blocks = (m + 2 * (qb::kRowThreads / 32) - 1) / (2 * (qb::kRowThreads / 32));
-    if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
-    if (blocks < 1) blocks = 1;
-    qb_row_kernel<NT, 2><<<(unsigned)blocks, qb::kRowThreads, 0, stream>>>(s, m, n, k, beta, rule, alpha, topk_idx,
-                                                                           counts, status, tie_slot, skip, sT);
+    if (sT) launch_row_tt<NT, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+    else launch_row_tt<NT, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
 }
 
 // sT != nullptr: this row pass also writes s transposed into sT (the first pass of a call).
