@@ -342,11 +342,10 @@ __device__ __forceinline__ void block_select_bin(const unsigned* hist, int nbins
     __syncthreads();
 }
 
-// Add 1 to hist[d] for every active lane, one atomic per distinct d in the warp.
+// Add 1 to hist[d] for every active lane (shared-memory atomics; lanes on the same bin are
+// serialised by the hardware, which costs less than grouping them first).
 __device__ __forceinline__ void warp_hist_add(unsigned* hist, bool active, uint32_t d) {
-    const uint32_t grp = __match_any_sync(0xffffffffu, active ? d : 0xffffffffu);
-    const int lane = threadIdx.x & 31;
-    if (active && (grp & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[d], (unsigned)__popc(grp));
+    if (active) atomicAdd(&hist[d], 1u);
 }
 
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, unsigned* red) {
