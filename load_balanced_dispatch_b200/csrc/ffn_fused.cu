@@ -444,13 +444,17 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     }
 }
 
-// y rows of tokens whose pick was dropped (k = 1, dest_row < 0): the residual, or zeros.
+// y rows of tokens whose pick was dropped (k = 1, dest_row < 0): the residual, or zeros. CTA 0
+// also clears the FFN's tile counters (the FFN launch that follows waits for this one), so no
+// memset sits between the launches.
 __global__ void __launch_bounds__(256)
 combine_dropped_kernel(const int32_t* __restrict__ dest_row, const uint4* __restrict__ residual, int64_t m,
-                       int64_t vec_per_row, uint4* __restrict__ y) {
+                       int64_t vec_per_row, uint4* __restrict__ y, int* __restrict__ counters, int ncounters) {
     const int lane = threadIdx.x & 31;
     pdl_trigger();
     pdl_wait();
+    if (blockIdx.x == 0)
+        for (int c = threadIdx.x; c < ncounters; c += blockDim.x) counters[c] = 0;
     const int64_t warps = (int64_t)gridDim.x * 8;
     for (int64_t i0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * 32; i0 < m; i0 += warps * 32) {
         const int64_t i = i0 + lane;
@@ -467,12 +471,13 @@ combine_dropped_kernel(const int32_t* __restrict__ dest_row, const uint4* __rest
 }
 
 cudaError_t launch_combine_dropped(const int32_t* dest_row, const void* residual, int64_t m, int d, void* y,
-                                   cudaStream_t stream) {
+                                   int* counters, int ncounters, cudaStream_t stream) {
     if (m == 0) return cudaSuccess;
     int64_t blocks = (m + 255) / 256;
     if (blocks > (int64_t)num_sms() * 4) blocks = (int64_t)num_sms() * 4;
     return launch_pdl(combine_dropped_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, dest_row,
-                      static_cast<const uint4*>(residual), m, (int64_t)d * 2 / 16, static_cast<uint4*>(y));
+                      static_cast<const uint4*>(residual), m, (int64_t)d * 2 / 16, static_cast<uint4*>(y), counters,
+                      ncounters);
 }
 
 // xbuf: the expert-major rows [max_rows, d], or with gth the token-major x [gth->m, d] whose
@@ -541,13 +546,10 @@ cudaError_t launch_ffn_tc_combine(const void* xbuf, const void* w1, const void* 
                                   const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* hbuf,
                                   const int32_t* src_token, const int32_t* dest_row, const float* gate,
                                   const void* residual, int64_t m, void* y, cudaStream_t stream) {
-    // counters first, so that the FFN directly follows a kernel (programmatic dependent launch)
+    // the dropped rows' kernel also clears the FFN's counters, so the FFN directly follows a
+    // kernel (programmatic dependent launch) and no memset sits in the chain
     int* counters = ffn_counters(hbuf, max_rows, d_ff);
-    if (max_rows > 0) {
-        cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)(n + 1), stream);
-        if (e != cudaSuccess) return e;
-    }
-    cudaError_t e = launch_combine_dropped(dest_row, residual, m, d, y, stream);
+    cudaError_t e = launch_combine_dropped(dest_row, residual, m, d, y, counters, max_rows > 0 ? n + 1 : 0, stream);
     if (e != cudaSuccess || max_rows == 0) return e;
     const FusedCombine cmb{src_token, gate, static_cast<const __nv_bfloat16*>(residual),
                            static_cast<__nv_bfloat16*>(y), m};

@@ -214,19 +214,20 @@ class MoELayer:
 
     def launches_per_forward(self) -> int:
         """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection
-        and the finish kernel; else 1), capacity 2
-        (count + scan, assign), dispatch 1 (0 when the FFN gathers its rows from x), FFN (bf16: one fused
-        launch, after a memset of its counters; fp32: 2), combine 1, statistics 1. With one pick per token
-        in bf16 the combine is the FFN's epilogue plus one launch for the dropped tokens' rows."""
+        and the finish kernel; else 1), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
+        gathers its rows from x), FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
+        combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus
+        one launch for the dropped tokens' rows (which also clears the FFN's counters)."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
         router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
+        capacity = 2
         dispatch = 1 if self.uses_dispatch() else 0
         if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped rows
             ffn, combine = 2, 0
         else:
             ffn, combine = (1 if bf16 else 2), 1
-        return router + 2 + dispatch + ffn + combine + 1
+        return router + capacity + dispatch + ffn + combine + 1
 
 
 def weights_to_device(inp: dict, dtype: torch.dtype, device="cuda") -> dict:

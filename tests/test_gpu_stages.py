@@ -109,7 +109,9 @@ def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
 # ---------------------------------------------------------------- capacity
 @pytest.mark.parametrize("m,n,k,cap,seg", [(1000, 8, 1, 160, 1000), (8192, 128, 1, 80, 8192), (4096, 64, 2, 256, 512),
                                            (777, 16, 3, 40, 777), (1536, 256, 8, 30, 256), (600, 5, 2, 0, 300),
-                                           (300, 4, 2, 10 ** 6, 100), (64, 64, 63, 1, 64)])
+                                           (300, 4, 2, 10 ** 6, 100), (64, 64, 63, 1, 64),
+                                           # a large one-segment shape (many chunks in one segment)
+                                           (16384, 64, 6, 16384 * 6, 16384)])
 def test_capacity_bitexact(m, n, k, cap, seg):
     idx = W.make_topk_idx(m, n, k, seed=m * 7 + n)
     ref = oracle.capacity(idx, m, k, n, cap, seg)
