@@ -44,6 +44,9 @@ constexpr int threads(bool gather) { return gather ? 320 : 192; }
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
+// a tile with at most BN / 2 valid columns (the last one when N % BN <= BN / 2) issues N = BN / 2
+// MMAs over the first half of its B tile; the epilogue never reads the other half
+constexpr uint32_t IDESC_HALF = ptx::idesc_bf16_f32(BM, BN / 2);
 constexpr int kEpiWarps = 4;
 constexpr int RING = 4;   // tile ids handed from the producer to the MMA and epilogue warps
 }  // namespace fz
@@ -253,10 +256,9 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                 ptx::mbar_arrive(&sh->tfree[slot]);
                 if (++slot == RING) { slot = 0; rphase ^= 1u; }
                 if (tile < 0) break;
-                int ph, lt_unused;
-                ticket_decode(sh, n, L, tile, ph, lt_unused);
-                const int K = ph == 1 ? d : d_ff;
-                const int nkb = (K + BK - 1) / BK;
+                const FusedTile t = fused_decode(sh, tile, L, n, d, d_ff);
+                const int nkb = (t.K + BK - 1) / BK;
+                const uint32_t idesc = t.N - t.n0 <= BN / 2 ? IDESC_HALF : IDESC;
                 if (!ptx::mbar_wait(&sh->tempty[acc], aphase ^ 1u, abort_flag)) break;
                 ptx::tc_fence_after();
                 const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
@@ -269,7 +271,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                     const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        ptx::umma_bf16(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+                        ptx::umma_bf16(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
                     ptx::umma_commit(&sh->empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
