@@ -1026,8 +1026,6 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     __shared__ double dist[2][kMaxExperts];
     __shared__ unsigned char chg[2][kMaxExperts];
     __shared__ double part_d[8][qb::kRepCols];
-    __shared__ double nd_own[qb::kRepCols];
-    __shared__ unsigned char nc_own[qb::kRepCols];
     __shared__ int part_p[8][qb::kRepCols];
     __shared__ int pred[kMaxExperts];
     __shared__ int front[kMaxExperts], nfront, wcount[kMaxExperts / 32];
@@ -1062,13 +1060,18 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     int cur = 0;
     bool settled = false;
     for (int round = 0; round <= n; ++round) {
-        compact_flags(chg[cur], n, front, &nfront, wcount);
-        const int nf = nfront;
-        if (nf == 0) { settled = true; break; }
+        // warp `part` relaxes from the changed experts among 32 part .. 32 part + 31 (a ballot of
+        // the change flags, no compaction); the rounds end when no flag is set in any CTA's copy
+        // (every CTA holds the same flags)
+        const int a0 = part * 32;
+        const bool mine = a0 + bl < n && chg[cur][a0 + bl];
+        uint32_t fm = __ballot_sync(0xffffffffu, mine);
+        if (!__syncthreads_or(mine)) { settled = true; break; }
         double best = INFINITY;
         if (own) {
-            for (int f = part; f < nf; f += 8) {
-                const int a = front[f];
+            while (fm) {
+                const int a = a0 + __ffs(fm) - 1;
+                fm &= fm - 1;
                 const double w = wsl[a * qb::kRepCols + bl];
                 if (a != b && w != INFINITY) {
                     const double c = dist[cur][a] + w;
@@ -1078,16 +1081,14 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         }
         part_d[part][bl] = best;
         __syncthreads();
-        if (part == 0 && own) {
+        if (part == 0 && own) {  // fold the 8 partials, then this column into every CTA's next-round buffers
             double nd = dist[cur][b];
             for (int p = 0; p < 8; ++p) nd = fmin(nd, part_d[p][bl]);
-            nd_own[bl] = nd;
-            nc_own[bl] = nd != dist[cur][b] ? 1 : 0;
-        }
-        __syncthreads();
-        if (own) {  // thread (part = target CTA, bl): this column into that CTA's next-round buffers
-            ptx::st_cluster_f64(ptx::mapa_shared(ptx::smem_u32(&dist[cur ^ 1][b]), (uint32_t)part), nd_own[bl]);
-            ptx::st_cluster_u8(ptx::mapa_shared(ptx::smem_u32(&chg[cur ^ 1][b]), (uint32_t)part), nc_own[bl]);
+            const unsigned char nc = nd != dist[cur][b] ? 1 : 0;
+            for (int r = 0; r < qb::kRepCtas; ++r) {
+                ptx::st_cluster_f64(ptx::mapa_shared(ptx::smem_u32(&dist[cur ^ 1][b]), (uint32_t)r), nd);
+                ptx::st_cluster_u8(ptx::mapa_shared(ptx::smem_u32(&chg[cur ^ 1][b]), (uint32_t)r), nc);
+            }
         }
         ptx::cluster_sync();
         cur ^= 1;

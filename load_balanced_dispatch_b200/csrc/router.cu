@@ -210,12 +210,20 @@ router_finish_kernel(const float* h, int64_t m, int n, int k, int fn, int renorm
     pdl_trigger();
     pdl_wait();
     const int64_t warps = (int64_t)gridDim.x * (kFinishThreads / 32);
-    for (int64_t row = (int64_t)blockIdx.x * (kFinishThreads / 32) + (threadIdx.x >> 5); row < m; row += warps) {
-        float hv[NT];
+    // the next row's logits are loaded before this row is finished (one row in flight ahead)
+    int64_t row = (int64_t)blockIdx.x * (kFinishThreads / 32) + (threadIdx.x >> 5);
+    float hv[NT];
 #pragma unroll
-        for (int q = 0; q < NT; ++q) hv[q] = (lane + 32 * q < n) ? h[row * n + lane + 32 * q] : 0.f;
+    for (int q = 0; q < NT; ++q) hv[q] = (row < m && lane + 32 * q < n) ? h[row * n + lane + 32 * q] : 0.f;
+    for (; row < m; row += warps) {
+        const int64_t nr = row + warps;
+        float nx[NT];
+#pragma unroll
+        for (int q = 0; q < NT; ++q) nx[q] = (nr < m && lane + 32 * q < n) ? h[nr * n + lane + 32 * q] : 0.f;
         __syncwarp();
         finish_row<NT>(hv, row, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+#pragma unroll
+        for (int q = 0; q < NT; ++q) hv[q] = nx[q];
     }
 }
 
