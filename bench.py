@@ -59,7 +59,7 @@ def peaks_all():
 # dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch at a shape, from the
 # ncu capture summarised under profiles/. Emptied whenever the kernel changes (the figure would be
 # stale), refilled from the next capture.
-FFN_DRAM_TRAFFIC = {"switch": 1.24e9 + 36.06e6}
+FFN_DRAM_TRAFFIC = {"switch": 1239.07e6 + 39.97e6}
 
 
 def ffn_roofline(cfg, offsets, ffn_ms, esz=2):
