@@ -414,6 +414,31 @@ def test_balance_solve_bitexact(m, n, k, iters, rule):
     assert (np.bincount(host(idx).ravel(), minlength=n) == m * k // n).all()
 
 
+@pytest.mark.parametrize("m,n,k", [(4096, 64, 4), (1000, 32, 8)])
+def test_balance_misaligned_scores(m, n, k):
+    # s starting 4 bytes past a 16-byte boundary: the row pass loads its tiles without bulk copies
+    # and the window sweep reads scalars; two chained STEPs and a SOLVE stay bit-exact
+    s = W.make_qb_scores(m, n, seed=m + 5)
+    buf = torch.empty((m * n + 1,), dtype=torch.float32, device="cuda")
+    sd = buf[1:].view(m, n)
+    sd.copy_(torch.from_numpy(s))
+    assert sd.data_ptr() % 16 == 4
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(2):
+        i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=b, mode=oracle.QB_STEP)
+        idx, beta, info = lb.moe_balance_assign(sd, k, beta=dev(b), mode=lb.MOE_QB_STEP)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(beta) == b_ref).all()
+        b = b_ref
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=12)
+    idx, beta, info = lb.moe_balance_assign(sd, k, mode=lb.MOE_QB_SOLVE, max_iters=12)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
+
+
 @pytest.mark.parametrize("m,n,k,seed", [(1024, 8, 2, 0), (2048, 16, 2, 2), (4096, 32, 4, 1), (512, 4, 1, 0)])
 def test_balance_solve_converges_inside_a_batch(m, n, k, seed):
     # mild skew: QB alone reaches exact balance after 6..45 beta updates (no repair), so the
