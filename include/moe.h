@@ -109,7 +109,9 @@ MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float
  * alternating QB algorithm box, and its practical one-step form under
  * "Mind the pitfall" (select with the old beta, then update beta).
  *
- *  s          [m, n] fp32 scores. (m * k) % n must be 0 and k < n.
+ *  s          [m, n] fp32 scores, row-major, any 4-byte alignment (rows that start on
+ *             16-byte boundaries take the faster bulk-copy and vector paths). (m * k) % n
+ *             must be 0 and k < n.
  *  beta       [n] fp32, in: previous beta (zeros for a cold start); out: new beta.
  *  mode       MOE_QB_STEP: x = topk(s - beta_old); one alpha/beta update -> beta_new.
  *             MOE_QB_SOLVE: alternate row/column passes until topk(s - beta) has
@@ -130,6 +132,10 @@ MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float
  * SOLVE synchronises `stream` between phases (its loop length depends on the
  * data) and returns MOE_ERR_NOT_CONVERGED if max_repair moves did not remove
  * the excess. STEP is fully asynchronous.
+ * workspace: moe_balance_assign_workspace_size bytes (device, caller-owned, any
+ * contents on entry; the call clears what it needs). It holds s transposed
+ * (SOLVE), alpha, the column pass's per-expert windows and candidate lists, and
+ * the exact finish's arc costs and membership bitmap.
  */
 MOE_API size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k, moe_qb_mode mode);
 MOE_API moe_status moe_balance_assign(const float* s, int64_t m, int32_t n, int32_t k, float* beta, moe_qb_mode mode,
