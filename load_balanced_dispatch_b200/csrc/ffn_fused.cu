@@ -20,8 +20,8 @@
 // One CTA per SM, 192 threads: warp 0 takes tickets and runs the TMA producer
 // (4-stage ring of a 128x64 A tile and a 256x64 B tile, 128-byte swizzle,
 // K-major, no multicast); warp 1's lane 0 issues tcgen05.mma kind::f16
-// (M=128, N=256, K=16, bf16 x bf16 -> fp32 in TMEM) and commits each stage
-// back; warps 2-5 drain one of two TMEM accumulators (tcgen05.ld, + bias,
+// (M=128, N=256, K=16, bf16 x bf16 -> fp32 in TMEM; N=128 for a tile with at
+// most 128 valid columns) and commits each stage back; warps 2-5 drain one of two TMEM accumulators (tcgen05.ld, + bias,
 // ReLU for GEMM1, bf16, 16-byte stores) while the other fills. Row tails past
 // an expert's end are computed and masked; column and K tails are TMA zero
 // fill. Every wait is bounded (about 2 s), after which the device error word
@@ -30,7 +30,8 @@
 // With one pick per token (k = 1) the GEMM2 epilogue can also do the gated
 // combine (moe_expert_ffn_combine): each output row is written, gated, to its
 // token's row of y, so ybuf and the combine launch disappear; the few dropped
-// tokens get their residual (or zeros) from combine_dropped_kernel.
+// tokens get their residual (or zeros) from combine_dropped_kernel, which also
+// clears the FFN's counters so that the FFN launch directly follows it.
 #include "groups.cuh"
 #include "tc_ptx.cuh"
 
