@@ -836,9 +836,10 @@ __global__ void qb_member_bits_kernel(const int32_t* __restrict__ topk_idx, int6
 
 // Arc costs of the expert graph for the listed rows a = rows[blockIdx.x]:
 // W[a][b] = min over tokens i holding a but not b of s_ia - s_ib (fp64), A[a][b] = that token
-// (lowest token among equal costs). Each row is split over gridDim.y CTAs, slice y taking the
-// y-th range of bitmap words (tokens), so the few rows a repair move invalidates still spread
-// over the GPU. The members of a in the slice come from the bitmap (compacted into shared memory,
+// (lowest token among equal costs). It builds every row once per SOLVE (later moves update W in
+// place: qb_arc_inc_kernel, qb_arc_recompute_kernel). Each row is split over gridDim.y CTAs,
+// slice y taking the y-th range of bitmap words (tokens), so the rows spread over the GPU.
+// The members of a in the slice come from the bitmap (compacted into shared memory,
 // kMemberCap at a time); warp w takes members in batches of kArcBatch, lanes own columns
 // b = lane + 32 q; the warps' minima are folded in warp order, and the last slice of the row to
 // finish folds the slices' partials in slice order.
