@@ -203,7 +203,9 @@ MOE_API moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_
  *  MOE_ERR_WORKSPACE before anything is enqueued; use moe_capacity_slots then.
  *  The first call on a device looks up the array's device address with
  *  cudaGetSymbolAddress while that device is current; make that first call
- *  before any stream capture.
+ *  before any stream capture. `stream` must belong to the current device
+ *  (MOE_ERR_INVALID_ARG otherwise). Invalid arguments are rejected before the
+ *  lookup, with the same checks and codes as moe_capacity_slots.
  *  All calls share the one array and it keeps the last call's contents (no
  *  word of it needs to start at zero: every word read is first written by the
  *  same call). Calls that overlap on the GPU -- on different streams, or from
@@ -224,6 +226,21 @@ MOE_API moe_status moe_capacity_slots_static(const int32_t* topk_idx, int64_t m,
  */
 MOE_API moe_status moe_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, const int32_t* src_token,
                         const int32_t* expert_offsets, int32_t n, int64_t max_rows, void* xbuf, moe_stream_t stream);
+
+/*
+ * Dispatch, token-major: the same expert-major rows as moe_dispatch, written by
+ * visiting tokens instead of rows, so each token's activations are read once
+ * however many of its picks are kept (with k picks per token moe_dispatch
+ * reads a token once per kept pick).
+ * Passage: as moe_dispatch ("Switch Transformer read for implementation",
+ * molayo1419.me: the first of the two permutations groups tokens by expert).
+ *  x [m, d] (dtype dt); dest_row [m, k] from moe_capacity_slots (-1 = dropped).
+ *  xbuf [max_rows, d] out: xbuf[dest_row[i, r]] = x[i] for every dest_row[i, r] >= 0;
+ *  a row index >= max_rows is skipped and sets the device error word.
+ *  Results: bit for bit those of moe_dispatch on the same capacity outputs.
+ */
+MOE_API moe_status moe_dispatch_tokens(const void* x, moe_dtype dt, int64_t m, int32_t d, int32_t k,
+                                       const int32_t* dest_row, int64_t max_rows, void* xbuf, moe_stream_t stream);
 
 /*
  * Expert FFN on the expert-major rows: for the rows of expert e,

@@ -30,7 +30,7 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
            "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step",
-           "moe_expert_ffn_gather")
+           "moe_expert_ffn_gather", "moe_dispatch_tokens")
 
 
 class MoEError(RuntimeError):
@@ -64,6 +64,7 @@ def lib() -> C.CDLL:
         L.moe_capacity_slots.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P, SZ, P]
         L.moe_capacity_slots_static.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P]
         L.moe_dispatch.argtypes = [P, I32, I64, I32, P, P, I32, I64, P, P]
+        L.moe_dispatch_tokens.argtypes = [P, I32, I64, I32, I32, P, I64, P, P]
         L.moe_expert_ffn_workspace_size.argtypes = [I32, I64, I32]
         L.moe_expert_ffn_workspace_size.restype = SZ
         L.moe_expert_ffn.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, SZ, P]
@@ -209,6 +210,19 @@ def moe_dispatch(x, src_token, expert_offsets, n, max_rows=None, xbuf=None, stre
         xbuf = torch.empty((max_rows, d), dtype=x.dtype, device=x.device)
     _check("moe_dispatch", lib().moe_dispatch(_ptr(x), _dtype_code(x), m, d, _ptr(src_token), _ptr(expert_offsets),
                                               n, max_rows, _ptr(xbuf), _stream(stream)))
+    return xbuf
+
+
+def moe_dispatch_tokens(x, dest_row, max_rows=None, xbuf=None, stream=None):
+    """xbuf[dest_row[i, r]] = x[i] for the kept picks, visiting tokens (each x row read once).
+    Returns xbuf [max_rows, d]; the same rows as moe_dispatch."""
+    m, d = x.shape
+    k = dest_row.shape[1]
+    max_rows = m * k if max_rows is None else max_rows
+    if xbuf is None:
+        xbuf = torch.empty((max_rows, d), dtype=x.dtype, device=x.device)
+    _check("moe_dispatch_tokens", lib().moe_dispatch_tokens(_ptr(x), _dtype_code(x), m, d, k, _ptr(dest_row),
+                                                            max_rows, _ptr(xbuf), _stream(stream)))
     return xbuf
 
 

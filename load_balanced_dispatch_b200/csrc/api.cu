@@ -19,6 +19,8 @@ cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, in
 size_t capacity_workspace_bytes(int64_t m, int32_t k, int32_t n, int64_t seg_len);
 cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const int32_t* src_token,
                             const int32_t* expert_offsets, int n, int64_t max_rows, void* xbuf, cudaStream_t stream);
+cudaError_t launch_dispatch_tokens(const void* x, moe_dtype dt, int64_t m, int d, int k, const int32_t* dest_row,
+                                   int64_t max_rows, void* xbuf, cudaStream_t stream);
 cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
                            const void* residual, int64_t m, int k, int d, void* y, cudaStream_t stream);
 cudaError_t launch_ffn(const void* xbuf, moe_dtype dt, const void* w1, const void* b1, const void* w2, const void* b2,
@@ -135,10 +137,13 @@ size_t moe_capacity_slots_workspace_size(int64_t m, int32_t k, int32_t n, int64_
     return capacity_workspace_bytes(m, k, n, seg_len);
 }
 
-moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_t k, int32_t n, int32_t capacity,
-                              int64_t seg_len, int32_t* slot, int32_t* dest_row, int32_t* src_token,
-                              int32_t* expert_offsets, int32_t* routed_count, int32_t* kept_count, void* workspace,
-                              size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+// Argument checks of the capacity stage, shared by moe_capacity_slots and moe_capacity_slots_static.
+static moe_status capacity_args_ok(const int32_t* topk_idx, int64_t m, int32_t k, int32_t n, int32_t capacity,
+                                   int64_t seg_len, const int32_t* slot, const int32_t* dest_row,
+                                   const int32_t* src_token, const int32_t* expert_offsets,
+                                   const int32_t* routed_count, const int32_t* kept_count) {
     REQUIRE(m >= 0, "m must be >= 0");
     REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
     REQUIRE(k >= 1 && k <= n, "k must be in [1, n]");
@@ -147,6 +152,18 @@ moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_t k, int
     REQUIRE(seg_len >= 1 && m % seg_len == 0, "seg_len must be >= 1 and divide m");
     REQUIRE(expert_offsets && routed_count && kept_count, "output pointers are required");
     REQUIRE(m == 0 || (topk_idx && slot && dest_row && src_token), "array pointers are required");
+    return MOE_OK;
+}
+
+extern "C" {
+
+moe_status moe_capacity_slots(const int32_t* topk_idx, int64_t m, int32_t k, int32_t n, int32_t capacity,
+                              int64_t seg_len, int32_t* slot, int32_t* dest_row, int32_t* src_token,
+                              int32_t* expert_offsets, int32_t* routed_count, int32_t* kept_count, void* workspace,
+                              size_t ws_bytes, moe_stream_t stream) {
+    const moe_status st = capacity_args_ok(topk_idx, m, k, n, capacity, seg_len, slot, dest_row, src_token,
+                                           expert_offsets, routed_count, kept_count);
+    if (st != MOE_OK) return st;
     const size_t need = capacity_workspace_bytes(m, k, n, seg_len);
     if (ws_bytes < need || (need && !workspace))
         return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
@@ -166,6 +183,18 @@ moe_status moe_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, const
     REQUIRE(max_rows == 0 || (aligned16(x) && aligned16(xbuf)), "x and xbuf must be 16-byte aligned");
     return check_launch(launch_dispatch(x, dt, m, d, src_token, expert_offsets, n, max_rows, xbuf, stream),
                         "moe_dispatch");
+}
+
+moe_status moe_dispatch_tokens(const void* x, moe_dtype dt, int64_t m, int32_t d, int32_t k, const int32_t* dest_row,
+                               int64_t max_rows, void* xbuf, moe_stream_t stream) {
+    REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
+    REQUIRE(m >= 0 && max_rows >= 0 && max_rows < ((int64_t)1 << 31), "bad m or max_rows");
+    REQUIRE(k >= 1 && k <= kMaxExperts && m * (int64_t)k < ((int64_t)1 << 31), "bad k");
+    REQUIRE(d >= 1 && (d * (dt == MOE_BF16 ? 2 : 4)) % 16 == 0, "d must be a multiple of %d", dt == MOE_BF16 ? 8 : 4);
+    REQUIRE(m == 0 || (x && dest_row && xbuf), "array pointers are required");
+    REQUIRE(m == 0 || (aligned16(x) && aligned16(xbuf)), "x and xbuf must be 16-byte aligned");
+    return check_launch(launch_dispatch_tokens(x, dt, m, d, k, dest_row, max_rows, xbuf, stream),
+                        "moe_dispatch_tokens");
 }
 
 size_t moe_expert_ffn_workspace_size(moe_dtype dt, int64_t max_rows, int32_t d_ff) {

@@ -53,20 +53,31 @@ extern "C" moe_status moe_capacity_slots_static(const int32_t* topk_idx, int64_t
                                                 int32_t capacity, int64_t seg_len, int32_t* slot, int32_t* dest_row,
                                                 int32_t* src_token, int32_t* expert_offsets, int32_t* routed_count,
                                                 int32_t* kept_count, moe_stream_t stream) {
-    if (seg_len >= 1 && m >= 0 && n >= 1 && n <= moe::kMaxExperts && k >= 1) {
-        const size_t need = moe::capacity_workspace_bytes(m, k, n, seg_len);
-        if (need > moe::kStaticCapacityScratchBytes)
-            return fail(MOE_ERR_WORKSPACE,
-                        "moe_capacity_slots_static: this problem needs %zu bytes of scratch, more than the fixed "
-                        "%zu-byte array; call moe_capacity_slots with a workspace instead",
-                        need, moe::kStaticCapacityScratchBytes);
-    }
+    // Invalid arguments are rejected first, so they never reach the one-time address lookup below.
+    const moe_status st = capacity_args_ok(topk_idx, m, k, n, capacity, seg_len, slot, dest_row, src_token,
+                                           expert_offsets, routed_count, kept_count);
+    if (st != MOE_OK) return st;
+    const size_t need = moe::capacity_workspace_bytes(m, k, n, seg_len);
+    if (need > moe::kStaticCapacityScratchBytes)
+        return fail(MOE_ERR_WORKSPACE,
+                    "moe_capacity_slots_static: this problem needs %zu bytes of scratch, more than the fixed "
+                    "%zu-byte array; call moe_capacity_slots with a workspace instead",
+                    need, moe::kStaticCapacityScratchBytes);
+    // The scratch address is per device: the stream must belong to the current device.
+    int cur = 0, sdev = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e == cudaSuccess) e = cudaStreamGetDevice(stream, &sdev);
+    if (e != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "moe_capacity_slots_static: device of the stream: %s", cudaGetErrorString(e));
+    if (sdev != cur)
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_capacity_slots_static: the stream belongs to device %d but device %d is current", sdev, cur);
     void* scratch = nullptr;
-    const cudaError_t e = moe::static_capacity_scratch(&scratch);
+    e = moe::static_capacity_scratch(&scratch);
     if (e != cudaSuccess)
         return fail(MOE_ERR_CUDA, "moe_capacity_slots_static: device address of the scratch array: %s",
                     cudaGetErrorString(e));
-    // Same validation and kernels as moe_capacity_slots; the scratch is fully written before it is read.
+    // Same kernels as moe_capacity_slots; the scratch is fully written before it is read.
     return moe_capacity_slots(topk_idx, m, k, n, capacity, seg_len, slot, dest_row, src_token, expert_offsets,
                               routed_count, kept_count, scratch, moe::kStaticCapacityScratchBytes, stream);
 }

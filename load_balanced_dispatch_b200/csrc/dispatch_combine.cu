@@ -6,8 +6,8 @@
 // overflow tokens keep only the residual. Switch Transformers paper review
 // (tildalice.io/?p=118), Step 3: y = p_i* E_i*(x).
 //
-// Both kernels are HBM-bound row copies: one warp per row, 16-byte vectors,
-// grid sized to a multiple of the SM count and striding over rows.
+// All kernels are HBM-bound row copies: one warp per row (or per token), 16-byte
+// vectors, grid sized to a multiple of the SM count and striding over rows.
 #include "common.cuh"
 
 namespace moe {
@@ -55,6 +55,53 @@ dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, con
             for (int u = 0; u < 8; ++u) {
                 const int64_t c = c0 + 32 * u;
                 if (c < vec_per_row) dst[c] = v[u];
+            }
+        }
+    }
+}
+
+// Token-major dispatch: xbuf[dest_row[i, r]] = x[i] for every kept pick (dest_row >= 0). Each
+// token's row is read from HBM once, whatever the number of its kept picks, and written to each
+// of its rows: the same xbuf as dispatch_kernel (the kept rows are exactly rows 0 .. rows-1).
+// One warp per token; a lane moves 16-byte vectors, eight loads in flight before the stores.
+__global__ void __launch_bounds__(kRowThreads)
+dispatch_tokens_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, int k,
+                       const int32_t* __restrict__ dest_row, int64_t max_rows, uint4* __restrict__ xbuf) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
+    for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
+        // the token's kept rows, gathered into lanes 0 .. nk-1 (k <= 32 per pass of picks)
+        for (int r0 = 0; r0 < k; r0 += 32) {
+            int32_t row = -1;
+            if (r0 + lane < k) row = dest_row[i * k + r0 + lane];
+            if (row >= max_rows) {
+                record_error(kErrRowOverflow);
+                row = -1;
+            }
+            const uint32_t kept = __ballot_sync(0xffffffffu, row >= 0);
+            if (!kept) continue;
+            const uint4* src = x + i * vec_per_row;
+            for (int64_t c0 = lane; c0 < vec_per_row; c0 += 32 * 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t c = c0 + 32 * u;
+                    if (c < vec_per_row) v[u] = src[c];
+                }
+                uint32_t rest = kept;
+                while (rest) {
+                    const int b = __ffs(rest) - 1;
+                    rest &= rest - 1;
+                    const int64_t dr = __shfl_sync(0xffffffffu, row, b);
+                    uint4* dst = xbuf + dr * vec_per_row;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int64_t c = c0 + 32 * u;
+                        if (c < vec_per_row) dst[c] = v[u];
+                    }
+                }
             }
         }
     }
@@ -111,6 +158,15 @@ cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const
     const int64_t bytes_per_row = (int64_t)d * (dt == MOE_BF16 ? 2 : 4);
     return launch_pdl(dispatch_kernel, dim3(row_grid(max_rows)), dim3(kRowThreads), 0, stream,
                       static_cast<const uint4*>(x), m, bytes_per_row / 16, src_token, expert_offsets, n, max_rows,
+                      static_cast<uint4*>(xbuf));
+}
+
+cudaError_t launch_dispatch_tokens(const void* x, moe_dtype dt, int64_t m, int d, int k, const int32_t* dest_row,
+                                   int64_t max_rows, void* xbuf, cudaStream_t stream) {
+    if (m == 0) return cudaSuccess;
+    const int64_t bytes_per_row = (int64_t)d * (dt == MOE_BF16 ? 2 : 4);
+    return launch_pdl(dispatch_tokens_kernel, dim3(row_grid(m)), dim3(kRowThreads), 0, stream,
+                      static_cast<const uint4*>(x), m, bytes_per_row / 16, k, dest_row, max_rows,
                       static_cast<uint4*>(xbuf));
 }
 

@@ -12,7 +12,7 @@ from dataclasses import dataclass
 import torch
 
 from . import (MOE_QB_MIDPOINT, MOE_QB_STEP, MOE_SIGMOID, MOE_SOFTMAX, moe_balance_assign, moe_balance_stats,
-               moe_capacity_slots, moe_combine, moe_dispatch, moe_expert_ffn, moe_expert_ffn_combine,
+               moe_capacity_slots, moe_combine, moe_dispatch_tokens, moe_expert_ffn, moe_expert_ffn_combine,
                moe_expert_ffn_gather, moe_router_topk, lib)
 
 
@@ -100,7 +100,8 @@ class MoELayer:
             moe_capacity_slots(b["topk_idx"], s.n, s.capacity, self.seg_len, out=b, workspace=self.ws["cap"], stream=st)
         elif i == 2:
             if self.uses_dispatch():  # otherwise the FFN gathers its rows from x
-                moe_dispatch(x, b["src_token"], b["expert_offsets"], s.n, self.rows_max, xbuf=b["xbuf"], stream=st)
+                # token-major: each token read once, written to each of its kept rows
+                moe_dispatch_tokens(x, b["dest_row"], self.rows_max, xbuf=b["xbuf"], stream=st)
         elif i == 3:
             if self.ffn_combine:
                 moe_expert_ffn_combine(b["xbuf"], w["w1"], w["b1"], w["w2"], w["b2"], b["expert_offsets"],

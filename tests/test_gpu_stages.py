@@ -158,6 +158,10 @@ def test_dispatch_combine(dtype, m, d, n, k, cap):
     xbuf = lb.moe_dispatch(xd, out["src_token"], out["expert_offsets"], n, m * k)
     torch.cuda.synchronize()
     assert (host(xbuf)[:rows] == oracle.dispatch(x, ref["src_token"], rows)).all()
+    # token-major dispatch: the same rows, each token read once
+    xbuf_t = lb.moe_dispatch_tokens(xd, out["dest_row"], m * k)
+    torch.cuda.synchronize()
+    assert (host(xbuf_t)[:rows] == oracle.dispatch(x, ref["src_token"], rows)).all()
     ybuf = rng.standard_normal((m * k, d)).astype(np.float32)
     if dtype == "bf16":
         ybuf = W.round_to_bf16(ybuf)

@@ -8,8 +8,10 @@ scratch array of its own. This test calls that entry point through the C ABI
 twice in a row, on different problems (the second smaller than the first, so
 stale scratch contents from the first call are present), and checks that every
 output equals the one of moe_capacity_slots with a caller workspace, bit for
-bit (these are integer results). It also checks that a problem needing more
-than the fixed array is rejected before anything runs.
+bit (these are integer results). A second pair runs small-then-large (so the
+large call uses scratch words the small one never touched), then an empty problem.
+It also checks that a problem needing more than the fixed array, or one with
+invalid arguments, is rejected before anything runs.
 """
 import numpy as np
 import pytest
@@ -52,6 +54,38 @@ def test_static_scratch_matches_workspace_version_on_two_calls(lib):
     _compare(W.make_topk_idx(65536, 64, 2, seed=11), 64, 256, 4096)
     # call 2: a smaller single-segment top-1 problem over 128 experts with heavy drops
     _compare(W.make_topk_idx(8192, 128, 1, seed=12), 128, 40, 8192)
+
+
+def test_static_scratch_small_then_large_and_empty(lib):
+    # small first, then large: the large call's per-chunk words lie past anything the small one wrote
+    _compare(W.make_topk_idx(1024, 16, 2, seed=13), 16, 100, 512)
+    _compare(W.make_topk_idx(32768, 64, 4, seed=14), 64, 300, 8192)
+    # no tokens: the empty layout (all offsets 0), from both entry points
+    n = 32
+    empty = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+
+    def outs():
+        return dict(slot=torch.empty((0, 2), dtype=torch.int32, device="cuda"),
+                    dest_row=torch.empty((0, 2), dtype=torch.int32, device="cuda"),
+                    src_token=torch.empty((1,), dtype=torch.int32, device="cuda"),
+                    expert_offsets=torch.full((n + 1,), 7, dtype=torch.int32, device="cuda"),
+                    routed_count=torch.empty((1, n), dtype=torch.int32, device="cuda"),
+                    kept_count=torch.empty((1, n), dtype=torch.int32, device="cuda"))
+    ref = lb.moe_capacity_slots(empty, n, 10, 1, out=outs())
+    got = lb.moe_capacity_slots_static(empty, n, 10, 1, out=outs())
+    torch.cuda.synchronize()
+    lb.sync_status()
+    assert torch.equal(got["expert_offsets"], ref["expert_offsets"])
+    assert int(got["expert_offsets"].abs().sum().item()) == 0
+
+
+def test_static_scratch_rejects_invalid_arguments_first(lib):
+    # seg_len that does not divide m: the same MOE_ERR_INVALID_ARG as moe_capacity_slots
+    fake = torch.empty(16, dtype=torch.int32, device="cuda")
+    p = fake.data_ptr()
+    rc = lib.moe_capacity_slots_static(p, 10, 1, 4, 2, 3, p, p, p, p, p, p, None)
+    assert rc == 1
+    assert "seg_len" in lb.last_error()
 
 
 def test_static_scratch_rejects_problems_larger_than_the_array(lib):
