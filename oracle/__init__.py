@@ -58,6 +58,7 @@ def lib():
         _lib.orc_qb_col.restype = None
         _lib.orc_is_optimal.argtypes = [P, L, I, P, I, D]
         _lib.orc_qb_sign_step.argtypes = [P, L, I, I, P, F, I, P, P]
+        _lib.orc_balance_step_minibatch.argtypes = [P, L, I, I, P, I, L, P, P]
     return _lib
 
 
@@ -136,12 +137,13 @@ def combine(ybuf, dest_row, topk_gate, residual, m, k, d, gate_bf16=0):
 
 
 def balance_stats(probs, topk_idx, m, n, k, seg_len, alpha=1e-2, bias=None, gamma=1e-3):
-    """Returns dict(f [nseg+1,n], P [nseg+1,n] or None, aux [nseg+2] or None, vio [3], bias_new or None)."""
+    """Returns dict(f [nseg+1,n], P [nseg+1,n] or None, aux [nseg+3] or None, vio [3], bias_new or None).
+    aux: per segment, micro-batch mean, global-batch, hybrid (global + 0.01 micro)."""
     nseg = m // seg_len
     probs = None if probs is None else np.ascontiguousarray(probs, dtype=np.float64)
     f = np.empty((nseg + 1, n), np.float64)
     P = np.empty((nseg + 1, n), np.float64)
-    aux = np.empty(nseg + 2, np.float64)
+    aux = np.empty(nseg + 3, np.float64)
     vio = np.empty(3, np.float64)
     bias = _f32(bias)
     bias_out = None if bias is None else np.empty(n, np.float32)
@@ -177,6 +179,20 @@ def qb_sign_step(s, k, beta, gamma, rule=QB_MIDPOINT):
     rc = lib().orc_qb_sign_step(_p(s), m, n, k, _p(beta), np.float32(gamma), rule, _p(idx), _p(info))
     if rc:
         raise OracleError("orc_qb_sign_step", rc)
+    return idx, beta, info
+
+
+def balance_step_minibatch(s, k, beta, seg_len, rule=QB_MIDPOINT):
+    """The practical QB step with beta computed per mini-batch of seg_len tokens and averaged:
+    returns (topk_idx [m,k] ascending experts, beta_out [n] f32, info [4])."""
+    s = _f32(s)
+    m, n = s.shape
+    beta = np.array(beta, dtype=np.float32, copy=True)
+    idx = np.empty((m, k), np.int32)
+    info = np.zeros(4, np.int32)
+    rc = lib().orc_balance_step_minibatch(_p(s), m, n, k, _p(beta), rule, seg_len, _p(idx), _p(info))
+    if rc:
+        raise OracleError("orc_balance_step_minibatch", rc)
     return idx, beta, info
 
 

@@ -275,8 +275,11 @@ void orc_combine(const double* ybuf, const int32_t* dest_row, const double* topk
  * Counts are taken from the routing decision (before capacity). For k > 1,
  * f_i = count_i / (k * m_seg) so that sum_i f_i = 1.
  *   f, P  : [(nseg + 1) * n], row nseg is the whole batch (pooled counts).
- *   aux   : [nseg + 2]; aux[s] per segment, aux[nseg] mean over segments
- *           (micro-batch loss), aux[nseg + 1] on pooled f and P (global).
+ *   aux   : [nseg + 3]; aux[s] per segment, aux[nseg] mean over segments
+ *           (micro-batch loss), aux[nseg + 1] on pooled f and P (global),
+ *           aux[nseg + 2] the hybrid loss of [QW] "balancing efficiency and
+ *           effectiveness": the global-batch loss plus the micro-batch loss with
+ *           the constant weight 0.01, aux[nseg + 1] + 0.01 * aux[nseg].
  *   vio   : [3] MaxVio, MinVio, AvgVio of the pooled counts: F_i = count_i /
  *           sum(count) * n - 1 -> max, min, mean |F_i|.
  *   bias  : b_i <- b_i - gamma * sign(F_i - 1/n) in fp32, with the sign decided
@@ -318,7 +321,11 @@ int orc_balance_stats(const double* probs, const int32_t* topk_idx, int64_t m, i
             g += f[nseg * n + e] * P[nseg * n + e];
         }
     }
-    if (probs) { aux[nseg] = micro / (double)nseg; aux[nseg + 1] = alpha * (double)n * g; }
+    if (probs) {
+        aux[nseg] = micro / (double)nseg;
+        aux[nseg + 1] = alpha * (double)n * g;
+        aux[nseg + 2] = aux[nseg + 1] + 0.01 * aux[nseg];
+    }
     if (vio) {
         double mx = -INFINITY, mn = INFINITY, av = 0.0, all = (double)m * (double)k;
         for (int e = 0; e < n; ++e) {
@@ -614,6 +621,50 @@ int orc_qb_sign_step(const float* s, int64_t m, int n, int k, float* beta_inout,
     }
     if (info) { info[0] = 1; info[1] = 0; info[2] = (int32_t)excess; info[3] = (int32_t)ties; }
     free(alpha); free(X); free(cnt); free(buf);
+    return ORC_OK;
+}
+
+/*
+ * The practical QB step on mini-batches ([QB] "Mind the pitfall", closing paragraph): an exact
+ * beta over the whole batch needs the (m k / n + 1)-th largest of m values per expert, too
+ * costly when m is in the millions, so the batch is split into mini-batches of seg_len tokens,
+ * beta is computed on each by the formula, and the results are averaged.
+ *   x = topk(s - beta_old) and alpha from s - beta_old for every token (the row pass of STEP:
+ *   selection with the old beta, before the update);
+ *   for each mini-batch b (tokens b L .. b L + L - 1, L = seg_len, C_b = L k / n): beta_b by the
+ *   column pass of those tokens alone;
+ *   beta_new_j = fp32( (sum over b = 0, 1, ... of (double) beta_b_j) / B ), B = m / L, the sum
+ *   taken in mini-batch order.
+ * seg_len = m is the STEP of orc_balance_assign. Requires L | m and (L k) % n == 0.
+ * topk_idx / info as orc_balance_assign's STEP (info[0] = 1).
+ */
+int orc_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* beta_inout, int rule, int64_t seg_len,
+                               int32_t* topk_idx, int32_t* info) {
+    if (n < 2 || k < 1 || k >= n || m < 1 || seg_len < 1 || m % seg_len != 0 || ((seg_len * k) % n) != 0)
+        return ORC_ERR_ARG;
+    if (rule != ORC_QB_MIDPOINT && rule != ORC_QB_BOUNDARY && rule != ORC_QB_BIP) return ORC_ERR_ARG;
+    const int64_t nb = m / seg_len, Cb = seg_len * k / n, C = m * k / n;
+    float* alpha = (float*)malloc(sizeof(float) * (size_t)m);
+    unsigned char* X = (unsigned char*)malloc((size_t)m * n);
+    int64_t* cnt = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
+    orc_kv* buf = (orc_kv*)malloc(sizeof(orc_kv) * (size_t)(seg_len > n ? seg_len : n));
+    float* bb = (float*)malloc(sizeof(float) * (size_t)n);
+    double* acc = (double*)calloc((size_t)n, sizeof(double));
+    int64_t ties = 0;
+    qb_row_pass(s, m, n, k, beta_inout, rule, alpha, X, cnt, &ties, buf);
+    for (int64_t b = 0; b < nb; ++b) {
+        qb_col_pass(s + b * seg_len * n, seg_len, n, Cb, alpha + b * seg_len, rule, bb, buf);
+        for (int j = 0; j < n; ++j) acc[j] += (double)bb[j];
+    }
+    for (int j = 0; j < n; ++j) beta_inout[j] = (float)(acc[j] / (double)nb);
+    int64_t excess = 0;
+    for (int e = 0; e < n; ++e) if (cnt[e] > C) excess += cnt[e] - C;
+    for (int64_t i = 0; i < m; ++i) {
+        int r = 0;
+        for (int j = 0; j < n; ++j) if (X[i * n + j]) topk_idx[i * k + (r++)] = j;
+    }
+    if (info) { info[0] = 1; info[1] = 0; info[2] = (int32_t)excess; info[3] = (int32_t)ties; }
+    free(alpha); free(X); free(cnt); free(buf); free(bb); free(acc);
     return ORC_OK;
 }
 

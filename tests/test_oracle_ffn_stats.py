@@ -72,7 +72,10 @@ def test_aux_balanced_golden(golden):
             m = 4 * n
             st = oracle.balance_stats(W.make_uniform_probs(m, n), W.make_round_robin_idx(m, n, k), m, n, k, m // 2,
                                       alpha=alpha)
-            assert (st["aux"] == float(g["expected_aux"][0])).all()
+            # per segment, micro-batch mean and global loss equal alpha; the hybrid loss adds
+            # 0.01 x the micro-batch loss to the global one: alpha (1 + 0.01)
+            assert (st["aux"][:-1] == float(g["expected_aux"][0])).all()
+            assert st["aux"][-1] == pytest.approx(alpha * 1.01, rel=1e-15)
             assert (st["f"] == 1.0 / n).all() and (st["P"] == 1.0 / n).all()
             assert (st["vio"] == 0).all()
 
@@ -87,7 +90,9 @@ def test_stats_hand_example():
     # global: f = [.75, .25], P = [0.6, 0.4] -> aux = 0.01*2*(0.45+0.1) = 0.011
     assert st["f"].tolist() == [[1.0, 0.0], [0.5, 0.5], [0.75, 0.25]]
     assert np.allclose(st["P"], [[0.75, 0.25], [0.45, 0.55], [0.6, 0.4]], rtol=1e-15)
-    assert np.allclose(st["aux"], [0.015, 0.01, 0.0125, 0.011], rtol=1e-14)
+    # hybrid ("Qwen global-batch load balance", balancing efficiency and effectiveness): the global
+    # loss plus the micro-batch loss with weight 0.01: 0.011 + 0.01 * 0.0125 = 0.011125
+    assert np.allclose(st["aux"], [0.015, 0.01, 0.0125, 0.011, 0.011125], rtol=1e-14)
     # MaxVio/MinVio/AvgVio of pooled counts [3, 1]: F = [3/4*2-1, 1/4*2-1] = [0.5, -0.5]
     assert st["vio"].tolist() == [0.5, -0.5, 0.5]
 
@@ -114,6 +119,8 @@ def test_f_sums_to_one_and_micro_equals_global_for_identical_segments():
     st2 = oracle.balance_stats(np.concatenate([pa, pb]), np.concatenate([ia, ib]), 2 * seg, n, 2, seg, alpha=0.01)
     assert st2["aux"][2] == pytest.approx(0.01 * n / 2, rel=1e-15)
     assert st2["aux"][3] == pytest.approx(0.01 * n / 4, rel=1e-15)
+    # the hybrid keeps a small pull towards micro-batch balance: global + 0.01 x micro
+    assert st2["aux"][4] == pytest.approx(0.01 * n / 4 + 0.01 * 0.01 * n / 2, rel=1e-14)
 
 
 def test_lossfree_bias_update_exact():

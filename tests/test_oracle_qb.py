@@ -301,3 +301,50 @@ def test_sign_step_with_zero_gamma_is_plain_topk():
     assert (beta_out == beta).all()
     _, ref, _ = oracle.qb_row(s, 2, beta)
     assert (np.sort(ref, axis=1) == idx).all()
+
+
+# ---------------------------------------------------------------- mini-batch beta ("Mind the pitfall")
+def test_minibatch_step_hand_example():
+    # m=4, n=2, k=1, two mini-batches of 2 tokens (C_b = 1), beta_old = 0.
+    # row pass: picks [0, 0, 1, 1]; alpha = mid of the two values = [2, 1, 1, 3].
+    # batch 0 (tokens 0, 1): u_0 = [3-2, 2-1] = [1, 1] -> beta = mid(1, 1) = 1;
+    #                        u_1 = [1-2, 0-1] = [-1, -1] -> -1.
+    # batch 1 (tokens 2, 3): u_0 = [0-1, 1-3] = [-1, -2] -> mid = -1.5; u_1 = [2-1, 5-3] = [1, 2] -> 1.5.
+    # average: beta = [(1 - 1.5) / 2, (-1 + 1.5) / 2] = [-0.25, 0.25].
+    s = np.array([[3, 1], [2, 0], [0, 2], [1, 5]], np.float32)
+    idx, beta, info = oracle.balance_step_minibatch(s, 1, np.zeros(2, np.float32), 2)
+    assert idx[:, 0].tolist() == [0, 0, 1, 1]
+    assert beta.tolist() == [-0.25, 0.25]
+    assert info.tolist() == [1, 0, 0, 0]
+    # the whole batch as one (C = 2): u_0 = [1, 1, -1, -2] -> mid(1, -1) = 0; u_1 = [-1, -1, 1, 2] -> 0
+    _, beta_all, _, _ = oracle.balance_assign(s, 1, mode=oracle.QB_STEP)
+    assert beta_all.tolist() == [0.0, 0.0]
+
+
+def test_minibatch_step_one_batch_is_step():
+    s = W.make_qb_scores(1024, 16, seed=5)
+    b0 = np.linspace(-0.2, 0.2, 16).astype(np.float32)
+    for rule in (oracle.QB_MIDPOINT, oracle.QB_BOUNDARY, oracle.QB_BIP):
+        i1, b1, f1 = oracle.balance_step_minibatch(s, 2, b0, 1024, rule=rule)
+        i2, b2, f2, _ = oracle.balance_assign(s, 2, beta=b0, mode=oracle.QB_STEP, rule=rule)
+        assert (i1 == i2).all() and (b1 == b2).all() and (f1 == f2).all()
+
+
+def test_minibatch_step_identical_batches_give_the_batch_beta():
+    # B copies of the same mini-batch: each beta_b is that batch's beta, and their mean is it exactly
+    s0 = W.make_qb_scores(256, 16, seed=6)
+    s = np.concatenate([s0] * 8)
+    _, b_one, _, _ = oracle.balance_assign(s0, 4, mode=oracle.QB_STEP)
+    idx, b_avg, _ = oracle.balance_step_minibatch(s, 4, np.zeros(16, np.float32), 256)
+    assert (b_avg == b_one).all()
+    # selection is the whole batch's topk(s - beta_old), as in STEP
+    i_step, _, _, _ = oracle.balance_assign(s, 4, mode=oracle.QB_STEP)
+    assert (idx == i_step).all()
+
+
+def test_minibatch_step_argument_errors():
+    s = np.zeros((12, 4), np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.balance_step_minibatch(s, 1, np.zeros(4, np.float32), 5)   # 5 does not divide 12
+    with pytest.raises(oracle.OracleError):
+        oracle.balance_step_minibatch(s, 1, np.zeros(4, np.float32), 6)   # 6 * 1 not divisible by 4
