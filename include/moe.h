@@ -92,14 +92,33 @@ MOE_API moe_status moe_sync_status(moe_stream_t stream);
  *  workspace  bf16 x with n <= 128: [3, n, d] bf16 split of W_r (w = w0 + w1 + w2, each
  *             bf16) so the projection runs on the tensor cores with exact products and
  *             fp32 accumulation; size from moe_router_topk_workspace_size (0 otherwise).
+ *             With w_r given, every call re-makes the split. With w_r == NULL (this
+ *             tensor-core path only) the call uses the split that moe_router_prepare
+ *             left in the workspace: the router weight is static across forwards, so it
+ *             is split once (the caller keeps the workspace unchanged in between).
  * All h, p, rho and keys are fp32. Errors: MOE_ERR_INVALID_ARG for bad shapes
- * or NULL required pointers; MOE_ERR_WORKSPACE for a missing or short workspace.
+ * or NULL required pointers (w_r == NULL off the tensor-core path); MOE_ERR_WORKSPACE
+ * for a missing or short workspace.
  */
 MOE_API size_t moe_router_topk_workspace_size(int32_t d, int32_t n, int32_t k, moe_dtype x_dtype);
 MOE_API moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, const float* logits_in, int64_t m,
                            int32_t d, int32_t n, int32_t k, moe_score_fn fn, int32_t renorm_topk,
                            const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
                            void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Prepare the router weight once: write the [3, n, d] bf16 split of W_r into the
+ * workspace of moe_router_topk, which later calls with w_r == NULL use as is.
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), selective
+ * precision: the router computes in fp32; the split keeps every product exact
+ * on the bf16 tensor cores (w = w0 + w1 + w2, each part bf16).
+ *  w_r [d, n] fp32; k and x_dtype as in moe_router_topk (they pick the path).
+ *  workspace: moe_router_topk_workspace_size(d, n, k, x_dtype) bytes, 16-byte aligned.
+ * Errors: MOE_ERR_UNSUPPORTED when the shape takes the fp32 FMA router (no split:
+ * pass w_r to moe_router_topk); MOE_ERR_INVALID_ARG; MOE_ERR_WORKSPACE.
+ */
+MOE_API moe_status moe_router_prepare(const float* w_r, int32_t d, int32_t n, int32_t k, moe_dtype x_dtype,
+                                      void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Optimal-assignment balancing (Quantile Balancing) with an exact finish.
@@ -158,6 +177,26 @@ MOE_API moe_status moe_balance_assign(const float* s, int64_t m, int32_t n, int3
 MOE_API moe_status moe_balance_sign_step(const float* s, int64_t m, int32_t n, int32_t k, float* beta, float gamma,
                                  moe_qb_threshold rule, int32_t* topk_idx, int32_t* info, void* workspace,
                                  size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The practical QB step with beta averaged over mini-batches.
+ * Passage: "MoE travelogue 6" (kexue.fm/archives/11619), Mind the pitfall, closing
+ * paragraph: with m in the millions the exact (m k / n + 1)-th largest per expert is
+ * too costly, so the batch is split into mini-batches, beta is computed on each by
+ * the formula, and the results are averaged.
+ *  x = topk(s - beta_old) and alpha from s - beta_old over the whole batch (as the
+ *  STEP of moe_balance_assign: select with the old beta, then update). Mini-batch b
+ *  holds tokens b seg_len .. (b + 1) seg_len - 1; its beta_b comes from its own
+ *  column pass with C_b = seg_len k / n and the threshold `rule`. The new beta is
+ *  beta_j = fp32((sum over b, in order, of (double) beta_b_j) / (m / seg_len)).
+ *  seg_len = m gives moe_balance_assign's STEP, bit for bit.
+ *  s, beta, rule, topk_idx, info, workspace: as moe_balance_assign (STEP; info[0] = 1).
+ *  Requires seg_len | m, (seg_len k) % n == 0 and m / seg_len <= 4096.
+ *  Fully asynchronous. Workspace: moe_balance_assign_workspace_size.
+ */
+MOE_API moe_status moe_balance_step_minibatch(const float* s, int64_t m, int32_t n, int32_t k, float* beta,
+                                              moe_qb_threshold rule, int64_t seg_len, int32_t* topk_idx,
+                                              int32_t* info, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Capacity slots and the expert-major row layout.
@@ -327,8 +366,10 @@ MOE_API moe_status moe_combine(const void* ybuf, moe_dtype dt, const int32_t* de
  *  topk_idx  [m, k] routing decision (counts are taken before capacity).
  *  seg_len   micro-batch length (divides m); nseg = m / seg_len.
  *  f, P      [nseg + 1, n] out (row nseg: whole batch). f_i = count_i / (k m_seg).
- *  aux       [nseg + 2] out: per segment, the mean over segments (micro-batch
- *            loss), and the loss on pooled f and P (global-batch loss).
+ *  aux       [nseg + 3] out: per segment, the mean over segments (micro-batch
+ *            loss), the loss on pooled f and P (global-batch loss), and the hybrid
+ *            loss of "Qwen global-batch load balance" (balancing efficiency and
+ *            effectiveness): the global-batch loss plus 0.01 x the micro-batch loss.
  *  vio       [3] out: MaxVio, MinVio, AvgVio of the pooled counts, or NULL.
  *  bias_inout [n] Loss-Free bias updated in place with step gamma, or NULL; the
  *            sign is decided exactly from the integer counts.

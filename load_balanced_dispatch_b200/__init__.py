@@ -30,7 +30,8 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_balance_stats_workspace_size",
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
            "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step",
-           "moe_expert_ffn_gather", "moe_dispatch_tokens")
+           "moe_expert_ffn_gather", "moe_dispatch_tokens", "moe_router_prepare",
+           "moe_balance_step_minibatch")
 
 
 class MoEError(RuntimeError):
@@ -56,6 +57,7 @@ def lib() -> C.CDLL:
         L.moe_router_topk_workspace_size.argtypes = [I32, I32, I32, I32]
         L.moe_router_topk_workspace_size.restype = SZ
         L.moe_router_topk.argtypes = [P, I32, P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
+        L.moe_router_prepare.argtypes = [P, I32, I32, I32, I32, P, SZ, P]
         L.moe_balance_assign_workspace_size.argtypes = [I64, I32, I32, I32]
         L.moe_balance_assign_workspace_size.restype = SZ
         L.moe_balance_assign.argtypes = [P, I64, I32, I32, P, I32, I32, I32, I32, P, P, P, SZ, P]
@@ -76,6 +78,7 @@ def lib() -> C.CDLL:
         L.moe_balance_stats_workspace_size.restype = SZ
         L.moe_balance_stats.argtypes = [P, P, I64, I32, I32, I64, F, P, P, P, P, P, F, P, SZ, P]
         L.moe_balance_sign_step.argtypes = [P, I64, I32, I32, P, F, I32, P, P, P, SZ, P]
+        L.moe_balance_step_minibatch.argtypes = [P, I64, I32, I32, P, I32, I64, P, P, P, SZ, P]
         L.moe_balance_totals_workspace_size.argtypes = [I64, I32]
         L.moe_balance_totals_workspace_size.restype = SZ
         L.moe_balance_totals.argtypes = [P, P, I64, I32, I32, P, P, SZ, P]
@@ -130,7 +133,8 @@ def sync_status(stream=None):
 
 def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias=None, logits_in=None,
                     probs_out=None, topk_idx=None, topk_gate=None, want_probs=True, workspace=None, stream=None):
-    """Router + top-k. Returns (topk_idx [m,k] int32, topk_gate [m,k] fp32, probs [m,n] fp32 or None)."""
+    """Router + top-k. Returns (topk_idx [m,k] int32, topk_gate [m,k] fp32, probs [m,n] fp32 or None).
+    w_r None: the workspace holds the split made by moe_router_prepare (tensor-core path only)."""
     if logits_in is not None:
         m, d = logits_in.shape[0], 0
         dev = logits_in.device
@@ -142,6 +146,8 @@ def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias
         xdt = _dtype_code(x)
         _need(x, x.dtype, (m, d), "x")
         _need(w_r, torch.float32, (d, n), "w_r")
+        if w_r is None and workspace is None:
+            raise ValueError("w_r None needs the workspace prepared by moe_router_prepare")
     _need(rank_bias, torch.float32, (n,), "rank_bias")
     if topk_idx is None:
         topk_idx = torch.empty((m, k), dtype=torch.int32, device=dev)
@@ -157,6 +163,20 @@ def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias
         _ptr(probs_out), _ptr(topk_idx), _ptr(topk_gate), _ptr(workspace),
         0 if workspace is None else workspace.numel(), _stream(stream)))
     return topk_idx, topk_gate, probs_out
+
+
+def moe_router_prepare(w_r, k, x_dtype=torch.bfloat16, workspace=None, stream=None):
+    """Split the static router weight once into the router workspace (tensor-core path). Returns the
+    workspace, for moe_router_topk(x, None, ..., workspace=ws)."""
+    d, n = w_r.shape
+    _need(w_r, torch.float32, (d, n), "w_r")
+    xdt = MOE_BF16 if x_dtype == torch.bfloat16 else MOE_F32
+    ws_bytes = lib().moe_router_topk_workspace_size(d, n, k, xdt)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=w_r.device)
+    _check("moe_router_prepare", lib().moe_router_prepare(_ptr(w_r), d, n, k, xdt, _ptr(workspace),
+                                                          workspace.numel(), _stream(stream)))
+    return workspace
 
 
 def moe_capacity_slots(topk_idx, n, capacity, seg_len=None, out=None, workspace=None, stream=None):
@@ -303,7 +323,7 @@ def moe_combine(ybuf, dest_row, topk_gate, residual=None, y=None, stream=None):
 
 def moe_balance_stats(probs, topk_idx, n, seg_len=None, alpha=1e-2, bias_inout=None, gamma=1e-3, out=None,
                       workspace=None, stream=None):
-    """f, P [nseg+1, n], aux [nseg+2], vio [3]; updates bias_inout in place when given."""
+    """f, P [nseg+1, n], aux [nseg+3], vio [3]; updates bias_inout in place when given."""
     m, k = topk_idx.shape
     seg_len = m if seg_len is None else seg_len
     nseg = m // seg_len
@@ -311,7 +331,7 @@ def moe_balance_stats(probs, topk_idx, n, seg_len=None, alpha=1e-2, bias_inout=N
     if out is None:
         out = dict(f=torch.empty((nseg + 1, n), dtype=torch.float32, device=dev),
                    P=torch.empty((nseg + 1, n), dtype=torch.float32, device=dev),
-                   aux=torch.empty((nseg + 2,), dtype=torch.float32, device=dev),
+                   aux=torch.empty((nseg + 3,), dtype=torch.float32, device=dev),
                    vio=torch.empty((3,), dtype=torch.float32, device=dev))
     ws_bytes = lib().moe_balance_stats_workspace_size(m, n, seg_len)
     if workspace is None:
@@ -374,6 +394,27 @@ def moe_balance_sign_step(s, k, beta, gamma, rule=MOE_QB_MIDPOINT, topk_idx=None
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
     _check("moe_balance_sign_step", lib().moe_balance_sign_step(
         _ptr(s), m, n, k, _ptr(beta), gamma, rule, _ptr(topk_idx), _ptr(info), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return topk_idx, beta, info
+
+
+def moe_balance_step_minibatch(s, k, beta, seg_len, rule=MOE_QB_MIDPOINT, topk_idx=None, info=None, workspace=None,
+                               stream=None):
+    """The practical QB step with beta averaged over mini-batches of seg_len tokens (beta updated in
+    place): (topk_idx [m,k] ascending experts, beta, info [4])."""
+    m, n = s.shape
+    dev = s.device
+    _need(s, torch.float32, (m, n), "s")
+    _need(beta, torch.float32, (n,), "beta")
+    if topk_idx is None:
+        topk_idx = torch.empty((m, k), dtype=torch.int32, device=dev)
+    if info is None:
+        info = torch.zeros((4,), dtype=torch.int32, device=dev)
+    ws_bytes = lib().moe_balance_assign_workspace_size(m, n, k, MOE_QB_STEP)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    _check("moe_balance_step_minibatch", lib().moe_balance_step_minibatch(
+        _ptr(s), m, n, k, _ptr(beta), rule, seg_len, _ptr(topk_idx), _ptr(info), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return topk_idx, beta, info
 

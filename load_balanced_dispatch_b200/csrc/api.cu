@@ -12,6 +12,7 @@ cudaError_t launch_router(const void* x, moe_dtype dt, const float* w_r, const f
                           int n, int k, int fn, int renorm, const float* rank_bias, float* probs_out,
                           int32_t* topk_idx, float* topk_gate, void* workspace, cudaStream_t stream);
 size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt);
+cudaError_t launch_router_split(const float* w_r, int d, int n, void* workspace, cudaStream_t stream);
 bool router_uses_tc(moe_dtype dt, const float* logits_in, int n, int k);
 cudaError_t launch_capacity(const int32_t* topk_idx, int64_t m, int k, int n, int32_t capacity, int64_t seg_len,
                             int32_t* slot, int32_t* dest_row, int32_t* src_token, int32_t* expert_offsets,
@@ -43,6 +44,9 @@ cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, in
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k);
 int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, float gamma, int rule,
                           int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream, const char** err);
+int run_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* beta, int rule, int64_t seg_len,
+                               int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream,
+                               const char** err);
 int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int mode, int rule, int max_iters,
                        int max_repair, int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream,
                        const char** err);
@@ -117,7 +121,10 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, c
     REQUIRE(x_dtype == MOE_F32 || x_dtype == MOE_BF16, "unknown dtype");
     REQUIRE(m == 0 || (topk_idx && topk_gate), "topk_idx and topk_gate are required");
     if (!logits_in) {
-        REQUIRE(m == 0 || (x && w_r), "x and w_r are required when logits_in is NULL");
+        REQUIRE(m == 0 || x, "x is required when logits_in is NULL");
+        REQUIRE(m == 0 || w_r || router_uses_tc(x_dtype, logits_in, n, k),
+                "w_r may be NULL only on the tensor-core path (bf16 x, n <= 128), with a workspace prepared by "
+                "moe_router_prepare");
         REQUIRE(d >= 1, "d must be >= 1");
         REQUIRE(x_dtype != MOE_BF16 || d % 8 == 0, "d must be a multiple of 8 for bf16 x");
         REQUIRE(x_dtype != MOE_BF16 || m == 0 || aligned16(x), "bf16 x must be 16-byte aligned");
@@ -131,6 +138,23 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, const float* w_r, c
     return check_launch(launch_router(x, x_dtype, w_r, logits_in, m, d, n, k, (int)fn, renorm_topk, rank_bias,
                                       probs_out, topk_idx, topk_gate, workspace, stream),
                         "moe_router_topk");
+}
+
+moe_status moe_router_prepare(const float* w_r, int32_t d, int32_t n, int32_t k, moe_dtype x_dtype, void* workspace,
+                              size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(k >= 1 && k <= n, "k must be in [1, n]");
+    REQUIRE(d >= 1, "d must be >= 1");
+    REQUIRE(x_dtype == MOE_F32 || x_dtype == MOE_BF16, "unknown dtype");
+    REQUIRE(w_r, "w_r is required");
+    if (!router_uses_tc(x_dtype, nullptr, n, k))
+        return fail(MOE_ERR_UNSUPPORTED, "moe_router_prepare: this shape takes the fp32 FMA router, which reads w_r "
+                                         "directly; pass w_r to moe_router_topk");
+    REQUIRE(d % 8 == 0, "d must be a multiple of 8 for bf16 x");
+    const size_t need = router_workspace_bytes(d, n, x_dtype);
+    if (ws_bytes < need || !workspace || !aligned16(workspace))
+        return fail(MOE_ERR_WORKSPACE, "moe_router_prepare: 16-byte aligned workspace of %zu bytes required", need);
+    return check_launch(launch_router_split(w_r, d, n, workspace, stream), "moe_router_prepare");
 }
 
 size_t moe_capacity_slots_workspace_size(int64_t m, int32_t k, int32_t n, int64_t seg_len) {
@@ -352,6 +376,27 @@ moe_status moe_balance_sign_step(const float* s, int64_t m, int32_t n, int32_t k
     const char* err = "";
     const int rc = run_balance_sign_step(s, m, n, k, beta, gamma, rule, topk_idx, info, workspace, stream, &err);
     if (rc != MOE_OK) return fail((moe_status)rc, "moe_balance_sign_step: %s", err);
+    return MOE_OK;
+}
+
+moe_status moe_balance_step_minibatch(const float* s, int64_t m, int32_t n, int32_t k, float* beta,
+                                      moe_qb_threshold rule, int64_t seg_len, int32_t* topk_idx, int32_t* info,
+                                      void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    REQUIRE(m >= 1, "m must be >= 1");
+    REQUIRE(n >= 2 && n <= kMaxExperts, "n must be in [2, %d]", kMaxExperts);
+    REQUIRE(k >= 1 && k < n, "k must be in [1, n - 1]");
+    REQUIRE(m * (int64_t)k < ((int64_t)1 << 31) && m * (int64_t)n < ((int64_t)1 << 34), "m too large");
+    REQUIRE(seg_len >= 1 && m % seg_len == 0, "seg_len must be >= 1 and divide m");
+    REQUIRE((seg_len * k) % n == 0, "seg_len * k must be divisible by n (each mini-batch's column count)");
+    REQUIRE(m / seg_len <= 4096, "at most 4096 mini-batches");
+    REQUIRE(rule == MOE_QB_MIDPOINT || rule == MOE_QB_BOUNDARY || rule == MOE_QB_BIP, "unknown threshold rule");
+    REQUIRE(s && beta && topk_idx && info, "s, beta, topk_idx and info are required");
+    const size_t need = balance_workspace_bytes(m, n, k);
+    if (ws_bytes < need || !workspace) return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+    const char* err = "";
+    const int rc = run_balance_step_minibatch(s, m, n, k, beta, rule, seg_len, topk_idx, info, workspace, stream, &err);
+    if (rc != MOE_OK) return fail((moe_status)rc, "moe_balance_step_minibatch: %s", err);
+    g_last_error[0] = 0;
     return MOE_OK;
 }
 

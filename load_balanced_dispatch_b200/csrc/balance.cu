@@ -50,6 +50,7 @@ constexpr int kColThreads = 512;  // qb_col_kernel block size (its scan buffer i
 enum { kStDone = 0, kStAugments = 1, kStError = 2, kStQbDone = 4, kStIters = 5, kStTies0 = 6, kStTies1 = 7,
        kStWords = 8 };
 constexpr int kBatch = 16;  // QB iterations enqueued between host checks
+constexpr int64_t kMaxMiniBatches = 4096;  // mini-batches of one averaged-beta step
 }  // namespace qb
 
 // Threshold between the q-th (a) and (q+1)-th (b) largest: midpoint, the (q+1)-th, or the
@@ -668,6 +669,85 @@ __device__ __forceinline__ void rank_select2(const unsigned* list, unsigned ncan
     __syncthreads();
 }
 
+// The C-th and (C+1)-th largest keys of fp32(col[i * stride] - alpha[i]) over i < m, by the full
+// radix path: a 12-bit digit histogram sweep, a sweep keeping the selected bin's keys (the largest
+// key below the bin is tracked), then the low digits over the kept keys (streamed from global
+// memory if the bin overflows the shared list). Called by every thread of the block; the keys
+// come back in every thread.
+__device__ void column_select_full(const float* __restrict__ col, int64_t stride, const float* __restrict__ alpha,
+                                   int64_t m, int64_t C, unsigned* hist, unsigned* scan, unsigned* cand,
+                                   unsigned* s_ncand_p, uint32_t* akey_out, uint32_t* bkey_out) {
+    const int tid = threadIdx.x, T = blockDim.x;
+    unsigned& s_ncand = *s_ncand_p;
+    unsigned ncand;
+    uint32_t akey, bkey;
+    // ---- full radix path
+    uint32_t below = 0;
+    for (int b = tid; b < 4096; b += T) hist[b] = 0;
+    __syncthreads();
+    for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) { warp_hist_add(hist, ok, key >> 20); });
+    __syncthreads();
+    int sel1;
+    int64_t want1;
+    unsigned cnt1;
+    block_select_bin(hist, 4096, C, scan, &sel1, &want1, &cnt1);
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
+        const uint32_t d = key >> 20;
+        if (ok && d < (uint32_t)sel1 && key > below) below = key;
+        warp_append(cand, &s_ncand, ok && d == (uint32_t)sel1, key);
+    });
+    below = block_max_u32(below, scan);
+    ncand = s_ncand;
+    if (ncand <= (unsigned)qb::kCandCap) {
+        unsigned mult;
+        int64_t greater;
+        select_in_list(cand, ncand, want1, hist, scan, &akey, &mult, &greater);
+        greater += C - want1;
+        if (greater + (int64_t)mult >= C + 1) {
+            bkey = akey;
+        } else {
+            const uint32_t best = list_max_below(cand, ncand, akey, scan);
+            bkey = best ? best : below;
+        }
+    } else {
+        // the bin overflows the list: its low digits stream from global memory
+        int sel2, sel3;
+        int64_t want2, want3;
+        unsigned cnt2, cnt3;
+        for (int b = tid; b < 4096; b += T) hist[b] = 0;
+        __syncthreads();
+        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
+            warp_hist_add(hist, ok && (key >> 20) == (uint32_t)sel1, (key >> 8) & 0xfffu);
+        });
+        __syncthreads();
+        block_select_bin(hist, 4096, want1, scan, &sel2, &want2, &cnt2);
+        const uint32_t pre2 = ((uint32_t)sel1 << 20) | ((uint32_t)sel2 << 8);
+        for (int b = tid; b < 256; b += T) hist[b] = 0;
+        __syncthreads();
+        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
+            warp_hist_add(hist, ok && (key & 0xffffff00u) == pre2, key & 0xffu);
+        });
+        __syncthreads();
+        block_select_bin(hist, 256, want2, scan, &sel3, &want3, &cnt3);
+        akey = pre2 | (uint32_t)sel3;
+        const int64_t greater = C - want3;
+        if (greater + (int64_t)cnt3 >= C + 1) {
+            bkey = akey;
+        } else {
+            uint32_t best = 0;
+            for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
+                if (ok && (key >> 20) == (uint32_t)sel1 && key < akey && key > best) best = key;
+            });
+            best = block_max_u32(best, scan);
+            bkey = best ? best : below;
+        }
+    }
+    *akey_out = akey;
+    *bkey_out = bkey;
+}
+
 // Column pass, part 2: beta_j = threshold between the C-th and (C+1)-th largest key of column j
 // of u = fp32(s - alpha). When both fell inside the window of part 1 (the usual case once the
 // iteration settles) they come from the column's candidate list, copied into shared memory:
@@ -739,69 +819,7 @@ qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t
         greater += above;
         bkey = greater + (int64_t)mult >= C + 1 ? akey : list_max_below(cand, ncand, akey, scan);
     } else {
-        // ---- full radix path
-        uint32_t below = 0;
-        for (int b = tid; b < 4096; b += T) hist[b] = 0;
-        __syncthreads();
-        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) { warp_hist_add(hist, ok, key >> 20); });
-        __syncthreads();
-        int sel1;
-        int64_t want1;
-        unsigned cnt1;
-        block_select_bin(hist, 4096, C, scan, &sel1, &want1, &cnt1);
-        if (tid == 0) s_ncand = 0;
-        __syncthreads();
-        for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
-            const uint32_t d = key >> 20;
-            if (ok && d < (uint32_t)sel1 && key > below) below = key;
-            warp_append(cand, &s_ncand, ok && d == (uint32_t)sel1, key);
-        });
-        below = block_max_u32(below, scan);
-        ncand = s_ncand;
-        if (ncand <= (unsigned)qb::kCandCap) {
-            unsigned mult;
-            int64_t greater;
-            select_in_list(cand, ncand, want1, hist, scan, &akey, &mult, &greater);
-            greater += C - want1;
-            if (greater + (int64_t)mult >= C + 1) {
-                bkey = akey;
-            } else {
-                const uint32_t best = list_max_below(cand, ncand, akey, scan);
-                bkey = best ? best : below;
-            }
-        } else {
-            // the bin overflows the list: its low digits stream from global memory
-            int sel2, sel3;
-            int64_t want2, want3;
-            unsigned cnt2, cnt3;
-            for (int b = tid; b < 4096; b += T) hist[b] = 0;
-            __syncthreads();
-            for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
-                warp_hist_add(hist, ok && (key >> 20) == (uint32_t)sel1, (key >> 8) & 0xfffu);
-            });
-            __syncthreads();
-            block_select_bin(hist, 4096, want1, scan, &sel2, &want2, &cnt2);
-            const uint32_t pre2 = ((uint32_t)sel1 << 20) | ((uint32_t)sel2 << 8);
-            for (int b = tid; b < 256; b += T) hist[b] = 0;
-            __syncthreads();
-            for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
-                warp_hist_add(hist, ok && (key & 0xffffff00u) == pre2, key & 0xffu);
-            });
-            __syncthreads();
-            block_select_bin(hist, 256, want2, scan, &sel3, &want3, &cnt3);
-            akey = pre2 | (uint32_t)sel3;
-            const int64_t greater = C - want3;
-            if (greater + (int64_t)cnt3 >= C + 1) {
-                bkey = akey;
-            } else {
-                uint32_t best = 0;
-                for_each_col_key(col, stride, alpha, m, [&](bool ok, uint32_t key) {
-                    if (ok && (key >> 20) == (uint32_t)sel1 && key < akey && key > best) best = key;
-                });
-                best = block_max_u32(best, scan);
-                bkey = best ? best : below;
-            }
-        }
+        column_select_full(col, stride, alpha, m, C, hist, scan, cand, &s_ncand, &akey, &bkey);
     }
     if (tid == 0) {
         const float bnew = qb_threshold(key_float(akey), key_float(bkey), rule);
@@ -812,6 +830,58 @@ qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t
         uint64_t wn = 2 * dist + (uint64_t)(akey - bkey) + qb::kWinMin;
         if (wn > qb::kWinMax) wn = qb::kWinMax;
         win[j] = (uint32_t)wn;
+    }
+}
+
+// The practical QB step on mini-batches ("MoE travelogue 6", Mind the pitfall, closing
+// paragraph): beta computed by the formula on each mini-batch of L tokens, then averaged. One CTA
+// per (expert j, mini-batch b): the C_b-th and (C_b + 1)-th largest of fp32(s_ij - alpha_i) over
+// the mini-batch's tokens, read from sT (contiguous). A mini-batch of at most kCandCap tokens has
+// all its keys copied into shared memory and selected there (ranks for at most one key per
+// thread, else radix digits); a longer one takes the full radix path over global memory.
+__global__ void __launch_bounds__(qb::kColThreads)
+qb_col_slice_kernel(const float* __restrict__ sT, int64_t m, int n, int64_t L, int64_t Cb,
+                    const float* __restrict__ alpha, int rule, float* __restrict__ beta_parts) {
+    extern __shared__ unsigned col_smem[];
+    unsigned* hist = col_smem;                 // 4096
+    unsigned* scan = hist + 4096;              // blockDim
+    unsigned* cand = scan + qb::kColThreads;   // kCandCap
+    __shared__ unsigned s_ncand;
+    __shared__ uint32_t s_sel[2];
+    const int tid = threadIdx.x;
+    const int j = blockIdx.x;
+    const int64_t b = blockIdx.y;
+    const float* col = sT + (int64_t)j * m + b * L;
+    const float* a = alpha + b * L;
+    uint32_t akey, bkey;
+    if (L <= (int64_t)qb::kCandCap) {
+        if (tid == 0) s_ncand = 0;
+        __syncthreads();
+        for_each_col_key(col, 1, a, L, [&](bool ok, uint32_t key) { warp_append(cand, &s_ncand, ok, key); });
+        __syncthreads();
+        const unsigned ncand = (unsigned)L;
+        if (ncand <= (unsigned)blockDim.x) {
+            rank_select2(cand, ncand, Cb, s_sel);
+            akey = s_sel[0];
+            bkey = s_sel[1];
+        } else {
+            unsigned mult;
+            int64_t greater;
+            select_in_list(cand, ncand, Cb, hist, scan, &akey, &mult, &greater);
+            bkey = greater + (int64_t)mult >= Cb + 1 ? akey : list_max_below(cand, ncand, akey, scan);
+        }
+    } else {
+        column_select_full(col, 1, a, L, Cb, hist, scan, cand, &s_ncand, &akey, &bkey);
+    }
+    if (tid == 0) beta_parts[b * n + j] = qb_threshold(key_float(akey), key_float(bkey), rule);
+}
+
+// beta_j = fp32((sum over b in order of (double) beta_parts[b][j]) / B).
+__global__ void qb_beta_mean_kernel(const float* __restrict__ beta_parts, int64_t nb, int n, float* __restrict__ beta) {
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        double acc = 0.0;
+        for (int64_t b = 0; b < nb; ++b) acc += (double)beta_parts[b * n + j];
+        beta[j] = (float)(acc / (double)nb);
     }
 }
 
@@ -1350,6 +1420,7 @@ struct QBWorkspace {
     int32_t* moves;        // [n][3] the last repair move: token, from, to per hop
     int32_t* nmoves;       // [2] hops of the last move, entries queued for recomputation
     int32_t* rec;          // [n * n] queued entries x * n + y
+    float* beta_parts;     // [kMaxMiniBatches][n] per-mini-batch beta of the mini-batch step
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -1382,6 +1453,7 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
     p = take(sizeof(int32_t) * 3 * (size_t)(n + 1));    if (w) w->moves = (int32_t*)p;
     p = take(sizeof(int32_t) * 2);                      if (w) w->nmoves = (int32_t*)p;
     p = take(sizeof(int32_t) * (size_t)n * n);          if (w) w->rec = (int32_t*)p;
+    p = take(sizeof(float) * (size_t)qb::kMaxMiniBatches * n); if (w) w->beta_parts = (float*)p;
     return off;
 }
 
@@ -1549,6 +1621,37 @@ int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, 
         else qb_sign_count_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
         qb_sign_update_kernel<<<1, 256, 0, stream>>>(sc, n, C, gamma, beta);
     }
+    qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
+    if ((ce = cudaGetLastError()) != cudaSuccess) goto fail;
+    return MOE_OK;
+fail:
+    *err = cudaGetErrorString(ce);
+    return MOE_ERR_CUDA;
+}
+
+// The practical QB step with beta averaged over mini-batches of seg_len tokens: the row pass of
+// STEP (selection with the old beta; it also writes s transposed), one column select per
+// (expert, mini-batch), the fixed-order mean. Fully asynchronous.
+int run_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* beta, int rule, int64_t seg_len,
+                               int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream,
+                               const char** err) {
+    QBWorkspace w;
+    qb_layout(m, n, k, &w, static_cast<char*>(workspace));
+    const int64_t C = m * k / n, nb = m / seg_len, Cb = seg_len * k / n;
+    cudaError_t ce;
+    static bool attr = false;
+    if (!attr) {
+        if ((ce = cudaFuncSetAttribute(qb_col_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)qb::kColSmem)) != cudaSuccess)
+            goto fail;
+        attr = true;
+    }
+    if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 2 * n), stream)) != cudaSuccess)
+        goto fail;
+    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, w.sT, stream);
+    qb_col_slice_kernel<<<dim3((unsigned)n, (unsigned)nb), qb::kColThreads, qb::kColSmem, stream>>>(
+        w.sT, m, n, seg_len, Cb, w.alpha, rule, w.beta_parts);
+    qb_beta_mean_kernel<<<1, 256, 0, stream>>>(w.beta_parts, nb, n, beta);
     qb_info_kernel<<<1, 32, 0, stream>>>(w.counts, n, C, w.status, 1, qb::kStTies0, info);
     if ((ce = cudaGetLastError()) != cudaSuccess) goto fail;
     return MOE_OK;

@@ -8,23 +8,25 @@
 // so x.W_r = x.w0 + x.w1 + x.w2 where every bf16 x bf16 product is exact and
 // the tensor core accumulates in fp32: fp32-accurate logits at tensor-core speed.
 //
-//   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand)
-//   router_tc_kernel     one CTA per 128 tokens and 64-wide column tile of experts
-//                        (n <= 128, so one or two tiles), 192 threads:
-//     warp 0 lane 0   TMA: x tile 128x64 + the three W parts of the tile per stage
-//     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = the tile width (3 parts x 4 K-steps per stage)
-//     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM
-//                     lane); each K block's product lands in a fresh TMEM accumulator
-//                     (two, ping-pong) and is added into fp32 registers with
-//                     round-to-nearest adds, which keeps the sum fp32-accurate;
-//                     then the warp parks its 32 rows in shared memory.
-//   Finish. With probs_out the logits are stored (coalesced) and router_finish_kernel
-//   (one warp per row, the whole GPU) finishes them in place. Without it, for k <= 8
-//   the CTAs of the two column tiles of the same tokens form a 2-CTA cluster: thread
-//   r of each finishes row r over its own columns and trades the row maximum, the
-//   exp-sum and its local top-k with the peer through distributed shared memory, and
-//   rank 0 writes the picks. For larger k without probs_out each CTA takes whole rows
-//   (one tile of all n experts) and a warp finishes each row.
+//   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand);
+//                        run once per weight by moe_router_prepare, or on every call.
+//   router_rows_kernel   (k <= 8) persistent, one CTA per SM, 192 threads, each CTA
+//                        taking 128-token blocks in turn with all n <= 128 experts:
+//     warp 0 lane 0   TMA: x tile 128x64 + the three W parts (all n rows) per stage
+//     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = n rounded up to 32 (3 parts x 4 K-steps)
+//     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM lane);
+//                     each K block's product lands in a fresh TMEM accumulator (two,
+//                     ping-pong) and is added into fp32 registers with round-to-nearest
+//                     adds, which keeps the sum fp32-accurate. After a block's last K
+//                     block the thread finishes its row in registers (softmax or
+//                     logistic, ranking key, top-k with ties to the lower index, gates)
+//                     while the MMA warp already runs the next block, and the scores go
+//                     out coalesced through a per-warp shared-memory transpose. Logits
+//                     never reach HBM.
+//   router_tc_kernel     (k > 8) one CTA per 128 tokens and column tile: with probs_out
+//                        the logits are stored and router_finish_kernel (a warp per row)
+//                        finishes them in place; without it each CTA takes whole rows and
+//                        a warp finishes each.
 #include "tc_ptx.cuh"
 
 namespace moe {
@@ -83,7 +85,8 @@ __global__ void router_split_kernel(const float* __restrict__ w_r, int d, int n,
 constexpr int KTHREAD = 8;  // largest k finished one row per thread
 
 namespace rtc {
-enum { kModeLogits = 0, kModeFused = 1, kModeRows = 2 };
+enum { kModeLogits = 0, kModeRows = 2 };
+constexpr int kParkPitch = 33;  // padded row pitch of a warp's 32 x 32 transpose tile
 }  // namespace rtc
 
 // Insert (key, j, p) into a best-first list of length k <= KTHREAD (ties: the lower index first).
@@ -102,132 +105,6 @@ __device__ __forceinline__ void topk_insert(float (&kk)[KTHREAD], int (&ki)[KTHR
             }
         }
     }
-}
-
-// Score function, ranking and top-k of 128 token rows whose logits are parked in shared memory
-// (`rows`, pitch NP + 1, this CTA's expert columns col0 .. col0 + NP - 1), one row per thread of
-// warps 2-5. With `paired`, the other CTA of the 2-CTA cluster holds the other column tile of the
-// same rows: the row maximum, the exp-sum and the local top-k lists are exchanged through
-// distributed shared memory (`xch`, read by the peer), and the peer's partial sums are added in
-// cluster-rank order so both CTAs agree bit for bit. CTA rank 0 writes the picks and gates; each
-// CTA stores its own columns of probs_out, coalesced. Called by all 192 threads of both CTAs:
-// every barrier is reached by every thread whatever happened before (`ok` only gates the work).
-template <int NP>
-__device__ void fused_finish(float* rows, float* xch, bool paired, bool ok, int64_t row0, int col0, int64_t m, int n,
-                             int k, int fn, int renorm, const float* __restrict__ rank_bias,
-                             float* __restrict__ probs_out, int32_t* __restrict__ topk_idx,
-                             float* __restrict__ topk_gate) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool worker = warp >= 2 && ok;
-    const int quad = warp & 3, r = quad * 32 + lane;
-    float* h = rows + r * (NP + 1);
-    float* xmax = xch;                                   // [128]
-    float* xsum = xch + 128;                             // [128]
-    float* lkey = xch + 256;                             // [128][KTHREAD]
-    int* lidx = reinterpret_cast<int*>(xch + 256 + 128 * KTHREAD);
-    float* lp = xch + 256 + 2 * 128 * KTHREAD;
-    const int nloc = max(0, min(NP, n - col0));          // real experts in this tile
-    const uint32_t peer = paired ? (ptx::cluster_ctarank() ^ 1u) : 0u;
-    const bool first = !paired || ptx::cluster_ctarank() == 0;
-    auto sync = [&]() {
-        if (paired) ptx::cluster_sync();
-        else __syncthreads();
-    };
-    auto peer_addr = [&](const void* p) { return ptx::mapa_shared(ptx::smem_u32(p), peer); };
-    const bool softmax = fn == MOE_SOFTMAX;
-
-    // 1. row maximum (softmax)
-    float mx = -INFINITY;
-    if (worker && softmax)
-        for (int j = 0; j < nloc; ++j) mx = fmaxf(mx, h[j]);
-    if (worker) xmax[r] = mx;
-    sync();
-    if (worker && paired && softmax) mx = fmaxf(mx, ptx::ld_cluster_f32(peer_addr(xmax + r)));
-    // 2. sum of exp(h - max), added in cluster-rank order
-    float s = 0.f;
-    if (worker && softmax)
-        for (int j = 0; j < nloc; ++j) s += expf(h[j] - mx);
-    if (worker) xsum[r] = s;
-    sync();
-    if (worker && paired && softmax) {
-        const float so = ptx::ld_cluster_f32(peer_addr(xsum + r));
-        s = first ? s + so : so + s;
-    }
-    // 3. scores (parked back over the logits), keys, this tile's top-k
-    float kk[KTHREAD], kp[KTHREAD];
-    int ki[KTHREAD];
-#pragma unroll
-    for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
-    if (worker) {
-        for (int j = 0; j < nloc; ++j) {
-            const float hj = h[j];
-            const float p = softmax ? expf(hj - mx) / s : 1.f / (1.f + expf(-hj));
-            h[j] = p;
-            const float key = rank_bias ? __fadd_rn(p, rank_bias[col0 + j]) : (softmax ? hj : p);
-            topk_insert(kk, ki, kp, k, key, col0 + j, p);
-        }
-#pragma unroll
-        for (int t = 0; t < KTHREAD; ++t)
-            if (t < k) { lkey[r * KTHREAD + t] = kk[t]; lidx[r * KTHREAD + t] = ki[t]; lp[r * KTHREAD + t] = kp[t]; }
-    }
-    sync();
-    // 4. merge with the peer's list: each entry's place = its own rank + the other list's entries
-    //    ranking before it (a strict order, so the places are a permutation); rank 0 writes
-    const int64_t row = row0 + r;
-    if (worker && first && row < m) {
-        float ok2[KTHREAD], op[KTHREAD];
-        int oi[KTHREAD];
-#pragma unroll
-        for (int t = 0; t < KTHREAD; ++t) {
-            ok2[t] = -INFINITY; oi[t] = 0x7fffffff; op[t] = 0.f;
-            if (paired && t < k) {
-                ok2[t] = ptx::ld_cluster_f32(peer_addr(lkey + r * KTHREAD + t));
-                oi[t] = ptx::ld_cluster_s32(peer_addr(lidx + r * KTHREAD + t));
-                op[t] = ptx::ld_cluster_f32(peer_addr(lp + r * KTHREAD + t));
-            }
-        }
-        int pa[KTHREAD], pb[KTHREAD];
-        float selsum = 0.f;
-#pragma unroll
-        for (int t = 0; t < KTHREAD; ++t) {
-            int ca = t, cb = t;
-#pragma unroll
-            for (int u = 0; u < KTHREAD; ++u) {
-                if (u < k && ranks_before(ok2[u], oi[u], kk[t], ki[t])) ++ca;
-                if (u < k && ranks_before(kk[u], ki[u], ok2[t], oi[t])) ++cb;
-            }
-            pa[t] = t < k ? ca : KTHREAD;
-            pb[t] = t < k ? cb : KTHREAD;
-            if (pa[t] < k) selsum += kp[t];
-            if (pb[t] < k) selsum += op[t];
-        }
-        const bool renorm_gate = softmax && renorm;
-#pragma unroll
-        for (int t = 0; t < KTHREAD; ++t) {
-            if (pa[t] < k) {
-                topk_idx[row * k + pa[t]] = ki[t];
-                topk_gate[row * k + pa[t]] = renorm_gate ? kp[t] / selsum : kp[t];
-            }
-            if (pb[t] < k) {
-                topk_idx[row * k + pb[t]] = oi[t];
-                topk_gate[row * k + pb[t]] = renorm_gate ? op[t] / selsum : op[t];
-            }
-        }
-    }
-    // 5. this tile's scores out, coalesced: the warp stores its 32 rows
-    if (worker && probs_out) {
-        __syncwarp();
-        for (int rr = 0; rr < 32; ++rr) {
-            const int64_t rw = row0 + quad * 32 + rr;
-            if (rw >= m) break;
-#pragma unroll
-            for (int q = 0; q < NP / 32; ++q) {
-                const int j = lane + 32 * q;
-                if (j < nloc) probs_out[rw * n + col0 + j] = rows[(quad * 32 + rr) * (NP + 1) + j];
-            }
-        }
-    }
-    sync();  // the peer has finished reading this CTA's exchange area
 }
 
 template <int NCH, int STAGES>
@@ -361,16 +238,219 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             }
         }
     }
-    if (mode == kModeFused)
-        fused_finish<NP>(reinterpret_cast<float*>(smem), reinterpret_cast<float*>(smem) + BM * (NP + 1),
-                         gridDim.y == 2, drain_ok, row0, col0, m, n, k, fn, renorm, rank_bias, probs_out, topk_idx,
-                         topk_gate);
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, tcols);
     }
+}
+
+// Persistent full-row router (k <= KTHREAD): see the file header. Every barrier wait is bounded;
+// on a timeout all roles leave their loops and TMEM is freed.
+template <int NCH, int STAGES>
+__global__ void __launch_bounds__(rtc::kThreads, 1)
+router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
+                   int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
+                   float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+    using namespace rtc;
+    constexpr int NP = NCH * 32;
+    constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* park = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [4 warps][32][kParkPitch]
+    RouterTcShared* sh = reinterpret_cast<RouterTcShared*>(park + 4 * 32 * kParkPitch);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = (d + BK - 1) / BK;
+    const int64_t nblocks = (m + BM - 1) / BM;
+    const uint32_t tcols = router_tmem_cols(NP);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        sh->abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::prefetch_tensormap(&map_x);
+        ptx::prefetch_tensormap(&map_w);
+    }
+    if (warp == 1) ptx::tmem_alloc(&sh->tmem_base, tcols);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    pdl_trigger();
+    pdl_wait();  // x (and the W split when made by this call) come from earlier launches
+    const uint32_t tmem = sh->tmem_base;
+    volatile int* abort_flag = &sh->abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                    uint8_t* st = smem + stage * STAGE_BYTES;
+                    ptx::mbar_expect_tx(&sh->full[stage], (uint32_t)STAGE_BYTES);
+                    ptx::tma_load_2d(st, &map_x, &sh->full[stage], kb * BK, (int)(tb * BM));
+                    for (int part = 0; part < 3; ++part)
+                        ptx::tma_load_3d(st + A_BYTES + part * NP * 128, &map_w, &sh->full[stage], kb * BK, 0, part);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, NP);
+            int stage = 0, buf = 0;
+            uint32_t phase = 0, bphase = 0;
+            bool ok = true;
+            for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!ptx::mbar_wait(&sh->tempty[buf], bphase ^ 1u, abort_flag)) { ok = false; break; }
+                    if (!ptx::mbar_wait(&sh->full[stage], phase, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = ptx::smem_u32(smem + stage * STAGE_BYTES);
+                    const uint64_t adesc = ptx::sw128_kmajor_desc(sa);
+                    // a fresh accumulator per K block; the small parts of W first, the leading part last
+                    for (int part = 2; part >= 0; --part) {
+                        const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + A_BYTES + part * NP * 128);
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            ptx::umma_bf16(tmem + (uint32_t)(buf * NP), adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                           (part != 2 || kk != 0) ? 1u : 0u);
+                    }
+                    ptx::umma_commit(&sh->empty[stage]);
+                    ptx::umma_commit(&sh->tfull[buf]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    if (++buf == 2) { buf = 0; bphase ^= 1u; }
+                }
+            }
+        }
+    } else {
+        const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31 belong to this warp
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        float* pk = park + quad * 32 * kParkPitch;
+        const bool softmax = fn == MOE_SOFTMAX;
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
+            float acc[NP];
+#pragma unroll
+            for (int j = 0; j < NP; ++j) acc[j] = 0.f;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                // two 32-column chunks in flight per wait
+#pragma unroll
+                for (int c = 0; c < NCH; c += 2) {
+                    uint32_t v[2][32];
+                    ptx::tmem_ld32_issue(trow + (uint32_t)(buf * NP + c * 32), v[0]);
+                    if (c + 1 < NCH) ptx::tmem_ld32_issue(trow + (uint32_t)(buf * NP + (c + 1) * 32), v[1]);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[0][q]));
+                    if (c + 1 < NCH) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            acc[(c + 1) * 32 + q] = __fadd_rn(acc[(c + 1) * 32 + q], __uint_as_float(v[1][q]));
+                    }
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&sh->tempty[buf]);
+                if (++buf == 2) { buf = 0; bphase ^= 1u; }
+            }
+            if (!ok) break;
+            // finish this thread's row: scores, ranking keys, top-k (ties -> lower index), gates
+            const int64_t row0w = tb * BM + quad * 32;
+            const int64_t row = row0w + lane;
+            float mx = -INFINITY, sum = 0.f;
+            if (softmax) {
+#pragma unroll
+                for (int j = 0; j < NP; ++j) if (j < n) mx = fmaxf(mx, acc[j]);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) if (j < n) sum += expf(acc[j] - mx);
+            }
+            float kk[KTHREAD], kp[KTHREAD];
+            int ki[KTHREAD];
+#pragma unroll
+            for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                if (j < n) {
+                    const float hj = acc[j];
+                    const float p = softmax ? expf(hj - mx) / sum : 1.f / (1.f + expf(-hj));
+                    const float key = rank_bias ? __fadd_rn(p, rank_bias[j]) : (softmax ? hj : p);
+                    topk_insert(kk, ki, kp, k, key, j, p);
+                    acc[j] = p;
+                }
+            }
+            if (row < m) {
+                float selsum = 0.f;
+#pragma unroll
+                for (int t = 0; t < KTHREAD; ++t) if (t < k) selsum += kp[t];
+                const bool renorm_gate = softmax && renorm;
+#pragma unroll
+                for (int t = 0; t < KTHREAD; ++t) {
+                    if (t < k) {
+                        topk_idx[row * k + t] = ki[t];
+                        topk_gate[row * k + t] = renorm_gate ? kp[t] / selsum : kp[t];
+                    }
+                }
+            }
+            if (probs_out) {
+                // the warp's 32 rows of scores, 32 columns at a time through shared memory: each
+                // store instruction writes 128 contiguous bytes of one row
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    __syncwarp();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) pk[lane * kParkPitch + q] = acc[c * 32 + q];
+                    __syncwarp();
+                    const int j = c * 32 + lane;
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const int64_t r = row0w + rr;
+                        if (r >= m) break;
+                        if (j < n) probs_out[r * n + j] = pk[rr * kParkPitch + lane];
+                    }
+                }
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, tcols);
+    }
+}
+
+inline size_t router_rows_smem(int np, int stages) {
+    return 1024 + (size_t)stages * router_stage_bytes(np) + (size_t)4 * 32 * rtc::kParkPitch * 4 +
+           sizeof(RouterTcShared);
+}
+
+// Ring depth of the rows kernel: as many stages as fit next to the transpose tiles (at most 6).
+constexpr int router_rows_stages(int nch) { return nch == 1 ? 6 : (nch == 2 ? 4 : 3); }
+
+template <int NCH>
+static cudaError_t launch_router_rows_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
+                                        int fn, int renorm, const float* rank_bias, float* probs_out,
+                                        int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
+    constexpr int ST = router_rows_stages(NCH);
+    const size_t smem = router_rows_smem(NCH * 32, ST);
+    static bool attr = false;
+    if (!attr) {
+        const cudaError_t e = cudaFuncSetAttribute(router_rows_kernel<NCH, ST>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
+    const unsigned grid = (unsigned)(blocks < num_sms() ? blocks : num_sms());
+    return launch_pdl(router_rows_kernel<NCH, ST>, dim3(grid), dim3(rtc::kThreads), smem, stream, mx, mw, m, d, n, k,
+                      fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
 }
 
 size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt) {
@@ -396,19 +476,11 @@ static cudaError_t launch_router_tc_st(const CUtensorMap& mx, const CUtensorMap&
     cfg.blockDim = dim3(rtc::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute at[2];
+    cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (mode == rtc::kModeFused && grid.y == 2) {
-        // the two column tiles of the same 128 tokens form a cluster (exchange through DSMEM)
-        at[1].id = cudaLaunchAttributeClusterDimension;
-        at[1].val.clusterDim.x = 1;
-        at[1].val.clusterDim.y = 2;
-        at[1].val.clusterDim.z = 1;
-        cfg.numAttrs = 2;
-    }
     return cudaLaunchKernelEx(&cfg, router_tc_kernel<NCH, ST>, mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out,
                               topk_idx, topk_gate, mode);
 }
@@ -435,27 +507,41 @@ static cudaError_t launch_router_tc_t(const CUtensorMap& mx, const CUtensorMap& 
 // Tensor-core router for bf16 activations with n <= 128 (the drain keeps a token's n logits in registers).
 bool router_tc_supported(int n, int k) { (void)k; return n <= rtc::NMAX; }
 
+// W_r [d, n] fp32 -> the [3, n, d] bf16 split in the workspace (moe_router_prepare, or every call).
+cudaError_t launch_router_split(const float* w_r, int d, int n, void* workspace, cudaStream_t stream) {
+    dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
+    return launch_pdl(router_split_kernel, tg, tb, 0, stream, w_r, d, n, static_cast<__nv_bfloat16*>(workspace));
+}
+
+// w_r == nullptr: the workspace already holds the split of the router weight (moe_router_prepare).
 cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, int n, int k, int fn, int renorm,
                              const float* rank_bias, float* probs_out, int32_t* topk_idx, float* topk_gate,
                              void* workspace, cudaStream_t stream) {
     if (!router_tc_supported(n, k)) return cudaErrorNotSupported;
     if (m == 0) return cudaSuccess;
     __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(workspace);
-    {
-        dim3 tb(32, 8), tg((unsigned)((d + 31) / 32), (unsigned)((n + 31) / 32));
-        const cudaError_t e = launch_pdl(router_split_kernel, tg, tb, 0, stream, w_r, d, n, wsplit);
+    if (w_r) {
+        const cudaError_t e = launch_router_split(w_r, d, n, workspace, stream);
         if (e != cudaSuccess) return e;
     }
-    // With probs_out the logits go to memory in 64-wide column tiles and router_finish_kernel (a
-    // warp per row, the whole GPU) finishes them in place: measured faster than finishing in this
-    // kernel, where only four warps per SM share the rows. Without probs_out (nothing to store
-    // them in) the rows are finished here: for k <= KTHREAD by the paired-tile cluster, one row
-    // per thread; for larger k each CTA keeps whole rows and a warp finishes each.
     const int np = router_np(n);
-    const int mode = probs_out ? rtc::kModeLogits : (k <= KTHREAD ? rtc::kModeFused : rtc::kModeRows);
-    const int tile = mode == rtc::kModeRows ? np : (np < 64 ? np : 64);
     CUtensorMap mx, mw;
     if (!map_2d(&mx, x, (uint64_t)m, (uint64_t)d, rtc::BM)) return cudaErrorInvalidValue;
+    if (k <= KTHREAD) {
+        // every expert in one tile: the drain threads finish their rows in registers
+        if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)np)) return cudaErrorInvalidValue;
+        switch (np / 32) {
+            case 1: return launch_router_rows_t<1>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+            case 2: return launch_router_rows_t<2>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+            case 3: return launch_router_rows_t<3>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+            default: return launch_router_rows_t<4>(mx, mw, m, d, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate, stream);
+        }
+    }
+    // k > KTHREAD. With probs_out the logits go to memory in 64-wide column tiles and
+    // router_finish_kernel (a warp per row, the whole GPU) finishes them in place; without it
+    // (nothing to store them in) each CTA keeps whole rows and a warp finishes each.
+    const int mode = probs_out ? rtc::kModeLogits : rtc::kModeRows;
+    const int tile = mode == rtc::kModeRows ? np : (np < 64 ? np : 64);
     if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)tile)) return cudaErrorInvalidValue;
     cudaError_t e;
     switch (tile / 32) {

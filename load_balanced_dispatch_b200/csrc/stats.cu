@@ -135,7 +135,12 @@ __device__ __forceinline__ void fold_blocks(const int32_t* cnt, const double* ps
 // Whole-batch results from the batch totals held by thread e < n (routed copies `tot`, probability
 // sum `pall`) over m tokens: f and P rows, the loss on them, the violations and the Loss-Free
 // update. Every thread of the block calls it (block reductions inside). Optional outputs may be NULL.
-__device__ void finish_batch(int64_t tot, double pall, int64_t m, int n, int k, bool has_probs, float alpha,
+// Weight of the micro-batch loss in the hybrid loss ("Qwen global-batch load balance", balancing
+// efficiency and effectiveness: the micro-batch loss added to the global-batch loss with 0.01).
+constexpr double kHybridMicroWeight = 0.01;
+
+// Whole-batch f, P, loss, violations and bias update; returns the loss (0 without scores).
+__device__ double finish_batch(int64_t tot, double pall, int64_t m, int n, int k, bool has_probs, float alpha,
                              float* __restrict__ f_row, float* __restrict__ P_row, float* __restrict__ aux_out,
                              float* __restrict__ vio, float* __restrict__ bias, float gamma, double* sh) {
     const int tid = threadIdx.x;
@@ -150,8 +155,9 @@ __device__ void finish_batch(int64_t tot, double pall, int64_t m, int n, int k, 
             gprod = fg * pg;
         }
     }
+    double g = 0.0;
     if (has_probs) {
-        const double g = (double)alpha * (double)n * block_sum_d(gprod, sh);
+        g = (double)alpha * (double)n * block_sum_d(gprod, sh);
         if (tid == 0 && aux_out) *aux_out = (float)g;
     }
     const double F = valid ? (double)tot / ((double)m * (double)k) * (double)n - 1.0 : 0.0;
@@ -168,6 +174,7 @@ __device__ void finish_batch(int64_t tot, double pall, int64_t m, int n, int k, 
         else if (lhs < rhs) b = __fadd_rn(b, gamma);
         bias[tid] = b;
     }
+    return g;
 }
 
 __global__ void __launch_bounds__(stats::kThreads, 2)
@@ -294,13 +301,16 @@ stats_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, i
     double pall = 0.0;
     fold_blocks(w.segcnt, w.segps, nseg, n, has_probs, pc, part, &tot, &pall);
     if (totals && tid < n) { totals[tid] = (double)tot; totals[n + tid] = has_probs ? pall : 0.0; }
+    double micro = 0.0;
     if (has_probs && aux && tid == 0) {
-        double micro = 0.0;
         for (int64_t s = 0; s < nseg; ++s) micro += __ldcg(w.segaux + s);
-        aux[nseg] = (float)(micro / (double)nseg);
+        micro /= (double)nseg;
+        aux[nseg] = (float)micro;
     }
-    finish_batch(tot, pall, m, n, k, has_probs, alpha, f ? f + nseg * n : nullptr, P ? P + nseg * n : nullptr,
-                 aux ? aux + nseg + 1 : nullptr, vio, bias, gamma, sh);
+    const double g = finish_batch(tot, pall, m, n, k, has_probs, alpha, f ? f + nseg * n : nullptr,
+                                  P ? P + nseg * n : nullptr, aux ? aux + nseg + 1 : nullptr, vio, bias, gamma, sh);
+    // the hybrid loss: the global-batch loss plus the weighted micro-batch loss
+    if (has_probs && aux && tid == 0) aux[nseg + 2] = (float)(g + kHybridMicroWeight * micro);
 }
 
 // Global-batch results from totals [2, n] summed over data-parallel ranks (m_total tokens).

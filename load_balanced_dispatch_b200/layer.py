@@ -13,7 +13,7 @@ import torch
 
 from . import (MOE_QB_MIDPOINT, MOE_QB_STEP, MOE_SIGMOID, MOE_SOFTMAX, moe_balance_assign, moe_balance_stats,
                moe_capacity_slots, moe_combine, moe_dispatch_tokens, moe_expert_ffn, moe_expert_ffn_combine,
-               moe_expert_ffn_gather, moe_router_topk, lib)
+               moe_expert_ffn_gather, moe_router_prepare, moe_router_topk, lib)
 
 
 @dataclass
@@ -64,7 +64,7 @@ class MoELayer:
             y=torch.empty((m, d), dtype=s.dtype, device=dev),
             f=torch.empty((nseg + 1, n), dtype=f32, device=dev),
             P=torch.empty((nseg + 1, n), dtype=f32, device=dev),
-            aux=torch.empty((nseg + 2,), dtype=f32, device=dev),
+            aux=torch.empty((nseg + 3,), dtype=f32, device=dev),
             vio=torch.empty((3,), dtype=f32, device=dev),
         )
         L = lib()
@@ -78,6 +78,10 @@ class MoELayer:
             stats=torch.empty((max(L.moe_balance_stats_workspace_size(m, n, seg), 1),), dtype=torch.uint8,
                               device=dev),
         )
+        # the router weight is static: on the tensor-core path its bf16 split is made once, here
+        self.router_prepared = L.moe_router_topk_workspace_size(d, n, k, dt) > 0
+        if self.router_prepared:
+            moe_router_prepare(self.w["w_r"], k, s.dtype, workspace=self.ws["router"])
         # one pick per token in bf16: the combine runs in the FFN's second GEMM (moe_expert_ffn_combine).
         # gather = True would let the FFN read its rows from x (moe_expert_ffn_gather: no dispatch, no
         # xbuf); measured slower, it is off
@@ -93,7 +97,8 @@ class MoELayer:
         s, b, w = self.shape, self.buf, self.w
         if i == 0:
             fn = MOE_SOFTMAX if s.score_fn == "softmax" else MOE_SIGMOID
-            moe_router_topk(x, w["w_r"], s.n, s.k, fn, s.renorm_topk, rank_bias=w.get("rank_bias"),
+            moe_router_topk(x, None if self.router_prepared else w["w_r"], s.n, s.k, fn, s.renorm_topk,
+                            rank_bias=w.get("rank_bias"),
                             probs_out=b["probs"], topk_idx=b["topk_idx"], topk_gate=b["topk_gate"],
                             workspace=self.ws["router"], stream=st)
         elif i == 1:
@@ -214,14 +219,15 @@ class MoELayer:
                                   stream=stream)
 
     def launches_per_forward(self) -> int:
-        """Kernel launches of one forward: router (bf16 with n <= 128: weight split, tensor-core projection
-        and the finish kernel; else 1), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
+        """Kernel launches of one forward: router (1; 2 for bf16 with k > 8: projection and finish), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
         gathers its rows from x), FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
         combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus
         one launch for the dropped tokens' rows (which also clears the FFN's counters)."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
-        router = 3 if (bf16 and s.n <= 128) else 1  # scores are always requested here
+        router = 1  # tensor-core rows kernel (split prepared once; k <= 8) or the fp32 FMA kernel
+        if bf16 and s.n <= 128 and s.k > 8:
+            router = 2  # tensor-core logits tiles + the finish kernel
         capacity = 2
         dispatch = 1 if self.uses_dispatch() else 0
         if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped rows

@@ -75,6 +75,15 @@ def test_invalid_arguments_rejected_before_any_launch(L):
     # bf16 router without its workspace
     rc = L.moe_router_topk(fake, 1, fake, None, 16, 64, 8, 2, 0, 0, None, None, fake, fake, None, 0, None)
     assert rc == 3 and "workspace" in _err(L)
+    # w_r NULL (a prepared split) is only for the tensor-core path: not for fp32 activations
+    rc = L.moe_router_topk(fake, 0, None, None, 16, 64, 8, 2, 0, 0, None, None, fake, fake, None, 0, None)
+    assert rc == 1 and "moe_router_prepare" in _err(L)
+    # preparing the split on the fp32 FMA path: nothing to prepare
+    rc = L.moe_router_prepare(fake, 64, 8, 2, 0, fake, 1 << 20, None)
+    assert rc == 2 and "FMA" in _err(L)
+    # preparing without a workspace
+    rc = L.moe_router_prepare(fake, 64, 8, 2, 1, None, 0, None)
+    assert rc == 3 and "workspace" in _err(L)
     # workspace too small
     rc = L.moe_capacity_slots(fake, 64, 1, 8, 10, 64, fake, fake, fake, fake, fake, fake, fake, 0, None)
     assert rc == 3 and "workspace" in _err(L)

@@ -66,7 +66,7 @@ def test_rank_totals_sum_to_the_global_batch():
     P = t0[1] / m0
     assert (f == ref["f"][-1]).all()
     assert np.allclose(P, ref["P"][-1], rtol=1e-12, atol=0)
-    assert 1e-2 * N * (f * P).sum() == pytest.approx(ref["aux"][-1], rel=1e-12)
+    assert 1e-2 * N * (f * P).sum() == pytest.approx(ref["aux"][-2], rel=1e-12)  # the global-batch loss
     # the Loss-Free update from the pooled counts, decided on integers
     c = t0[0].astype(np.int64)
     step = np.where(c * N > M * K, -1, np.where(c * N < M * K, 1, 0))

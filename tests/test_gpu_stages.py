@@ -89,8 +89,8 @@ def test_router_projection(dtype, m, d, n, k, fn, renorm, bias):
                                                       (700, 512, 64, 6, 1, 0, True), (64, 64, 16, 12, 0, 0, False),
                                                       (400, 128, 100, 8, 1, 0, True)])
 def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
-    # no probs_out: the tensor-core path finishes the rows in the kernel (paired tiles for n > 64,
-    # whole rows for k > 8) and stores nothing but the picks and gates
+    # no probs_out: the tensor-core path finishes the rows in the kernel (in the drain threads for
+    # k <= 8, a warp per row for k > 8) and stores nothing but the picks and gates
     rng = np.random.default_rng(d * 3 + n)
     x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
     w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
@@ -104,6 +104,31 @@ def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
     assert ok.mean() > 0.97
     assert (host(idx)[ok] == i_ref[ok]).all()
     assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-5)
+
+
+@pytest.mark.parametrize("m,d,n,k,fn,renorm,bias", [(40000, 256, 64, 2, 0, 1, False), (20000, 512, 128, 1, 0, 0, False),
+                                                      (19100, 192, 96, 6, 1, 0, True), (30001, 128, 32, 4, 0, 0, False)])
+def test_router_persistent_blocks_and_prepared_split(m, d, n, k, fn, renorm, bias):
+    # more 128-token blocks than SMs, so each CTA of the persistent kernel takes several in turn
+    # (ragged last block); the call with w_r = None on a workspace from moe_router_prepare gives
+    # the same bits as the call that splits W_r itself
+    rng = np.random.default_rng(m + d)
+    x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
+    w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
+    b = rng.uniform(-0.05, 0.05, n).astype(np.float32) if bias else None
+    p_ref, i_ref, g_ref, margin = oracle.router(x, w, m, d, n, k, fn, renorm, b)
+    xd, wd, bd = dev(x, torch.bfloat16), dev(w), None if b is None else dev(b)
+    idx, gate, probs = lb.moe_router_topk(xd, wd, n, k, fn, renorm, rank_bias=bd)
+    ws = lb.moe_router_prepare(wd, k, torch.bfloat16)
+    idx2, gate2, probs2 = lb.moe_router_topk(xd, None, n, k, fn, renorm, rank_bias=bd, workspace=ws)
+    torch.cuda.synchronize()
+    lb.sync_status()
+    assert torch.equal(idx, idx2) and torch.equal(gate, gate2) and torch.equal(probs, probs2)
+    ok = margin > MARGIN
+    assert ok.mean() > 0.97
+    assert (host(idx)[ok] == i_ref[ok]).all()
+    assert np.allclose(host(gate)[ok], g_ref[ok], rtol=1e-5)
+    assert np.allclose(host(probs), p_ref, rtol=1e-5, atol=1e-9)
 
 
 # ---------------------------------------------------------------- capacity
@@ -279,7 +304,10 @@ def test_balance_stats_golden_identity(golden):
         out = lb.moe_balance_stats(dev(W.make_uniform_probs(m, n)), dev(W.make_round_robin_idx(m, n, 2)), n, m // 2,
                                    float(g["alpha"][0]))
         torch.cuda.synchronize()
-        assert (host(out["aux"]) == np.float32(g["expected_aux"][0])).all()
+        aux = host(out["aux"])
+        assert (aux[:-1] == np.float32(g["expected_aux"][0])).all()
+        # the hybrid loss: the global loss + 0.01 x the micro-batch loss = 1.01 alpha at balance
+        assert aux[-1] == pytest.approx(1.01 * float(g["alpha"][0]), rel=TOL_STATS)
         assert (host(out["vio"]) == 0).all()
 
 
@@ -308,9 +336,38 @@ def test_balance_global_across_ranks(m, n, k, ranks, with_probs):
     assert (host(out["f"]) == ref["f"][-1].astype(np.float32)).all()
     if with_probs:
         assert np.allclose(host(out["P"]), ref["P"][-1], rtol=TOL_STATS, atol=0)
-        assert np.allclose(host(out["aux"])[0], ref["aux"][-1], rtol=TOL_STATS, atol=0)
+        assert np.allclose(host(out["aux"])[0], ref["aux"][-2], rtol=TOL_STATS, atol=0)  # the global-batch loss
     assert np.allclose(host(out["vio"]), ref["vio"], rtol=1e-6, atol=1e-7)
     assert (host(bd) == ref["bias"]).all()
+
+
+# ---------------------------------------------------------------- mini-batch beta
+@pytest.mark.parametrize("m,n,k,seg,rule", [(65536, 256, 8, 4096, 0), (65536, 256, 8, 32768, 0),
+                                            (6144, 64, 6, 1024, 1), (4000, 16, 4, 500, 2), (2048, 32, 2, 2048, 0),
+                                            (1024, 8, 1, 8, 0), (12000, 24, 3, 24000 // 8, 0)])
+def test_balance_step_minibatch_bitexact(m, n, k, seg, rule):
+    # picks, beta and info bit-exact against the oracle: mini-batches kept in shared memory
+    # (seg <= 16384), the full radix path (32768), many tiny mini-batches (seg = 8), one (seg = m)
+    s = W.make_qb_scores(m, n, seed=m + n + seg, skew_std=1.0)
+    b0 = np.random.default_rng(seg).uniform(-0.5, 0.5, n).astype(np.float32)
+    i_ref, b_ref, f_ref = oracle.balance_step_minibatch(s, k, b0, seg, rule=rule)
+    beta = dev(b0)
+    idx, beta, info = lb.moe_balance_step_minibatch(dev(s), k, beta, seg, rule=rule)
+    torch.cuda.synchronize()
+    lb.sync_status()
+    assert (host(idx) == i_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(info) == f_ref).all()
+
+
+def test_balance_step_minibatch_ties():
+    # coarse scores: many equal keys inside each mini-batch's column
+    m, n, k, seg = 8192, 32, 4, 1024
+    s = (np.round(W.make_qb_scores(m, n, seed=3) * 4) / 4).astype(np.float32)
+    i_ref, b_ref, f_ref = oracle.balance_step_minibatch(s, k, np.zeros(n, np.float32), seg)
+    idx, beta, info = lb.moe_balance_step_minibatch(dev(s), k, torch.zeros(n, device="cuda"), seg)
+    torch.cuda.synchronize()
+    assert (host(idx) == i_ref).all() and (host(beta) == b_ref).all() and (host(info) == f_ref).all()
 
 
 # ---------------------------------------------------------------- balanced assignment
