@@ -17,10 +17,12 @@
 //              flag (k + 1 rounds of a warp arg-max when that does not apply);
 //              the set is written in ascending expert order and counted per
 //              expert. The first row pass of a SOLVE also writes s transposed
-//              (sT [n, m]) for the column pass's full path.
-//   qb_colwin  the column pass's window sweep, over row-major s by the whole
-//              GPU: per column, the keys of u above a window around the
-//              previous beta_j are counted and those inside are listed.
+//              (sT [n, m]) for the column pass's full path. Before a column
+//              pass the row pass also runs that pass's window sweep on the rows
+//              it holds: once it has alpha_i, per column the keys of
+//              u = s - alpha above a window around the current beta_j are
+//              counted and those inside are listed (one read of s per
+//              iteration instead of two).
 //   qb_col     one CTA per expert column: when the C-th largest fell inside
 //              the window, the C-th and (C+1)-th largest come from the column's
 //              list (radix digits over order-preserving uint32 keys); otherwise
@@ -50,7 +52,18 @@ constexpr int kColThreads = 512;  // qb_col_kernel block size (its scan buffer i
 enum { kStDone = 0, kStAugments = 1, kStError = 2, kStQbDone = 4, kStIters = 5, kStTies0 = 6, kStTies1 = 7,
        kStWords = 8 };
 constexpr int kBatch = 16;  // QB iterations enqueued between host checks
+constexpr int kRowPairCap = 512;  // window pairs buffered per row-pass CTA (flushed at tile boundaries)
 constexpr int64_t kMaxMiniBatches = 4096;  // mini-batches of one averaged-beta step
+}  // namespace qb
+
+namespace qb {
+constexpr int kCandCap = 16384;                         // candidate keys kept in shared memory
+constexpr int kColUnroll = 4;                           // float4 pairs in flight per thread in a column sweep
+constexpr int kGCap = 8192;                             // window candidates kept per column (global lists)
+constexpr size_t kColSmem = 4096 * 4 + kColThreads * 4 + kCandCap * 4;
+// key-space half-widths of the window around the previous beta_j
+// kWinSweep: the sweep's windows are at most this wide
+constexpr uint32_t kWinDefault = 1u << 18, kWinMin = 1u << 12, kWinMax = 1u << 26, kWinSweep = 1u << 21;
 }  // namespace qb
 
 // Threshold between the q-th (a) and (q+1)-th (b) largest: midpoint, the (q+1)-th, or the
@@ -69,6 +82,11 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 }
 __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+// float_key with -0 folded by an IEEE add of +0 (branch-free; the same key for every float)
+__device__ __forceinline__ uint32_t float_key_nz(float f) {
+    const uint32_t b = __float_as_uint(__fadd_rn(f, 0.0f));
+    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
 }
 
 // Top-(k+1) of one row held by a warp: lane owns j = lane + 32 q (q < NT); key = float_key(v),
@@ -167,11 +185,53 @@ __device__ __forceinline__ bool row_topk_ranked(const uint32_t (&key)[NT], const
 // Each row takes the ranked selection, or the plain rounds when it does not apply. beta for the
 // lane's columns stays in registers. TRANS: the tile is also written out transposed (sT [n, m],
 // each expert's column contiguous) for the column pass's full path.
-template <int NT, bool TRANS>
+// The window sweep of the column pass, done by the row pass on the rows it holds (SWEEP): once a
+// warp has alpha_i, the keys of u_ij = fp32(s_ij - alpha_i) of its row are compared with a window
+// [lo_j, hi_j] around the current beta_j (half-width min(win_j, kWinSweep), the previous select's
+// width): keys above the window are counted (per lane, per column) and keys inside it are
+// buffered in shared memory as (column, key) pairs, which the CTA appends to the column's global
+// candidate list (g_cand[j], kGCap long, count g_ncand[j]) at tile boundaries once the buffer is
+// half full, and at the end. A column whose pairs do not fit is marked full (its count pushed
+// past kGCap), so the select takes the exact full path. This removes the second read of s.
+struct RowSweep {
+    const uint32_t* win;   // [n] window half-widths (0: default)
+    uint32_t* g_above;     // [n] keys above the window
+    uint32_t* g_ncand;     // [n] keys inside it
+    uint32_t* g_cand;      // [n][kGCap] the keys inside it
+};
+
+// Append the CTA's buffered (column, key) pairs to the global candidate lists (all threads).
+__device__ __forceinline__ void sweep_flush(const uint2* pairs, unsigned* npairs, uint32_t* scnt, uint32_t* sbase,
+                                            unsigned char* sfull, int n, const RowSweep& sw) {
+    const int tid = threadIdx.x, T = blockDim.x;
+    const unsigned np = min(*npairs, (unsigned)qb::kRowPairCap);
+    for (unsigned p = tid; p < np; p += T) atomicAdd(&scnt[pairs[p].x], 1u);
+    __syncthreads();
+    for (int j = tid; j < n; j += T) {
+        // a full column: its count goes past kGCap, its pairs are not stored
+        const uint32_t add = sfull[j] ? scnt[j] + (uint32_t)qb::kGCap + 1u : scnt[j];
+        sbase[j] = add ? atomicAdd(&sw.g_ncand[j], add) : 0u;
+        if (sfull[j]) sbase[j] = (uint32_t)qb::kGCap;
+        scnt[j] = 0;
+    }
+    __syncthreads();
+    for (unsigned p = tid; p < np; p += T) {
+        const uint2 pr = pairs[p];
+        const uint32_t pos = sbase[pr.x] + atomicAdd(&scnt[pr.x], 1u);
+        if (pos < (uint32_t)qb::kGCap) sw.g_cand[(int64_t)pr.x * qb::kGCap + pos] = pr.y;
+    }
+    __syncthreads();
+    for (int j = tid; j < n; j += T) { scnt[j] = 0; sfull[j] = 0; }
+    if (tid == 0) *npairs = 0;
+    __syncthreads();
+}
+
+template <int NT, bool TRANS, bool SWEEP>
 __global__ void __launch_bounds__(qb::kRowThreads, 3)
 qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
               float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
-              int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT, int bulk) {
+              int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT, int bulk,
+              RowSweep sw) {
     if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
     constexpr int RT = qb::kRowTile;
     extern __shared__ __align__(128) float rtile[];  // [2][RT * n]
@@ -182,14 +242,22 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
     __shared__ uint32_t s_key[qb::kRowThreads];
     __shared__ int s_j[qb::kRowThreads];
     __shared__ float s_v[qb::kRowThreads];
+    // window sweep: buffered pairs and per-column scratch of the flush
+    __shared__ uint2 pairs[SWEEP ? qb::kRowPairCap : 1];
+    __shared__ uint32_t scnt[SWEEP ? kMaxExperts : 1], sbase[SWEEP ? kMaxExperts : 1];
+    __shared__ unsigned char sfull[SWEEP ? kMaxExperts : 1];
+    __shared__ unsigned npairs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wbase = tid & ~31;  // this warp's 32 shared slots
     const int64_t ntiles = (m + RT - 1) / RT;
     const int64_t tile_floats = (int64_t)RT * n;
     const uint32_t tile_bytes = (uint32_t)(tile_floats * sizeof(float));
     for (int j = tid; j < n; j += blockDim.x) cnt[j] = 0;
+    if (SWEEP)
+        for (int j = tid; j < n; j += blockDim.x) { scnt[j] = 0; sfull[j] = 0; }
     if (tid == 0) {
         nties = 0;
+        npairs = 0;
         abort_flag = 0;
         ptx::mbar_init(&bar[0], 1);
         ptx::mbar_init(&bar[1], 1);
@@ -199,6 +267,21 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
     float bq[NT];
 #pragma unroll
     for (int q = 0; q < NT; ++q) bq[q] = lane + 32 * q < n ? beta[lane + 32 * q] : 0.f;
+    // the lane's windows (padding columns get lo = hi = the largest key, which no float reaches)
+    uint32_t lo[NT], hi[NT], above[NT];
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+        above[q] = 0;
+        lo[q] = hi[q] = 0xffffffffu;
+        const int j = lane + 32 * q;
+        if (SWEEP && j < n) {
+            const uint32_t pk = float_key(bq[q]);
+            uint32_t w = sw.win[j] ? sw.win[j] : qb::kWinDefault;
+            if (w > qb::kWinSweep) w = qb::kWinSweep;
+            lo[q] = pk > w ? pk - w : 0u;
+            hi[q] = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
+        }
+    }
     const uint32_t lt = (1u << lane) - 1u;
     const bool prune = k < 32 && k < n;
     // copies issued and consumed per buffer (thread 0's bookkeeping, for a clean exit on abort)
@@ -275,8 +358,35 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
                 alpha[i] = qb_threshold(vk, vk1, rule);
                 if (vk == vk1) atomicAdd(&nties, 1);
             }
+            if (SWEEP) {
+                // vk, vk1 are the same in every lane: so is alpha_i
+                const float a = qb_threshold(vk, vk1, rule);
+                uint32_t inw = 0;
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    if (lane + 32 * q < n) {
+                        const uint32_t key = float_key_nz(__fsub_rn(row[lane + 32 * q], a));
+                        above[q] += key > hi[q] ? 1u : 0u;
+                        inw |= (key >= lo[q] && key <= hi[q]) ? (1u << q) : 0u;
+                    }
+                }
+                if (__any_sync(0xffffffffu, inw != 0)) {
+#pragma unroll
+                    for (int q = 0; q < NT; ++q) {
+                        if ((inw >> q) & 1u) {
+                            const int j = lane + 32 * q;
+                            const unsigned p = atomicAdd(&npairs, 1u);
+                            if (p < (unsigned)qb::kRowPairCap)
+                                pairs[p] = make_uint2((uint32_t)j, float_key_nz(__fsub_rn(row[j], a)));
+                            else
+                                sfull[j] = 1;
+                        }
+                    }
+                }
+            }
         }
         __syncthreads();  // every warp is done with the buffer
+        if (SWEEP && npairs >= (unsigned)qb::kRowPairCap / 2) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw);
         if (tid == 0) {
             const int64_t tn = t + 2 * (int64_t)gridDim.x;
             if (bulk && tn < ntiles && (tn + 1) * RT <= m) {
@@ -301,6 +411,19 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
     for (int j = tid; j < n; j += blockDim.x)
         if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
     if (tid == 0 && nties) atomicAdd(&status[tie_slot], nties);
+    if (SWEEP) {
+        // keys above the windows: lanes -> shared (scnt is free between flushes) -> global
+#pragma unroll
+        for (int q = 0; q < NT; ++q)
+            if (lane + 32 * q < n && above[q]) atomicAdd(&scnt[lane + 32 * q], above[q]);
+        __syncthreads();
+        for (int j = tid; j < n; j += blockDim.x) {
+            if (scnt[j]) atomicAdd(&sw.g_above[j], scnt[j]);
+            scnt[j] = 0;
+        }
+        __syncthreads();
+        if (npairs) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw);
+    }
 }
 
 // Block-wide bin selection: scanning bins from the top, the bin where the cumulative count
@@ -371,18 +494,6 @@ __device__ __forceinline__ unsigned block_sum_u32(unsigned v, unsigned* red) {
     return r;
 }
 
-namespace qb {
-constexpr int kCandCap = 16384;                         // candidate keys kept in shared memory
-constexpr int kColUnroll = 4;                           // float4 pairs in flight per thread in a column sweep
-constexpr int kGCap = 8192;                             // window candidates kept per column (global lists)
-constexpr int kWinThreads = 256;                        // qb_colwin_kernel block size
-constexpr int kPairCap = 4096;                          // (column, key) pairs buffered per window-sweep CTA
-constexpr int kWinRows = 4;                             // rows in flight per warp in the window sweep
-constexpr size_t kColSmem = 4096 * 4 + kColThreads * 4 + kCandCap * 4;
-// key-space half-widths of the window around the previous beta_j
-// kWinSweep: the sweep's windows are at most this wide
-constexpr uint32_t kWinDefault = 1u << 18, kWinMin = 1u << 12, kWinMax = 1u << 26, kWinSweep = 1u << 21;
-}  // namespace qb
 
 // Visit every key float_key(fp32(col[i * stride] - alpha[i])) of a column, warp-uniformly (f gets
 // ok = false for padding lanes). A contiguous column (stride 1, m a multiple of 4: every column
@@ -500,151 +611,6 @@ __device__ __forceinline__ uint32_t list_max_below(const unsigned* list, unsigne
     return block_max_u32(best, scan);
 }
 
-// Column pass, part 1: the window sweep over row-major s. For every column j the keys of
-// u_ij = fp32(s_ij - alpha_i) are compared with a window [lo_j, hi_j] around the previous beta_j
-// (half-width min(win_j, kWinSweep)): keys above it are counted and keys inside it are appended
-// to column j's candidate list (g_cand[j], kGCap long; the count g_ncand[j] goes on past it).
-// Warp per row, kWinRows rows in flight per warp; lane owns the columns win_col(lane, q) (VEC:
-// 16-byte loads, four adjacent columns per load). The per-key work is branch-free; a row with a
-// key inside some window takes the append path. A CTA buffers its (column, key) pairs in shared
-// memory and reserves room in the global lists once per column at the end; a column whose pairs
-// did not fit is marked full (its count pushed past kGCap), so it takes the exact full path.
-// All SMs sweep together, so the pass runs at the rate of one read of s.
-// check: stop at once when the row pass just made left every count at C (sets kStQbDone).
-template <bool VEC>
-__device__ __forceinline__ int win_col(int lane, int q) {
-    return VEC ? 128 * (q >> 2) + 4 * lane + (q & 3) : lane + 32 * q;
-}
-
-// float_key with -0 folded by an IEEE add of +0 (branch-free; the same key for every float)
-__device__ __forceinline__ uint32_t float_key_nz(float f) {
-    const uint32_t b = __float_as_uint(__fadd_rn(f, 0.0f));
-    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
-}
-
-template <int NT, bool VEC>
-__global__ void __launch_bounds__(qb::kWinThreads, 2)
-qb_colwin_kernel(const float* __restrict__ s, int64_t m, int n, int64_t C, const float* __restrict__ alpha,
-                 const float* __restrict__ beta, const uint32_t* __restrict__ win, const int32_t* __restrict__ counts,
-                 int32_t* __restrict__ status, int check, uint32_t* __restrict__ g_above,
-                 uint32_t* __restrict__ g_ncand, uint32_t* __restrict__ g_cand) {
-    static_assert(!VEC || NT % 4 == 0, "vector columns come in fours");
-    constexpr int R = qb::kWinRows;
-    __shared__ uint32_t sabove[kMaxExperts], scnt[kMaxExperts], sbase[kMaxExperts];
-    __shared__ unsigned char sfull[kMaxExperts];
-    __shared__ uint2 pairs[qb::kPairCap];
-    __shared__ unsigned npairs;
-    __shared__ int balanced;
-    const int tid = threadIdx.x, lane = tid & 31;
-    if (check) {
-        if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
-        if (tid == 0) balanced = 1;
-        __syncthreads();
-        for (int e = tid; e < n; e += blockDim.x)
-            if (counts[e] != C) balanced = 0;
-        __syncthreads();
-        if (balanced) {
-            if (blockIdx.x == 0 && tid == 0) status[qb::kStQbDone] = 1;
-            return;
-        }
-    }
-    for (int j = tid; j < n; j += blockDim.x) { sabove[j] = 0; scnt[j] = 0; sfull[j] = 0; }
-    if (tid == 0) npairs = 0;
-    // padding columns get the empty window lo = hi = the largest key, which no float reaches
-    uint32_t lo[NT], hi[NT], above[NT];
-#pragma unroll
-    for (int q = 0; q < NT; ++q) {
-        const int j = win_col<VEC>(lane, q);
-        above[q] = 0;
-        lo[q] = 0xffffffffu;
-        hi[q] = 0xffffffffu;
-        if (j < n) {
-            const uint32_t pk = float_key(beta[j]);
-            uint32_t w = win[j] ? win[j] : qb::kWinDefault;
-            if (w > qb::kWinSweep) w = qb::kWinSweep;
-            lo[q] = pk > w ? pk - w : 0u;
-            hi[q] = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
-        }
-    }
-    __syncthreads();
-    constexpr int WPB = qb::kWinThreads / 32;
-    const int64_t nw = (int64_t)gridDim.x * WPB;
-    for (int64_t i0 = (int64_t)blockIdx.x * WPB + (tid >> 5); i0 < m; i0 += R * nw) {
-        float a[R], v[R][NT];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t i = i0 + r * nw;
-            const bool ok = i < m;
-            a[r] = ok ? alpha[i] : 0.f;
-            if (VEC) {
-#pragma unroll
-                for (int h = 0; h < NT / 4; ++h) {
-                    const int c = 128 * h + 4 * lane;
-                    const float4 t = (ok && c < n) ? *reinterpret_cast<const float4*>(s + i * n + c)
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[r][4 * h] = t.x;
-                    v[r][4 * h + 1] = t.y;
-                    v[r][4 * h + 2] = t.z;
-                    v[r][4 * h + 3] = t.w;
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < NT; ++q) {
-                    const int j = lane + 32 * q;
-                    v[r][q] = (ok && j < n) ? s[i * n + j] : 0.f;
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const bool ok = i0 + r * nw < m;  // warp-uniform
-            uint32_t inw = 0;
-#pragma unroll
-            for (int q = 0; q < NT; ++q) {
-                const uint32_t key = float_key_nz(__fsub_rn(v[r][q], a[r]));
-                above[q] += (ok && key > hi[q]) ? 1u : 0u;
-                inw |= (ok && key >= lo[q] && key <= hi[q]) ? (1u << q) : 0u;
-            }
-            if (__any_sync(0xffffffffu, inw != 0)) {
-#pragma unroll
-                for (int q = 0; q < NT; ++q) {
-                    if ((inw >> q) & 1u) {
-                        const int j = win_col<VEC>(lane, q);
-                        const unsigned p = atomicAdd(&npairs, 1u);
-                        if (p < (unsigned)qb::kPairCap)
-                            pairs[p] = make_uint2((uint32_t)j, float_key_nz(__fsub_rn(v[r][q], a[r])));
-                        else
-                            sfull[j] = 1;
-                    }
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < NT; ++q) {
-        const int j = win_col<VEC>(lane, q);
-        if (j < n && above[q]) atomicAdd(&sabove[j], above[q]);
-    }
-    __syncthreads();
-    const unsigned np = min(npairs, (unsigned)qb::kPairCap);
-    for (unsigned p = tid; p < np; p += blockDim.x) atomicAdd(&scnt[pairs[p].x], 1u);
-    __syncthreads();
-    for (int j = tid; j < n; j += blockDim.x) {
-        if (sabove[j]) atomicAdd(&g_above[j], sabove[j]);
-        // a full column: its count goes past kGCap, its pairs are not stored
-        const uint32_t add = sfull[j] ? scnt[j] + (uint32_t)qb::kGCap + 1u : scnt[j];
-        sbase[j] = add ? atomicAdd(&g_ncand[j], add) : 0u;
-        if (sfull[j]) sbase[j] = (uint32_t)qb::kGCap;
-        scnt[j] = 0;
-    }
-    __syncthreads();
-    for (unsigned p = tid; p < np; p += blockDim.x) {
-        const uint2 pr = pairs[p];
-        const uint32_t pos = sbase[pr.x] + atomicAdd(&scnt[pr.x], 1u);
-        if (pos < (uint32_t)qb::kGCap) g_cand[(int64_t)pr.x * qb::kGCap + pos] = pr.y;
-    }
-}
-
 // The want-th and (want+1)-th largest keys (1-based, want + 1 <= ncand) of a short shared list,
 // by ranks: a key holds rank r when fewer than r keys are above it and at least r are at or
 // above it. One candidate per thread (ncand <= blockDim.x), four list keys per shared load.
@@ -748,8 +714,8 @@ __device__ void column_select_full(const float* __restrict__ col, int64_t stride
     *bkey_out = bkey;
 }
 
-// Column pass, part 2: beta_j = threshold between the C-th and (C+1)-th largest key of column j
-// of u = fp32(s - alpha). When both fell inside the window of part 1 (the usual case once the
+// Column pass: beta_j = threshold between the C-th and (C+1)-th largest key of column j
+// of u = fp32(s - alpha). When both fell inside the window of the row pass's sweep (the usual case once the
 // iteration settles) they come from the column's candidate list, copied into shared memory:
 // by ranks when the list is short, else by radix digits. Otherwise the full radix path over the
 // column: a 12-bit digit histogram sweep, a sweep keeping the selected bin's keys (the largest
@@ -778,6 +744,13 @@ qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t
     }
     if (check) {
         if (*(volatile int32_t*)&status[qb::kStQbDone]) return;
+        // stop once the row pass just made left every count at C
+        int unbalanced = 0;
+        for (int e = threadIdx.x; e < n; e += blockDim.x) unbalanced |= info_counts[e] != C;
+        if (!__syncthreads_or(unbalanced)) {
+            if (blockIdx.x == 0 && threadIdx.x == 0) status[qb::kStQbDone] = 1;
+            return;
+        }
         if (blockIdx.x == 0) {
             for (int e = threadIdx.x; e < n; e += blockDim.x) counts_next[e] = 0;
             if (threadIdx.x == 0) {
@@ -1459,14 +1432,14 @@ static size_t qb_layout(int64_t m, int n, int k, QBWorkspace* w, char* base) {
 
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k) { return qb_layout(m, n, k, nullptr, nullptr); }
 
-template <int NT, bool TRANS>
+template <int NT, bool TRANS, bool SWEEP>
 static void launch_row_tt(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                           int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
-                          cudaStream_t stream) {
+                          const RowSweep& sw, cudaStream_t stream) {
     const size_t smem = 2 * (size_t)qb::kRowTile * n * sizeof(float);
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(qb_row_kernel<NT, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(qb_row_kernel<NT, TRANS, SWEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(2 * (size_t)qb::kRowTile * kMaxExperts * sizeof(float)));
         attr = true;
     }
@@ -1478,54 +1451,41 @@ static void launch_row_tt(const float* s, int64_t m, int n, int k, const float* 
     if (blocks < 1) blocks = 1;
     // bulk copies need a 16-byte aligned s (every tile then starts on a 16-byte boundary)
     const int bulk = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
-    qb_row_kernel<NT, TRANS><<<(unsigned)blocks, qb::kRowThreads, smem, stream>>>(
-        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk);
+    qb_row_kernel<NT, TRANS, SWEEP><<<(unsigned)blocks, qb::kRowThreads, smem, stream>>>(
+        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk, sw);
 }
 
 template <int NT>
 static void launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                          int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
-                         cudaStream_t stream) {
-    if (sT) launch_row_tt<NT, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
-    else launch_row_tt<NT, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+                         const RowSweep* sw, cudaStream_t stream) {
+    const RowSweep none{nullptr, nullptr, nullptr, nullptr};
+    if (sw) {
+        if (sT) launch_row_tt<NT, true, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
+        else launch_row_tt<NT, false, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
+    } else {
+        if (sT) launch_row_tt<NT, true, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
+        else launch_row_tt<NT, false, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
+    }
 }
 
 // sT != nullptr: this row pass also writes s transposed into sT (the first pass of a call).
+// sw != nullptr: it also runs the column pass's window sweep on its rows.
 static void launch_row(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                        int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
-                       cudaStream_t stream) {
-    if (n <= 32) launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
-    else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
-    else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
-    else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, stream);
+                       const RowSweep* sw, cudaStream_t stream) {
+    if (n <= 32) launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
+    else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
+    else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
+    else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
 }
 
-template <int NT, bool VEC>
-static void launch_colwin_t(const float* s, int64_t m, int n, int64_t C, const QBWorkspace& w, const float* beta,
-                            const int32_t* counts, int check, cudaStream_t stream) {
-    constexpr int WPB = qb::kWinThreads / 32;
-    int64_t blocks = (m + qb::kWinRows * WPB - 1) / (qb::kWinRows * WPB);
-    if (blocks > (int64_t)kNumSMs * 2) blocks = (int64_t)kNumSMs * 2;
-    if (blocks < 1) blocks = 1;
-    qb_colwin_kernel<NT, VEC><<<(unsigned)blocks, qb::kWinThreads, 0, stream>>>(
-        s, m, n, C, w.alpha, beta, w.win, counts, w.status, check, w.g_above, w.g_ncand, w.g_cand);
-}
-
-// The column pass: the window sweep over s, then one select CTA per column. sT: s transposed
-// (SOLVE), read by the select kernel's full path when the window missed; nullptr: that path
-// reads the column from s with stride n.
+// The column pass's select: one CTA per column (the window sweep ran inside the row pass). sT: s
+// transposed (SOLVE), read by the select kernel's full path when the window missed; nullptr:
+// that path reads the column from s with stride n.
 static void launch_col(const float* s, const float* sT, int64_t m, int n, int64_t C, const QBWorkspace& w, int rule,
                        float* beta, const int32_t* counts, int32_t* counts_next, int iter, int check,
                        cudaStream_t stream, int32_t* info = nullptr) {
-    // 16-byte rows when every row of s starts on a 16-byte boundary
-    const bool vec = n % 4 == 0 && (reinterpret_cast<uintptr_t>(s) & 15) == 0;
-    if (vec) {
-        if (n <= 128) launch_colwin_t<4, true>(s, m, n, C, w, beta, counts, check, stream);
-        else launch_colwin_t<8, true>(s, m, n, C, w, beta, counts, check, stream);
-    } else if (n <= 32) launch_colwin_t<1, false>(s, m, n, C, w, beta, counts, check, stream);
-    else if (n <= 64) launch_colwin_t<2, false>(s, m, n, C, w, beta, counts, check, stream);
-    else if (n <= 128) launch_colwin_t<4, false>(s, m, n, C, w, beta, counts, check, stream);
-    else launch_colwin_t<8, false>(s, m, n, C, w, beta, counts, check, stream);
     qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(s, sT, m, n, C, w.alpha, rule, beta, counts_next,
                                                                 w.status, iter, check, w.win, w.g_above, w.g_ncand,
                                                                 w.g_cand, counts, qb::kStTies0, info);
@@ -1609,7 +1569,8 @@ int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, 
     cudaError_t ce;
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 2 * n), stream)) != cudaSuccess)
         goto fail;
-    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
+    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, nullptr,
+               stream);
     {
         int64_t blocks = (m + 7) / 8;
         if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
@@ -1648,7 +1609,7 @@ int run_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* b
     }
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 2 * n), stream)) != cudaSuccess)
         goto fail;
-    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, w.sT, stream);
+    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, w.sT, nullptr, stream);
     qb_col_slice_kernel<<<dim3((unsigned)n, (unsigned)nb), qb::kColThreads, qb::kColSmem, stream>>>(
         w.sT, m, n, seg_len, Cb, w.alpha, rule, w.beta_parts);
     qb_beta_mean_kernel<<<1, 256, 0, stream>>>(w.beta_parts, nb, n, beta);
@@ -1667,6 +1628,7 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
     QBWorkspace w;
     qb_layout(m, n, k, &w, static_cast<char*>(workspace));
     const int64_t C = m * k / n;
+    const RowSweep sweep{w.win, w.g_above, w.g_ncand, w.g_cand};
     cudaError_t ce;
     static bool col_attr = false;
     if (!col_attr) {
@@ -1680,7 +1642,8 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
         goto cuda_fail;
     if (mode == MOE_QB_STEP) {
         // one pass each; a window miss reads its column from s (no transposed copy)
-        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, stream);
+        launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, &sweep,
+                   stream);
         launch_col(s, nullptr, m, n, C, w, rule, beta, w.counts, w.counts + n, 0, 0, stream, info);
         if ((ce = cudaGetLastError()) != cudaSuccess) goto cuda_fail;
         return MOE_OK;
@@ -1692,8 +1655,10 @@ int run_balance_assign(const float* s, int64_t m, int n, int k, float* beta, int
             const int u1 = u0 + qb::kBatch - 1 < max_iters ? u0 + qb::kBatch - 1 : max_iters;
             for (int u = u0; u <= u1; ++u) {
                 int32_t* cnt = w.counts + (u % 2) * n;
+                // the sweep feeds the column pass that follows (none after the last row pass)
                 launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, cnt, w.status,
-                           u % 2 ? qb::kStTies1 : qb::kStTies0, 1, u == 0 ? w.sT : nullptr, stream);
+                           u % 2 ? qb::kStTies1 : qb::kStTies0, 1, u == 0 ? w.sT : nullptr,
+                           u < max_iters ? &sweep : nullptr, stream);
                 if (u < max_iters)
                     launch_col(s, w.sT, m, n, C, w, rule, beta, cnt, w.counts + ((u + 1) % 2) * n, u, 1, stream);
             }

@@ -528,11 +528,17 @@ static int* ffn_counters(void* hbuf, int64_t max_rows, int d_ff) {
     return reinterpret_cast<int*>(static_cast<char*>(hbuf) + hbytes);
 }
 
+cudaError_t launch_ffn_pair(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
+                            const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
+                            int* counters, cudaStream_t stream);
+
+// moe_expert_ffn in bf16: the two-SM tiles of ffn_pair.cu (the one-SM kernel here serves the
+// fused-combine and row-gather variants).
 cudaError_t launch_ffn_tc(const void* xbuf, const void* w1, const void* b1, const void* w2, const void* b2,
                           const int32_t* offsets, int n, int d, int d_ff, int64_t max_rows, void* ybuf, void* hbuf,
                           cudaStream_t stream) {
-    return launch_ffn_fused(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf,
-                            ffn_counters(hbuf, max_rows, d_ff), stream);
+    return launch_ffn_pair(xbuf, w1, b1, w2, b2, offsets, n, d, d_ff, max_rows, ybuf, hbuf,
+                           ffn_counters(hbuf, max_rows, d_ff), stream);
 }
 
 // The FFN reading its rows straight from x by src_token (the dispatch fused into the first GEMM).
