@@ -355,6 +355,54 @@ MOE_API moe_status moe_combine(const void* ybuf, moe_dtype dt, const int32_t* de
                        const void* residual, int64_t m, int32_t k, int32_t d, void* y, moe_stream_t stream);
 
 /*
+ * Expert parallelism over G ranks (one GPU each), three calls around the owner's FFN.
+ * Passage: "Switch Transformer read for implementation" (molayo1419.me), Expert
+ * Parallelism (experts on different devices: the dispatch and the return of the
+ * outputs become exchanges between devices, kept apart from the compute); "Switch
+ * Transformers paper review" (tildalice.io/?p=118), distributed training and
+ * communication cost (an all-to-all before the experts and one after them).
+ *
+ * Rank q owns experts q E .. q E + E - 1, E = n / G (n % G == 0). Each rank routes its
+ * own m tokens over all n experts and runs moe_capacity_slots on them (capacity is per
+ * source rank). The caller gathers every rank's expert_offsets [n + 1] into
+ * offsets_all [G, n + 1] (rank-major; one all-gather of n + 1 int32 per rank). Owner
+ * q's receive buffer then holds its local experts in order, each expert's rows from
+ * source rank 0 first, then rank 1, ..., each source's rows in its own expert-major
+ * order: the rows the one-GPU layer gives the expert on the concatenated batch with
+ * one capacity segment per rank.
+ *
+ * moe_ep_plan: from offsets_all (device), this rank's send_base [n] (the row of expert
+ *   e's owner's buffer where this rank's rows of e start) and recv_offsets [E + 1] (the
+ *   row offsets of this rank's local experts in its own receive buffer; recv_offsets[E]
+ *   = its rows). recv_offsets and this rank's E experts' weights are what moe_expert_ffn
+ *   takes (n = E) to run the owner's FFN on its receive buffer.
+ * moe_ep_dispatch: x [m, d] -> the owners' receive buffers. peer_xrecv is a DEVICE array
+ *   of G device pointers, entry q = rank q's receive buffer [max_recv_rows, d] mapped into
+ *   this GPU's address space (peer access: CUDA IPC or symmetric memory; entry `rank` is
+ *   this rank's own buffer). Each token is read once and stored to each kept pick's row
+ *   of its owner's buffer (plain 16-byte stores, no TMA). ep_row [m, k] out: the pick's
+ *   row in its owner's buffer, or -1 (dropped). topk_idx, dest_row, expert_offsets: this
+ *   rank's router and capacity outputs; send_base from moe_ep_plan.
+ * moe_ep_combine: y[i] = (residual[i]) + sum over kept picks r of g_ir * yrecv_q[ep_row[i, r]]
+ *   with q = topk_idx[i, r] / E, read through peer_yrecv (a DEVICE array of G pointers to
+ *   the ranks' expert outputs [max_recv_rows, d]); fp32 accumulation in pick order and,
+ *   for bf16, gates rounded to bf16 first: the operations of moe_combine, so the result is
+ *   bit for bit the one-GPU layer's.
+ * Ordering across ranks is the caller's: every rank's dispatch completes before any owner
+ * runs its FFN, and every FFN before any combine reads it (the kernels wait on nothing).
+ * Errors: MOE_ERR_INVALID_ARG; a row outside [0, max_recv_rows) sets the device error word.
+ */
+MOE_API moe_status moe_ep_plan(const int32_t* offsets_all, int32_t G, int32_t n, int32_t rank, int32_t* send_base,
+                               int32_t* recv_offsets, moe_stream_t stream);
+MOE_API moe_status moe_ep_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, int32_t k, int32_t n, int32_t G,
+                                   const int32_t* topk_idx, const int32_t* dest_row, const int32_t* expert_offsets,
+                                   const int32_t* send_base, void* const* peer_xrecv, int64_t max_recv_rows,
+                                   int32_t* ep_row, moe_stream_t stream);
+MOE_API moe_status moe_ep_combine(const void* const* peer_yrecv, moe_dtype dt, const int32_t* ep_row,
+                                  const int32_t* topk_idx, int32_t n, int32_t G, const float* topk_gate,
+                                  const void* residual, int64_t m, int32_t k, int32_t d, void* y, moe_stream_t stream);
+
+/*
  * Load statistics, auxiliary loss and the Loss-Free bias update.
  * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), auxiliary
  * load balancing loss L = alpha N sum_i f_i P_i; "Qwen global-batch load

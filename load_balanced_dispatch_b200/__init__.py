@@ -31,7 +31,7 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
            "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step",
            "moe_expert_ffn_gather", "moe_dispatch_tokens", "moe_router_prepare",
-           "moe_balance_step_minibatch")
+           "moe_balance_step_minibatch", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine")
 
 
 class MoEError(RuntimeError):
@@ -67,6 +67,9 @@ def lib() -> C.CDLL:
         L.moe_capacity_slots_static.argtypes = [P, I64, I32, I32, I32, I64, P, P, P, P, P, P, P]
         L.moe_dispatch.argtypes = [P, I32, I64, I32, P, P, I32, I64, P, P]
         L.moe_dispatch_tokens.argtypes = [P, I32, I64, I32, I32, P, I64, P, P]
+        L.moe_ep_plan.argtypes = [P, I32, I32, I32, P, P, P]
+        L.moe_ep_dispatch.argtypes = [P, I32, I64, I32, I32, I32, I32, P, P, P, P, P, I64, P, P]
+        L.moe_ep_combine.argtypes = [P, I32, P, P, I32, I32, P, P, I64, I32, I32, P, P]
         L.moe_expert_ffn_workspace_size.argtypes = [I32, I64, I32]
         L.moe_expert_ffn_workspace_size.restype = SZ
         L.moe_expert_ffn.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, I64, P, P, SZ, P]
@@ -244,6 +247,50 @@ def moe_dispatch_tokens(x, dest_row, max_rows=None, xbuf=None, stream=None):
     _check("moe_dispatch_tokens", lib().moe_dispatch_tokens(_ptr(x), _dtype_code(x), m, d, k, _ptr(dest_row),
                                                             max_rows, _ptr(xbuf), _stream(stream)))
     return xbuf
+
+
+def moe_ep_plan(offsets_all, rank, send_base=None, recv_offsets=None, stream=None):
+    """Expert parallelism, the exchange plan of one rank from every rank's expert_offsets
+    offsets_all [G, n+1]: (send_base [n], recv_offsets [n/G + 1])."""
+    G, n1 = offsets_all.shape
+    n = n1 - 1
+    dev = offsets_all.device
+    _need(offsets_all, torch.int32, (G, n + 1), "offsets_all")
+    if send_base is None:
+        send_base = torch.empty((n,), dtype=torch.int32, device=dev)
+    if recv_offsets is None:
+        recv_offsets = torch.empty((n // G + 1,), dtype=torch.int32, device=dev)
+    _check("moe_ep_plan", lib().moe_ep_plan(_ptr(offsets_all), G, n, rank, _ptr(send_base), _ptr(recv_offsets),
+                                            _stream(stream)))
+    return send_base, recv_offsets
+
+
+def moe_ep_dispatch(x, topk_idx, dest_row, expert_offsets, send_base, peer_xrecv, G, max_recv_rows, ep_row=None,
+                    stream=None):
+    """Store each kept row of this rank's tokens into its expert owner's receive buffer. peer_xrecv:
+    a device int64 tensor [G] of buffer addresses (this GPU's view). Returns ep_row [m, k]."""
+    m, d = x.shape
+    k = topk_idx.shape[1]
+    n = expert_offsets.numel() - 1
+    if ep_row is None:
+        ep_row = torch.empty((m, k), dtype=torch.int32, device=x.device)
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(
+        _ptr(x), _dtype_code(x), m, d, k, n, G, _ptr(topk_idx), _ptr(dest_row), _ptr(expert_offsets),
+        _ptr(send_base), _ptr(peer_xrecv), max_recv_rows, _ptr(ep_row), _stream(stream)))
+    return ep_row
+
+
+def moe_ep_combine(peer_yrecv, dtype, ep_row, topk_idx, n, G, topk_gate, residual=None, y=None, d=None, stream=None):
+    """y = (residual) + gated sum of the owners' output rows (peer loads). peer_yrecv: device int64 [G]."""
+    m, k = ep_row.shape
+    if y is None:
+        y = torch.empty((m, d), dtype=dtype, device=ep_row.device)
+    d = y.shape[1]
+    code = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    _check("moe_ep_combine", lib().moe_ep_combine(
+        _ptr(peer_yrecv), code, _ptr(ep_row), _ptr(topk_idx), n, G, _ptr(topk_gate), _ptr(residual), m, k, d,
+        _ptr(y), _stream(stream)))
+    return y
 
 
 def moe_expert_ffn(xbuf, w1, b1, w2, b2, expert_offsets, ybuf=None, workspace=None, stream=None):

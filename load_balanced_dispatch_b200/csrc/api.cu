@@ -42,6 +42,15 @@ cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, in
                                 float* f, float* P, float* aux, float* vio, float* bias, float gamma,
                                 cudaStream_t stream);
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k);
+cudaError_t launch_ep_plan(const int32_t* offsets_all, int G, int n, int rank, int32_t* send_base,
+                           int32_t* recv_offsets, cudaStream_t stream);
+cudaError_t launch_ep_dispatch(const void* x, moe_dtype dt, int64_t m, int d, int k, int n, int G,
+                               const int32_t* topk_idx, const int32_t* dest_row, const int32_t* offsets,
+                               const int32_t* send_base, void* const* peers, int64_t max_recv_rows, int32_t* ep_row,
+                               cudaStream_t stream);
+cudaError_t launch_ep_combine(const void* const* peers, moe_dtype dt, const int32_t* ep_row, const int32_t* topk_idx,
+                              int n, int G, const float* gate, const void* residual, int64_t m, int k, int d, void* y,
+                              cudaStream_t stream);
 int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, float gamma, int rule,
                           int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream, const char** err);
 int run_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* beta, int rule, int64_t seg_len,
@@ -398,6 +407,49 @@ moe_status moe_balance_step_minibatch(const float* s, int64_t m, int32_t n, int3
     if (rc != MOE_OK) return fail((moe_status)rc, "moe_balance_step_minibatch: %s", err);
     g_last_error[0] = 0;
     return MOE_OK;
+}
+
+moe_status moe_ep_plan(const int32_t* offsets_all, int32_t G, int32_t n, int32_t rank, int32_t* send_base,
+                       int32_t* recv_offsets, moe_stream_t stream) {
+    REQUIRE(G >= 1 && n >= 1 && n <= kMaxExperts && n % G == 0, "n must be in [1, %d] and divisible by G",
+            kMaxExperts);
+    REQUIRE(rank >= 0 && rank < G, "rank must be in [0, G)");
+    REQUIRE(offsets_all && send_base && recv_offsets, "offsets_all, send_base and recv_offsets are required");
+    return check_launch(launch_ep_plan(offsets_all, G, n, rank, send_base, recv_offsets, stream), "moe_ep_plan");
+}
+
+moe_status moe_ep_dispatch(const void* x, moe_dtype dt, int64_t m, int32_t d, int32_t k, int32_t n, int32_t G,
+                           const int32_t* topk_idx, const int32_t* dest_row, const int32_t* expert_offsets,
+                           const int32_t* send_base, void* const* peer_xrecv, int64_t max_recv_rows, int32_t* ep_row,
+                           moe_stream_t stream) {
+    REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
+    REQUIRE(m >= 0 && max_recv_rows >= 0 && max_recv_rows < ((int64_t)1 << 31), "bad m or max_recv_rows");
+    REQUIRE(G >= 1 && n >= 1 && n <= kMaxExperts && n % G == 0, "n must be in [1, %d] and divisible by G",
+            kMaxExperts);
+    REQUIRE(k >= 1 && k <= n && m * (int64_t)k < ((int64_t)1 << 31), "bad k");
+    REQUIRE(d >= 1 && (d * (dt == MOE_BF16 ? 2 : 4)) % 16 == 0, "d must be a multiple of %d", dt == MOE_BF16 ? 8 : 4);
+    REQUIRE(m == 0 || (x && topk_idx && dest_row && expert_offsets && send_base && peer_xrecv && ep_row),
+            "array pointers are required");
+    REQUIRE(m == 0 || aligned16(x), "x must be 16-byte aligned");
+    return check_launch(launch_ep_dispatch(x, dt, m, d, k, n, G, topk_idx, dest_row, expert_offsets, send_base,
+                                           peer_xrecv, max_recv_rows, ep_row, stream),
+                        "moe_ep_dispatch");
+}
+
+moe_status moe_ep_combine(const void* const* peer_yrecv, moe_dtype dt, const int32_t* ep_row, const int32_t* topk_idx,
+                          int32_t n, int32_t G, const float* topk_gate, const void* residual, int64_t m, int32_t k,
+                          int32_t d, void* y, moe_stream_t stream) {
+    REQUIRE(dt == MOE_F32 || dt == MOE_BF16, "unknown dtype");
+    REQUIRE(m >= 0 && k >= 1 && k <= kMaxExperts, "bad m or k");
+    REQUIRE(G >= 1 && n >= 1 && n <= kMaxExperts && n % G == 0, "n must be in [1, %d] and divisible by G",
+            kMaxExperts);
+    REQUIRE(d >= 1 && (d * (dt == MOE_BF16 ? 2 : 4)) % 16 == 0, "d must be a multiple of %d", dt == MOE_BF16 ? 8 : 4);
+    REQUIRE(m == 0 || (peer_yrecv && ep_row && topk_idx && topk_gate && y), "array pointers are required");
+    REQUIRE(aligned16(y) && aligned16(residual), "y and residual must be 16-byte aligned");
+    REQUIRE(residual == nullptr || residual != y, "residual must not alias y");
+    return check_launch(launch_ep_combine(peer_yrecv, dt, ep_row, topk_idx, n, G, topk_gate, residual, m, k, d, y,
+                                          stream),
+                        "moe_ep_combine");
 }
 
 size_t moe_balance_assign_workspace_size(int64_t m, int32_t n, int32_t k, moe_qb_mode mode) {
