@@ -59,6 +59,7 @@ def lib():
         _lib.orc_is_optimal.argtypes = [P, L, I, P, I, D]
         _lib.orc_qb_sign_step.argtypes = [P, L, I, I, P, F, I, P, P]
         _lib.orc_balance_step_minibatch.argtypes = [P, L, I, I, P, I, L, P, P]
+        _lib.orc_balance_loss_grad.argtypes = [P, P, L, I, I, L, I, D, D, D, P]
     return _lib
 
 
@@ -153,6 +154,17 @@ def balance_stats(probs, topk_idx, m, n, k, seg_len, alpha=1e-2, bias=None, gamm
         raise OracleError("orc_balance_stats", rc)
     return dict(f=f, P=None if probs is None else P, aux=None if probs is None else aux, vio=vio,
                 bias=bias_out)
+
+
+def balance_loss_grad(probs, topk_idx, m, n, k, seg_len, fn=SOFTMAX, alpha=1e-2, w_micro=0.0, w_global=1.0):
+    """Gradient of w_global L_global + w_micro L_micro with respect to the router logits: [m, n] f64."""
+    probs = np.ascontiguousarray(probs, dtype=np.float64)
+    out = np.empty((m, n), np.float64)
+    rc = lib().orc_balance_loss_grad(_p(probs), _p(_i32(topk_idx)), m, n, k, seg_len, fn, alpha, w_micro, w_global,
+                                     _p(out))
+    if rc:
+        raise OracleError("orc_balance_loss_grad", rc)
+    return out
 
 
 def balance_assign(s, k, beta=None, mode=QB_SOLVE, rule=QB_MIDPOINT, max_iters=64, max_repair=1 << 20,

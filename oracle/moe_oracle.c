@@ -349,6 +349,49 @@ int orc_balance_stats(const double* probs, const int32_t* topk_idx, int64_t m, i
     return ORC_OK;
 }
 
+/*
+ * Router gradient of the balance loss ([SWR] auxiliary load balancing loss: f_i comes from the
+ * argmax and carries no gradient, so the gradient flows through P_i, the mean router score).
+ * The loss is L = w_global * L_global + w_micro * L_micro with
+ *   L_global = alpha N sum_i f_i P_i over the whole batch (pooled counts, m tokens),
+ *   L_micro  = (1 / S) sum_s alpha N sum_i f^s_i P^s_i over the S segments of seg_len tokens
+ * (w_global = 1, w_micro = 0.01 is the hybrid loss of [QW]). With f fixed,
+ *   dL/dp_i(t) = w_global alpha N f_i / m + w_micro alpha N f^s_i / (S seg_len)   (t in segment s),
+ * and through the score function
+ *   softmax: dL/dh_j(t) = p_j(t) (dL/dp_j(t) - sum_i p_i(t) dL/dp_i(t)),
+ *   sigmoid: dL/dh_j(t) = dL/dp_j(t) p_j(t) (1 - p_j(t)).
+ * f is counted from topk_idx as in orc_balance_stats (count / (k m_seg)). dlogits [m, n].
+ */
+int orc_balance_loss_grad(const double* probs, const int32_t* topk_idx, int64_t m, int n, int k, int64_t seg_len,
+                          int fn, double alpha, double w_micro, double w_global, double* dlogits) {
+    if (seg_len <= 0 || m % seg_len != 0 || k < 1 || k > n || (fn != ORC_SOFTMAX && fn != ORC_SIGMOID))
+        return ORC_ERR_ARG;
+    const int64_t S = m / seg_len;
+    double* fg = (double*)calloc((size_t)n, sizeof(double));
+    double* fs = (double*)calloc((size_t)n, sizeof(double));
+    double* g = (double*)malloc(sizeof(double) * (size_t)n);
+    for (int64_t q = 0; q < m * k; ++q) fg[topk_idx[q]] += 1.0;
+    for (int e = 0; e < n; ++e) fg[e] /= (double)k * (double)m;
+    for (int64_t s = 0; s < S; ++s) {
+        memset(fs, 0, sizeof(double) * (size_t)n);
+        for (int64_t q = s * seg_len * k; q < (s + 1) * seg_len * k; ++q) fs[topk_idx[q]] += 1.0;
+        for (int e = 0; e < n; ++e) {
+            fs[e] /= (double)k * (double)seg_len;
+            g[e] = w_global * alpha * (double)n * fg[e] / (double)m +
+                   w_micro * alpha * (double)n * fs[e] / ((double)S * (double)seg_len);
+        }
+        for (int64_t t = s * seg_len; t < (s + 1) * seg_len; ++t) {
+            const double* p = probs + t * n;
+            double c = 0.0;
+            for (int j = 0; j < n; ++j) c += p[j] * g[j];
+            for (int j = 0; j < n; ++j)
+                dlogits[t * n + j] = fn == ORC_SOFTMAX ? p[j] * (g[j] - c) : g[j] * p[j] * (1.0 - p[j]);
+        }
+    }
+    free(fg); free(fs); free(g);
+    return ORC_OK;
+}
+
 /* ---------------------------------------------------------------------------
  * Optimal assignment ([QB]).
  *

@@ -132,3 +132,48 @@ def test_lossfree_bias_update_exact():
     exp = np.array([b[0] - g, b[1], b[2] - g, b[3] + g], np.float32)
     assert st["bias"].tolist() == exp.tolist()
     assert st["P"] is None and st["aux"] is None
+
+
+# ---------------------------------------------------------------- router gradient of the balance loss
+def _loss(h, idx, m, n, k, seg, fn, w_micro, w_global, alpha=1e-2):
+    """The balance loss at logits h with the routing (hence f) held fixed: the oracle's router
+    scores from h, then the oracle's micro-batch and global-batch losses."""
+    probs = oracle.router(None, None, m, 0, n, k, fn, 0, None, logits_in=h)[0]
+    aux = oracle.balance_stats(probs, idx, m, n, k, seg, alpha)["aux"]
+    nseg = m // seg
+    return w_global * aux[nseg + 1] + w_micro * aux[nseg]
+
+
+@pytest.mark.parametrize("fn,w_micro,w_global", [(oracle.SOFTMAX, 0.01, 1.0), (oracle.SOFTMAX, 1.0, 0.0),
+                                                 (oracle.SIGMOID, 0.0, 1.0)])
+def test_loss_grad_matches_finite_differences(fn, w_micro, w_global):
+    # "Switch Transformers paper review", auxiliary loss: f_i is fixed by the argmax, the gradient
+    # flows through P_i. Central differences of the oracle's own loss, routing held fixed.
+    m, n, k, seg = 48, 8, 2, 16
+    rng = np.random.default_rng(4)
+    h = rng.standard_normal((m, n)).astype(np.float32)
+    idx = W.make_topk_idx(m, n, k, seed=8, skew=1.0)
+    probs = oracle.router(None, None, m, 0, n, k, fn, 0, None, logits_in=h)[0]
+    g = oracle.balance_loss_grad(probs, idx, m, n, k, seg, fn, 1e-2, w_micro, w_global)
+    for t, j in [(0, 0), (5, 3), (17, 7), (33, 1), (47, 6)]:
+        hp, hm = h.copy(), h.copy()
+        hp[t, j] = np.float32(h[t, j] + np.float32(2e-3))
+        hm[t, j] = np.float32(h[t, j] - np.float32(2e-3))
+        step = float(hp[t, j]) - float(hm[t, j])
+        fd = (_loss(hp, idx, m, n, k, seg, fn, w_micro, w_global) -
+              _loss(hm, idx, m, n, k, seg, fn, w_micro, w_global)) / step
+        assert fd == pytest.approx(g[t, j], rel=1e-4, abs=1e-12)
+
+
+def test_loss_grad_softmax_rows_sum_to_zero_and_vanish_at_balance():
+    m, n, k, seg = 64, 8, 2, 32
+    rng = np.random.default_rng(5)
+    p = rng.random((m, n))
+    p /= p.sum(1, keepdims=True)
+    g = oracle.balance_loss_grad(p, W.make_topk_idx(m, n, k, seed=2), m, n, k, seg, oracle.SOFTMAX, 1e-2, 0.01, 1.0)
+    # softmax is unchanged by adding a constant to a token's logits: each gradient row sums to 0
+    assert np.abs(g.sum(1)).max() < 1e-18
+    assert np.abs(g).max() > 1e-6
+    # f_i = 1/n in every segment: dL/dp is the same for every expert, so the gradient vanishes
+    g0 = oracle.balance_loss_grad(p, W.make_round_robin_idx(m, n, k), m, n, k, seg, oracle.SOFTMAX, 1e-2, 0.01, 1.0)
+    assert np.abs(g0).max() < 1e-18
