@@ -362,7 +362,11 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 if (++buf == 2) { buf = 0; bphase ^= 1u; }
             }
             if (!ok) break;
-            // finish this thread's row: scores, ranking keys, top-k (ties -> lower index), gates
+            // finish this thread's row: scores, ranking keys, top-k (ties -> lower index), gates.
+            // The row maximum and exp-sum come from the registers; the per-expert work then runs
+            // 32 columns at a time through the warp's shared-memory tile, in a loop that is not
+            // unrolled (an unrolled pass over every expert makes the code too large for the
+            // instruction cache), and each chunk's scores go out coalesced from the same tile.
             const int64_t row0w = tb * BM + quad * 32;
             const int64_t row = row0w + lane;
             float mx = -INFINITY, sum = 0.f;
@@ -376,14 +380,32 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
             int ki[KTHREAD];
 #pragma unroll
             for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
+            float* mine = pk + lane * kParkPitch;  // this thread's row of the tile (odd pitch: no bank conflicts)
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                if (j < n) {
-                    const float hj = acc[j];
+            for (int c = 0; c < NCH; ++c) {
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) mine[q] = acc[c * 32 + q];
+                __syncwarp();
+                const int jn = min(32, n - c * 32);
+#pragma unroll 1
+                for (int q = 0; q < jn; ++q) {
+                    const int j = c * 32 + q;
+                    const float hj = mine[q];
                     const float p = softmax ? expf(hj - mx) / sum : 1.f / (1.f + expf(-hj));
                     const float key = rank_bias ? __fadd_rn(p, rank_bias[j]) : (softmax ? hj : p);
                     topk_insert(kk, ki, kp, k, key, j, p);
-                    acc[j] = p;
+                    mine[q] = p;
+                }
+                __syncwarp();
+                if (probs_out) {
+                    // the warp's 32 rows of this chunk: each store writes 128 contiguous bytes of a row
+                    const int j = c * 32 + lane;
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const int64_t r = row0w + rr;
+                        if (r >= m) break;
+                        if (j < n) probs_out[r * n + j] = pk[rr * kParkPitch + lane];
+                    }
                 }
             }
             if (row < m) {
@@ -396,23 +418,6 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     if (t < k) {
                         topk_idx[row * k + t] = ki[t];
                         topk_gate[row * k + t] = renorm_gate ? kp[t] / selsum : kp[t];
-                    }
-                }
-            }
-            if (probs_out) {
-                // the warp's 32 rows of scores, 32 columns at a time through shared memory: each
-                // store instruction writes 128 contiguous bytes of one row
-#pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    __syncwarp();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) pk[lane * kParkPitch + q] = acc[c * 32 + q];
-                    __syncwarp();
-                    const int j = c * 32 + lane;
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const int64_t r = row0w + rr;
-                        if (r >= m) break;
-                        if (j < n) probs_out[r * n + j] = pk[rr * kParkPitch + lane];
                     }
                 }
             }
