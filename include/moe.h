@@ -429,6 +429,25 @@ MOE_API moe_status moe_balance_stats(const float* probs, const int32_t* topk_idx
                              float* bias_inout, float gamma, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Router gradient of the balance loss (the backward of the statistics stage).
+ * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), auxiliary load
+ * balancing loss: f_i is set by the argmax and is not differentiable, P_i (the mean
+ * score) is, so minimising f_i P_i sends the gradient through P_i; "Qwen global-batch
+ * load balance" (agentlenshq.com) for the micro-batch / global-batch losses.
+ *  Loss: w_global L_global + w_micro L_micro (L_global = alpha n sum_i f^G_i P^G_i,
+ *  L_micro = mean over segments of alpha n sum_i f^s_i P^s_i; w_global = 1, w_micro =
+ *  0.01 is the hybrid loss aux[nseg + 2] of moe_balance_stats).
+ *  probs   [m, n] router scores of moe_router_topk (p for MOE_SOFTMAX, rho for MOE_SIGMOID).
+ *  f       [nseg + 1, n] of moe_balance_stats with the same seg_len (held fixed).
+ *  dlogits [m, n] out: dL/dh, h the router logits: softmax p_j (g_j - sum_i p_i g_i),
+ *          sigmoid g_j p_j (1 - p_j), with g_i = w_global alpha n f^G_i / m +
+ *          w_micro alpha n f^s_i / (nseg seg_len) for a token of segment s. fp32.
+ */
+MOE_API moe_status moe_balance_loss_grad(const float* probs, moe_score_fn fn, const float* f, int64_t m, int32_t n,
+                                         int64_t seg_len, float alpha, float w_micro, float w_global, float* dlogits,
+                                         moe_stream_t stream);
+
+/*
  * Global-batch statistics across data-parallel ranks, step 1 of 3: this rank's totals.
  * Passage: "Qwen global-batch load balance for MoE LLM training" (agentlenshq.com):
  * the global batch spans every data-parallel rank, so f_i is synchronised across the

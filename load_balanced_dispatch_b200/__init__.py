@@ -31,7 +31,8 @@ EXPORTS = ("moe_last_error", "moe_sync_status", "moe_router_topk_workspace_size"
            "moe_balance_stats", "moe_capacity_slots_static", "moe_balance_totals_workspace_size",
            "moe_balance_totals", "moe_balance_global", "moe_expert_ffn_combine", "moe_balance_sign_step",
            "moe_expert_ffn_gather", "moe_dispatch_tokens", "moe_router_prepare",
-           "moe_balance_step_minibatch", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine")
+           "moe_balance_step_minibatch", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
+           "moe_balance_loss_grad")
 
 
 class MoEError(RuntimeError):
@@ -68,6 +69,7 @@ def lib() -> C.CDLL:
         L.moe_dispatch.argtypes = [P, I32, I64, I32, P, P, I32, I64, P, P]
         L.moe_dispatch_tokens.argtypes = [P, I32, I64, I32, I32, P, I64, P, P]
         L.moe_ep_plan.argtypes = [P, I32, I32, I32, P, P, P]
+        L.moe_balance_loss_grad.argtypes = [P, I32, P, I64, I32, I64, F, F, F, P, P]
         L.moe_ep_dispatch.argtypes = [P, I32, I64, I32, I32, I32, I32, P, P, P, P, P, I64, P, P]
         L.moe_ep_combine.argtypes = [P, I32, P, P, I32, I32, P, P, I64, I32, I32, P, P]
         L.moe_expert_ffn_workspace_size.argtypes = [I32, I64, I32]
@@ -388,6 +390,20 @@ def moe_balance_stats(probs, topk_idx, n, seg_len=None, alpha=1e-2, bias_inout=N
         _ptr(out["aux"] if probs is not None else None), _ptr(out["vio"]), _ptr(bias_inout), gamma, _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return out
+
+
+def moe_balance_loss_grad(probs, f, seg_len=None, score_fn=MOE_SOFTMAX, alpha=1e-2, w_micro=0.01, w_global=1.0,
+                          dlogits=None, stream=None):
+    """Router-logit gradient of w_global L_global + w_micro L_micro, f held fixed. Returns dlogits [m, n]."""
+    m, n = probs.shape
+    seg_len = m if seg_len is None else seg_len
+    _need(probs, torch.float32, (m, n), "probs")
+    _need(f, torch.float32, (m // seg_len + 1, n), "f")
+    if dlogits is None:
+        dlogits = torch.empty((m, n), dtype=torch.float32, device=probs.device)
+    _check("moe_balance_loss_grad", lib().moe_balance_loss_grad(
+        _ptr(probs), score_fn, _ptr(f), m, n, seg_len, alpha, w_micro, w_global, _ptr(dlogits), _stream(stream)))
+    return dlogits
 
 
 def moe_balance_totals(probs, topk_idx, n, totals=None, workspace=None, stream=None):

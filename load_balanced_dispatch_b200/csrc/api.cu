@@ -42,6 +42,8 @@ cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, in
                                 float* f, float* P, float* aux, float* vio, float* bias, float gamma,
                                 cudaStream_t stream);
 size_t balance_workspace_bytes(int64_t m, int32_t n, int32_t k);
+cudaError_t launch_loss_grad(const float* probs, int fn, const float* f, int64_t m, int n, int64_t seg_len, float alpha,
+                             float w_micro, float w_global, float* dlogits, cudaStream_t stream);
 cudaError_t launch_ep_plan(const int32_t* offsets_all, int G, int n, int rank, int32_t* send_base,
                            int32_t* recv_offsets, cudaStream_t stream);
 cudaError_t launch_ep_dispatch(const void* x, moe_dtype dt, int64_t m, int d, int k, int n, int G,
@@ -338,6 +340,18 @@ moe_status moe_balance_stats(const float* probs, const int32_t* topk_idx, int64_
     return check_launch(launch_stats(probs, topk_idx, m, n, k, seg_len, alpha, f, P, aux, vio, bias_inout, gamma,
                                      workspace, stream, nullptr),
                         "moe_balance_stats");
+}
+
+moe_status moe_balance_loss_grad(const float* probs, moe_score_fn fn, const float* f, int64_t m, int32_t n,
+                                 int64_t seg_len, float alpha, float w_micro, float w_global, float* dlogits,
+                                 moe_stream_t stream) {
+    REQUIRE(m >= 0, "m must be >= 0");
+    REQUIRE(n >= 1 && n <= kMaxExperts, "n must be in [1, %d]", kMaxExperts);
+    REQUIRE(fn == MOE_SOFTMAX || fn == MOE_SIGMOID, "unknown score function");
+    REQUIRE(seg_len >= 1 && m % seg_len == 0, "seg_len must be >= 1 and divide m");
+    REQUIRE(m == 0 || (probs && f && dlogits), "probs, f and dlogits are required");
+    return check_launch(launch_loss_grad(probs, (int)fn, f, m, n, seg_len, alpha, w_micro, w_global, dlogits, stream),
+                        "moe_balance_loss_grad");
 }
 
 size_t moe_balance_totals_workspace_size(int64_t m, int32_t n) { return stats_workspace_bytes(m, n, m); }

@@ -351,4 +351,65 @@ cudaError_t launch_stats_global(const double* totals, int64_t m_total, int n, in
     return cudaGetLastError();
 }
 
+// Router gradient of w_global L_global + w_micro L_micro ("Switch Transformers paper review",
+// auxiliary loss: f_i is fixed by the routing decision, the gradient flows through P_i, the mean
+// score). For token t of segment s: dL/dp_i = g_i = w_global alpha n f^G_i / m
+// + w_micro alpha n f^s_i / (nseg seg_len); softmax: dL/dh_j = p_j (g_j - sum_i p_i g_i);
+// sigmoid: dL/dh_j = g_j p_j (1 - p_j). One warp per token, lane j holds experts lane + 32 q;
+// reads the scores once and writes the gradient once (HBM-bound).
+template <int NT>
+__global__ void __launch_bounds__(256)
+loss_grad_kernel(const float* __restrict__ probs, int fn, const float* __restrict__ f, int64_t m, int n,
+                 int64_t seg_len, int64_t nseg, float alpha, float w_micro, float w_global,
+                 float* __restrict__ dlogits) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    const float cg = w_global * alpha * (float)n / (float)m;
+    const float cm = w_micro * alpha * (float)n / ((float)nseg * (float)seg_len);
+    for (int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); t < m; t += warps) {
+        const int64_t seg = t / seg_len;
+        float p[NT], g[NT];
+        float c = 0.f;
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+            const int j = lane + 32 * q;
+            p[q] = 0.f;
+            g[q] = 0.f;
+            if (j < n) {
+                p[q] = probs[t * n + j];
+                g[q] = fmaf(cg, f[nseg * n + j], cm * f[seg * n + j]);
+                c = fmaf(p[q], g[q], c);
+            }
+        }
+        c = warp_sum(c);
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+            const int j = lane + 32 * q;
+            if (j < n)
+                dlogits[t * n + j] = fn == MOE_SOFTMAX ? p[q] * (g[q] - c) : g[q] * p[q] * (1.f - p[q]);
+        }
+    }
+}
+
+cudaError_t launch_loss_grad(const float* probs, int fn, const float* f, int64_t m, int n, int64_t seg_len, float alpha,
+                             float w_micro, float w_global, float* dlogits, cudaStream_t stream) {
+    if (m == 0) return cudaSuccess;
+    int64_t blocks = (m + 7) / 8;
+    if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
+    const int64_t nseg = m / seg_len;
+    if (n <= 32)
+        return launch_pdl(loss_grad_kernel<1>, dim3((unsigned)blocks), dim3(256), 0, stream, probs, fn, f, m, n,
+                          seg_len, nseg, alpha, w_micro, w_global, dlogits);
+    if (n <= 64)
+        return launch_pdl(loss_grad_kernel<2>, dim3((unsigned)blocks), dim3(256), 0, stream, probs, fn, f, m, n,
+                          seg_len, nseg, alpha, w_micro, w_global, dlogits);
+    if (n <= 128)
+        return launch_pdl(loss_grad_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, stream, probs, fn, f, m, n,
+                          seg_len, nseg, alpha, w_micro, w_global, dlogits);
+    return launch_pdl(loss_grad_kernel<8>, dim3((unsigned)blocks), dim3(256), 0, stream, probs, fn, f, m, n, seg_len,
+                      nseg, alpha, w_micro, w_global, dlogits);
+}
+
 }  // namespace moe

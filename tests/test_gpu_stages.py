@@ -341,6 +341,21 @@ def test_balance_global_across_ranks(m, n, k, ranks, with_probs):
     assert (host(bd) == ref["bias"]).all()
 
 
+# ---------------------------------------------------------------- router gradient of the balance loss
+@pytest.mark.parametrize("m,n,k,seg,fn,w_micro,w_global", [(4096, 64, 2, 512, 0, 0.01, 1.0), (2000, 8, 1, 250, 0, 1.0, 0.0),
+                                                          (3000, 256, 8, 3000, 0, 0.0, 1.0),
+                                                          (1024, 100, 6, 128, 1, 0.01, 1.0)])
+def test_balance_loss_grad(m, n, k, seg, fn, w_micro, w_global):
+    rng = np.random.default_rng(m + n)
+    logits = rng.standard_normal((m, n)).astype(np.float32)
+    idx, _, probs = lb.moe_router_topk(None, None, n, k, fn, 0, logits_in=dev(logits))
+    st = lb.moe_balance_stats(probs, idx, n, seg, 1e-2)
+    g = lb.moe_balance_loss_grad(probs, st["f"], seg, fn, 1e-2, w_micro, w_global)
+    torch.cuda.synchronize()
+    ref = oracle.balance_loss_grad(host(probs), host(idx), m, n, k, seg, fn, 1e-2, w_micro, w_global)
+    assert norm_err(host(g), ref) <= TOL_STATS
+
+
 # ---------------------------------------------------------------- mini-batch beta
 @pytest.mark.parametrize("m,n,k,seg,rule", [(65536, 256, 8, 4096, 0), (65536, 256, 8, 32768, 0),
                                             (6144, 64, 6, 1024, 1), (4000, 16, 4, 500, 2), (2048, 32, 2, 2048, 0),
