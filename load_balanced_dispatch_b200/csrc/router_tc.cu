@@ -15,14 +15,14 @@
 //     warp 0 lane 0   TMA: x tile 128x64 + the three W parts (all n rows) per stage
 //     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = n rounded up to 32 (3 parts x 4 K-steps)
 //     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM lane);
-//                     each K block's product lands in a fresh TMEM accumulator (two,
-//                     ping-pong) and is added into fp32 registers with round-to-nearest
+//                     each K block's product lands in a fresh TMEM accumulator (four,
+//                     taken in turn, so the MMAs run up to four K blocks ahead of the
+//                     drain) and is added into fp32 registers with round-to-nearest
 //                     adds, which keeps the sum fp32-accurate. After a block's last K
-//                     block the thread finishes its row in registers (softmax or
-//                     logistic, ranking key, top-k with ties to the lower index, gates)
-//                     while the MMA warp already runs the next block, and the scores go
-//                     out coalesced through a per-warp shared-memory transpose. Logits
-//                     never reach HBM.
+//                     block the thread finishes its row (softmax or logistic, ranking
+//                     key, top-k with ties to the lower index, gates) while the MMA warp
+//                     already runs the next block, and the scores go out coalesced
+//                     through a per-warp shared-memory transpose. Logits never reach HBM.
 //   router_tc_kernel     (k > 8) one CTA per 128 tokens and column tile: with probs_out
 //                        the logits are stored and router_finish_kernel (a warp per row)
 //                        finishes them in place; without it each CTA takes whole rows and
@@ -37,6 +37,16 @@ constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 drain + epil
 constexpr int A_BYTES = BM * BK * 2;
 }  // namespace rtc
 
+// Shared state of the rows kernel: up to kRowsMaxStages ring stages, kRowsAcc TMEM accumulators.
+namespace rtc {
+constexpr int kRowsMaxStages = 6, kRowsAcc = 4;
+}  // namespace rtc
+struct RouterRowsShared {
+    uint64_t full[rtc::kRowsMaxStages], empty[rtc::kRowsMaxStages], tfull[rtc::kRowsAcc], tempty[rtc::kRowsAcc];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
 struct RouterTcShared {
     uint64_t full[rtc::kMaxStages], empty[rtc::kMaxStages], tfull[2], tempty[2];
     uint32_t tmem_base;
@@ -45,6 +55,12 @@ struct RouterTcShared {
 
 __host__ __device__ inline int router_np(int n) { return ((n + 31) / 32) * 32; }
 __host__ __device__ inline int router_stage_bytes(int np) { return rtc::A_BYTES + 3 * np * 128; }
+// TMEM columns of the rows kernel: kRowsAcc accumulators of np columns, rounded up to a power of 2.
+__host__ __device__ inline uint32_t router_rows_tmem_cols(int np) {
+    uint32_t c = 32;
+    while ((int)c < rtc::kRowsAcc * np) c <<= 1;
+    return c;
+}
 __host__ __device__ inline uint32_t router_tmem_cols(int np) {
     uint32_t c = 32;
     while ((int)c < 2 * np) c <<= 1;
@@ -116,6 +132,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     using namespace rtc;
     constexpr int NP = NCH * 32;
     constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
+    static_assert(STAGES <= kMaxStages, "ring deeper than the barrier arrays");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     RouterTcShared* sh = reinterpret_cast<RouterTcShared*>(smem + STAGES * STAGE_BYTES);
@@ -256,18 +273,20 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     using namespace rtc;
     constexpr int NP = NCH * 32;
     constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
+    constexpr int NACC = kRowsAcc;
+    static_assert(STAGES <= kRowsMaxStages, "ring deeper than the barrier arrays");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* park = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [4 warps][32][kParkPitch]
-    RouterTcShared* sh = reinterpret_cast<RouterTcShared*>(park + 4 * 32 * kParkPitch);
+    RouterRowsShared* sh = reinterpret_cast<RouterRowsShared*>(park + 4 * 32 * kParkPitch);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = (d + BK - 1) / BK;
     const int64_t nblocks = (m + BM - 1) / BM;
-    const uint32_t tcols = router_tmem_cols(NP);
+    const uint32_t tcols = router_rows_tmem_cols(NP);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        for (int b = 0; b < NACC; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
         sh->abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::prefetch_tensormap(&map_x);
@@ -323,7 +342,7 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     ptx::umma_commit(&sh->empty[stage]);
                     ptx::umma_commit(&sh->tfull[buf]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                    if (++buf == 2) { buf = 0; bphase ^= 1u; }
+                    if (++buf == NACC) { buf = 0; bphase ^= 1u; }
                 }
             }
         }
@@ -359,7 +378,7 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 }
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&sh->tempty[buf]);
-                if (++buf == 2) { buf = 0; bphase ^= 1u; }
+                if (++buf == NACC) { buf = 0; bphase ^= 1u; }
             }
             if (!ok) break;
             // finish this thread's row: scores, ranking keys, top-k (ties -> lower index), gates.
@@ -433,7 +452,7 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
 
 inline size_t router_rows_smem(int np, int stages) {
     return 1024 + (size_t)stages * router_stage_bytes(np) + (size_t)4 * 32 * rtc::kParkPitch * 4 +
-           sizeof(RouterTcShared);
+           sizeof(RouterRowsShared);
 }
 
 // Ring depth of the rows kernel: as many stages as fit next to the transpose tiles (at most 6).
