@@ -265,14 +265,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 
 // Persistent full-row router (k <= KTHREAD): see the file header. Every barrier wait is bounded;
 // on a timeout all roles leave their loops and TMEM is freed.
-template <int NCH, int STAGES>
+template <int NCH, int STAGES, int H>
 __global__ void __launch_bounds__(rtc::kThreads, 1)
 router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
                    int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
                    float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
     using namespace rtc;
     constexpr int NP = NCH * 32;
-    constexpr int STAGE_BYTES = A_BYTES + 3 * NP * 128;
+    // a stage holds H consecutive 64-deep K blocks: x boxes first, then each W part's boxes
+    constexpr int W_BYTES = NP * 128;
+    constexpr int STAGE_BYTES = H * (A_BYTES + 3 * W_BYTES);
     constexpr int NACC = kRowsAcc;
     static_assert(STAGES <= kRowsMaxStages, "ring deeper than the barrier arrays");
     extern __shared__ uint8_t smem_raw[];
@@ -280,7 +282,7 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     float* park = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [4 warps][32][kParkPitch]
     RouterRowsShared* sh = reinterpret_cast<RouterRowsShared*>(park + 4 * 32 * kParkPitch);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nkb = (d + BK - 1) / BK;
+    const int nkb = ((d + BK - 1) / BK + H - 1) / H * H;  // a stage's blocks past d are zero fill
     const int64_t nblocks = (m + BM - 1) / BM;
     const uint32_t tcols = router_rows_tmem_cols(NP);
 
@@ -307,13 +309,18 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
             uint32_t phase = 0;
             bool ok = true;
             for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = 0; kb < nkb; kb += H) {
                     if (!ptx::mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* st = smem + stage * STAGE_BYTES;
                     ptx::mbar_expect_tx(&sh->full[stage], (uint32_t)STAGE_BYTES);
-                    ptx::tma_load_2d(st, &map_x, &sh->full[stage], kb * BK, (int)(tb * BM));
+#pragma unroll
+                    for (int h = 0; h < H; ++h)
+                        ptx::tma_load_2d(st + h * A_BYTES, &map_x, &sh->full[stage], (kb + h) * BK, (int)(tb * BM));
                     for (int part = 0; part < 3; ++part)
-                        ptx::tma_load_3d(st + A_BYTES + part * NP * 128, &map_w, &sh->full[stage], kb * BK, 0, part);
+#pragma unroll
+                        for (int h = 0; h < H; ++h)
+                            ptx::tma_load_3d(st + H * A_BYTES + (part * H + h) * W_BYTES, &map_w, &sh->full[stage],
+                                             (kb + h) * BK, 0, part);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -325,24 +332,27 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
             uint32_t phase = 0, bphase = 0;
             bool ok = true;
             for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!ptx::mbar_wait(&sh->tempty[buf], bphase ^ 1u, abort_flag)) { ok = false; break; }
+                for (int kb = 0; kb < nkb; kb += H) {
                     if (!ptx::mbar_wait(&sh->full[stage], phase, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
                     const uint32_t sa = ptx::smem_u32(smem + stage * STAGE_BYTES);
-                    const uint64_t adesc = ptx::sw128_kmajor_desc(sa);
-                    // a fresh accumulator per K block; the small parts of W first, the leading part last
-                    for (int part = 2; part >= 0; --part) {
-                        const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + A_BYTES + part * NP * 128);
+                    for (int h = 0; h < H; ++h) {
+                        if (!ptx::mbar_wait(&sh->tempty[buf], bphase ^ 1u, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        const uint64_t adesc = ptx::sw128_kmajor_desc(sa + h * A_BYTES);
+                        // a fresh accumulator per K block; the small parts of W first, the leading part last
+                        for (int part = 2; part >= 0; --part) {
+                            const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + H * A_BYTES + (part * H + h) * W_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            ptx::umma_bf16(tmem + (uint32_t)(buf * NP), adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                           (part != 2 || kk != 0) ? 1u : 0u);
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                ptx::umma_bf16(tmem + (uint32_t)(buf * NP), adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                               (part != 2 || kk != 0) ? 1u : 0u);
+                        }
+                        ptx::umma_commit(&sh->tfull[buf]);
+                        if (++buf == NACC) { buf = 0; bphase ^= 1u; }
                     }
+                    if (!ok) break;
                     ptx::umma_commit(&sh->empty[stage]);
-                    ptx::umma_commit(&sh->tfull[buf]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                    if (++buf == NACC) { buf = 0; bphase ^= 1u; }
                 }
             }
         }
@@ -450,31 +460,34 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     }
 }
 
-inline size_t router_rows_smem(int np, int stages) {
-    return 1024 + (size_t)stages * router_stage_bytes(np) + (size_t)4 * 32 * rtc::kParkPitch * 4 +
+inline size_t router_rows_smem(int np, int stages, int h) {
+    return 1024 + (size_t)stages * h * router_stage_bytes(np) + (size_t)4 * 32 * rtc::kParkPitch * 4 +
            sizeof(RouterRowsShared);
 }
 
-// Ring depth of the rows kernel: as many stages as fit next to the transpose tiles (at most 6).
-constexpr int router_rows_stages(int nch) { return nch == 1 ? 6 : (nch == 2 ? 4 : 3); }
+// Ring of the rows kernel: H K blocks per stage (two for up to 64 experts: each x row is then
+// read 256 contiguous bytes at a time), and as many stages as fit next to the transpose tiles.
+constexpr int router_rows_h(int nch) { return nch <= 2 ? 2 : 1; }
+constexpr int router_rows_stages(int nch) { return nch == 1 ? 3 : (nch == 2 ? 2 : 3); }
 
 template <int NCH>
 static cudaError_t launch_router_rows_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
                                         int fn, int renorm, const float* rank_bias, float* probs_out,
                                         int32_t* topk_idx, float* topk_gate, cudaStream_t stream) {
-    constexpr int ST = router_rows_stages(NCH);
-    const size_t smem = router_rows_smem(NCH * 32, ST);
+    constexpr int ST = router_rows_stages(NCH), H = router_rows_h(NCH);
+    const size_t smem = router_rows_smem(NCH * 32, ST, H);
     static bool attr = false;
     if (!attr) {
-        const cudaError_t e = cudaFuncSetAttribute(router_rows_kernel<NCH, ST>,
+        const cudaError_t e = cudaFuncSetAttribute(router_rows_kernel<NCH, ST, H>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
-    const unsigned grid = (unsigned)(blocks < num_sms() ? blocks : num_sms());
-    return launch_pdl(router_rows_kernel<NCH, ST>, dim3(grid), dim3(rtc::kThreads), smem, stream, mx, mw, m, d, n, k,
-                      fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+    const int64_t cap = (int64_t)num_sms();
+    const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
+    return launch_pdl(router_rows_kernel<NCH, ST, H>, dim3(grid), dim3(rtc::kThreads), smem, stream, mx, mw, m, d, n,
+                      k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
 }
 
 size_t router_workspace_bytes(int32_t d, int32_t n, moe_dtype dt) {
