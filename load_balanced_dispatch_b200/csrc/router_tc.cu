@@ -10,19 +10,21 @@
 //
 //   router_split_kernel  W_r [d, n] fp32 -> workspace [3, n, d] bf16 (K-major B operand);
 //                        run once per weight by moe_router_prepare, or on every call.
-//   router_rows_kernel   (k <= 8) persistent, one CTA per SM, 192 threads, each CTA
+//   router_rows_kernel   (k <= 8) persistent, one CTA per SM, 320 threads, each CTA
 //                        taking 128-token blocks in turn with all n <= 128 experts:
-//     warp 0 lane 0   TMA: x tile 128x64 + the three W parts (all n rows) per stage
+//     warp 0 lane 0   TMA: x tiles 128x64 + the three W parts (all n rows), two 64-deep
+//                     K blocks per stage for n <= 64
 //     warp 1 lane 0   tcgen05.mma kind::f16 M=128, N = n rounded up to 32 (3 parts x 4 K-steps)
 //     warps 2-5       drain: thread t of warp w owns token row 32(w%4) + t (its TMEM lane);
 //                     each K block's product lands in a fresh TMEM accumulator (four,
 //                     taken in turn, so the MMAs run up to four K blocks ahead of the
 //                     drain) and is added into fp32 registers with round-to-nearest
 //                     adds, which keeps the sum fp32-accurate. After a block's last K
-//                     block the thread finishes its row (softmax or logistic, ranking
-//                     key, top-k with ties to the lower index, gates) while the MMA warp
-//                     already runs the next block, and the scores go out coalesced
-//                     through a per-warp shared-memory transpose. Logits never reach HBM.
+//                     block the rows go to a shared-memory logits tile.
+//     warps 6-9       finish: a warp per row, 32 rows per warp (softmax or logistic,
+//                     ranking key, top-k with ties to the lower index, gates, scores
+//                     stored coalesced) while the drain accumulates the next block.
+//                     Logits never reach HBM.
 //   router_tc_kernel     (k > 8) one CTA per 128 tokens and column tile: with probs_out
 //                        the logits are stored and router_finish_kernel (a warp per row)
 //                        finishes them in place; without it each CTA takes whole rows and
@@ -40,9 +42,11 @@ constexpr int A_BYTES = BM * BK * 2;
 // Shared state of the rows kernel: up to kRowsMaxStages ring stages, kRowsAcc TMEM accumulators.
 namespace rtc {
 constexpr int kRowsMaxStages = 6, kRowsAcc = 4;
+constexpr int kRowsThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 drain, warps 6-9 finish
 }  // namespace rtc
 struct RouterRowsShared {
     uint64_t full[rtc::kRowsMaxStages], empty[rtc::kRowsMaxStages], tfull[rtc::kRowsAcc], tempty[rtc::kRowsAcc];
+    uint64_t park_full, park_empty;  // a token block's logits handed from the drain to the finish warps
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -102,7 +106,6 @@ constexpr int KTHREAD = 8;  // largest k finished one row per thread
 
 namespace rtc {
 enum { kModeLogits = 0, kModeRows = 2 };
-constexpr int kParkPitch = 33;  // padded row pitch of a warp's 32 x 32 transpose tile
 }  // namespace rtc
 
 // Insert (key, j, p) into a best-first list of length k <= KTHREAD (ties: the lower index first).
@@ -266,7 +269,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
 // Persistent full-row router (k <= KTHREAD): see the file header. Every barrier wait is bounded;
 // on a timeout all roles leave their loops and TMEM is freed.
 template <int NCH, int STAGES, int H>
-__global__ void __launch_bounds__(rtc::kThreads, 1)
+__global__ void __launch_bounds__(rtc::kRowsThreads, 1)
 router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
                    int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
                    float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
@@ -276,11 +279,12 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     constexpr int W_BYTES = NP * 128;
     constexpr int STAGE_BYTES = H * (A_BYTES + 3 * W_BYTES);
     constexpr int NACC = kRowsAcc;
+    constexpr int PITCH = NP + 1;  // odd row pitch of the logits tile: no shared-memory bank conflicts
     static_assert(STAGES <= kRowsMaxStages, "ring deeper than the barrier arrays");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* park = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [4 warps][32][kParkPitch]
-    RouterRowsShared* sh = reinterpret_cast<RouterRowsShared*>(park + 4 * 32 * kParkPitch);
+    float* park = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [BM][PITCH] logits of one block
+    RouterRowsShared* sh = reinterpret_cast<RouterRowsShared*>(park + BM * PITCH);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = ((d + BK - 1) / BK + H - 1) / H * H;  // a stage's blocks past d are zero fill
     const int64_t nblocks = (m + BM - 1) / BM;
@@ -289,6 +293,8 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
         for (int b = 0; b < NACC; ++b) { ptx::mbar_init(&sh->tfull[b], 1); ptx::mbar_init(&sh->tempty[b], 128); }
+        ptx::mbar_init(&sh->park_full, 128);
+        ptx::mbar_init(&sh->park_empty, 128);
         sh->abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::prefetch_tensormap(&map_x);
@@ -298,7 +304,6 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    pdl_trigger();
     pdl_wait();  // x (and the W split when made by this call) come from earlier launches
     const uint32_t tmem = sh->tmem_base;
     volatile int* abort_flag = &sh->abort_flag;
@@ -356,13 +361,13 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 }
             }
         }
-    } else {
-        const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31 belong to this warp
+    } else if (warp < 6) {
+        // drain: thread t of this warp owns the block's row 32 quad + t (its TMEM lane)
+        const int quad = warp & 3;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        float* pk = park + quad * 32 * kParkPitch;
-        const bool softmax = fn == MOE_SOFTMAX;
+        float* prow = park + (quad * 32 + lane) * PITCH;
         int buf = 0;
-        uint32_t bphase = 0;
+        uint32_t bphase = 0, pphase = 0;
         bool ok = true;
         for (int64_t tb = blockIdx.x; tb < nblocks && ok; tb += gridDim.x) {
             float acc[NP];
@@ -391,67 +396,36 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 if (++buf == NACC) { buf = 0; bphase ^= 1u; }
             }
             if (!ok) break;
-            // finish this thread's row: scores, ranking keys, top-k (ties -> lower index), gates.
-            // The row maximum and exp-sum come from the registers; the per-expert work then runs
-            // 32 columns at a time through the warp's shared-memory tile, in a loop that is not
-            // unrolled (an unrolled pass over every expert makes the code too large for the
-            // instruction cache), and each chunk's scores go out coalesced from the same tile.
-            const int64_t row0w = tb * BM + quad * 32;
-            const int64_t row = row0w + lane;
-            float mx = -INFINITY, sum = 0.f;
-            if (softmax) {
+            // hand the block's logits to the finish warps once they are done with the previous block
+            if (!ptx::mbar_wait(&sh->park_empty, pphase ^ 1u, abort_flag)) break;
 #pragma unroll
-                for (int j = 0; j < NP; ++j) if (j < n) mx = fmaxf(mx, acc[j]);
+            for (int j = 0; j < NP; ++j) prow[j] = acc[j];
+            ptx::mbar_arrive(&sh->park_full);
+            pphase ^= 1u;
+        }
+    } else {
+        // finish: warp f takes rows 32 f .. 32 f + 31 of each block, one row at a time with the
+        // whole warp (lane holds experts lane + 32 q): scores, ranking keys, top-k, gates, and the
+        // scores stored coalesced, while the drain accumulates the next block
+        const int fw = warp - 6;
+        uint32_t pphase = 0;
+        for (int64_t tb = blockIdx.x; tb < nblocks; tb += gridDim.x) {
+            if (!ptx::mbar_wait(&sh->park_full, pphase, abort_flag)) break;
+            for (int rr = 0; rr < 32; ++rr) {
+                const int r = fw * 32 + rr;
+                const int64_t row = tb * BM + r;
+                if (row >= m) break;
+                float hv[NCH];
 #pragma unroll
-                for (int j = 0; j < NP; ++j) if (j < n) sum += expf(acc[j] - mx);
+                for (int q = 0; q < NCH; ++q) hv[q] = park[r * PITCH + lane + 32 * q];
+                finish_row<NCH>(hv, row, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
             }
-            float kk[KTHREAD], kp[KTHREAD];
-            int ki[KTHREAD];
-#pragma unroll
-            for (int t = 0; t < KTHREAD; ++t) { kk[t] = -INFINITY; ki[t] = 0x7fffffff; kp[t] = 0.f; }
-            float* mine = pk + lane * kParkPitch;  // this thread's row of the tile (odd pitch: no bank conflicts)
-#pragma unroll
-            for (int c = 0; c < NCH; ++c) {
-                __syncwarp();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) mine[q] = acc[c * 32 + q];
-                __syncwarp();
-                const int jn = min(32, n - c * 32);
-#pragma unroll 1
-                for (int q = 0; q < jn; ++q) {
-                    const int j = c * 32 + q;
-                    const float hj = mine[q];
-                    const float p = softmax ? expf(hj - mx) / sum : 1.f / (1.f + expf(-hj));
-                    const float key = rank_bias ? __fadd_rn(p, rank_bias[j]) : (softmax ? hj : p);
-                    topk_insert(kk, ki, kp, k, key, j, p);
-                    mine[q] = p;
-                }
-                __syncwarp();
-                if (probs_out) {
-                    // the warp's 32 rows of this chunk: each store writes 128 contiguous bytes of a row
-                    const int j = c * 32 + lane;
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const int64_t r = row0w + rr;
-                        if (r >= m) break;
-                        if (j < n) probs_out[r * n + j] = pk[rr * kParkPitch + lane];
-                    }
-                }
-            }
-            if (row < m) {
-                float selsum = 0.f;
-#pragma unroll
-                for (int t = 0; t < KTHREAD; ++t) if (t < k) selsum += kp[t];
-                const bool renorm_gate = softmax && renorm;
-#pragma unroll
-                for (int t = 0; t < KTHREAD; ++t) {
-                    if (t < k) {
-                        topk_idx[row * k + t] = ki[t];
-                        topk_gate[row * k + t] = renorm_gate ? kp[t] / selsum : kp[t];
-                    }
-                }
-            }
+            __syncwarp();
+            ptx::mbar_arrive(&sh->park_empty);
+            pphase ^= 1u;
         }
     }
+    pdl_trigger();  // the dependent launch may start while this grid drains
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -461,14 +435,14 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
 }
 
 inline size_t router_rows_smem(int np, int stages, int h) {
-    return 1024 + (size_t)stages * h * router_stage_bytes(np) + (size_t)4 * 32 * rtc::kParkPitch * 4 +
+    return 1024 + (size_t)stages * h * router_stage_bytes(np) + (size_t)rtc::BM * (np + 1) * 4 +
            sizeof(RouterRowsShared);
 }
 
 // Ring of the rows kernel: H K blocks per stage (two for up to 64 experts: each x row is then
-// read 256 contiguous bytes at a time), and as many stages as fit next to the transpose tiles.
+// read 256 contiguous bytes at a time), and as many stages as fit next to the logits tile.
 constexpr int router_rows_h(int nch) { return nch <= 2 ? 2 : 1; }
-constexpr int router_rows_stages(int nch) { return nch == 1 ? 3 : (nch == 2 ? 2 : 3); }
+constexpr int router_rows_stages(int nch) { return nch == 1 ? 3 : (nch == 2 ? 2 : (nch == 3 ? 3 : 2)); }
 
 template <int NCH>
 static cudaError_t launch_router_rows_t(const CUtensorMap& mx, const CUtensorMap& mw, int64_t m, int d, int n, int k,
@@ -486,7 +460,7 @@ static cudaError_t launch_router_rows_t(const CUtensorMap& mx, const CUtensorMap
     const int64_t blocks = (m + rtc::BM - 1) / rtc::BM;
     const int64_t cap = (int64_t)num_sms();
     const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
-    return launch_pdl(router_rows_kernel<NCH, ST, H>, dim3(grid), dim3(rtc::kThreads), smem, stream, mx, mw, m, d, n,
+    return launch_pdl(router_rows_kernel<NCH, ST, H>, dim3(grid), dim3(rtc::kRowsThreads), smem, stream, mx, mw, m, d, n,
                       k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
 }
 
