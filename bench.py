@@ -60,10 +60,11 @@ def peaks_all():
                 "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED, "source": "fallback"}
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one ffn_fused_tc launch at a shape, from the
-# ncu capture summarised under profiles/. Emptied whenever the kernel changes (the figure would be
-# stale), refilled from the next capture.
-FFN_DRAM_TRAFFIC = {"switch": 1239.07e6 + 39.97e6}
+# dram__bytes_read.sum + dram__bytes_write.sum of one FFN launch at a shape, from the ncu captures
+# summarised under profiles/ (switch: ffn_fused_tc, the one-pick FFN with the combine in its
+# epilogue; lossfree and global: ffn_pair_tc). An entry is removed whenever its kernel changes
+# (the figure would be stale) and refilled from the next capture.
+FFN_DRAM_TRAFFIC = {"switch": 1239.07e6 + 39.97e6, "lossfree": 1418.98e6 + 647.99e6, "global": 5.11e9 + 753.91e6}
 
 
 def ffn_roofline(cfg, offsets, ffn_ms, esz=2):
