@@ -67,7 +67,6 @@ dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, con
 __global__ void __launch_bounds__(kRowThreads)
 dispatch_tokens_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, int k,
                        const int32_t* __restrict__ dest_row, int64_t max_rows, uint4* __restrict__ xbuf) {
-    pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
@@ -105,6 +104,7 @@ dispatch_tokens_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_r
             }
         }
     }
+    pdl_trigger();  // after this CTA's rows: the dependent launch starts as the grid drains
 }
 
 // y[i] = (residual[i]) + sum_r g_ir * ybuf[dest_row[i,r]]  (fp32 accumulation, picks in order).
@@ -117,7 +117,6 @@ combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row,
     constexpr int V = Vec16<T>::N;
     constexpr int U = 4;
     const int lane = threadIdx.x & 31;
-    pdl_trigger();
     pdl_wait();
     const int nvec = d / V;
     const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
@@ -161,6 +160,7 @@ combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row,
             }
         }
     }
+    pdl_trigger();  // after this CTA's tokens: the dependent launch starts as the grid drains
 }
 
 cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const int32_t* src_token,

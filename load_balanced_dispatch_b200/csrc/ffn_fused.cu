@@ -178,7 +178,6 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         ptx::prefetch_tensormap(&map_w2);
     }
     if (warp == 1) ptx::tmem_alloc(&sh->tmem_base, TMEM_COLS);
-    pdl_trigger();
     pdl_wait();  // expert_offsets, xbuf and the counters come from earlier launches
     if (warp == 2) build_group_table(offsets, n, ntn1, BM, max_rows, sh->g1);
     if (warp == 3) build_group_table(offsets, n, ntn2, BM, max_rows, sh->g2);
@@ -439,6 +438,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
             if (++acc == 2) { acc = 0; aphase ^= 1u; }
         }
     }
+    pdl_trigger();  // the dependent launch may start while this grid drains
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {

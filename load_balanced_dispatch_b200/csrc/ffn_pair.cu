@@ -120,7 +120,6 @@ ffn_pair_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
         ptx::prefetch_tensormap(&map_w2);
     }
     if (warp == 1) ptx::tmem_alloc_pair(&sh->tmem_base, TMEM_COLS);
-    pdl_trigger();
     pdl_wait();  // expert_offsets, xbuf and the counters come from earlier launches
     if (warp == 2) build_group_table(offsets, n, ntn1, BM, max_rows, sh->g1);
     if (warp == 3) build_group_table(offsets, n, ntn2, BM, max_rows, sh->g2);
@@ -311,6 +310,7 @@ ffn_pair_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
             if (++acc == 2) { acc = 0; aphase ^= 1u; }
         }
     }
+    pdl_trigger();  // the dependent launch may start while the pairs drain
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync();  // neither CTA frees its TMEM while the pair may still use it

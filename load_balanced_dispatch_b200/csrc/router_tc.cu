@@ -59,12 +59,6 @@ struct RouterTcShared {
 
 __host__ __device__ inline int router_np(int n) { return ((n + 31) / 32) * 32; }
 __host__ __device__ inline int router_stage_bytes(int np) { return rtc::A_BYTES + 3 * np * 128; }
-// TMEM columns of the rows kernel: kRowsAcc accumulators of np columns, rounded up to a power of 2.
-__host__ __device__ inline uint32_t router_rows_tmem_cols(int np) {
-    uint32_t c = 32;
-    while ((int)c < rtc::kRowsAcc * np) c <<= 1;
-    return c;
-}
 __host__ __device__ inline uint32_t router_tmem_cols(int np) {
     uint32_t c = 32;
     while ((int)c < 2 * np) c <<= 1;
@@ -275,10 +269,13 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                    float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
     using namespace rtc;
     constexpr int NP = NCH * 32;
-    // a stage holds H consecutive 64-deep K blocks: x boxes first, then each W part's boxes
+    // a stage holds H consecutive 64-deep K blocks: x boxes first, then per block the three W
+    // parts' boxes, adjacent (so that for n <= 64 one N = 3 NP MMA takes all three parts)
     constexpr int W_BYTES = NP * 128;
     constexpr int STAGE_BYTES = H * (A_BYTES + 3 * W_BYTES);
-    constexpr int NACC = kRowsAcc;
+    constexpr bool FUSEP = NP <= 64;               // the three parts in one MMA, separate columns
+    constexpr int WIDTH = FUSEP ? 3 * NP : NP;     // TMEM columns of one accumulator
+    constexpr int NACC = (FUSEP && NP == 64) ? 2 : kRowsAcc;
     constexpr int PITCH = NP + 1;  // odd row pitch of the logits tile: no shared-memory bank conflicts
     static_assert(STAGES <= kRowsMaxStages, "ring deeper than the barrier arrays");
     extern __shared__ uint8_t smem_raw[];
@@ -288,7 +285,8 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = ((d + BK - 1) / BK + H - 1) / H * H;  // a stage's blocks past d are zero fill
     const int64_t nblocks = (m + BM - 1) / BM;
-    const uint32_t tcols = router_rows_tmem_cols(NP);
+    uint32_t tcols = 32;
+    while ((int)tcols < NACC * WIDTH) tcols <<= 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&sh->full[s], 1); ptx::mbar_init(&sh->empty[s], 1); }
@@ -321,10 +319,10 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
 #pragma unroll
                     for (int h = 0; h < H; ++h)
                         ptx::tma_load_2d(st + h * A_BYTES, &map_x, &sh->full[stage], (kb + h) * BK, (int)(tb * BM));
-                    for (int part = 0; part < 3; ++part)
 #pragma unroll
-                        for (int h = 0; h < H; ++h)
-                            ptx::tma_load_3d(st + H * A_BYTES + (part * H + h) * W_BYTES, &map_w, &sh->full[stage],
+                    for (int h = 0; h < H; ++h)
+                        for (int part = 0; part < 3; ++part)
+                            ptx::tma_load_3d(st + H * A_BYTES + (h * 3 + part) * W_BYTES, &map_w, &sh->full[stage],
                                              (kb + h) * BK, 0, part);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -332,7 +330,7 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = ptx::idesc_bf16_f32(BM, NP);
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, WIDTH);
             int stage = 0, buf = 0;
             uint32_t phase = 0, bphase = 0;
             bool ok = true;
@@ -344,13 +342,23 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                         if (!ptx::mbar_wait(&sh->tempty[buf], bphase ^ 1u, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
                         const uint64_t adesc = ptx::sw128_kmajor_desc(sa + h * A_BYTES);
-                        // a fresh accumulator per K block; the small parts of W first, the leading part last
-                        for (int part = 2; part >= 0; --part) {
-                            const uint64_t bdesc = ptx::sw128_kmajor_desc(sa + H * A_BYTES + (part * H + h) * W_BYTES);
+                        const uint32_t wbase = sa + H * A_BYTES + h * 3 * W_BYTES;
+                        if (FUSEP) {
+                            // a fresh accumulator per K block; part p's products in columns p NP ..
+                            const uint64_t bdesc = ptx::sw128_kmajor_desc(wbase);
 #pragma unroll
                             for (int kk = 0; kk < BK / 16; ++kk)
-                                ptx::umma_bf16(tmem + (uint32_t)(buf * NP), adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                               (part != 2 || kk != 0) ? 1u : 0u);
+                                ptx::umma_bf16(tmem + (uint32_t)(buf * WIDTH), adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                               kk != 0 ? 1u : 0u);
+                        } else {
+                            // a fresh accumulator per K block; the small parts of W first, the leading part last
+                            for (int part = 2; part >= 0; --part) {
+                                const uint64_t bdesc = ptx::sw128_kmajor_desc(wbase + part * W_BYTES);
+#pragma unroll
+                                for (int kk = 0; kk < BK / 16; ++kk)
+                                    ptx::umma_bf16(tmem + (uint32_t)(buf * WIDTH), adesc + 2 * kk, bdesc + 2 * kk,
+                                                   idesc, (part != 2 || kk != 0) ? 1u : 0u);
+                            }
                         }
                         ptx::umma_commit(&sh->tfull[buf]);
                         if (++buf == NACC) { buf = 0; bphase ^= 1u; }
@@ -376,19 +384,41 @@ router_rows_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                // two 32-column chunks in flight per wait
+                if (FUSEP) {
+                    // per 32 experts: the three parts' products in flight together, added smallest
+                    // first ((w2 + w1) + w0), then into the running sum (all round to nearest)
 #pragma unroll
-                for (int c = 0; c < NCH; c += 2) {
-                    uint32_t v[2][32];
-                    ptx::tmem_ld32_issue(trow + (uint32_t)(buf * NP + c * 32), v[0]);
-                    if (c + 1 < NCH) ptx::tmem_ld32_issue(trow + (uint32_t)(buf * NP + (c + 1) * 32), v[1]);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[0][q]));
-                    if (c + 1 < NCH) {
+                    for (int c = 0; c < NCH; ++c) {
+                        uint32_t v[2][32];
+                        ptx::tmem_ld32_issue(trow + (uint32_t)(buf * WIDTH + 2 * NP + c * 32), v[0]);
+                        ptx::tmem_ld32_issue(trow + (uint32_t)(buf * WIDTH + NP + c * 32), v[1]);
+                        ptx::tmem_wait_ld();
 #pragma unroll
                         for (int q = 0; q < 32; ++q)
-                            acc[(c + 1) * 32 + q] = __fadd_rn(acc[(c + 1) * 32 + q], __uint_as_float(v[1][q]));
+                            v[1][q] = __float_as_uint(__fadd_rn(__uint_as_float(v[0][q]), __uint_as_float(v[1][q])));
+                        ptx::tmem_ld32_issue(trow + (uint32_t)(buf * WIDTH + c * 32), v[0]);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q],
+                                                        __fadd_rn(__uint_as_float(v[1][q]), __uint_as_float(v[0][q])));
+                    }
+                } else {
+                    // two 32-column chunks in flight per wait
+#pragma unroll
+                    for (int c = 0; c < NCH; c += 2) {
+                        uint32_t v[2][32];
+                        ptx::tmem_ld32_issue(trow + (uint32_t)(buf * WIDTH + c * 32), v[0]);
+                        if (c + 1 < NCH) ptx::tmem_ld32_issue(trow + (uint32_t)(buf * WIDTH + (c + 1) * 32), v[1]);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            acc[c * 32 + q] = __fadd_rn(acc[c * 32 + q], __uint_as_float(v[0][q]));
+                        if (c + 1 < NCH) {
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                acc[(c + 1) * 32 + q] = __fadd_rn(acc[(c + 1) * 32 + q], __uint_as_float(v[1][q]));
+                        }
                     }
                 }
                 ptx::tc_fence_before();
