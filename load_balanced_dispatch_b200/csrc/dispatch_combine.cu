@@ -107,57 +107,46 @@ dispatch_tokens_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_r
     pdl_trigger();  // after this CTA's rows: the dependent launch starts as the grid drains
 }
 
-// y[i] = (residual[i]) + sum_r g_ir * ybuf[dest_row[i,r]]  (fp32 accumulation, picks in order).
-// One warp per token; a lane takes U 16-byte column chunks at a time, so U x k row loads are in
-// flight together.
+// y[i] = (residual[i]) + sum_r g_ir * ybuf[dest_row[i,r]]  (fp32 accumulation).
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
 combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row, const float* __restrict__ gate,
                const T* __restrict__ residual, int64_t m, int k, int d, int gate_bf16, T* __restrict__ y) {
     constexpr int V = Vec16<T>::N;
-    constexpr int U = 4;
     const int lane = threadIdx.x & 31;
     pdl_wait();
     const int nvec = d / V;
     const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
     for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
-        for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
-            float acc[U][V];
+        // two 16-byte column chunks per lane at a time: their k row loads are independent
+        for (int c0 = lane; c0 < nvec; c0 += 64) {
+            const int c1 = c0 + 32;
+            const bool has1 = c1 < nvec;
+            float acc0[V], acc1[V];
+            if (residual) {
+                Vec16<T>::load(residual + i * d + (int64_t)c0 * V, acc0);
+                if (has1) Vec16<T>::load(residual + i * d + (int64_t)c1 * V, acc1);
+            } else {
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (residual && c < nvec) {
-                    Vec16<T>::load(residual + i * d + (int64_t)c * V, acc[u]);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < V; ++q) acc[u][q] = 0.f;
-                }
+                for (int q = 0; q < V; ++q) { acc0[q] = 0.f; acc1[q] = 0.f; }
             }
             for (int r = 0; r < k; ++r) {
                 const int32_t row = dest_row[i * k + r];
                 if (row < 0) continue;
                 float g = gate[i * k + r];
                 if (gate_bf16) g = round_to_bf16(g);
+                float v0[V], v1[V];
                 const T* yr = ybuf + (int64_t)row * d;
-                float v[U][V];
+                Vec16<T>::load(yr + (int64_t)c0 * V, v0);
+                if (has1) Vec16<T>::load(yr + (int64_t)c1 * V, v1);
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int c = c0 + 32 * u;
-                    if (c < nvec) Vec16<T>::load(yr + (int64_t)c * V, v[u]);
-                }
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if (c0 + 32 * u < nvec) {
-#pragma unroll
-                        for (int q = 0; q < V; ++q) acc[u][q] = fmaf(g, v[u][q], acc[u][q]);
-                    }
+                for (int q = 0; q < V; ++q) {
+                    acc0[q] = fmaf(g, v0[q], acc0[q]);
+                    if (has1) acc1[q] = fmaf(g, v1[q], acc1[q]);
                 }
             }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nvec) Vec16<T>::store(y + i * d + (int64_t)c * V, acc[u]);
-            }
+            Vec16<T>::store(y + i * d + (int64_t)c0 * V, acc0);
+            if (has1) Vec16<T>::store(y + i * d + (int64_t)c1 * V, acc1);
         }
     }
     pdl_trigger();  // after this CTA's tokens: the dependent launch starts as the grid drains
