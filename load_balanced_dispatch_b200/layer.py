@@ -219,15 +219,15 @@ class MoELayer:
                                   stream=stream)
 
     def launches_per_forward(self) -> int:
-        """Kernel launches of one forward: router (1; 2 for bf16 with k > 8: projection and finish), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
+        """Kernel launches of one forward: router (bf16 with n <= 128: projection and finish, 2; else 1), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
         gathers its rows from x), FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
         combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus
         one launch for the dropped tokens' rows (which also clears the FFN's counters)."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
-        router = 1  # tensor-core rows kernel (split prepared once; k <= 8) or the fp32 FMA kernel
-        if bf16 and s.n <= 128 and s.k > 8:
-            router = 2  # tensor-core logits tiles + the finish kernel
+        # bf16 with n <= 128: tensor-core logits tiles + the finish kernel (the W_r split is made
+        # once, at construction); otherwise the fp32 FMA kernel
+        router = 2 if (bf16 and s.n <= 128) else 1
         capacity = 2
         dispatch = 1 if self.uses_dispatch() else 0
         if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped rows

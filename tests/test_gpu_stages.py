@@ -89,8 +89,8 @@ def test_router_projection(dtype, m, d, n, k, fn, renorm, bias):
                                                       (700, 512, 64, 6, 1, 0, True), (64, 64, 16, 12, 0, 0, False),
                                                       (400, 128, 100, 8, 1, 0, True)])
 def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
-    # no probs_out: the tensor-core path finishes the rows in the kernel (in the drain threads for
-    # k <= 8, a warp per row for k > 8) and stores nothing but the picks and gates
+    # no probs_out: the tensor-core path keeps whole rows per CTA and a warp finishes each row in
+    # the kernel; nothing but the picks and gates is stored
     rng = np.random.default_rng(d * 3 + n)
     x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
     w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
@@ -108,10 +108,9 @@ def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
 
 @pytest.mark.parametrize("m,d,n,k,fn,renorm,bias", [(40000, 256, 64, 2, 0, 1, False), (20000, 512, 128, 1, 0, 0, False),
                                                       (19100, 192, 96, 6, 1, 0, True), (30001, 128, 32, 4, 0, 0, False)])
-def test_router_persistent_blocks_and_prepared_split(m, d, n, k, fn, renorm, bias):
-    # more 128-token blocks than SMs, so each CTA of the persistent kernel takes several in turn
-    # (ragged last block); the call with w_r = None on a workspace from moe_router_prepare gives
-    # the same bits as the call that splits W_r itself
+def test_router_many_blocks_and_prepared_split(m, d, n, k, fn, renorm, bias):
+    # more 128-token blocks than two waves of CTAs (ragged last block); the call with w_r = None
+    # on a workspace from moe_router_prepare gives the same bits as the call that splits W_r itself
     rng = np.random.default_rng(m + d)
     x = W.round_to_bf16(rng.standard_normal((m, d)).astype(np.float32))
     w = (rng.standard_normal((d, n)) / np.sqrt(d)).astype(np.float32)
