@@ -128,9 +128,10 @@ MOE_API moe_status moe_router_prepare(const float* w_r, int32_t d, int32_t n, in
  * alternating QB algorithm box, and its practical one-step form under
  * "Mind the pitfall" (select with the old beta, then update beta).
  *
- *  s          [m, n] fp32 scores, row-major, any 4-byte alignment (rows that start on
- *             16-byte boundaries take the faster bulk-copy and vector paths). (m * k) % n
- *             must be 0 and k < n.
+ *  s          [m, n] fp32 scores, row-major, finite (no NaN or infinity: the results are
+ *             unspecified otherwise), any 4-byte alignment (rows that start on 16-byte
+ *             boundaries take the faster bulk-copy and vector paths). (m * k) % n must be 0
+ *             and k < n.
  *  beta       [n] fp32, in: previous beta (zeros for a cold start); out: new beta.
  *  mode       MOE_QB_STEP: x = topk(s - beta_old); one alpha/beta update -> beta_new.
  *             MOE_QB_SOLVE: alternate row/column passes until topk(s - beta) has

@@ -200,11 +200,13 @@ struct RowSweep {
     uint32_t* g_cand;      // [n][kGCap] the keys inside it
 };
 
-// Append the CTA's buffered (column, key) pairs to the global candidate lists (all threads).
+// Append the CTA's buffered (column, key) pairs to the global candidate lists (all threads); the
+// buffer holds min(*npairs, cap) pairs.
 __device__ __forceinline__ void sweep_flush(const uint2* pairs, unsigned* npairs, uint32_t* scnt, uint32_t* sbase,
-                                            unsigned char* sfull, int n, const RowSweep& sw) {
+                                            unsigned char* sfull, int n, const RowSweep& sw,
+                                            unsigned cap = (unsigned)qb::kRowPairCap) {
     const int tid = threadIdx.x, T = blockDim.x;
-    const unsigned np = min(*npairs, (unsigned)qb::kRowPairCap);
+    const unsigned np = min(*npairs, cap);
     for (unsigned p = tid; p < np; p += T) atomicAdd(&scnt[pairs[p].x], 1u);
     __syncthreads();
     for (int j = tid; j < n; j += T) {
@@ -423,6 +425,437 @@ qb_row_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float*
         }
         __syncthreads();
         if (npairs) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Thread-per-row form of the row pass (used when k + 1 <= the number of column groups).
+//
+// A warp owns a tile of 32 consecutive rows of s in shared memory (one bulk copy per row into a
+// padded row stride, so that 16-byte reads of one column chunk by the 32 threads hit distinct
+// banks) and each thread selects for one row:
+//   1. group maxima: the row's columns in 32 groups of NT consecutive columns; gm_g = max over
+//      the group of v = fp32(s - beta);
+//   2. T = the (k+1)-th largest of the 32 group maxima (a sorting network in registers): k + 1
+//      distinct elements reach T, so T is a lower bound of the row's (k+1)-th largest v;
+//   3. the elements with v >= T' (T' = T, or lower for the window sweep, below) are listed in
+//      ascending column order (one byte each), scanning only the groups whose maximum reaches T';
+//   4. the listed elements with v >= T are sorted by key (a second network); the k-th and
+//      (k+1)-th keys give vk and vk1 (the same values as the ranked selection; only the sign of
+//      a zero may differ, and nothing downstream sees it), and the picks are the listed
+//      elements with a larger key plus, on a tie at the k-th key, the first ones in column order.
+// Window sweep (SWEEP): a key u = fp32(s_ij - alpha_i) can only reach the window [lo_j, hi_j]
+// if fp32(s_ij - beta_j) >= T - D, where D = max_j (beta_j - pred(lo_j)) over the columns
+// (pred(lo_j): the largest float whose key is below lo_j), because alpha_i >= vk1 >= T:
+// fp32(s - a) >= L implies s - a > pred(L), so s - beta_j > alpha_i - D. T' = T - D (rounded
+// down) therefore lists every element the sweep can count, and the sweep runs on the list.
+// A row whose list overflows kTprCap entries falls back to the warp-per-row code on its tile
+// row (ranked selection or rounds, and the full sweep of the row).
+namespace qb {
+constexpr int kTprWarps = 5;        // warps (32-row tiles) per CTA, one CTA per SM
+constexpr int kTprCap = 32;         // listed elements per row
+constexpr int kTprPairCap = 3072;   // window pairs buffered per CTA (the rest go straight to the lists)
+}  // namespace qb
+
+template <int NT>
+__host__ __device__ constexpr int tpr_ld() { return 32 * NT + 4; }  // 32 NT / 4 + 1 is odd: consecutive rows' chunks in distinct banks
+template <int NT>
+constexpr size_t tpr_dyn_smem() {
+    return (size_t)qb::kTprWarps * 32 * tpr_ld<NT>() * sizeof(float) + (size_t)qb::kTprWarps * qb::kTprCap * 32;
+}
+
+__device__ __forceinline__ float vmax2(float a, float b) { return fmaxf(a, b); }
+__device__ __forceinline__ float vmin2(float a, float b) { return fminf(a, b); }
+__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) { return max(a, b); }
+__device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b) { return min(a, b); }
+
+// Sorts N values held in registers into descending order (bitonic network, N a power of two).
+template <typename V, int N>
+__device__ __forceinline__ void sort_desc(V (&a)[N]) {
+    constexpr int LOG = N == 32 ? 5 : N == 16 ? 4 : N == 8 ? 3 : N == 4 ? 2 : 1;
+    static_assert((1 << LOG) == N, "a power of two up to 32");
+#pragma unroll
+    for (int ls = 1; ls <= LOG; ++ls)
+#pragma unroll
+        for (int lt = ls - 1; lt >= 0; --lt)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int p = i ^ (1 << lt);
+                if (p > i) {
+                    const V x = a[i], y = a[p];
+                    const V hi = vmax2(x, y), lo = vmin2(x, y);
+                    if ((i & (1 << ls)) == 0) { a[i] = hi; a[p] = lo; }
+                    else { a[i] = lo; a[p] = hi; }
+                }
+            }
+}
+
+// a[idx] for a register array: a tree of selects on the bits of idx (no local-memory copy).
+template <typename V>
+__device__ __forceinline__ V value_at(const V (&a)[32], int idx) {
+    V b[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) b[q] = (idx & 16) ? a[q + 16] : a[q];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) b[q] = (idx & 8) ? b[q + 8] : b[q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) b[q] = (idx & 4) ? b[q + 4] : b[q];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) b[q] = (idx & 2) ? b[q + 2] : b[q];
+    return (idx & 1) ? b[1] : b[0];
+}
+
+// One (column, key) pair inside the window, from the lanes in `mask` (warp-aggregated reservation
+// in the CTA buffer; the pairs that do not fit go straight to the column's global list).
+__device__ __forceinline__ void tpr_append(bool in, uint32_t j, uint32_t key, uint2* pairs, unsigned* npairs,
+                                           const RowSweep& sw) {
+    const unsigned full = __activemask();
+    const unsigned b = __ballot_sync(full, in);
+    if (!b) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(b) - 1;
+    unsigned base = 0;
+    if (lane == leader) base = atomicAdd(npairs, (unsigned)__popc(b));
+    base = __shfl_sync(full, base, leader);
+    if (in) {
+        const unsigned pos = base + (unsigned)__popc(b & ((1u << lane) - 1u));
+        if (pos < (unsigned)qb::kTprPairCap) {
+            pairs[pos] = make_uint2(j, key);
+        } else {
+            const uint32_t g = atomicAdd(&sw.g_ncand[j], 1u);
+            if (g < (uint32_t)qb::kGCap) sw.g_cand[(int64_t)j * qb::kGCap + g] = key;
+        }
+    }
+}
+
+template <int NT, bool TRANS, bool SWEEP>
+__global__ void __launch_bounds__(qb::kTprWarps * 32, 1)
+qb_row_tpr_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
+                  float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
+                  int32_t* __restrict__ status, int tie_slot, int skip_if_done, float* __restrict__ sT, int bulk,
+                  RowSweep sw) {
+    if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
+    constexpr int W = qb::kTprWarps, LD = tpr_ld<NT>(), NC = 32 * NT, CAP = qb::kTprCap;
+    extern __shared__ __align__(128) float tiles[];  // [W][32][LD], then the lists [W][CAP][32] bytes
+    unsigned char* lists = reinterpret_cast<unsigned char*>(tiles + (size_t)W * 32 * LD);
+    __shared__ __align__(16) float bsh[NC];                        // beta, 0 past n
+    __shared__ uint32_t lo_s[SWEEP ? NC : 1], hi_s[SWEEP ? NC : 1];  // the sweep's windows
+    __shared__ int cnt[kMaxExperts];
+    __shared__ uint32_t above_s[SWEEP ? kMaxExperts : 1];
+    __shared__ uint2 pairs[SWEEP ? qb::kTprPairCap : 1];
+    __shared__ uint32_t scnt[SWEEP ? kMaxExperts : 1], sbase[SWEEP ? kMaxExperts : 1];
+    __shared__ unsigned char sfull[SWEEP ? kMaxExperts : 1];
+    __shared__ __align__(8) uint64_t bar[W];
+    __shared__ uint32_t f_key[W * 32];
+    __shared__ int f_j[W * 32];
+    __shared__ float f_v[W * 32];
+    __shared__ unsigned npairs;
+    __shared__ int nties, abort_flag;
+    __shared__ unsigned long long dmax_bits;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned full = 0xffffffffu;
+    float* tile = tiles + (size_t)warp * 32 * LD;
+    unsigned char* list = lists + (size_t)warp * CAP * 32;
+
+    for (int j = tid; j < NC; j += blockDim.x) {
+        bsh[j] = j < n ? beta[j] : 0.f;
+        if (SWEEP) {
+            uint32_t lo = 0xffffffffu, hi = 0xffffffffu;  // padding columns: no key reaches them
+            if (j < n) {
+                const uint32_t pk = float_key(beta[j]);
+                uint32_t w = sw.win[j] ? sw.win[j] : qb::kWinDefault;
+                if (w > qb::kWinSweep) w = qb::kWinSweep;
+                lo = pk > w ? pk - w : 0u;
+                hi = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
+            }
+            lo_s[j] = lo;
+            hi_s[j] = hi;
+        }
+    }
+    for (int j = tid; j < kMaxExperts; j += blockDim.x) {
+        cnt[j] = 0;
+        if (SWEEP) { above_s[j] = 0; scnt[j] = 0; sfull[j] = 0; }
+    }
+    // tile columns n .. NC - 1 hold -inf for good (the row copies write columns below n only)
+    if (n < NC)
+        for (int q = tid; q < W * 32 * (NC - n); q += blockDim.x)
+            tiles[(q / (NC - n)) * LD + n + q % (NC - n)] = -INFINITY;
+    if (tid == 0) { npairs = 0; nties = 0; abort_flag = 0; dmax_bits = 0ull; }
+    if (lane == 0) ptx::mbar_init(&bar[warp], 1);
+    ptx::fence_barrier_init();
+    __syncthreads();
+    double dmax = 0.0;
+    if (SWEEP) {
+        double d = 0.0;
+        for (int j = tid; j < n; j += blockDim.x) {
+            const uint32_t lo = lo_s[j];
+            double dj;
+            if (lo <= 0x00800000u) {
+                dj = INFINITY;  // the window reaches -inf: every element is listed
+            } else {
+                uint32_t pk = lo - 1u;
+                if (pk == 0x7fffffffu) pk = 0x7ffffffeu;  // below +0 the next float is -denorm_min
+                dj = __dsub_ru((double)bsh[j], (double)key_float(pk));
+            }
+            d = fmax(d, dj);
+        }
+        atomicMax(&dmax_bits, (unsigned long long)__double_as_longlong(d));  // d >= 0: the bits order like the values
+        __syncthreads();
+        dmax = __longlong_as_double((long long)dmax_bits);
+    }
+
+    const int64_t ntiles = (m + 31) / 32;
+    const int64_t nw = (int64_t)gridDim.x * W;
+    const int64_t gw = (int64_t)warp * gridDim.x + blockIdx.x;  // tiles b, b + G, ... spread over the CTA's warps
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t used = 0, issued = 0;  // row copies consumed / issued into this warp's tile
+    const int ngroups = (n + NT - 1) / NT;
+    const uint32_t gvalid = ngroups >= 32 ? 0xffffffffu : ((1u << ngroups) - 1u);
+
+    auto issue = [&](int64_t t) {
+        const int64_t i0 = t * 32;
+        const int rows = (int)min((int64_t)32, m - i0);
+        if (lane == 0) ptx::mbar_expect_tx(&bar[warp], (uint32_t)rows * (uint32_t)n * 4u);
+        __syncwarp();
+        if (lane < rows) ptx::bulk_load(tile + lane * LD, s + (i0 + lane) * n, (uint32_t)n * 4u, &bar[warp]);
+        ++issued;
+    };
+    if (bulk && gw < ntiles) issue(gw);
+
+    for (int64_t t = gw; t < ntiles; t += nw) {
+        const int64_t i0 = t * 32;
+        const int rows = (int)min((int64_t)32, m - i0);
+        if (bulk) {
+            const bool ok = ptx::mbar_wait(&bar[warp], used & 1u, &abort_flag);
+            if (!__all_sync(full, ok)) break;
+            ++used;
+        } else {
+            for (int r = 0; r < rows; ++r)
+                for (int q = lane; q < n; q += 32) tile[r * LD + q] = s[(i0 + r) * n + q];
+            __syncwarp();
+        }
+        if (__any_sync(full, *(volatile int*)&abort_flag != 0)) break;
+        const bool valid = lane < rows;
+        const int64_t i = i0 + lane;
+        const float* row = tile + lane * LD;
+
+        if (TRANS && valid) {
+            for (int c = 0; c < NC / 4; ++c) {
+                const float4 sv = *reinterpret_cast<const float4*>(row + 4 * c);
+                const float e4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * c + e < n) sT[(int64_t)(4 * c + e) * m + i] = e4[e];
+            }
+        }
+
+        // 1. group maxima of v = fp32(s - beta)
+        float gm[32];
+#pragma unroll
+        for (int g = 0; g < 32; ++g) gm[g] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < NC / 4; ++c) {
+            const float4 sv = *reinterpret_cast<const float4*>(row + 4 * c);
+            const float4 bv = *reinterpret_cast<const float4*>(bsh + 4 * c);
+            const float v0 = __fsub_rn(sv.x, bv.x), v1 = __fsub_rn(sv.y, bv.y), v2 = __fsub_rn(sv.z, bv.z),
+                        v3 = __fsub_rn(sv.w, bv.w);
+            if constexpr (NT >= 4) {
+                gm[4 * c / NT] = fmaxf(gm[4 * c / NT], fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
+            } else if constexpr (NT == 2) {
+                gm[2 * c] = fmaxf(gm[2 * c], fmaxf(v0, v1));
+                gm[2 * c + 1] = fmaxf(gm[2 * c + 1], fmaxf(v2, v3));
+            } else {
+                gm[4 * c] = v0; gm[4 * c + 1] = v1; gm[4 * c + 2] = v2; gm[4 * c + 3] = v3;
+            }
+        }
+        // 2. T and the listing threshold
+        float T, Tl;
+        uint32_t gbits = 0;
+        {
+            float srt[32];
+#pragma unroll
+            for (int g = 0; g < 32; ++g) srt[g] = gm[g];
+            sort_desc(srt);
+            T = value_at(srt, k);
+            Tl = SWEEP ? __double2float_rd(__dsub_rd((double)T, dmax)) : T;
+#pragma unroll
+            for (int g = 0; g < 32; ++g) gbits |= (gm[g] >= Tl ? 1u : 0u) << g;
+            gbits &= gvalid;
+        }
+        // 3. the listed elements, ascending column
+        int nc = 0;
+        {
+            uint32_t bits = valid ? gbits : 0u;
+            while (bits) {
+                const int g = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                const int j0 = g * NT;
+                float sv[NT], bv[NT];
+                if constexpr (NT >= 4) {
+#pragma unroll
+                    for (int e = 0; e < NT; e += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(row + j0 + e);
+                        const float4 b4 = *reinterpret_cast<const float4*>(bsh + j0 + e);
+                        sv[e] = a4.x; sv[e + 1] = a4.y; sv[e + 2] = a4.z; sv[e + 3] = a4.w;
+                        bv[e] = b4.x; bv[e + 1] = b4.y; bv[e + 2] = b4.z; bv[e + 3] = b4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NT; ++e) { sv[e] = row[j0 + e]; bv[e] = bsh[j0 + e]; }
+                }
+#pragma unroll
+                for (int e = 0; e < NT; ++e) {
+                    const bool c = (j0 + e < n) && __fsub_rn(sv[e], bv[e]) >= Tl;
+                    if (c) {
+                        if (nc < CAP) list[nc * 32 + lane] = (unsigned char)(j0 + e);
+                        ++nc;
+                    }
+                }
+            }
+        }
+        const bool ovf = valid && nc > CAP;
+        const bool mine = valid && !ovf;
+        const int pmax = __reduce_max_sync(full, mine ? nc : 0);
+        // 4. keys of the listed elements with v >= T, sorted
+        uint32_t kk[CAP];
+#pragma unroll
+        for (int p = 0; p < CAP; ++p) {
+            uint32_t key = 0u;
+            if (p < pmax && p < nc && mine) {
+                const int j = list[p * 32 + lane];
+                const float v = __fsub_rn(row[j], bsh[j]);
+                key = v >= T ? float_key_nz(v) : 0u;
+            }
+            kk[p] = key;
+        }
+        uint32_t KK = 0, KK1 = 0;
+        int A = 0;
+        {
+            uint32_t srt[CAP];
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) srt[p] = kk[p];
+            sort_desc(srt);
+            KK = value_at(srt, k - 1);
+            KK1 = value_at(srt, k);
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) A += srt[p] > KK ? 1 : 0;
+        }
+        const float vk = key_float(KK), vk1 = key_float(KK1);
+        const float a = qb_threshold(vk, vk1, rule);
+        if (mine) {
+            alpha[i] = a;
+            int np = 0, eq = 0;
+            const int need_eq = k - A;
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) {
+                if (p < pmax) {
+                    const uint32_t key = kk[p];
+                    const bool pick = key > KK || (key == KK && eq < need_eq);
+                    eq += key == KK ? 1 : 0;
+                    if (pick) {
+                        const int j = list[p * 32 + lane];
+                        topk_idx[i * k + np] = j;
+                        atomicAdd(&cnt[j], 1);
+                        ++np;
+                    }
+                }
+            }
+        }
+        {
+            const unsigned tb = __ballot_sync(full, mine && vk == vk1);
+            if (lane == 0 && tb) atomicAdd(&nties, __popc(tb));
+        }
+        if (SWEEP) {
+            // the sweep on the list: keys above the window counted, keys inside it appended
+            for (int p = 0; p < pmax; ++p) {
+                bool in = false;
+                uint32_t j = 0, key = 0;
+                if (mine && p < nc) {
+                    j = list[p * 32 + lane];
+                    key = float_key_nz(__fsub_rn(row[j], a));
+                    if (key > hi_s[j]) atomicAdd(&above_s[j], 1u);
+                    else in = key >= lo_s[j];
+                }
+                tpr_append(in, j, key, pairs, &npairs, sw);
+            }
+        }
+        // rows whose list overflowed: the warp-per-row code on the tile row
+        uint32_t ob = __ballot_sync(full, ovf);
+        while (ob) {
+            const int r = __ffs(ob) - 1;
+            ob &= ob - 1u;
+            const int64_t ir = i0 + r;
+            const float* rw = tile + r * LD;
+            float v[NT];
+            uint32_t key[NT];
+#pragma unroll
+            for (int q = 0; q < NT; ++q) {
+                const int j = lane + 32 * q;
+                const bool ok = j < n;
+                v[q] = ok ? __fsub_rn(rw[j], bsh[j]) : 0.f;
+                key[q] = ok ? float_key(v[q]) : 0u;
+            }
+            float wk, wk1;
+            if (!(k < 32 && k < n && row_topk_ranked<NT>(key, v, k, ir, f_key + warp * 32, f_j + warp * 32,
+                                                          f_v + warp * 32, topk_idx, cnt, wk, wk1))) {
+                uint32_t taken;
+                row_topk_rounds<NT>(key, v, n, k, taken, wk, wk1);
+                int pos = 0;
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const bool bit = (taken >> q) & 1u;
+                    const uint32_t mask = __ballot_sync(full, bit);
+                    if (bit) {
+                        topk_idx[ir * k + pos + __popc(mask & lt)] = lane + 32 * q;
+                        atomicAdd(&cnt[lane + 32 * q], 1);
+                    }
+                    pos += __popc(mask);
+                }
+            }
+            const float wa = qb_threshold(wk, wk1, rule);
+            if (lane == 0) {
+                alpha[ir] = wa;
+                if (wk == wk1) atomicAdd(&nties, 1);
+            }
+            if (SWEEP) {
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const int j = lane + 32 * q;
+                    bool in = false;
+                    uint32_t uk = 0;
+                    if (j < n) {
+                        uk = float_key_nz(__fsub_rn(rw[j], wa));
+                        if (uk > hi_s[j]) atomicAdd(&above_s[j], 1u);
+                        else in = uk >= lo_s[j];
+                    }
+                    tpr_append(in, (uint32_t)j, uk, pairs, &npairs, sw);
+                }
+            }
+        }
+        __syncwarp();  // every lane is done with the tile
+        const int64_t tn = t + nw;
+        if (bulk && tn < ntiles) {
+            ptx::fence_proxy_async_shared();
+            issue(tn);
+        }
+    }
+    __syncthreads();
+    if (abort_flag) {
+        // a wait gave up: let this warp's copies still in flight land before the CTA exits (bounded)
+        if (lane == 0)
+            for (uint32_t c = used; c < issued; ++c)
+                for (int it = 0; it < (1 << 22) && !ptx::mbar_try_wait(&bar[warp], c & 1u); ++it) {
+                }
+        if (tid == 0) status[qb::kStError] = 1;
+        return;
+    }
+    for (int j = tid; j < n; j += blockDim.x)
+        if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
+    if (tid == 0 && nties) atomicAdd(&status[tie_slot], nties);
+    if (SWEEP) {
+        for (int j = tid; j < n; j += blockDim.x)
+            if (above_s[j]) atomicAdd(&sw.g_above[j], above_s[j]);
+        if (npairs) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw, (unsigned)qb::kTprPairCap);
     }
 }
 
@@ -1455,11 +1888,43 @@ static void launch_row_tt(const float* s, int64_t m, int n, int k, const float* 
         s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk, sw);
 }
 
+template <int NT, bool TRANS, bool SWEEP>
+static void launch_row_tpr_tt(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
+                              int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
+                              const RowSweep& sw, cudaStream_t stream) {
+    const size_t smem = tpr_dyn_smem<NT>();
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(qb_row_tpr_kernel<NT, TRANS, SWEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        attr = true;
+    }
+    const int64_t ntiles = (m + 31) / 32;
+    int64_t blocks = (ntiles + qb::kTprWarps - 1) / qb::kTprWarps;
+    if (blocks > kNumSMs) blocks = kNumSMs;
+    if (blocks < 1) blocks = 1;
+    // one bulk copy per row: a 16-byte aligned s and rows of a multiple of 16 bytes
+    const int bulk = (reinterpret_cast<uintptr_t>(s) & 15) == 0 && n % 4 == 0;
+    qb_row_tpr_kernel<NT, TRANS, SWEEP><<<(unsigned)blocks, qb::kTprWarps * 32, smem, stream>>>(
+        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk, sw);
+}
+
 template <int NT>
 static void launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                          int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
                          const RowSweep* sw, cudaStream_t stream) {
     const RowSweep none{nullptr, nullptr, nullptr, nullptr};
+    if (k >= 1 && k + 1 <= (n + NT - 1) / NT) {
+        // thread-per-row selection: the (k+1)-th largest of the 32 column-group maxima exists
+        if (sw) {
+            if (sT) launch_row_tpr_tt<NT, true, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
+            else launch_row_tpr_tt<NT, false, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
+        } else {
+            if (sT) launch_row_tpr_tt<NT, true, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
+            else launch_row_tpr_tt<NT, false, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
+        }
+        return;
+    }
     if (sw) {
         if (sT) launch_row_tt<NT, true, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
         else launch_row_tt<NT, false, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);

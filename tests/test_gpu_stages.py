@@ -514,6 +514,40 @@ def test_balance_misaligned_scores(m, n, k):
     assert (host(idx) == i_ref).all()
 
 
+@pytest.mark.parametrize("m,n,k,kind", [(8192, 256, 8, "tied_rows"), (4040, 101, 5, "odd_n"),
+                                        (4096, 256, 40, "large_k"), (1024, 64, 40, "large_k"),
+                                        (6048, 96, 23, "k_at_groups"), (2016, 32, 31, "k_at_groups")])
+def test_balance_row_pass_forms(m, n, k, kind):
+    # the row pass's two forms: the thread-per-row selection (k + 1 <= the number of column groups)
+    # with its warp-per-row fallback for rows whose listed elements overflow (every 7th row constant,
+    # every 5th on a coarse grid: many equal values), rows of n not a multiple of 4 (plain loads),
+    # and the warp-per-row kernel when k + 1 exceeds the groups; chained STEPs and a SOLVE
+    s = W.make_qb_scores(m, n, seed=m + n + k)
+    if kind == "tied_rows":
+        s[3::7] = np.float32(0.5)
+        s[1::5] = np.round(s[1::5] * 2) / 2
+    b = np.zeros(n, dtype=np.float32)
+    for _ in range(3):
+        i_ref, b_ref, info_ref, _ = oracle.balance_assign(s, k, beta=b, mode=oracle.QB_STEP)
+        idx, beta, info = lb.moe_balance_assign(dev(s), k, beta=dev(b), mode=lb.MOE_QB_STEP)
+        torch.cuda.synchronize()
+        assert (host(idx) == i_ref).all()
+        assert (host(beta) == b_ref).all()
+        assert (host(info) == info_ref).all()
+        b = b_ref
+    if kind == "tied_rows":
+        # whole rows of equal values give the exact finish zero-cost cycles between experts, where
+        # its path reconstruction is not defined: STEPs only
+        return
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=10)
+    assert rc == oracle.OK
+    idx, beta, info = lb.moe_balance_assign(dev(s), k, mode=lb.MOE_QB_SOLVE, max_iters=10)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
+
+
 @pytest.mark.parametrize("m,n,k,seed", [(1024, 8, 2, 0), (2048, 16, 2, 2), (4096, 32, 4, 1), (512, 4, 1, 0)])
 def test_balance_solve_converges_inside_a_batch(m, n, k, seed):
     # mild skew: QB alone reaches exact balance after 6..45 beta updates (no repair), so the
