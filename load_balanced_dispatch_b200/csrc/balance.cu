@@ -766,17 +766,45 @@ qb_row_tpr_kernel(const float* __restrict__ s, int64_t m, int n, int k, const fl
             if (lane == 0 && tb) atomicAdd(&nties, __popc(tb));
         }
         if (SWEEP) {
-            // the sweep on the list: keys above the window counted, keys inside it appended
-            for (int p = 0; p < pmax; ++p) {
-                bool in = false;
-                uint32_t j = 0, key = 0;
-                if (mine && p < nc) {
-                    j = list[p * 32 + lane];
-                    key = float_key_nz(__fsub_rn(row[j], a));
-                    if (key > hi_s[j]) atomicAdd(&above_s[j], 1u);
-                    else in = key >= lo_s[j];
+            // the sweep on the list: keys above the window counted, keys inside it appended (one
+            // reservation in the CTA buffer per warp and tile)
+            uint32_t inmask = 0;
+            int nin = 0;
+            if (mine)
+                for (int p = 0; p < nc; ++p) {
+                    const int j = list[p * 32 + lane];
+                    const uint32_t key = float_key_nz(__fsub_rn(row[j], a));
+                    if (key > hi_s[j]) {
+                        atomicAdd(&above_s[j], 1u);
+                    } else if (key >= lo_s[j]) {
+                        inmask |= 1u << p;
+                        ++nin;
+                    }
                 }
-                tpr_append(in, j, key, pairs, &npairs, sw);
+            int incl = nin;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(full, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int total = __shfl_sync(full, incl, 31);
+            if (total) {
+                unsigned base = 0;
+                if (lane == 31) base = atomicAdd(&npairs, (unsigned)total);
+                unsigned pos = __shfl_sync(full, base, 31) + (unsigned)(incl - nin);
+                while (inmask) {
+                    const int p = __ffs(inmask) - 1;
+                    inmask &= inmask - 1u;
+                    const uint32_t j = list[p * 32 + lane];
+                    const uint32_t key = float_key_nz(__fsub_rn(row[j], a));
+                    if (pos < (unsigned)qb::kTprPairCap) {
+                        pairs[pos] = make_uint2(j, key);
+                    } else {
+                        const uint32_t g = atomicAdd(&sw.g_ncand[j], 1u);
+                        if (g < (uint32_t)qb::kGCap) sw.g_cand[(int64_t)j * qb::kGCap + g] = key;
+                    }
+                    ++pos;
+                }
             }
         }
         // rows whose list overflowed: the warp-per-row code on the tile row
@@ -852,6 +880,365 @@ qb_row_tpr_kernel(const float* __restrict__ s, int64_t m, int n, int k, const fl
     for (int j = tid; j < n; j += blockDim.x)
         if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
     if (tid == 0 && nties) atomicAdd(&status[tie_slot], nties);
+    if (SWEEP) {
+        for (int j = tid; j < n; j += blockDim.x)
+            if (above_s[j]) atomicAdd(&sw.g_above[j], above_s[j]);
+        if (npairs) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw, (unsigned)qb::kTprPairCap);
+    }
+}
+
+// The same selection without a shared-memory copy of the rows (the passes that write no
+// transposed copy): a warp reads its 32 rows from global memory with each lane holding one
+// column group of a row (coalesced), forms the group maxima with beta in registers and hands
+// them to the row threads through a small shared array; the row threads then read the groups
+// that reach T' of their own row again (from L2) and keep the listed elements' scores in their
+// shared list. Sixteen warps per SM instead of five: the selection is latency-bound, and the
+// rows no longer occupy shared memory.
+namespace qb {
+constexpr int kTpr2Warps = 16;
+}  // namespace qb
+
+constexpr size_t tpr2_dyn_smem() {
+    return (size_t)qb::kTpr2Warps * ((32 * 33 + qb::kTprCap * 32) * sizeof(float) + qb::kTprCap * 32);
+}
+
+// NT consecutive scores from p (the first `valid` of them exist; the rest read as -inf)
+template <int NT>
+__device__ __forceinline__ void load_group(const float* p, bool vec, int valid, float (&out)[NT]) {
+    if (vec && valid >= NT) {
+        if constexpr (NT >= 4) {
+#pragma unroll
+            for (int e = 0; e < NT; e += 4) {
+                const float4 q = __ldg(reinterpret_cast<const float4*>(p + e));
+                out[e] = q.x; out[e + 1] = q.y; out[e + 2] = q.z; out[e + 3] = q.w;
+            }
+            return;
+        } else if constexpr (NT == 2) {
+            const float2 q = __ldg(reinterpret_cast<const float2*>(p));
+            out[0] = q.x; out[1] = q.y;
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < NT; ++e) out[e] = e < valid ? __ldg(p + e) : -INFINITY;
+}
+
+// SIGN (SignSGD step): also count_j = #{i : fp32(s_ij - alpha_i) > beta_j}. Such an element has
+// s_ij - beta_j > alpha_i >= T (fp32(x) > beta_j implies x > beta_j), so v_ij >= T: it is listed.
+template <int NT, bool SWEEP, bool SIGN>
+__global__ void __launch_bounds__(qb::kTpr2Warps * 32, 1)
+qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const float* __restrict__ beta, int rule,
+                   float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
+                   int32_t* __restrict__ status, int tie_slot, int skip_if_done, RowSweep sw,
+                   int32_t* __restrict__ sign_counts) {
+    if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
+    constexpr int W = qb::kTpr2Warps, NC = 32 * NT, CAP = qb::kTprCap, GS = 33;
+    extern __shared__ __align__(16) float dsm[];  // per warp: [32][33] group maxima, [CAP][32] listed scores; then [W][CAP][32] columns
+    __shared__ __align__(16) float bsh[NC];
+    __shared__ uint32_t lo_s[SWEEP ? NC : 1], hi_s[SWEEP ? NC : 1];
+    __shared__ int cnt[kMaxExperts];
+    __shared__ uint32_t above_s[(SWEEP || SIGN) ? kMaxExperts : 1];  // keys above the window, or the sign counts
+    __shared__ uint2 pairs[SWEEP ? qb::kTprPairCap : 1];
+    __shared__ uint32_t scnt[SWEEP ? kMaxExperts : 1], sbase[SWEEP ? kMaxExperts : 1];
+    __shared__ unsigned char sfull[SWEEP ? kMaxExperts : 1];
+    __shared__ uint32_t f_key[W * 32];
+    __shared__ int f_j[W * 32];
+    __shared__ float f_v[W * 32];
+    __shared__ unsigned npairs;
+    __shared__ int nties;
+    __shared__ unsigned long long dmax_bits;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned full = 0xffffffffu;
+    float* gmx = dsm + (size_t)warp * (32 * GS + CAP * 32);
+    float* ls = gmx + 32 * GS;
+    unsigned char* lj = reinterpret_cast<unsigned char*>(dsm + (size_t)W * (32 * GS + CAP * 32)) + (size_t)warp * CAP * 32;
+
+    for (int j = tid; j < NC; j += blockDim.x) {
+        bsh[j] = j < n ? beta[j] : 0.f;
+        if (SWEEP) {
+            uint32_t lo = 0xffffffffu, hi = 0xffffffffu;
+            if (j < n) {
+                const uint32_t pk = float_key(beta[j]);
+                uint32_t w = sw.win[j] ? sw.win[j] : qb::kWinDefault;
+                if (w > qb::kWinSweep) w = qb::kWinSweep;
+                lo = pk > w ? pk - w : 0u;
+                hi = pk < 0xffffffffu - w ? pk + w : 0xffffffffu;
+            }
+            lo_s[j] = lo;
+            hi_s[j] = hi;
+        }
+    }
+    for (int j = tid; j < kMaxExperts; j += blockDim.x) {
+        cnt[j] = 0;
+        if (SWEEP || SIGN) above_s[j] = 0;
+        if (SWEEP) { scnt[j] = 0; sfull[j] = 0; }
+    }
+    if (tid == 0) { npairs = 0; nties = 0; dmax_bits = 0ull; }
+    __syncthreads();
+    double dmax = 0.0;
+    if (SWEEP) {
+        double d = 0.0;
+        for (int j = tid; j < n; j += blockDim.x) {
+            const uint32_t lo = lo_s[j];
+            double dj;
+            if (lo <= 0x00800000u) {
+                dj = INFINITY;
+            } else {
+                uint32_t pk = lo - 1u;
+                if (pk == 0x7fffffffu) pk = 0x7ffffffeu;
+                dj = __dsub_ru((double)bsh[j], (double)key_float(pk));
+            }
+            d = fmax(d, dj);
+        }
+        atomicMax(&dmax_bits, (unsigned long long)__double_as_longlong(d));
+        __syncthreads();
+        dmax = __longlong_as_double((long long)dmax_bits);
+    }
+
+    const int64_t ntiles = (m + 31) / 32;
+    const int64_t nw = (int64_t)gridDim.x * W;
+    const int64_t gw = (int64_t)warp * gridDim.x + blockIdx.x;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int ngroups = (n + NT - 1) / NT;
+    const uint32_t gvalid = ngroups >= 32 ? 0xffffffffu : ((1u << ngroups) - 1u);
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0 && n % 4 == 0;
+    // this lane's column group in the coalesced pass, and its beta
+    const int gj0 = lane * NT;
+    float bl[NT];
+#pragma unroll
+    for (int e = 0; e < NT; ++e) bl[e] = bsh[gj0 + e];
+
+    for (int64_t t = gw; t < ntiles; t += nw) {
+        const int64_t i0 = t * 32;
+        const int rows = (int)min((int64_t)32, m - i0);
+        // 1. group maxima, 8 rows per batch (lane = column group)
+#pragma unroll 1
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+            float sv[8][NT];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                if (r0 + rr < rows && gj0 < n) {
+                    load_group<NT>(s + (i0 + r0 + rr) * n + gj0, vec, n - gj0, sv[rr]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NT; ++e) sv[rr][e] = -INFINITY;
+                }
+            }
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                float g = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < NT; ++e) g = fmaxf(g, __fsub_rn(sv[rr][e], bl[e]));
+                gmx[(r0 + rr) * GS + lane] = g;
+            }
+        }
+        __syncwarp();
+        const bool valid = lane < rows;
+        const int64_t i = i0 + lane;
+        // 2. T and the listing threshold
+        float T, Tl;
+        uint32_t gbits = 0;
+        {
+            float srt[32];
+#pragma unroll
+            for (int g = 0; g < 32; ++g) srt[g] = gmx[lane * GS + g];
+            sort_desc(srt);
+            T = value_at(srt, k);
+            Tl = SWEEP ? __double2float_rd(__dsub_rd((double)T, dmax)) : T;
+#pragma unroll
+            for (int g = 0; g < 32; ++g) gbits |= (gmx[lane * GS + g] >= Tl ? 1u : 0u) << g;
+            gbits &= gvalid;
+        }
+        // 3. the listed elements of the groups reaching T', two groups' loads in flight
+        int nc = 0;
+        {
+            const float* rowp = s + i * n;
+            uint32_t bits = valid ? gbits : 0u;
+            while (bits) {
+                const int g1 = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                const int g2 = bits ? __ffs(bits) - 1 : -1;
+                if (bits) bits &= bits - 1u;
+                float s1[NT], s2[NT];
+                load_group<NT>(rowp + g1 * NT, vec, n - g1 * NT, s1);
+                if (g2 >= 0) load_group<NT>(rowp + g2 * NT, vec, n - g2 * NT, s2);
+#pragma unroll
+                for (int e = 0; e < NT; ++e) {
+                    const int j = g1 * NT + e;
+                    if (j < n && __fsub_rn(s1[e], bsh[j]) >= Tl) {
+                        if (nc < CAP) { ls[nc * 32 + lane] = s1[e]; lj[nc * 32 + lane] = (unsigned char)j; }
+                        ++nc;
+                    }
+                }
+                if (g2 >= 0) {
+#pragma unroll
+                    for (int e = 0; e < NT; ++e) {
+                        const int j = g2 * NT + e;
+                        if (j < n && __fsub_rn(s2[e], bsh[j]) >= Tl) {
+                            if (nc < CAP) { ls[nc * 32 + lane] = s2[e]; lj[nc * 32 + lane] = (unsigned char)j; }
+                            ++nc;
+                        }
+                    }
+                }
+            }
+        }
+        const bool ovf = valid && nc > CAP;
+        const bool mine = valid && !ovf;
+        const int pmax = __reduce_max_sync(full, mine ? nc : 0);
+        // 4. the k-th and (k+1)-th keys of the listed elements with v >= T
+        uint32_t KK = 0, KK1 = 0;
+        int A = 0;
+        {
+            uint32_t kk[CAP];
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) {
+                uint32_t key = 0u;
+                if (p < pmax && p < nc && mine) {
+                    const int j = lj[p * 32 + lane];
+                    const float v = __fsub_rn(ls[p * 32 + lane], bsh[j]);
+                    key = v >= T ? float_key_nz(v) : 0u;
+                }
+                kk[p] = key;
+            }
+            sort_desc(kk);
+            KK = value_at(kk, k - 1);
+            KK1 = value_at(kk, k);
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) A += kk[p] > KK ? 1 : 0;
+        }
+        const float vk = key_float(KK), vk1 = key_float(KK1);
+        const float a = qb_threshold(vk, vk1, rule);
+        if (mine) {
+            alpha[i] = a;
+            int np = 0, eq = 0;
+            const int need_eq = k - A;
+            for (int p = 0; p < nc; ++p) {
+                const int j = lj[p * 32 + lane];
+                const float v = __fsub_rn(ls[p * 32 + lane], bsh[j]);
+                const uint32_t key = v >= T ? float_key_nz(v) : 0u;
+                const bool pick = key > KK || (key == KK && eq < need_eq);
+                eq += key == KK ? 1 : 0;
+                if (pick) {
+                    topk_idx[i * k + np] = j;
+                    atomicAdd(&cnt[j], 1);
+                    ++np;
+                }
+                if (SIGN && key != 0u && __fsub_rn(ls[p * 32 + lane], a) > bsh[j]) atomicAdd(&above_s[j], 1u);
+            }
+        }
+        {
+            const unsigned tb = __ballot_sync(full, mine && vk == vk1);
+            if (lane == 0 && tb) atomicAdd(&nties, __popc(tb));
+        }
+        if (SWEEP) {
+            uint32_t inmask = 0;
+            int nin = 0;
+            if (mine)
+                for (int p = 0; p < nc; ++p) {
+                    const int j = lj[p * 32 + lane];
+                    const uint32_t key = float_key_nz(__fsub_rn(ls[p * 32 + lane], a));
+                    if (key > hi_s[j]) {
+                        atomicAdd(&above_s[j], 1u);
+                    } else if (key >= lo_s[j]) {
+                        inmask |= 1u << p;
+                        ++nin;
+                    }
+                }
+            int incl = nin;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(full, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int total = __shfl_sync(full, incl, 31);
+            if (total) {
+                unsigned base = 0;
+                if (lane == 31) base = atomicAdd(&npairs, (unsigned)total);
+                unsigned pos = __shfl_sync(full, base, 31) + (unsigned)(incl - nin);
+                while (inmask) {
+                    const int p = __ffs(inmask) - 1;
+                    inmask &= inmask - 1u;
+                    const uint32_t j = lj[p * 32 + lane];
+                    const uint32_t key = float_key_nz(__fsub_rn(ls[p * 32 + lane], a));
+                    if (pos < (unsigned)qb::kTprPairCap) {
+                        pairs[pos] = make_uint2(j, key);
+                    } else {
+                        const uint32_t g = atomicAdd(&sw.g_ncand[j], 1u);
+                        if (g < (uint32_t)qb::kGCap) sw.g_cand[(int64_t)j * qb::kGCap + g] = key;
+                    }
+                    ++pos;
+                }
+            }
+        }
+        // rows whose list overflowed: the warp-per-row code, the row read again from global memory
+        uint32_t ob = __ballot_sync(full, ovf);
+        while (ob) {
+            const int r = __ffs(ob) - 1;
+            ob &= ob - 1u;
+            const int64_t ir = i0 + r;
+            const float* rw = s + ir * n;
+            float v[NT];
+            uint32_t key[NT];
+#pragma unroll
+            for (int q = 0; q < NT; ++q) {
+                const int j = lane + 32 * q;
+                const bool ok = j < n;
+                v[q] = ok ? __fsub_rn(__ldg(rw + j), bsh[j]) : 0.f;
+                key[q] = ok ? float_key(v[q]) : 0u;
+            }
+            float wk, wk1;
+            if (!(k < 32 && k < n && row_topk_ranked<NT>(key, v, k, ir, f_key + warp * 32, f_j + warp * 32,
+                                                          f_v + warp * 32, topk_idx, cnt, wk, wk1))) {
+                uint32_t taken;
+                row_topk_rounds<NT>(key, v, n, k, taken, wk, wk1);
+                int pos = 0;
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const bool bit = (taken >> q) & 1u;
+                    const uint32_t mask = __ballot_sync(full, bit);
+                    if (bit) {
+                        topk_idx[ir * k + pos + __popc(mask & lt)] = lane + 32 * q;
+                        atomicAdd(&cnt[lane + 32 * q], 1);
+                    }
+                    pos += __popc(mask);
+                }
+            }
+            const float wa = qb_threshold(wk, wk1, rule);
+            if (lane == 0) {
+                alpha[ir] = wa;
+                if (wk == wk1) atomicAdd(&nties, 1);
+            }
+            if (SIGN) {
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const int j = lane + 32 * q;
+                    if (j < n && __fsub_rn(__ldg(rw + j), wa) > bsh[j]) atomicAdd(&above_s[j], 1u);
+                }
+            }
+            if (SWEEP) {
+#pragma unroll
+                for (int q = 0; q < NT; ++q) {
+                    const int j = lane + 32 * q;
+                    bool in = false;
+                    uint32_t uk = 0;
+                    if (j < n) {
+                        uk = float_key_nz(__fsub_rn(__ldg(rw + j), wa));
+                        if (uk > hi_s[j]) atomicAdd(&above_s[j], 1u);
+                        else in = uk >= lo_s[j];
+                    }
+                    tpr_append(in, (uint32_t)j, uk, pairs, &npairs, sw);
+                }
+            }
+        }
+        __syncwarp();  // the group maxima and lists are rewritten by the next tile
+    }
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x)
+        if (cnt[j]) atomicAdd(&counts[j], cnt[j]);
+    if (tid == 0 && nties) atomicAdd(&status[tie_slot], nties);
+    if (SIGN)
+        for (int j = tid; j < n; j += blockDim.x)
+            if (above_s[j]) atomicAdd(&sign_counts[j], (int)above_s[j]);
     if (SWEEP) {
         for (int j = tid; j < n; j += blockDim.x)
             if (above_s[j]) atomicAdd(&sw.g_above[j], above_s[j]);
@@ -1909,13 +2296,40 @@ static void launch_row_tpr_tt(const float* s, int64_t m, int n, int k, const flo
         s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, bulk, sw);
 }
 
+template <int NT, bool SWEEP, bool SIGN>
+static void launch_row_tpr2_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
+                              int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip,
+                              const RowSweep& sw, int32_t* sign_counts, cudaStream_t stream) {
+    const size_t smem = tpr2_dyn_smem();
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(qb_row_tpr2_kernel<NT, SWEEP, SIGN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        attr = true;
+    }
+    const int64_t ntiles = (m + 31) / 32;
+    int64_t blocks = (ntiles + qb::kTpr2Warps - 1) / qb::kTpr2Warps;
+    if (blocks > kNumSMs) blocks = kNumSMs;
+    if (blocks < 1) blocks = 1;
+    qb_row_tpr2_kernel<NT, SWEEP, SIGN><<<(unsigned)blocks, qb::kTpr2Warps * 32, smem, stream>>>(
+        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sw, sign_counts);
+}
+
+// Returns true when the launched pass also counted sign_counts (then no separate count is needed).
 template <int NT>
-static void launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
+static bool launch_row_t(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                          int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
-                         const RowSweep* sw, cudaStream_t stream) {
+                         const RowSweep* sw, int32_t* sign_counts, cudaStream_t stream) {
     const RowSweep none{nullptr, nullptr, nullptr, nullptr};
     if (k >= 1 && k + 1 <= (n + NT - 1) / NT) {
-        // thread-per-row selection: the (k+1)-th largest of the 32 column-group maxima exists
+        // thread-per-row selection: the (k+1)-th largest of the 32 column-group maxima exists;
+        // without a transposed copy to write, the rows are read from global memory
+        if (!sT) {
+            if (sign_counts) launch_row_tpr2_t<NT, false, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, none, sign_counts, stream);
+            else if (sw) launch_row_tpr2_t<NT, true, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, *sw, nullptr, stream);
+            else launch_row_tpr2_t<NT, false, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, none, nullptr, stream);
+            return sign_counts != nullptr;
+        }
         if (sw) {
             if (sT) launch_row_tpr_tt<NT, true, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
             else launch_row_tpr_tt<NT, false, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
@@ -1923,7 +2337,7 @@ static void launch_row_t(const float* s, int64_t m, int n, int k, const float* b
             if (sT) launch_row_tpr_tt<NT, true, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
             else launch_row_tpr_tt<NT, false, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
         }
-        return;
+        return false;
     }
     if (sw) {
         if (sT) launch_row_tt<NT, true, true>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, *sw, stream);
@@ -1932,17 +2346,20 @@ static void launch_row_t(const float* s, int64_t m, int n, int k, const float* b
         if (sT) launch_row_tt<NT, true, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
         else launch_row_tt<NT, false, false>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, none, stream);
     }
+    return false;
 }
 
 // sT != nullptr: this row pass also writes s transposed into sT (the first pass of a call).
 // sw != nullptr: it also runs the column pass's window sweep on its rows.
-static void launch_row(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
+// sign_counts != nullptr (with sT and sw null): the pass may also count the sign step's
+// indicators; the return value says whether it did.
+static bool launch_row(const float* s, int64_t m, int n, int k, const float* beta, int rule, float* alpha,
                        int32_t* topk_idx, int32_t* counts, int32_t* status, int tie_slot, int skip, float* sT,
-                       const RowSweep* sw, cudaStream_t stream) {
-    if (n <= 32) launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
-    else if (n <= 64) launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
-    else if (n <= 128) launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
-    else launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, stream);
+                       const RowSweep* sw, cudaStream_t stream, int32_t* sign_counts = nullptr) {
+    if (n <= 32) return launch_row_t<1>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, sign_counts, stream);
+    if (n <= 64) return launch_row_t<2>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, sign_counts, stream);
+    if (n <= 128) return launch_row_t<4>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, sign_counts, stream);
+    return launch_row_t<8>(s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sT, sw, sign_counts, stream);
 }
 
 // The column pass's select: one CTA per column (the window sweep ran inside the row pass). sT: s
@@ -2034,14 +2451,15 @@ int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, 
     cudaError_t ce;
     if ((ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * (qb::kStWords + 2 * n), stream)) != cudaSuccess)
         goto fail;
-    launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status, qb::kStTies0, 0, nullptr, nullptr,
-               stream);
     {
+        int32_t* sc = w.counts + n;  // chi counts, separate from the pick counts
+        const bool counted = launch_row(s, m, n, k, beta, rule, w.alpha, topk_idx, w.counts, w.status,
+                                        qb::kStTies0, 0, nullptr, nullptr, stream, sc);
         int64_t blocks = (m + 7) / 8;
         if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
         if (blocks < 1) blocks = 1;
-        int32_t* sc = w.counts + n;  // chi counts, separate from the pick counts
-        if (n <= 32) qb_sign_count_kernel<1><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
+        if (counted) {
+        } else if (n <= 32) qb_sign_count_kernel<1><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
         else if (n <= 64) qb_sign_count_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
         else if (n <= 128) qb_sign_count_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
         else qb_sign_count_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(s, m, n, w.alpha, beta, sc);
