@@ -114,7 +114,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                                          "--format=csv,noheader,nounits", "-lms", "20"], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -139,7 +139,8 @@ class ClockSampler:
                 if len(parts) < 10:
                     continue
                 try:
-                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    whole, _, frac = parts[0].partition(".")
+                    ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + (float("0." + frac) if frac else 0.0)
                     rows.append(dict(ts=ts, sm=float(parts[2]), smax=float(parts[3]), active=parts[5],
                                      hw=parts[6], hwt=parts[7], swt=parts[8], pcap=parts[9]))
                 except Exception:
@@ -147,7 +148,12 @@ class ClockSampler:
         os.unlink(self.path)
         if not rows:
             return None
-        inside = [r for r in rows if self.t0 - 1 <= r["ts"] <= self.t1 + 1] or rows
+        # the samples taken while the timed steps ran (20 ms apart); when the region is shorter than
+        # the sampling interval, the samples nearest to it
+        inside = [r for r in rows if self.t0 - 0.02 <= r["ts"] <= self.t1 + 0.02]
+        if not inside:
+            mid = 0.5 * (self.t0 + self.t1)
+            inside = sorted(rows, key=lambda r: abs(r["ts"] - mid))[:3]
         load = [r for r in inside if r["sm"] > 0.5 * r["smax"]] or inside
         reasons = set()
         for r in inside:
