@@ -10,10 +10,10 @@
 // segment):
 //   count+scan -- per-chunk expert histogram (shared-memory integer atomics);
 //             the last CTA to finish (ticket after a fence) runs the scan:
-//             thread e walks the chunks of every segment in order: chunk
-//             prefix within its segment, routed/kept counts, the expert
-//             offsets (block exclusive scan over e) and each (segment,
-//             expert) base row;
+//             chunk prefixes within each segment, routed/kept counts, the
+//             expert offsets (block exclusive scan over e) and each (segment,
+//             expert) base row -- a thread per (segment, expert) pair when
+//             they fit, else groups of threads walking the segments in order;
 //   assign -- per chunk, a stable in-order rank for every assignment
 //             (warp __match_any_sync groups + per-warp running counters in
 //             shared memory, warps owning consecutive sub-ranges), then
@@ -151,6 +151,59 @@ __device__ __forceinline__ void cap_scan_body(const int32_t* hist, int n, int64_
     if (tid == 0) expert_offsets[n] = (int32_t)total;
 }
 
+// The same scan with one thread per (segment, expert) pair, when the pairs fit in shared memory
+// and a segment has at most kPairChunks chunks: each thread loads all of its pair's chunk counts
+// at once and writes the pair's prefixes in chunk order (one round of L2 latency instead of one
+// per segment), then thread e adds expert e's kept totals over the segments in segment order.
+namespace cap {
+constexpr int kPairCap = 4096;
+constexpr int kPairChunks = 32;
+}
+__device__ __forceinline__ void cap_scan_pairs(const int32_t* hist, int n, int64_t nseg, int64_t cps,
+                                               int32_t capacity, int32_t* __restrict__ prefix,
+                                               int32_t* __restrict__ seg_base, int32_t* __restrict__ expert_offsets,
+                                               int32_t* __restrict__ routed_count, int32_t* __restrict__ kept_count) {
+    __shared__ int32_t kept_sh[cap::kPairCap];
+    __shared__ int64_t sh[cap::kThreads];
+    const int tid = threadIdx.x;
+    const int64_t npairs = nseg * n;
+    for (int64_t pr = tid; pr < npairs; pr += blockDim.x) {
+        const int64_t s = pr / n;
+        const int e = (int)(pr - s * n);
+        const int32_t* hs = hist + s * cps * n + e;
+        int32_t h[cap::kPairChunks];
+#pragma unroll
+        for (int c = 0; c < cap::kPairChunks; ++c) h[c] = c < cps ? __ldcg(hs + (int64_t)c * n) : 0;
+        int32_t* ps = prefix + s * cps * n + e;
+        int32_t run = 0;
+#pragma unroll
+        for (int c = 0; c < cap::kPairChunks; ++c)
+            if (c < cps) {
+                ps[(int64_t)c * n] = run;
+                run += h[c];
+            }
+        const int32_t kept = run < capacity ? run : capacity;
+        routed_count[pr] = run;
+        kept_count[pr] = kept;
+        kept_sh[pr] = kept;
+    }
+    __syncthreads();
+    int64_t ktot = 0;
+    if (tid < n)
+        for (int64_t s = 0; s < nseg; ++s) ktot += kept_sh[s * n + tid];
+    int64_t total;
+    const int64_t off = block_exclusive_scan(tid < n ? ktot : 0, sh, total);
+    if (tid < n) {
+        expert_offsets[tid] = (int32_t)off;
+        int64_t base = off;
+        for (int64_t s = 0; s < nseg; ++s) {
+            seg_base[s * n + tid] = (int32_t)base;
+            base += kept_sh[s * n + tid];
+        }
+    }
+    if (tid == 0) expert_offsets[n] = (int32_t)total;
+}
+
 // Per-chunk expert histogram (shared-memory integer atomics); the last CTA to finish (a ticket
 // taken after a fence) then runs the scan over all chunks.
 __global__ void __launch_bounds__(cap::kThreads)
@@ -180,7 +233,10 @@ cap_count_scan_kernel(const int32_t* __restrict__ idx, int k, int n, int64_t seg
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    cap_scan_body(hist, n, nseg, cps, capacity, prefix, seg_base, expert_offsets, routed_count, kept_count);
+    if (nseg * n <= cap::kPairCap && cps <= cap::kPairChunks)
+        cap_scan_pairs(hist, n, nseg, cps, capacity, prefix, seg_base, expert_offsets, routed_count, kept_count);
+    else
+        cap_scan_body(hist, n, nseg, cps, capacity, prefix, seg_base, expert_offsets, routed_count, kept_count);
 }
 
 __global__ void __launch_bounds__(cap::kThreads)

@@ -135,7 +135,9 @@ def test_router_many_blocks_and_prepared_split(m, d, n, k, fn, renorm, bias):
                                            (777, 16, 3, 40, 777), (1536, 256, 8, 30, 256), (600, 5, 2, 0, 300),
                                            (300, 4, 2, 10 ** 6, 100), (64, 64, 63, 1, 64),
                                            # a large one-segment shape (many chunks in one segment)
-                                           (16384, 64, 6, 16384 * 6, 16384)])
+                                           (16384, 64, 6, 16384 * 6, 16384),
+                                           # more (segment, expert) pairs than the pair scan holds
+                                           (32768, 64, 2, 40, 256)])
 def test_capacity_bitexact(m, n, k, cap, seg):
     idx = W.make_topk_idx(m, n, k, seed=m * 7 + n)
     ref = oracle.capacity(idx, m, k, n, cap, seg)
