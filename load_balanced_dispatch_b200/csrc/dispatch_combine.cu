@@ -152,6 +152,75 @@ combine_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row,
     pdl_trigger();  // after this CTA's tokens: the dependent launch starts as the grid drains
 }
 
+// The same combine for k <= KMAX: a token's rows and gates are read once (lane r holds pick r's),
+// and each pass covers U 16-byte column chunks per lane with every kept row's loads issued before
+// the adds (the adds in pick order, as above: the same bits).
+template <typename T, int KMAX, int U>
+__global__ void __launch_bounds__(kRowThreads)
+combine_rows_kernel(const T* __restrict__ ybuf, const int32_t* __restrict__ dest_row, const float* __restrict__ gate,
+                    const T* __restrict__ residual, int64_t m, int k, int d, int gate_bf16, T* __restrict__ y) {
+    constexpr int V = Vec16<T>::N;
+    const int lane = threadIdx.x & 31;
+    pdl_wait();
+    const int nvec = d / V;
+    const int64_t warps = (int64_t)gridDim.x * (kRowThreads / 32);
+    for (int64_t i = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); i < m; i += warps) {
+        int32_t myrow = -1;
+        float myg = 0.f;
+        if (lane < k) {
+            myrow = dest_row[i * k + lane];
+            myg = gate[i * k + lane];
+            if (gate_bf16) myg = round_to_bf16(myg);
+        }
+        int32_t rows[KMAX];
+        float gs[KMAX];
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) {
+            rows[r] = __shfl_sync(0xffffffffu, myrow, r);
+            gs[r] = __shfl_sync(0xffffffffu, myg, r);
+        }
+        for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
+            float acc[U][V];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + 32 * u;
+                if (residual && c < nvec) {
+                    Vec16<T>::load(residual + i * d + (int64_t)c * V, acc[u]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < V; ++q) acc[u][q] = 0.f;
+                }
+            }
+            uint4 raw[KMAX][U];
+#pragma unroll
+            for (int r = 0; r < KMAX; ++r)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + 32 * u;
+                    if (r < k && rows[r] >= 0 && c < nvec)
+                        raw[r][u] = *reinterpret_cast<const uint4*>(ybuf + (int64_t)rows[r] * d + (int64_t)c * V);
+                }
+#pragma unroll
+            for (int r = 0; r < KMAX; ++r) {
+                if (r >= k || rows[r] < 0) continue;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float v[V];
+                    Vec16<T>::load(reinterpret_cast<const T*>(&raw[r][u]), v);
+#pragma unroll
+                    for (int q = 0; q < V; ++q) acc[u][q] = fmaf(gs[r], v[q], acc[u][q]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + 32 * u;
+                if (c < nvec) Vec16<T>::store(y + i * d + (int64_t)c * V, acc[u]);
+            }
+        }
+    }
+    pdl_trigger();
+}
+
 cudaError_t launch_dispatch(const void* x, moe_dtype dt, int64_t m, int d, const int32_t* src_token,
                             const int32_t* expert_offsets, int n, int64_t max_rows, void* xbuf,
                             cudaStream_t stream) {
@@ -173,6 +242,18 @@ cudaError_t launch_dispatch_tokens(const void* x, moe_dtype dt, int64_t m, int d
 cudaError_t launch_combine(const void* ybuf, moe_dtype dt, const int32_t* dest_row, const float* topk_gate,
                            const void* residual, int64_t m, int k, int d, void* y, cudaStream_t stream) {
     if (m == 0) return cudaSuccess;
+    if (dt == MOE_BF16 && k <= 8) {
+        // two chunks per lane per pass: 155.6 us at 65536 x 4096, k = 2, against 169.7 us for
+        // combine_kernel and 187.7 us with four chunks per pass
+#define MOE_COMBINE_ROWS(KM)                                                                                     \
+    return launch_pdl(combine_rows_kernel<__nv_bfloat16, KM, 2>, dim3(row_grid(m)), dim3(kRowThreads), 0, stream, \
+                      static_cast<const __nv_bfloat16*>(ybuf), dest_row, topk_gate,                             \
+                      static_cast<const __nv_bfloat16*>(residual), m, k, d, 1, static_cast<__nv_bfloat16*>(y))
+        if (k <= 2) MOE_COMBINE_ROWS(2);
+        if (k <= 4) MOE_COMBINE_ROWS(4);
+        MOE_COMBINE_ROWS(8);
+#undef MOE_COMBINE_ROWS
+    }
     if (dt == MOE_BF16) {
         return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(row_grid(m)), dim3(kRowThreads), 0, stream,
                           static_cast<const __nv_bfloat16*>(ybuf), dest_row, topk_gate,
