@@ -119,6 +119,81 @@ __device__ __forceinline__ void finish_row(const float (&h)[NT], int64_t row, in
     }
 }
 
+// One row finished by one thread from its n <= NV logits in registers v (k <= K): the operations of
+// finish_row, except that the softmax sum adds the terms in expert order (not a warp tree). The
+// K best (key, expert, score) are kept sorted while the experts are scanned in ascending order; a
+// key enters only if it beats the K-th kept one, so ties keep the lower index.
+// v is overwritten with the scores.
+template <int NV, int K>
+__device__ __forceinline__ void finish_row_thread(float (&v)[NV], int64_t row, int n, int k, int fn, int renorm,
+                                                  const float* rank_bias, float* probs_out, int32_t* topk_idx,
+                                                  float* topk_gate) {
+    float tk[K], tp[K];
+    int ti[K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) { tk[q] = -INFINITY; tp[q] = 0.f; ti[q] = 0; }
+    auto offer = [&](float key, int j, float pj) {
+        if (key > tk[K - 1]) {
+#pragma unroll
+            for (int q = K - 1; q > 0; --q) {
+                if (key > tk[q - 1]) { tk[q] = tk[q - 1]; ti[q] = ti[q - 1]; tp[q] = tp[q - 1]; }
+                else if (key > tk[q]) { tk[q] = key; ti[q] = j; tp[q] = pj; }
+            }
+            if (key > tk[0]) { tk[0] = key; ti[0] = j; tp[0] = pj; }
+        }
+    };
+    if (fn == MOE_SOFTMAX) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) if (j < n) mx = fmaxf(mx, v[j]);
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const float e = j < n ? expf(v[j] - mx) : 0.f;
+            if (!rank_bias && j < n) offer(v[j], j, e);  // the logit ranks; the score is divided below
+            v[j] = e;
+            s += e;
+        }
+#pragma unroll
+        for (int j = 0; j < NV; ++j) v[j] = v[j] / s;
+        if (rank_bias) {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) if (j < n) offer(__fadd_rn(v[j], __ldg(rank_bias + j)), j, v[j]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < K; ++q) tp[q] = tp[q] / s;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            v[j] = 1.f / (1.f + expf(-v[j]));
+            if (j < n) offer(rank_bias ? __fadd_rn(v[j], __ldg(rank_bias + j)) : v[j], j, v[j]);
+        }
+    }
+    if (probs_out) {
+        float* pr = probs_out + row * n;
+        if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(probs_out) & 15) == 0) {
+#pragma unroll
+            for (int c = 0; c < NV / 4; ++c)
+                if (4 * c < n)
+                    *reinterpret_cast<float4*>(pr + 4 * c) = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) if (j < n) pr[j] = v[j];
+        }
+    }
+    float selsum = 0.f;
+#pragma unroll
+    for (int q = 0; q < K; ++q) if (q < k) selsum += tp[q];
+    const bool rn = fn == MOE_SOFTMAX && renorm;
+#pragma unroll
+    for (int q = 0; q < K; ++q)
+        if (q < k) {
+            topk_idx[row * k + q] = ti[q];
+            topk_gate[row * k + q] = rn ? tp[q] / selsum : tp[q];
+        }
+}
+
 template <typename T, int NT>
 __global__ void __launch_bounds__(router::kThreads)
 router_topk_kernel(const T* __restrict__ x, const float* __restrict__ w_r, const float* __restrict__ logits_in,

@@ -17,11 +17,12 @@
 //                     lane); each K block's product lands in a fresh TMEM accumulator
 //                     (two, ping-pong) and is added into fp32 registers with
 //                     round-to-nearest adds, which keeps the sum fp32-accurate.
-//   Finish. With probs_out the tile's logits are stored (coalesced) and
-//   router_finish_kernel (one warp per row, the whole GPU) finishes them in place:
-//   softmax or logistic, ranking key, top-k with ties to the lower index, gates.
-//   Without probs_out each CTA takes whole rows (one tile of all n experts) and a warp
-//   finishes each row in the kernel.
+//   Finish: softmax or logistic, ranking key, top-k with ties to the lower index, gates.
+//   Logits mode: the tile's logits are stored (coalesced) and router_finish_kernel (one
+//   warp per row, the whole GPU) finishes them in place. Rows mode (no probs_out, or
+//   n <= 64 on a grid of more tiles than SMs): each CTA takes whole rows (one tile of all
+//   n experts) and finishes them in the kernel, a thread per row up to 64 experts (from
+//   the drain thread's registers), a warp per row above.
 #include "tc_ptx.cuh"
 
 namespace moe {
@@ -85,7 +86,7 @@ enum { kModeLogits = 0, kModeRows = 2 };
 // (N = 3 NP) forms all three products, so each K step reads the x tile from shared memory once
 // instead of three times; the drain adds the parts' block products in fp32, small parts first.
 template <int NCH, int STAGES, bool FUSED>
-__global__ void __launch_bounds__(rtc::kThreads, 1)
+__global__ void __launch_bounds__(rtc::kThreads, STAGES == 2 ? 2 : 1)  // two-stage rings: two CTAs per SM
 router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w, int64_t m,
                  int d, int n, int k, int fn, int renorm, const float* __restrict__ rank_bias,
                  float* __restrict__ probs_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
@@ -215,8 +216,20 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             ptx::mbar_arrive(&sh->tempty[buf]);
             if (++buf == 2) { buf = 0; bphase ^= 1u; }
         }
-        // park the warp's 32 logit rows in the (now idle) stage memory
-        if (drain_ok) {
+        bool finished = false;
+        if constexpr (NP <= 64) {
+            if (drain_ok && mode == kModeRows && k <= 8) {
+                // whole rows in this CTA: the thread finishes the row it drained, from its registers
+                const int64_t r = row0 + quad * 32 + lane;
+                if (r < m) {
+                    if (k <= 2) finish_row_thread<NP, 2>(acc, r, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+                    else finish_row_thread<NP, 8>(acc, r, n, k, fn, renorm, rank_bias, probs_out, topk_idx, topk_gate);
+                }
+                finished = true;
+            }
+        }
+        if (drain_ok && !finished) {
+            // park the warp's 32 logit rows in the (now idle) stage memory
             float* rows = reinterpret_cast<float*>(smem) + (size_t)quad * 32 * (NP + 1);
 #pragma unroll
             for (int j = 0; j < NP; ++j) rows[lane * (NP + 1) + j] = acc[j];
@@ -234,7 +247,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                     }
                 }
             } else if (mode == kModeRows) {
-                // whole rows in this CTA (no scores out): a warp finishes each row
+                // whole rows in this CTA (more than 64 experts): a warp finishes each row
                 for (int rr = 0; rr < 32; ++rr) {
                     const int64_t r = row0 + quad * 32 + rr;
                     if (r >= m) break;
@@ -336,14 +349,19 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, int64_t m, int d, 
     const int np = router_np(n);
     CUtensorMap mx, mw;
     if (!map_2d(&mx, x, (uint64_t)m, (uint64_t)d, rtc::BM)) return cudaErrorInvalidValue;
-    // With probs_out the logits go to memory in 64-wide column tiles and router_finish_kernel (a
-    // warp per row, the whole GPU) finishes them in place; without it (nothing to store them in)
-    // each CTA keeps whole rows and a warp finishes each. Measured against a persistent kernel
-    // that finished the rows in the same launch (a logits tile in shared memory, four finish
-    // warps): 162 against 204 us at 65536 x 4096 x 64, 19 against 45 us at 8192 x 768 x 128. One
-    // CTA per SM left its K-block pipeline latency-bound (33% issue-active); here two CTAs share
-    // an SM and the finish runs on every SM's warps.
-    const int mode = probs_out ? rtc::kModeLogits : rtc::kModeRows;
+    // Two ways to finish the rows. Logits mode: the projection stores the fp32 logits in 64-wide
+    // column tiles and router_finish_kernel (a warp per row, over the whole GPU) finishes them in
+    // place. Rows mode: a CTA holds whole rows (one column tile of all n experts) and finishes
+    // them itself -- each drain thread its own row from its registers up to 64 experts, a warp
+    // per row above. Rows mode is taken without probs_out, and with it when n <= 64 and there are
+    // more 128-row tiles than SMs (two CTAs per SM: one CTA's finish runs while the other streams
+    // x): 146.5 against 163.6 us at 65536 x 4096 x 64. With one CTA per SM the finish would run
+    // on an otherwise idle SM, and logits mode is faster (38.2 against 41.5 us at
+    // 16384 x 2048 x 64). A persistent kernel that finished the rows in the same launch (a
+    // logits tile in shared memory, four finish warps) measured 204 against 162 us at
+    // 65536 x 4096 x 64, its one K-block pipeline per SM latency-bound (33% issue-active).
+    const bool many_tiles = (m + rtc::BM - 1) / rtc::BM > (int64_t)num_sms();
+    const int mode = (probs_out && !(np <= 64 && many_tiles)) ? rtc::kModeLogits : rtc::kModeRows;
     const int tile = mode == rtc::kModeRows ? np : (np < 64 ? np : 64);
     if (!map_3d(&mw, wsplit, 3, (uint64_t)n, (uint64_t)d, (uint32_t)tile)) return cudaErrorInvalidValue;
     cudaError_t e;

@@ -219,15 +219,20 @@ class MoELayer:
                                   stream=stream)
 
     def launches_per_forward(self) -> int:
-        """Kernel launches of one forward: router (bf16 with n <= 128: projection and finish, 2; else 1), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
+        """Kernel launches of one forward: router (bf16 with n <= 128: projection and finish, 2, except
+        n <= 64 with more 128-token tiles than SMs, where the projection kernel finishes the rows, 1;
+        else 1), capacity 2 (count + scan, assign), dispatch 1 (0 when the FFN
         gathers its rows from x), FFN (bf16: one fused launch, after a memset of its counters; fp32: 2),
         combine 1, statistics 1. With one pick per token in bf16 the combine is the FFN's epilogue plus
         one launch for the dropped tokens' rows (which also clears the FFN's counters)."""
         s = self.shape
         bf16 = s.dtype == torch.bfloat16
         # bf16 with n <= 128: tensor-core logits tiles + the finish kernel (the W_r split is made
-        # once, at construction); otherwise the fp32 FMA kernel
-        router = 2 if (bf16 and s.n <= 128) else 1
+        # once, at construction), or one launch when the projection kernel finishes whole rows
+        # (n <= 64 and more 128-token tiles than SMs); otherwise the fp32 FMA kernel
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        rows_mode = s.n <= 64 and (s.m + 127) // 128 > sms
+        router = 2 if (bf16 and s.n <= 128 and not rows_mode) else 1
         capacity = 2
         dispatch = 1 if self.uses_dispatch() else 0
         if self.ffn_combine:  # the FFN with the combine in its epilogue, plus the dropped rows
