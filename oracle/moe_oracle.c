@@ -478,8 +478,12 @@ static void qb_col_pass(const float* s, int64_t m, int n, int64_t C, const float
  *   W[a][b] = min_i (s_ia - s_ib) in fp64, the argmin token is the lowest index.
  *   distances: every over-full expert starts at 0; rounds of
  *   dist'[b] = min(dist[b], min_a dist[a] + W[a][b]) (all b from the previous
- *   round's dist) until nothing changes; pred[b] = lowest a with
- *   dist[a] + W[a][b] == dist[b].
+ *   round's dist) until nothing changes; settle[b] = the round (1-based) of b's
+ *   last decrease, 0 for the over-full experts; pred[b] = lowest a with
+ *   dist[a] + W[a][b] == dist[b] and settle[a] < settle[b]. (The value that set
+ *   dist[b] in its last round came from an a already final by then, so such an
+ *   a exists; settle decreases along pred, so the path ends at an over-full
+ *   expert even when zero-cost cycles make several arcs tight.)
  *   target: under-full expert with the least distance (lowest index on ties);
  *   every arc of its path moves its argmin token.
  * Stops when all counts equal C or after max_repair moves.
@@ -491,6 +495,7 @@ static int qb_repair(const float* s, int64_t m, int n, int64_t C, unsigned char*
     double* dist = (double*)malloc(sizeof(double) * (size_t)n);
     double* nd = (double*)malloc(sizeof(double) * (size_t)n);
     int* pred = (int*)malloc(sizeof(int) * (size_t)n);
+    int* settle = (int*)malloc(sizeof(int) * (size_t)n);
     int* path = (int*)malloc(sizeof(int) * (size_t)(n + 1));
     int* sel = (int*)malloc(sizeof(int) * (size_t)n);
     int* unsel = (int*)malloc(sizeof(int) * (size_t)n);
@@ -514,7 +519,7 @@ static int qb_repair(const float* s, int64_t m, int n, int64_t C, unsigned char*
                 }
             }
         }
-        for (int e = 0; e < n; ++e) dist[e] = cnt[e] > C ? 0.0 : INFINITY;
+        for (int e = 0; e < n; ++e) { dist[e] = cnt[e] > C ? 0.0 : INFINITY; settle[e] = 0; }
         int settled = 0;
         for (int round = 0; round <= n; ++round) {
             int changed = 0;
@@ -526,7 +531,7 @@ static int qb_repair(const float* s, int64_t m, int n, int64_t C, unsigned char*
                     if (c < best) best = c;
                 }
                 nd[b] = best;
-                if (best != dist[b]) changed = 1;
+                if (best != dist[b]) { changed = 1; settle[b] = round + 1; }
             }
             memcpy(dist, nd, sizeof(double) * (size_t)n);
             if (!changed) { settled = 1; break; }
@@ -537,7 +542,7 @@ static int qb_repair(const float* s, int64_t m, int n, int64_t C, unsigned char*
             if (dist[b] == INFINITY) continue;
             for (int a = 0; a < n; ++a) {
                 if (a == b || dist[a] == INFINITY || W[a * n + b] == INFINITY) continue;
-                if (dist[a] + W[a * n + b] == dist[b]) { pred[b] = a; break; }
+                if (dist[a] + W[a * n + b] == dist[b] && settle[a] < settle[b]) { pred[b] = a; break; }
             }
         }
         int target = -1;
@@ -561,7 +566,7 @@ static int qb_repair(const float* s, int64_t m, int n, int64_t C, unsigned char*
         cnt[target]++;
         (*augments)++;
     }
-    free(W); free(A); free(dist); free(nd); free(pred); free(path); free(sel); free(unsel);
+    free(W); free(A); free(dist); free(nd); free(pred); free(settle); free(path); free(sel); free(unsel);
     return status;
 }
 

@@ -95,6 +95,22 @@ def test_lp_medium(m, n, k, iters, seed):
     assert oracle.is_optimal(s, idx)
 
 
+@pytest.mark.parametrize("m,n,k,seed", [(64, 8, 2, 0), (96, 6, 2, 1), (128, 8, 3, 2), (48, 4, 1, 3), (64, 8, 2, 4)])
+def test_solve_with_zero_cost_cycles(m, n, k, seed):
+    # half-integer scores with every third row constant: many tokens swap two experts at the same
+    # cost, so the expert graph has zero-cost cycles and several arcs into an expert are tight.
+    # The exact finish must still follow a path back to an over-full expert (predecessors settled
+    # in an earlier Bellman-Ford round) and reach the LP optimum.
+    s = (np.round(np.random.default_rng(seed).standard_normal((m, n)) * 2) / 2).astype(np.float32)
+    s[::3] = np.float32(0.5)
+    idx, _, info, rc = oracle.balance_assign(s, k, max_iters=3)
+    assert rc == oracle.OK and info[2] == 0 and info[1] > 0
+    _check_balanced(idx, m, n, k)
+    obj, _ = _lp(s, k)
+    assert _objective(s, idx) == pytest.approx(obj, rel=1e-12, abs=1e-9)
+    assert oracle.is_optimal(s, idx)
+
+
 def test_hungarian_k1():
     m, n = 120, 6
     s = W.make_qb_scores(m, n, seed=7)
