@@ -1876,7 +1876,9 @@ constexpr int kRepCols = 32;      // columns of W per CTA (n <= 256)
 // writes its columns' new distances and change flags into the next-round buffers of every CTA
 // of the cluster (distributed shared memory) and one cluster barrier ends the round, so every
 // CTA holds the same full distance vector. Then the predecessors (lowest a with
-// dist[a] + W[a][b] == dist[b]) of each CTA's columns go to CTA 0, whose thread 0 takes the
+// dist[a] + W[a][b] == dist[b] whose distance settled in an earlier round than b's: the value that
+// set dist[b] in its last round came from such an a, and with zero-cost cycles several arcs can be
+// tight) of each CTA's columns go to CTA 0, whose thread 0 takes the
 // nearest under-full expert (lowest index on ties), walks the path and moves each arc's token,
 // and CTA 0 lists the rows of W the moves invalidate (the old set of every moved token, plus the
 // expert it moved to) for the next arc launch. All decisions that end loops or return are made
@@ -1892,6 +1894,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     __shared__ double part_d[8][qb::kRepCols];
     __shared__ int part_p[8][qb::kRepCols];
     __shared__ int pred[kMaxExperts];
+    __shared__ int settle[kMaxExperts];  // the round (1-based) of each expert's last decrease, 0 for the roots
     __shared__ int front[kMaxExperts], nfront, wcount[kMaxExperts / 32];
     __shared__ int any_over;
     const int tid = threadIdx.x, bl = tid & 31, part = tid >> 5;
@@ -1913,6 +1916,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         chg[0][e] = over ? 1 : 0;
         chg[1][e] = 0;
         pred[e] = -1;
+        settle[e] = 0;
         if (over) atomicOr(&any_over, 1);
     }
     __syncthreads();
@@ -1923,6 +1927,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
     ptx::cluster_sync();  // every CTA's buffers are initialised before any remote write
     int cur = 0;
     bool settled = false;
+    int my_settle = 0;  // column b's settle round (the fold threads)
     for (int round = 0; round <= n; ++round) {
         // warp `part` relaxes from the changed experts among 32 part .. 32 part + 31 (a ballot of
         // the change flags, no compaction); the rounds end when no flag is set in any CTA's copy
@@ -1949,6 +1954,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
             double nd = dist[cur][b];
             for (int p = 0; p < 8; ++p) nd = fmin(nd, part_d[p][bl]);
             const unsigned char nc = nd != dist[cur][b] ? 1 : 0;
+            if (nc) my_settle = round + 1;
             for (int r = 0; r < qb::kRepCtas; ++r) {
                 ptx::st_cluster_f64(ptx::mapa_shared(ptx::smem_u32(&dist[cur ^ 1][b]), (uint32_t)r), nd);
                 ptx::st_cluster_u8(ptx::mapa_shared(ptx::smem_u32(&chg[cur ^ 1][b]), (uint32_t)r), nc);
@@ -1966,6 +1972,11 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         }
         return;
     }
+    // every CTA learns every column's settle round
+    if (part == 0 && own)
+        for (int r = 0; r < qb::kRepCtas; ++r)
+            ptx::st_cluster_s32(ptx::mapa_shared(ptx::smem_u32(&settle[b]), (uint32_t)r), my_settle);
+    ptx::cluster_sync();
     // predecessors of this CTA's columns, over the reachable experts, to CTA 0
     for (int e = tid; e < kMaxExperts; e += blockDim.x) chg[cur ^ 1][e] = (e < n && dist[cur][e] != INFINITY) ? 1 : 0;
     __syncthreads();
@@ -1977,7 +1988,7 @@ qb_repair_step_kernel(int n, int64_t C, int k, const double* __restrict__ W, con
         for (int f = part; f < nr; f += 8) {
             const int a = front[f];
             const double w = wsl[a * qb::kRepCols + bl];
-            if (a != b && w != INFINITY && dist[cur][a] + w == db && a < pa) pa = a;
+            if (a != b && w != INFINITY && dist[cur][a] + w == db && settle[a] < settle[b] && a < pa) pa = a;
         }
     }
     part_p[part][bl] = pa;

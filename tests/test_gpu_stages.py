@@ -538,12 +538,26 @@ def test_balance_row_pass_forms(m, n, k, kind):
         assert (host(info) == info_ref).all()
         b = b_ref
     if kind == "tied_rows":
-        # whole rows of equal values give the exact finish zero-cost cycles between experts, where
-        # its path reconstruction is not defined: STEPs only
-        return
+        return  # the SOLVE of heavily tied scores: test_balance_solve_zero_cost_cycles
     i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=10)
     assert rc == oracle.OK
     idx, beta, info = lb.moe_balance_assign(dev(s), k, mode=lb.MOE_QB_SOLVE, max_iters=10)
+    torch.cuda.synchronize()
+    assert (host(info) == info_ref).all()
+    assert (host(beta) == b_ref).all()
+    assert (host(idx) == i_ref).all()
+
+
+@pytest.mark.parametrize("m,n,k,seed", [(1024, 16, 2, 0), (2048, 32, 4, 1), (1536, 64, 8, 2)])
+def test_balance_solve_zero_cost_cycles(m, n, k, seed):
+    # half-integer scores with every third row constant: the exact finish runs thousands of moves on
+    # an expert graph with zero-cost cycles (several tight arcs into an expert); the predecessor
+    # settled in the earlier round keeps every path acyclic. Picks, beta and info bit-exact.
+    s = (np.round(np.random.default_rng(seed).standard_normal((m, n)) * 2) / 2).astype(np.float32)
+    s[::3] = np.float32(0.5)
+    i_ref, b_ref, info_ref, rc = oracle.balance_assign(s, k, mode=oracle.QB_SOLVE, max_iters=6)
+    assert rc == oracle.OK and info_ref[1] > 0
+    idx, beta, info = lb.moe_balance_assign(dev(s), k, mode=lb.MOE_QB_SOLVE, max_iters=6)
     torch.cuda.synchronize()
     assert (host(info) == info_ref).all()
     assert (host(beta) == b_ref).all()
