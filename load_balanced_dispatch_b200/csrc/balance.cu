@@ -10,19 +10,25 @@
 // so every decision is reproducible bit for bit.
 //
 // Kernels:
-//   qb_row     one warp per token: v = s_i - beta in registers (n/32 values per
-//              lane); the keys that can be among the k + 1 best are found from
-//              the lane maxima and gathered one per lane, and their ranks give
-//              the top-k set, the k-th and (k+1)-th values (alpha) and a tie
-//              flag (k + 1 rounds of a warp arg-max when that does not apply);
-//              the set is written in ascending expert order and counted per
-//              expert. The first row pass of a SOLVE also writes s transposed
-//              (sT [n, m]) for the column pass's full path. Before a column
-//              pass the row pass also runs that pass's window sweep on the rows
-//              it holds: once it has alpha_i, per column the keys of
-//              u = s - alpha above a window around the current beta_j are
-//              counted and those inside are listed (one read of s per
-//              iteration instead of two).
+//   qb_row_tpr2 the row pass, one thread per token (when k + 1 <= the number of
+//              column groups): a warp reads 32 rows coalesced and forms the
+//              row's 32 column-group maxima of v = s - beta; T, the (k+1)-th
+//              largest of them, bounds the row's (k+1)-th value from below; the
+//              thread lists its row's elements at or above T (or the lower T'
+//              that also covers the window sweep), sorts their keys and takes
+//              the top-k set (ascending expert order), the k-th and (k+1)-th
+//              values (alpha) and a tie flag. Before a column pass it also runs
+//              that pass's window sweep on the listed elements (keys of
+//              u = s - alpha above a window around the current beta_j counted,
+//              those inside listed), and in the sign step it counts
+//              fp32(s - alpha) > beta_j, so s is read once per iteration.
+//   qb_row_tpr the same selection on rows staged in shared memory, for the
+//              first row pass of a SOLVE, which also writes s transposed
+//              (sT [n, m]) for the column pass's full path.
+//   qb_row     one warp per token (k + 1 above the group count, and rows whose
+//              list overflows): the lane maxima bound the (k+1)-th key, the
+//              keys reaching it are ranked (k + 1 rounds of a warp arg-max when
+//              more than 32 reach it).
 //   qb_col     one CTA per expert column: when the C-th largest fell inside
 //              the window, the C-th and (C+1)-th largest come from the column's
 //              list (radix digits over order-preserving uint32 keys); otherwise
@@ -34,8 +40,9 @@
 //              (fp64, lowest token on ties); an 8-CTA cluster (W's columns
 //              split over the CTAs' shared memory) runs Jacobi Bellman-Ford
 //              rounds from the over-full experts, picks the nearest under-full
-//              expert (lowest index on ties) and moves each arc's argmin
-//              token. The number of moves equals the excess, so the host
+//              expert (lowest index on ties), follows predecessors settled in
+//              an earlier round back to an over-full expert and moves each
+//              arc's argmin token. The number of moves equals the excess, so the host
 //              enqueues exactly that many rounds without waiting in between.
 #include "common.cuh"
 #include "tc_ptx.cuh"
