@@ -938,6 +938,7 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
                    float* __restrict__ alpha, int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts,
                    int32_t* __restrict__ status, int tie_slot, int skip_if_done, RowSweep sw,
                    int32_t* __restrict__ sign_counts) {
+    pdl_wait();  // beta, the status words and the counters come from the previous launches
     if (skip_if_done && *(volatile int32_t*)&status[qb::kStQbDone]) return;
     constexpr int W = qb::kTpr2Warps, NC = 32 * NT, CAP = qb::kTprCap, GS = 33;
     extern __shared__ __align__(16) float dsm[];  // per warp: [32][33] group maxima, [CAP][32] listed scores; then [W][CAP][32] columns
@@ -1251,6 +1252,7 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
             if (above_s[j]) atomicAdd(&sw.g_above[j], above_s[j]);
         if (npairs) sweep_flush(pairs, &npairs, scnt, sbase, sfull, n, sw, (unsigned)qb::kTprPairCap);
     }
+    pdl_trigger();
 }
 
 // Block-wide bin selection: scanning bins from the top, the bin where the cumulative count
@@ -1558,6 +1560,7 @@ qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t
               int32_t* __restrict__ status, int iter, int check, uint32_t* __restrict__ win,
               uint32_t* __restrict__ g_above, uint32_t* __restrict__ g_ncand, const uint32_t* __restrict__ g_cand,
               const int32_t* __restrict__ info_counts, int tie_slot, int32_t* __restrict__ info) {
+    pdl_wait();  // the row pass's counts, alpha and window lists
     if (info && blockIdx.x == 0 && threadIdx.x < 32) {
         int64_t ex = 0;
         for (int e = threadIdx.x; e < n; e += 32) ex += info_counts[e] > C ? info_counts[e] - C : 0;
@@ -1631,6 +1634,7 @@ qb_col_kernel(const float* __restrict__ s, const float* __restrict__ sT, int64_t
         if (wn > qb::kWinMax) wn = qb::kWinMax;
         win[j] = (uint32_t)wn;
     }
+    pdl_trigger();
 }
 
 // The practical QB step on mini-batches ("MoE travelogue 6", Mind the pitfall, closing
@@ -2329,8 +2333,9 @@ static void launch_row_tpr2_t(const float* s, int64_t m, int n, int k, const flo
     int64_t blocks = (ntiles + qb::kTpr2Warps - 1) / qb::kTpr2Warps;
     if (blocks > kNumSMs) blocks = kNumSMs;
     if (blocks < 1) blocks = 1;
-    qb_row_tpr2_kernel<NT, SWEEP, SIGN><<<(unsigned)blocks, qb::kTpr2Warps * 32, smem, stream>>>(
-        s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sw, sign_counts);
+    // programmatic dependent launch: the pass's prologue overlaps the previous launch's tail
+    launch_pdl(qb_row_tpr2_kernel<NT, SWEEP, SIGN>, dim3((unsigned)blocks), dim3(qb::kTpr2Warps * 32), smem, stream,
+               s, m, n, k, beta, rule, alpha, topk_idx, counts, status, tie_slot, skip, sw, sign_counts);
 }
 
 // Returns true when the launched pass also counted sign_counts (then no separate count is needed).
@@ -2386,9 +2391,9 @@ static bool launch_row(const float* s, int64_t m, int n, int k, const float* bet
 static void launch_col(const float* s, const float* sT, int64_t m, int n, int64_t C, const QBWorkspace& w, int rule,
                        float* beta, const int32_t* counts, int32_t* counts_next, int iter, int check,
                        cudaStream_t stream, int32_t* info = nullptr) {
-    qb_col_kernel<<<n, qb::kColThreads, qb::kColSmem, stream>>>(s, sT, m, n, C, w.alpha, rule, beta, counts_next,
-                                                                w.status, iter, check, w.win, w.g_above, w.g_ncand,
-                                                                w.g_cand, counts, qb::kStTies0, info);
+    launch_pdl(qb_col_kernel, dim3((unsigned)n), dim3(qb::kColThreads), qb::kColSmem, stream, s, sT, m, n, C,
+               (const float*)w.alpha, rule, beta, counts_next, w.status, iter, check, w.win, w.g_above, w.g_ncand,
+               (const uint32_t*)w.g_cand, counts, (int)qb::kStTies0, info);
 }
 
 template <int NT>
