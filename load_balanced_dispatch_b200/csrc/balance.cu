@@ -497,6 +497,19 @@ __device__ __forceinline__ void sort_desc(V (&a)[N]) {
             }
 }
 
+// a[idx & 15] for a 16-entry register array (a tree of selects).
+template <typename V>
+__device__ __forceinline__ V value_at(const V (&a)[16], int idx) {
+    V b[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) b[q] = (idx & 8) ? a[q + 8] : a[q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) b[q] = (idx & 4) ? b[q + 4] : b[q];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) b[q] = (idx & 2) ? b[q + 2] : b[q];
+    return (idx & 1) ? b[1] : b[0];
+}
+
 // a[idx] for a register array: a tree of selects on the bits of idx (no local-memory copy).
 template <typename V>
 __device__ __forceinline__ V value_at(const V (&a)[32], int idx) {
@@ -1108,11 +1121,23 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
                 }
                 kk[p] = key;
             }
-            sort_desc(kk);
-            KK = value_at(kk, k - 1);
-            KK1 = value_at(kk, k);
+            if (pmax <= 16) {
+                // at most 16 listed elements in every row of the warp (then k < 16): a 16-wide network
+                uint32_t k16[16];
 #pragma unroll
-            for (int p = 0; p < CAP; ++p) A += kk[p] > KK ? 1 : 0;
+                for (int p = 0; p < 16; ++p) k16[p] = kk[p];
+                sort_desc(k16);
+                KK = value_at(k16, k - 1);
+                KK1 = value_at(k16, k);
+#pragma unroll
+                for (int p = 0; p < 16; ++p) A += k16[p] > KK ? 1 : 0;
+            } else {
+                sort_desc(kk);
+                KK = value_at(kk, k - 1);
+                KK1 = value_at(kk, k);
+#pragma unroll
+                for (int p = 0; p < CAP; ++p) A += kk[p] > KK ? 1 : 0;
+            }
         }
         const float vk = key_float(KK), vk1 = key_float(KK1);
         const float a = qb_threshold(vk, vk1, rule);
