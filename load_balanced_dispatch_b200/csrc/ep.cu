@@ -89,7 +89,10 @@ ep_dispatch_kernel(const uint4* __restrict__ x, int64_t m, int64_t vec_per_row, 
             const uint32_t kept = __ballot_sync(0xffffffffu, row >= 0);
             if (!kept) continue;
             const uint4* src = x + i * vec_per_row;
-            for (int64_t c0 = lane; c0 < vec_per_row; c0 += 32 * 8) {
+            // the pass count is warp-uniform, so every lane reaches the shuffles below (rows of
+            // fewer than 32 vectors leave the upper lanes without columns, not outside the loop)
+            for (int64_t cb = 0; cb < vec_per_row; cb += 32 * 8) {
+                const int64_t c0 = cb + lane;
                 uint4 v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {

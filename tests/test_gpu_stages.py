@@ -169,7 +169,10 @@ def test_capacity_rejects_bad_expert_ids():
 
 # ---------------------------------------------------------------- dispatch / combine
 @pytest.mark.parametrize("dtype,m,d,n,k,cap", [("bf16", 1000, 768, 16, 2, 100), ("fp32", 513, 64, 8, 1, 80),
-                                               ("bf16", 300, 4096, 64, 2, 0)])
+                                               ("bf16", 300, 4096, 64, 2, 0),
+                                               # rows of fewer than 32 16-byte vectors with several picks
+                                               ("bf16", 777, 128, 64, 2, 40), ("bf16", 500, 64, 8, 3, 150),
+                                               ("bf16", 400, 8, 4, 3, 1000), ("fp32", 333, 20, 16, 5, 90)])
 def test_dispatch_combine(dtype, m, d, n, k, cap):
     rng = np.random.default_rng(d)
     x = rng.standard_normal((m, d)).astype(np.float32)
