@@ -207,7 +207,9 @@ def test_dispatch_combine(dtype, m, d, n, k, cap):
 @pytest.mark.parametrize("dtype,rows_per,d,d_ff", [("fp32", [100, 0, 37, 256, 1], 64, 256),
                                                    ("bf16", [64, 80, 0, 3, 129, 77], 768, 3072),
                                                    ("bf16", [130, 1, 0, 256], 2048, 1408),
-                                                   ("bf16", [0, 300], 256, 512)])
+                                                   ("bf16", [0, 300], 256, 512),
+                                                   # 512-column tiles (d and d_ff multiples of 512)
+                                                   ("bf16", [300, 0, 17, 513, 256], 512, 1024)])
 def test_expert_ffn(dtype, rows_per, d, d_ff):
     n = len(rows_per)
     rng = np.random.default_rng(d + d_ff)
@@ -257,7 +259,8 @@ def test_expert_ffn_combine_matches_two_calls(m, n, d, d_ff, cap):
 
 
 @pytest.mark.parametrize("m,n,k,d,d_ff,cap", [(2000, 16, 2, 768, 3072, 300), (1000, 64, 6, 2048, 1408, 10 ** 6),
-                                              (777, 8, 3, 256, 512, 40), (512, 4, 1, 128, 256, 0)])
+                                              (777, 8, 3, 256, 512, 40), (512, 4, 1, 128, 256, 0),
+                                              (1500, 8, 2, 1024, 512, 300)])
 def test_expert_ffn_gather_matches_dispatch(m, n, k, d, d_ff, cap):
     # the FFN loading its rows from x by src_token gives bit for bit the FFN of the dispatched
     # copy, including dropped picks, ragged experts and a capacity that empties every expert
