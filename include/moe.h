@@ -70,6 +70,19 @@ MOE_API void moe_last_error(char* buf, size_t len);
 MOE_API moe_status moe_sync_status(moe_stream_t stream);
 
 /*
+ * Self-test of the bounded waits (no passage: an engineering check). One warp
+ * waits until the int32 *flag (device memory) is at least 1, polling it the
+ * way the FFN's second-GEMM tiles poll their per-expert counters, for at most
+ * limit_cycles SM clock cycles (0 .. 4e9; the library's own waits use 4e9,
+ * about 2 s). If nothing sets the flag the wait gives up, the device error
+ * word records a pipeline timeout, and the kernel returns: the next
+ * moe_sync_status reports MOE_ERR_INTERNAL ("a pipeline wait timed out") and
+ * the context stays usable. Asynchronous on `stream`; the flag is only read.
+ * Errors: MOE_ERR_INVALID_ARG (NULL flag, limit out of range), MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_selftest_wait(const int32_t* flag, int64_t limit_cycles, moe_stream_t stream);
+
+/*
  * Router and top-k selection.
  * Passage: "Switch Transformers paper review" (tildalice.io/?p=118), Switch
  * Routing Steps 1-3 (h = x W_r, p = softmax(h), i* = argmax p, gate p_i*) and

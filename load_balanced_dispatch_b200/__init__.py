@@ -55,6 +55,7 @@ def lib() -> C.CDLL:
         L.moe_last_error.argtypes = [C.c_char_p, SZ]
         L.moe_last_error.restype = None
         L.moe_sync_status.argtypes = [P]
+        L.moe_selftest_wait.argtypes = [P, I64, P]
         L.moe_router_topk_workspace_size.argtypes = [I32, I32, I32, I32]
         L.moe_router_topk_workspace_size.restype = SZ
         L.moe_router_topk.argtypes = [P, I32, P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
@@ -134,6 +135,13 @@ def _need(t, dtype, shape, name):
 def sync_status(stream=None):
     """Synchronise the stream and raise if a kernel recorded a device-side error."""
     _check("moe_sync_status", lib().moe_sync_status(_stream(stream)))
+
+
+def moe_selftest_wait(flag, limit_cycles, stream=None):
+    """One warp waits (at most limit_cycles SM cycles) for the int32 device scalar `flag` to reach 1;
+    if nothing sets it, the device error word records a pipeline timeout (see sync_status)."""
+    _need(flag, torch.int32, (1,), "flag")
+    _check("moe_selftest_wait", lib().moe_selftest_wait(_ptr(flag), int(limit_cycles), _stream(stream)))
 
 
 def moe_router_topk(x, w_r, n, k, score_fn=MOE_SOFTMAX, renorm_topk=0, rank_bias=None, logits_in=None,

@@ -53,6 +53,7 @@ cudaError_t launch_ep_dispatch(const void* x, moe_dtype dt, int64_t m, int d, in
 cudaError_t launch_ep_combine(const void* const* peers, moe_dtype dt, const int32_t* ep_row, const int32_t* topk_idx,
                               int n, int G, const float* gate, const void* residual, int64_t m, int k, int d, void* y,
                               cudaStream_t stream);
+cudaError_t launch_selftest_wait(const int32_t* flag, int64_t limit_cycles, cudaStream_t stream);
 int run_balance_sign_step(const float* s, int64_t m, int n, int k, float* beta, float gamma, int rule,
                           int32_t* topk_idx, int32_t* info, void* workspace, cudaStream_t stream, const char** err);
 int run_balance_step_minibatch(const float* s, int64_t m, int n, int k, float* beta, int rule, int64_t seg_len,
@@ -114,6 +115,12 @@ moe_status moe_sync_status(moe_stream_t stream) {
     }
     g_last_error[0] = 0;
     return MOE_OK;
+}
+
+moe_status moe_selftest_wait(const int32_t* flag, int64_t limit_cycles, moe_stream_t stream) {
+    REQUIRE(flag, "flag is required");
+    REQUIRE(limit_cycles >= 0 && limit_cycles <= 4000000000LL, "limit_cycles must be in [0, 4e9]");
+    return check_launch(launch_selftest_wait(flag, limit_cycles, stream), "moe_selftest_wait");
 }
 
 size_t moe_router_topk_workspace_size(int32_t d, int32_t n, int32_t k, moe_dtype x_dtype) {

@@ -211,17 +211,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                     // all GEMM1 tiles of expert e, each signalled by its 4 epilogue warps
                     const int rows_e = sh->g1.row_start[t.e + 1] - sh->g1.row_start[t.e];
                     const int need = ((rows_e + BM - 1) / BM) * ntn1 * kEpiWarps;
-                    const long long t0 = clock64();
-                    bool ok = true;
-                    while (ptx::ld_acquire_gpu(done1 + t.e) < need) {
-                        if (*abort_flag || clock64() - t0 > ptx::kWaitCycles) {
-                            if (!*abort_flag) { *abort_flag = 1; record_error(kErrPipelineTimeout); }
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    if (!ok) break;
+                    if (!ptx::wait_count_geq(done1 + t.e, need, abort_flag, ptx::kWaitCycles)) break;
                     ptx::fence_proxy_async_global();
                 }
                 const CUtensorMap* ma = t.phase == 1 ? &map_x : &map_h;

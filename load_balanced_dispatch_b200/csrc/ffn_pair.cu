@@ -196,17 +196,7 @@ ffn_pair_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 if (t.phase == 2) {
                     // every GEMM1 tile of expert e, each signalled by every epilogue warp of its pair
                     const int need = t.mtiles * ntn1 * EPI * 2;
-                    const long long t0 = clock64();
-                    bool ok = true;
-                    while (ptx::ld_acquire_gpu(done1 + t.e) < need) {
-                        if (*abort_flag || clock64() - t0 > ptx::kWaitCycles) {
-                            if (!*abort_flag) { *abort_flag = 1; record_error(kErrPipelineTimeout); }
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    if (!ok) break;
+                    if (!ptx::wait_count_geq(done1 + t.e, need, abort_flag, ptx::kWaitCycles)) break;
                     ptx::fence_proxy_async_global();
                 }
                 const CUtensorMap* ma = t.phase == 1 ? &map_x : &map_h;

@@ -125,6 +125,24 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Waits until the counter *p (written by other CTAs) reaches `need`, polling with acquire loads.
+// Bounded: after `limit` SM clock cycles, or at once when *abort_flag (if given) is already set,
+// it gives up and returns false; a wait that ran out records kErrPipelineTimeout in the device
+// error word and sets *abort_flag, so the CTA's other roles leave their loops too.
+__device__ __forceinline__ bool wait_count_geq(const int* p, int need, volatile int* abort_flag, long long limit) {
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(p) < need) {
+        if ((abort_flag && *abort_flag) || clock64() - t0 > limit) {
+            if (!(abort_flag && *abort_flag)) {
+                if (abort_flag) *abort_flag = 1;
+                record_error(kErrPipelineTimeout);
+            }
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
+}
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

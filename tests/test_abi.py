@@ -106,3 +106,8 @@ def test_invalid_arguments_rejected_before_any_launch(L):
     # residual aliasing the output
     rc = L.moe_combine(fake, 1, fake, fake, fake, 4, 1, 64, fake, None)
     assert rc == 1 and "alias" in _err(L)
+    # the bounded-wait self-test: a flag is required, and the limit is at most the library's own
+    rc = L.moe_selftest_wait(None, C.c_int64(1000), None)
+    assert rc == 1 and "flag" in _err(L)
+    rc = L.moe_selftest_wait(fake, C.c_int64(5_000_000_000), None)
+    assert rc == 1 and "limit_cycles" in _err(L)

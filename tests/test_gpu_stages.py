@@ -582,3 +582,25 @@ def test_balance_solve_converges_inside_a_batch(m, n, k, seed):
     assert (host(info) == info_ref).all()
     assert (host(beta) == b_ref).all()
     assert (host(idx) == i_ref).all()
+
+
+# ---------------------------------------------------------------- bounded waits
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    # a wait (the FFN's counter wait) on a flag that nothing sets runs out after its limit,
+    # reports the pipeline timeout through the device error word, and the context keeps working
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lb.moe_selftest_wait(flag, 20_000_000)  # about 10 ms of SM clock cycles
+    with pytest.raises(lb.MoEError, match="timed out"):
+        lb.sync_status()
+    lb.sync_status()  # reading the word cleared it
+    flag.fill_(1)
+    lb.moe_selftest_wait(flag, 20_000_000)  # the flag is set: no wait, no error
+    lb.sync_status()
+    # a regular call after the timeout still gives the oracle's bits
+    m, n, k, cap = 1000, 8, 2, 200
+    idx = W.make_topk_idx(m, n, k, seed=3)
+    ref = oracle.capacity(idx, m, k, n, cap, m)
+    out = lb.moe_capacity_slots(dev(idx), n, cap)
+    lb.sync_status()
+    assert (host(out["slot"]) == ref["slot"]).all()
+    assert (host(out["expert_offsets"]) == ref["expert_offsets"]).all()
