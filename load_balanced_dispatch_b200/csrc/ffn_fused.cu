@@ -335,7 +335,9 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         int acc = 0, slot = 0;
         uint32_t aphase = 0, rphase = 0;
         for (;;) {
-            if (!ptx::mbar_wait(&sh->tready[slot], rphase, abort_flag)) break;
+            // every lane waits; the warp leaves together if any lane gave up (a timeout): the
+            // warp-collective TMEM loads below need all 32 lanes
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sh->tready[slot], rphase, abort_flag))) break;
             const int tile = *(volatile int*)&sh->tile_ring[slot];
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&sh->tfree[slot]);
@@ -351,7 +353,7 @@ ffn_fused_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(be + lane * 8) = *reinterpret_cast<const uint4*>(gb + col);
                 __syncwarp();
             }
-            if (!ptx::mbar_wait(&sh->tfull[acc], aphase, abort_flag)) break;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sh->tfull[acc], aphase, abort_flag))) break;
             ptx::tc_fence_after();
             const int64_t r = t.row0 + quad * 32 + lane;
             bool row_ok = r < t.row_end;

@@ -285,7 +285,9 @@ ffn_pair_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
         int acc = 0, slot = 0;
         uint32_t aphase = 0, rphase = 0;
         for (;;) {
-            if (!ptx::mbar_wait_cluster(&sh->tready[slot], rphase, abort_flag)) break;
+            // every lane waits; the warp leaves together if any lane gave up (a timeout): the
+            // warp-collective TMEM loads and __syncwarp below need all 32 lanes
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_cluster(&sh->tready[slot], rphase, abort_flag))) break;
             const int tile = *(volatile int*)&sh->tile_ring[slot];
             __syncwarp();
             if (lane == 0) {
@@ -311,7 +313,7 @@ ffn_pair_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 }
                 __syncwarp();
             }
-            if (!ptx::mbar_wait_cluster(&sh->tfull[acc], aphase, abort_flag)) break;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_cluster(&sh->tfull[acc], aphase, abort_flag))) break;
             ptx::tc_fence_after();
             const int64_t r = t.row0 + (int64_t)HM * rank + quad * 32 + lane;
             const bool row_ok = r < t.row_end;

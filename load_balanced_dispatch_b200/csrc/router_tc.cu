@@ -182,7 +182,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
         int buf = 0;
         uint32_t bphase = 0;
         for (int kb = 0; kb < nkb; ++kb) {
-            if (!ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag)) { drain_ok = false; break; }
+            // every lane waits; the warp leaves together if any lane gave up (a timeout), since the
+            // TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sh->tfull[buf], bphase, abort_flag))) { drain_ok = false; break; }
             ptx::tc_fence_after();
             if (FUSED) {
                 // per 32-column chunk, the three parts' block products: (p2 + p1) + p0, then into acc
