@@ -154,7 +154,11 @@ def _compare_layer(cfg, got, ref, sample=None):
 
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("switch", dict(m=1024, d=256, d_ff=512)),
                                      ("lossfree", dict(m=1024, d=256, d_ff=352)),
-                                     ("global", dict(m=2048, d=256, d_ff=512, seg_len=512))])
+                                     ("global", dict(m=2048, d=256, d_ff=512, seg_len=512)),
+                                     # more 128-token tiles than SMs (the router finishes whole rows),
+                                     # rows of 16 vectors in dispatch and combine, half-width GEMM2 tiles
+                                     ("global", dict(m=19456, d=128, d_ff=256, seg_len=4864,
+                                                     wr_std=1.0 / np.sqrt(128)))])
 @pytest.mark.parametrize("residual", [False, True])
 def test_layer_reduced(name, kw, residual):
     cfg = _scaled(name, **kw)
