@@ -107,7 +107,10 @@ def test_router_projection_without_scores(m, d, n, k, fn, renorm, bias):
 
 
 @pytest.mark.parametrize("m,d,n,k,fn,renorm,bias", [(40000, 256, 64, 2, 0, 1, False), (20000, 512, 128, 1, 0, 0, False),
-                                                      (19100, 192, 96, 6, 1, 0, True), (30001, 128, 32, 4, 0, 0, False)])
+                                                      (19100, 192, 96, 6, 1, 0, True), (30001, 128, 32, 4, 0, 0, False),
+                                                      # the per-thread row finish with sigmoid scores and a
+                                                      # ranking bias, and with k = 8 renormalised gates
+                                                      (25000, 128, 64, 6, 1, 0, True), (20000, 64, 64, 8, 0, 1, False)])
 def test_router_many_blocks_and_prepared_split(m, d, n, k, fn, renorm, bias):
     # more 128-token blocks than two waves of CTAs (ragged last block); the call with w_r = None
     # on a workspace from moe_router_prepare gives the same bits as the call that splits W_r itself
