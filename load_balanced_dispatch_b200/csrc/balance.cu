@@ -922,6 +922,21 @@ constexpr size_t tpr2_dyn_smem() {
     return (size_t)qb::kTpr2Warps * ((32 * 33 + qb::kTprCap * 32) * sizeof(float) + qb::kTprCap * 32);
 }
 
+// bsh[g NT .. g NT + NT - 1] (a 16-byte aligned run when NT is a multiple of 4)
+template <int NT>
+__device__ __forceinline__ void group_betas(const float* bsh, int g, float (&out)[NT]) {
+    if constexpr (NT % 4 == 0) {
+#pragma unroll
+        for (int e = 0; e < NT; e += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(bsh + g * NT + e);
+            out[e] = q.x; out[e + 1] = q.y; out[e + 2] = q.z; out[e + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < NT; ++e) out[e] = bsh[g * NT + e];
+    }
+}
+
 // NT consecutive scores from p (the first `valid` of them exist; the rest read as -inf)
 template <int NT>
 __device__ __forceinline__ void load_group(const float* p, bool vec, int valid, float (&out)[NT]) {
@@ -1083,10 +1098,14 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
                 float s1[NT], s2[NT];
                 load_group<NT>(rowp + g1 * NT, vec, n - g1 * NT, s1);
                 if (g2 >= 0) load_group<NT>(rowp + g2 * NT, vec, n - g2 * NT, s2);
+                // the group's betas in one piece (bsh holds 32 NT entries, zero past n)
+                float b1v[NT], b2v[NT];
+                group_betas<NT>(bsh, g1, b1v);
+                if (g2 >= 0) group_betas<NT>(bsh, g2, b2v);
 #pragma unroll
                 for (int e = 0; e < NT; ++e) {
                     const int j = g1 * NT + e;
-                    if (j < n && __fsub_rn(s1[e], bsh[j]) >= Tl) {
+                    if (j < n && __fsub_rn(s1[e], b1v[e]) >= Tl) {
                         if (nc < CAP) { ls[nc * 32 + lane] = s1[e]; lj[nc * 32 + lane] = (unsigned char)j; }
                         ++nc;
                     }
@@ -1095,7 +1114,7 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
 #pragma unroll
                     for (int e = 0; e < NT; ++e) {
                         const int j = g2 * NT + e;
-                        if (j < n && __fsub_rn(s2[e], bsh[j]) >= Tl) {
+                        if (j < n && __fsub_rn(s2[e], b2v[e]) >= Tl) {
                             if (nc < CAP) { ls[nc * 32 + lane] = s2[e]; lj[nc * 32 + lane] = (unsigned char)j; }
                             ++nc;
                         }
@@ -1111,15 +1130,24 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
         int A = 0;
         {
             uint32_t kk[CAP];
-#pragma unroll
-            for (int p = 0; p < CAP; ++p) {
+            // the keys of list slots p < pmax (slots 16 .. CAP - 1 only when some row of the warp has them)
+            auto slot_key = [&](int p) {
                 uint32_t key = 0u;
-                if (p < pmax && p < nc && mine) {
+                if (p < nc && mine) {
                     const int j = lj[p * 32 + lane];
                     const float v = __fsub_rn(ls[p * 32 + lane], bsh[j]);
                     key = v >= T ? float_key_nz(v) : 0u;
                 }
-                kk[p] = key;
+                return key;
+            };
+#pragma unroll
+            for (int p = 0; p < 16; ++p) kk[p] = p < pmax ? slot_key(p) : 0u;
+            if (pmax > 16) {
+#pragma unroll
+                for (int p = 16; p < CAP; ++p) kk[p] = p < pmax ? slot_key(p) : 0u;
+            } else {
+#pragma unroll
+                for (int p = 16; p < CAP; ++p) kk[p] = 0u;
             }
             if (pmax <= 16) {
                 // at most 16 listed elements in every row of the warp (then k < 16): a 16-wide network
