@@ -1169,13 +1169,18 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
         }
         const float vk = key_float(KK), vk1 = key_float(KK1);
         const float a = qb_threshold(vk, vk1, rule);
+        // one pass over the list: the picks, the sign counts, and the sweep's window test of
+        // u = fp32(s - alpha_i) (the list positions inside the window in inmask)
+        uint32_t inmask = 0;
+        int nin = 0;
         if (mine) {
             alpha[i] = a;
             int np = 0, eq = 0;
             const int need_eq = k - A;
             for (int p = 0; p < nc; ++p) {
                 const int j = lj[p * 32 + lane];
-                const float v = __fsub_rn(ls[p * 32 + lane], bsh[j]);
+                const float sv = ls[p * 32 + lane], bj = bsh[j];
+                const float v = __fsub_rn(sv, bj);
                 const uint32_t key = v >= T ? float_key_nz(v) : 0u;
                 const bool pick = key > KK || (key == KK && eq < need_eq);
                 eq += key == KK ? 1 : 0;
@@ -1184,7 +1189,16 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
                     atomicAdd(&cnt[j], 1);
                     ++np;
                 }
-                if (SIGN && key != 0u && __fsub_rn(ls[p * 32 + lane], a) > bsh[j]) atomicAdd(&above_s[j], 1u);
+                if (SIGN && key != 0u && __fsub_rn(sv, a) > bj) atomicAdd(&above_s[j], 1u);
+                if (SWEEP) {
+                    const uint32_t ua = float_key_nz(__fsub_rn(sv, a));
+                    if (ua > hi_s[j]) {
+                        atomicAdd(&above_s[j], 1u);
+                    } else if (ua >= lo_s[j]) {
+                        inmask |= 1u << p;
+                        ++nin;
+                    }
+                }
             }
         }
         {
@@ -1192,19 +1206,6 @@ qb_row_tpr2_kernel(const float* __restrict__ s, int64_t m, int n, int k, const f
             if (lane == 0 && tb) atomicAdd(&nties, __popc(tb));
         }
         if (SWEEP) {
-            uint32_t inmask = 0;
-            int nin = 0;
-            if (mine)
-                for (int p = 0; p < nc; ++p) {
-                    const int j = lj[p * 32 + lane];
-                    const uint32_t key = float_key_nz(__fsub_rn(ls[p * 32 + lane], a));
-                    if (key > hi_s[j]) {
-                        atomicAdd(&above_s[j], 1u);
-                    } else if (key >= lo_s[j]) {
-                        inmask |= 1u << p;
-                        ++nin;
-                    }
-                }
             int incl = nin;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
